@@ -1,0 +1,13 @@
+"""CPU oracle for paged decode attention (fp64 NumPy) and a reference model of
+the block manager.
+
+TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.  Only ``tests/``, the smoke
+check in ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may
+import, call or run anything in this folder.  It shares no code with the CUDA
+path and never imports the product package.
+"""
+from .paged_attention import attend, cache_write, decode_step, gather_context, paged_decode
+from .block_manager import BlockManagerError, BlockManagerModel
+
+__all__ = ["attend", "cache_write", "decode_step", "gather_context", "paged_decode",
+           "BlockManagerError", "BlockManagerModel"]

@@ -1,0 +1,144 @@
+"""Reference model of the block manager (pure Python).
+
+TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.  Only the tests, the smoke check
+in ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may use it.
+
+Rules, from "The KV Cache and PagedAttention":
+  * a text's cache is cut into equal blocks; its logical blocks map to
+    physical blocks anywhere in the pool (§Like Pages of Memory);
+  * the block table holds, per logical block, the physical block and how many
+    places are filled; a new physical block is handed out only when all the
+    text's earlier blocks are full (§The Block Table);
+  * when a text is done its blocks go back to the pool (§The Block Table);
+  * parallel samples of one prompt point at the same physical blocks, each
+    block counting the texts that use it; a text about to write into a shared
+    block first gets a copy, writes there, and the original's count drops by
+    one (§Shared, Copied on Write);
+  * a text holds all its blocks or none (§When Memory Runs Out): an operation
+    that cannot get every block it needs changes nothing.
+
+Free-list policy (the pages leave it open): blocks are taken from the front of
+the free list and returned to its back; the initial order is given.  The
+"places filled" field is kept as the text's token count (filled places of
+block j = min(B, n - j*B)).
+
+Pinned by tests/golden/cow_two_answers.json (the pages' two-answer example)
+and by invariants checked in tests/test_block_manager.py.
+"""
+from __future__ import annotations
+
+from collections import deque
+from typing import Dict, List, Optional, Sequence, Tuple
+
+
+class BlockManagerError(Exception):
+    def __init__(self, kind: str, msg: str = ""):
+        super().__init__(f"{kind}: {msg}")
+        self.kind = kind
+
+
+class BlockManagerModel:
+    def __init__(self, num_blocks: int, block_size: int,
+                 initial_order: Optional[Sequence[int]] = None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise BlockManagerError("invalid", "num_blocks and block_size must be > 0")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        order = list(range(num_blocks)) if initial_order is None else [int(b) for b in initial_order]
+        if sorted(order) != list(range(num_blocks)):
+            raise BlockManagerError("invalid", "initial order is not a permutation")
+        self.free: deque = deque(order)
+        self.ref: List[int] = [0] * num_blocks
+        self.tables: Dict[int, List[int]] = {}
+        self.tokens: Dict[int, int] = {}
+
+    # -- helpers -----------------------------------------------------------
+    def _take(self) -> int:
+        b = self.free.popleft()
+        self.ref[b] = 1
+        return b
+
+    def _need(self, n: int) -> None:
+        if len(self.free) < n:
+            raise BlockManagerError("out_of_blocks", f"need {n}, have {len(self.free)}")
+
+    # -- operations --------------------------------------------------------
+    def add_seq(self, seq_id: int, num_tokens: int) -> None:
+        """A new text whose first ``num_tokens`` tokens (its prompt) are
+        stored at once: ceil(n / B) fresh blocks."""
+        if seq_id in self.tables:
+            raise BlockManagerError("exists", str(seq_id))
+        if num_tokens < 0:
+            raise BlockManagerError("invalid", "negative token count")
+        n_blocks = -(-num_tokens // self.block_size)
+        self._need(n_blocks)
+        self.tables[seq_id] = [self._take() for _ in range(n_blocks)]
+        self.tokens[seq_id] = num_tokens
+
+    def fork(self, parent: int, child: int) -> None:
+        """The child shares every block of the parent; each count goes up by one."""
+        if parent not in self.tables:
+            raise BlockManagerError("no_seq", str(parent))
+        if child in self.tables:
+            raise BlockManagerError("exists", str(child))
+        self.tables[child] = list(self.tables[parent])
+        self.tokens[child] = self.tokens[parent]
+        for b in self.tables[child]:
+            self.ref[b] += 1
+
+    def append_slot(self, seq_id: int) -> Tuple[int, int, int]:
+        """Room for the text's next token.  Returns (slot, cow_src, cow_dst);
+        the copy pair is (-1, -1) when no copy is needed.  The caller copies
+        block cow_src to cow_dst before writing the token."""
+        if seq_id not in self.tables:
+            raise BlockManagerError("no_seq", str(seq_id))
+        table = self.tables[seq_id]
+        n = self.tokens[seq_id]
+        place = n % self.block_size
+        src = dst = -1
+        if place == 0:
+            self._need(1)
+            table.append(self._take())
+        else:
+            last = table[-1]
+            if self.ref[last] > 1:
+                self._need(1)
+                dst = self._take()
+                self.ref[last] -= 1
+                table[-1] = dst
+                src = last
+        self.tokens[seq_id] = n + 1
+        return table[-1] * self.block_size + place, src, dst
+
+    def free_seq(self, seq_id: int) -> None:
+        """The text is done: every block's count drops by one; blocks that
+        reach zero go back to the pool, in table order."""
+        if seq_id not in self.tables:
+            raise BlockManagerError("no_seq", str(seq_id))
+        for b in self.tables.pop(seq_id):
+            if self.ref[b] <= 0:
+                raise BlockManagerError("corrupt", f"count of block {b} below zero")
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+        del self.tokens[seq_id]
+
+    # -- queries -----------------------------------------------------------
+    def num_free(self) -> int:
+        return len(self.free)
+
+    def refcount(self, block: int) -> int:
+        return self.ref[block]
+
+    def export(self, seq_ids: Sequence[int], max_blocks_per_seq: int):
+        """Block tables (``-1`` past each text's last block) and token counts."""
+        tables, lens = [], []
+        for s in seq_ids:
+            if s not in self.tables:
+                raise BlockManagerError("no_seq", str(s))
+            t = self.tables[s]
+            if len(t) > max_blocks_per_seq:
+                raise BlockManagerError("table_full", f"{len(t)} > {max_blocks_per_seq}")
+            tables.append(t + [-1] * (max_blocks_per_seq - len(t)))
+            lens.append(self.tokens[s])
+        return tables, lens

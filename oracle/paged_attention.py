@@ -1,0 +1,140 @@
+"""CPU oracle: paged decode attention and the KV-cache write, in fp64.
+
+TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.  Only the tests, the smoke check
+in ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it.
+It shares no code with the CUDA path and imports nothing from the package.
+
+What it computes is the plain definition.  Paging changes where the keys and
+values live, not what attention computes ("The KV Cache and PagedAttention",
+§Like Pages of Memory: logical blocks are contiguous to the text, physical
+blocks sit anywhere; §The Block Table: attention follows the block table and
+fetches each block's keys and values).  So the oracle
+
+  1. writes the new token's key and value into its slot ("KV cache", §How it
+     works: the new position's key and value are written into the cache;
+     "The KV Cache and PagedAttention", §One Token at a Time: only the new
+     token's key and value are computed, the earlier ones are kept);
+  2. gathers each text's tokens through its block table into one contiguous
+     fp64 buffer (token t sits in logical block t // B at place t % B);
+  3. runs textbook attention for the one new query: weights
+     softmax(scale * q . k_t) over every stored key including the new one
+     ("KV cache", §How it works), output sum_t w_t v_t.
+
+Readings where the pages are silent (each also listed in the design notes):
+  * pool layout ``[num_blocks][num_heads][block_size][head_dim]`` for K and V;
+  * the context length counts the token written in this step (write, then
+    attend);
+  * ``scale`` is a parameter (the workloads use 1/sqrt(head_dim) in fp32);
+  * a text with no tokens gets a zero output;
+  * a negative slot marks a padding token that is not written;
+  * table entries past the text's last block are never read.
+
+Precision: inputs are the exact fp16/bf16 values widened to fp64; every step
+is fp64; softmax subtracts the maximum before exponentiating (an identity, so
+the result is the same number up to rounding).
+
+Pinned by tests/test_oracle.py against: torch's fp64 attention on unpaged
+contiguous tensors, scalar brute force with ``math.fsum`` on tiny inputs,
+closed forms (one token gives its value; equal scores give the mean of the
+values; one dominant score gives its value), bit-identity under a relabelling
+of physical blocks, under a change of block size, and for texts that share
+prefix blocks, and a hand-worked cache write.
+"""
+from __future__ import annotations
+
+from typing import Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+
+def cache_write(k_cache: np.ndarray, v_cache: np.ndarray, k: np.ndarray, v: np.ndarray,
+                slot_mapping: Sequence[int], block_size: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Return copies of the caches with token t's key/value placed at slot
+    ``slot_mapping[t]``: physical block ``slot // block_size``, place
+    ``slot % block_size``.  Negative slots are skipped.
+
+    A pure copy of values, so it works on any dtype, including raw uint16
+    bit patterns; the result is exact.  Caches are ``[N][H][B][D]``; k and v
+    are ``[T][H][D]``."""
+    kc = k_cache.copy()
+    vc = v_cache.copy()
+    for t, slot in enumerate(slot_mapping):
+        slot = int(slot)
+        if slot < 0:
+            continue
+        block, place = divmod(slot, block_size)
+        kc[block, :, place, :] = k[t]
+        vc[block, :, place, :] = v[t]
+    return kc, vc
+
+
+def gather_context(cache: np.ndarray, block_table: Sequence[int], context_len: int,
+                   block_size: int) -> np.ndarray:
+    """Contiguous fp64 ``[L][H][D]`` copy of one text's keys (or values):
+    token t comes from physical block ``block_table[t // block_size]``, place
+    ``t % block_size``."""
+    L = int(context_len)
+    H, D = cache.shape[1], cache.shape[3]
+    out = np.empty((L, H, D), dtype=np.float64)
+    for t in range(L):
+        phys = int(block_table[t // block_size])
+        out[t] = cache[phys, :, t % block_size, :]
+    return out
+
+
+def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> np.ndarray:
+    """Attention of one query per head over L stored keys/values, fp64.
+
+    q ``[H][D]``, K and V ``[L][H][D]``; returns ``[H][D]``.
+    z_t = scale * sum_d q[d] K[t, d];  w = softmax(z);  out = sum_t w_t V[t].
+    With L == 0 the output is zero."""
+    q = np.asarray(q, dtype=np.float64)
+    H, D = q.shape
+    L = K.shape[0]
+    out = np.zeros((H, D), dtype=np.float64)
+    if L == 0:
+        return out
+    for h in range(H):
+        z = float(scale) * (K[:, h, :] @ q[h])
+        e = np.exp(z - z.max())
+        w = e / e.sum()
+        out[h] = w @ V[:, h, :]
+    return out
+
+
+def paged_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                 block_tables: np.ndarray, context_lens: Sequence[int], scale: float,
+                 block_size: int,
+                 pairs: Optional[Iterable[Tuple[int, int]]] = None) -> np.ndarray:
+    """Decode attention over paged caches, fp64 ``[S][H][D]``.
+
+    With ``pairs`` (a list of (seq, head)), only those outputs are computed
+    (the rest stay zero); this is how large workloads are checked one output
+    at a time."""
+    S, H, D = q.shape
+    out = np.zeros((S, H, D), dtype=np.float64)
+    if pairs is None:
+        for s in range(S):
+            K = gather_context(k_cache, block_tables[s], context_lens[s], block_size)
+            V = gather_context(v_cache, block_tables[s], context_lens[s], block_size)
+            out[s] = attend(q[s], K, V, scale)
+        return out
+    by_seq = {}
+    for s, h in pairs:
+        by_seq.setdefault(int(s), []).append(int(h))
+    for s, heads in by_seq.items():
+        K = gather_context(k_cache, block_tables[s], context_lens[s], block_size)
+        V = gather_context(v_cache, block_tables[s], context_lens[s], block_size)
+        full = attend(q[s][heads], K[:, heads, :], V[:, heads, :], scale)
+        for i, h in enumerate(heads):
+            out[s, h] = full[i]
+    return out
+
+
+def decode_step(q, k, v, k_cache, v_cache, slot_mapping, block_tables, context_lens,
+                scale, block_size, pairs=None):
+    """One decode step of one layer: write the new tokens, then attend.
+    Returns (out fp64, k_cache', v_cache')."""
+    kc, vc = cache_write(k_cache, v_cache, k, v, slot_mapping, block_size)
+    out = paged_decode(q, kc, vc, block_tables, context_lens, scale, block_size, pairs)
+    return out, kc, vc

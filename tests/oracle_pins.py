@@ -1,0 +1,292 @@
+"""Checks that pin the oracle to something other than itself.
+
+Each ``pin_*`` takes the decode function under test, with the oracle's
+signature ``fn(q, k_cache, v_cache, block_tables, context_lens, scale,
+block_size) -> out``, and raises AssertionError when it disagrees with what
+the pages and the mathematics fix.  tests/test_oracle.py runs them on the
+oracle; tests/test_oracle_mutants.py runs them on copies of the oracle with
+planted mistakes and requires each copy to fail at least one.
+
+The ground truth here is built in the opposite direction to the oracle: texts
+are drawn as contiguous [L][H][D] tensors first, then scattered into a paged
+pool through a random block table, so a wrong gather cannot agree with it.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def load_golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def f64(t):
+    return t.to(torch.float64).numpy() if isinstance(t, torch.Tensor) else np.asarray(t, np.float64)
+
+
+# ---------------------------------------------------------------------------
+# contiguous texts -> paged pool (independent of the oracle's gather)
+# ---------------------------------------------------------------------------
+
+def random_texts(lens, H, D, seed, dtype=torch.float16):
+    g = torch.Generator().manual_seed(seed)
+    K = [torch.randn(L, H, D, generator=g).to(dtype) for L in lens]
+    V = [torch.randn(L, H, D, generator=g).to(dtype) for L in lens]
+    q = torch.randn(len(lens), H, D, generator=g).to(dtype)
+    return q, K, V
+
+
+def scatter_to_pool(K, V, block_size, num_blocks, seed, dtype=torch.float16):
+    """Place token t of text s at (table[s][t // B], t % B), blocks drawn from
+    a seeded permutation; unused rows are NaN."""
+    H, D = K[0].shape[1], K[0].shape[2]
+    g = torch.Generator().manual_seed(seed + 77)
+    perm = torch.randperm(num_blocks, generator=g).tolist()
+    kc = torch.full((num_blocks, H, block_size, D), float("nan"), dtype=dtype)
+    vc = torch.full((num_blocks, H, block_size, D), float("nan"), dtype=dtype)
+    nblk = [-(-k.shape[0] // block_size) for k in K]
+    tables = np.full((len(K), max([1] + nblk)), -1, dtype=np.int64)
+    at = 0
+    for s, (k, v) in enumerate(zip(K, V)):
+        for j in range(nblk[s]):
+            phys = perm[at]
+            at += 1
+            tables[s, j] = phys
+            lo, hi = j * block_size, min(k.shape[0], (j + 1) * block_size)
+            kc[phys, :, : hi - lo, :] = k[lo:hi].permute(1, 0, 2)
+            vc[phys, :, : hi - lo, :] = v[lo:hi].permute(1, 0, 2)
+    return kc, vc, tables
+
+
+def sdpa_contiguous(q, K, V, scale):
+    """torch's attention in fp64 on the unpaged texts (a library routine,
+    written independently of the oracle)."""
+    outs = []
+    for s in range(len(K)):
+        if K[s].shape[0] == 0:
+            outs.append(torch.zeros(q.shape[1], q.shape[2], dtype=torch.float64))
+            continue
+        qs = q[s].to(torch.float64)[:, None, :]             # [H][1][D]
+        ks = K[s].to(torch.float64).permute(1, 0, 2)         # [H][L][D]
+        vs = V[s].to(torch.float64).permute(1, 0, 2)
+        o = torch.nn.functional.scaled_dot_product_attention(qs, ks, vs, scale=scale)
+        outs.append(o[:, 0, :])
+    return torch.stack(outs).numpy()
+
+
+def brute_force(q, K, V, scale):
+    """Scalar loops with math.exp / math.fsum."""
+    S, H, D = q.shape
+    out = np.zeros((S, H, D))
+    qn = f64(q)
+    for s in range(S):
+        Ks, Vs = f64(K[s]), f64(V[s])
+        L = Ks.shape[0]
+        if L == 0:
+            continue
+        for h in range(H):
+            z = [scale * math.fsum(qn[s, h, d] * Ks[t, h, d] for d in range(D)) for t in range(L)]
+            zmax = max(z)
+            e = [math.exp(x - zmax) for x in z]
+            tot = math.fsum(e)
+            for d in range(D):
+                out[s, h, d] = math.fsum(e[t] * Vs[t, h, d] for t in range(L)) / tot
+    return out
+
+
+# ---------------------------------------------------------------------------
+# pins
+# ---------------------------------------------------------------------------
+
+LENS_SMALL = [5, 9, 16, 23, 1, 31]
+
+
+def pin_unpaged_sdpa(fn):
+    for B, dtype, seed in ((4, torch.float16, 11), (8, torch.bfloat16, 12), (16, torch.float16, 13)):
+        H, D = 3, 16
+        q, K, V = random_texts(LENS_SMALL, H, D, seed, dtype)
+        kc, vc, tables = scatter_to_pool(K, V, B, 40, seed, dtype)
+        scale = 1.0 / math.sqrt(D)
+        got = fn(f64(q), f64(kc), f64(vc), tables, LENS_SMALL, scale, B)
+        ref = sdpa_contiguous(q, K, V, scale)
+        err = np.abs(got - ref).max()
+        assert err <= 1e-12, f"unpaged sdpa B={B}: max err {err}"
+
+
+def pin_brute_force(fn):
+    lens = [5, 9, 16, 23]
+    H, D, B = 2, 8, 4
+    q, K, V = random_texts(lens, H, D, 21)
+    kc, vc, tables = scatter_to_pool(K, V, B, 16, 21)
+    scale = 0.3535
+    got = fn(f64(q), f64(kc), f64(vc), tables, lens, scale, B)
+    ref = brute_force(q, K, V, scale)
+    err = np.abs(got - ref).max()
+    assert err <= 1e-12, f"brute force: max err {err}"
+
+
+def pin_golden_closed_form(fn):
+    g = load_golden("attention_closed_form.json")
+    got = fn(np.array(g["q"]), np.array(g["k_cache"]), np.array(g["v_cache"]),
+             np.array(g["block_tables"]), g["context_lens"], g["scale"], g["block_size"])
+    err = np.abs(got - np.array(g["expected_out"])).max()
+    assert err <= g["tol"], f"closed form: {got.ravel()} vs {g['expected_out']}"
+
+
+def pin_single_token(fn):
+    """One token: its weight is exactly 1, so the output is its value, exactly."""
+    H, D, B = 4, 32, 4
+    q, K, V = random_texts([1, 1, 1], H, D, 31)
+    kc, vc, tables = scatter_to_pool(K, V, B, 8, 31)
+    got = fn(f64(q), f64(kc), f64(vc), tables, [1, 1, 1], 0.17677669, B)
+    for s in range(3):
+        assert np.array_equal(got[s], f64(V[s])[0]), "single token output != its value"
+
+
+def pin_uniform_scores(fn):
+    """q = 0 (and, separately, all keys equal): every weight is 1/L, so the
+    output is the mean of the values."""
+    H, D, B = 2, 16, 4
+    lens = [7, 12]
+    q, K, V = random_texts(lens, H, D, 41)
+    kc, vc, tables = scatter_to_pool(K, V, B, 8, 41)
+    zero_q = np.zeros_like(f64(q))
+    got = fn(zero_q, f64(kc), f64(vc), tables, lens, 0.25, B)
+    for s, L in enumerate(lens):
+        mean = f64(V[s]).mean(axis=0)
+        assert np.abs(got[s] - mean).max() <= 1e-12, "q=0 is not the mean of V"
+    Keq = [torch.ones_like(k) * 0.5 for k in K]
+    kc2, vc2, tables2 = scatter_to_pool(Keq, V, B, 8, 42)
+    got2 = fn(f64(q), f64(kc2), f64(vc2), tables2, lens, 0.25, B)
+    for s, L in enumerate(lens):
+        mean = f64(V[s]).mean(axis=0)
+        assert np.abs(got2[s] - mean).max() <= 1e-12, "equal keys are not the mean of V"
+
+
+def pin_dominant_key(fn):
+    """One key far ahead of the others (score gap > 800): the others' weights
+    underflow, so the output is that key's value."""
+    H, D, B = 1, 4, 4
+    L = 10
+    rng = np.random.default_rng(5)
+    K = rng.normal(size=(L, H, D))
+    V = rng.normal(size=(L, H, D))
+    q = np.zeros((1, H, D))
+    q[0, 0, 0] = 1.0
+    K[:, 0, 0] = 0.0
+    K[6, 0, 0] = 1000.0
+    Kt, Vt = [torch.tensor(K)], [torch.tensor(V)]
+    kc, vc, tables = scatter_to_pool(Kt, Vt, B, 6, 51, torch.float64)
+    got = fn(q, f64(kc), f64(vc), tables, [L], 1.0, B)
+    assert np.abs(got[0, 0] - V[6, 0]).max() <= 1e-12, "dominant key's value not returned"
+
+
+def pin_relabel_invariance(fn):
+    """Renumbering the physical blocks (pool and tables together) changes
+    nothing, bit for bit."""
+    H, D, B, N = 3, 16, 4, 40
+    q, K, V = random_texts(LENS_SMALL, H, D, 61)
+    kc, vc, tables = scatter_to_pool(K, V, B, N, 61)
+    base = fn(f64(q), f64(kc), f64(vc), tables, LENS_SMALL, 0.25, B)
+    perm = np.random.default_rng(7).permutation(N)
+    kc2 = np.empty_like(f64(kc))
+    vc2 = np.empty_like(f64(vc))
+    kc2[perm] = f64(kc)
+    vc2[perm] = f64(vc)
+    t2 = np.where(tables >= 0, perm[np.maximum(tables, 0)], -1)
+    got = fn(f64(q), kc2, vc2, t2, LENS_SMALL, 0.25, B)
+    assert np.array_equal(base, got), "not invariant under block relabelling"
+
+
+def pin_block_size_invariance(fn):
+    """The same texts stored with blocks of 4, 8, 16 or 32 give the same
+    output, bit for bit."""
+    H, D = 2, 16
+    q, K, V = random_texts(LENS_SMALL, H, D, 71)
+    outs = []
+    for B in (4, 8, 16, 32):
+        kc, vc, tables = scatter_to_pool(K, V, B, 64, 71 + B)
+        outs.append(fn(f64(q), f64(kc), f64(vc), tables, LENS_SMALL, 0.25, B))
+    for o in outs[1:]:
+        assert np.array_equal(outs[0], o), "output depends on block size"
+
+
+def pin_shared_prefix(fn):
+    """A text reading shared prefix blocks gives the same output as a copy of
+    it whose blocks are private; two texts with the same table, length and
+    query give the same output."""
+    H, D, B = 2, 8, 4
+    q, K, V = random_texts([10, 10], H, D, 81)
+    K[1][:8] = K[0][:8]
+    V[1][:8] = V[0][:8]
+    kc, vc, tables = scatter_to_pool(K, V, B, 12, 81)
+    private = fn(f64(q), f64(kc), f64(vc), tables, [10, 10], 0.3, B)
+    shared_tables = tables.copy()
+    shared_tables[1, :2] = tables[0, :2]
+    shared = fn(f64(q), f64(kc), f64(vc), shared_tables, [10, 10], 0.3, B)
+    assert np.array_equal(private, shared), "shared prefix blocks change the output"
+    q2 = q.clone()
+    q2[1] = q2[0]
+    same = fn(f64(q2), f64(kc), f64(vc), np.stack([tables[0], tables[0]]), [10, 10], 0.3, B)
+    assert np.array_equal(same[0], same[1]), "identical texts differ"
+
+
+def pin_nan_tail_and_unused_entries(fn):
+    """Rows past the context (NaN) and table entries past the last block
+    (garbage) never reach the output; an empty text gives zeros."""
+    H, D, B = 2, 8, 4
+    q, K, V = random_texts([6, 3, 0], H, D, 91)
+    kc, vc, tables = scatter_to_pool(K, V, B, 8, 91)
+    t = np.concatenate([tables, np.full((3, 2), 10**6)], axis=1)
+    got = fn(f64(q), f64(kc), f64(vc), t, [6, 3, 0], 0.3, B)
+    assert np.isfinite(got).all(), "NaN padding leaked"
+    assert np.array_equal(got[2], np.zeros((H, D))), "empty text is not zero"
+
+
+ATTENTION_PINS = [pin_unpaged_sdpa, pin_brute_force, pin_golden_closed_form, pin_single_token,
+                  pin_uniform_scores, pin_dominant_key, pin_relabel_invariance,
+                  pin_block_size_invariance, pin_shared_prefix, pin_nan_tail_and_unused_entries]
+
+
+def pin_cache_write_golden(write_fn):
+    g = load_golden("cache_write_tiny.json")
+    shape = (g["num_blocks"], g["num_heads"], g["block_size"], g["head_dim"])
+    kc = np.zeros(shape, dtype=np.uint16)
+    vc = np.zeros(shape, dtype=np.uint16)
+    k = np.array(g["k"], dtype=np.uint16)
+    v = np.array(g["v"], dtype=np.uint16)
+    kc2, vc2 = write_fn(kc, vc, k, v, g["slot_mapping"], g["block_size"])
+    assert np.array_equal(kc2, np.array(g["expected_k_cache"], dtype=np.uint16)), "k cache write"
+    assert np.array_equal(vc2, np.array(g["expected_v_cache"], dtype=np.uint16)), "v cache write"
+    assert not kc.any() and not vc.any(), "write modified its input"
+
+
+def pin_cache_write_then_read(write_fn):
+    """Writing every token of contiguous texts through their slots rebuilds
+    the pool that the independent scatter builds."""
+    H, D, B = 2, 8, 4
+    lens = [5, 9, 3]
+    q, K, V = random_texts(lens, H, D, 101)
+    kc_ref, vc_ref, tables = scatter_to_pool(K, V, B, 10, 101)
+    kc = torch.full_like(kc_ref, float("nan")).view(torch.int16).numpy()
+    vc = torch.full_like(vc_ref, float("nan")).view(torch.int16).numpy()
+    ks, vs, slots = [], [], []
+    for s, L in enumerate(lens):
+        for t in range(L):
+            ks.append(K[s][t].view(torch.int16).numpy())
+            vs.append(V[s][t].view(torch.int16).numpy())
+            slots.append(int(tables[s, t // B]) * B + t % B)
+    kc2, vc2 = write_fn(kc, vc, np.stack(ks), np.stack(vs), slots, B)
+    assert np.array_equal(kc2, kc_ref.view(torch.int16).numpy()), "rebuilt k pool differs"
+    assert np.array_equal(vc2, vc_ref.view(torch.int16).numpy()), "rebuilt v pool differs"
+
+
+WRITE_PINS = [pin_cache_write_golden, pin_cache_write_then_read]

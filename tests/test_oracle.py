@@ -1,0 +1,54 @@
+"""The oracle against its pins (CPU only)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import oracle_pins as P
+
+
+@pytest.mark.parametrize("pin", P.ATTENTION_PINS, ids=lambda f: f.__name__)
+def test_attention_pin(pin):
+    pin(oracle.paged_decode)
+
+
+@pytest.mark.parametrize("pin", P.WRITE_PINS, ids=lambda f: f.__name__)
+def test_write_pin(pin):
+    pin(oracle.cache_write)
+
+
+def test_step_writes_before_attending():
+    """The token written in this step is one of the keys the query attends to
+    ("KV cache", How it works: the stored keys plus the new key)."""
+    H, D, B = 2, 8, 4
+    q, K, V = P.random_texts([7], H, D, 111)
+    kc, vc, tables = P.scatter_to_pool([K[0][:6]], [V[0][:6]], B, 4, 111)
+    slot = int(tables[0, 6 // B]) * B + 6 % B
+    out, kc2, vc2 = oracle.decode_step(P.f64(q), P.f64(K[0][6:7]), P.f64(V[0][6:7]), P.f64(kc),
+                                       P.f64(vc), [slot], tables, [7], 0.3, B)
+    ref = P.sdpa_contiguous(q, K, V, 0.3)
+    assert np.abs(out - ref).max() <= 1e-12
+
+
+def test_pairs_subset_matches_full():
+    H, D, B = 3, 8, 4
+    lens = [5, 9, 16]
+    q, K, V = P.random_texts(lens, H, D, 121)
+    kc, vc, tables = P.scatter_to_pool(K, V, B, 16, 121)
+    full = oracle.paged_decode(P.f64(q), P.f64(kc), P.f64(vc), tables, lens, 0.3, B)
+    pairs = [(0, 2), (2, 0), (2, 1), (1, 1)]
+    part = oracle.paged_decode(P.f64(q), P.f64(kc), P.f64(vc), tables, lens, 0.3, B, pairs=pairs)
+    for s, h in pairs:
+        assert np.array_equal(full[s, h], part[s, h])
+
+
+def test_tiny_workload_runs_and_is_finite():
+    """The tiny workload end to end through the oracle: NaN poison in unused
+    rows never reaches the output."""
+    from paged_kv_cache_326_b200 import workloads as W
+    w = W.tiny(device="cpu")
+    out, kc, vc = oracle.decode_step(
+        P.f64(w.q), P.f64(w.k), P.f64(w.v), P.f64(w.k_cache), P.f64(w.v_cache),
+        w.slot_mapping.numpy(), w.block_tables.numpy(), w.context_lens.numpy(), w.scale,
+        w.block_size)
+    assert out.shape == (4, 8, 64) and np.isfinite(out).all()

@@ -1,0 +1,145 @@
+"""Each copy of the oracle below has one planted mistake of the kind a
+careless implementation makes; the pins must catch every one (CPU only)."""
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_pins as P
+
+
+def _decode_with(attend_fn=None, gather_fn=None, len_fn=None):
+    attend_fn = attend_fn or oracle.attend
+    gather_fn = gather_fn or oracle.gather_context
+    len_fn = len_fn or (lambda L: L)
+
+    def fn(q, k_cache, v_cache, block_tables, context_lens, scale, block_size):
+        S, H, D = q.shape
+        out = np.zeros((S, H, D))
+        for s in range(S):
+            L = len_fn(int(context_lens[s]))
+            K = gather_fn(k_cache, block_tables[s], L, block_size)
+            V = gather_fn(v_cache, block_tables[s], L, block_size)
+            out[s] = attend_fn(q[s], K, V, scale)
+        return out
+    return fn
+
+
+def gather_swapped_index(cache, table, L, B):
+    H, D = cache.shape[1], cache.shape[3]
+    out = np.empty((L, H, D))
+    for t in range(L):
+        out[t] = cache[int(table[t % B]) if t % B < len(table) else 0, :, min(t // B, B - 1), :]
+    return out
+
+
+def gather_off_by_one_place(cache, table, L, B):
+    H, D = cache.shape[1], cache.shape[3]
+    out = np.empty((L, H, D))
+    for t in range(L):
+        out[t] = cache[int(table[t // B]), :, (t + 1) % B, :]
+    return out
+
+
+def attend_no_scale(q, K, V, scale):
+    return oracle.attend(q, K, V, 1.0)
+
+
+def attend_k_v_swapped(q, K, V, scale):
+    return oracle.attend(q, V, K, scale)
+
+
+def attend_unnormalised(q, K, V, scale):
+    H, D = q.shape
+    out = np.zeros((H, D))
+    for h in range(H):
+        z = scale * (K[:, h, :] @ q[h])
+        out[h] = np.exp(z - z.max()) @ V[:, h, :]
+    return out
+
+
+def attend_wrong_head(q, K, V, scale):
+    H = q.shape[0]
+    return oracle.attend(q, K[:, [(h + 1) % H for h in range(H)], :], V, scale)
+
+
+def attend_mean_of_keys(q, K, V, scale):
+    H, D = q.shape
+    out = np.zeros((H, D))
+    for h in range(H):
+        z = scale * (K[:, h, :] @ q[h])
+        w = np.exp(z - z.max())
+        out[h] = (w / w.sum()) @ K[:, h, :]
+    return out
+
+
+def attend_weights_transposed_sign(q, K, V, scale):
+    return oracle.attend(-q, K, V, scale)
+
+
+MUTANTS = {
+    "block/place swapped": _decode_with(gather_fn=gather_swapped_index),
+    "place off by one": _decode_with(gather_fn=gather_off_by_one_place),
+    "scale dropped": _decode_with(attend_fn=attend_no_scale),
+    "K and V swapped": _decode_with(attend_fn=attend_k_v_swapped),
+    "softmax not normalised": _decode_with(attend_fn=attend_unnormalised),
+    "wrong head's keys": _decode_with(attend_fn=attend_wrong_head),
+    "keys mixed instead of values": _decode_with(attend_fn=attend_mean_of_keys),
+    "score sign flipped": _decode_with(attend_fn=attend_weights_transposed_sign),
+    "new token left out": _decode_with(len_fn=lambda L: max(L - 1, 0)),
+}
+
+
+def _fails_some_pin(fn):
+    failed = []
+    for pin in P.ATTENTION_PINS:
+        try:
+            pin(fn)
+        except (AssertionError, IndexError, ValueError):
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_attention_mistake_is_caught(name):
+    assert _fails_some_pin(MUTANTS[name]), f"no pin catches: {name}"
+
+
+def test_unmodified_oracle_passes_all_pins():
+    assert _fails_some_pin(oracle.paged_decode) == []
+
+
+def write_block_place_swapped(kc, vc, k, v, slots, B):
+    kc, vc = kc.copy(), vc.copy()
+    for t, s in enumerate(slots):
+        if s < 0:
+            continue
+        place, block = divmod(int(s), B)
+        if place < kc.shape[2] and block < kc.shape[0]:
+            kc[block, :, place, :] = k[t]
+            vc[block, :, place, :] = v[t]
+    return kc, vc
+
+
+def write_ignores_negative_check(kc, vc, k, v, slots, B):
+    kc, vc = kc.copy(), vc.copy()
+    for t, s in enumerate(slots):
+        block, place = divmod(int(s), B)
+        kc[block, :, place, :] = k[t]
+        vc[block, :, place, :] = v[t]
+    return kc, vc
+
+
+def write_k_into_v(kc, vc, k, v, slots, B):
+    return oracle.cache_write(kc, vc, v, k, slots, B)
+
+
+@pytest.mark.parametrize("fn", [write_block_place_swapped, write_ignores_negative_check,
+                                write_k_into_v], ids=lambda f: f.__name__)
+def test_planted_write_mistake_is_caught(fn):
+    failed = 0
+    for pin in P.WRITE_PINS:
+        try:
+            pin(fn)
+        except (AssertionError, IndexError):
+            failed += 1
+    assert failed, fn.__name__
