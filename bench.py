@@ -1,0 +1,386 @@
+"""Benchmark: one decode step of an OPT-13B-shaped layer, batch 64.
+
+A step is the whole hot path once: the write of each text's new key/value
+(pa_kv_cache_write), then paged decode attention over every text's cache
+(pa_paged_attn_decode: the decode kernel plus its log-sum-exp merge).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is KV bytes read per step / device
+time per step (GB/s, whole job over all ranks); ``e2e`` repeats it with the
+step's inputs copied from pinned host memory and the output copied back inside
+the timed region.  Under torchrun each rank runs its own independent batch
+(weak scaling, no collective on the data path).  ``--impl reference`` times the
+fp64 CPU oracle on the host instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode KV HBM GB/s (% of B200 peak) and decode tokens/s, 1 GPU"
+WORKLOAD = "opt13b_batch64"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_opt13b_batch64_traffic.json")
+KERNEL_SOURCES = ["paged_kv_cache_326_b200/csrc/paged_attn_decode.cu",
+                  "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: copy, burst)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def traffic_per_launch():
+    """DRAM bytes per decode call from the committed ncu summary, if it was
+    taken on the kernel as it is now; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        if t.get("kernel_source_hash") == kernel_source_hash():
+            return float(t["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+def kv_bytes(context_lens, num_heads, head_dim, elem_bytes) -> int:
+    from paged_kv_cache_326_b200.accounting import decode_kv_bytes
+    return decode_kv_bytes(context_lens, num_heads, head_dim, elem_bytes)
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def oracle_runner(w, num_pairs):
+    """The oracle over the first ``num_pairs`` (text, head) pairs of the
+    workload, in text-major order.  Inputs are prepared outside the timed
+    region.  Returns (run, kv_bytes_of_the_sample)."""
+    from threadpoolctl import threadpool_limits
+    from tests.gpu_helpers import oracle_inputs, run_oracle
+    H = w.num_heads
+    pairs = [(p // H, p % H) for p in range(num_pairs)]
+    seqs = sorted({s for s, _ in pairs})
+    oi = oracle_inputs(w.q, w.k, w.v, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                       w.slot_mapping, w.block_size, seqs)
+    lens = w.context_lens.tolist()
+    sample_bytes = sum(lens[s] for s, _ in pairs) * 2 * w.head_dim * w.q.element_size()
+    full = num_pairs == len(seqs) * H
+
+    def run():
+        with threadpool_limits(limits=1):
+            run_oracle(oi, w.scale, w.block_size, None if full else pairs)
+    return run, sample_bytes
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The oracle as it stands, on the host, over the whole batch, repeated
+    until ``budget_s`` seconds of work (at least once)."""
+    run, sample_bytes = oracle_runner(w, w.num_seqs * w.num_heads)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 20:
+            break
+    return {"value": sample_bytes * reps / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"all {w.num_seqs} texts x {w.num_heads} heads of the batch-64 step, "
+                      f"{reps} run(s), {el:.1f} s, numpy fp64, BLAS limited to 1 thread"}
+
+
+def run_reference(args, world, rank):
+    """The oracle timed as the reference arm: each step is the first n
+    (text, head) pairs of the batch, n sized so warm-up + timed steps take
+    about two minutes in all."""
+    from paged_kv_cache_326_b200 import workloads as W
+    if rank != 0:
+        return 0
+    w = W.opt13b_batch64(device="cpu")
+    H = w.num_heads
+    probe, _ = oracle_runner(w, H)
+    t0 = time.perf_counter()
+    probe()
+    per_pair = (time.perf_counter() - t0) / H
+    budget = min(2.0, 120.0 / (args.steps + args.warmup))
+    n = int(max(1, min(w.num_seqs * H, budget / max(per_pair, 1e-6))))
+    run, sample_bytes = oracle_runner(w, n)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t0
+    ms = el / args.steps * 1e3
+    value = sample_bytes / (el / args.steps) / 1e9
+    desc = (f"first {n} (text, head) pairs of the {w.num_seqs}x{H} batch per step, "
+            f"numpy fp64, 1 BLAS thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+
+    import paged_kv_cache_326_b200 as P
+    from paged_kv_cache_326_b200 import workloads as W
+    P.lib()   # fails loudly if the library was not built
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    w = W.opt13b_batch64(seed=2 + rank, device=dev)
+    S, H, D = w.q.shape
+    eb = w.q.element_size()
+    lens = w.context_lens.tolist()
+    step_kv = kv_bytes(lens, H, D, eb)
+    decode_bytes = step_kv + 2 * S * H * D * eb + sum(4 * -(-L // w.block_size) for L in lens) + 4 * S
+    out = torch.empty_like(w.q)
+    ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+        P.pa_paged_attn_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                               w.scale, workspace=ws, status=status)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}: {P.pa_status_string(status.item())}")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+            ev[i][1].record(stream)
+            P.pa_paged_attn_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                   w.context_lens, w.scale, workspace=ws, status=status)
+            ev[i][2].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clk = clocks.summary()
+    total_ms = start.elapsed_time(stop)
+    decode_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
+    write_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+
+    # end to end: inputs from pinned host memory, output back to the host
+    hq = w.q.cpu().pin_memory()
+    hk = w.k.cpu().pin_memory()
+    hv = w.v.cpu().pin_memory()
+    hslot = w.slot_mapping.cpu().pin_memory()
+    htab = w.block_tables.cpu().pin_memory()
+    hlen = w.context_lens.cpu().pin_memory()
+    hout = torch.empty_like(hq).pin_memory()
+    dq, dk, dv = torch.empty_like(w.q), torch.empty_like(w.k), torch.empty_like(w.v)
+    dslot, dtab, dlen = (torch.empty_like(w.slot_mapping), torch.empty_like(w.block_tables),
+                         torch.empty_like(w.context_lens))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hslot, htab, hlen))
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        for d, h in ((dq, hq), (dk, hk), (dv, hv), (dslot, hslot), (dtab, htab), (dlen, hlen)):
+            d.copy_(h, non_blocking=True)
+        P.pa_kv_cache_write(dk, dv, w.k_cache, w.v_cache, dslot, status=status)
+        P.pa_paged_attn_decode(out, dq, w.k_cache, w.v_cache, dtab, dlen, w.scale, workspace=ws,
+                               status=status)
+        hout.copy_(out, non_blocking=True)
+
+    Ke = max(3, min(K, 1000))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_stop = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_stop) / Ke
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}: {P.pa_status_string(status.item())}")
+
+    ms_step = total_ms / K
+    times = torch.tensor([ms_step, e2e_ms, decode_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    ms_step, e2e_ms, decode_ms = times.tolist()
+
+    peak, peak_src = hbm_peak()
+    achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
+    value = world * step_kv / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "num_seqs": S, "num_heads": H, "head_dim": D,
+                   "block_size": w.block_size, "context_lens": "uniform [128, 2048], seed 2+rank",
+                   "num_blocks": w.num_blocks, "kv_bytes_per_step": step_kv,
+                   "l2": "inputs larger than L2 (KV read per step >> 126 MB)",
+                   "parallelism": f"independent batch per GPU x{world}"},
+        "decode_tokens_per_s": world * S / (ms_step * 1e-3),
+        "pct_of_nominal_8tbs": 100.0 * (value / world) / NOMINAL_HBM_GBS,
+        "kernel_ms": {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic_per_launch(),
+                     "kernel": "pa_paged_attn_decode (decode kernel + split reduce)",
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": decode_bytes},
+        "e2e": {"value": world * step_kv / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        w_cpu = w
+        line["cpu_baseline"] = cpu_baseline(w_cpu)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

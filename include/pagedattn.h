@@ -1,0 +1,211 @@
+/*
+ * pagedattn.h — C ABI of libpagedattn.so: paged decode attention, the KV-cache
+ * write, and a host-side block manager, for NVIDIA B200 (sm_100a).
+ *
+ * The method is PagedAttention as described in "The KV Cache and
+ * PagedAttention" (sections "Like Pages of Memory", "The Block Table",
+ * "Shared, Copied on Write") and "KV cache" ("How it works"): each text's keys
+ * and values are cut into fixed-size blocks that may sit anywhere in a pool;
+ * a per-text block table maps logical to physical blocks; in each generation
+ * step the new token's key and value are written into their slot and its
+ * query attends over every stored key of its text, the new one included.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer to tensor data is a DEVICE pointer owned by the caller,
+ *    except the block manager's arguments, which are HOST pointers.  The
+ *    library never allocates, frees or keeps device memory.
+ *  - Tensors are dense and row-major ("contiguous").  Element types are
+ *    IEEE fp16 or bfloat16 (pa_dtype), 2 bytes each.
+ *  - Pool layout: k_cache and v_cache are each
+ *        [num_blocks][num_heads][block_size][head_dim]
+ *    so the keys of one (block, head) pair are one contiguous
+ *    block_size*head_dim*2-byte tile.  Slot s is place s % block_size of
+ *    physical block s / block_size.
+ *  - Device calls are asynchronous on `stream` (NULL = the legacy default
+ *    stream).  A non-zero return means nothing was launched, except
+ *    PA_ERR_CUDA after a launch, which reports cudaGetLastError().
+ *  - Data errors that only the GPU can see (a table entry outside the pool, a
+ *    context length past the table, a slot past the pool, a wait that gave
+ *    up) are recorded in *d_status, a caller-owned device int32 that should be
+ *    zero before the call: the first error code seen is stored there (later
+ *    ones do not overwrite it).  d_status may be NULL.  No call traps,
+ *    asserts or aborts on bad data; offending reads and writes are skipped.
+ *  - Support: head_dim in {64, 128}; block_size in {4, 8, 16, 32};
+ *    num_seqs <= 4096; num_heads <= 1024.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                       /* same type as cudaStream_t */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = -1,        /* bad argument (null pointer, unsupported size, workspace too small) */
+  PA_ERR_CUDA = -2,           /* a CUDA runtime call failed */
+  PA_ERR_OUT_OF_BLOCKS = -3,  /* block manager: pool exhausted; state unchanged */
+  PA_ERR_NO_SEQ = -4,         /* block manager: unknown sequence id */
+  PA_ERR_EXISTS = -5,         /* block manager: sequence id already present */
+  PA_ERR_TABLE_FULL = -6,     /* block manager: a table does not fit max_blocks_per_seq */
+  PA_ERR_BAD_BLOCK = -7,      /* device: block table entry outside [0, num_blocks) */
+  PA_ERR_BAD_LEN = -8,        /* device: context length < 0 or > max_blocks_per_seq*block_size */
+  PA_ERR_BAD_SLOT = -9,       /* device: slot >= num_blocks*block_size */
+  PA_ERR_TIMEOUT = -10,       /* device: a bounded wait on a shared-memory barrier gave up */
+  PA_ERR_CORRUPT = -11        /* block manager: internal counts inconsistent */
+};
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* pa_status_string(int code);
+
+/*
+ * pa_kv_cache_write — store each new token's key and value in its slot.
+ *
+ * Definition: "KV cache", section "How it works" (the token's own key and
+ * value are written into the cache) and "The KV Cache and PagedAttention",
+ * section "One Token at a Time" (only the new token's key and value are
+ * computed; earlier ones are kept).  For t < num_tokens with slot_mapping[t]
+ * >= 0:  k_cache[slot/B][h][slot%B][:] = k[t][h][:]  (and v likewise), for
+ * every head h.  A pure copy: the stored bits equal the input bits.
+ *
+ *   k, v           [num_tokens][num_heads][head_dim]  dt, device, read
+ *   k_cache,v_cache pool, layout above, device, written at the given slots only
+ *   slot_mapping   [num_tokens] int64, device; a negative slot skips the token
+ *   num_blocks     pool size in blocks (bounds check: slot < num_blocks*B,
+ *                  else PA_ERR_BAD_SLOT in *d_status and the token is skipped)
+ *   d_status       nullable device int32 (see conventions)
+ * Two tokens with the same slot race; the pages never produce that.
+ * num_tokens == 0 is a no-op.  Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
+                      const int64_t* slot_mapping, int num_tokens, int num_heads, int head_dim,
+                      int block_size, int64_t num_blocks, pa_dtype dt, int32_t* d_status,
+                      pa_stream_t stream);
+
+/*
+ * pa_paged_attn_decode_workspace_size — bytes of device scratch that
+ * pa_paged_attn_decode needs for these sizes on the CURRENT device (it
+ * depends on the device's SM count).  Host only; allocates nothing.
+ * Returns 0 for unsupported sizes.
+ */
+size_t pa_paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
+                                           int block_size, int max_blocks_per_seq);
+
+/*
+ * pa_paged_attn_decode — decode-phase attention through block tables.
+ *
+ * Definition: "KV cache", section "How it works": the query of the new
+ * position is compared against the stored keys (the new key included) and the
+ * attention weights mix the stored values; "The KV Cache and PagedAttention",
+ * section "The Block Table": attention follows the block table and fetches
+ * each block's keys and values.  For text s with L = context_lens[s] tokens
+ * and every head h:
+ *     z_t = scale * sum_d q[s][h][d] * K_t[d],   t < L,
+ *     out[s][h][:] = sum_t softmax(z)_t * V_t[:],
+ * where token t lives in physical block block_tables[s][t / B], place t % B.
+ * Arithmetic: fp32 products and sums, online (running-max) softmax, result
+ * rounded to dt (round to nearest even).  L == 0 gives zeros.
+ *
+ *   out            [num_seqs][num_heads][head_dim] dt, device, written
+ *   q              [num_seqs][num_heads][head_dim] dt, device
+ *   k_cache,v_cache pool (layout above), device; only rows t < L are read
+ *   block_tables   [num_seqs][max_blocks_per_seq] int32, device; entries at or
+ *                  past ceil(L/B) are ignored
+ *   context_lens   [num_seqs] int32, device; counts the token written this
+ *                  step (call pa_kv_cache_write first, same stream)
+ *   scale          usually 1/sqrt(head_dim)
+ *   num_blocks     pool size in blocks (bounds check of table entries)
+ *   workspace      device scratch of at least
+ *                  pa_paged_attn_decode_workspace_size(...) bytes, 256-byte
+ *                  aligned; no initial contents needed; must not be shared by
+ *                  calls that may run at the same time
+ *   d_status       nullable device int32 (see conventions)
+ * Work is split over all SMs in equal runs of 16-token (head_dim 128) or
+ * 32-token (head_dim 64) chunks; a text whose run spans several warps is
+ * merged with a log-sum-exp reduction (a second kernel on the same stream).
+ * For fixed inputs, sizes and device the result is bitwise reproducible.
+ * Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, float scale,
+                         int num_seqs, int num_heads, int head_dim, int block_size,
+                         int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt,
+                         void* workspace, size_t workspace_bytes, int32_t* d_status,
+                         pa_stream_t stream);
+
+/*
+ * Tuning and test options (process-wide, not thread-safe; set before use).
+ *   PA_OPT_WAIT_LIMIT_NS  bound on each shared-memory barrier wait in the
+ *                         decode kernel, in ns (default 1e9).  A negative
+ *                         value makes every wait give up at once, which
+ *                         exercises the PA_ERR_TIMEOUT path: the kernel then
+ *                         drains its copies in flight (bounded by 1 s) and
+ *                         returns with *d_status = PA_ERR_TIMEOUT.
+ *   PA_OPT_DECODE_WARPS   number of working warps of the decode kernel
+ *                         (0 = all SMs, the default).  1 gives a single-pass
+ *                         run in which no text is split.
+ * Returns PA_OK or PA_ERR_INVALID for an unknown key.
+ */
+enum { PA_OPT_WAIT_LIMIT_NS = 1, PA_OPT_DECODE_WARPS = 2 };
+int pa_set_option(int key, int64_t value);
+
+/* ------------------------------------------------------------------------ */
+/* Host block manager ("The KV Cache and PagedAttention", sections "The     */
+/* Block Table", "Shared, Copied on Write", "When Memory Runs Out").  Pure  */
+/* host code; all pointers are host pointers; not thread-safe per handle.   */
+/* ------------------------------------------------------------------------ */
+typedef struct pa_bm pa_bm;
+
+/* A pool of num_blocks blocks of block_size tokens.  The free list starts in
+ * block order (shuffle_seed == 0) or in a seeded random order; blocks are
+ * taken from its front and returned to its back.  NULL on bad arguments. */
+pa_bm* pa_bm_create(int64_t num_blocks, int block_size, uint64_t shuffle_seed);
+void pa_bm_destroy(pa_bm* bm);
+
+/* New text whose first num_tokens tokens (the prompt) are stored at once:
+ * ceil(num_tokens / B) fresh blocks.  All or nothing. */
+int pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int num_tokens);
+
+/* child shares every block of parent; each block's count rises by one. */
+int pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child);
+
+/* Room for the text's next token.  A fresh block is taken only when the last
+ * block is full ("a new block only when the earlier ones are full").  If the
+ * last block is partial and shared, it is copied first: *cow_src/*cow_dst
+ * receive the pair (the caller copies the block's rows on the device before
+ * writing), the original's count drops by one; otherwise both are -1.
+ * *slot receives the token's slot.  All or nothing. */
+int pa_bm_append_slot(pa_bm* bm, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                      int32_t* cow_dst);
+
+/* The text is done: each block's count drops by one; blocks that reach zero
+ * return to the free list, in table order. */
+int pa_bm_free_seq(pa_bm* bm, int64_t seq_id);
+
+int64_t pa_bm_num_free(const pa_bm* bm);
+/* Reference count of a block, or PA_ERR_INVALID for an id outside the pool. */
+int pa_bm_refcount(const pa_bm* bm, int32_t block);
+/* Tokens stored for the text, or a negative status. */
+int64_t pa_bm_num_tokens(const pa_bm* bm, int64_t seq_id);
+
+/* Writes block_tables[n][max_blocks_per_seq] (int32, -1 past each text's last
+ * block) and context_lens[n] (token counts) into caller host buffers, in the
+ * order of seq_ids.  PA_ERR_TABLE_FULL if a table is longer than
+ * max_blocks_per_seq; nothing is written on error. */
+int pa_bm_export(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* block_tables,
+                 int max_blocks_per_seq, int32_t* context_lens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

@@ -1,0 +1,28 @@
+"""Byte accounting for the KV cache.
+
+"The KV Cache and PagedAttention", section "800 KB a Token": each token keeps a
+key and a value in every layer, so one token costs
+2 x hidden x layers x bytes-per-number (OPT-13B: 2 x 5,120 x 40 x 2 = 819,200
+bytes).  Section "What Came After": when several heads share one set of keys
+and values, only the shared sets count (hidden = kv_heads x head_dim).
+"""
+from __future__ import annotations
+
+from typing import Iterable
+
+
+def kv_bytes_per_token(num_kv_heads: int, head_dim: int, num_layers: int, elem_bytes: int) -> int:
+    return 2 * num_kv_heads * head_dim * num_layers * elem_bytes
+
+
+def decode_kv_bytes(context_lens: Iterable[int], num_kv_heads: int, head_dim: int,
+                    elem_bytes: int) -> int:
+    """K and V bytes that one decode step of one layer must read: every
+    stored token of every text, keys and values (unfilled places excluded)."""
+    return sum(int(L) for L in context_lens) * kv_bytes_per_token(num_kv_heads, head_dim, 1,
+                                                                  elem_bytes)
+
+
+def tokens_that_fit(cache_bytes: int, num_kv_heads: int, head_dim: int, num_layers: int,
+                    elem_bytes: int) -> int:
+    return cache_bytes // kv_bytes_per_token(num_kv_heads, head_dim, num_layers, elem_bytes)

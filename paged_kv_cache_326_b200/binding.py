@@ -1,0 +1,279 @@
+"""Python binding of libpagedattn.so (ctypes): argument marshalling only.
+
+Every function carries the name of the C entry point it calls (see
+include/pagedattn.h for the definitions).  Tensors are torch tensors; the
+binding checks their device, dtype and contiguity, reads the sizes from their
+shapes and passes raw pointers and the current CUDA stream.  All arithmetic
+runs in the library's CUDA kernels.  There is no fallback: if the shared
+library is missing, loading it raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Dict, Optional, Sequence, Tuple
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
+
+PA_OK = 0
+PA_ERR_INVALID = -1
+PA_ERR_CUDA = -2
+PA_ERR_OUT_OF_BLOCKS = -3
+PA_ERR_NO_SEQ = -4
+PA_ERR_EXISTS = -5
+PA_ERR_TABLE_FULL = -6
+PA_ERR_BAD_BLOCK = -7
+PA_ERR_BAD_LEN = -8
+PA_ERR_BAD_SLOT = -9
+PA_ERR_TIMEOUT = -10
+PA_ERR_CORRUPT = -11
+
+PA_F16 = 0
+PA_BF16 = 1
+
+PA_OPT_WAIT_LIMIT_NS = 1
+PA_OPT_DECODE_WARPS = 2
+
+_KIND = {PA_ERR_INVALID: "invalid", PA_ERR_CUDA: "cuda", PA_ERR_OUT_OF_BLOCKS: "out_of_blocks",
+         PA_ERR_NO_SEQ: "no_seq", PA_ERR_EXISTS: "exists", PA_ERR_TABLE_FULL: "table_full",
+         PA_ERR_CORRUPT: "corrupt"}
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        self.kind = _KIND.get(code, "error")
+        super().__init__(f"{where}: {pa_status_string(code)} ({code})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+_vp, _i32, _i64, _u64, _f32, _sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                     ctypes.c_uint64, ctypes.c_float, ctypes.c_size_t)
+
+_SIGNATURES = {
+    "pa_status_string": (ctypes.c_char_p, [_i32]),
+    "pa_set_option": (_i32, [_i32, _i64]),
+    "pa_kv_cache_write": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i32,
+                                 _vp, _vp]),
+    "pa_paged_attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "pa_paged_attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _i32,
+                                    _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
+    "pa_bm_create": (_vp, [_i64, _i32, _u64]),
+    "pa_bm_destroy": (None, [_vp]),
+    "pa_bm_add_seq": (_i32, [_vp, _i64, _i32]),
+    "pa_bm_fork": (_i32, [_vp, _i64, _i64]),
+    "pa_bm_append_slot": (_i32, [_vp, _i64, ctypes.POINTER(_i64), ctypes.POINTER(ctypes.c_int32),
+                                 ctypes.POINTER(ctypes.c_int32)]),
+    "pa_bm_free_seq": (_i32, [_vp, _i64]),
+    "pa_bm_num_free": (_i64, [_vp]),
+    "pa_bm_refcount": (_i32, [_vp, ctypes.c_int32]),
+    "pa_bm_num_tokens": (_i64, [_vp, _i64]),
+    "pa_bm_export": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (built by ``python -m paged_kv_cache_326_b200.build``)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                                      "`python -m paged_kv_cache_326_b200.build`")
+                l = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in _SIGNATURES.items():
+                    fn = getattr(l, name)
+                    fn.restype = res
+                    fn.argtypes = args
+                _lib = l
+    return _lib
+
+
+def _check(code: int, where: str) -> None:
+    if code != PA_OK:
+        raise PagedAttnError(code, where)
+
+
+def pa_status_string(code: int) -> str:
+    return lib().pa_status_string(int(code)).decode()
+
+
+def pa_set_option(key: int, value: int) -> None:
+    _check(lib().pa_set_option(int(key), int(value)), "pa_set_option")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: fp16 or bf16")
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream, device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _status_ptr(status: Optional[torch.Tensor]) -> Optional[int]:
+    if status is None:
+        return None
+    return _cuda(status, "status", torch.int32)
+
+
+def pa_kv_cache_write(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
+                      v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                      status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """k, v: [T][H][D]; caches [N][H][B][D]; slot_mapping [T] int64."""
+    T, H, D = k.shape
+    N, H2, B, D2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
+        raise ValueError("shape mismatch between k/v and the caches")
+    if slot_mapping.shape != (T,):
+        raise ValueError("slot_mapping must be [num_tokens]")
+    for t in (v, k_cache, v_cache):
+        if t.dtype != k.dtype:
+            raise TypeError("k, v and the caches must share a dtype")
+    code = lib().pa_kv_cache_write(
+        _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(slot_mapping, "slot_mapping", torch.int64), T, H, D, B, N, _dtype_code(k),
+        _status_ptr(status), _stream(stream, k.device))
+    _check(code, "pa_kv_cache_write")
+
+
+def pa_paged_attn_decode_workspace_size(num_seqs: int, num_heads: int, head_dim: int,
+                                        block_size: int, max_blocks_per_seq: int) -> int:
+    return int(lib().pa_paged_attn_decode_workspace_size(num_seqs, num_heads, head_dim,
+                                                          block_size, max_blocks_per_seq))
+
+
+_ws_cache: Dict[Tuple[int, int], torch.Tensor] = {}
+
+
+def workspace_for(q: torch.Tensor, block_size: int, max_blocks_per_seq: int) -> torch.Tensor:
+    """A cached device workspace big enough for these sizes (allocated by
+    torch, never by the library)."""
+    S, H, D = q.shape
+    need = pa_paged_attn_decode_workspace_size(S, H, D, block_size, max_blocks_per_seq)
+    if need == 0:
+        raise PagedAttnError(PA_ERR_INVALID, "pa_paged_attn_decode_workspace_size")
+    key = (q.device.index if q.device.index is not None else torch.cuda.current_device(), need)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def pa_paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                         v_cache: torch.Tensor, block_tables: torch.Tensor,
+                         context_lens: torch.Tensor, scale: float,
+                         workspace: Optional[torch.Tensor] = None,
+                         status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out, q: [S][H][D]; caches [N][H][B][D]; block_tables [S][max_blocks]
+    int32; context_lens [S] int32."""
+    S, H, D = q.shape
+    N, H2, B, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S][max_blocks], context_lens [S]")
+    for t in (out, k_cache, v_cache):
+        if t.dtype != q.dtype:
+            raise TypeError("q, out and the caches must share a dtype")
+    MB = block_tables.shape[1]
+    if workspace is None:
+        workspace = workspace_for(q, B, MB)
+    code = lib().pa_paged_attn_decode(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(context_lens, "context_lens", torch.int32), float(scale), S, H, D, B, MB, N,
+        _dtype_code(q), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _status_ptr(status), _stream(stream, q.device))
+    _check(code, "pa_paged_attn_decode")
+    return out
+
+
+# aliases under the names the method's description uses
+kv_cache_write = pa_kv_cache_write
+paged_attn_decode = pa_paged_attn_decode
+
+
+class BlockManager:
+    """Host block manager (pa_bm_* in the C ABI)."""
+
+    def __init__(self, num_blocks: int, block_size: int, shuffle_seed: int = 0):
+        self._h = lib().pa_bm_create(int(num_blocks), int(block_size), int(shuffle_seed))
+        if not self._h:
+            raise PagedAttnError(PA_ERR_INVALID, "pa_bm_create")
+        self.num_blocks = int(num_blocks)
+        self.block_size = int(block_size)
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib().pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, seq_id: int, num_tokens: int) -> None:
+        _check(lib().pa_bm_add_seq(self._h, int(seq_id), int(num_tokens)), "pa_bm_add_seq")
+
+    def fork(self, parent: int, child: int) -> None:
+        _check(lib().pa_bm_fork(self._h, int(parent), int(child)), "pa_bm_fork")
+
+    def append_slot(self, seq_id: int) -> Tuple[int, int, int]:
+        slot = ctypes.c_int64()
+        src = ctypes.c_int32()
+        dst = ctypes.c_int32()
+        _check(lib().pa_bm_append_slot(self._h, int(seq_id), ctypes.byref(slot), ctypes.byref(src),
+                                       ctypes.byref(dst)), "pa_bm_append_slot")
+        return slot.value, src.value, dst.value
+
+    def free_seq(self, seq_id: int) -> None:
+        _check(lib().pa_bm_free_seq(self._h, int(seq_id)), "pa_bm_free_seq")
+
+    def num_free(self) -> int:
+        return int(lib().pa_bm_num_free(self._h))
+
+    def refcount(self, block: int) -> int:
+        r = lib().pa_bm_refcount(self._h, int(block))
+        if r < 0:
+            raise PagedAttnError(r, "pa_bm_refcount")
+        return r
+
+    def num_tokens(self, seq_id: int) -> int:
+        r = int(lib().pa_bm_num_tokens(self._h, int(seq_id)))
+        if r < 0:
+            raise PagedAttnError(r, "pa_bm_num_tokens")
+        return r
+
+    def export(self, seq_ids: Sequence[int], max_blocks_per_seq: int):
+        """(block_tables [n][max_blocks] int32, context_lens [n] int32) as CPU tensors."""
+        n = len(seq_ids)
+        ids = torch.tensor(list(seq_ids), dtype=torch.int64)
+        tables = torch.empty((n, max_blocks_per_seq), dtype=torch.int32)
+        lens = torch.empty(n, dtype=torch.int32)
+        _check(lib().pa_bm_export(self._h, ids.data_ptr(), n, tables.data_ptr(),
+                                  int(max_blocks_per_seq), lens.data_ptr()), "pa_bm_export")
+        return tables, lens

@@ -1,0 +1,124 @@
+// C ABI of libpagedattn.so (declared and documented in include/pagedattn.h):
+// argument checks, then the launchers in kv_cache_write.cu and
+// paged_attn_decode.cu.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "kernels.h"
+#include "pagedattn.h"
+
+namespace {
+
+std::atomic<int64_t> g_wait_limit_ns{1000000000};
+std::atomic<int64_t> g_decode_warps{0};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(int num_heads, int head_dim, int block_size) {
+  return num_heads >= 1 && num_heads <= 1024 && (head_dim == 64 || head_dim == 128) &&
+         (block_size == 4 || block_size == 8 || block_size == 16 || block_size == 32);
+}
+
+int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return PA_OK;
+  if (e == cudaErrorInvalidValue) return PA_ERR_INVALID;
+  return PA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(int code) {
+  switch (code) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID: return "invalid argument";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_OUT_OF_BLOCKS: return "out of blocks";
+    case PA_ERR_NO_SEQ: return "unknown sequence";
+    case PA_ERR_EXISTS: return "sequence exists";
+    case PA_ERR_TABLE_FULL: return "block table longer than max_blocks_per_seq";
+    case PA_ERR_BAD_BLOCK: return "block table entry outside the pool";
+    case PA_ERR_BAD_LEN: return "context length outside [0, max_blocks_per_seq*block_size]";
+    case PA_ERR_BAD_SLOT: return "slot outside the pool";
+    case PA_ERR_TIMEOUT: return "bounded wait gave up";
+    case PA_ERR_CORRUPT: return "block manager counts inconsistent";
+    default: return "unknown status";
+  }
+}
+
+int pa_set_option(int key, int64_t value) {
+  switch (key) {
+    case PA_OPT_WAIT_LIMIT_NS: g_wait_limit_ns = value; return PA_OK;
+    case PA_OPT_DECODE_WARPS:
+      if (value < 0 || value > (int64_t{1} << 24)) return PA_ERR_INVALID;
+      g_decode_warps = value;
+      return PA_OK;
+    default: return PA_ERR_INVALID;
+  }
+}
+
+int pa_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
+                      const int64_t* slot_mapping, int num_tokens, int num_heads, int head_dim,
+                      int block_size, int64_t num_blocks, pa_dtype dt, int32_t* d_status,
+                      pa_stream_t stream) {
+  if (num_tokens < 0 || !shape_ok(num_heads, head_dim, block_size) || num_blocks <= 0 ||
+      (dt != PA_F16 && dt != PA_BF16))
+    return PA_ERR_INVALID;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  return from_cuda(pa::launch_kv_cache_write(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                             num_heads, head_dim, block_size, num_blocks,
+                                             d_status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t pa_paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
+                                           int block_size, int max_blocks_per_seq) {
+  return pa::decode_workspace_bytes(num_seqs, num_heads, head_dim, block_size,
+                                    max_blocks_per_seq, g_decode_warps.load());
+}
+
+int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, float scale,
+                         int num_seqs, int num_heads, int head_dim, int block_size,
+                         int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt,
+                         void* workspace, size_t workspace_bytes, int32_t* d_status,
+                         pa_stream_t stream) {
+  if (num_seqs == 0) return PA_OK;
+  if (!pa::decode_sizes_supported(num_seqs, num_heads, head_dim, block_size,
+                                  max_blocks_per_seq) ||
+      num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16))
+    return PA_ERR_INVALID;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return PA_ERR_INVALID;
+  pa::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.scale = scale;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.is_bf16 = dt == PA_BF16;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  a.status = d_status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.forced_warps = g_decode_warps.load();
+  return from_cuda(pa::launch_paged_attn_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,179 @@
+// Host block manager: free list, per-block reference counts, copy-on-write.
+//
+// "The KV Cache and PagedAttention": a text's logical blocks map to physical
+// blocks anywhere in the pool (section "Like Pages of Memory"); a new block is
+// handed out only when all the text's earlier blocks are full and a finished
+// text's blocks go back to the pool (section "The Block Table"); samples of one
+// prompt share its blocks, each block counting its users, and a text about to
+// write into a shared block first gets a copy (section "Shared, Copied on
+// Write"); a text holds all its blocks or none (section "When Memory Runs
+// Out"), so every operation here either succeeds completely or changes nothing.
+#include <cstdint>
+#include <deque>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "pagedattn.h"
+
+struct pa_bm {
+  int64_t num_blocks;
+  int block_size;
+  std::deque<int32_t> free_list;                 // take front, return back
+  std::vector<int32_t> ref;                      // texts using each block
+  struct Seq {
+    std::vector<int32_t> blocks;
+    int64_t tokens;
+  };
+  std::unordered_map<int64_t, Seq> seqs;
+};
+
+namespace {
+
+// SplitMix64 (Steele, Lea, Flood, "Fast splittable pseudorandom number
+// generators", OOPSLA 2014): drives the Fisher-Yates shuffle of the initial
+// free list when a seed is given.
+uint64_t splitmix64(uint64_t& x) {
+  uint64_t z = (x += 0x9E3779B97F4A7C15ull);
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+int32_t take(pa_bm* bm) {
+  int32_t b = bm->free_list.front();
+  bm->free_list.pop_front();
+  bm->ref[b] = 1;
+  return b;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_bm* pa_bm_create(int64_t num_blocks, int block_size, uint64_t shuffle_seed) {
+  if (num_blocks <= 0 || num_blocks > INT32_MAX || block_size <= 0) return nullptr;
+  pa_bm* bm = new (std::nothrow) pa_bm();
+  if (!bm) return nullptr;
+  bm->num_blocks = num_blocks;
+  bm->block_size = block_size;
+  std::vector<int32_t> order(static_cast<size_t>(num_blocks));
+  for (int64_t i = 0; i < num_blocks; ++i) order[i] = static_cast<int32_t>(i);
+  if (shuffle_seed != 0) {
+    uint64_t st = shuffle_seed;
+    for (int64_t i = num_blocks - 1; i > 0; --i) {
+      int64_t j = static_cast<int64_t>(splitmix64(st) % static_cast<uint64_t>(i + 1));
+      std::swap(order[i], order[j]);
+    }
+  }
+  bm->free_list.assign(order.begin(), order.end());
+  bm->ref.assign(static_cast<size_t>(num_blocks), 0);
+  return bm;
+}
+
+void pa_bm_destroy(pa_bm* bm) { delete bm; }
+
+int pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int num_tokens) {
+  if (!bm || num_tokens < 0) return PA_ERR_INVALID;
+  if (bm->seqs.count(seq_id)) return PA_ERR_EXISTS;
+  int64_t need = (static_cast<int64_t>(num_tokens) + bm->block_size - 1) / bm->block_size;
+  if (static_cast<int64_t>(bm->free_list.size()) < need) return PA_ERR_OUT_OF_BLOCKS;
+  pa_bm::Seq s;
+  s.tokens = num_tokens;
+  s.blocks.reserve(static_cast<size_t>(need));
+  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(take(bm));
+  bm->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+int pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child) {
+  if (!bm) return PA_ERR_INVALID;
+  auto it = bm->seqs.find(parent);
+  if (it == bm->seqs.end()) return PA_ERR_NO_SEQ;
+  if (bm->seqs.count(child)) return PA_ERR_EXISTS;
+  pa_bm::Seq copy = it->second;
+  for (int32_t b : copy.blocks) bm->ref[b] += 1;
+  bm->seqs.emplace(child, std::move(copy));
+  return PA_OK;
+}
+
+int pa_bm_append_slot(pa_bm* bm, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                      int32_t* cow_dst) {
+  if (!bm || !slot || !cow_src || !cow_dst) return PA_ERR_INVALID;
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) return PA_ERR_NO_SEQ;
+  pa_bm::Seq& s = it->second;
+  const int64_t place = s.tokens % bm->block_size;
+  int32_t src = -1, dst = -1;
+  if (place == 0) {
+    if (bm->free_list.empty()) return PA_ERR_OUT_OF_BLOCKS;
+    s.blocks.push_back(take(bm));
+  } else {
+    int32_t last = s.blocks.back();
+    if (bm->ref[last] > 1) {
+      if (bm->free_list.empty()) return PA_ERR_OUT_OF_BLOCKS;
+      dst = take(bm);
+      bm->ref[last] -= 1;
+      s.blocks.back() = dst;
+      src = last;
+    }
+  }
+  s.tokens += 1;
+  *slot = static_cast<int64_t>(s.blocks.back()) * bm->block_size + place;
+  *cow_src = src;
+  *cow_dst = dst;
+  return PA_OK;
+}
+
+int pa_bm_free_seq(pa_bm* bm, int64_t seq_id) {
+  if (!bm) return PA_ERR_INVALID;
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) return PA_ERR_NO_SEQ;
+  for (int32_t b : it->second.blocks)
+    if (bm->ref[b] <= 0) return PA_ERR_CORRUPT;
+  for (int32_t b : it->second.blocks) {
+    if (--bm->ref[b] == 0) bm->free_list.push_back(b);
+  }
+  bm->seqs.erase(it);
+  return PA_OK;
+}
+
+int64_t pa_bm_num_free(const pa_bm* bm) {
+  return bm ? static_cast<int64_t>(bm->free_list.size()) : PA_ERR_INVALID;
+}
+
+int pa_bm_refcount(const pa_bm* bm, int32_t block) {
+  if (!bm || block < 0 || block >= bm->num_blocks) return PA_ERR_INVALID;
+  return bm->ref[block];
+}
+
+int64_t pa_bm_num_tokens(const pa_bm* bm, int64_t seq_id) {
+  if (!bm) return PA_ERR_INVALID;
+  auto it = bm->seqs.find(seq_id);
+  return it == bm->seqs.end() ? PA_ERR_NO_SEQ : it->second.tokens;
+}
+
+int pa_bm_export(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* block_tables,
+                 int max_blocks_per_seq, int32_t* context_lens) {
+  if (!bm || n < 0 || max_blocks_per_seq <= 0 || (n > 0 && (!seq_ids || !block_tables ||
+                                                             !context_lens)))
+    return PA_ERR_INVALID;
+  for (int i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end()) return PA_ERR_NO_SEQ;
+    if (static_cast<int64_t>(it->second.blocks.size()) > max_blocks_per_seq)
+      return PA_ERR_TABLE_FULL;
+    if (it->second.tokens > INT32_MAX) return PA_ERR_INVALID;
+  }
+  for (int i = 0; i < n; ++i) {
+    const pa_bm::Seq& s = bm->seqs.find(seq_ids[i])->second;
+    int32_t* row = block_tables + static_cast<int64_t>(i) * max_blocks_per_seq;
+    size_t k = 0;
+    for (; k < s.blocks.size(); ++k) row[k] = s.blocks[k];
+    for (; k < static_cast<size_t>(max_blocks_per_seq); ++k) row[k] = -1;
+    context_lens[i] = static_cast<int32_t>(s.tokens);
+  }
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// Internal launcher declarations shared by the C-ABI layer and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace pa {
+
+cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
+                                  const int64_t* slot_mapping, int num_tokens, int num_heads,
+                                  int head_dim, int block_size, int64_t num_blocks,
+                                  int32_t* status, cudaStream_t stream);
+
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float scale;
+  int num_seqs;
+  int num_heads;
+  int head_dim;
+  int block_size;
+  int max_blocks_per_seq;
+  int64_t num_blocks;
+  int is_bf16;
+  void* workspace;
+  size_t workspace_bytes;
+  int32_t* status;
+  int64_t wait_limit_ns;
+  int64_t forced_warps;  // 0 = fill the device
+};
+
+bool decode_sizes_supported(int num_seqs, int num_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq);
+
+// Size of the decode workspace for these sizes on the current device, or 0
+// if the sizes are unsupported.
+size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int block_size,
+                              int max_blocks_per_seq, int64_t forced_warps);
+
+// Launches the decode kernel and the split reduce on `stream`.
+// Returns cudaErrorInvalidValue for unsupported sizes or a short workspace.
+cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace pa

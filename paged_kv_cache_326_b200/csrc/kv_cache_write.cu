@@ -1,0 +1,65 @@
+// kv_cache_write: scatter each new token's key and value into its slot.
+//
+// "KV cache", section "How it works": the new position's key and value are
+// written into the cache; "The KV Cache and PagedAttention", section "One Token
+// at a Time": only the new token's key and value are computed each iteration.
+//
+// One thread moves one 16-byte vector of K and the matching one of V.  A
+// token's H*D elements are contiguous in the input and land in H tiles of the
+// pool (one per head, stride block_size*head_dim), each a contiguous row of
+// head_dim elements, so both the loads and the stores are full 16-byte
+// transactions and consecutive threads touch consecutive bytes of a row.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace pa {
+
+__global__ void __launch_bounds__(256)
+kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                      uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                      const int64_t* __restrict__ slot_mapping, int num_tokens, int num_heads,
+                      int vec_per_row, int block_size, int64_t num_slots, int32_t* status) {
+  const int64_t per_token = static_cast<int64_t>(num_heads) * vec_per_row;
+  const int64_t total = per_token * num_tokens;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int64_t r = i - t * per_token;
+    const int64_t h = r / vec_per_row;
+    const int64_t c = r - h * vec_per_row;
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (r == 0) set_status(status, -9 /* PA_ERR_BAD_SLOT */);
+      continue;
+    }
+    const int64_t blk = slot / block_size;
+    const int64_t place = slot - blk * block_size;
+    const int64_t dst = ((blk * num_heads + h) * block_size + place) * vec_per_row + c;
+    k_cache[dst] = __ldg(k + i);
+    v_cache[dst] = __ldg(v + i);
+  }
+}
+
+cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
+                                  const int64_t* slot_mapping, int num_tokens, int num_heads,
+                                  int head_dim, int block_size, int64_t num_blocks,
+                                  int32_t* status, cudaStream_t stream) {
+  const int vec_per_row = head_dim / 8;  // 8 two-byte elements per 16 bytes
+  const int64_t total = static_cast<int64_t>(num_tokens) * num_heads * vec_per_row;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > (1 << 20)) blocks = 1 << 20;
+  kv_cache_write_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_heads, vec_per_row, block_size,
+      num_blocks * block_size, status);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

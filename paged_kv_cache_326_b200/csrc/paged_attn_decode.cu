@@ -1,0 +1,670 @@
+// paged_attn_decode: decode-phase attention through block tables, and the
+// log-sum-exp merge of partial results.
+//
+// What it computes ("KV cache", section "How it works"; "The KV Cache and
+// PagedAttention", section "The Block Table"): for text s and head h, the new
+// query q[s][h] attends over the L_s stored keys, the new one included; token
+// t lives in physical block block_tables[s][t / B] at place t % B:
+//     out[s][h] = sum_t softmax_t(scale * q . K_t) * V_t.
+//
+// How (B200 design, not the pages' A100 kernel):
+//  * The work is HBM-bound (about one flop per byte), so no tensor cores: each
+//    (text, head) is a GEMV over its keys and another over its values.
+//  * The unit of work is a CHUNK: CH consecutive tokens of one (text, head)
+//    (CH = 16 at head_dim 128, 32 at head_dim 64, so a chunk's keys are 4 KB
+//    and keys + values 8 KB).  All chunks of all (text, head) pairs are laid
+//    out in one flat order (text-major, then head, then chunk) and cut into
+//    equal runs, one per warp of a persistent grid that fills every SM.  So
+//    long and short texts alike keep all 148 SMs busy to the end, with no
+//    tail wave.  A (text, head) whose chunks fall into several warps' runs
+//    produces one partial result per warp (running max m, sum l, unnormalised
+//    output o), merged by split_reduce_kernel; one that falls inside a single
+//    run is finished in place.
+//  * Each warp is its own pipeline: lane 0 issues bulk (TMA) copies of the
+//    chunk's key rows and value rows, straight from their physical blocks,
+//    into a ring of STAGES shared-memory stages, each with an mbarrier that
+//    counts the bytes landed; all 32 lanes consume.  The issue runs STAGES
+//    chunks ahead and crosses (text, head) boundaries, so the copy engine
+//    never idles at a boundary.  Only valid rows are copied: the unfilled tail
+//    of a text's last block is never read from HBM.
+//  * Block-table entries and context lengths for the next 32 chunks are
+//    fetched one per lane, 32 chunks before they are needed, and handed to
+//    the issuing lane with shuffles, so no table lookup sits on the critical
+//    path.
+//  * Dot products: a key row of head_dim elements is read by D/8 lanes as
+//    16-byte vectors and reduced with shuffles; the softmax is the online
+//    (running-max) form in fp32, in base 2 with log2(e) folded into the scale.
+//  * Every wait is bounded; a wait that gives up records PA_ERR_TIMEOUT,
+//    drains the copies in flight (bounded too) and returns.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <utility>
+
+#include "dtype.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace pa {
+
+namespace {
+
+constexpr int kDecodeWarps = 4;   // warps per CTA
+constexpr int kDecodeStages = 3;  // ring depth per warp
+constexpr int kMaxSeqs = 4096;
+constexpr int kHeaderInts = 4;    // total chunks, chunks per warp, warps, spare
+constexpr int kDrainLimitNs = 1000000000;
+
+__host__ __device__ constexpr int chunk_tokens(int D) { return 2048 / D; }
+__host__ __device__ constexpr int stage_bytes(int D) { return 2 * 4096 + 2 * D + 128; }
+__host__ __device__ constexpr int warp_area_bytes(int D, int stages) { return stages * stage_bytes(D) + 128; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t header_bytes(int num_seqs) {
+  return align_up(sizeof(int32_t) * (kHeaderInts + num_seqs + 1), 256);
+}
+
+struct DecodeParams {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float qk_scale_log2;
+  int num_seqs;
+  int num_heads;
+  int max_blocks_per_seq;
+  int64_t num_blocks;
+  int num_work_warps;
+  int32_t* header;
+  float* records;
+  int32_t* status;
+  int64_t wait_limit_ns;
+};
+
+// Per-lane look-ahead entry: where flat chunk (run start + position) lives.
+template <int NB>
+struct Lookahead {
+  int s, h, j, len;  // len is the raw context length (clamped at use)
+  int blk[NB];
+};
+
+}  // namespace
+
+template <typename T, int D, int B, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32)
+paged_decode_kernel(const DecodeParams p) {
+  constexpr int CH = chunk_tokens(D);        // tokens per chunk
+  constexpr int LPT = D / 8;                 // lanes per token row (16-byte vectors)
+  constexpr int TPI = 32 / LPT;              // token rows per warp-wide load
+  constexpr int ITERS = CH / TPI;            // loads per chunk (8)
+  constexpr int NB = CH >= B ? CH / B : 1;   // physical blocks a chunk touches
+  constexpr int TILE = CH * D;               // elements of K (or V) per chunk
+  constexpr int STRIDE = stage_bytes(D);
+  constexpr int AREA = warp_area_bytes(D, STAGES);
+  static_assert(CH % TPI == 0 && (CH % B == 0 || B % CH == 0), "shape");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  int32_t* prefix = reinterpret_cast<int32_t*>(smem + WARPS * AREA);
+  __shared__ int32_t warp_tot[WARPS];
+
+  const int S = p.num_seqs;
+  const int H = p.num_heads;
+  const int cap = p.max_blocks_per_seq * B;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+
+  // ---- prologue: prefix[s] = H * (chunks of texts before s), block-wide scan
+  {
+    const int nthr = WARPS * 32;
+    const int per = (S + nthr - 1) / nthr;
+    const int s0 = min(S, tid * per), s1 = min(S, s0 + per);
+    int local = 0;
+    for (int s = s0; s < s1; ++s) {
+      int L = __ldg(p.context_lens + s);
+      if (L < 0 || L > cap) {
+        if (blockIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
+        L = min(max(L, 0), cap);
+      }
+      local += (L + CH - 1) / CH;
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    int run = before + incl - local;
+    for (int s = s0; s < s1; ++s) {
+      int L = min(max(__ldg(p.context_lens + s), 0), cap);
+      prefix[s] = run * H;
+      run += (L + CH - 1) / CH;
+    }
+    if (tid == nthr - 1) prefix[S] = run * H;
+    __syncthreads();
+  }
+  const int total = prefix[S];
+  const int W = p.num_work_warps;
+  const int cpw = (total + W - 1) / W;
+  if (blockIdx.x == 0) {
+    if (tid == 0) {
+      p.header[0] = total;
+      p.header[1] = cpw;
+      p.header[2] = W;
+      p.header[3] = 0;
+    }
+    for (int s = tid; s <= S; s += WARPS * 32) p.header[kHeaderInts + s] = prefix[s];
+  }
+
+  const int w = blockIdx.x * WARPS + warp;
+  if (w >= W || total == 0) return;
+  const int c0 = w * cpw;
+  const int c1 = min(total, c0 + cpw);
+  if (c0 >= c1) return;
+  const int n = c1 - c0;
+
+  uint8_t* area = smem + warp * AREA;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(area + STAGES * STRIDE);
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  const uint64_t policy = l2_evict_first_policy();
+  const T* __restrict__ kc = static_cast<const T*>(p.k_cache);
+  const T* __restrict__ vc = static_cast<const T*>(p.v_cache);
+  const T* __restrict__ qg = static_cast<const T*>(p.q);
+
+  int step = 1;
+  while (step * 2 <= S) step *= 2;
+
+  // Where flat chunk c0 + pos lives.  Reads only shared memory before issuing
+  // its global loads, whose results are not used for 32 - STAGES chunks.
+  auto lookahead = [&](int pos) {
+    Lookahead<NB> e;
+    const int c = c0 + min(pos, n - 1);
+    int s = 0;
+    for (int st = step; st > 0; st >>= 1)
+      if (s + st < S && prefix[s + st] <= c) s += st;
+    const int seg0 = prefix[s];
+    const int ns = (prefix[s + 1] - seg0) / H;
+    const int within = c - seg0;
+    const int h = within / ns;
+    const int j = within - h * ns;
+    e.s = s;
+    e.h = h;
+    e.j = j;
+    e.len = __ldg(p.context_lens + s);
+    const int32_t* row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      const int idx = (j * CH) / B + k;
+      e.blk[k] = idx < p.max_blocks_per_seq ? __ldg(row + idx) : -1;
+    }
+    return e;
+  };
+
+  Lookahead<NB> win0 = lookahead(lane);
+  Lookahead<NB> win1 = lookahead(32 + lane);
+  int base = 0;
+
+  // Issue the copies of chunk `pos` into stage pos % STAGES (lane 0 copies,
+  // every lane takes part in the shuffles).
+  auto issue = [&](int pos) {
+    if (pos >= n) return;
+    int src = pos - base;
+    const bool hi = src >= 32;
+    src &= 31;
+    const int s = __shfl_sync(0xffffffffu, hi ? win1.s : win0.s, src);
+    const int h = __shfl_sync(0xffffffffu, hi ? win1.h : win0.h, src);
+    const int j = __shfl_sync(0xffffffffu, hi ? win1.j : win0.j, src);
+    const int len_raw = __shfl_sync(0xffffffffu, hi ? win1.len : win0.len, src);
+    int blk[NB];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) blk[k] = __shfl_sync(0xffffffffu, hi ? win1.blk[k] : win0.blk[k], src);
+    if (lane == 0) {
+      const int st = pos % STAGES;
+      uint8_t* stage = area + st * STRIDE;
+      T* sK = reinterpret_cast<T*>(stage);
+      T* sV = sK + TILE;
+      T* sQ = sV + TILE;
+      int32_t* flag = reinterpret_cast<int32_t*>(stage + 2 * 4096 + 2 * D);
+      const int len = min(max(len_raw, 0), cap);
+      const int nvalid = min(CH, len - j * CH);
+      const bool first = (pos == 0) || (j == 0);
+      // rows of this chunk that each touched block supplies
+      bool bad = false;
+#pragma unroll
+      for (int k = 0; k < NB; ++k) {
+        const int rows = (CH >= B) ? min(B, nvalid - k * B) : nvalid;
+        if (rows > 0 && (blk[k] < 0 || blk[k] >= p.num_blocks)) bad = true;
+      }
+      if (bad) set_status(p.status, -7 /* PA_ERR_BAD_BLOCK */);
+      fence_proxy_async_smem();
+      *flag = bad ? 1 : 0;
+      const uint32_t qbytes = first ? D * 2 : 0;
+      const uint32_t kvbytes = bad ? 0 : 2u * nvalid * D * 2;
+      mbar_arrive_expect_tx(&bars[st], qbytes + kvbytes);
+      if (first)
+        bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * H + h) * D, D * 2, &bars[st], policy);
+      if (!bad) {
+        if constexpr (CH >= B) {
+#pragma unroll
+          for (int k = 0; k < NB; ++k) {
+            const int rows = min(B, nvalid - k * B);
+            if (rows > 0) {
+              const int64_t off = (static_cast<int64_t>(blk[k]) * H + h) * B * D;
+              bulk_copy_g2s(sK + k * B * D, kc + off, rows * D * 2, &bars[st], policy);
+              bulk_copy_g2s(sV + k * B * D, vc + off, rows * D * 2, &bars[st], policy);
+            }
+          }
+        } else {
+          const int row0 = (j * CH) % B;
+          const int64_t off = ((static_cast<int64_t>(blk[0]) * H + h) * B + row0) * D;
+          bulk_copy_g2s(sK, kc + off, nvalid * D * 2, &bars[st], policy);
+          bulk_copy_g2s(sV, vc + off, nvalid * D * 2, &bars[st], policy);
+        }
+      }
+    }
+  };
+
+#pragma unroll
+  for (int pos = 0; pos < STAGES; ++pos) issue(pos);
+
+  const int dchunk = lane % LPT;
+  const int tsub = lane / LPT;
+  float qf[8];
+  float acc[8];
+  float m = -INFINITY, lsum = 0.f;
+  int piece_j0 = 0;
+
+  for (int pos = 0; pos < n; ++pos) {
+    if (pos - base == 32) {
+      base += 32;
+      win0 = win1;
+      win1 = lookahead(base + 32 + lane);
+    }
+    const int src = pos - base;
+    const int s = __shfl_sync(0xffffffffu, win0.s, src);
+    const int h = __shfl_sync(0xffffffffu, win0.h, src);
+    const int j = __shfl_sync(0xffffffffu, win0.j, src);
+    const int len = min(max(__shfl_sync(0xffffffffu, win0.len, src), 0), cap);
+    const int st = pos % STAGES;
+    const uint32_t parity = (pos / STAGES) & 1;
+
+    if (!mbar_wait_bounded(&bars[st], parity, p.wait_limit_ns)) {
+      set_status(p.status, -10 /* PA_ERR_TIMEOUT */);
+      for (int d = pos; d < min(pos + STAGES, n); ++d)
+        mbar_wait_bounded(&bars[d % STAGES], (d / STAGES) & 1, kDrainLimitNs);
+      return;
+    }
+
+    const uint8_t* stage = area + st * STRIDE;
+    const T* sK = reinterpret_cast<const T*>(stage);
+    const T* sV = sK + TILE;
+    const T* sQ = sV + TILE;
+    const int bad = *reinterpret_cast<const int32_t*>(stage + 2 * 4096 + 2 * D);
+
+    if (pos == 0 || j == 0) {
+      piece_j0 = j;
+      float qraw[8];
+      unpack8<T>(*reinterpret_cast<const uint4*>(sQ + dchunk * 8), qraw);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        qf[k] = qraw[k] * p.qk_scale_log2;
+        acc[k] = 0.f;
+      }
+      m = -INFINITY;
+      lsum = 0.f;
+    }
+    const int nvalid = bad ? 0 : min(CH, len - j * CH);
+
+    // scores (base-2 logits) of this lane's token rows
+    float sc[ITERS];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      float kf[8];
+      unpack8<T>(*reinterpret_cast<const uint4*>(sK + (it * TPI + tsub) * D + dchunk * 8), kf);
+      float d0 = qf[0] * kf[0];
+#pragma unroll
+      for (int k = 1; k < 8; ++k) d0 = fmaf(qf[k], kf[k], d0);
+      sc[it] = d0;
+    }
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+#pragma unroll
+      for (int off = LPT / 2; off >= 1; off >>= 1) sc[it] += __shfl_xor_sync(0xffffffffu, sc[it], off);
+    }
+    if (nvalid < CH) {
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it)
+        if (it * TPI + tsub >= nvalid) sc[it] = -INFINITY;
+    }
+    float cm = sc[0];
+#pragma unroll
+    for (int it = 1; it < ITERS; ++it) cm = fmaxf(cm, sc[it]);
+#pragma unroll
+    for (int off = LPT; off < 32; off <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+    const float m_new = fmaxf(m, cm);
+    if (m_new != -INFINITY) {
+      const float alpha = fast_exp2(m - m_new);
+      float psum = 0.f;
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) {
+        sc[it] = fast_exp2(sc[it] - m_new);
+        psum += sc[it];
+      }
+      lsum = fmaf(lsum, alpha, psum);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] *= alpha;
+      m = m_new;
+      if (nvalid == CH) {
+#pragma unroll
+        for (int it = 0; it < ITERS; ++it) {
+          float vf[8];
+          unpack8<T>(*reinterpret_cast<const uint4*>(sV + (it * TPI + tsub) * D + dchunk * 8), vf);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = fmaf(sc[it], vf[k], acc[k]);
+        }
+      } else {
+#pragma unroll
+        for (int it = 0; it < ITERS; ++it) {
+          if (it * TPI + tsub < nvalid) {
+            float vf[8];
+            unpack8<T>(*reinterpret_cast<const uint4*>(sV + (it * TPI + tsub) * D + dchunk * 8), vf);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = fmaf(sc[it], vf[k], acc[k]);
+          }
+        }
+      }
+    }
+
+    const int ns = (len + CH - 1) / CH;
+    if (pos == n - 1 || j == ns - 1) {
+      float l_all = lsum;
+      float o[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] = acc[k];
+#pragma unroll
+      for (int off = LPT; off < 32; off <<= 1) {
+        l_all += __shfl_xor_sync(0xffffffffu, l_all, off);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
+      }
+      const int64_t sh = static_cast<int64_t>(s) * H + h;
+      if (piece_j0 == 0 && j == ns - 1) {
+        if (tsub == 0) {
+          const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) o[k] *= inv;
+          *reinterpret_cast<uint4*>(static_cast<T*>(p.out) + sh * D + dchunk * 8) = pack8<T>(o);
+        }
+      } else {
+        float* rec = p.records + (static_cast<int64_t>(w) + sh) * (D + 4);
+        if (lane == 0) {
+          rec[0] = m;
+          rec[1] = l_all;
+        }
+        if (tsub == 0) {
+          float4* dst = reinterpret_cast<float4*>(rec + 4 + dchunk * 8);
+          dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+          dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+        }
+      }
+    }
+
+    __syncwarp();
+    issue(pos + STAGES);
+  }
+}
+
+// Merge of the partial results of one (text, head) whose chunks were split
+// over several warps: with M = max_i m_i and f_i = 2^(m_i - M),
+//     out = (sum_i f_i o_i) / (sum_i f_i l_i),
+// which equals the softmax-weighted sum over all the text's tokens exactly
+// (up to rounding).  Texts with no tokens get zeros here.  Partials are read
+// in warp order, so the result is reproducible.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
+                    const float* __restrict__ records, int num_seqs, int num_heads) {
+  constexpr int PER = D / 32;  // elements per lane
+  const int lane = threadIdx.x & 31;
+  const int seg = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (seg >= num_seqs * num_heads) return;
+  const int s = seg / num_heads;
+  const int h = seg - s * num_heads;
+  const int32_t* prefix = header + kHeaderInts;
+  const int cpw = header[1];
+  const int seg0 = prefix[s];
+  const int ns = (prefix[s + 1] - seg0) / num_heads;
+  T* o = out + static_cast<int64_t>(seg) * D + lane * PER;
+  if (ns == 0) {
+    if constexpr (PER == 4) {
+      *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
+    } else {
+      *reinterpret_cast<uint32_t*>(o) = 0u;
+    }
+    return;
+  }
+  const int a = seg0 + h * ns;
+  const int w_lo = a / cpw;
+  const int w_hi = (a + ns - 1) / cpw;
+  if (w_lo == w_hi) return;  // finished in place by the decode kernel
+  float M = -INFINITY;
+  for (int w = w_lo; w <= w_hi; ++w)
+    M = fmaxf(M, records[(static_cast<int64_t>(w) + seg) * (D + 4)]);
+  float L = 0.f;
+  float acc[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+  for (int w = w_lo; w <= w_hi; ++w) {
+    const float* rec = records + (static_cast<int64_t>(w) + seg) * (D + 4);
+    const float f = M == -INFINITY ? 0.f : fast_exp2(rec[0] - M);
+    L = fmaf(f, rec[1], L);
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc[k] = fmaf(f, rec[4 + lane * PER + k], acc[k]);
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if constexpr (PER == 4) {
+    uint2 v;
+    v.x = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
+    v.y = Elem<T>::from_float2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(o) = v;
+  } else {
+    *reinterpret_cast<uint32_t*>(o) = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
+  }
+}
+
+namespace {
+
+int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+size_t decode_smem_bytes(int D, int num_seqs) {
+  const int area = D == 128 ? warp_area_bytes(128, kDecodeStages) : warp_area_bytes(64, kDecodeStages);
+  return static_cast<size_t>(kDecodeWarps) * area + align_up(sizeof(int32_t) * (num_seqs + 1), 16);
+}
+
+// Resident CTAs per SM of `kernel` with `smem` dynamic shared memory, cached
+// per (device, kernel, smem).  Also raises the kernel's shared-memory limit.
+int resident_ctas(const void* kernel, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, size_t>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(dev, kernel, smem);
+  const auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int occ = 0;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kDecodeWarps * 32, smem) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    occ = 0;
+  }
+  cache[key] = occ;
+  return occ;
+}
+
+struct Plan {
+  int grid = 0;
+  int work_warps = 0;
+  size_t smem = 0;
+};
+
+// Persistent grid: every SM filled with resident CTAs, but never more warps
+// than there can be chunks.
+Plan plan_decode(const void* kernel, int D, int B, int num_seqs, int num_heads,
+                 int max_blocks_per_seq, int64_t forced_warps) {
+  Plan pl;
+  pl.smem = decode_smem_bytes(D, num_seqs);
+  const int occ = resident_ctas(kernel, pl.smem);
+  const int sms = device_sm_count();
+  if (occ <= 0 || sms <= 0) return pl;
+  const int CH = chunk_tokens(D);
+  const int64_t cap = static_cast<int64_t>(max_blocks_per_seq) * B;
+  const int64_t chunks_max = static_cast<int64_t>(num_seqs) * num_heads * ((cap + CH - 1) / CH);
+  int64_t warps = static_cast<int64_t>(sms) * occ * kDecodeWarps;
+  const int64_t useful = ((chunks_max + kDecodeWarps - 1) / kDecodeWarps) * kDecodeWarps;
+  if (warps > useful) warps = useful;
+  if (forced_warps > 0) warps = forced_warps;
+  if (warps < 1) warps = 1;
+  pl.work_warps = static_cast<int>(warps);
+  pl.grid = static_cast<int>((warps + kDecodeWarps - 1) / kDecodeWarps);
+  return pl;
+}
+
+size_t records_bytes(int64_t records, int D) {
+  return static_cast<size_t>(records) * (D + 4) * sizeof(float);
+}
+
+template <typename T, int D, int B>
+const void* decode_kernel_ptr() {
+  return reinterpret_cast<const void*>(&paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages>);
+}
+
+template <typename T, int D, int B>
+cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
+  const Plan pl = plan_decode(decode_kernel_ptr<T, D, B>(), D, B, a.num_seqs, a.num_heads,
+                              a.max_blocks_per_seq, a.forced_warps);
+  if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
+  const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_heads;
+  const size_t need = header_bytes(a.num_seqs) + records_bytes(pl.work_warps + segs, D);
+  if (a.workspace_bytes < need) return cudaErrorInvalidValue;
+  DecodeParams p;
+  p.out = a.out;
+  p.q = a.q;
+  p.k_cache = a.k_cache;
+  p.v_cache = a.v_cache;
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  p.qk_scale_log2 = a.scale * 1.4426950408889634f;  // log2(e)
+  p.num_seqs = a.num_seqs;
+  p.num_heads = a.num_heads;
+  p.max_blocks_per_seq = a.max_blocks_per_seq;
+  p.num_blocks = a.num_blocks;
+  p.num_work_warps = pl.work_warps;
+  p.header = static_cast<int32_t*>(a.workspace);
+  p.records = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + header_bytes(a.num_seqs));
+  p.status = a.status;
+  p.wait_limit_ns = a.wait_limit_ns;
+  paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages>
+      <<<pl.grid, kDecodeWarps * 32, pl.smem, stream>>>(p);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int per_cta = 8;
+  const int64_t grid2 = (segs + per_cta - 1) / per_cta;
+  split_reduce_kernel<T, D><<<static_cast<unsigned>(grid2), per_cta * 32, 0, stream>>>(
+      static_cast<T*>(a.out), p.header, p.records, a.num_seqs, a.num_heads);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t dispatch_block(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.block_size) {
+    case 4: return launch_typed<T, D, 4>(a, stream);
+    case 8: return launch_typed<T, D, 8>(a, stream);
+    case 16: return launch_typed<T, D, 16>(a, stream);
+    case 32: return launch_typed<T, D, 32>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T>
+cudaError_t dispatch_dim(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.head_dim) {
+    case 64: return dispatch_block<T, 64>(a, stream);
+    case 128: return dispatch_block<T, 128>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D>
+const void* kernel_for(int block_size, bool bf16) {
+  switch (block_size) {
+    case 4: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 4>() : decode_kernel_ptr<__half, D, 4>();
+    case 8: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 8>() : decode_kernel_ptr<__half, D, 8>();
+    case 16: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 16>() : decode_kernel_ptr<__half, D, 16>();
+    case 32: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 32>() : decode_kernel_ptr<__half, D, 32>();
+    default: return nullptr;
+  }
+}
+
+}  // namespace
+
+bool decode_sizes_supported(int num_seqs, int num_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq) {
+  if (num_seqs < 1 || num_seqs > kMaxSeqs || num_heads < 1 || num_heads > 1024) return false;
+  if (head_dim != 64 && head_dim != 128) return false;
+  if (block_size != 4 && block_size != 8 && block_size != 16 && block_size != 32) return false;
+  if (max_blocks_per_seq < 1) return false;
+  const int64_t CH = chunk_tokens(head_dim);
+  const int64_t cap = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+  const int64_t chunks = static_cast<int64_t>(num_seqs) * num_heads * ((cap + CH - 1) / CH);
+  return chunks < (int64_t{1} << 30) && cap < (int64_t{1} << 30);
+}
+
+size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int block_size,
+                              int max_blocks_per_seq, int64_t forced_warps) {
+  if (!decode_sizes_supported(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq))
+    return 0;
+  int64_t warps = 0;
+  for (int bf16 = 0; bf16 < 2; ++bf16) {
+    const void* k = head_dim == 128 ? kernel_for<128>(block_size, bf16)
+                                    : kernel_for<64>(block_size, bf16);
+    const Plan pl = plan_decode(k, head_dim, block_size, num_seqs, num_heads,
+                                max_blocks_per_seq, forced_warps);
+    if (pl.grid <= 0) return 0;
+    if (pl.work_warps > warps) warps = pl.work_warps;
+  }
+  const int64_t segs = static_cast<int64_t>(num_seqs) * num_heads;
+  return header_bytes(num_seqs) + records_bytes(warps + segs, head_dim);
+}
+
+cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
+  if (!decode_sizes_supported(a.num_seqs, a.num_heads, a.head_dim, a.block_size,
+                              a.max_blocks_per_seq))
+    return cudaErrorInvalidValue;
+  return a.is_bf16 ? dispatch_dim<__nv_bfloat16>(a, stream) : dispatch_dim<__half>(a, stream);
+}
+
+}  // namespace pa

@@ -1,0 +1,57 @@
+"""Run decode steps (write + paged attention) of one workload R times.
+
+    python -m paged_kv_cache_326_b200.run_case [--workload NAME] [--num-seqs S] [--reps R]
+
+For profilers: it makes no timing claims.  Workloads: ``opt13b_batch64``
+(optionally cut to the first S texts, pool sized 1.5x what they need),
+``tiny``, ``skewed`` (bf16, blocks of 16).
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+import paged_kv_cache_326_b200 as P
+from paged_kv_cache_326_b200 import workloads as W
+
+
+def make(name: str, num_seqs: int, device):
+    if name == "tiny":
+        return W.tiny(device=device)
+    if name == "skewed":
+        return W.skewed(device=device)
+    if name == "opt13b_batch64":
+        if num_seqs <= 0 or num_seqs >= 64:
+            return W.opt13b_batch64(device=device)
+        lens = W.opt13b_batch64_lens()[:num_seqs]
+        need = sum(W.blocks_needed(L, 16) for L in lens)
+        return W.make_decode(f"opt13b_first{num_seqs}", lens, num_heads=40, head_dim=128,
+                             block_size=16, num_blocks=(3 * need + 1) // 2, dtype=torch.float16,
+                             seed=2, device=device, max_blocks_per_seq=128)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="opt13b_batch64")
+    ap.add_argument("--num-seqs", type=int, default=0)
+    ap.add_argument("--reps", type=int, default=3)
+    args = ap.parse_args()
+    dev = torch.device("cuda", 0)
+    w = make(args.workload, args.num_seqs, dev)
+    out = torch.empty_like(w.q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(args.reps):
+        P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+        P.pa_paged_attn_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                               w.scale, status=status)
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
+    kv = sum(w.context_lens.tolist()) * 2 * w.num_heads * w.head_dim * w.q.element_size()
+    print(f"{w.name}: {w.num_seqs} texts, KV bytes per step {kv}, status ok")
+
+
+if __name__ == "__main__":
+    main()

@@ -139,7 +139,7 @@ def slots_of(block_tables: torch.Tensor, positions: torch.Tensor, block_size: in
     """Slot of token ``positions[s]`` of text s: physical block of its logical
     block, times the block size, plus its place in the block."""
     pos = positions.to(torch.int64)
-    phys = block_tables.to(torch.int64).gather(1, (pos // block_size)[:, None])[:, 0]
+    phys = block_tables.to(torch.int64).gather(1, (pos.clamp(min=0) // block_size)[:, None])[:, 0]
     return torch.where(pos >= 0, phys * block_size + pos % block_size,
                        torch.full_like(pos, -1))
 
