@@ -503,21 +503,32 @@ size_t decode_smem_bytes(int D, int num_seqs) {
 }
 
 // Resident CTAs per SM of `kernel` with `smem` dynamic shared memory, cached
-// per (device, kernel, smem).  Also raises the kernel's shared-memory limit.
-int resident_ctas(const void* kernel, size_t smem) {
+// per (device, kernel, smem).  The kernel's dynamic shared-memory limit is
+// raised once per (device, kernel) to the most any call can need, so a call
+// with fewer texts never lowers it below what a larger one uses.
+int resident_ctas(const void* kernel, size_t smem, int head_dim) {
   static std::mutex mu;
   static std::map<std::tuple<int, const void*, size_t>, int> cache;
+  static std::map<std::pair<int, const void*>, bool> raised;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lock(mu);
   const auto key = std::make_tuple(dev, kernel, smem);
   const auto it = cache.find(key);
   if (it != cache.end()) return it->second;
+  const auto rkey = std::make_pair(dev, kernel);
+  if (!raised.count(rkey)) {
+    const size_t most = decode_smem_bytes(head_dim, kMaxSeqs);
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(most)) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    raised[rkey] = true;
+  }
   int occ = 0;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kDecodeWarps * 32, smem) !=
-          cudaSuccess) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kDecodeWarps * 32, smem) !=
+      cudaSuccess) {
     cudaGetLastError();
     occ = 0;
   }
@@ -537,7 +548,7 @@ Plan plan_decode(const void* kernel, int D, int B, int num_seqs, int num_heads,
                  int max_blocks_per_seq, int64_t forced_warps) {
   Plan pl;
   pl.smem = decode_smem_bytes(D, num_seqs);
-  const int occ = resident_ctas(kernel, pl.smem);
+  const int occ = resident_ctas(kernel, pl.smem, D);
   const int sms = device_sm_count();
   if (occ <= 0 || sms <= 0) return pl;
   const int CH = chunk_tokens(D);
