@@ -14,7 +14,8 @@
  * --------------------------------
  *  - Every pointer to tensor data is a DEVICE pointer owned by the caller,
  *    except the block manager's arguments, which are HOST pointers.  The
- *    library never allocates, frees or keeps device memory.
+ *    library never allocates or frees device memory; the only device memory
+ *    it keeps is the static scratch of pa_paged_attn_decode_noalloc.
  *  - Tensors are dense and row-major ("contiguous").  Element types are
  *    IEEE fp16 or bfloat16 (pa_dtype), 2 bytes each.
  *  - Pool layout: k_cache and v_cache are each
@@ -61,7 +62,8 @@ enum {
   PA_ERR_BAD_LEN = -8,        /* device: context length < 0 or > max_blocks_per_seq*block_size */
   PA_ERR_BAD_SLOT = -9,       /* device: slot >= num_blocks*block_size */
   PA_ERR_TIMEOUT = -10,       /* device: a bounded wait on a shared-memory barrier gave up */
-  PA_ERR_CORRUPT = -11        /* block manager: internal counts inconsistent */
+  PA_ERR_CORRUPT = -11,       /* block manager: internal counts inconsistent */
+  PA_ERR_TOO_LARGE = -12      /* sizes need more scratch than pa_paged_attn_decode_noalloc holds */
 };
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -141,6 +143,34 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
                          int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt,
                          void* workspace, size_t workspace_bytes, int32_t* d_status,
                          pa_stream_t stream);
+
+/*
+ * pa_paged_attn_decode_noalloc — pa_paged_attn_decode without a caller
+ * workspace, for callers that cannot allocate device memory (a host framework
+ * that owns every device allocation, a fixed memory budget, a loop where an
+ * allocation and the device synchronisation it may bring are not allowed).
+ * The pages have no counterpart: this is a deployment convenience.
+ *
+ * Same arguments, computation, result and errors as pa_paged_attn_decode,
+ * minus workspace/workspace_bytes.  Its scratch is a static device array of
+ * 8 MiB inside the library; every GPU that loads the library holds it until
+ * the process exits.  Sizes whose workspace
+ * (pa_paged_attn_decode_workspace_size) exceeds 8 MiB are rejected with
+ * PA_ERR_TOO_LARGE before anything is launched (8 MiB covers, e.g., 256 texts
+ * x 40 heads x 128 on a 148-SM B200).  The call allocates and frees nothing.
+ *
+ * The first call on each device looks up the array's device address (a host
+ * runtime call, cudaGetSymbolAddress); make that first call before any
+ * stream capture.  All calls share the one array and leave their contents in
+ * it (nothing in it needs to start at zero): calls that may overlap on the
+ * GPU, on any streams, race and must be serialised by the caller.
+ */
+int pa_paged_attn_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, int num_seqs,
+                                 int num_heads, int head_dim, int block_size,
+                                 int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt,
+                                 int32_t* d_status, pa_stream_t stream);
 
 /*
  * Tuning and test options (process-wide, not thread-safe; set before use).

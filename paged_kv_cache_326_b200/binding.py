@@ -30,6 +30,7 @@ PA_ERR_BAD_LEN = -8
 PA_ERR_BAD_SLOT = -9
 PA_ERR_TIMEOUT = -10
 PA_ERR_CORRUPT = -11
+PA_ERR_TOO_LARGE = -12
 
 PA_F16 = 0
 PA_BF16 = 1
@@ -39,7 +40,7 @@ PA_OPT_DECODE_WARPS = 2
 
 _KIND = {PA_ERR_INVALID: "invalid", PA_ERR_CUDA: "cuda", PA_ERR_OUT_OF_BLOCKS: "out_of_blocks",
          PA_ERR_NO_SEQ: "no_seq", PA_ERR_EXISTS: "exists", PA_ERR_TABLE_FULL: "table_full",
-         PA_ERR_CORRUPT: "corrupt"}
+         PA_ERR_CORRUPT: "corrupt", PA_ERR_TOO_LARGE: "too_large"}
 
 
 class PagedAttnError(RuntimeError):
@@ -63,6 +64,8 @@ _SIGNATURES = {
     "pa_paged_attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "pa_paged_attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _i32,
                                     _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
+    "pa_paged_attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
+                                            _i32, _i32, _i64, _i32, _vp, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_i32, [_vp, _i64, _i32]),
@@ -207,6 +210,32 @@ def pa_paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tens
         _dtype_code(q), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _status_ptr(status), _stream(stream, q.device))
     _check(code, "pa_paged_attn_decode")
+    return out
+
+
+def pa_paged_attn_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                                 v_cache: torch.Tensor, block_tables: torch.Tensor,
+                                 context_lens: torch.Tensor, scale: float,
+                                 status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pa_paged_attn_decode with the library's own static 8 MiB scratch: for
+    callers that cannot allocate device memory.  Calls that may overlap on
+    the GPU share that scratch and race.  Raises PagedAttnError with code
+    PA_ERR_TOO_LARGE when the sizes need more scratch than it holds."""
+    S, H, D = q.shape
+    N, H2, B, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S][max_blocks], context_lens [S]")
+    for t in (out, k_cache, v_cache):
+        if t.dtype != q.dtype:
+            raise TypeError("q, out and the caches must share a dtype")
+    code = lib().pa_paged_attn_decode_noalloc(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(context_lens, "context_lens", torch.int32), float(scale), S, H, D, B,
+        block_tables.shape[1], N, _dtype_code(q), _status_ptr(status), _stream(stream, q.device))
+    _check(code, "pa_paged_attn_decode_noalloc")
     return out
 
 

@@ -29,6 +29,10 @@ int from_cuda(cudaError_t e) {
 
 }  // namespace
 
+namespace pa {
+int64_t option_decode_warps() { return g_decode_warps.load(); }
+}  // namespace pa
+
 extern "C" {
 
 const char* pa_status_string(int code) {
@@ -45,6 +49,7 @@ const char* pa_status_string(int code) {
     case PA_ERR_BAD_SLOT: return "slot outside the pool";
     case PA_ERR_TIMEOUT: return "bounded wait gave up";
     case PA_ERR_CORRUPT: return "block manager counts inconsistent";
+    case PA_ERR_TOO_LARGE: return "sizes need more scratch than the no-allocation entry point holds";
     default: return "unknown status";
   }
 }

@@ -1,0 +1,72 @@
+// pa_paged_attn_decode_noalloc: paged decode attention for callers that cannot
+// allocate device memory.
+//
+// Some callers cannot call cudaMalloc, or cannot hand this library a buffer
+// of their own: a host framework that owns every device allocation and gives
+// out no scratch, a fixed device-memory budget set before serving starts, or a
+// latency-bound loop where an allocation (which may synchronise the device)
+// is not allowed.  This entry point runs the same kernels as
+// pa_paged_attn_decode, but its scratch is a file-scope device array that the
+// library carries with it, so the caller passes only inputs and outputs.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "kernels.h"
+#include "pagedattn.h"
+
+namespace {
+
+// 8 MiB of scratch, zero at load, kept by every GPU that loads the library
+// until the process exits.  Enough for, e.g., 256 texts x 40 heads x 128.
+constexpr size_t kScratchBytes = size_t{8} << 20;
+static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_decode_scratch on the current device, looked up once
+// per device.  In host code the array's name is only a host-side stand-in,
+// never a device address, so it is resolved with cudaGetSymbolAddress.
+int scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return PA_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_paged_attn_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                            const void* v_cache, const int32_t* block_tables,
+                                            const int32_t* context_lens, float scale,
+                                            int num_seqs, int num_heads, int head_dim,
+                                            int block_size, int max_blocks_per_seq,
+                                            int64_t num_blocks, pa_dtype dt, int32_t* d_status,
+                                            pa_stream_t stream) {
+  if (num_seqs == 0) return PA_OK;
+  const size_t need = pa::decode_workspace_bytes(num_seqs, num_heads, head_dim, block_size,
+                                                 max_blocks_per_seq, pa::option_decode_warps());
+  if (need == 0) return PA_ERR_INVALID;
+  if (need > kScratchBytes) return PA_ERR_TOO_LARGE;
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != PA_OK) return rc;
+  return pa_paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                              num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq,
+                              num_blocks, dt, scratch, kScratchBytes, d_status, stream);
+}

@@ -42,6 +42,9 @@ bool decode_sizes_supported(int num_seqs, int num_heads, int head_dim, int block
 size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int block_size,
                               int max_blocks_per_seq, int64_t forced_warps);
 
+// Current PA_OPT_DECODE_WARPS setting.
+int64_t option_decode_warps();
+
 // Launches the decode kernel and the split reduce on `stream`.
 // Returns cudaErrorInvalidValue for unsupported sizes or a short workspace.
 cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream);
