@@ -128,13 +128,16 @@ size_t pa_paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head
  *   num_blocks     pool size in blocks (bounds check of table entries)
  *   workspace      device scratch of at least
  *                  pa_paged_attn_decode_workspace_size(...) bytes, 256-byte
- *                  aligned; no initial contents needed; must not be shared by
+ *                  aligned; no initial contents needed (its arrival counters
+ *                  are tagged with a per-call epoch); must not be shared by
  *                  calls that may run at the same time
  *   d_status       nullable device int32 (see conventions)
  * Work is split over all SMs in equal runs of 16-token (head_dim 128) or
- * 32-token (head_dim 64) chunks; a text whose run spans several warps is
- * merged with a log-sum-exp reduction (a second kernel on the same stream).
- * For fixed inputs, sizes and device the result is bitwise reproducible.
+ * 32-token (head_dim 64) chunks; a (text, head) whose chunks span several
+ * warps' runs is merged with a log-sum-exp reduction by the last of those
+ * warps to finish.  One kernel launch, with programmatic dependent launch
+ * after pa_kv_cache_write.  For fixed inputs, sizes and device the result is
+ * bitwise reproducible.
  * Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
  */
 int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const void* v_cache,

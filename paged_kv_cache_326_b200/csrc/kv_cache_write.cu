@@ -23,6 +23,11 @@ kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                       uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                       const int64_t* __restrict__ slot_mapping, int num_tokens, int num_heads,
                       int vec_per_row, int block_size, int64_t num_slots, int32_t* status) {
+  // Programmatic dependent launch: wait for the previous kernel's writes
+  // (for example the last decode still reading this pool), then let the
+  // decode kernel that follows get its CTAs resident.
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t per_token = static_cast<int64_t>(num_heads) * vec_per_row;
   const int64_t total = per_token * num_tokens;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -55,10 +60,21 @@ cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, v
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
   if (blocks > (1 << 20)) blocks = 1 << 20;
-  kv_cache_write_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_heads, vec_per_row, block_size,
-      num_blocks * block_size, status);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(
+      &cfg, kv_cache_write_kernel, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, num_tokens,
+      num_heads, vec_per_row, block_size, num_blocks * block_size, status);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

@@ -18,8 +18,9 @@
 //    long and short texts alike keep all 148 SMs busy to the end, with no
 //    tail wave.  A (text, head) whose chunks fall into several warps' runs
 //    produces one partial result per warp (running max m, sum l, unnormalised
-//    output o), merged by split_reduce_kernel; one that falls inside a single
-//    run is finished in place.
+//    output o); the last of those warps to finish merges them (log-sum-exp),
+//    so no second kernel is needed.  One that falls inside a single run is
+//    finished in place.
 //  * Each warp is its own pipeline: lane 0 issues bulk (TMA) copies of the
 //    chunk's key rows and value rows, straight from their physical blocks,
 //    into a ring of STAGES shared-memory stages, each with an mbarrier that
@@ -36,8 +37,12 @@
 //    (running-max) form in fp32, in base 2 with log2(e) folded into the scale.
 //  * Every wait is bounded; a wait that gives up records PA_ERR_TIMEOUT,
 //    drains the copies in flight (bounded too) and returns.
+//  * Launched with programmatic dependent launch, so its CTAs are resident
+//    while the preceding cache write finishes; griddepcontrol.wait holds every
+//    read until that kernel's writes are visible.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <map>
 #include <mutex>
@@ -52,10 +57,15 @@ namespace pa {
 
 namespace {
 
-constexpr int kDecodeWarps = 4;   // warps per CTA
-constexpr int kDecodeStages = 3;  // ring depth per warp
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 3
+#endif
+constexpr int kDecodeWarps = PA_DECODE_WARPS;    // warps per CTA
+constexpr int kDecodeStages = PA_DECODE_STAGES;  // ring depth per warp
 constexpr int kMaxSeqs = 4096;
-constexpr int kHeaderInts = 4;    // total chunks, chunks per warp, warps, spare
 constexpr int kDrainLimitNs = 1000000000;
 
 __host__ __device__ constexpr int chunk_tokens(int D) { return 2048 / D; }
@@ -64,9 +74,13 @@ __host__ __device__ constexpr int warp_area_bytes(int D, int stages) { return st
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t header_bytes(int num_seqs) {
-  return align_up(sizeof(int32_t) * (kHeaderInts + num_seqs + 1), 256);
-}
+// Arrival counters, one 64-bit word per (text, head): the call's epoch in
+// the top 40 bits, the number of partials stored so far in the low 24.  A
+// word whose epoch is not this call's counts as zero, so the workspace never
+// needs clearing.
+size_t counters_bytes(int64_t segs) { return align_up(sizeof(unsigned long long) * segs, 256); }
+constexpr int kCountBits = 24;
+constexpr unsigned long long kEpochMask = (1ull << 40) - 1;
 
 struct DecodeParams {
   void* out;
@@ -81,7 +95,8 @@ struct DecodeParams {
   int max_blocks_per_seq;
   int64_t num_blocks;
   int num_work_warps;
-  int32_t* header;
+  unsigned long long* counters;
+  unsigned long long epoch;  // 40-bit, never 0
   float* records;
   int32_t* status;
   int64_t wait_limit_ns;
@@ -93,6 +108,83 @@ struct Lookahead {
   int s, h, j, len;  // len is the raw context length (clamped at use)
   int blk[NB];
 };
+
+// Count one more stored partial of a (text, head) in this call; returns the
+// count including this one.
+// The compare-and-swap is acq_rel at GPU scope: it releases this warp's
+// partial (ordered before it by __syncwarp) and, for the last arriver,
+// acquires everyone else's.
+__device__ __forceinline__ unsigned long long cas_acq_rel(unsigned long long* p,
+                                                         unsigned long long cmp,
+                                                         unsigned long long val) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
+               : "=l"(old)
+               : "l"(p), "l"(cmp), "l"(val)
+               : "memory");
+  return old;
+}
+
+__device__ __forceinline__ uint32_t arrive_count(unsigned long long* ctr, unsigned long long epoch) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  while (true) {
+    const unsigned long long want =
+        (cur >> kCountBits) == epoch ? cur + 1 : (epoch << kCountBits) | 1ull;
+    const unsigned long long prev = cas_acq_rel(ctr, cur, want);
+    if (prev == cur) return static_cast<uint32_t>(want & ((1ull << kCountBits) - 1));
+    cur = prev;
+  }
+}
+
+// Merge the partials of one (text, head), stored by warps w_lo..w_hi: with
+// M = max_i m_i and f_i = 2^(m_i - M),
+//     out = (sum_i f_i o_i) / (sum_i f_i l_i),
+// which equals the softmax-weighted sum over all the text's tokens (up to
+// rounding).  Partials are read in warp order, so the result does not depend
+// on which warp merges.  Reads go through L2 (other SMs wrote them).
+template <typename T, int D>
+__device__ __forceinline__ void merge_partials(const float* records, T* out, int64_t sh, int w_lo,
+                                               int w_hi, int lane) {
+  constexpr int PER = D / 32;
+  // running maxima: one partial per lane, then a warp max
+  float M = -INFINITY;
+  for (int w0 = w_lo; w0 <= w_hi; w0 += 32) {
+    const int w = w0 + lane;
+    if (w <= w_hi) M = fmaxf(M, __ldcg(records + (w + sh) * (D + 4)));
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float L = 0.f;
+  float acc[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+  for (int w = w_lo; w <= w_hi; ++w) {
+    const float* rec = records + (w + sh) * (D + 4);
+    const float f = M == -INFINITY ? 0.f : fast_exp2(__ldcg(rec) - M);
+    L = fmaf(f, __ldcg(rec + 1), L);
+    if constexpr (PER == 4) {
+      const float4 o = __ldcg(reinterpret_cast<const float4*>(rec + 4) + lane);
+      acc[0] = fmaf(f, o.x, acc[0]);
+      acc[1] = fmaf(f, o.y, acc[1]);
+      acc[2] = fmaf(f, o.z, acc[2]);
+      acc[3] = fmaf(f, o.w, acc[3]);
+    } else {
+      const float2 o = __ldcg(reinterpret_cast<const float2*>(rec + 4) + lane);
+      acc[0] = fmaf(f, o.x, acc[0]);
+      acc[1] = fmaf(f, o.y, acc[1]);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  T* o = out + sh * D + lane * PER;
+  if constexpr (PER == 4) {
+    uint2 v;
+    v.x = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
+    v.y = Elem<T>::from_float2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(o) = v;
+  } else {
+    *reinterpret_cast<uint32_t*>(o) = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
+  }
+}
 
 }  // namespace
 
@@ -119,6 +211,9 @@ paged_decode_kernel(const DecodeParams p) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+
+  // Inputs may come from the kernel launched just before (the cache write).
+  griddep_wait();
 
   // ---- prologue: prefix[s] = H * (chunks of texts before s), block-wide scan
   {
@@ -156,14 +251,12 @@ paged_decode_kernel(const DecodeParams p) {
   const int total = prefix[S];
   const int W = p.num_work_warps;
   const int cpw = (total + W - 1) / W;
-  if (blockIdx.x == 0) {
-    if (tid == 0) {
-      p.header[0] = total;
-      p.header[1] = cpw;
-      p.header[2] = W;
-      p.header[3] = 0;
+  // Texts with no tokens get zeros (spread over the CTAs).
+  for (int s = blockIdx.x; s < S; s += gridDim.x) {
+    if (prefix[s + 1] == prefix[s]) {
+      uint4* o = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + static_cast<int64_t>(s) * H * D);
+      for (int i = tid; i < H * D / 8; i += WARPS * 32) o[i] = make_uint4(0u, 0u, 0u, 0u);
     }
-    for (int s = tid; s <= S; s += WARPS * 32) p.header[kHeaderInts + s] = prefix[s];
   }
 
   const int w = blockIdx.x * WARPS + warp;
@@ -391,6 +484,11 @@ paged_decode_kernel(const DecodeParams p) {
       }
     }
 
+    // This stage is consumed: refill it before the epilogue, whose global
+    // stores and (rarely) merge must not leave the copy engine idle.
+    __syncwarp();
+    issue(pos + STAGES);
+
     const int ns = (len + CH - 1) / CH;
     if (pos == n - 1 || j == ns - 1) {
       float l_all = lsum;
@@ -422,69 +520,21 @@ paged_decode_kernel(const DecodeParams p) {
           dst[0] = make_float4(o[0], o[1], o[2], o[3]);
           dst[1] = make_float4(o[4], o[5], o[6], o[7]);
         }
+        // Publish the partial, count it; the warp that stores the last one
+        // of this (text, head) merges them all.
+        __syncwarp();
+        const int a = prefix[s] + h * ns;
+        const int w_lo = a / cpw;
+        const int w_hi = (a + ns - 1) / cpw;
+        uint32_t cnt = 0;
+        if (lane == 0) cnt = arrive_count(p.counters + sh, p.epoch);
+        cnt = __shfl_sync(0xffffffffu, cnt, 0);
+        if (cnt == static_cast<uint32_t>(w_hi - w_lo + 1)) {
+          __syncwarp();  // order lane 0's acquire before every lane's reads
+          merge_partials<T, D>(p.records, static_cast<T*>(p.out), sh, w_lo, w_hi, lane);
+        }
       }
     }
-
-    __syncwarp();
-    issue(pos + STAGES);
-  }
-}
-
-// Merge of the partial results of one (text, head) whose chunks were split
-// over several warps: with M = max_i m_i and f_i = 2^(m_i - M),
-//     out = (sum_i f_i o_i) / (sum_i f_i l_i),
-// which equals the softmax-weighted sum over all the text's tokens exactly
-// (up to rounding).  Texts with no tokens get zeros here.  Partials are read
-// in warp order, so the result is reproducible.
-template <typename T, int D>
-__global__ void __launch_bounds__(256)
-split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
-                    const float* __restrict__ records, int num_seqs, int num_heads) {
-  constexpr int PER = D / 32;  // elements per lane
-  const int lane = threadIdx.x & 31;
-  const int seg = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (seg >= num_seqs * num_heads) return;
-  const int s = seg / num_heads;
-  const int h = seg - s * num_heads;
-  const int32_t* prefix = header + kHeaderInts;
-  const int cpw = header[1];
-  const int seg0 = prefix[s];
-  const int ns = (prefix[s + 1] - seg0) / num_heads;
-  T* o = out + static_cast<int64_t>(seg) * D + lane * PER;
-  if (ns == 0) {
-    if constexpr (PER == 4) {
-      *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
-    } else {
-      *reinterpret_cast<uint32_t*>(o) = 0u;
-    }
-    return;
-  }
-  const int a = seg0 + h * ns;
-  const int w_lo = a / cpw;
-  const int w_hi = (a + ns - 1) / cpw;
-  if (w_lo == w_hi) return;  // finished in place by the decode kernel
-  float M = -INFINITY;
-  for (int w = w_lo; w <= w_hi; ++w)
-    M = fmaxf(M, records[(static_cast<int64_t>(w) + seg) * (D + 4)]);
-  float L = 0.f;
-  float acc[PER];
-#pragma unroll
-  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  for (int w = w_lo; w <= w_hi; ++w) {
-    const float* rec = records + (static_cast<int64_t>(w) + seg) * (D + 4);
-    const float f = M == -INFINITY ? 0.f : fast_exp2(rec[0] - M);
-    L = fmaf(f, rec[1], L);
-#pragma unroll
-    for (int k = 0; k < PER; ++k) acc[k] = fmaf(f, rec[4 + lane * PER + k], acc[k]);
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  if constexpr (PER == 4) {
-    uint2 v;
-    v.x = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
-    v.y = Elem<T>::from_float2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(o) = v;
-  } else {
-    *reinterpret_cast<uint32_t*>(o) = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
   }
 }
 
@@ -536,6 +586,17 @@ int resident_ctas(const void* kernel, size_t smem, int head_dim) {
   return occ;
 }
 
+// A fresh 40-bit epoch per launch (never 0, so a zeroed workspace holds no
+// live counts).
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> counter{0};
+  unsigned long long e;
+  do {
+    e = (counter.fetch_add(1) + 1) & kEpochMask;
+  } while (e == 0);
+  return e;
+}
+
 struct Plan {
   int grid = 0;
   int work_warps = 0;
@@ -579,7 +640,7 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
                               a.max_blocks_per_seq, a.forced_warps);
   if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
   const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_heads;
-  const size_t need = header_bytes(a.num_seqs) + records_bytes(pl.work_warps + segs, D);
+  const size_t need = counters_bytes(segs) + records_bytes(pl.work_warps + segs, D);
   if (a.workspace_bytes < need) return cudaErrorInvalidValue;
   DecodeParams p;
   p.out = a.out;
@@ -594,18 +655,23 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   p.max_blocks_per_seq = a.max_blocks_per_seq;
   p.num_blocks = a.num_blocks;
   p.num_work_warps = pl.work_warps;
-  p.header = static_cast<int32_t*>(a.workspace);
-  p.records = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + header_bytes(a.num_seqs));
+  p.counters = static_cast<unsigned long long*>(a.workspace);
+  p.epoch = next_epoch();
+  p.records = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + counters_bytes(segs));
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
-  paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages>
-      <<<pl.grid, kDecodeWarps * 32, pl.smem, stream>>>(p);
-  cudaError_t err = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(kDecodeWarps * 32);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages>, p);
   if (err != cudaSuccess) return err;
-  const int per_cta = 8;
-  const int64_t grid2 = (segs + per_cta - 1) / per_cta;
-  split_reduce_kernel<T, D><<<static_cast<unsigned>(grid2), per_cta * 32, 0, stream>>>(
-      static_cast<T*>(a.out), p.header, p.records, a.num_seqs, a.num_heads);
   return cudaGetLastError();
 }
 
@@ -668,7 +734,7 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int blo
     if (pl.work_warps > warps) warps = pl.work_warps;
   }
   const int64_t segs = static_cast<int64_t>(num_seqs) * num_heads;
-  return header_bytes(num_seqs) + records_bytes(warps + segs, head_dim);
+  return counters_bytes(segs) + records_bytes(warps + segs, head_dim);
 }
 
 cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
