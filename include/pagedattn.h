@@ -128,16 +128,17 @@ size_t pa_paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head
  *   num_blocks     pool size in blocks (bounds check of table entries)
  *   workspace      device scratch of at least
  *                  pa_paged_attn_decode_workspace_size(...) bytes, 256-byte
- *                  aligned; no initial contents needed (its arrival counters
- *                  are tagged with a per-call epoch); must not be shared by
+ *                  aligned; no initial contents needed (its grain counter is
+ *                  tagged with a per-call epoch); must not be shared by
  *                  calls that may run at the same time
  *   d_status       nullable device int32 (see conventions)
- * Work is split over all SMs in equal runs of 16-token (head_dim 128) or
- * 32-token (head_dim 64) chunks; a (text, head) whose chunks span several
- * warps' runs is merged with a log-sum-exp reduction by the last of those
- * warps to finish.  One kernel launch, with programmatic dependent launch
- * after pa_kv_cache_write.  For fixed inputs, sizes and device the result is
- * bitwise reproducible.
+ * Work is split over all SMs in 16-token (head_dim 128) or 32-token
+ * (head_dim 64) chunks: static runs, then grains from a shared counter; a
+ * (text, head) whose chunks span several work units is merged with a
+ * log-sum-exp reduction by a second kernel on the same stream.  Both use
+ * programmatic dependent launch.  For fixed inputs, sizes and device the
+ * result is bitwise reproducible (which warp takes a grain does not change
+ * how it is computed or merged).
  * Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
  */
 int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -156,10 +157,10 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
  *
  * Same arguments, computation, result and errors as pa_paged_attn_decode,
  * minus workspace/workspace_bytes.  Its scratch is a static device array of
- * 8 MiB inside the library; every GPU that loads the library holds it until
+ * 16 MiB inside the library; every GPU that loads the library holds it until
  * the process exits.  Sizes whose workspace
- * (pa_paged_attn_decode_workspace_size) exceeds 8 MiB are rejected with
- * PA_ERR_TOO_LARGE before anything is launched (8 MiB covers, e.g., 256 texts
+ * (pa_paged_attn_decode_workspace_size) exceeds 16 MiB are rejected with
+ * PA_ERR_TOO_LARGE before anything is launched (16 MiB covers, e.g., 256 texts
  * x 40 heads x 128 on a 148-SM B200).  The call allocates and frees nothing.
  *
  * The first call on each device looks up the array's device address (a host

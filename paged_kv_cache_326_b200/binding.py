@@ -217,7 +217,7 @@ def pa_paged_attn_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: to
                                  v_cache: torch.Tensor, block_tables: torch.Tensor,
                                  context_lens: torch.Tensor, scale: float,
                                  status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """pa_paged_attn_decode with the library's own static 8 MiB scratch: for
+    """pa_paged_attn_decode with the library's own static 16 MiB scratch: for
     callers that cannot allocate device memory.  Calls that may overlap on
     the GPU share that scratch and race.  Raises PagedAttnError with code
     PA_ERR_TOO_LARGE when the sizes need more scratch than it holds."""

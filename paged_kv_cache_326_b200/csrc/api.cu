@@ -58,7 +58,7 @@ int pa_set_option(int key, int64_t value) {
   switch (key) {
     case PA_OPT_WAIT_LIMIT_NS: g_wait_limit_ns = value; return PA_OK;
     case PA_OPT_DECODE_WARPS:
-      if (value < 0 || value > (int64_t{1} << 24)) return PA_ERR_INVALID;
+      if (value < 0 || value > (int64_t{1} << 20)) return PA_ERR_INVALID;
       g_decode_warps = value;
       return PA_OK;
     default: return PA_ERR_INVALID;

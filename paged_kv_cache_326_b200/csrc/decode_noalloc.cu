@@ -18,9 +18,9 @@
 
 namespace {
 
-// 8 MiB of scratch, zero at load, kept by every GPU that loads the library
+// 16 MiB of scratch, zero at load, kept by every GPU that loads the library
 // until the process exits.  Enough for, e.g., 256 texts x 40 heads x 128.
-constexpr size_t kScratchBytes = size_t{8} << 20;
+constexpr size_t kScratchBytes = size_t{16} << 20;
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -1,5 +1,5 @@
 // paged_attn_decode: decode-phase attention through block tables, and the
-// log-sum-exp merge of partial results.
+// log-sum-exp merge of partial results (split_reduce_kernel).
 //
 // What it computes ("KV cache", section "How it works"; "The KV Cache and
 // PagedAttention", section "The Block Table"): for text s and head h, the new
@@ -13,33 +13,40 @@
 //  * The unit of work is a CHUNK: CH consecutive tokens of one (text, head)
 //    (CH = 16 at head_dim 128, 32 at head_dim 64, so a chunk's keys are 4 KB
 //    and keys + values 8 KB).  All chunks of all (text, head) pairs are laid
-//    out in one flat order (text-major, then head, then chunk) and cut into
-//    equal runs, one per warp of a persistent grid that fills every SM.  So
-//    long and short texts alike keep all 148 SMs busy to the end, with no
-//    tail wave.  A (text, head) whose chunks fall into several warps' runs
-//    produces one partial result per warp (running max m, sum l, unnormalised
-//    output o); the last of those warps to finish merges them (log-sum-exp),
-//    so no second kernel is needed.  One that falls inside a single run is
-//    finished in place.
+//    out in one flat order (text-major, then head, then chunk).  A persistent
+//    grid fills every SM; each warp first streams a static run of that order
+//    (about 70% of an even share), then takes grains of the rest from a
+//    shared counter.  Measured on B200, warps given equal bytes finish up to a
+//    third apart (SMs do not get equal shares of HBM bandwidth); the grains
+//    absorb that, so long and short texts alike keep all 148 SMs busy to the
+//    end.
+//  * A (text, head) whose chunks fall into several work units yields one
+//    partial result per unit (running max m, sum l, unnormalised output o),
+//    merged by split_reduce_kernel (log-sum-exp).  The merge is a second,
+//    tiny kernel rather than an in-kernel "last arriver" step because the
+//    GPU-scope atomics and fences that step needs stall the whole SM's
+//    streaming (measured: 12% to 27% slower per launch), while kernel order
+//    needs none.  A (text, head) that falls inside one unit is finished in
+//    place.
 //  * Each warp is its own pipeline: lane 0 issues bulk (TMA) copies of the
 //    chunk's key rows and value rows, straight from their physical blocks,
 //    into a ring of STAGES shared-memory stages, each with an mbarrier that
 //    counts the bytes landed; all 32 lanes consume.  The issue runs STAGES
-//    chunks ahead and crosses (text, head) boundaries, so the copy engine
-//    never idles at a boundary.  Only valid rows are copied: the unfilled tail
-//    of a text's last block is never read from HBM.
-//  * Block-table entries and context lengths for the next 32 chunks are
-//    fetched one per lane, 32 chunks before they are needed, and handed to
-//    the issuing lane with shuffles, so no table lookup sits on the critical
-//    path.
+//    chunks ahead and crosses (text, head) and unit boundaries, so the copy
+//    engine never idles at a boundary.  Only valid rows are copied: the
+//    unfilled tail of a text's last block is never read from HBM.
+//  * Block-table entries and context lengths are fetched one chunk per lane
+//    for a whole window of up to 32 chunks, a window ahead of use, and handed
+//    to the issuing lane with shuffles, so no table lookup sits on the
+//    critical path.
 //  * Dot products: a key row of head_dim elements is read by D/8 lanes as
 //    16-byte vectors and reduced with shuffles; the softmax is the online
 //    (running-max) form in fp32, in base 2 with log2(e) folded into the scale.
 //  * Every wait is bounded; a wait that gives up records PA_ERR_TIMEOUT,
 //    drains the copies in flight (bounded too) and returns.
-//  * Launched with programmatic dependent launch, so its CTAs are resident
-//    while the preceding cache write finishes; griddepcontrol.wait holds every
-//    read until that kernel's writes are visible.
+//  * Both kernels launch with programmatic dependent launch, so their CTAs
+//    are resident while the kernel before them finishes; griddepcontrol.wait
+//    holds every read until that kernel's writes are visible.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -66,20 +73,37 @@ namespace {
 constexpr int kDecodeWarps = PA_DECODE_WARPS;    // warps per CTA
 constexpr int kDecodeStages = PA_DECODE_STAGES;  // ring depth per warp
 constexpr int kMaxSeqs = 4096;
+// Work split: each warp first streams a static run of about kStaticPermille
+// per mille of an even share; the rest is handed out in grains from a shared
+// counter, at least kMinGrain chunks each and about kGrainsPerWarp per warp.
+#ifndef PA_STATIC_PERMILLE
+#define PA_STATIC_PERMILLE 700
+#endif
+#ifndef PA_MIN_GRAIN
+#define PA_MIN_GRAIN 16
+#endif
+constexpr int kStaticPermille = PA_STATIC_PERMILLE;
+constexpr int kGrainsPerWarp = 12;
+constexpr int kMinGrain = PA_MIN_GRAIN;
 constexpr int kDrainLimitNs = 1000000000;
-
 __host__ __device__ constexpr int chunk_tokens(int D) { return 2048 / D; }
 __host__ __device__ constexpr int stage_bytes(int D) { return 2 * 4096 + 2 * D + 128; }
 __host__ __device__ constexpr int warp_area_bytes(int D, int stages) { return stages * stage_bytes(D) + 128; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Arrival counters, one 64-bit word per (text, head): the call's epoch in
-// the top 40 bits, the number of partials stored so far in the low 24.  A
-// word whose epoch is not this call's counts as zero, so the workspace never
-// needs clearing.
-size_t counters_bytes(int64_t segs) { return align_up(sizeof(unsigned long long) * segs, 256); }
-constexpr int kCountBits = 24;
+// Workspace: a header (the work split, then prefix[S+1]), the grain counter,
+// then the partial records.  The header is written by CTA 0 of the decode
+// kernel and read by the merge kernel.
+constexpr int kHeaderInts = 8;  // total, q, G, W, 4 spare
+size_t header_bytes(int num_seqs) {
+  return align_up(sizeof(int32_t) * (kHeaderInts + num_seqs + 1), 256);
+}
+constexpr size_t kGrabBytes = 256;
+// The grain counter holds the call's epoch above bit 30; a stale epoch (an
+// earlier call's, or never set) reads as zero, so the workspace never needs
+// clearing.
+constexpr unsigned long long kGrabMask = (1ull << 30) - 1;
 constexpr unsigned long long kEpochMask = (1ull << 40) - 1;
 
 struct DecodeParams {
@@ -95,8 +119,9 @@ struct DecodeParams {
   int max_blocks_per_seq;
   int64_t num_blocks;
   int num_work_warps;
-  unsigned long long* counters;
-  unsigned long long epoch;  // 40-bit, never 0
+  int32_t* header;                // work split + prefix, for the merge kernel
+  unsigned long long* grab;       // grain counter
+  unsigned long long epoch;       // 40-bit, never 0
   float* records;
   int32_t* status;
   int64_t wait_limit_ns;
@@ -111,32 +136,7 @@ struct Lookahead {
 
 // Count one more stored partial of a (text, head) in this call; returns the
 // count including this one.
-// The compare-and-swap is acq_rel at GPU scope: it releases this warp's
-// partial (ordered before it by __syncwarp) and, for the last arriver,
-// acquires everyone else's.
-__device__ __forceinline__ unsigned long long cas_acq_rel(unsigned long long* p,
-                                                         unsigned long long cmp,
-                                                         unsigned long long val) {
-  unsigned long long old;
-  asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
-               : "=l"(old)
-               : "l"(p), "l"(cmp), "l"(val)
-               : "memory");
-  return old;
-}
-
-__device__ __forceinline__ uint32_t arrive_count(unsigned long long* ctr, unsigned long long epoch) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
-  while (true) {
-    const unsigned long long want =
-        (cur >> kCountBits) == epoch ? cur + 1 : (epoch << kCountBits) | 1ull;
-    const unsigned long long prev = cas_acq_rel(ctr, cur, want);
-    if (prev == cur) return static_cast<uint32_t>(want & ((1ull << kCountBits) - 1));
-    cur = prev;
-  }
-}
-
-// Merge the partials of one (text, head), stored by warps w_lo..w_hi: with
+// Merge the partials of one (text, head), stored by units w_lo..w_hi: with
 // M = max_i m_i and f_i = 2^(m_i - M),
 //     out = (sum_i f_i o_i) / (sum_i f_i l_i),
 // which equals the softmax-weighted sum over all the text's tokens (up to
@@ -146,32 +146,50 @@ template <typename T, int D>
 __device__ __forceinline__ void merge_partials(const float* records, T* out, int64_t sh, int w_lo,
                                                int w_hi, int lane) {
   constexpr int PER = D / 32;
-  // running maxima: one partial per lane, then a warp max
+  const int n = w_hi - w_lo + 1;
+  // running max over the partials, one partial per lane
   float M = -INFINITY;
-  for (int w0 = w_lo; w0 <= w_hi; w0 += 32) {
-    const int w = w0 + lane;
-    if (w <= w_hi) M = fmaxf(M, __ldcg(records + (w + sh) * (D + 4)));
-  }
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(records + (w_lo + i + sh) * (D + 4)));
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float L = 0.f;
   float acc[PER];
 #pragma unroll
   for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  for (int w = w_lo; w <= w_hi; ++w) {
-    const float* rec = records + (w + sh) * (D + 4);
-    const float f = M == -INFINITY ? 0.f : fast_exp2(__ldcg(rec) - M);
-    L = fmaf(f, __ldcg(rec + 1), L);
-    if constexpr (PER == 4) {
-      const float4 o = __ldcg(reinterpret_cast<const float4*>(rec + 4) + lane);
-      acc[0] = fmaf(f, o.x, acc[0]);
-      acc[1] = fmaf(f, o.y, acc[1]);
-      acc[2] = fmaf(f, o.z, acc[2]);
-      acc[3] = fmaf(f, o.w, acc[3]);
-    } else {
-      const float2 o = __ldcg(reinterpret_cast<const float2*>(rec + 4) + lane);
-      acc[0] = fmaf(f, o.x, acc[0]);
-      acc[1] = fmaf(f, o.y, acc[1]);
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    // weight f_i = 2^(m_i - M) of partial i0 + lane, and its share of the sum
+    float f = 0.f, lf = 0.f;
+    if (i0 + lane < n) {
+      const float* rec = records + (w_lo + i0 + lane + sh) * (D + 4);
+      f = M == -INFINITY ? 0.f : fast_exp2(__ldcg(rec) - M);
+      lf = f * __ldcg(rec + 1);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) lf += __shfl_xor_sync(0xffffffffu, lf, off);
+    L += lf;
+    // outputs: eight partials' loads in flight at a time
+    const int cnt = min(32, n - i0);
+    for (int b = 0; b < cnt; b += 8) {
+      float o[8][PER];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float* rec = records + (w_lo + i0 + min(b + u, cnt - 1) + sh) * (D + 4) + 4 + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(rec));
+          o[u][0] = v.x; o[u][1] = v.y; o[u][2] = v.z; o[u][3] = v.w;
+        } else {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(rec));
+          o[u][0] = v.x; o[u][1] = v.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float fu = __shfl_sync(0xffffffffu, f, min(b + u, 31));
+        if (b + u < cnt) {
+#pragma unroll
+          for (int k = 0; k < PER; ++k) acc[k] = fmaf(fu, o[u][k], acc[k]);
+        }
+      }
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -189,7 +207,7 @@ __device__ __forceinline__ void merge_partials(const float* records, T* out, int
 }  // namespace
 
 template <typename T, int D, int B, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32)
+__global__ void __launch_bounds__(WARPS * 32, 2)
 paged_decode_kernel(const DecodeParams p) {
   constexpr int CH = chunk_tokens(D);        // tokens per chunk
   constexpr int LPT = D / 8;                 // lanes per token row (16-byte vectors)
@@ -250,7 +268,22 @@ paged_decode_kernel(const DecodeParams p) {
   }
   const int total = prefix[S];
   const int W = p.num_work_warps;
-  const int cpw = (total + W - 1) / W;
+  // Static runs of q chunks (units 0..W-1), then grains of G chunks (units
+  // W, W+1, ...) covering the rest of the flat order.
+  int q = W == 1 ? total : static_cast<int>(static_cast<long long>(total) * kStaticPermille / 1000 / W);
+  if (q < 32 && W > 1) q = 0;
+  const int dyn_base = W * q;
+  const int dyn = total - dyn_base;
+  const int G = max(kMinGrain, (dyn + kGrainsPerWarp * W - 1) / (kGrainsPerWarp * W));
+  if (blockIdx.x == 0) {
+    if (tid == 0) {
+      p.header[0] = total;
+      p.header[1] = q;
+      p.header[2] = G;
+      p.header[3] = W;
+    }
+    for (int i = tid; i <= S; i += WARPS * 32) p.header[kHeaderInts + i] = prefix[i];
+  }
   // Texts with no tokens get zeros (spread over the CTAs).
   for (int s = blockIdx.x; s < S; s += gridDim.x) {
     if (prefix[s + 1] == prefix[s]) {
@@ -261,10 +294,6 @@ paged_decode_kernel(const DecodeParams p) {
 
   const int w = blockIdx.x * WARPS + warp;
   if (w >= W || total == 0) return;
-  const int c0 = w * cpw;
-  const int c1 = min(total, c0 + cpw);
-  if (c0 >= c1) return;
-  const int n = c1 - c0;
 
   uint8_t* area = smem + warp * AREA;
   uint64_t* bars = reinterpret_cast<uint64_t*>(area + STAGES * STRIDE);
@@ -283,11 +312,100 @@ paged_decode_kernel(const DecodeParams p) {
   int step = 1;
   while (step * 2 <= S) step *= 2;
 
-  // Where flat chunk c0 + pos lives.  Reads only shared memory before issuing
-  // its global loads, whose results are not used for 32 - STAGES chunks.
-  auto lookahead = [&](int pos) {
+  // ---- work units and their windows ----------------------------------
+  // A unit is a run of consecutive flat chunks: first this warp's static run,
+  // then grains taken from the shared counter.  Units are cut into windows of
+  // at most 32 chunks (one chunk per lane for the look-ahead); a unit's last
+  // two windows are balanced, so only the very last window of all the work
+  // can be shorter than the copy ring.
+  const unsigned long long e34 = p.epoch & ((1ull << 34) - 1);
+  // Chunk offset of the grain whose counter value is `old` (lane 0).  The
+  // counter carries this call's epoch above bit 30; a stale epoch (left by an
+  // earlier call, or never set) is replaced by compare-and-swap, so the
+  // workspace never needs clearing.
+  auto grab_resolve = [&](unsigned long long old) -> int {
+    if ((old >> 30) == e34) return static_cast<int>(old & kGrabMask);
+    unsigned long long seen = old + static_cast<unsigned long long>(G);
+    while (true) {
+      if ((seen >> 30) == e34) {
+        const unsigned long long o2 = atomicAdd(p.grab, static_cast<unsigned long long>(G));
+        if ((o2 >> 30) == e34) return static_cast<int>(o2 & kGrabMask);
+        seen = o2 + static_cast<unsigned long long>(G);
+        continue;
+      }
+      const unsigned long long prev =
+          atomicCAS(p.grab, seen, (e34 << 30) | static_cast<unsigned long long>(G));
+      if (prev == seen) return 0;
+      seen = prev;
+    }
+  };
+  bool static_taken = false, exhausted = false, pend_live = false;
+  unsigned long long pend = 0;  // lane 0: counter value of the next grain
+  int u_start = 0, u_count = 0, u_id = -1, u_off = 0;
+  auto grab_issue = [&]() {
+    if (lane == 0) pend = atomicAdd(p.grab, static_cast<unsigned long long>(G));
+    pend_live = true;
+  };
+  auto next_unit = [&]() {
+    if (!static_taken) {
+      static_taken = true;
+      if (q > 0) {
+        u_start = w * q;
+        u_count = q;
+        u_id = w;
+        u_off = 0;
+        if (dyn > 0) grab_issue();
+        return;
+      }
+    }
+    if (dyn <= 0) {
+      exhausted = true;
+      return;
+    }
+    if (!pend_live) grab_issue();
+    int off = 0;
+    if (lane == 0) off = grab_resolve(pend);
+    off = __shfl_sync(0xffffffffu, off, 0);
+    pend_live = false;
+    if (off >= dyn) {
+      exhausted = true;
+      return;
+    }
+    u_start = dyn_base + off;
+    u_count = min(G, dyn - off);
+    u_id = W + off / G;
+    u_off = 0;
+    grab_issue();  // the next grain, resolved when this one runs out
+  };
+  // Next window of this warp's work: start chunk, count (0 = no more), unit.
+  auto next_window = [&](int& ws, int& wc, int& wu) {
+    if (!exhausted && u_off >= u_count) next_unit();
+    if (exhausted) {
+      ws = 0;
+      wc = 0;
+      wu = -1;
+      return;
+    }
+    const int rem = u_count - u_off;
+    const int n = rem <= 32 ? rem : (rem < 64 ? rem / 2 : 32);
+    ws = u_start + u_off;
+    wc = n;
+    wu = u_id;
+    u_off += n;
+  };
+
+  // Where each chunk of a window lives, one chunk per lane.  Reads only
+  // shared memory before issuing its global loads, whose results are not
+  // used until the copy issue reaches this window.
+  auto lookahead = [&](int ws, int wc) {
     Lookahead<NB> e;
-    const int c = c0 + min(pos, n - 1);
+    if (wc <= 0) {
+      e.s = e.h = e.j = e.len = 0;
+#pragma unroll
+      for (int k = 0; k < NB; ++k) e.blk[k] = -1;
+      return e;
+    }
+    const int c = ws + min(lane, wc - 1);
     int s = 0;
     for (int st = step; st > 0; st >>= 1)
       if (s + st < S && prefix[s + st] <= c) s += st;
@@ -309,17 +427,29 @@ paged_decode_kernel(const DecodeParams p) {
     return e;
   };
 
-  Lookahead<NB> win0 = lookahead(lane);
-  Lookahead<NB> win1 = lookahead(32 + lane);
-  int base = 0;
+  int ws0, wc0, wu0, ws1, wc1, wu1;
+  next_window(ws0, wc0, wu0);
+  next_window(ws1, wc1, wu1);
+  Lookahead<NB> win0 = lookahead(ws0, wc0);
+  Lookahead<NB> win1 = lookahead(ws1, wc1);
+  int i0 = 0;       // consumer's index in window 0
+  int issued = 0;   // chunks whose copies were issued (stage = issued % STAGES)
 
-  // Issue the copies of chunk `pos` into stage pos % STAGES (lane 0 copies,
-  // every lane takes part in the shuffles).
-  auto issue = [&](int pos) {
-    if (pos >= n) return;
-    int src = pos - base;
-    const bool hi = src >= 32;
-    src &= 31;
+  // Issue the copies of the chunk `k` places after the start of window 0 into
+  // the next stage (lane 0 copies, every lane takes part in the shuffles).
+  auto issue = [&](int k) {
+    bool hi;
+    int src;
+    if (k < wc0) {
+      hi = false;
+      src = k;
+    } else if (k - wc0 < wc1) {
+      hi = true;
+      src = k - wc0;
+    } else {
+      return;  // no more work
+    }
+    const bool unit_start = src == 0 && (hi ? wu1 != wu0 : issued == 0);
     const int s = __shfl_sync(0xffffffffu, hi ? win1.s : win0.s, src);
     const int h = __shfl_sync(0xffffffffu, hi ? win1.h : win0.h, src);
     const int j = __shfl_sync(0xffffffffu, hi ? win1.j : win0.j, src);
@@ -327,8 +457,9 @@ paged_decode_kernel(const DecodeParams p) {
     int blk[NB];
 #pragma unroll
     for (int k = 0; k < NB; ++k) blk[k] = __shfl_sync(0xffffffffu, hi ? win1.blk[k] : win0.blk[k], src);
+    const int st = issued % STAGES;
+    ++issued;
     if (lane == 0) {
-      const int st = pos % STAGES;
       uint8_t* stage = area + st * STRIDE;
       T* sK = reinterpret_cast<T*>(stage);
       T* sV = sK + TILE;
@@ -336,7 +467,7 @@ paged_decode_kernel(const DecodeParams p) {
       int32_t* flag = reinterpret_cast<int32_t*>(stage + 2 * 4096 + 2 * D);
       const int len = min(max(len_raw, 0), cap);
       const int nvalid = min(CH, len - j * CH);
-      const bool first = (pos == 0) || (j == 0);
+      const bool first = unit_start || j == 0;
       // rows of this chunk that each touched block supplies
       bool bad = false;
 #pragma unroll
@@ -374,7 +505,7 @@ paged_decode_kernel(const DecodeParams p) {
   };
 
 #pragma unroll
-  for (int pos = 0; pos < STAGES; ++pos) issue(pos);
+  for (int k = 0; k < STAGES; ++k) issue(k);
 
   const int dchunk = lane % LPT;
   const int tsub = lane / LPT;
@@ -382,24 +513,19 @@ paged_decode_kernel(const DecodeParams p) {
   float acc[8];
   float m = -INFINITY, lsum = 0.f;
   int piece_j0 = 0;
+  int prev_unit = -1;
 
-  for (int pos = 0; pos < n; ++pos) {
-    if (pos - base == 32) {
-      base += 32;
-      win0 = win1;
-      win1 = lookahead(base + 32 + lane);
-    }
-    const int src = pos - base;
-    const int s = __shfl_sync(0xffffffffu, win0.s, src);
-    const int h = __shfl_sync(0xffffffffu, win0.h, src);
-    const int j = __shfl_sync(0xffffffffu, win0.j, src);
-    const int len = min(max(__shfl_sync(0xffffffffu, win0.len, src), 0), cap);
+  for (int pos = 0; wc0 > 0; ++pos) {
+    const int s = __shfl_sync(0xffffffffu, win0.s, i0);
+    const int h = __shfl_sync(0xffffffffu, win0.h, i0);
+    const int j = __shfl_sync(0xffffffffu, win0.j, i0);
+    const int len = min(max(__shfl_sync(0xffffffffu, win0.len, i0), 0), cap);
     const int st = pos % STAGES;
     const uint32_t parity = (pos / STAGES) & 1;
 
     if (!mbar_wait_bounded(&bars[st], parity, p.wait_limit_ns)) {
       set_status(p.status, -10 /* PA_ERR_TIMEOUT */);
-      for (int d = pos; d < min(pos + STAGES, n); ++d)
+      for (int d = pos; d < issued; ++d)
         mbar_wait_bounded(&bars[d % STAGES], (d / STAGES) & 1, kDrainLimitNs);
       return;
     }
@@ -410,7 +536,7 @@ paged_decode_kernel(const DecodeParams p) {
     const T* sQ = sV + TILE;
     const int bad = *reinterpret_cast<const int32_t*>(stage + 2 * 4096 + 2 * D);
 
-    if (pos == 0 || j == 0) {
+    if (j == 0 || wu0 != prev_unit) {
       piece_j0 = j;
       float qraw[8];
       unpack8<T>(*reinterpret_cast<const uint4*>(sQ + dchunk * 8), qraw);
@@ -487,10 +613,11 @@ paged_decode_kernel(const DecodeParams p) {
     // This stage is consumed: refill it before the epilogue, whose global
     // stores and (rarely) merge must not leave the copy engine idle.
     __syncwarp();
-    issue(pos + STAGES);
+    issue(i0 + STAGES);
 
     const int ns = (len + CH - 1) / CH;
-    if (pos == n - 1 || j == ns - 1) {
+    const bool unit_ends = i0 + 1 == wc0 && (wc1 == 0 || wu1 != wu0);
+    if (unit_ends || j == ns - 1) {
       float l_all = lsum;
       float o[8];
 #pragma unroll
@@ -510,7 +637,7 @@ paged_decode_kernel(const DecodeParams p) {
           *reinterpret_cast<uint4*>(static_cast<T*>(p.out) + sh * D + dchunk * 8) = pack8<T>(o);
         }
       } else {
-        float* rec = p.records + (static_cast<int64_t>(w) + sh) * (D + 4);
+        float* rec = p.records + (static_cast<int64_t>(wu0) + sh) * (D + 4);
         if (lane == 0) {
           rec[0] = m;
           rec[1] = l_all;
@@ -520,22 +647,50 @@ paged_decode_kernel(const DecodeParams p) {
           dst[0] = make_float4(o[0], o[1], o[2], o[3]);
           dst[1] = make_float4(o[4], o[5], o[6], o[7]);
         }
-        // Publish the partial, count it; the warp that stores the last one
-        // of this (text, head) merges them all.
-        __syncwarp();
-        const int a = prefix[s] + h * ns;
-        const int w_lo = a / cpw;
-        const int w_hi = (a + ns - 1) / cpw;
-        uint32_t cnt = 0;
-        if (lane == 0) cnt = arrive_count(p.counters + sh, p.epoch);
-        cnt = __shfl_sync(0xffffffffu, cnt, 0);
-        if (cnt == static_cast<uint32_t>(w_hi - w_lo + 1)) {
-          __syncwarp();  // order lane 0's acquire before every lane's reads
-          merge_partials<T, D>(p.records, static_cast<T*>(p.out), sh, w_lo, w_hi, lane);
-        }
       }
     }
+
+    prev_unit = wu0;
+    if (++i0 == wc0) {  // window 0 done: the next one moves up
+      ws0 = ws1;
+      wc0 = wc1;
+      wu0 = wu1;
+      win0 = win1;
+      next_window(ws1, wc1, wu1);
+      win1 = lookahead(ws1, wc1);
+      i0 = 0;
+    }
   }
+}
+
+// Merge kernel: for every (text, head) whose chunks fell into several work
+// units, combine the units' partials (log-sum-exp); the decode kernel has
+// already written every other output.  Launched right after the decode
+// kernel with programmatic dependent launch: its CTAs become resident early
+// and griddepcontrol.wait holds them until the decode kernel's writes are
+// visible.  One warp per (text, head).
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
+                    const float* __restrict__ records, int num_seqs, int num_heads) {
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int seg = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (seg >= num_seqs * num_heads) return;
+  const int s = seg / num_heads;
+  const int h = seg - s * num_heads;
+  const int q = header[1], G = header[2], W = header[3];
+  const int32_t* prefix = header + kHeaderInts;
+  const int seg0 = prefix[s];
+  const int ns = (prefix[s + 1] - seg0) / num_heads;
+  if (ns == 0) return;  // zero-filled by the decode kernel
+  const int dyn_base = W * q;
+  auto unit_of = [&](int c) { return c < dyn_base ? c / q : W + (c - dyn_base) / G; };
+  const int a = seg0 + h * ns;
+  const int u_lo = unit_of(a);
+  const int u_hi = unit_of(a + ns - 1);
+  if (u_lo == u_hi) return;  // finished in place by the decode kernel
+  merge_partials<T, D>(records, out, seg, u_lo, u_hi, lane);
 }
 
 namespace {
@@ -625,6 +780,10 @@ Plan plan_decode(const void* kernel, int D, int B, int num_seqs, int num_heads,
   return pl;
 }
 
+// Units (static runs plus grains) a launch with `warps` working warps can
+// create: grains number at most kGrainsPerWarp per warp.
+int64_t max_units(int64_t warps) { return warps * (kGrainsPerWarp + 1) + 1; }
+
 size_t records_bytes(int64_t records, int D) {
   return static_cast<size_t>(records) * (D + 4) * sizeof(float);
 }
@@ -640,7 +799,8 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
                               a.max_blocks_per_seq, a.forced_warps);
   if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
   const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_heads;
-  const size_t need = counters_bytes(segs) + records_bytes(pl.work_warps + segs, D);
+  const size_t need = header_bytes(a.num_seqs) + kGrabBytes +
+                      records_bytes(max_units(pl.work_warps) + segs, D);
   if (a.workspace_bytes < need) return cudaErrorInvalidValue;
   DecodeParams p;
   p.out = a.out;
@@ -655,9 +815,11 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   p.max_blocks_per_seq = a.max_blocks_per_seq;
   p.num_blocks = a.num_blocks;
   p.num_work_warps = pl.work_warps;
-  p.counters = static_cast<unsigned long long*>(a.workspace);
+  char* ws = static_cast<char*>(a.workspace);
+  p.header = reinterpret_cast<int32_t*>(ws);
+  p.grab = reinterpret_cast<unsigned long long*>(ws + header_bytes(a.num_seqs));
   p.epoch = next_epoch();
-  p.records = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + counters_bytes(segs));
+  p.records = reinterpret_cast<float*>(ws + header_bytes(a.num_seqs) + kGrabBytes);
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
   cudaLaunchConfig_t cfg = {};
@@ -671,6 +833,14 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(&cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages>, p);
+  if (err != cudaSuccess) return err;
+  const int per_cta = 8;  // warps, one per (text, head)
+  cfg.gridDim = dim3(static_cast<unsigned>((segs + per_cta - 1) / per_cta));
+  cfg.blockDim = dim3(per_cta * 32);
+  cfg.dynamicSmemBytes = 0;
+  err = cudaLaunchKernelEx(&cfg, split_reduce_kernel<T, D>, static_cast<T*>(a.out),
+                           static_cast<const int32_t*>(p.header),
+                           static_cast<const float*>(p.records), a.num_seqs, a.num_heads);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
@@ -734,7 +904,7 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int blo
     if (pl.work_warps > warps) warps = pl.work_warps;
   }
   const int64_t segs = static_cast<int64_t>(num_seqs) * num_heads;
-  return counters_bytes(segs) + records_bytes(warps + segs, head_dim);
+  return header_bytes(num_seqs) + kGrabBytes + records_bytes(max_units(warps) + segs, head_dim);
 }
 
 cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {

@@ -219,7 +219,7 @@ def test_run_to_run_bitwise_determinism():
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
-@pytest.mark.parametrize("warps", [1, 7, 100000])
+@pytest.mark.parametrize("warps", [1, 7, 4096])
 def test_split_and_single_pass_agree(warps):
     """1 warp: no text is split (single pass).  Many warps: every text is cut
     into many partials merged by the log-sum-exp reduce.  Both match the

@@ -68,12 +68,12 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(P, make):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(P):
-    """Sizes whose workspace exceeds the static 8 MiB come back as
+    """Sizes whose workspace exceeds the static 16 MiB come back as
     PA_ERR_TOO_LARGE before any launch (null data pointers are never
     touched)."""
     lib = P.lib()
     S, H, D, B, MB = 4096, 64, 128, 16, 128
-    assert P.pa_paged_attn_decode_workspace_size(S, H, D, B, MB) > (8 << 20)
+    assert P.pa_paged_attn_decode_workspace_size(S, H, D, B, MB) > (16 << 20)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = lib.pa_paged_attn_decode_noalloc(None, None, None, None, None, None, ctypes.c_float(1.0),
                                           S, H, D, B, MB, 1 << 20, P.binding.PA_F16,
