@@ -1,10 +1,13 @@
 """Benchmark: one decode step of an OPT-13B-shaped layer, batch 64.
 
-A step is the whole hot path once: the write of each text's new key/value
-(pa_kv_cache_write), then paged decode attention over every text's cache
-(pa_paged_attn_decode: the decode kernel plus its log-sum-exp merge).
+A step is the whole hot path once: the write of each text's new key/value,
+then paged decode attention over every text's cache.  By default it is the
+one-launch entry point pa_decode_step (write + attention in the decode
+kernel, then the log-sum-exp merge kernel); ``--path calls`` times the two
+calls pa_kv_cache_write + pa_paged_attn_decode instead.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--path fused|calls]
 
 Prints one JSON line (rank 0).  ``value`` is KV bytes read per step / device
 time per step (GB/s, whole job over all ranks); ``e2e`` repeats it with the
@@ -232,6 +235,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["fused", "calls"], default="fused")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -256,14 +260,29 @@ def main():
     lens = w.context_lens.tolist()
     step_kv = kv_bytes(lens, H, D, eb)
     decode_bytes = step_kv + 2 * S * H * D * eb + sum(4 * -(-L // w.block_size) for L in lens) + 4 * S
+    write_bytes = 4 * S * H * D * eb + 8 * S   # k, v read and stored; slots
+    fused = args.path == "fused"
+    if fused:
+        decode_bytes += write_bytes
     out = torch.empty_like(w.q)
     ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
+    def write_part(k, v, slots):
+        if not fused:
+            P.pa_kv_cache_write(k, v, w.k_cache, w.v_cache, slots, status=status)
+
+    def decode_part(q, k, v, slots, tables, lens):
+        if fused:
+            P.pa_decode_step(out, q, k, v, w.k_cache, w.v_cache, slots, tables, lens, w.scale,
+                             workspace=ws, status=status)
+        else:
+            P.pa_paged_attn_decode(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
+                                   workspace=ws, status=status)
+
     def step():
-        P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
-        P.pa_paged_attn_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
-                               w.scale, workspace=ws, status=status)
+        write_part(w.k, w.v, w.slot_mapping)
+        decode_part(w.q, w.k, w.v, w.slot_mapping, w.block_tables, w.context_lens)
 
     def barrier():
         if world > 1:
@@ -287,10 +306,9 @@ def main():
         start.record(stream)
         for i in range(K):
             ev[i][0].record(stream)
-            P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+            write_part(w.k, w.v, w.slot_mapping)
             ev[i][1].record(stream)
-            P.pa_paged_attn_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables,
-                                   w.context_lens, w.scale, workspace=ws, status=status)
+            decode_part(w.q, w.k, w.v, w.slot_mapping, w.block_tables, w.context_lens)
             ev[i][2].record(stream)
         stop.record(stream)
         torch.cuda.synchronize()
@@ -317,9 +335,8 @@ def main():
     def e2e_step():
         for d, h in ((dq, hq), (dk, hk), (dv, hv), (dslot, hslot), (dtab, htab), (dlen, hlen)):
             d.copy_(h, non_blocking=True)
-        P.pa_kv_cache_write(dk, dv, w.k_cache, w.v_cache, dslot, status=status)
-        P.pa_paged_attn_decode(out, dq, w.k_cache, w.v_cache, dtab, dlen, w.scale, workspace=ws,
-                               status=status)
+        write_part(dk, dv, dslot)
+        decode_part(dq, dk, dv, dslot, dtab, dlen)
         hout.copy_(out, non_blocking=True)
 
     Ke = max(3, min(K, 1000))
@@ -358,17 +375,20 @@ def main():
                    "block_size": w.block_size, "context_lens": "uniform [128, 2048], seed 2+rank",
                    "num_blocks": w.num_blocks, "kv_bytes_per_step": step_kv,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB)",
-                   "parallelism": f"independent batch per GPU x{world}"},
+                   "parallelism": f"independent batch per GPU x{world}",
+                   "path": "pa_decode_step" if fused else "pa_kv_cache_write + pa_paged_attn_decode"},
         "decode_tokens_per_s": world * S / (ms_step * 1e-3),
         "pct_of_nominal_8tbs": 100.0 * (value / world) / NOMINAL_HBM_GBS,
-        "kernel_ms": {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms},
+        "kernel_ms": ({"pa_decode_step": decode_ms} if fused else
+                      {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic_per_launch(),
-                     "kernel": "pa_paged_attn_decode (decode kernel + split reduce)",
+                     "kernel": ("pa_decode_step (decode kernel with the cache write, + merge kernel)"
+                                if fused else "pa_paged_attn_decode (decode kernel + merge kernel)"),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": decode_bytes},
         "e2e": {"value": world * step_kv / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 3 * K,
+        "gpu_launches": (2 if fused else 3) * K,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -149,6 +149,33 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
                          pa_stream_t stream);
 
 /*
+ * pa_decode_step — one whole decode step of one layer in one launch (plus the
+ * merge): the cache write of pa_kv_cache_write for one new token per text,
+ * then the attention of pa_paged_attn_decode.  A B200 fusion of the pages'
+ * two steps ("KV cache", section "How it works": the new token's key and
+ * value are written into the cache and take part in its own attention).
+ *
+ *   k, v           [num_seqs][num_heads][head_dim] dt: each text's new token
+ *   slot_mapping   [num_seqs] int64: its slot (negative: not stored)
+ *   other arguments as for pa_paged_attn_decode (same workspace size).
+ *
+ * Result: the pool afterwards and `out` are exactly those of
+ * pa_kv_cache_write(k, v, ..., slot_mapping, num_tokens = num_seqs) followed
+ * by pa_paged_attn_decode, provided slot_mapping[s] is the slot of position
+ * context_lens[s] - 1 of text s (what the block manager's append_slot
+ * returns) and no text reads another text's new slot (written blocks are
+ * private after copy-on-write).  The attention takes position
+ * context_lens[s] - 1 from k[s], v[s] directly, so the launch never waits on
+ * its own write.  Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_decode_step(void* out, const void* q, const void* k, const void* v, void* k_cache,
+                   void* v_cache, const int64_t* slot_mapping, const int32_t* block_tables,
+                   const int32_t* context_lens, float scale, int num_seqs, int num_heads,
+                   int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                   pa_dtype dt, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                   pa_stream_t stream);
+
+/*
  * pa_paged_attn_decode_noalloc — pa_paged_attn_decode without a caller
  * workspace, for callers that cannot allocate device memory (a host framework
  * that owns every device allocation, a fixed memory budget, a loop where an

@@ -64,6 +64,8 @@ _SIGNATURES = {
     "pa_paged_attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "pa_paged_attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _i32,
                                     _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
+    "pa_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
+                              _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_paged_attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
                                             _i32, _i32, _i64, _i32, _vp, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
@@ -210,6 +212,40 @@ def pa_paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tens
         _dtype_code(q), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _status_ptr(status), _stream(stream, q.device))
     _check(code, "pa_paged_attn_decode")
+    return out
+
+
+def pa_decode_step(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                   k_cache: torch.Tensor, v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                   block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                   workspace: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Cache write of each text's new token plus decode attention, one launch.
+    q, k, v, out: [S][H][D]; slot_mapping [S] int64 (the slot of position
+    context_lens[s] - 1)."""
+    S, H, D = q.shape
+    N, H2, B, D2 = k_cache.shape
+    if (out.shape != q.shape or k.shape != q.shape or v.shape != q.shape
+            or v_cache.shape != k_cache.shape or (H2, D2) != (H, D)):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S][max_blocks], context_lens [S]")
+    if slot_mapping.shape != (S,):
+        raise ValueError("slot_mapping must be [num_seqs]")
+    for t in (out, k, v, k_cache, v_cache):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, out and the caches must share a dtype")
+    MB = block_tables.shape[1]
+    if workspace is None:
+        workspace = workspace_for(q, B, MB)
+    code = lib().pa_decode_step(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache"),
+        _cuda(v_cache, "v_cache"), _cuda(slot_mapping, "slot_mapping", torch.int64),
+        _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(context_lens, "context_lens", torch.int32), float(scale), S, H, D, B, MB, N,
+        _dtype_code(q), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _status_ptr(status), _stream(stream, q.device))
+    _check(code, "pa_decode_step")
     return out
 
 

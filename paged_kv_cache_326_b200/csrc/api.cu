@@ -126,4 +126,47 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
   return from_cuda(pa::launch_paged_attn_decode(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int pa_decode_step(void* out, const void* q, const void* k, const void* v, void* k_cache,
+                   void* v_cache, const int64_t* slot_mapping, const int32_t* block_tables,
+                   const int32_t* context_lens, float scale, int num_seqs, int num_heads,
+                   int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                   pa_dtype dt, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                   pa_stream_t stream) {
+  if (num_seqs == 0) return PA_OK;
+  if (!pa::decode_sizes_supported(num_seqs, num_heads, head_dim, block_size,
+                                  max_blocks_per_seq) ||
+      num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16))
+    return PA_ERR_INVALID;
+  if (!out || !q || !k || !v || !k_cache || !v_cache || !slot_mapping || !block_tables ||
+      !context_lens || !workspace)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return PA_ERR_INVALID;
+  pa::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.scale = scale;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.is_bf16 = dt == PA_BF16;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  a.status = d_status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.forced_warps = g_decode_warps.load();
+  a.k_new = k;
+  a.v_new = v;
+  a.slot_mapping = slot_mapping;
+  return from_cuda(pa::launch_paged_attn_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -32,6 +32,10 @@ struct DecodeArgs {
   int32_t* status;
   int64_t wait_limit_ns;
   int64_t forced_warps;  // 0 = fill the device
+  // Fused decode step (pa_decode_step) only; all null otherwise.
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  const int64_t* slot_mapping = nullptr;
 };
 
 bool decode_sizes_supported(int num_seqs, int num_heads, int head_dim, int block_size,

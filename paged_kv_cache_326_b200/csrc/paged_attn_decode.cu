@@ -119,6 +119,9 @@ struct DecodeParams {
   int max_blocks_per_seq;
   int64_t num_blocks;
   int num_work_warps;
+  const void* k_new;              // fused step only: the new token's k, v [S][H][D]
+  const void* v_new;
+  const int64_t* slot_mapping;    // fused step only: their slots
   int32_t* header;                // work split + prefix, for the merge kernel
   unsigned long long* grab;       // grain counter
   unsigned long long epoch;       // 40-bit, never 0
@@ -206,7 +209,10 @@ __device__ __forceinline__ void merge_partials(const float* records, T* out, int
 
 }  // namespace
 
-template <typename T, int D, int B, int WARPS, int STAGES>
+// FUSED: also store each text's new key/value at its slot, and take the
+// text's last position (the new token) from the inputs instead of the pool,
+// so nothing in this launch waits on its own write.
+template <typename T, int D, int B, int WARPS, int STAGES, bool FUSED>
 __global__ void __launch_bounds__(WARPS * 32, 2)
 paged_decode_kernel(const DecodeParams p) {
   constexpr int CH = chunk_tokens(D);        // tokens per chunk
@@ -293,7 +299,41 @@ paged_decode_kernel(const DecodeParams p) {
   }
 
   const int w = blockIdx.x * WARPS + warp;
-  if (w >= W || total == 0) return;
+  // Fused step: the cache write, 16-byte vectors spread over the working
+  // warps (as in kv_cache_write_kernel).  No read in this launch touches
+  // these slots, so each warp does its share whenever it has a moment: right
+  // after issuing its first copies, while it waits for them.
+  auto fused_write = [&]() {
+    if constexpr (FUSED) {
+      const int vpr = D / 8;
+      const int64_t per_text = static_cast<int64_t>(H) * vpr;
+      const int64_t nvec = per_text * S;
+      const int64_t num_slots = p.num_blocks * B;
+      uint4* kcw = static_cast<uint4*>(const_cast<void*>(p.k_cache));
+      uint4* vcw = static_cast<uint4*>(const_cast<void*>(p.v_cache));
+      for (int64_t i = static_cast<int64_t>(w) * 32 + lane; i < nvec;
+           i += static_cast<int64_t>(W) * 32) {
+        const int64_t s = i / per_text;
+        const int64_t r = i - s * per_text;
+        const int64_t slot = __ldg(p.slot_mapping + s);
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+          if (r == 0) set_status(p.status, -9 /* PA_ERR_BAD_SLOT */);
+          continue;
+        }
+        const int64_t h = r / vpr, c = r - (r / vpr) * vpr;
+        const int64_t blk = slot / B, place = slot - blk * B;
+        const int64_t dst = ((blk * H + h) * B + place) * vpr + c;
+        kcw[dst] = __ldg(static_cast<const uint4*>(p.k_new) + i);
+        vcw[dst] = __ldg(static_cast<const uint4*>(p.v_new) + i);
+      }
+    }
+  };
+  if (w >= W) return;
+  if (total == 0) {
+    fused_write();
+    return;
+  }
 
   uint8_t* area = smem + warp * AREA;
   uint64_t* bars = reinterpret_cast<uint64_t*>(area + STAGES * STRIDE);
@@ -484,10 +524,14 @@ paged_decode_kernel(const DecodeParams p) {
       if (first)
         bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * H + h) * D, D * 2, &bars[st], policy);
       if (!bad) {
+        // Fused step: the chunk holding the text's last position takes that
+        // row from the new k/v instead of the pool.
+        const bool new_row = FUSED && j * CH + nvalid == len;
+        const int pool_rows = nvalid - (new_row ? 1 : 0);
         if constexpr (CH >= B) {
 #pragma unroll
           for (int k = 0; k < NB; ++k) {
-            const int rows = min(B, nvalid - k * B);
+            const int rows = min(B, pool_rows - k * B);
             if (rows > 0) {
               const int64_t off = (static_cast<int64_t>(blk[k]) * H + h) * B * D;
               bulk_copy_g2s(sK + k * B * D, kc + off, rows * D * 2, &bars[st], policy);
@@ -497,8 +541,17 @@ paged_decode_kernel(const DecodeParams p) {
         } else {
           const int row0 = (j * CH) % B;
           const int64_t off = ((static_cast<int64_t>(blk[0]) * H + h) * B + row0) * D;
-          bulk_copy_g2s(sK, kc + off, nvalid * D * 2, &bars[st], policy);
-          bulk_copy_g2s(sV, vc + off, nvalid * D * 2, &bars[st], policy);
+          if (pool_rows > 0) {
+            bulk_copy_g2s(sK, kc + off, pool_rows * D * 2, &bars[st], policy);
+            bulk_copy_g2s(sV, vc + off, pool_rows * D * 2, &bars[st], policy);
+          }
+        }
+        if (new_row) {
+          const int64_t src_off = (static_cast<int64_t>(s) * H + h) * D;
+          bulk_copy_g2s(sK + pool_rows * D, static_cast<const T*>(p.k_new) + src_off, D * 2,
+                        &bars[st], policy);
+          bulk_copy_g2s(sV + pool_rows * D, static_cast<const T*>(p.v_new) + src_off, D * 2,
+                        &bars[st], policy);
         }
       }
     }
@@ -506,6 +559,7 @@ paged_decode_kernel(const DecodeParams p) {
 
 #pragma unroll
   for (int k = 0; k < STAGES; ++k) issue(k);
+  fused_write();
 
   const int dchunk = lane % LPT;
   const int tsub = lane / LPT;
@@ -788,14 +842,15 @@ size_t records_bytes(int64_t records, int D) {
   return static_cast<size_t>(records) * (D + 4) * sizeof(float);
 }
 
-template <typename T, int D, int B>
+template <typename T, int D, int B, bool FUSED = false>
 const void* decode_kernel_ptr() {
-  return reinterpret_cast<const void*>(&paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages>);
+  return reinterpret_cast<const void*>(
+      &paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED>);
 }
 
-template <typename T, int D, int B>
+template <typename T, int D, int B, bool FUSED>
 cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
-  const Plan pl = plan_decode(decode_kernel_ptr<T, D, B>(), D, B, a.num_seqs, a.num_heads,
+  const Plan pl = plan_decode(decode_kernel_ptr<T, D, B, FUSED>(), D, B, a.num_seqs, a.num_heads,
                               a.max_blocks_per_seq, a.forced_warps);
   if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
   const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_heads;
@@ -822,6 +877,9 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   p.records = reinterpret_cast<float*>(ws + header_bytes(a.num_seqs) + kGrabBytes);
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.k_new = a.k_new;
+  p.v_new = a.v_new;
+  p.slot_mapping = a.slot_mapping;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(kDecodeWarps * 32);
@@ -832,7 +890,8 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages>, p);
+  cudaError_t err = cudaLaunchKernelEx(
+      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED>, p);
   if (err != cudaSuccess) return err;
   const int per_cta = 8;  // warps, one per (text, head)
   cfg.gridDim = dim3(static_cast<unsigned>((segs + per_cta - 1) / per_cta));
@@ -845,33 +904,33 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <typename T, int D>
+template <typename T, int D, bool FUSED>
 cudaError_t dispatch_block(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.block_size) {
-    case 4: return launch_typed<T, D, 4>(a, stream);
-    case 8: return launch_typed<T, D, 8>(a, stream);
-    case 16: return launch_typed<T, D, 16>(a, stream);
-    case 32: return launch_typed<T, D, 32>(a, stream);
+    case 4: return launch_typed<T, D, 4, FUSED>(a, stream);
+    case 8: return launch_typed<T, D, 8, FUSED>(a, stream);
+    case 16: return launch_typed<T, D, 16, FUSED>(a, stream);
+    case 32: return launch_typed<T, D, 32, FUSED>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T>
+template <typename T, bool FUSED>
 cudaError_t dispatch_dim(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.head_dim) {
-    case 64: return dispatch_block<T, 64>(a, stream);
-    case 128: return dispatch_block<T, 128>(a, stream);
+    case 64: return dispatch_block<T, 64, FUSED>(a, stream);
+    case 128: return dispatch_block<T, 128, FUSED>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D>
+template <int D, bool FUSED>
 const void* kernel_for(int block_size, bool bf16) {
   switch (block_size) {
-    case 4: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 4>() : decode_kernel_ptr<__half, D, 4>();
-    case 8: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 8>() : decode_kernel_ptr<__half, D, 8>();
-    case 16: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 16>() : decode_kernel_ptr<__half, D, 16>();
-    case 32: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 32>() : decode_kernel_ptr<__half, D, 32>();
+    case 4: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 4, FUSED>() : decode_kernel_ptr<__half, D, 4, FUSED>();
+    case 8: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 8, FUSED>() : decode_kernel_ptr<__half, D, 8, FUSED>();
+    case 16: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 16, FUSED>() : decode_kernel_ptr<__half, D, 16, FUSED>();
+    case 32: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 32, FUSED>() : decode_kernel_ptr<__half, D, 32, FUSED>();
     default: return nullptr;
   }
 }
@@ -895,9 +954,11 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int blo
   if (!decode_sizes_supported(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq))
     return 0;
   int64_t warps = 0;
-  for (int bf16 = 0; bf16 < 2; ++bf16) {
-    const void* k = head_dim == 128 ? kernel_for<128>(block_size, bf16)
-                                    : kernel_for<64>(block_size, bf16);
+  for (int variant = 0; variant < 4; ++variant) {
+    const bool bf16 = variant & 1, fused = variant & 2;
+    const void* k = head_dim == 128
+                        ? (fused ? kernel_for<128, true>(block_size, bf16) : kernel_for<128, false>(block_size, bf16))
+                        : (fused ? kernel_for<64, true>(block_size, bf16) : kernel_for<64, false>(block_size, bf16));
     const Plan pl = plan_decode(k, head_dim, block_size, num_seqs, num_heads,
                                 max_blocks_per_seq, forced_warps);
     if (pl.grid <= 0) return 0;
@@ -911,7 +972,11 @@ cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (!decode_sizes_supported(a.num_seqs, a.num_heads, a.head_dim, a.block_size,
                               a.max_blocks_per_seq))
     return cudaErrorInvalidValue;
-  return a.is_bf16 ? dispatch_dim<__nv_bfloat16>(a, stream) : dispatch_dim<__half>(a, stream);
+  if (a.slot_mapping)  // fused decode step
+    return a.is_bf16 ? dispatch_dim<__nv_bfloat16, true>(a, stream)
+                     : dispatch_dim<__half, true>(a, stream);
+  return a.is_bf16 ? dispatch_dim<__nv_bfloat16, false>(a, stream)
+                   : dispatch_dim<__half, false>(a, stream);
 }
 
 }  // namespace pa

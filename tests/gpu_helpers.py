@@ -113,5 +113,15 @@ def gpu_step(w, status=None, out=None):
     return out
 
 
+def gpu_step_fused(w, status=None, out=None):
+    """The same step through the one-launch entry point pa_decode_step."""
+    import paged_kv_cache_326_b200 as P
+    if out is None:
+        out = torch.empty_like(w.q)
+    P.pa_decode_step(out, w.q, w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, w.block_tables,
+                     w.context_lens, w.scale, status=status)
+    return out
+
+
 def new_status(device="cuda"):
     return torch.zeros(1, dtype=torch.int32, device=device)

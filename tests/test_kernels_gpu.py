@@ -9,7 +9,8 @@ import torch
 
 import oracle
 from paged_kv_cache_326_b200 import workloads as W
-from tests.gpu_helpers import compare, gpu_step, new_status, oracle_inputs, run_oracle
+from tests.gpu_helpers import (compare, gpu_step, gpu_step_fused, new_status, oracle_inputs,
+                               run_oracle)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,8 +31,8 @@ def _pairs_mask(pairs, S_sel, seqs, H, D):
     return m
 
 
-def parity(w, seqs=None, heads_per_seq=None, seed=0, check_pool=False):
-    """GPU decode step vs the oracle.  Returns the Closeness."""
+def parity(w, seqs=None, heads_per_seq=None, seed=0, check_pool=False, step=gpu_step):
+    """GPU decode step (two calls, or the fused one) vs the oracle."""
     S, H, D = w.q.shape
     seqs = np.arange(S) if seqs is None else np.asarray(seqs)
     pairs = None
@@ -44,7 +45,7 @@ def parity(w, seqs=None, heads_per_seq=None, seed=0, check_pool=False):
         kb = w.k_cache.view(torch.int16).cpu().numpy()
         vb = w.v_cache.view(torch.int16).cpu().numpy()
     st = new_status()
-    out = gpu_step(w, st)
+    out = step(w, st)
     torch.cuda.synchronize()
     assert st.item() == 0, st.item()
     if check_pool:
@@ -299,3 +300,54 @@ def test_bounded_wait_gives_up_with_status_and_context_survives():
         P.pa_set_option(P.binding.PA_OPT_WAIT_LIMIT_NS, 1_000_000_000)
     assert st.item() == P.binding.PA_ERR_TIMEOUT
     parity(W.tiny(device="cuda"))
+
+
+# ---------------------------------------------------------------------------
+# the one-launch step (pa_decode_step)
+# ---------------------------------------------------------------------------
+
+def test_fused_step_tiny():
+    parity(W.tiny(device="cuda"), check_pool=True, step=gpu_step_fused)
+
+
+def test_fused_step_opt13b_batch64():
+    c = parity(W.opt13b_batch64(device="cuda"), check_pool=True, step=gpu_step_fused)
+    print("fused opt13b_batch64", c)
+
+
+def test_fused_step_skewed_bf16():
+    c = parity(W.skewed(block_size=16, device="cuda"), heads_per_seq=4, seed=7,
+               step=gpu_step_fused)
+    print("fused skewed", c)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("head_dim", [64, 128])
+@pytest.mark.parametrize("block_size", [4, 8, 16, 32])
+def test_fused_step_every_shape_ragged(dtype, head_dim, block_size):
+    w = W.make_decode("shape", SHAPE_LENS, num_heads=3, head_dim=head_dim, block_size=block_size,
+                      num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in SHAPE_LENS),
+                      dtype=dtype, seed=head_dim + block_size, device="cuda",
+                      max_blocks_per_seq=160 // block_size)
+    parity(w, check_pool=True, step=gpu_step_fused)
+
+
+def test_fused_step_equals_two_calls_bitwise():
+    """Same inputs, same split: the one-launch step and write-then-decode give
+    the same output and the same pool, bit for bit."""
+    a = W.opt13b_batch64(device="cuda")
+    b = W.opt13b_batch64(device="cuda")
+    out_a = gpu_step(a)
+    out_b = gpu_step_fused(b)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, out_b)
+    assert torch.equal(a.k_cache.view(torch.int16), b.k_cache.view(torch.int16))
+    assert torch.equal(a.v_cache.view(torch.int16), b.v_cache.view(torch.int16))
+
+
+def test_fused_step_single_token_returns_its_value():
+    w = W.make_decode("one", [1] * 7, num_heads=5, head_dim=128, block_size=16, num_blocks=16,
+                      dtype=torch.float16, seed=3, device="cuda")
+    out = gpu_step_fused(w)
+    torch.cuda.synchronize()
+    assert torch.equal(out, w.v)
