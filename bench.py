@@ -58,13 +58,14 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
 
 
-def traffic_per_launch():
-    """DRAM bytes per decode call from the committed ncu summary, if it was
-    taken on the kernel as it is now; else None."""
+def traffic_per_launch(path: str):
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    capture, if it was taken on this path and on the kernel as it is now;
+    else None."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
-        if t.get("kernel_source_hash") == kernel_source_hash():
+        if t.get("kernel_source_hash") == kernel_source_hash() and t.get("path") == path:
             return float(t["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -382,7 +383,7 @@ def main():
         "kernel_ms": ({"pa_decode_step": decode_ms} if fused else
                       {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic_per_launch(),
+                     "frac": achieved / peak, "traffic": traffic_per_launch(args.path),
                      "kernel": ("pa_decode_step (decode kernel with the cache write, + merge kernel)"
                                 if fused else "pa_paged_attn_decode (decode kernel + merge kernel)"),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": decode_bytes},

@@ -1,6 +1,7 @@
 """Run decode steps (write + paged attention) of one workload R times.
 
     python -m paged_kv_cache_326_b200.run_case [--workload NAME] [--num-seqs S] [--reps R]
+                                               [--path fused|calls]
 
 For profilers: it makes no timing claims.  Workloads: ``opt13b_batch64``
 (optionally cut to the first S texts, pool sized 1.5x what they need),
@@ -37,15 +38,20 @@ def main():
     ap.add_argument("--workload", default="opt13b_batch64")
     ap.add_argument("--num-seqs", type=int, default=0)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--path", choices=["fused", "calls"], default="fused")
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
     w = make(args.workload, args.num_seqs, dev)
     out = torch.empty_like(w.q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     for _ in range(args.reps):
-        P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
-        P.pa_paged_attn_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
-                               w.scale, status=status)
+        if args.path == "fused":
+            P.pa_decode_step(out, w.q, w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping,
+                             w.block_tables, w.context_lens, w.scale, status=status)
+        else:
+            P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+            P.pa_paged_attn_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                   w.context_lens, w.scale, status=status)
     torch.cuda.synchronize()
     if status.item() != 0:
         raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
