@@ -139,21 +139,6 @@ def kv_bytes(context_lens, num_heads, head_dim, elem_bytes) -> int:
     return decode_kv_bytes(context_lens, num_heads, head_dim, elem_bytes)
 
 
-def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        backend = "gloo" if args.impl == "reference" else "nccl"
-        if backend == "nccl":
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
-    return world, rank, local
-
-
 def oracle_runner(w, num_pairs):
     """The oracle over the first ``num_pairs`` (text, head) pairs of the
     workload, in text-major order.  Inputs are prepared outside the timed
@@ -240,12 +225,12 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
-    world, rank, local = dist_setup(args)
+    from paged_kv_cache_326_b200 import dist
+    ranks = dist.init("gloo" if args.impl == "reference" else "nccl")
+    world, rank, local = ranks.world, ranks.rank, ranks.local
     if args.impl == "reference":
         rc = run_reference(args, world, rank)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        dist.finish(ranks)
         return rc
 
     import paged_kv_cache_326_b200 as P
@@ -255,7 +240,7 @@ def main():
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
 
-    w = W.opt13b_batch64(seed=2 + rank, device=dev)
+    w = W.opt13b_batch64(seed=dist.batch_seed(2, ranks), device=dev)
     S, H, D = w.q.shape
     eb = w.q.element_size()
     lens = w.context_lens.tolist()
@@ -286,9 +271,7 @@ def main():
         decode_part(w.q, w.k, w.v, w.slot_mapping, w.block_tables, w.context_lens)
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+        dist.barrier(ranks)
 
     for _ in range(args.warmup):
         step()
@@ -358,11 +341,7 @@ def main():
         raise RuntimeError(f"device status {status.item()}: {P.pa_status_string(status.item())}")
 
     ms_step = total_ms / K
-    times = torch.tensor([ms_step, e2e_ms, decode_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    ms_step, e2e_ms, decode_ms = times.tolist()
+    ms_step, e2e_ms, decode_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms, decode_ms], dev)
 
     peak, peak_src = hbm_peak()
     achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
@@ -397,9 +376,7 @@ def main():
         line["cpu_baseline"] = cpu_baseline(w_cpu)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    dist.finish(ranks)
     return 0
 
 
