@@ -38,7 +38,9 @@ contiguous tensors, scalar brute force with ``math.fsum`` on tiny inputs,
 closed forms (one token gives its value; equal scores give the mean of the
 values; one dominant score gives its value), bit-identity under a relabelling
 of physical blocks, under a change of block size, and for texts that share
-prefix blocks, and a hand-worked cache write.
+prefix blocks, and a hand-worked cache write; grouped-query attention against
+the same pool with key/value heads replicated per query head, torch's fp64
+attention on repeated heads, and brute force for one shared head.
 """
 from __future__ import annotations
 
@@ -102,22 +104,36 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> np.ndar
     return out
 
 
+def kv_head_of(num_heads: int, num_kv_heads: int) -> np.ndarray:
+    """Query head h reads key/value head h // (num_heads / num_kv_heads):
+    consecutive query heads share one set of keys and values ("The KV Cache
+    and PagedAttention", §What Came After; num_kv_heads == num_heads is plain
+    multi-head attention, num_kv_heads == 1 one set for all heads)."""
+    if num_kv_heads <= 0 or num_heads % num_kv_heads:
+        raise ValueError("num_heads must be a multiple of num_kv_heads")
+    return np.arange(num_heads) // (num_heads // num_kv_heads)
+
+
 def paged_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
                  block_tables: np.ndarray, context_lens: Sequence[int], scale: float,
                  block_size: int,
                  pairs: Optional[Iterable[Tuple[int, int]]] = None) -> np.ndarray:
     """Decode attention over paged caches, fp64 ``[S][H][D]``.
 
+    The caches may hold fewer heads than q (grouped-query attention): query
+    head h then reads key/value head ``kv_head_of(H, H_kv)[h]``.
+
     With ``pairs`` (a list of (seq, head)), only those outputs are computed
     (the rest stay zero); this is how large workloads are checked one output
     at a time."""
     S, H, D = q.shape
+    kvh = kv_head_of(H, k_cache.shape[1])
     out = np.zeros((S, H, D), dtype=np.float64)
     if pairs is None:
         for s in range(S):
             K = gather_context(k_cache, block_tables[s], context_lens[s], block_size)
             V = gather_context(v_cache, block_tables[s], context_lens[s], block_size)
-            out[s] = attend(q[s], K, V, scale)
+            out[s] = attend(q[s], K[:, kvh, :], V[:, kvh, :], scale)
         return out
     by_seq = {}
     for s, h in pairs:
@@ -125,7 +141,8 @@ def paged_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
     for s, heads in by_seq.items():
         K = gather_context(k_cache, block_tables[s], context_lens[s], block_size)
         V = gather_context(v_cache, block_tables[s], context_lens[s], block_size)
-        full = attend(q[s][heads], K[:, heads, :], V[:, heads, :], scale)
+        sel = kvh[heads]
+        full = attend(q[s][heads], K[:, sel, :], V[:, sel, :], scale)
         for i, h in enumerate(heads):
             out[s, h] = full[i]
     return out

@@ -290,3 +290,54 @@ def pin_cache_write_then_read(write_fn):
 
 
 WRITE_PINS = [pin_cache_write_golden, pin_cache_write_then_read]
+
+
+# ---------------------------------------------------------------------------
+# grouped-query attention (several query heads share one key/value head)
+# ---------------------------------------------------------------------------
+
+def pin_gqa_equals_replicated_mha(fn):
+    """Sharing a key/value head between G query heads is the same as giving
+    each query head its own copy: a pool with the heads repeated (np.repeat,
+    built independently) gives the same output bit for bit."""
+    Hq, Hkv, D, B = 8, 2, 16, 4
+    lens = [5, 9, 16, 1]
+    q, _, _ = random_texts(lens, Hq, D, 201)
+    _, K, V = random_texts(lens, Hkv, D, 202)
+    kc, vc, tables = scatter_to_pool(K, V, B, 24, 203)
+    got = fn(f64(q), f64(kc), f64(vc), tables, lens, 0.25, B)
+    rep = np.repeat
+    ref = fn(f64(q), rep(f64(kc), Hq // Hkv, axis=1), rep(f64(vc), Hq // Hkv, axis=1), tables,
+             lens, 0.25, B)
+    assert np.array_equal(got, ref), "GQA differs from replicated MHA"
+
+
+def pin_gqa_unpaged_sdpa(fn):
+    """GQA against torch's fp64 attention on unpaged texts whose key/value
+    heads are repeated for each query head."""
+    Hq, Hkv, D, B = 6, 3, 16, 8
+    lens = [7, 23, 2]
+    q, _, _ = random_texts(lens, Hq, D, 211)
+    _, K, V = random_texts(lens, Hkv, D, 212)
+    kc, vc, tables = scatter_to_pool(K, V, B, 12, 213)
+    got = fn(f64(q), f64(kc), f64(vc), tables, lens, 0.3, B)
+    Kr = [k.repeat_interleave(Hq // Hkv, dim=1) for k in K]
+    Vr = [v.repeat_interleave(Hq // Hkv, dim=1) for v in V]
+    ref = sdpa_contiguous(q, Kr, Vr, 0.3)
+    assert np.abs(got - ref).max() <= 1e-12, "GQA vs sdpa"
+
+
+def pin_mqa_single_head(fn):
+    """One key/value head for all query heads (multi-query): head h's output
+    is attention of q_h over the one shared head."""
+    Hq, D, B = 4, 8, 4
+    lens = [6, 11]
+    q, _, _ = random_texts(lens, Hq, D, 221)
+    _, K, V = random_texts(lens, 1, D, 222)
+    kc, vc, tables = scatter_to_pool(K, V, B, 8, 223)
+    got = fn(f64(q), f64(kc), f64(vc), tables, lens, 0.5, B)
+    ref = brute_force(q, [k.expand(-1, Hq, -1) for k in K], [v.expand(-1, Hq, -1) for v in V], 0.5)
+    assert np.abs(got - ref).max() <= 1e-12, "MQA vs brute force"
+
+
+GQA_PINS = [pin_gqa_equals_replicated_mha, pin_gqa_unpaged_sdpa, pin_mqa_single_head]

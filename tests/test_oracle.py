@@ -52,3 +52,14 @@ def test_tiny_workload_runs_and_is_finite():
         w.slot_mapping.numpy(), w.block_tables.numpy(), w.context_lens.numpy(), w.scale,
         w.block_size)
     assert out.shape == (4, 8, 64) and np.isfinite(out).all()
+
+
+@pytest.mark.parametrize("pin", P.GQA_PINS, ids=lambda f: f.__name__)
+def test_gqa_pin(pin):
+    pin(oracle.paged_decode)
+
+
+def test_kv_head_of_rejects_uneven_groups():
+    with pytest.raises(ValueError):
+        oracle.kv_head_of(6, 4)
+    assert list(oracle.kv_head_of(8, 2)) == [0, 0, 0, 0, 1, 1, 1, 1]

@@ -143,3 +143,30 @@ def test_planted_write_mistake_is_caught(fn):
         except (AssertionError, IndexError):
             failed += 1
     assert failed, fn.__name__
+
+
+def decode_gqa_heads_by_modulo(q, k_cache, v_cache, block_tables, context_lens, scale, B):
+    """Planted mistake: query head h reads key/value head h % H_kv."""
+    S, H, D = q.shape
+    kvh = np.arange(H) % k_cache.shape[1]
+    out = np.zeros((S, H, D))
+    for s in range(S):
+        K = oracle.gather_context(k_cache, block_tables[s], context_lens[s], B)
+        V = oracle.gather_context(v_cache, block_tables[s], context_lens[s], B)
+        out[s] = oracle.attend(q[s], K[:, kvh, :], V[:, kvh, :], scale)
+    return out
+
+
+def test_planted_gqa_head_mapping_mistake_is_caught():
+    failed = []
+    for pin in P.GQA_PINS:
+        try:
+            pin(decode_gqa_heads_by_modulo)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed
+
+
+def test_unmodified_oracle_passes_gqa_pins():
+    for pin in P.GQA_PINS:
+        pin(oracle.paged_decode)
