@@ -222,6 +222,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
+    ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa"],
+                    default="opt13b_batch64",
+                    help="llama2_70b_gqa: 64 query heads on 8 key/value heads (two calls)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -240,18 +243,24 @@ def main():
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
 
-    w = W.opt13b_batch64(seed=dist.batch_seed(2, ranks), device=dev)
+    gqa = args.workload == "llama2_70b_gqa"
+    if gqa:
+        args.path = "calls"   # the one-launch step is multi-head only
+        w = W.llama2_70b_gqa(seed=dist.batch_seed(6, ranks), device=dev)
+    else:
+        w = W.opt13b_batch64(seed=dist.batch_seed(2, ranks), device=dev)
     S, H, D = w.q.shape
+    Hkv = w.k_cache.shape[1]
     eb = w.q.element_size()
     lens = w.context_lens.tolist()
-    step_kv = kv_bytes(lens, H, D, eb)
+    step_kv = kv_bytes(lens, Hkv, D, eb)
     decode_bytes = step_kv + 2 * S * H * D * eb + sum(4 * -(-L // w.block_size) for L in lens) + 4 * S
-    write_bytes = 4 * S * H * D * eb + 8 * S   # k, v read and stored; slots
+    write_bytes = 4 * S * Hkv * D * eb + 8 * S   # k, v read and stored; slots
     fused = args.path == "fused"
     if fused:
         decode_bytes += write_bytes
     out = torch.empty_like(w.q)
-    ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq)
+    ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq, Hkv)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def write_part(k, v, slots):
@@ -262,6 +271,9 @@ def main():
         if fused:
             P.pa_decode_step(out, q, k, v, w.k_cache, w.v_cache, slots, tables, lens, w.scale,
                              workspace=ws, status=status)
+        elif gqa:
+            P.pa_paged_attn_decode_gqa(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
+                                       workspace=ws, status=status)
         else:
             P.pa_paged_attn_decode(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
                                    workspace=ws, status=status)
@@ -351,8 +363,10 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "num_seqs": S, "num_heads": H, "head_dim": D,
-                   "block_size": w.block_size, "context_lens": "uniform [128, 2048], seed 2+rank",
+        "config": {"workload": args.workload, "num_seqs": S, "num_heads": H,
+                   "num_kv_heads": Hkv, "head_dim": D, "block_size": w.block_size,
+                   "context_lens": ("uniform [128, 4096], seed 6+rank" if gqa else
+                                    "uniform [128, 2048], seed 2+rank"),
                    "num_blocks": w.num_blocks, "kv_bytes_per_step": step_kv,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB)",
                    "parallelism": f"independent batch per GPU x{world}",
@@ -362,16 +376,19 @@ def main():
         "kernel_ms": ({"pa_decode_step": decode_ms} if fused else
                       {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic_per_launch(args.path),
+                     "frac": achieved / peak,
+                     "traffic": None if gqa else traffic_per_launch(args.path),
                      "kernel": ("pa_decode_step (decode kernel with the cache write, + merge kernel)"
-                                if fused else "pa_paged_attn_decode (decode kernel + merge kernel)"),
+                                if fused else
+                                "pa_paged_attn_decode_gqa (decode kernel + merge kernel)" if gqa
+                                else "pa_paged_attn_decode (decode kernel + merge kernel)"),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": decode_bytes},
         "e2e": {"value": world * step_kv / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": (2 if fused else 3) * K,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not gqa:
         w_cpu = w
         line["cpu_baseline"] = cpu_baseline(w_cpu)
     if rank == 0:

@@ -64,6 +64,9 @@ _SIGNATURES = {
     "pa_paged_attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "pa_paged_attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _i32,
                                     _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
+    "pa_paged_attn_decode_gqa_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
+    "pa_paged_attn_decode_gqa": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _i32,
+                                        _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
                               _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_paged_attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
@@ -171,11 +174,23 @@ def pa_paged_attn_decode_workspace_size(num_seqs: int, num_heads: int, head_dim:
 _ws_cache: Dict[Tuple[int, int], torch.Tensor] = {}
 
 
-def workspace_for(q: torch.Tensor, block_size: int, max_blocks_per_seq: int) -> torch.Tensor:
+def pa_paged_attn_decode_gqa_workspace_size(num_seqs: int, num_heads: int, num_kv_heads: int,
+                                            head_dim: int, block_size: int,
+                                            max_blocks_per_seq: int) -> int:
+    return int(lib().pa_paged_attn_decode_gqa_workspace_size(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq))
+
+
+def workspace_for(q: torch.Tensor, block_size: int, max_blocks_per_seq: int,
+                  num_kv_heads: Optional[int] = None) -> torch.Tensor:
     """A cached device workspace big enough for these sizes (allocated by
     torch, never by the library)."""
     S, H, D = q.shape
-    need = pa_paged_attn_decode_workspace_size(S, H, D, block_size, max_blocks_per_seq)
+    if num_kv_heads is None or num_kv_heads == H:
+        need = pa_paged_attn_decode_workspace_size(S, H, D, block_size, max_blocks_per_seq)
+    else:
+        need = pa_paged_attn_decode_gqa_workspace_size(S, H, num_kv_heads, D, block_size,
+                                                       max_blocks_per_seq)
     if need == 0:
         raise PagedAttnError(PA_ERR_INVALID, "pa_paged_attn_decode_workspace_size")
     key = (q.device.index if q.device.index is not None else torch.cuda.current_device(), need)
@@ -212,6 +227,35 @@ def pa_paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tens
         _dtype_code(q), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _status_ptr(status), _stream(stream, q.device))
     _check(code, "pa_paged_attn_decode")
+    return out
+
+
+def pa_paged_attn_decode_gqa(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                             v_cache: torch.Tensor, block_tables: torch.Tensor,
+                             context_lens: torch.Tensor, scale: float,
+                             workspace: Optional[torch.Tensor] = None,
+                             status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Grouped-query decode: out, q [S][H][D]; caches [N][H_kv][B][D] with H a
+    multiple of H_kv (query head h reads key/value head h // (H / H_kv))."""
+    S, H, D = q.shape
+    N, Hkv, B, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D or H % Hkv:
+        raise ValueError("shape mismatch (num_heads must be a multiple of num_kv_heads)")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S][max_blocks], context_lens [S]")
+    for t in (out, k_cache, v_cache):
+        if t.dtype != q.dtype:
+            raise TypeError("q, out and the caches must share a dtype")
+    MB = block_tables.shape[1]
+    if workspace is None:
+        workspace = workspace_for(q, B, MB, Hkv)
+    code = lib().pa_paged_attn_decode_gqa(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(context_lens, "context_lens", torch.int32), float(scale), S, H, Hkv, D, B, MB, N,
+        _dtype_code(q), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _status_ptr(status), _stream(stream, q.device))
+    _check(code, "pa_paged_attn_decode_gqa")
     return out
 
 

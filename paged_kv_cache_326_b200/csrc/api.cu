@@ -83,18 +83,30 @@ int pa_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache
 
 size_t pa_paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
                                            int block_size, int max_blocks_per_seq) {
-  return pa::decode_workspace_bytes(num_seqs, num_heads, head_dim, block_size,
+  return pa::decode_workspace_bytes(num_seqs, num_heads, num_heads, head_dim, block_size,
                                     max_blocks_per_seq, g_decode_warps.load());
 }
 
-int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                         const int32_t* block_tables, const int32_t* context_lens, float scale,
-                         int num_seqs, int num_heads, int head_dim, int block_size,
-                         int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt,
-                         void* workspace, size_t workspace_bytes, int32_t* d_status,
-                         pa_stream_t stream) {
+size_t pa_paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                               int head_dim, int block_size,
+                                               int max_blocks_per_seq) {
+  return pa::decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                    max_blocks_per_seq, g_decode_warps.load());
+}
+
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the decode entry points, then the launch.
+int decode_common(void* out, const void* q, const void* k_cache, const void* v_cache,
+                  const int32_t* block_tables, const int32_t* context_lens, float scale,
+                  int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                  int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt, void* workspace,
+                  size_t workspace_bytes, int32_t* d_status, pa_stream_t stream,
+                  const void* k_new, const void* v_new, const int64_t* slot_mapping) {
   if (num_seqs == 0) return PA_OK;
-  if (!pa::decode_sizes_supported(num_seqs, num_heads, head_dim, block_size,
+  if (!pa::decode_sizes_supported(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                   max_blocks_per_seq) ||
       num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16))
     return PA_ERR_INVALID;
@@ -103,6 +115,8 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return PA_ERR_INVALID;
+  if (slot_mapping && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
+    return PA_ERR_INVALID;
   pa::DecodeArgs a;
   a.out = out;
   a.q = q;
@@ -113,6 +127,7 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
   a.scale = scale;
   a.num_seqs = num_seqs;
   a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
   a.head_dim = head_dim;
   a.block_size = block_size;
   a.max_blocks_per_seq = max_blocks_per_seq;
@@ -123,7 +138,37 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
   a.status = d_status;
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.forced_warps = g_decode_warps.load();
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.slot_mapping = slot_mapping;
   return from_cuda(pa::launch_paged_attn_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, float scale,
+                         int num_seqs, int num_heads, int head_dim, int block_size,
+                         int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt,
+                         void* workspace, size_t workspace_bytes, int32_t* d_status,
+                         pa_stream_t stream) {
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       dt, workspace, workspace_bytes, d_status, stream, nullptr, nullptr, nullptr);
+}
+
+int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             float scale, int num_seqs, int num_heads, int num_kv_heads,
+                             int head_dim, int block_size, int max_blocks_per_seq,
+                             int64_t num_blocks, pa_dtype dt, void* workspace,
+                             size_t workspace_bytes, int32_t* d_status, pa_stream_t stream) {
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                       num_blocks, dt, workspace, workspace_bytes, d_status, stream, nullptr,
+                       nullptr, nullptr);
 }
 
 int pa_decode_step(void* out, const void* q, const void* k, const void* v, void* k_cache,
@@ -132,41 +177,10 @@ int pa_decode_step(void* out, const void* q, const void* k, const void* v, void*
                    int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
                    pa_dtype dt, void* workspace, size_t workspace_bytes, int32_t* d_status,
                    pa_stream_t stream) {
-  if (num_seqs == 0) return PA_OK;
-  if (!pa::decode_sizes_supported(num_seqs, num_heads, head_dim, block_size,
-                                  max_blocks_per_seq) ||
-      num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16))
-    return PA_ERR_INVALID;
-  if (!out || !q || !k || !v || !k_cache || !v_cache || !slot_mapping || !block_tables ||
-      !context_lens || !workspace)
-    return PA_ERR_INVALID;
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
-      !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return PA_ERR_INVALID;
-  pa::DecodeArgs a;
-  a.out = out;
-  a.q = q;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.block_tables = block_tables;
-  a.context_lens = context_lens;
-  a.scale = scale;
-  a.num_seqs = num_seqs;
-  a.num_heads = num_heads;
-  a.head_dim = head_dim;
-  a.block_size = block_size;
-  a.max_blocks_per_seq = max_blocks_per_seq;
-  a.num_blocks = num_blocks;
-  a.is_bf16 = dt == PA_BF16;
-  a.workspace = workspace;
-  a.workspace_bytes = workspace_bytes;
-  a.status = d_status;
-  a.wait_limit_ns = g_wait_limit_ns.load();
-  a.forced_warps = g_decode_warps.load();
-  a.k_new = k;
-  a.v_new = v;
-  a.slot_mapping = slot_mapping;
-  return from_cuda(pa::launch_paged_attn_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+  if (num_seqs != 0 && !slot_mapping) return PA_ERR_INVALID;
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       dt, workspace, workspace_bytes, d_status, stream, k, v, slot_mapping);
 }
 
 }  // extern "C"

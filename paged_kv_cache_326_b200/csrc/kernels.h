@@ -21,7 +21,8 @@ struct DecodeArgs {
   const int32_t* context_lens;
   float scale;
   int num_seqs;
-  int num_heads;
+  int num_heads;     // query heads
+  int num_kv_heads;  // key/value heads of the pool (== num_heads: multi-head)
   int head_dim;
   int block_size;
   int max_blocks_per_seq;
@@ -38,13 +39,13 @@ struct DecodeArgs {
   const int64_t* slot_mapping = nullptr;
 };
 
-bool decode_sizes_supported(int num_seqs, int num_heads, int head_dim, int block_size,
-                            int max_blocks_per_seq);
+bool decode_sizes_supported(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                            int block_size, int max_blocks_per_seq);
 
 // Size of the decode workspace for these sizes on the current device, or 0
 // if the sizes are unsupported.
-size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int block_size,
-                              int max_blocks_per_seq, int64_t forced_warps);
+size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_blocks_per_seq, int64_t forced_warps);
 
 // Current PA_OPT_DECODE_WARPS setting.
 int64_t option_decode_warps();

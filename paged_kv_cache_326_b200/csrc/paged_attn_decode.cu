@@ -87,15 +87,18 @@ constexpr int kGrainsPerWarp = 12;
 constexpr int kMinGrain = PA_MIN_GRAIN;
 constexpr int kDrainLimitNs = 1000000000;
 __host__ __device__ constexpr int chunk_tokens(int D) { return 2048 / D; }
-__host__ __device__ constexpr int stage_bytes(int D) { return 2 * 4096 + 2 * D + 128; }
-__host__ __device__ constexpr int warp_area_bytes(int D, int stages) { return stages * stage_bytes(D) + 128; }
+// One stage: K rows (4 KB), V rows (4 KB), the unit's GS query rows, a flag.
+__host__ __device__ constexpr int stage_bytes(int D, int gs) { return 2 * 4096 + gs * 2 * D + 128; }
+__host__ __device__ constexpr int warp_area_bytes(int D, int stages, int gs) {
+  return stages * stage_bytes(D, gs) + 128;
+}
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace: a header (the work split, then prefix[S+1]), the grain counter,
 // then the partial records.  The header is written by CTA 0 of the decode
 // kernel and read by the merge kernel.
-constexpr int kHeaderInts = 8;  // total, q, G, W, 4 spare
+constexpr int kHeaderInts = 8;  // total, q, grain, W, 4 spare
 size_t header_bytes(int num_seqs) {
   return align_up(sizeof(int32_t) * (kHeaderInts + num_seqs + 1), 256);
 }
@@ -115,7 +118,10 @@ struct DecodeParams {
   const int32_t* context_lens;
   float qk_scale_log2;
   int num_seqs;
-  int num_heads;
+  int num_heads;      // virtual heads: key/value heads x subsets (the flat order's heads)
+  int num_q_heads;    // query heads of q and out
+  int num_kv_heads;   // key/value heads of the pool
+  int nsub;           // subsets per key/value head (GS query heads each)
   int max_blocks_per_seq;
   int64_t num_blocks;
   int num_work_warps;
@@ -146,13 +152,14 @@ struct Lookahead {
 // rounding).  Partials are read in warp order, so the result does not depend
 // on which warp merges.  Reads go through L2 (other SMs wrote them).
 template <typename T, int D>
-__device__ __forceinline__ void merge_partials(const float* records, T* out, int64_t sh, int w_lo,
-                                               int w_hi, int lane) {
+__device__ __forceinline__ void merge_partials(const float* records, int64_t rec_stride,
+                                               T* out_row, int64_t sh, int w_lo, int w_hi,
+                                               int lane) {
   constexpr int PER = D / 32;
   const int n = w_hi - w_lo + 1;
   // running max over the partials, one partial per lane
   float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(records + (w_lo + i + sh) * (D + 4)));
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(records + (w_lo + i + sh) * rec_stride));
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float L = 0.f;
@@ -163,7 +170,7 @@ __device__ __forceinline__ void merge_partials(const float* records, T* out, int
     // weight f_i = 2^(m_i - M) of partial i0 + lane, and its share of the sum
     float f = 0.f, lf = 0.f;
     if (i0 + lane < n) {
-      const float* rec = records + (w_lo + i0 + lane + sh) * (D + 4);
+      const float* rec = records + (w_lo + i0 + lane + sh) * rec_stride;
       f = M == -INFINITY ? 0.f : fast_exp2(__ldcg(rec) - M);
       lf = f * __ldcg(rec + 1);
     }
@@ -176,7 +183,7 @@ __device__ __forceinline__ void merge_partials(const float* records, T* out, int
       float o[8][PER];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const float* rec = records + (w_lo + i0 + min(b + u, cnt - 1) + sh) * (D + 4) + 4 + lane * PER;
+        const float* rec = records + (w_lo + i0 + min(b + u, cnt - 1) + sh) * rec_stride + 4 + lane * PER;
         if constexpr (PER == 4) {
           const float4 v = __ldcg(reinterpret_cast<const float4*>(rec));
           o[u][0] = v.x; o[u][1] = v.y; o[u][2] = v.z; o[u][3] = v.w;
@@ -196,7 +203,7 @@ __device__ __forceinline__ void merge_partials(const float* records, T* out, int
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-  T* o = out + sh * D + lane * PER;
+  T* o = out_row + lane * PER;
   if constexpr (PER == 4) {
     uint2 v;
     v.x = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
@@ -212,7 +219,10 @@ __device__ __forceinline__ void merge_partials(const float* records, T* out, int
 // FUSED: also store each text's new key/value at its slot, and take the
 // text's last position (the new token) from the inputs instead of the pool,
 // so nothing in this launch waits on its own write.
-template <typename T, int D, int B, int WARPS, int STAGES, bool FUSED>
+// GS: query heads per work unit (1 = multi-head attention).  With grouped-
+// query attention the GS query heads of a unit share one key/value head, so
+// every K/V row copied is used GS times from registers.
+template <typename T, int D, int B, int WARPS, int STAGES, bool FUSED, int GS>
 __global__ void __launch_bounds__(WARPS * 32, 2)
 paged_decode_kernel(const DecodeParams p) {
   constexpr int CH = chunk_tokens(D);        // tokens per chunk
@@ -221,8 +231,8 @@ paged_decode_kernel(const DecodeParams p) {
   constexpr int ITERS = CH / TPI;            // loads per chunk (8)
   constexpr int NB = CH >= B ? CH / B : 1;   // physical blocks a chunk touches
   constexpr int TILE = CH * D;               // elements of K (or V) per chunk
-  constexpr int STRIDE = stage_bytes(D);
-  constexpr int AREA = warp_area_bytes(D, STAGES);
+  constexpr int STRIDE = stage_bytes(D, GS);
+  constexpr int AREA = warp_area_bytes(D, STAGES, GS);
   static_assert(CH % TPI == 0 && (CH % B == 0 || B % CH == 0), "shape");
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -230,7 +240,12 @@ paged_decode_kernel(const DecodeParams p) {
   __shared__ int32_t warp_tot[WARPS];
 
   const int S = p.num_seqs;
-  const int H = p.num_heads;
+  const int H = p.num_heads;  // virtual heads in the flat order
+  const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, NSUB = p.nsub;
+  const int G = Hq / Hkv;       // query heads per key/value head
+  // virtual head -> its key/value head and its first query head
+  auto kv_head = [&](int vh) { return vh / NSUB; };
+  auto q_head0 = [&](int vh) { return (vh / NSUB) * G + (vh % NSUB) * GS; };
   const int cap = p.max_blocks_per_seq * B;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -274,18 +289,18 @@ paged_decode_kernel(const DecodeParams p) {
   }
   const int total = prefix[S];
   const int W = p.num_work_warps;
-  // Static runs of q chunks (units 0..W-1), then grains of G chunks (units
+  // Static runs of q chunks (units 0..W-1), then grains of `grain` chunks (units
   // W, W+1, ...) covering the rest of the flat order.
   int q = W == 1 ? total : static_cast<int>(static_cast<long long>(total) * kStaticPermille / 1000 / W);
   if (q < 32 && W > 1) q = 0;
   const int dyn_base = W * q;
   const int dyn = total - dyn_base;
-  const int G = max(kMinGrain, (dyn + kGrainsPerWarp * W - 1) / (kGrainsPerWarp * W));
+  const int grain = max(kMinGrain, (dyn + kGrainsPerWarp * W - 1) / (kGrainsPerWarp * W));
   if (blockIdx.x == 0) {
     if (tid == 0) {
       p.header[0] = total;
       p.header[1] = q;
-      p.header[2] = G;
+      p.header[2] = grain;
       p.header[3] = W;
     }
     for (int i = tid; i <= S; i += WARPS * 32) p.header[kHeaderInts + i] = prefix[i];
@@ -293,8 +308,8 @@ paged_decode_kernel(const DecodeParams p) {
   // Texts with no tokens get zeros (spread over the CTAs).
   for (int s = blockIdx.x; s < S; s += gridDim.x) {
     if (prefix[s + 1] == prefix[s]) {
-      uint4* o = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + static_cast<int64_t>(s) * H * D);
-      for (int i = tid; i < H * D / 8; i += WARPS * 32) o[i] = make_uint4(0u, 0u, 0u, 0u);
+      uint4* o = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + static_cast<int64_t>(s) * Hq * D);
+      for (int i = tid; i < Hq * D / 8; i += WARPS * 32) o[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 
@@ -306,7 +321,7 @@ paged_decode_kernel(const DecodeParams p) {
   auto fused_write = [&]() {
     if constexpr (FUSED) {
       const int vpr = D / 8;
-      const int64_t per_text = static_cast<int64_t>(H) * vpr;
+      const int64_t per_text = static_cast<int64_t>(Hkv) * vpr;
       const int64_t nvec = per_text * S;
       const int64_t num_slots = p.num_blocks * B;
       uint4* kcw = static_cast<uint4*>(const_cast<void*>(p.k_cache));
@@ -323,7 +338,7 @@ paged_decode_kernel(const DecodeParams p) {
         }
         const int64_t h = r / vpr, c = r - (r / vpr) * vpr;
         const int64_t blk = slot / B, place = slot - blk * B;
-        const int64_t dst = ((blk * H + h) * B + place) * vpr + c;
+        const int64_t dst = ((blk * Hkv + h) * B + place) * vpr + c;
         kcw[dst] = __ldg(static_cast<const uint4*>(p.k_new) + i);
         vcw[dst] = __ldg(static_cast<const uint4*>(p.v_new) + i);
       }
@@ -365,16 +380,16 @@ paged_decode_kernel(const DecodeParams p) {
   // workspace never needs clearing.
   auto grab_resolve = [&](unsigned long long old) -> int {
     if ((old >> 30) == e34) return static_cast<int>(old & kGrabMask);
-    unsigned long long seen = old + static_cast<unsigned long long>(G);
+    unsigned long long seen = old + static_cast<unsigned long long>(grain);
     while (true) {
       if ((seen >> 30) == e34) {
-        const unsigned long long o2 = atomicAdd(p.grab, static_cast<unsigned long long>(G));
+        const unsigned long long o2 = atomicAdd(p.grab, static_cast<unsigned long long>(grain));
         if ((o2 >> 30) == e34) return static_cast<int>(o2 & kGrabMask);
-        seen = o2 + static_cast<unsigned long long>(G);
+        seen = o2 + static_cast<unsigned long long>(grain);
         continue;
       }
       const unsigned long long prev =
-          atomicCAS(p.grab, seen, (e34 << 30) | static_cast<unsigned long long>(G));
+          atomicCAS(p.grab, seen, (e34 << 30) | static_cast<unsigned long long>(grain));
       if (prev == seen) return 0;
       seen = prev;
     }
@@ -383,7 +398,7 @@ paged_decode_kernel(const DecodeParams p) {
   unsigned long long pend = 0;  // lane 0: counter value of the next grain
   int u_start = 0, u_count = 0, u_id = -1, u_off = 0;
   auto grab_issue = [&]() {
-    if (lane == 0) pend = atomicAdd(p.grab, static_cast<unsigned long long>(G));
+    if (lane == 0) pend = atomicAdd(p.grab, static_cast<unsigned long long>(grain));
     pend_live = true;
   };
   auto next_unit = [&]() {
@@ -412,8 +427,8 @@ paged_decode_kernel(const DecodeParams p) {
       return;
     }
     u_start = dyn_base + off;
-    u_count = min(G, dyn - off);
-    u_id = W + off / G;
+    u_count = min(grain, dyn - off);
+    u_id = W + off / grain;
     u_off = 0;
     grab_issue();  // the next grain, resolved when this one runs out
   };
@@ -504,7 +519,7 @@ paged_decode_kernel(const DecodeParams p) {
       T* sK = reinterpret_cast<T*>(stage);
       T* sV = sK + TILE;
       T* sQ = sV + TILE;
-      int32_t* flag = reinterpret_cast<int32_t*>(stage + 2 * 4096 + 2 * D);
+      int32_t* flag = reinterpret_cast<int32_t*>(stage + 2 * 4096 + GS * 2 * D);
       const int len = min(max(len_raw, 0), cap);
       const int nvalid = min(CH, len - j * CH);
       const bool first = unit_start || j == 0;
@@ -518,11 +533,12 @@ paged_decode_kernel(const DecodeParams p) {
       if (bad) set_status(p.status, -7 /* PA_ERR_BAD_BLOCK */);
       fence_proxy_async_smem();
       *flag = bad ? 1 : 0;
-      const uint32_t qbytes = first ? D * 2 : 0;
+      const uint32_t qbytes = first ? GS * D * 2 : 0;
       const uint32_t kvbytes = bad ? 0 : 2u * nvalid * D * 2;
       mbar_arrive_expect_tx(&bars[st], qbytes + kvbytes);
       if (first)
-        bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * H + h) * D, D * 2, &bars[st], policy);
+        bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D, GS * D * 2, &bars[st],
+                      policy);
       if (!bad) {
         // Fused step: the chunk holding the text's last position takes that
         // row from the new k/v instead of the pool.
@@ -533,21 +549,21 @@ paged_decode_kernel(const DecodeParams p) {
           for (int k = 0; k < NB; ++k) {
             const int rows = min(B, pool_rows - k * B);
             if (rows > 0) {
-              const int64_t off = (static_cast<int64_t>(blk[k]) * H + h) * B * D;
+              const int64_t off = (static_cast<int64_t>(blk[k]) * Hkv + kv_head(h)) * B * D;
               bulk_copy_g2s(sK + k * B * D, kc + off, rows * D * 2, &bars[st], policy);
               bulk_copy_g2s(sV + k * B * D, vc + off, rows * D * 2, &bars[st], policy);
             }
           }
         } else {
           const int row0 = (j * CH) % B;
-          const int64_t off = ((static_cast<int64_t>(blk[0]) * H + h) * B + row0) * D;
+          const int64_t off = ((static_cast<int64_t>(blk[0]) * Hkv + kv_head(h)) * B + row0) * D;
           if (pool_rows > 0) {
             bulk_copy_g2s(sK, kc + off, pool_rows * D * 2, &bars[st], policy);
             bulk_copy_g2s(sV, vc + off, pool_rows * D * 2, &bars[st], policy);
           }
         }
         if (new_row) {
-          const int64_t src_off = (static_cast<int64_t>(s) * H + h) * D;
+          const int64_t src_off = (static_cast<int64_t>(s) * Hkv + kv_head(h)) * D;
           bulk_copy_g2s(sK + pool_rows * D, static_cast<const T*>(p.k_new) + src_off, D * 2,
                         &bars[st], policy);
           bulk_copy_g2s(sV + pool_rows * D, static_cast<const T*>(p.v_new) + src_off, D * 2,
@@ -563,9 +579,10 @@ paged_decode_kernel(const DecodeParams p) {
 
   const int dchunk = lane % LPT;
   const int tsub = lane / LPT;
-  float qf[8];
-  float acc[8];
-  float m = -INFINITY, lsum = 0.f;
+  // Per query head of this unit (GS of them share every K/V row read).
+  float qf[GS][8];
+  float acc[GS][8];
+  float m[GS], lsum[GS];
   int piece_j0 = 0;
   int prev_unit = -1;
 
@@ -588,118 +605,147 @@ paged_decode_kernel(const DecodeParams p) {
     const T* sK = reinterpret_cast<const T*>(stage);
     const T* sV = sK + TILE;
     const T* sQ = sV + TILE;
-    const int bad = *reinterpret_cast<const int32_t*>(stage + 2 * 4096 + 2 * D);
+    const int bad = *reinterpret_cast<const int32_t*>(stage + 2 * 4096 + GS * 2 * D);
 
     if (j == 0 || wu0 != prev_unit) {
       piece_j0 = j;
-      float qraw[8];
-      unpack8<T>(*reinterpret_cast<const uint4*>(sQ + dchunk * 8), qraw);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        qf[k] = qraw[k] * p.qk_scale_log2;
-        acc[k] = 0.f;
+      for (int g = 0; g < GS; ++g) {
+        float qraw[8];
+        unpack8<T>(*reinterpret_cast<const uint4*>(sQ + g * D + dchunk * 8), qraw);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          qf[g][k] = qraw[k] * p.qk_scale_log2;
+          acc[g][k] = 0.f;
+        }
+        m[g] = -INFINITY;
+        lsum[g] = 0.f;
       }
-      m = -INFINITY;
-      lsum = 0.f;
     }
     const int nvalid = bad ? 0 : min(CH, len - j * CH);
 
-    // scores (base-2 logits) of this lane's token rows
-    float sc[ITERS];
+    // scores (base-2 logits) of this lane's token rows, for every head
+    float sc[GS][ITERS];
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       float kf[8];
       unpack8<T>(*reinterpret_cast<const uint4*>(sK + (it * TPI + tsub) * D + dchunk * 8), kf);
-      float d0 = qf[0] * kf[0];
 #pragma unroll
-      for (int k = 1; k < 8; ++k) d0 = fmaf(qf[k], kf[k], d0);
-      sc[it] = d0;
+      for (int g = 0; g < GS; ++g) {
+        float d0 = qf[g][0] * kf[0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) d0 = fmaf(qf[g][k], kf[k], d0);
+        sc[g][it] = d0;
+      }
     }
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
+    for (int g = 0; g < GS; ++g)
 #pragma unroll
-      for (int off = LPT / 2; off >= 1; off >>= 1) sc[it] += __shfl_xor_sync(0xffffffffu, sc[it], off);
-    }
+      for (int it = 0; it < ITERS; ++it) {
+#pragma unroll
+        for (int off = LPT / 2; off >= 1; off >>= 1)
+          sc[g][it] += __shfl_xor_sync(0xffffffffu, sc[g][it], off);
+      }
     if (nvalid < CH) {
 #pragma unroll
       for (int it = 0; it < ITERS; ++it)
-        if (it * TPI + tsub >= nvalid) sc[it] = -INFINITY;
+        if (it * TPI + tsub >= nvalid) {
+#pragma unroll
+          for (int g = 0; g < GS; ++g) sc[g][it] = -INFINITY;
+        }
     }
-    float cm = sc[0];
 #pragma unroll
-    for (int it = 1; it < ITERS; ++it) cm = fmaxf(cm, sc[it]);
+    for (int g = 0; g < GS; ++g) {
+      float cm = sc[g][0];
 #pragma unroll
-    for (int off = LPT; off < 32; off <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
-    const float m_new = fmaxf(m, cm);
-    if (m_new != -INFINITY) {
-      const float alpha = fast_exp2(m - m_new);
-      float psum = 0.f;
+      for (int it = 1; it < ITERS; ++it) cm = fmaxf(cm, sc[g][it]);
 #pragma unroll
-      for (int it = 0; it < ITERS; ++it) {
-        sc[it] = fast_exp2(sc[it] - m_new);
-        psum += sc[it];
-      }
-      lsum = fmaf(lsum, alpha, psum);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] *= alpha;
-      m = m_new;
-      if (nvalid == CH) {
+      for (int off = LPT; off < 32; off <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+      const float m_new = fmaxf(m[g], cm);
+      if (m_new != -INFINITY) {
+        const float alpha = fast_exp2(m[g] - m_new);
+        float psum = 0.f;
 #pragma unroll
         for (int it = 0; it < ITERS; ++it) {
+          sc[g][it] = fast_exp2(sc[g][it] - m_new);
+          psum += sc[g][it];
+        }
+        lsum[g] = fmaf(lsum[g], alpha, psum);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[g][k] *= alpha;
+        m[g] = m_new;
+      } else {
+#pragma unroll
+        for (int it = 0; it < ITERS; ++it) sc[g][it] = 0.f;
+      }
+    }
+    if (nvalid == CH) {
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) {
+        float vf[8];
+        unpack8<T>(*reinterpret_cast<const uint4*>(sV + (it * TPI + tsub) * D + dchunk * 8), vf);
+#pragma unroll
+        for (int g = 0; g < GS; ++g)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
+      }
+    } else {
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) {
+        if (it * TPI + tsub < nvalid) {
           float vf[8];
           unpack8<T>(*reinterpret_cast<const uint4*>(sV + (it * TPI + tsub) * D + dchunk * 8), vf);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[k] = fmaf(sc[it], vf[k], acc[k]);
-        }
-      } else {
+          for (int g = 0; g < GS; ++g)
 #pragma unroll
-        for (int it = 0; it < ITERS; ++it) {
-          if (it * TPI + tsub < nvalid) {
-            float vf[8];
-            unpack8<T>(*reinterpret_cast<const uint4*>(sV + (it * TPI + tsub) * D + dchunk * 8), vf);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = fmaf(sc[it], vf[k], acc[k]);
-          }
+            for (int k = 0; k < 8; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
         }
       }
     }
 
     // This stage is consumed: refill it before the epilogue, whose global
-    // stores and (rarely) merge must not leave the copy engine idle.
+    // stores must not leave the copy engine idle.
     __syncwarp();
     issue(i0 + STAGES);
 
     const int ns = (len + CH - 1) / CH;
     const bool unit_ends = i0 + 1 == wc0 && (wc1 == 0 || wu1 != wu0);
     if (unit_ends || j == ns - 1) {
-      float l_all = lsum;
-      float o[8];
+      const int64_t sh = static_cast<int64_t>(s) * H + h;          // (text, virtual head)
+      const int64_t qrow = static_cast<int64_t>(s) * Hq + q_head0(h);  // first query head
+      const bool whole = piece_j0 == 0 && j == ns - 1;
+      float* recs = p.records + (static_cast<int64_t>(wu0) + sh) * (GS * (D + 4));
 #pragma unroll
-      for (int k = 0; k < 8; ++k) o[k] = acc[k];
+      for (int g = 0; g < GS; ++g) {
+        float l_all = lsum[g];
+        float o[8];
 #pragma unroll
-      for (int off = LPT; off < 32; off <<= 1) {
-        l_all += __shfl_xor_sync(0xffffffffu, l_all, off);
+        for (int k = 0; k < 8; ++k) o[k] = acc[g][k];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
-      }
-      const int64_t sh = static_cast<int64_t>(s) * H + h;
-      if (piece_j0 == 0 && j == ns - 1) {
-        if (tsub == 0) {
-          const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+        for (int off = LPT; off < 32; off <<= 1) {
+          l_all += __shfl_xor_sync(0xffffffffu, l_all, off);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) o[k] *= inv;
-          *reinterpret_cast<uint4*>(static_cast<T*>(p.out) + sh * D + dchunk * 8) = pack8<T>(o);
+          for (int k = 0; k < 8; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
         }
-      } else {
-        float* rec = p.records + (static_cast<int64_t>(wu0) + sh) * (D + 4);
-        if (lane == 0) {
-          rec[0] = m;
-          rec[1] = l_all;
-        }
-        if (tsub == 0) {
-          float4* dst = reinterpret_cast<float4*>(rec + 4 + dchunk * 8);
-          dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-          dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+        if (whole) {
+          if (tsub == 0) {
+            const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o[k] *= inv;
+            *reinterpret_cast<uint4*>(static_cast<T*>(p.out) + (qrow + g) * D + dchunk * 8) =
+                pack8<T>(o);
+          }
+        } else {
+          float* rec = recs + g * (D + 4);
+          if (lane == 0) {
+            rec[0] = m[g];
+            rec[1] = l_all;
+          }
+          if (tsub == 0) {
+            float4* dst = reinterpret_cast<float4*>(rec + 4 + dchunk * 8);
+            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+          }
         }
       }
     }
@@ -723,28 +769,35 @@ paged_decode_kernel(const DecodeParams p) {
 // kernel with programmatic dependent launch: its CTAs become resident early
 // and griddepcontrol.wait holds them until the decode kernel's writes are
 // visible.  One warp per (text, head).
-template <typename T, int D>
+template <typename T, int D, int GS>
 __global__ void __launch_bounds__(256)
 split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
-                    const float* __restrict__ records, int num_seqs, int num_heads) {
+                    const float* __restrict__ records, int num_seqs, int num_vheads,
+                    int num_q_heads, int nsub) {
   griddep_wait();
   const int lane = threadIdx.x & 31;
   const int seg = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (seg >= num_seqs * num_heads) return;
-  const int s = seg / num_heads;
-  const int h = seg - s * num_heads;
-  const int q = header[1], G = header[2], W = header[3];
+  if (seg >= num_seqs * num_vheads) return;
+  const int s = seg / num_vheads;
+  const int vh = seg - s * num_vheads;
+  const int q = header[1], grain = header[2], W = header[3];
   const int32_t* prefix = header + kHeaderInts;
   const int seg0 = prefix[s];
-  const int ns = (prefix[s + 1] - seg0) / num_heads;
+  const int ns = (prefix[s + 1] - seg0) / num_vheads;
   if (ns == 0) return;  // zero-filled by the decode kernel
   const int dyn_base = W * q;
-  auto unit_of = [&](int c) { return c < dyn_base ? c / q : W + (c - dyn_base) / G; };
-  const int a = seg0 + h * ns;
+  auto unit_of = [&](int c) { return c < dyn_base ? c / q : W + (c - dyn_base) / grain; };
+  const int a = seg0 + vh * ns;
   const int u_lo = unit_of(a);
   const int u_hi = unit_of(a + ns - 1);
   if (u_lo == u_hi) return;  // finished in place by the decode kernel
-  merge_partials<T, D>(records, out, seg, u_lo, u_hi, lane);
+  const int group = num_q_heads / (num_vheads / nsub);  // query heads per key/value head
+  const int qh0 = (vh / nsub) * group + (vh % nsub) * GS;
+#pragma unroll 1
+  for (int g = 0; g < GS; ++g)
+    merge_partials<T, D>(records + g * (D + 4), GS * (D + 4),
+                         out + (static_cast<int64_t>(s) * num_q_heads + qh0 + g) * D, seg, u_lo,
+                         u_hi, lane);
 }
 
 namespace {
@@ -756,16 +809,33 @@ int device_sm_count() {
   return sms;
 }
 
-size_t decode_smem_bytes(int D, int num_seqs) {
-  const int area = D == 128 ? warp_area_bytes(128, kDecodeStages) : warp_area_bytes(64, kDecodeStages);
-  return static_cast<size_t>(kDecodeWarps) * area + align_up(sizeof(int32_t) * (num_seqs + 1), 16);
+size_t decode_smem_bytes(int D, int num_seqs, int gs) {
+  return static_cast<size_t>(kDecodeWarps) * warp_area_bytes(D, kDecodeStages, gs) +
+         align_up(sizeof(int32_t) * (num_seqs + 1), 16);
+}
+
+// How query heads map onto work: a key/value head's G query heads are split
+// into nsub subsets of GS (GS in {4, 2, 1}, the largest that divides G); the
+// flat order runs over Hkv * nsub "virtual heads".  Multi-head attention is
+// G = GS = nsub = 1.
+struct HeadLayout {
+  int group = 1, gs = 1, nsub = 1, vheads = 0;
+};
+HeadLayout head_layout(int num_heads, int num_kv_heads) {
+  HeadLayout l;
+  if (num_kv_heads < 1 || num_heads < 1 || num_heads % num_kv_heads) return l;
+  l.group = num_heads / num_kv_heads;
+  l.gs = l.group % 4 == 0 ? 4 : (l.group % 2 == 0 ? 2 : 1);
+  l.nsub = l.group / l.gs;
+  l.vheads = num_kv_heads * l.nsub;
+  return l;
 }
 
 // Resident CTAs per SM of `kernel` with `smem` dynamic shared memory, cached
 // per (device, kernel, smem).  The kernel's dynamic shared-memory limit is
 // raised once per (device, kernel) to the most any call can need, so a call
 // with fewer texts never lowers it below what a larger one uses.
-int resident_ctas(const void* kernel, size_t smem, int head_dim) {
+int resident_ctas(const void* kernel, size_t smem, int head_dim, int gs) {
   static std::mutex mu;
   static std::map<std::tuple<int, const void*, size_t>, int> cache;
   static std::map<std::pair<int, const void*>, bool> raised;
@@ -777,7 +847,7 @@ int resident_ctas(const void* kernel, size_t smem, int head_dim) {
   if (it != cache.end()) return it->second;
   const auto rkey = std::make_pair(dev, kernel);
   if (!raised.count(rkey)) {
-    const size_t most = decode_smem_bytes(head_dim, kMaxSeqs);
+    const size_t most = decode_smem_bytes(head_dim, kMaxSeqs, gs);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(most)) != cudaSuccess) {
       cudaGetLastError();
@@ -815,10 +885,10 @@ struct Plan {
 // Persistent grid: every SM filled with resident CTAs, but never more warps
 // than there can be chunks.
 Plan plan_decode(const void* kernel, int D, int B, int num_seqs, int num_heads,
-                 int max_blocks_per_seq, int64_t forced_warps) {
+                 int max_blocks_per_seq, int64_t forced_warps, int gs) {
   Plan pl;
-  pl.smem = decode_smem_bytes(D, num_seqs);
-  const int occ = resident_ctas(kernel, pl.smem, D);
+  pl.smem = decode_smem_bytes(D, num_seqs, gs);
+  const int occ = resident_ctas(kernel, pl.smem, D, gs);
   const int sms = device_sm_count();
   if (occ <= 0 || sms <= 0) return pl;
   const int CH = chunk_tokens(D);
@@ -838,24 +908,24 @@ Plan plan_decode(const void* kernel, int D, int B, int num_seqs, int num_heads,
 // create: grains number at most kGrainsPerWarp per warp.
 int64_t max_units(int64_t warps) { return warps * (kGrainsPerWarp + 1) + 1; }
 
-size_t records_bytes(int64_t records, int D) {
-  return static_cast<size_t>(records) * (D + 4) * sizeof(float);
+size_t records_bytes(int64_t records, int D, int gs) {
+  return static_cast<size_t>(records) * gs * (D + 4) * sizeof(float);
 }
 
-template <typename T, int D, int B, bool FUSED = false>
+template <typename T, int D, int B, bool FUSED, int GS>
 const void* decode_kernel_ptr() {
   return reinterpret_cast<const void*>(
-      &paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED>);
+      &paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS>);
 }
 
-template <typename T, int D, int B, bool FUSED>
-cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
-  const Plan pl = plan_decode(decode_kernel_ptr<T, D, B, FUSED>(), D, B, a.num_seqs, a.num_heads,
-                              a.max_blocks_per_seq, a.forced_warps);
+template <typename T, int D, int B, bool FUSED, int GS>
+cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
+  const Plan pl = plan_decode(decode_kernel_ptr<T, D, B, FUSED, GS>(), D, B, a.num_seqs,
+                              hl.vheads, a.max_blocks_per_seq, a.forced_warps, GS);
   if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
-  const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_heads;
+  const int64_t segs = static_cast<int64_t>(a.num_seqs) * hl.vheads;
   const size_t need = header_bytes(a.num_seqs) + kGrabBytes +
-                      records_bytes(max_units(pl.work_warps) + segs, D);
+                      records_bytes(max_units(pl.work_warps) + segs, D, GS);
   if (a.workspace_bytes < need) return cudaErrorInvalidValue;
   DecodeParams p;
   p.out = a.out;
@@ -866,7 +936,10 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   p.context_lens = a.context_lens;
   p.qk_scale_log2 = a.scale * 1.4426950408889634f;  // log2(e)
   p.num_seqs = a.num_seqs;
-  p.num_heads = a.num_heads;
+  p.num_heads = hl.vheads;
+  p.num_q_heads = a.num_heads;
+  p.num_kv_heads = a.num_kv_heads;
+  p.nsub = hl.nsub;
   p.max_blocks_per_seq = a.max_blocks_per_seq;
   p.num_blocks = a.num_blocks;
   p.num_work_warps = pl.work_warps;
@@ -891,92 +964,118 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(
-      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED>, p);
+      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS>, p);
   if (err != cudaSuccess) return err;
-  const int per_cta = 8;  // warps, one per (text, head)
+  const int per_cta = 8;  // warps, one per (text, virtual head)
   cfg.gridDim = dim3(static_cast<unsigned>((segs + per_cta - 1) / per_cta));
   cfg.blockDim = dim3(per_cta * 32);
   cfg.dynamicSmemBytes = 0;
-  err = cudaLaunchKernelEx(&cfg, split_reduce_kernel<T, D>, static_cast<T*>(a.out),
+  err = cudaLaunchKernelEx(&cfg, split_reduce_kernel<T, D, GS>, static_cast<T*>(a.out),
                            static_cast<const int32_t*>(p.header),
-                           static_cast<const float*>(p.records), a.num_seqs, a.num_heads);
+                           static_cast<const float*>(p.records), a.num_seqs, hl.vheads,
+                           a.num_heads, hl.nsub);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
-template <typename T, int D, bool FUSED>
-cudaError_t dispatch_block(const DecodeArgs& a, cudaStream_t stream) {
+template <typename T, int D, bool FUSED, int GS>
+cudaError_t dispatch_block(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
   switch (a.block_size) {
-    case 4: return launch_typed<T, D, 4, FUSED>(a, stream);
-    case 8: return launch_typed<T, D, 8, FUSED>(a, stream);
-    case 16: return launch_typed<T, D, 16, FUSED>(a, stream);
-    case 32: return launch_typed<T, D, 32, FUSED>(a, stream);
+    case 4: return launch_typed<T, D, 4, FUSED, GS>(a, hl, stream);
+    case 8: return launch_typed<T, D, 8, FUSED, GS>(a, hl, stream);
+    case 16: return launch_typed<T, D, 16, FUSED, GS>(a, hl, stream);
+    case 32: return launch_typed<T, D, 32, FUSED, GS>(a, hl, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T, bool FUSED>
-cudaError_t dispatch_dim(const DecodeArgs& a, cudaStream_t stream) {
+template <typename T, bool FUSED, int GS>
+cudaError_t dispatch_dim(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
   switch (a.head_dim) {
-    case 64: return dispatch_block<T, 64, FUSED>(a, stream);
-    case 128: return dispatch_block<T, 128, FUSED>(a, stream);
+    case 64: return dispatch_block<T, 64, FUSED, GS>(a, hl, stream);
+    case 128: return dispatch_block<T, 128, FUSED, GS>(a, hl, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D, bool FUSED>
+template <typename T>
+cudaError_t dispatch_heads(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
+  if (a.slot_mapping)  // fused decode step: multi-head only
+    return hl.gs == 1 ? dispatch_dim<T, true, 1>(a, hl, stream) : cudaErrorInvalidValue;
+  switch (hl.gs) {
+    case 1: return dispatch_dim<T, false, 1>(a, hl, stream);
+    case 2: return dispatch_dim<T, false, 2>(a, hl, stream);
+    case 4: return dispatch_dim<T, false, 4>(a, hl, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D, bool FUSED, int GS>
 const void* kernel_for(int block_size, bool bf16) {
   switch (block_size) {
-    case 4: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 4, FUSED>() : decode_kernel_ptr<__half, D, 4, FUSED>();
-    case 8: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 8, FUSED>() : decode_kernel_ptr<__half, D, 8, FUSED>();
-    case 16: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 16, FUSED>() : decode_kernel_ptr<__half, D, 16, FUSED>();
-    case 32: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 32, FUSED>() : decode_kernel_ptr<__half, D, 32, FUSED>();
+    case 4: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 4, FUSED, GS>() : decode_kernel_ptr<__half, D, 4, FUSED, GS>();
+    case 8: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 8, FUSED, GS>() : decode_kernel_ptr<__half, D, 8, FUSED, GS>();
+    case 16: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 16, FUSED, GS>() : decode_kernel_ptr<__half, D, 16, FUSED, GS>();
+    case 32: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 32, FUSED, GS>() : decode_kernel_ptr<__half, D, 32, FUSED, GS>();
+    default: return nullptr;
+  }
+}
+
+template <int D>
+const void* kernel_for_variant(int block_size, bool bf16, bool fused, int gs) {
+  if (fused) return gs == 1 ? kernel_for<D, true, 1>(block_size, bf16) : nullptr;
+  switch (gs) {
+    case 1: return kernel_for<D, false, 1>(block_size, bf16);
+    case 2: return kernel_for<D, false, 2>(block_size, bf16);
+    case 4: return kernel_for<D, false, 4>(block_size, bf16);
     default: return nullptr;
   }
 }
 
 }  // namespace
 
-bool decode_sizes_supported(int num_seqs, int num_heads, int head_dim, int block_size,
-                            int max_blocks_per_seq) {
+bool decode_sizes_supported(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                            int block_size, int max_blocks_per_seq) {
   if (num_seqs < 1 || num_seqs > kMaxSeqs || num_heads < 1 || num_heads > 1024) return false;
+  const HeadLayout hl = head_layout(num_heads, num_kv_heads);
+  if (hl.vheads < 1 || hl.vheads > 1024) return false;
   if (head_dim != 64 && head_dim != 128) return false;
   if (block_size != 4 && block_size != 8 && block_size != 16 && block_size != 32) return false;
   if (max_blocks_per_seq < 1) return false;
   const int64_t CH = chunk_tokens(head_dim);
   const int64_t cap = static_cast<int64_t>(max_blocks_per_seq) * block_size;
-  const int64_t chunks = static_cast<int64_t>(num_seqs) * num_heads * ((cap + CH - 1) / CH);
+  const int64_t chunks = static_cast<int64_t>(num_seqs) * hl.vheads * ((cap + CH - 1) / CH);
   return chunks < (int64_t{1} << 30) && cap < (int64_t{1} << 30);
 }
 
-size_t decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int block_size,
-                              int max_blocks_per_seq, int64_t forced_warps) {
-  if (!decode_sizes_supported(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq))
+size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_blocks_per_seq, int64_t forced_warps) {
+  if (!decode_sizes_supported(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                              max_blocks_per_seq))
     return 0;
+  const HeadLayout hl = head_layout(num_heads, num_kv_heads);
   int64_t warps = 0;
   for (int variant = 0; variant < 4; ++variant) {
     const bool bf16 = variant & 1, fused = variant & 2;
-    const void* k = head_dim == 128
-                        ? (fused ? kernel_for<128, true>(block_size, bf16) : kernel_for<128, false>(block_size, bf16))
-                        : (fused ? kernel_for<64, true>(block_size, bf16) : kernel_for<64, false>(block_size, bf16));
-    const Plan pl = plan_decode(k, head_dim, block_size, num_seqs, num_heads,
-                                max_blocks_per_seq, forced_warps);
+    if (fused && hl.gs != 1) continue;
+    const void* k = head_dim == 128 ? kernel_for_variant<128>(block_size, bf16, fused, hl.gs)
+                                    : kernel_for_variant<64>(block_size, bf16, fused, hl.gs);
+    const Plan pl = plan_decode(k, head_dim, block_size, num_seqs, hl.vheads, max_blocks_per_seq,
+                                forced_warps, hl.gs);
     if (pl.grid <= 0) return 0;
     if (pl.work_warps > warps) warps = pl.work_warps;
   }
-  const int64_t segs = static_cast<int64_t>(num_seqs) * num_heads;
-  return header_bytes(num_seqs) + kGrabBytes + records_bytes(max_units(warps) + segs, head_dim);
+  const int64_t segs = static_cast<int64_t>(num_seqs) * hl.vheads;
+  return header_bytes(num_seqs) + kGrabBytes + records_bytes(max_units(warps) + segs, head_dim, hl.gs);
 }
 
 cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
-  if (!decode_sizes_supported(a.num_seqs, a.num_heads, a.head_dim, a.block_size,
+  if (!decode_sizes_supported(a.num_seqs, a.num_heads, a.num_kv_heads, a.head_dim, a.block_size,
                               a.max_blocks_per_seq))
     return cudaErrorInvalidValue;
-  if (a.slot_mapping)  // fused decode step
-    return a.is_bf16 ? dispatch_dim<__nv_bfloat16, true>(a, stream)
-                     : dispatch_dim<__half, true>(a, stream);
-  return a.is_bf16 ? dispatch_dim<__nv_bfloat16, false>(a, stream)
-                   : dispatch_dim<__half, false>(a, stream);
+  const HeadLayout hl = head_layout(a.num_heads, a.num_kv_heads);
+  return a.is_bf16 ? dispatch_heads<__nv_bfloat16>(a, hl, stream)
+                   : dispatch_heads<__half>(a, hl, stream);
 }
 
 }  // namespace pa

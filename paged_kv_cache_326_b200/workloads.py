@@ -148,11 +148,14 @@ def make_decode(name: str, context_lens: Sequence[int], num_heads: int, head_dim
                 block_size: int, num_blocks: int, dtype: torch.dtype, seed: int,
                 device="cpu", max_blocks_per_seq: Optional[int] = None,
                 block_order: Optional[torch.Tensor] = None,
-                poison: bool = True) -> DecodeInputs:
+                poison: bool = True, num_kv_heads: Optional[int] = None) -> DecodeInputs:
     """Generic single-layer decode step.
 
     Physical blocks are handed to the texts, in text order, from a seeded
-    random permutation of the pool (or from ``block_order`` if given)."""
+    random permutation of the pool (or from ``block_order`` if given).  With
+    ``num_kv_heads`` < ``num_heads`` the pool and the new k, v hold only the
+    shared key/value heads (grouped-query attention)."""
+    num_kv_heads = num_heads if num_kv_heads is None else num_kv_heads
     dev = torch.device(device)
     g_cpu = _gen(seed, "cpu")
     lens = [int(x) for x in context_lens]
@@ -171,12 +174,12 @@ def make_decode(name: str, context_lens: Sequence[int], num_heads: int, head_dim
         at += nb[s]
     lens_t = torch.tensor(lens, dtype=torch.int32)
     g = _gen(seed + 1000003, dev)
-    shape_pool = (num_blocks, num_heads, block_size, head_dim)
+    shape_pool = (num_blocks, num_kv_heads, block_size, head_dim)
     k_cache = _randn(shape_pool, dtype, g, dev)
     v_cache = _randn(shape_pool, dtype, g, dev)
     q = _randn((S, num_heads, head_dim), dtype, g, dev)
-    k = _randn((S, num_heads, head_dim), dtype, g, dev)
-    v = _randn((S, num_heads, head_dim), dtype, g, dev)
+    k = _randn((S, num_kv_heads, head_dim), dtype, g, dev)
+    v = _randn((S, num_kv_heads, head_dim), dtype, g, dev)
     tables_d = tables.to(dev)
     lens_d = lens_t.to(dev)
     if poison:
@@ -198,6 +201,19 @@ def tiny(seed: int = 1, device="cpu", dtype=torch.float16) -> DecodeInputs:
     seeded random order, fp16, and the write of the 4 new tokens."""
     return make_decode("tiny", [5, 9, 16, 23], num_heads=8, head_dim=64, block_size=4,
                        num_blocks=64, dtype=dtype, seed=seed, device=device)
+
+
+def llama2_70b_gqa(seed: int = 6, device="cpu", dtype=torch.float16, num_seqs: int = 64,
+                   num_blocks: int = 12288) -> DecodeInputs:
+    """One layer of a Llama-2-70B-shaped decode ("The KV Cache and
+    PagedAttention", section "What Came After": 64 query heads sharing 8
+    key/value heads): head_dim 128, blocks of 16, lengths uniform in
+    [128, 4096] (Llama 2's context), fp16."""
+    g = np.random.default_rng(seed)
+    lens = [int(x) for x in g.integers(128, 4096, size=num_seqs, endpoint=True)]
+    return make_decode("llama2_70b_gqa", lens, num_heads=64, head_dim=128, block_size=16,
+                       num_blocks=num_blocks, dtype=dtype, seed=seed, device=device,
+                       max_blocks_per_seq=4096 // 16, num_kv_heads=8)
 
 
 def opt13b_batch64_lens(seed: int = 2) -> List[int]:

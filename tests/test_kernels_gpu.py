@@ -351,3 +351,61 @@ def test_fused_step_single_token_returns_its_value():
     out = gpu_step_fused(w)
     torch.cuda.synchronize()
     assert torch.equal(out, w.v)
+
+
+# ---------------------------------------------------------------------------
+# grouped-query attention (pa_paged_attn_decode_gqa)
+# ---------------------------------------------------------------------------
+
+def gpu_step_gqa(w, status=None, out=None):
+    import paged_kv_cache_326_b200 as P
+    P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+    if out is None:
+        out = torch.empty_like(w.q)
+    P.pa_paged_attn_decode_gqa(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                               w.scale, status=status)
+    return out
+
+
+GQA_LENS = [0, 1, 17, 100, 300, 1000, 2048, 33]
+
+
+@pytest.mark.parametrize("heads", [(16, 8), (12, 4), (32, 8), (64, 8), (16, 1), (8, 8)],
+                         ids=lambda hk: f"q{hk[0]}kv{hk[1]}")
+def test_gqa_group_sizes(heads):
+    Hq, Hkv = heads
+    w = W.make_decode("gqa", GQA_LENS, num_heads=Hq, head_dim=128, block_size=16,
+                      num_blocks=2 * sum(W.blocks_needed(L, 16) for L in GQA_LENS),
+                      dtype=torch.float16, seed=Hq + Hkv, device="cuda",
+                      max_blocks_per_seq=2048 // 16, num_kv_heads=Hkv)
+    c = parity(w, check_pool=True, step=gpu_step_gqa)
+    print(f"gqa q{Hq} kv{Hkv}", c)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("block_size", [4, 32])
+def test_gqa_head_dim_64(dtype, block_size):
+    w = W.make_decode("gqa64", SHAPE_LENS, num_heads=32, head_dim=64, block_size=block_size,
+                      num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in SHAPE_LENS),
+                      dtype=dtype, seed=block_size, device="cuda",
+                      max_blocks_per_seq=160 // block_size, num_kv_heads=8)
+    parity(w, check_pool=True, step=gpu_step_gqa)
+
+
+def test_gqa_llama2_70b_shape():
+    w = W.llama2_70b_gqa(device="cuda")
+    c = parity(w, heads_per_seq=8, seed=6, step=gpu_step_gqa)
+    print("gqa llama2_70b", c)
+
+
+@pytest.mark.parametrize("warps", [1, 4096])
+def test_gqa_split_and_single_pass(warps):
+    import paged_kv_cache_326_b200 as P
+    w = W.make_decode("gqa_split", [300, 17, 1, 1000, 0, 511], num_heads=32, head_dim=128,
+                      block_size=16, num_blocks=256, dtype=torch.bfloat16, seed=11, device="cuda",
+                      max_blocks_per_seq=64, num_kv_heads=8)
+    P.pa_set_option(P.binding.PA_OPT_DECODE_WARPS, warps)
+    try:
+        parity(w, step=gpu_step_gqa)
+    finally:
+        P.pa_set_option(P.binding.PA_OPT_DECODE_WARPS, 0)
