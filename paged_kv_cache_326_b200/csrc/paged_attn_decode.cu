@@ -49,16 +49,10 @@
 //    holds every read until that kernel's writes are visible.
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstdint>
-#include <map>
-#include <mutex>
-#include <tuple>
-#include <utility>
 
-#include "dtype.cuh"
+#include "decode_common.cuh"
 #include "kernels.h"
-#include "ptx.cuh"
 
 namespace pa {
 
@@ -72,146 +66,10 @@ namespace {
 #endif
 constexpr int kDecodeWarps = PA_DECODE_WARPS;    // warps per CTA
 constexpr int kDecodeStages = PA_DECODE_STAGES;  // ring depth per warp
-constexpr int kMaxSeqs = 4096;
-// Work split: each warp first streams a static run of about kStaticPermille
-// per mille of an even share; the rest is handed out in grains from a shared
-// counter, at least kMinGrain chunks each and about kGrainsPerWarp per warp.
-#ifndef PA_STATIC_PERMILLE
-#define PA_STATIC_PERMILLE 700
-#endif
-#ifndef PA_MIN_GRAIN
-#define PA_MIN_GRAIN 16
-#endif
-constexpr int kStaticPermille = PA_STATIC_PERMILLE;
-constexpr int kGrainsPerWarp = 12;
-constexpr int kMinGrain = PA_MIN_GRAIN;
-constexpr int kDrainLimitNs = 1000000000;
-__host__ __device__ constexpr int chunk_tokens(int D) { return 2048 / D; }
 // One stage: K rows (4 KB), V rows (4 KB), the unit's GS query rows, a flag.
 __host__ __device__ constexpr int stage_bytes(int D, int gs) { return 2 * 4096 + gs * 2 * D + 128; }
 __host__ __device__ constexpr int warp_area_bytes(int D, int stages, int gs) {
   return stages * stage_bytes(D, gs) + 128;
-}
-
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-// Workspace: a header (the work split, then prefix[S+1]), the grain counter,
-// then the partial records.  The header is written by CTA 0 of the decode
-// kernel and read by the merge kernel.
-constexpr int kHeaderInts = 8;  // total, q, grain, W, 4 spare
-size_t header_bytes(int num_seqs) {
-  return align_up(sizeof(int32_t) * (kHeaderInts + num_seqs + 1), 256);
-}
-constexpr size_t kGrabBytes = 256;
-// The grain counter holds the call's epoch above bit 30; a stale epoch (an
-// earlier call's, or never set) reads as zero, so the workspace never needs
-// clearing.
-constexpr unsigned long long kGrabMask = (1ull << 30) - 1;
-constexpr unsigned long long kEpochMask = (1ull << 40) - 1;
-
-struct DecodeParams {
-  void* out;
-  const void* q;
-  const void* k_cache;
-  const void* v_cache;
-  const int32_t* block_tables;
-  const int32_t* context_lens;
-  float qk_scale_log2;
-  int num_seqs;
-  int num_heads;      // virtual heads: key/value heads x subsets (the flat order's heads)
-  int num_q_heads;    // query heads of q and out
-  int num_kv_heads;   // key/value heads of the pool
-  int nsub;           // subsets per key/value head (GS query heads each)
-  int max_blocks_per_seq;
-  int64_t num_blocks;
-  int num_work_warps;
-  const void* k_new;              // fused step only: the new token's k, v [S][H][D]
-  const void* v_new;
-  const int64_t* slot_mapping;    // fused step only: their slots
-  int32_t* header;                // work split + prefix, for the merge kernel
-  unsigned long long* grab;       // grain counter
-  unsigned long long epoch;       // 40-bit, never 0
-  float* records;
-  int32_t* status;
-  int64_t wait_limit_ns;
-};
-
-// Per-lane look-ahead entry: where flat chunk (run start + position) lives.
-template <int NB>
-struct Lookahead {
-  int s, h, j, len;  // len is the raw context length (clamped at use)
-  int blk[NB];
-};
-
-// Count one more stored partial of a (text, head) in this call; returns the
-// count including this one.
-// Merge the partials of one (text, head), stored by units w_lo..w_hi: with
-// M = max_i m_i and f_i = 2^(m_i - M),
-//     out = (sum_i f_i o_i) / (sum_i f_i l_i),
-// which equals the softmax-weighted sum over all the text's tokens (up to
-// rounding).  Partials are read in warp order, so the result does not depend
-// on which warp merges.  Reads go through L2 (other SMs wrote them).
-template <typename T, int D>
-__device__ __forceinline__ void merge_partials(const float* records, int64_t rec_stride,
-                                               T* out_row, int64_t sh, int w_lo, int w_hi,
-                                               int lane) {
-  constexpr int PER = D / 32;
-  const int n = w_hi - w_lo + 1;
-  // running max over the partials, one partial per lane
-  float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(records + (w_lo + i + sh) * rec_stride));
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float L = 0.f;
-  float acc[PER];
-#pragma unroll
-  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    // weight f_i = 2^(m_i - M) of partial i0 + lane, and its share of the sum
-    float f = 0.f, lf = 0.f;
-    if (i0 + lane < n) {
-      const float* rec = records + (w_lo + i0 + lane + sh) * rec_stride;
-      f = M == -INFINITY ? 0.f : fast_exp2(__ldcg(rec) - M);
-      lf = f * __ldcg(rec + 1);
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) lf += __shfl_xor_sync(0xffffffffu, lf, off);
-    L += lf;
-    // outputs: eight partials' loads in flight at a time
-    const int cnt = min(32, n - i0);
-    for (int b = 0; b < cnt; b += 8) {
-      float o[8][PER];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float* rec = records + (w_lo + i0 + min(b + u, cnt - 1) + sh) * rec_stride + 4 + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(rec));
-          o[u][0] = v.x; o[u][1] = v.y; o[u][2] = v.z; o[u][3] = v.w;
-        } else {
-          const float2 v = __ldcg(reinterpret_cast<const float2*>(rec));
-          o[u][0] = v.x; o[u][1] = v.y;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float fu = __shfl_sync(0xffffffffu, f, min(b + u, 31));
-        if (b + u < cnt) {
-#pragma unroll
-          for (int k = 0; k < PER; ++k) acc[k] = fmaf(fu, o[u][k], acc[k]);
-        }
-      }
-    }
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  T* o = out_row + lane * PER;
-  if constexpr (PER == 4) {
-    uint2 v;
-    v.x = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
-    v.y = Elem<T>::from_float2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(o) = v;
-  } else {
-    *reinterpret_cast<uint32_t*>(o) = Elem<T>::from_float2(acc[0] * inv, acc[1] * inv);
-  }
 }
 
 }  // namespace
@@ -254,95 +112,16 @@ paged_decode_kernel(const DecodeParams p) {
   // Inputs may come from the kernel launched just before (the cache write).
   griddep_wait();
 
-  // ---- prologue: prefix[s] = H * (chunks of texts before s), block-wide scan
-  {
-    const int nthr = WARPS * 32;
-    const int per = (S + nthr - 1) / nthr;
-    const int s0 = min(S, tid * per), s1 = min(S, s0 + per);
-    int local = 0;
-    for (int s = s0; s < s1; ++s) {
-      int L = __ldg(p.context_lens + s);
-      if (L < 0 || L > cap) {
-        if (blockIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
-        L = min(max(L, 0), cap);
-      }
-      local += (L + CH - 1) / CH;
-    }
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int before = 0;
-    for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    int run = before + incl - local;
-    for (int s = s0; s < s1; ++s) {
-      int L = min(max(__ldg(p.context_lens + s), 0), cap);
-      prefix[s] = run * H;
-      run += (L + CH - 1) / CH;
-    }
-    if (tid == nthr - 1) prefix[S] = run * H;
-    __syncthreads();
-  }
-  const int total = prefix[S];
-  const int W = p.num_work_warps;
-  // Static runs of q chunks (units 0..W-1), then grains of `grain` chunks (units
-  // W, W+1, ...) covering the rest of the flat order.
-  int q = W == 1 ? total : static_cast<int>(static_cast<long long>(total) * kStaticPermille / 1000 / W);
-  if (q < 32 && W > 1) q = 0;
-  const int dyn_base = W * q;
-  const int dyn = total - dyn_base;
-  const int grain = max(kMinGrain, (dyn + kGrainsPerWarp * W - 1) / (kGrainsPerWarp * W));
-  if (blockIdx.x == 0) {
-    if (tid == 0) {
-      p.header[0] = total;
-      p.header[1] = q;
-      p.header[2] = grain;
-      p.header[3] = W;
-    }
-    for (int i = tid; i <= S; i += WARPS * 32) p.header[kHeaderInts + i] = prefix[i];
-  }
-  // Texts with no tokens get zeros (spread over the CTAs).
-  for (int s = blockIdx.x; s < S; s += gridDim.x) {
-    if (prefix[s + 1] == prefix[s]) {
-      uint4* o = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + static_cast<int64_t>(s) * Hq * D);
-      for (int i = tid; i < Hq * D / 8; i += WARPS * 32) o[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
+  const WorkSplit sp = decode_prologue<T, D, CH, WARPS * 32>(p, prefix, warp_tot, cap);
+  const int total = sp.total;
+  const int W = sp.W;
 
   const int w = blockIdx.x * WARPS + warp;
-  // Fused step: the cache write, 16-byte vectors spread over the working
-  // warps (as in kv_cache_write_kernel).  No read in this launch touches
-  // these slots, so each warp does its share whenever it has a moment: right
-  // after issuing its first copies, while it waits for them.
+  // One-launch step: the cache write.  No read in this launch touches these
+  // slots, so each warp does its share whenever it has a moment: right after
+  // issuing its first copies, while it waits for them.
   auto fused_write = [&]() {
-    if constexpr (FUSED) {
-      const int vpr = D / 8;
-      const int64_t per_text = static_cast<int64_t>(Hkv) * vpr;
-      const int64_t nvec = per_text * S;
-      const int64_t num_slots = p.num_blocks * B;
-      uint4* kcw = static_cast<uint4*>(const_cast<void*>(p.k_cache));
-      uint4* vcw = static_cast<uint4*>(const_cast<void*>(p.v_cache));
-      for (int64_t i = static_cast<int64_t>(w) * 32 + lane; i < nvec;
-           i += static_cast<int64_t>(W) * 32) {
-        const int64_t s = i / per_text;
-        const int64_t r = i - s * per_text;
-        const int64_t slot = __ldg(p.slot_mapping + s);
-        if (slot < 0) continue;
-        if (slot >= num_slots) {
-          if (r == 0) set_status(p.status, -9 /* PA_ERR_BAD_SLOT */);
-          continue;
-        }
-        const int64_t h = r / vpr, c = r - (r / vpr) * vpr;
-        const int64_t blk = slot / B, place = slot - blk * B;
-        const int64_t dst = ((blk * Hkv + h) * B + place) * vpr + c;
-        kcw[dst] = __ldg(static_cast<const uint4*>(p.k_new) + i);
-        vcw[dst] = __ldg(static_cast<const uint4*>(p.v_new) + i);
-      }
-    }
+    if constexpr (FUSED) fused_cache_write<D, B>(p, w, W, lane);
   };
   if (w >= W) return;
   if (total == 0) {
@@ -364,123 +143,9 @@ paged_decode_kernel(const DecodeParams p) {
   const T* __restrict__ vc = static_cast<const T*>(p.v_cache);
   const T* __restrict__ qg = static_cast<const T*>(p.q);
 
-  int step = 1;
-  while (step * 2 <= S) step *= 2;
-
-  // ---- work units and their windows ----------------------------------
-  // A unit is a run of consecutive flat chunks: first this warp's static run,
-  // then grains taken from the shared counter.  Units are cut into windows of
-  // at most 32 chunks (one chunk per lane for the look-ahead); a unit's last
-  // two windows are balanced, so only the very last window of all the work
-  // can be shorter than the copy ring.
-  const unsigned long long e34 = p.epoch & ((1ull << 34) - 1);
-  // Chunk offset of the grain whose counter value is `old` (lane 0).  The
-  // counter carries this call's epoch above bit 30; a stale epoch (left by an
-  // earlier call, or never set) is replaced by compare-and-swap, so the
-  // workspace never needs clearing.
-  auto grab_resolve = [&](unsigned long long old) -> int {
-    if ((old >> 30) == e34) return static_cast<int>(old & kGrabMask);
-    unsigned long long seen = old + static_cast<unsigned long long>(grain);
-    while (true) {
-      if ((seen >> 30) == e34) {
-        const unsigned long long o2 = atomicAdd(p.grab, static_cast<unsigned long long>(grain));
-        if ((o2 >> 30) == e34) return static_cast<int>(o2 & kGrabMask);
-        seen = o2 + static_cast<unsigned long long>(grain);
-        continue;
-      }
-      const unsigned long long prev =
-          atomicCAS(p.grab, seen, (e34 << 30) | static_cast<unsigned long long>(grain));
-      if (prev == seen) return 0;
-      seen = prev;
-    }
-  };
-  bool static_taken = false, exhausted = false, pend_live = false;
-  unsigned long long pend = 0;  // lane 0: counter value of the next grain
-  int u_start = 0, u_count = 0, u_id = -1, u_off = 0;
-  auto grab_issue = [&]() {
-    if (lane == 0) pend = atomicAdd(p.grab, static_cast<unsigned long long>(grain));
-    pend_live = true;
-  };
-  auto next_unit = [&]() {
-    if (!static_taken) {
-      static_taken = true;
-      if (q > 0) {
-        u_start = w * q;
-        u_count = q;
-        u_id = w;
-        u_off = 0;
-        if (dyn > 0) grab_issue();
-        return;
-      }
-    }
-    if (dyn <= 0) {
-      exhausted = true;
-      return;
-    }
-    if (!pend_live) grab_issue();
-    int off = 0;
-    if (lane == 0) off = grab_resolve(pend);
-    off = __shfl_sync(0xffffffffu, off, 0);
-    pend_live = false;
-    if (off >= dyn) {
-      exhausted = true;
-      return;
-    }
-    u_start = dyn_base + off;
-    u_count = min(grain, dyn - off);
-    u_id = W + off / grain;
-    u_off = 0;
-    grab_issue();  // the next grain, resolved when this one runs out
-  };
-  // Next window of this warp's work: start chunk, count (0 = no more), unit.
-  auto next_window = [&](int& ws, int& wc, int& wu) {
-    if (!exhausted && u_off >= u_count) next_unit();
-    if (exhausted) {
-      ws = 0;
-      wc = 0;
-      wu = -1;
-      return;
-    }
-    const int rem = u_count - u_off;
-    const int n = rem <= 32 ? rem : (rem < 64 ? rem / 2 : 32);
-    ws = u_start + u_off;
-    wc = n;
-    wu = u_id;
-    u_off += n;
-  };
-
-  // Where each chunk of a window lives, one chunk per lane.  Reads only
-  // shared memory before issuing its global loads, whose results are not
-  // used until the copy issue reaches this window.
-  auto lookahead = [&](int ws, int wc) {
-    Lookahead<NB> e;
-    if (wc <= 0) {
-      e.s = e.h = e.j = e.len = 0;
-#pragma unroll
-      for (int k = 0; k < NB; ++k) e.blk[k] = -1;
-      return e;
-    }
-    const int c = ws + min(lane, wc - 1);
-    int s = 0;
-    for (int st = step; st > 0; st >>= 1)
-      if (s + st < S && prefix[s + st] <= c) s += st;
-    const int seg0 = prefix[s];
-    const int ns = (prefix[s + 1] - seg0) / H;
-    const int within = c - seg0;
-    const int h = within / ns;
-    const int j = within - h * ns;
-    e.s = s;
-    e.h = h;
-    e.j = j;
-    e.len = __ldg(p.context_lens + s);
-    const int32_t* row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
-#pragma unroll
-    for (int k = 0; k < NB; ++k) {
-      const int idx = (j * CH) / B + k;
-      e.blk[k] = idx < p.max_blocks_per_seq ? __ldg(row + idx) : -1;
-    }
-    return e;
-  };
+  Scheduler<CH, B, NB> sched(p, prefix, sp, w, lane);
+  auto next_window = [&](int& ws, int& wc, int& wu) { sched.next_window(ws, wc, wu); };
+  auto lookahead = [&](int ws, int wc) { return sched.lookahead(ws, wc); };
 
   int ws0, wc0, wu0, ws1, wc1, wu1;
   next_window(ws0, wc0, wu0);
@@ -763,64 +428,15 @@ paged_decode_kernel(const DecodeParams p) {
   }
 }
 
-// Merge kernel: for every (text, head) whose chunks fell into several work
-// units, combine the units' partials (log-sum-exp); the decode kernel has
-// already written every other output.  Launched right after the decode
-// kernel with programmatic dependent launch: its CTAs become resident early
-// and griddepcontrol.wait holds them until the decode kernel's writes are
-// visible.  One warp per (text, head).
-template <typename T, int D, int GS>
-__global__ void __launch_bounds__(256)
-split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
-                    const float* __restrict__ records, int num_seqs, int num_vheads,
-                    int num_q_heads, int nsub) {
-  griddep_wait();
-  const int lane = threadIdx.x & 31;
-  const int seg = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (seg >= num_seqs * num_vheads) return;
-  const int s = seg / num_vheads;
-  const int vh = seg - s * num_vheads;
-  const int q = header[1], grain = header[2], W = header[3];
-  const int32_t* prefix = header + kHeaderInts;
-  const int seg0 = prefix[s];
-  const int ns = (prefix[s + 1] - seg0) / num_vheads;
-  if (ns == 0) return;  // zero-filled by the decode kernel
-  const int dyn_base = W * q;
-  auto unit_of = [&](int c) { return c < dyn_base ? c / q : W + (c - dyn_base) / grain; };
-  const int a = seg0 + vh * ns;
-  const int u_lo = unit_of(a);
-  const int u_hi = unit_of(a + ns - 1);
-  if (u_lo == u_hi) return;  // finished in place by the decode kernel
-  const int group = num_q_heads / (num_vheads / nsub);  // query heads per key/value head
-  const int qh0 = (vh / nsub) * group + (vh % nsub) * GS;
-#pragma unroll 1
-  for (int g = 0; g < GS; ++g)
-    merge_partials<T, D>(records + g * (D + 4), GS * (D + 4),
-                         out + (static_cast<int64_t>(s) * num_q_heads + qh0 + g) * D, seg, u_lo,
-                         u_hi, lane);
-}
-
 namespace {
-
-int device_sm_count() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return sms;
-}
 
 size_t decode_smem_bytes(int D, int num_seqs, int gs) {
   return static_cast<size_t>(kDecodeWarps) * warp_area_bytes(D, kDecodeStages, gs) +
          align_up(sizeof(int32_t) * (num_seqs + 1), 16);
 }
 
-// How query heads map onto work: a key/value head's G query heads are split
-// into nsub subsets of GS (GS in {4, 2, 1}, the largest that divides G); the
-// flat order runs over Hkv * nsub "virtual heads".  Multi-head attention is
-// G = GS = nsub = 1.
-struct HeadLayout {
-  int group = 1, gs = 1, nsub = 1, vheads = 0;
-};
+// CUDA-core kernel: a key/value head's G query heads are split into nsub
+// subsets of GS (GS in {4, 2, 1}, the largest that divides G).
 HeadLayout head_layout(int num_heads, int num_kv_heads) {
   HeadLayout l;
   if (num_kv_heads < 1 || num_heads < 1 || num_heads % num_kv_heads) return l;
@@ -831,85 +447,12 @@ HeadLayout head_layout(int num_heads, int num_kv_heads) {
   return l;
 }
 
-// Resident CTAs per SM of `kernel` with `smem` dynamic shared memory, cached
-// per (device, kernel, smem).  The kernel's dynamic shared-memory limit is
-// raised once per (device, kernel) to the most any call can need, so a call
-// with fewer texts never lowers it below what a larger one uses.
-int resident_ctas(const void* kernel, size_t smem, int head_dim, int gs) {
-  static std::mutex mu;
-  static std::map<std::tuple<int, const void*, size_t>, int> cache;
-  static std::map<std::pair<int, const void*>, bool> raised;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(dev, kernel, smem);
-  const auto it = cache.find(key);
-  if (it != cache.end()) return it->second;
-  const auto rkey = std::make_pair(dev, kernel);
-  if (!raised.count(rkey)) {
-    const size_t most = decode_smem_bytes(head_dim, kMaxSeqs, gs);
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(most)) != cudaSuccess) {
-      cudaGetLastError();
-      return 0;
-    }
-    raised[rkey] = true;
-  }
-  int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kDecodeWarps * 32, smem) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    occ = 0;
-  }
-  cache[key] = occ;
-  return occ;
-}
-
-// A fresh 40-bit epoch per launch (never 0, so a zeroed workspace holds no
-// live counts).
-unsigned long long next_epoch() {
-  static std::atomic<unsigned long long> counter{0};
-  unsigned long long e;
-  do {
-    e = (counter.fetch_add(1) + 1) & kEpochMask;
-  } while (e == 0);
-  return e;
-}
-
-struct Plan {
-  int grid = 0;
-  int work_warps = 0;
-  size_t smem = 0;
-};
-
-// Persistent grid: every SM filled with resident CTAs, but never more warps
-// than there can be chunks.
-Plan plan_decode(const void* kernel, int D, int B, int num_seqs, int num_heads,
-                 int max_blocks_per_seq, int64_t forced_warps, int gs) {
-  Plan pl;
-  pl.smem = decode_smem_bytes(D, num_seqs, gs);
-  const int occ = resident_ctas(kernel, pl.smem, D, gs);
-  const int sms = device_sm_count();
-  if (occ <= 0 || sms <= 0) return pl;
-  const int CH = chunk_tokens(D);
-  const int64_t cap = static_cast<int64_t>(max_blocks_per_seq) * B;
-  const int64_t chunks_max = static_cast<int64_t>(num_seqs) * num_heads * ((cap + CH - 1) / CH);
-  int64_t warps = static_cast<int64_t>(sms) * occ * kDecodeWarps;
-  const int64_t useful = ((chunks_max + kDecodeWarps - 1) / kDecodeWarps) * kDecodeWarps;
-  if (warps > useful) warps = useful;
-  if (forced_warps > 0) warps = forced_warps;
-  if (warps < 1) warps = 1;
-  pl.work_warps = static_cast<int>(warps);
-  pl.grid = static_cast<int>((warps + kDecodeWarps - 1) / kDecodeWarps);
-  return pl;
-}
-
-// Units (static runs plus grains) a launch with `warps` working warps can
-// create: grains number at most kGrainsPerWarp per warp.
-int64_t max_units(int64_t warps) { return warps * (kGrainsPerWarp + 1) + 1; }
-
-size_t records_bytes(int64_t records, int D, int gs) {
-  return static_cast<size_t>(records) * gs * (D + 4) * sizeof(float);
+// Persistent grid for one decode kernel variant.
+Plan plan_variant(const void* kernel, int D, int B, int num_seqs, int vheads,
+                  int max_blocks_per_seq, int64_t forced_warps, int gs) {
+  return plan_decode(kernel, decode_smem_bytes(D, num_seqs, gs), decode_smem_bytes(D, kMaxSeqs, gs),
+                     kDecodeWarps, chunk_tokens(D), B, num_seqs, vheads, max_blocks_per_seq,
+                     forced_warps);
 }
 
 template <typename T, int D, int B, bool FUSED, int GS>
@@ -920,8 +463,8 @@ const void* decode_kernel_ptr() {
 
 template <typename T, int D, int B, bool FUSED, int GS>
 cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
-  const Plan pl = plan_decode(decode_kernel_ptr<T, D, B, FUSED, GS>(), D, B, a.num_seqs,
-                              hl.vheads, a.max_blocks_per_seq, a.forced_warps, GS);
+  const Plan pl = plan_variant(decode_kernel_ptr<T, D, B, FUSED, GS>(), D, B, a.num_seqs,
+                               hl.vheads, a.max_blocks_per_seq, a.forced_warps, GS);
   if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
   const int64_t segs = static_cast<int64_t>(a.num_seqs) * hl.vheads;
   const size_t need = header_bytes(a.num_seqs) + kGrabBytes +
@@ -940,6 +483,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   p.num_q_heads = a.num_heads;
   p.num_kv_heads = a.num_kv_heads;
   p.nsub = hl.nsub;
+  p.gs = GS;
   p.max_blocks_per_seq = a.max_blocks_per_seq;
   p.num_blocks = a.num_blocks;
   p.num_work_warps = pl.work_warps;
@@ -966,14 +510,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   cudaError_t err = cudaLaunchKernelEx(
       &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS>, p);
   if (err != cudaSuccess) return err;
-  const int per_cta = 8;  // warps, one per (text, virtual head)
-  cfg.gridDim = dim3(static_cast<unsigned>((segs + per_cta - 1) / per_cta));
-  cfg.blockDim = dim3(per_cta * 32);
-  cfg.dynamicSmemBytes = 0;
-  err = cudaLaunchKernelEx(&cfg, split_reduce_kernel<T, D, GS>, static_cast<T*>(a.out),
-                           static_cast<const int32_t*>(p.header),
-                           static_cast<const float*>(p.records), a.num_seqs, hl.vheads,
-                           a.num_heads, hl.nsub);
+  err = launch_merge<T, D>(p, GS, stream);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
@@ -1060,8 +597,8 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
     if (fused && hl.gs != 1) continue;
     const void* k = head_dim == 128 ? kernel_for_variant<128>(block_size, bf16, fused, hl.gs)
                                     : kernel_for_variant<64>(block_size, bf16, fused, hl.gs);
-    const Plan pl = plan_decode(k, head_dim, block_size, num_seqs, hl.vheads, max_blocks_per_seq,
-                                forced_warps, hl.gs);
+    const Plan pl = plan_variant(k, head_dim, block_size, num_seqs, hl.vheads, max_blocks_per_seq,
+                                 forced_warps, hl.gs);
     if (pl.grid <= 0) return 0;
     if (pl.work_warps > warps) warps = pl.work_warps;
   }
