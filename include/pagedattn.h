@@ -176,6 +176,42 @@ int pa_decode_step(void* out, const void* q, const void* k, const void* v, void*
                    pa_stream_t stream);
 
 /*
+ * pa_paged_attn_decode_gqa_workspace_size — as
+ * pa_paged_attn_decode_workspace_size, for pa_paged_attn_decode_gqa with
+ * num_kv_heads key/value heads.  Returns 0 for unsupported sizes (including
+ * num_heads not a multiple of num_kv_heads).
+ */
+size_t pa_paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                               int head_dim, int block_size,
+                                               int max_blocks_per_seq);
+
+/*
+ * pa_paged_attn_decode_gqa — pa_paged_attn_decode for a pool holding fewer
+ * key/value heads than there are query heads (grouped-query attention; one
+ * key/value head is multi-query attention): "The KV Cache and
+ * PagedAttention", section "What Came After" (several query heads share one
+ * set of stored keys and values, shrinking the cache).  With
+ * G = num_heads / num_kv_heads, query head h reads key/value head h / G:
+ *     z_t = scale * sum_d q[s][h][d] * K_t[h / G][d],
+ *     out[s][h][:] = sum_t softmax(z)_t * V_t[h / G][:].
+ *
+ *   q, out         [num_seqs][num_heads][head_dim] dt, device
+ *   k_cache,v_cache [num_blocks][num_kv_heads][block_size][head_dim] dt
+ *   workspace      pa_paged_attn_decode_gqa_workspace_size(...) bytes
+ *   other arguments, arithmetic, errors as for pa_paged_attn_decode.
+ * num_kv_heads == num_heads is exactly pa_paged_attn_decode.  Each key/value
+ * row is read from HBM once per (text, key/value head) and used by all the
+ * query heads that share it.  num_heads must be a multiple of num_kv_heads
+ * (else PA_ERR_INVALID).
+ */
+int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             float scale, int num_seqs, int num_heads, int num_kv_heads,
+                             int head_dim, int block_size, int max_blocks_per_seq,
+                             int64_t num_blocks, pa_dtype dt, void* workspace,
+                             size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
+
+/*
  * pa_paged_attn_decode_noalloc — pa_paged_attn_decode without a caller
  * workspace, for callers that cannot allocate device memory (a host framework
  * that owns every device allocation, a fixed memory budget, a loop where an
