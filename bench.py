@@ -37,14 +37,27 @@ METRIC = "paged decode KV HBM GB/s (% of B200 peak) and decode tokens/s, 1 GPU"
 WORKLOAD = "opt13b_batch64"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_opt13b_batch64_traffic.json")
-KERNEL_SOURCES = ["paged_kv_cache_326_b200/csrc/paged_attn_decode.cu",
-                  "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]
+# Per workload: the committed ncu DRAM-traffic capture of its decode kernel and
+# the sources that kernel is built from (the capture counts only while they
+# are unchanged).
+TRAFFIC = {
+    "opt13b_batch64": (
+        os.path.join(ROOT, "profiles", "paged_decode_opt13b_batch64_traffic.json"),
+        ["paged_kv_cache_326_b200/csrc/paged_attn_decode.cu",
+         "paged_kv_cache_326_b200/csrc/decode_common.cuh",
+         "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
+    "llama2_70b_gqa": (
+        os.path.join(ROOT, "profiles", "paged_decode_mma_llama2_70b_gqa_traffic.json"),
+        ["paged_kv_cache_326_b200/csrc/paged_attn_decode_mma.cu",
+         "paged_kv_cache_326_b200/csrc/decode_common.cuh",
+         "paged_kv_cache_326_b200/csrc/mma_ptx.cuh",
+         "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
+}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(workload: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in TRAFFIC[workload][1]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -58,14 +71,14 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
 
 
-def traffic_per_launch(path: str):
+def traffic_per_launch(workload: str, path: str):
     """DRAM bytes per launch of the decode kernel from the committed ncu
     capture, if it was taken on this path and on the kernel as it is now;
     else None."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(TRAFFIC[workload][0]) as f:
             t = json.load(f)
-        if t.get("kernel_source_hash") == kernel_source_hash() and t.get("path") == path:
+        if t.get("kernel_source_hash") == kernel_source_hash(workload) and t.get("path") == path:
             return float(t["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -151,8 +164,13 @@ def oracle_runner(w, num_pairs):
     oi = oracle_inputs(w.q, w.k, w.v, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
                        w.slot_mapping, w.block_size, seqs)
     lens = w.context_lens.tolist()
-    sample_bytes = sum(lens[s] for s, _ in pairs) * 2 * w.head_dim * w.q.element_size()
     full = num_pairs == len(seqs) * H
+    # bytes of the KV cache the sample covers (each key/value head once)
+    Hkv = w.k_cache.shape[1]
+    if full:
+        sample_bytes = sum(lens[s] for s in seqs) * 2 * Hkv * w.head_dim * w.q.element_size()
+    else:
+        sample_bytes = sum(lens[s] for s, _ in pairs) * 2 * w.head_dim * w.q.element_size()
 
     def run():
         with threadpool_limits(limits=1):
@@ -172,7 +190,7 @@ def cpu_baseline(w, budget_s=12.0):
         if el >= budget_s or reps >= 20:
             break
     return {"value": sample_bytes * reps / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"all {w.num_seqs} texts x {w.num_heads} heads of the batch-64 step, "
+            "sample": f"all {w.num_seqs} texts x {w.num_heads} query heads of the step ({w.name}), "
                       f"{reps} run(s), {el:.1f} s, numpy fp64, BLAS limited to 1 thread"}
 
 
@@ -222,6 +240,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
+    ap.add_argument("--gqa-kernel", choices=["auto", "cores", "tensor"], default="auto",
+                    help="grouped-query workload: kernel choice (PA_OPT_GQA_KERNEL)")
     ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa"],
                     default="opt13b_batch64",
                     help="llama2_70b_gqa: 64 query heads on 8 key/value heads (two calls)")
@@ -244,6 +264,8 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     gqa = args.workload == "llama2_70b_gqa"
+    P.pa_set_option(P.PA_OPT_GQA_KERNEL, {"auto": 0, "cores": 1, "tensor": 2}[args.gqa_kernel])
+    gqa_kernel = "CUDA-core" if args.gqa_kernel == "cores" else "tensor-core"
     if gqa:
         args.path = "calls"   # the one-launch step is multi-head only
         w = W.llama2_70b_gqa(seed=dist.batch_seed(6, ranks), device=dev)
@@ -370,17 +392,19 @@ def main():
                    "num_blocks": w.num_blocks, "kv_bytes_per_step": step_kv,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB)",
                    "parallelism": f"independent batch per GPU x{world}",
-                   "path": "pa_decode_step" if fused else "pa_kv_cache_write + pa_paged_attn_decode"},
+                   "path": ("pa_decode_step" if fused else
+                            f"pa_kv_cache_write + pa_paged_attn_decode_gqa ({gqa_kernel})" if gqa
+                            else "pa_kv_cache_write + pa_paged_attn_decode")},
         "decode_tokens_per_s": world * S / (ms_step * 1e-3),
         "pct_of_nominal_8tbs": 100.0 * (value / world) / NOMINAL_HBM_GBS,
         "kernel_ms": ({"pa_decode_step": decode_ms} if fused else
                       {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": None if gqa else traffic_per_launch(args.path),
+                     "traffic": traffic_per_launch(args.workload, args.path),
                      "kernel": ("pa_decode_step (decode kernel with the cache write, + merge kernel)"
                                 if fused else
-                                "pa_paged_attn_decode_gqa (decode kernel + merge kernel)" if gqa
+                                f"pa_paged_attn_decode_gqa ({gqa_kernel} decode kernel + merge kernel)" if gqa
                                 else "pa_paged_attn_decode (decode kernel + merge kernel)"),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": decode_bytes},
         "e2e": {"value": world * step_kv / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -388,7 +412,7 @@ def main():
         "gpu_launches": (2 if fused else 3) * K,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not gqa:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         w_cpu = w
         line["cpu_baseline"] = cpu_baseline(w_cpu)
     if rank == 0:

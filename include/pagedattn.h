@@ -201,7 +201,11 @@ size_t pa_paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int 
  *   other arguments, arithmetic, errors as for pa_paged_attn_decode.
  * num_kv_heads == num_heads is exactly pa_paged_attn_decode.  Each key/value
  * row is read from HBM once per (text, key/value head) and used by all the
- * query heads that share it.  num_heads must be a multiple of num_kv_heads
+ * query heads that share it (up to 16 per read; larger groups are split into
+ * equal subsets that each read the rows).  The tensor-core kernel (see
+ * PA_OPT_GQA_KERNEL) copies whole 16-token (32 at head_dim 64) runs of a
+ * block, so rows past L in a text's last block are read and ignored; they
+ * lie inside the pool, and their contents (NaN included) do not affect out.  num_heads must be a multiple of num_kv_heads
  * (else PA_ERR_INVALID).
  */
 int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -250,9 +254,20 @@ int pa_paged_attn_decode_noalloc(void* out, const void* q, const void* k_cache,
  *   PA_OPT_DECODE_WARPS   number of working warps of the decode kernel
  *                         (0 = all SMs, the default).  1 gives a single-pass
  *                         run in which no text is split.
- * Returns PA_OK or PA_ERR_INVALID for an unknown key.
+ *   PA_OPT_GQA_KERNEL     which kernel pa_paged_attn_decode_gqa runs when
+ *                         num_heads > num_kv_heads: 0 (default) the
+ *                         tensor-core kernel where it applies (block_size 8,
+ *                         16 or 32 and num_blocks * num_kv_heads * block_size
+ *                         < 2^31), else the CUDA-core one; 1 always the
+ *                         CUDA-core kernel; 2 always the tensor-core kernel
+ *                         (PA_ERR_INVALID where it does not apply).  Both
+ *                         compute the same function with fp32 sums; the
+ *                         tensor-core kernel carries the softmax weights into
+ *                         the weighted sum of values as the sum of two dt
+ *                         values (about 16 significant bits).
+ * Returns PA_OK or PA_ERR_INVALID for an unknown key or value.
  */
-enum { PA_OPT_WAIT_LIMIT_NS = 1, PA_OPT_DECODE_WARPS = 2 };
+enum { PA_OPT_WAIT_LIMIT_NS = 1, PA_OPT_DECODE_WARPS = 2, PA_OPT_GQA_KERNEL = 3 };
 int pa_set_option(int key, int64_t value);
 
 /* ------------------------------------------------------------------------ */

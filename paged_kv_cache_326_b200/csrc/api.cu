@@ -13,6 +13,7 @@ namespace {
 
 std::atomic<int64_t> g_wait_limit_ns{1000000000};
 std::atomic<int64_t> g_decode_warps{0};
+std::atomic<int64_t> g_gqa_kernel{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -31,6 +32,7 @@ int from_cuda(cudaError_t e) {
 
 namespace pa {
 int64_t option_decode_warps() { return g_decode_warps.load(); }
+int64_t option_gqa_kernel() { return g_gqa_kernel.load(); }
 }  // namespace pa
 
 extern "C" {
@@ -60,6 +62,10 @@ int pa_set_option(int key, int64_t value) {
     case PA_OPT_DECODE_WARPS:
       if (value < 0 || value > (int64_t{1} << 20)) return PA_ERR_INVALID;
       g_decode_warps = value;
+      return PA_OK;
+    case PA_OPT_GQA_KERNEL:
+      if (value < 0 || value > 2) return PA_ERR_INVALID;
+      g_gqa_kernel = value;
       return PA_OK;
     default: return PA_ERR_INVALID;
   }

@@ -49,6 +49,17 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
 
 // Current PA_OPT_DECODE_WARPS setting.
 int64_t option_decode_warps();
+// Current PA_OPT_GQA_KERNEL setting (0 automatic, 1 CUDA cores, 2 tensor cores).
+int64_t option_gqa_kernel();
+
+// Tensor-core grouped-query decode (paged_attn_decode_mma.cu): whether the
+// head layout and block size suit it, whether the pool fits its 32-bit TMA
+// row coordinates, its workspace size, and the launch.
+bool mma_decode_shape_ok(int num_heads, int num_kv_heads, int head_dim, int block_size);
+bool mma_decode_pool_ok(int num_kv_heads, int block_size, int64_t num_blocks);
+size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int max_blocks_per_seq, int64_t forced_warps);
+cudaError_t launch_paged_attn_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 
 // Launches the decode kernel and the split reduce on `stream`.
 // Returns cudaErrorInvalidValue for unsupported sizes or a short workspace.

@@ -603,13 +603,30 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
     if (pl.work_warps > warps) warps = pl.work_warps;
   }
   const int64_t segs = static_cast<int64_t>(num_seqs) * hl.vheads;
-  return header_bytes(num_seqs) + kGrabBytes + records_bytes(max_units(warps) + segs, head_dim, hl.gs);
+  size_t bytes =
+      header_bytes(num_seqs) + kGrabBytes + records_bytes(max_units(warps) + segs, head_dim, hl.gs);
+  // Grouped-query shapes may run on either kernel: size for both.
+  if (mma_decode_shape_ok(num_heads, num_kv_heads, head_dim, block_size)) {
+    const size_t mma = mma_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                  block_size, max_blocks_per_seq, forced_warps);
+    if (mma == 0) return 0;
+    if (mma > bytes) bytes = mma;
+  }
+  return bytes;
 }
 
 cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (!decode_sizes_supported(a.num_seqs, a.num_heads, a.num_kv_heads, a.head_dim, a.block_size,
                               a.max_blocks_per_seq))
     return cudaErrorInvalidValue;
+  // Grouped-query attention: tensor cores unless PA_OPT_GQA_KERNEL asks for
+  // the CUDA cores (or the shape or pool does not suit them).
+  const int64_t mode = option_gqa_kernel();
+  const bool mma_ok = !a.slot_mapping &&
+                      mma_decode_shape_ok(a.num_heads, a.num_kv_heads, a.head_dim, a.block_size) &&
+                      mma_decode_pool_ok(a.num_kv_heads, a.block_size, a.num_blocks);
+  if (mode == 2 && !mma_ok) return cudaErrorInvalidValue;
+  if (mma_ok && mode != 1) return launch_paged_attn_decode_mma(a, stream);
   const HeadLayout hl = head_layout(a.num_heads, a.num_kv_heads);
   return a.is_bf16 ? dispatch_heads<__nv_bfloat16>(a, hl, stream)
                    : dispatch_heads<__half>(a, hl, stream);

@@ -5,7 +5,10 @@
 
 For profilers: it makes no timing claims.  Workloads: ``opt13b_batch64``
 (optionally cut to the first S texts, pool sized 1.5x what they need),
-``tiny``, ``skewed`` (bf16, blocks of 16).
+``tiny``, ``skewed`` (bf16, blocks of 16), ``llama2_70b_gqa`` (64 query heads
+on 8 key/value heads; always the two-call path, the one-launch step being
+multi-head only).  ``--gqa-kernel`` picks its kernel (0 automatic, 1 CUDA
+cores, 2 tensor cores).
 """
 from __future__ import annotations
 
@@ -22,6 +25,8 @@ def make(name: str, num_seqs: int, device):
         return W.tiny(device=device)
     if name == "skewed":
         return W.skewed(device=device)
+    if name == "llama2_70b_gqa":
+        return W.llama2_70b_gqa(device=device, num_seqs=num_seqs if num_seqs > 0 else 64)
     if name == "opt13b_batch64":
         if num_seqs <= 0 or num_seqs >= 64:
             return W.opt13b_batch64(device=device)
@@ -39,13 +44,20 @@ def main():
     ap.add_argument("--num-seqs", type=int, default=0)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
+    ap.add_argument("--gqa-kernel", type=int, choices=[0, 1, 2], default=0)
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
     w = make(args.workload, args.num_seqs, dev)
+    gqa = w.k_cache.shape[1] != w.num_heads
+    P.pa_set_option(P.PA_OPT_GQA_KERNEL, args.gqa_kernel)
     out = torch.empty_like(w.q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     for _ in range(args.reps):
-        if args.path == "fused":
+        if gqa:
+            P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+            P.pa_paged_attn_decode_gqa(out, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                       w.context_lens, w.scale, status=status)
+        elif args.path == "fused":
             P.pa_decode_step(out, w.q, w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping,
                              w.block_tables, w.context_lens, w.scale, status=status)
         else:
@@ -55,7 +67,7 @@ def main():
     torch.cuda.synchronize()
     if status.item() != 0:
         raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
-    kv = sum(w.context_lens.tolist()) * 2 * w.num_heads * w.head_dim * w.q.element_size()
+    kv = sum(w.context_lens.tolist()) * 2 * w.k_cache.shape[1] * w.head_dim * w.q.element_size()
     print(f"{w.name}: {w.num_seqs} texts, KV bytes per step {kv}, status ok")
 
 

@@ -368,38 +368,65 @@ def gpu_step_gqa(w, status=None, out=None):
 
 
 GQA_LENS = [0, 1, 17, 100, 300, 1000, 2048, 33]
+# PA_OPT_GQA_KERNEL values: the tensor-core kernel, the CUDA-core kernel.
+GQA_KERNELS = {"tensor": 2, "cores": 1}
 
 
-@pytest.mark.parametrize("heads", [(16, 8), (12, 4), (32, 8), (64, 8), (16, 1), (8, 8)],
+@pytest.fixture(params=list(GQA_KERNELS))
+def gqa_kernel(request):
+    """Run the test once on each grouped-query kernel."""
+    import paged_kv_cache_326_b200 as P
+    P.pa_set_option(P.PA_OPT_GQA_KERNEL, GQA_KERNELS[request.param])
+    yield request.param
+    P.pa_set_option(P.PA_OPT_GQA_KERNEL, 0)
+
+
+def _tensor_applies(Hq, Hkv, block_size):
+    return Hq != Hkv and block_size >= 8
+
+
+@pytest.mark.parametrize("heads", [(16, 8), (12, 4), (6, 2), (40, 8), (32, 8), (64, 8),
+                                   (48, 2), (16, 1), (64, 1), (8, 8)],
                          ids=lambda hk: f"q{hk[0]}kv{hk[1]}")
-def test_gqa_group_sizes(heads):
+def test_gqa_group_sizes(heads, gqa_kernel):
+    """Group sizes 2 to 64: whole column tiles (8, 16), padded ones (3, 5, 6),
+    groups split into subsets (24, 32, 64), and plain multi-head (8, 8)."""
     Hq, Hkv = heads
+    if gqa_kernel == "tensor" and not _tensor_applies(Hq, Hkv, 16):
+        pytest.skip("multi-head attention runs on the CUDA-core kernel")
     w = W.make_decode("gqa", GQA_LENS, num_heads=Hq, head_dim=128, block_size=16,
                       num_blocks=2 * sum(W.blocks_needed(L, 16) for L in GQA_LENS),
                       dtype=torch.float16, seed=Hq + Hkv, device="cuda",
                       max_blocks_per_seq=2048 // 16, num_kv_heads=Hkv)
     c = parity(w, check_pool=True, step=gpu_step_gqa)
-    print(f"gqa q{Hq} kv{Hkv}", c)
+    print(f"gqa {gqa_kernel} q{Hq} kv{Hkv}", c)
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
-@pytest.mark.parametrize("block_size", [4, 32])
-def test_gqa_head_dim_64(dtype, block_size):
-    w = W.make_decode("gqa64", SHAPE_LENS, num_heads=32, head_dim=64, block_size=block_size,
+@pytest.mark.parametrize("head_dim", [64, 128])
+@pytest.mark.parametrize("block_size", [4, 8, 16, 32])
+def test_gqa_every_shape_ragged(dtype, head_dim, block_size, gqa_kernel):
+    """Every head_dim x block size x dtype, ragged lengths (partial chunks and
+    partial blocks, whose unwritten rows hold NaN), 16 query heads on 4
+    key/value heads."""
+    if gqa_kernel == "tensor" and not _tensor_applies(16, 4, block_size):
+        pytest.skip("blocks of 4 run on the CUDA-core kernel")
+    w = W.make_decode("gqa_shape", SHAPE_LENS, num_heads=16, head_dim=head_dim,
+                      block_size=block_size,
                       num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in SHAPE_LENS),
-                      dtype=dtype, seed=block_size, device="cuda",
-                      max_blocks_per_seq=160 // block_size, num_kv_heads=8)
+                      dtype=dtype, seed=head_dim + block_size, device="cuda",
+                      max_blocks_per_seq=160 // block_size, num_kv_heads=4)
     parity(w, check_pool=True, step=gpu_step_gqa)
 
 
-def test_gqa_llama2_70b_shape():
+def test_gqa_llama2_70b_shape(gqa_kernel):
     w = W.llama2_70b_gqa(device="cuda")
     c = parity(w, heads_per_seq=8, seed=6, step=gpu_step_gqa)
-    print("gqa llama2_70b", c)
+    print(f"gqa {gqa_kernel} llama2_70b", c)
 
 
 @pytest.mark.parametrize("warps", [1, 4096])
-def test_gqa_split_and_single_pass(warps):
+def test_gqa_split_and_single_pass(warps, gqa_kernel):
     import paged_kv_cache_326_b200 as P
     w = W.make_decode("gqa_split", [300, 17, 1, 1000, 0, 511], num_heads=32, head_dim=128,
                       block_size=16, num_blocks=256, dtype=torch.bfloat16, seed=11, device="cuda",
@@ -409,3 +436,82 @@ def test_gqa_split_and_single_pass(warps):
         parity(w, step=gpu_step_gqa)
     finally:
         P.pa_set_option(P.binding.PA_OPT_DECODE_WARPS, 0)
+
+
+def test_gqa_single_token_returns_its_value(gqa_kernel):
+    """One stored token: softmax weight 1, so every query head of a group gets
+    its key/value head's value (the tensor-core kernel rounds the weight 1.0
+    to fp16 exactly, so this stays bit-exact)."""
+    w = W.make_decode("gqa_one", [1] * 5, num_heads=16, head_dim=128, block_size=16,
+                      num_blocks=8, dtype=torch.float16, seed=13, device="cuda", num_kv_heads=2)
+    out = gpu_step_gqa(w)
+    torch.cuda.synchronize()
+    assert torch.equal(out, w.v.repeat_interleave(8, dim=1))
+
+
+def test_gqa_kernels_agree_and_are_deterministic():
+    """Both kernels compute the same function: equal within the tolerance;
+    each is bitwise reproducible run to run."""
+    import paged_kv_cache_326_b200 as P
+    w = W.llama2_70b_gqa(device="cuda", num_seqs=16)
+    P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping)
+    res = {}
+    try:
+        for name, mode in GQA_KERNELS.items():
+            P.pa_set_option(P.PA_OPT_GQA_KERNEL, mode)
+            outs = []
+            for _ in range(2):
+                out = torch.empty_like(w.q)
+                P.pa_paged_attn_decode_gqa(out, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                           w.context_lens, w.scale)
+                outs.append(out)
+            torch.cuda.synchronize()
+            assert torch.equal(outs[0], outs[1]), name
+            res[name] = outs[0]
+    finally:
+        P.pa_set_option(P.PA_OPT_GQA_KERNEL, 0)
+    diff = (res["tensor"].float() - res["cores"].float()).abs()
+    assert diff.max().item() <= 4e-3, diff.max().item()
+
+
+def test_gqa_tensor_kernel_refuses_shapes_it_does_not_cover():
+    import paged_kv_cache_326_b200 as P
+    w = W.make_decode("gqa_b4", [5, 9], num_heads=8, head_dim=64, block_size=4, num_blocks=16,
+                      dtype=torch.float16, seed=3, device="cuda", num_kv_heads=2)
+    out = torch.empty_like(w.q)
+    P.pa_set_option(P.PA_OPT_GQA_KERNEL, 2)
+    try:
+        with pytest.raises(P.PagedAttnError):
+            P.pa_paged_attn_decode_gqa(out, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                       w.context_lens, w.scale)
+    finally:
+        P.pa_set_option(P.PA_OPT_GQA_KERNEL, 0)
+
+
+def test_gqa_bad_block_and_timeout_are_reported(gqa_kernel):
+    """A table entry outside the pool and a wait that gives up are recorded
+    in the status word; the kernel skips the block / returns, and the next
+    call is correct."""
+    import paged_kv_cache_326_b200 as P
+    mk = lambda: W.make_decode("gqa_err", [40, 17, 100], num_heads=16, head_dim=128,
+                               block_size=16, num_blocks=32, dtype=torch.float16, seed=5,
+                               device="cuda", num_kv_heads=2)
+    w = mk()
+    w.block_tables[2, 1] = w.num_blocks + 3
+    st = new_status()
+    gpu_step_gqa(w, st)
+    torch.cuda.synchronize()
+    assert st.item() == P.binding.PA_ERR_BAD_BLOCK
+    w = mk()
+    P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping)
+    st = new_status()
+    P.pa_set_option(P.binding.PA_OPT_WAIT_LIMIT_NS, -1)
+    try:
+        out = torch.empty_like(w.q)
+        P.pa_paged_attn_decode_gqa(out, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                   w.context_lens, w.scale, status=st)
+        torch.cuda.synchronize()
+    finally:
+        P.pa_set_option(P.binding.PA_OPT_WAIT_LIMIT_NS, 1_000_000_000)
+    assert st.item() == P.binding.PA_ERR_TIMEOUT
+    parity(mk(), step=gpu_step_gqa)
