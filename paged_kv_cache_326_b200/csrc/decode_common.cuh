@@ -434,7 +434,8 @@ __device__ __forceinline__ void merge_partials(const float* records, int64_t rec
 // query heads; the decode kernel has already written every other output.
 // Launched right after the decode kernel with programmatic dependent launch:
 // its CTAs become resident early and griddepcontrol.wait holds them until the
-// decode kernel's writes are visible.  One warp per (text, virtual head).
+// decode kernel's writes are visible.  One warp per (text, virtual head,
+// query head of the subset).
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
@@ -442,8 +443,10 @@ split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
                     int num_q_heads, int nsub, int gs) {
   griddep_wait();
   const int lane = threadIdx.x & 31;
-  const int seg = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (seg >= num_seqs * num_vheads) return;
+  const int item = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (item >= num_seqs * num_vheads * gs) return;
+  const int seg = item / gs;
+  const int g = item - seg * gs;
   const int s = seg / num_vheads;
   const int vh = seg - s * num_vheads;
   WorkSplit sp;
@@ -461,12 +464,10 @@ split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
   const int u_hi = sp.unit_of(a + ns - 1);
   if (u_lo == u_hi) return;  // finished in place by the decode kernel
   const int group = num_q_heads / (num_vheads / nsub);  // query heads per key/value head
-  const int qh0 = (vh / nsub) * group + (vh % nsub) * gs;
-#pragma unroll 1
-  for (int g = 0; g < gs; ++g)
-    merge_partials<T, D>(records + g * (D + 4), static_cast<int64_t>(gs) * (D + 4),
-                         out + (static_cast<int64_t>(s) * num_q_heads + qh0 + g) * D, seg, u_lo,
-                         u_hi, lane);
+  const int qh = (vh / nsub) * group + (vh % nsub) * gs + g;
+  merge_partials<T, D>(records + g * (D + 4), static_cast<int64_t>(gs) * (D + 4),
+                       out + (static_cast<int64_t>(s) * num_q_heads + qh) * D, seg, u_lo, u_hi,
+                       lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -563,10 +564,10 @@ inline Plan plan_decode(const void* kernel, size_t smem, size_t smem_max, int wa
 // launch on the same stream).
 template <typename T, int D>
 cudaError_t launch_merge(const DecodeParams& p, int gs, cudaStream_t stream) {
-  const int64_t segs = static_cast<int64_t>(p.num_seqs) * p.num_heads;
-  const int per_cta = 8;  // warps, one per (text, virtual head)
+  const int64_t items = static_cast<int64_t>(p.num_seqs) * p.num_heads * gs;
+  const int per_cta = 8;  // warps, one per (text, virtual head, query head of the subset)
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((segs + per_cta - 1) / per_cta));
+  cfg.gridDim = dim3(static_cast<unsigned>((items + per_cta - 1) / per_cta));
   cfg.blockDim = dim3(per_cta * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;

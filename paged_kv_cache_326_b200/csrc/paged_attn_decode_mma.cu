@@ -101,8 +101,10 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
 
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, NSUB = p.nsub, GS = p.gs;
   const int G = Hq / Hkv;
-  auto kv_head = [&](int vh) { return vh / NSUB; };
-  auto q_head0 = [&](int vh) { return (vh / NSUB) * G + (vh % NSUB) * GS; };
+  // virtual head -> key/value head and first query head (one subset per
+  // key/value head, the usual case, needs no division)
+  auto kv_head = [&](int vh) { return NSUB == 1 ? vh : vh / NSUB; };
+  auto q_head0 = [&](int vh) { return NSUB == 1 ? vh * G : (vh / NSUB) * G + (vh % NSUB) * GS; };
   const int cap = p.max_blocks_per_seq * B;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -401,8 +403,9 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
     const int tq = (lane & 3) * 2;
 #pragma unroll
     for (int mt = 0; mt < TM; ++mt) {
+      const bool tail = nvalid < (mt + 1) * 16;  // warp-uniform
       uint32_t mask_lo = 0xffffffffu, mask_hi = 0xffffffffu;
-      if (nvalid < (mt + 1) * 16) {
+      if (tail) {
         const int t0 = mt * 16 + tq;
         mask_lo = (t0 < nvalid ? 0x0000ffffu : 0u) | (t0 + 1 < nvalid ? 0xffff0000u : 0u);
         mask_hi = (t0 + 8 < nvalid ? 0x0000ffffu : 0u) | (t0 + 9 < nvalid ? 0xffff0000u : 0u);
@@ -412,10 +415,12 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
         uint32_t a[4];
         ldsm_x4_trans(swz<CH>(sV, mt * 16 + (lane >> 4) * 8 + (lane & 7), md * 16 + ((lane >> 3) & 1) * 8),
                       a);
-        a[0] &= mask_lo;
-        a[1] &= mask_lo;
-        a[2] &= mask_hi;
-        a[3] &= mask_hi;
+        if (tail) {
+          a[0] &= mask_lo;
+          a[1] &= mask_lo;
+          a[2] &= mask_hi;
+          a[3] &= mask_hi;
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_16816<T>(o[md][nt], a, pb[mt][nt][0], pb[mt][nt][1]);
