@@ -6,9 +6,9 @@ check in ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may
 import, call or run anything in this folder.  It shares no code with the CUDA
 path and never imports the product package.
 """
-from .paged_attention import (attend, cache_write, decode_step, gather_context, kv_head_of,
-                              paged_decode)
+from .paged_attention import (attend, cache_write, copy_blocks, decode_step, gather_context,
+                              kv_head_of, paged_decode)
 from .block_manager import BlockManagerError, BlockManagerModel
 
-__all__ = ["attend", "cache_write", "decode_step", "gather_context", "kv_head_of", "paged_decode",
+__all__ = ["attend", "cache_write", "copy_blocks", "decode_step", "gather_context", "kv_head_of", "paged_decode",
            "BlockManagerError", "BlockManagerModel"]

@@ -33,6 +33,12 @@ Precision: inputs are the exact fp16/bf16 values widened to fp64; every step
 is fp64; softmax subtracts the maximum before exponentiating (an identity, so
 the result is the same number up to rounding).
 
+Block copies (``copy_blocks``): whole blocks copied from a source pool to a
+destination pool ("The KV Cache and PagedAttention", §Shared, Copied on
+Write: a text about to write into a block it shares gets its own copy of the
+block first; §When Memory Runs Out: blocks are moved out of the pool to CPU
+memory and back).
+
 Pinned by tests/test_oracle.py against: torch's fp64 attention on unpaged
 contiguous tensors, scalar brute force with ``math.fsum`` on tiny inputs,
 closed forms (one token gives its value; equal scores give the mean of the
@@ -40,7 +46,11 @@ values; one dominant score gives its value), bit-identity under a relabelling
 of physical blocks, under a change of block size, and for texts that share
 prefix blocks, and a hand-worked cache write; grouped-query attention against
 the same pool with key/value heads replicated per query head, torch's fp64
-attention on repeated heads, and brute force for one shared head.
+attention on repeated heads, and brute force for one shared head; block
+copies against the worked copy-on-write example of the pages (each answer
+reads the prompt plus its own token and nothing of the other's), torch's
+index_copy_ on raw bit patterns, and a copy out and back that restores every
+block.
 """
 from __future__ import annotations
 
@@ -68,6 +78,21 @@ def cache_write(k_cache: np.ndarray, v_cache: np.ndarray, k: np.ndarray, v: np.n
         kc[block, :, place, :] = k[t]
         vc[block, :, place, :] = v[t]
     return kc, vc
+
+
+def copy_blocks(src_k: np.ndarray, src_v: np.ndarray, dst_k: np.ndarray, dst_v: np.ndarray,
+                pairs: Sequence[Tuple[int, int]]) -> Tuple[np.ndarray, np.ndarray]:
+    """Return copies of the destination pools in which, for every pair
+    (src, dst), block dst holds block src of the source pools: every head,
+    every place, every bit.  Every pair reads the source pools as they were
+    before the call (the source arrays are never written, even when they are
+    the destination arrays too).  Pools are ``[N][H][B][D]`` of any dtype."""
+    kd = dst_k.copy()
+    vd = dst_v.copy()
+    for src, dst in pairs:
+        kd[int(dst)] = src_k[int(src)]
+        vd[int(dst)] = src_v[int(src)]
+    return kd, vd
 
 
 def gather_context(cache: np.ndarray, block_table: Sequence[int], context_len: int,

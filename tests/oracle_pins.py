@@ -341,3 +341,92 @@ def pin_mqa_single_head(fn):
 
 
 GQA_PINS = [pin_gqa_equals_replicated_mha, pin_gqa_unpaged_sdpa, pin_mqa_single_head]
+
+
+# ---------------------------------------------------------------------------
+# block copies (copy-on-write, moving blocks between pools)
+# ---------------------------------------------------------------------------
+
+def pin_copy_on_write_worked_example(copy_fn):
+    """The pages' worked example ("The KV Cache and PagedAttention", Shared,
+    Copied on Write; golden cow_two_answers.json): two answers share a
+    6-token prompt in blocks 0 and 1 of 4 places; the first answer's write
+    copies block 1 to block 2 and lands at slot 10, the second writes in
+    place at slot 6.  Afterwards each answer reads the prompt followed by its
+    own token, and neither sees the other's."""
+    g = load_golden("cow_two_answers.json")
+    B, N, P = g["block_size"], g["num_blocks"], g["prompt_tokens"]
+    H, D = 2, 8
+    rng = np.random.default_rng(301)
+    prompt = rng.standard_normal((P, H, D))
+    tok = rng.standard_normal((2, H, D))          # each answer's new key (values alike)
+    kc = np.full((N, H, B, D), np.nan)
+    for t in range(P):                            # the prompt in blocks 0, 1 (in order)
+        kc[t // B, :, t % B] = prompt[t]
+    vc = kc.copy()
+    a1 = g["answer1_append"]
+    kc, vc = copy_fn(kc, vc, kc, vc, [(a1["cow_src"], a1["cow_dst"])])
+    kc, vc = cache_write_plain(kc, vc, tok[0:1], tok[0:1], [a1["slot"]], B)
+    a2 = g["answer2_append"]
+    assert a2["cow_src"] < 0
+    kc, vc = cache_write_plain(kc, vc, tok[1:2], tok[1:2], [a2["slot"]], B)
+    for i, name in enumerate(["answer1", "answer2"]):
+        table = g["after_answer2"]["tables"][name]
+        got = np.stack([kc[table[t // B], :, t % B] for t in range(P + 1)])
+        want = np.concatenate([prompt, tok[i:i + 1]])
+        assert np.array_equal(got, want), f"{name} does not read the prompt plus its own token"
+
+
+def cache_write_plain(kc, vc, k, v, slots, B):
+    """A write done here, by plain indexing (the pin must not lean on the
+    oracle's own cache_write)."""
+    kc, vc = kc.copy(), vc.copy()
+    for t, slot in enumerate(slots):
+        kc[slot // B, :, slot % B] = k[t]
+        vc[slot // B, :, slot % B] = v[t]
+    return kc, vc
+
+
+def pin_copy_blocks_bits_vs_index_copy(copy_fn):
+    """Raw 16-bit patterns (NaN payloads and signed zeros included) land
+    unchanged: the result equals torch's index_copy_ of the chosen source
+    blocks into the destination pool."""
+    rng = np.random.default_rng(311)
+    shape_s, shape_d = (12, 3, 4, 8), (9, 3, 4, 8)
+    src_k = rng.integers(0, 1 << 16, size=shape_s, dtype=np.uint16)
+    src_v = rng.integers(0, 1 << 16, size=shape_s, dtype=np.uint16)
+    src_k[0, 0, 0, :3] = [0x7E01, 0x8000, 0xFC00]
+    dst_k = rng.integers(0, 1 << 16, size=shape_d, dtype=np.uint16)
+    dst_v = rng.integers(0, 1 << 16, size=shape_d, dtype=np.uint16)
+    pairs = [(0, 4), (11, 0), (5, 8), (5, 2)]
+    before = dst_k.copy()
+    kd, vd = copy_fn(src_k, src_v, dst_k, dst_v, pairs)
+    idx_s = torch.tensor([p[0] for p in pairs])
+    idx_d = torch.tensor([p[1] for p in pairs])
+    for got, src, dst in ((kd, src_k, dst_k), (vd, src_v, dst_v)):
+        s16, d16 = torch.from_numpy(src.view(np.int16)), torch.from_numpy(dst.view(np.int16))
+        ref = d16.clone().index_copy_(0, idx_d, s16.index_select(0, idx_s)).numpy()
+        assert np.array_equal(got.view(np.int16), ref), "block copy differs from index_copy_"
+    assert np.array_equal(dst_k, before), "copy modified its input"
+
+
+def pin_copy_out_and_back(copy_fn):
+    """Moving blocks out to another pool and back into new places (a swap
+    out and in) restores every value, and blocks not named stay as they were."""
+    rng = np.random.default_rng(321)
+    kc = rng.standard_normal((10, 2, 4, 8))
+    vc = rng.standard_normal((10, 2, 4, 8))
+    host_k = np.zeros((3, 2, 4, 8))
+    host_v = np.zeros((3, 2, 4, 8))
+    out_pairs = [(7, 0), (2, 1), (9, 2)]
+    hk, hv = copy_fn(kc, vc, host_k, host_v, out_pairs)
+    back_pairs = [(0, 3), (1, 5), (2, 6)]
+    kc2, vc2 = copy_fn(hk, hv, kc, vc, back_pairs)
+    for (src, _), (_, dst) in zip(out_pairs, back_pairs):
+        assert np.array_equal(kc2[dst], kc[src]) and np.array_equal(vc2[dst], vc[src])
+    untouched = [b for b in range(10) if b not in (3, 5, 6)]
+    assert np.array_equal(kc2[untouched], kc[untouched]) and np.array_equal(vc2[untouched], vc[untouched])
+
+
+COPY_PINS = [pin_copy_on_write_worked_example, pin_copy_blocks_bits_vs_index_copy,
+             pin_copy_out_and_back]

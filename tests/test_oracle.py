@@ -17,6 +17,11 @@ def test_write_pin(pin):
     pin(oracle.cache_write)
 
 
+@pytest.mark.parametrize("pin", P.COPY_PINS, ids=lambda f: f.__name__)
+def test_copy_pin(pin):
+    pin(oracle.copy_blocks)
+
+
 def test_step_writes_before_attending():
     """The token written in this step is one of the keys the query attends to
     ("KV cache", How it works: the stored keys plus the new key)."""

@@ -170,3 +170,56 @@ def test_planted_gqa_head_mapping_mistake_is_caught():
 def test_unmodified_oracle_passes_gqa_pins():
     for pin in P.GQA_PINS:
         pin(oracle.paged_decode)
+
+
+# --- block copies: planted mistakes -------------------------------------------
+
+def copy_swaps_src_and_dst(sk, sv, dk, dv, pairs):
+    return oracle.copy_blocks(sk, sv, dk, dv, [(d, s) for s, d in pairs])
+
+
+def copy_k_into_v(sk, sv, dk, dv, pairs):
+    return oracle.copy_blocks(sk, sk, dk, dv, pairs)
+
+
+def copy_first_head_only(sk, sv, dk, dv, pairs):
+    kd, vd = dk.copy(), dv.copy()
+    for s, d in pairs:
+        kd[d, 0] = sk[s, 0]
+        vd[d, 0] = sv[s, 0]
+    return kd, vd
+
+
+def copy_misses_last_place(sk, sv, dk, dv, pairs):
+    kd, vd = dk.copy(), dv.copy()
+    for s, d in pairs:
+        kd[d, :, :-1] = sk[s, :, :-1]
+        vd[d, :, :-1] = sv[s, :, :-1]
+    return kd, vd
+
+
+def copy_in_place_sequentially(sk, sv, dk, dv, pairs):
+    """Writes into the source arrays themselves (a later pair may then read
+    an earlier pair's result)."""
+    for s, d in pairs:
+        dk[d] = sk[s]
+        dv[d] = sv[s]
+    return dk, dv
+
+
+@pytest.mark.parametrize("fn", [copy_swaps_src_and_dst, copy_k_into_v, copy_first_head_only,
+                                copy_misses_last_place, copy_in_place_sequentially],
+                         ids=lambda f: f.__name__)
+def test_planted_copy_mistake_is_caught(fn):
+    failed = 0
+    for pin in P.COPY_PINS:
+        try:
+            pin(fn)
+        except (AssertionError, IndexError):
+            failed += 1
+    assert failed, fn.__name__
+
+
+def test_unmodified_oracle_passes_copy_pins():
+    for pin in P.COPY_PINS:
+        pin(oracle.copy_blocks)
