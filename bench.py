@@ -232,6 +232,120 @@ def run_reference(args, world, rank):
     return 0
 
 
+def run_cow_copy(args, ranks, world, rank, local):
+    """Copy-on-write bursts: each step copies one burst of 224 whole blocks
+    (32 prompts x 7 samples, 40 heads x 16 x 128 fp16, K and V) with
+    pa_copy_blocks; bursts rotate over 8 disjoint sets of blocks."""
+    import numpy as np
+    import paged_kv_cache_326_b200 as P
+    from paged_kv_cache_326_b200 import dist, workloads as W
+    P.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    kc, vc, bursts = W.cow_bursts(seed=dist.batch_seed(4, ranks), device=dev)
+    N, H, B, D = kc.shape
+    block_bytes = H * B * D * kc.element_size()
+    n = bursts[0].shape[0]
+    # Least DRAM traffic a burst needs: each distinct source block read once
+    # (its 7 copies share one read), each destination written once; K and V.
+    uniq_src = bursts[0][:, 0].unique().numel()
+    step_bytes = (uniq_src + n) * 2 * block_bytes
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(i):
+        P.pa_copy_blocks(kc, vc, kc, vc, bursts[i % len(bursts)], status=status)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        dist.barrier(ranks)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier(ranks)
+    clk = clocks.summary()
+    ms_step = start.elapsed_time(stop) / K
+    kernel_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+
+    # end to end: each step's pairs uploaded from pinned host memory, the
+    # status word read back
+    hpairs = [b.cpu().pin_memory() for b in bursts]
+    dpairs = torch.empty_like(bursts[0])
+    hstat = torch.zeros(1, dtype=torch.int32).pin_memory()
+    Ke = max(1, K // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(Ke):
+        dpairs.copy_(hpairs[i % len(hpairs)], non_blocking=True)
+        P.pa_copy_blocks(kc, vc, kc, vc, dpairs, status=status)
+        hstat.copy_(status, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    ms_step, e2e_ms, kernel_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms, kernel_ms], dev)
+    peak, peak_src = hbm_peak()
+    achieved = step_bytes / (kernel_ms * 1e-3) / 1e9
+    line = {
+        "metric": "paged block copy GB/s (distinct blocks read + blocks written)",
+        "value": world * step_bytes / (ms_step * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": "cow_copy", "pairs_per_step": n, "num_heads": H,
+                   "block_size": B, "head_dim": D, "block_bytes": block_bytes,
+                   "num_blocks": N, "bursts": len(bursts),
+                   "l2": f"{len(bursts)} disjoint bursts in rotation "
+                         f"({len(bursts) * step_bytes / 1e9:.2f} GB of blocks >> 126 MB L2)",
+                   "parallelism": f"independent pool per GPU x{world}"},
+        "kernel_ms": {"copy_blocks": kernel_ms},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "copy_blocks_kernel",
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": step_bytes},
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": dpairs.numel() * 4, "d2h_bytes_per_step": 4,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        pairs = bursts[0].cpu().numpy()
+        used = np.unique(pairs)
+        remap = {int(b): i for i, b in enumerate(used)}
+        local_pairs = [(remap[int(a)], remap[int(b)]) for a, b in pairs]
+        sk = kc[torch.as_tensor(used, device=dev)].cpu().numpy()
+        sv = vc[torch.as_tensor(used, device=dev)].cpu().numpy()
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.copy_blocks(sk, sv, sk, sv, local_pairs)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= 10.0 or reps >= 200:
+                break
+        line["cpu_baseline"] = {
+            "value": step_bytes * reps / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"burst 0 ({n} pairs) on a host pool of the {len(used)} blocks it names, "
+                      f"{reps} run(s), {el:.1f} s, numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -242,9 +356,10 @@ def main():
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
     ap.add_argument("--gqa-kernel", choices=["auto", "cores", "tensor"], default="auto",
                     help="grouped-query workload: kernel choice (PA_OPT_GQA_KERNEL)")
-    ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa"],
+    ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa", "cow_copy"],
                     default="opt13b_batch64",
-                    help="llama2_70b_gqa: 64 query heads on 8 key/value heads (two calls)")
+                    help="llama2_70b_gqa: 64 query heads on 8 key/value heads (two calls); "
+                         "cow_copy: copy-on-write bursts of whole blocks (pa_copy_blocks)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -253,6 +368,11 @@ def main():
     world, rank, local = ranks.world, ranks.rank, ranks.local
     if args.impl == "reference":
         rc = run_reference(args, world, rank)
+        dist.finish(ranks)
+        return rc
+
+    if args.workload == "cow_copy":
+        rc = run_cow_copy(args, ranks, world, rank, local)
         dist.finish(ranks)
         return rc
 

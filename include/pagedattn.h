@@ -216,6 +216,38 @@ int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, cons
                              size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
 
 /*
+ * pa_copy_blocks — copy whole blocks from one pool to another, or within one
+ * pool: the device side of copy-on-write ("The KV Cache and
+ * PagedAttention", section "Shared, Copied on Write": before a text writes
+ * into a block it shares, the block is copied to a free one, the text writes
+ * into the copy and the original's count drops by one; pa_bm_append_slot
+ * returns the pair) and of moving blocks out of the pool and back (section
+ * "When Memory Runs Out": blocks set aside in CPU memory).
+ *
+ *   src_k, src_v   [src_num_blocks][num_heads][block_size][head_dim] dt
+ *   dst_k, dst_v   [dst_num_blocks][num_heads][block_size][head_dim] dt; may
+ *                  be src_k, src_v (copy-on-write)
+ *   block_pairs    [num_pairs][2] int32: (source block, destination block)
+ * For every pair, destination block dst of both pools receives source block
+ * src: every head and place, bit for bit (a pure copy).  Every pair reads
+ * the sources as they were before the call, so no block may be the
+ * destination of two pairs, nor a destination and a source in one call (the
+ * block manager's pairs never are); otherwise the result is unspecified.
+ * Pools and block_pairs may be device memory of the current device, managed
+ * memory, or pinned host memory mapped at the same address (e.g. a CPU
+ * pool for blocks moved out); anything else is PA_ERR_INVALID, checked on the
+ * host before launch.  A block id outside its pool is recorded as
+ * PA_ERR_BAD_BLOCK in *d_status and that pair is skipped.  num_pairs == 0 is
+ * a no-op.  Launched with programmatic dependent launch: it waits for the
+ * kernel before it on the stream, and the next kernel waits for it.
+ * Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks, void* dst_k,
+                   void* dst_v, int64_t dst_num_blocks, const int32_t* block_pairs,
+                   int num_pairs, int num_heads, int head_dim, int block_size, pa_dtype dt,
+                   int32_t* d_status, pa_stream_t stream);
+
+/*
  * pa_paged_attn_decode_noalloc — pa_paged_attn_decode without a caller
  * workspace, for callers that cannot allocate device memory (a host framework
  * that owns every device allocation, a fixed memory budget, a loop where an

@@ -72,6 +72,8 @@ _SIGNATURES = {
                               _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_paged_attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
                                             _i32, _i32, _i64, _i32, _vp, _vp]),
+    "pa_copy_blocks": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32,
+                              _vp, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_i32, [_vp, _i64, _i32]),
@@ -164,6 +166,41 @@ def pa_kv_cache_write(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
         _cuda(slot_mapping, "slot_mapping", torch.int64), T, H, D, B, N, _dtype_code(k),
         _status_ptr(status), _stream(stream, k.device))
     _check(code, "pa_kv_cache_write")
+
+
+def _pool(t: torch.Tensor, name: str) -> int:
+    """A pool the GPU can address: a CUDA tensor, or a pinned CPU tensor (the
+    library checks the mapping before launch)."""
+    if not isinstance(t, torch.Tensor) or not (t.is_cuda or t.is_pinned()):
+        raise TypeError(f"{name} must be a CUDA tensor or a pinned CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def pa_copy_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor,
+                   dst_v: torch.Tensor, block_pairs: torch.Tensor,
+                   status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Pools [N][H][B][D] (source and destination may differ in N, or be the
+    same tensors); block_pairs [n][2] int32 (source block, destination
+    block), on the GPU."""
+    Ns, H, B, D = src_k.shape
+    Nd = dst_k.shape[0]
+    if (src_v.shape != src_k.shape or dst_k.shape[1:] != src_k.shape[1:] or
+            dst_v.shape != dst_k.shape):
+        raise ValueError("pool shapes differ")
+    if block_pairs.dim() != 2 or block_pairs.shape[1] != 2:
+        raise ValueError("block_pairs must be [n][2]")
+    for t in (src_v, dst_k, dst_v):
+        if t.dtype != src_k.dtype:
+            raise TypeError("pools must share a dtype")
+    dev = block_pairs.device
+    code = lib().pa_copy_blocks(
+        _pool(src_k, "src_k"), _pool(src_v, "src_v"), Ns, _pool(dst_k, "dst_k"),
+        _pool(dst_v, "dst_v"), Nd, _cuda(block_pairs, "block_pairs", torch.int32),
+        block_pairs.shape[0], H, D, B, _dtype_code(src_k), _status_ptr(status),
+        _stream(stream, dev))
+    _check(code, "pa_copy_blocks")
 
 
 def pa_paged_attn_decode_workspace_size(num_seqs: int, num_heads: int, head_dim: int,

@@ -22,6 +22,23 @@ bool shape_ok(int num_heads, int head_dim, int block_size) {
          (block_size == 4 || block_size == 8 || block_size == 16 || block_size == 32);
 }
 
+// Memory the current device can read and write at this address: its own
+// device memory, managed memory, or pinned host memory mapped at the same
+// address (unified addressing).
+bool device_accessible(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (a.type == cudaMemoryTypeDevice) return a.device == dev;
+  if (a.type == cudaMemoryTypeManaged) return true;
+  if (a.type == cudaMemoryTypeHost) return a.devicePointer == p;
+  return false;
+}
+
 int from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return PA_OK;
   if (e == cudaErrorInvalidValue) return PA_ERR_INVALID;
@@ -163,6 +180,27 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
   return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
                        num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
                        dt, workspace, workspace_bytes, d_status, stream, nullptr, nullptr, nullptr);
+}
+
+int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks, void* dst_k,
+                   void* dst_v, int64_t dst_num_blocks, const int32_t* block_pairs,
+                   int num_pairs, int num_heads, int head_dim, int block_size, pa_dtype dt,
+                   int32_t* d_status, pa_stream_t stream) {
+  if (num_pairs < 0 || !shape_ok(num_heads, head_dim, block_size) || src_num_blocks <= 0 ||
+      dst_num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16))
+    return PA_ERR_INVALID;
+  if (num_pairs == 0) return PA_OK;
+  if (!src_k || !src_v || !dst_k || !dst_v || !block_pairs) return PA_ERR_INVALID;
+  if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v) ||
+      (reinterpret_cast<uintptr_t>(block_pairs) & 3u) != 0)
+    return PA_ERR_INVALID;
+  if (!device_accessible(src_k) || !device_accessible(src_v) || !device_accessible(dst_k) ||
+      !device_accessible(dst_v) || !device_accessible(block_pairs))
+    return PA_ERR_INVALID;
+  const int64_t block_bytes = static_cast<int64_t>(num_heads) * block_size * head_dim * 2;
+  return from_cuda(pa::launch_copy_blocks(src_k, src_v, dst_k, dst_v, block_pairs, num_pairs,
+                                          block_bytes, src_num_blocks, dst_num_blocks, d_status,
+                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -12,6 +12,14 @@ cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, v
                                   int head_dim, int block_size, int64_t num_blocks,
                                   int32_t* status, cudaStream_t stream);
 
+// Whole-block copies: for each (src, dst) in pairs[num_pairs][2], block dst of
+// the destination K and V pools receives block src of the source pools
+// (block_bytes each).  Ids outside their pool: PA_ERR_BAD_BLOCK, skipped.
+cudaError_t launch_copy_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                               const int32_t* pairs, int num_pairs, int64_t block_bytes,
+                               int64_t src_num_blocks, int64_t dst_num_blocks, int32_t* status,
+                               cudaStream_t stream);
+
 struct DecodeArgs {
   void* out;
   const void* q;

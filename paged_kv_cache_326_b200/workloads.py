@@ -404,3 +404,32 @@ def full_step(seed: int = 5, device="cpu", dtype=torch.float16, num_layers: int 
     return FullStepInputs(k_cache=k_cache, v_cache=v_cache, context_lens=lens_d,
                           block_tables=tables, slot_mapping=slots, q=qs, k=ks, v=vs,
                           scale=fp32_scale(head_dim), block_size=block_size, seed=seed)
+
+
+def cow_bursts(seed: int = 4, device="cpu", dtype=torch.float16, num_bursts: int = 8,
+               prompts: int = 32, samples: int = 8, num_heads: int = 40, head_dim: int = 128,
+               block_size: int = 16, num_blocks: int = 8192):
+    """Copy-on-write bursts at the OPT-13B layer shape: in each burst, every
+    one of ``prompts`` prompts has its partial last block copied for
+    ``samples - 1`` of its samples (the last one writes in place), i.e. the
+    copies of one decode step right after parallel sampling forks.  Sources
+    and destinations of all bursts are distinct blocks drawn from a seeded
+    permutation of the pool, so rotating through the bursts touches about
+    ``num_bursts * prompts * samples`` blocks (far more than L2 holds).
+
+    Returns (k_cache, v_cache, [pairs of each burst as [n][2] int32])."""
+    dev = torch.device(device)
+    per = prompts * samples
+    if num_bursts * per > num_blocks:
+        raise ValueError("pool too small for the bursts")
+    order = torch.randperm(num_blocks, generator=_gen(seed, "cpu"))
+    bursts = []
+    for b in range(num_bursts):
+        ids = order[b * per:(b + 1) * per].view(prompts, samples)
+        src = ids[:, :1].expand(prompts, samples - 1)
+        dst = ids[:, 1:]
+        bursts.append(torch.stack([src.reshape(-1), dst.reshape(-1)], dim=1)
+                      .to(torch.int32).contiguous().to(dev))
+    g = _gen(seed + 1000003, dev)
+    shape = (num_blocks, num_heads, block_size, head_dim)
+    return _randn(shape, dtype, g, dev), _randn(shape, dtype, g, dev), bursts
