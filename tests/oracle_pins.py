@@ -430,3 +430,76 @@ def pin_copy_out_and_back(copy_fn):
 
 COPY_PINS = [pin_copy_on_write_worked_example, pin_copy_blocks_bits_vs_index_copy,
              pin_copy_out_and_back]
+
+
+# ---------------------------------------------------------------------------
+# 8-bit (E4M3) KV cache
+# ---------------------------------------------------------------------------
+
+def _torch_e4m3(x32: np.ndarray) -> np.ndarray:
+    """torch's float32 -> float8_e4m3fn cast (round to nearest even), as codes."""
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_e4m3_every_fp16_vs_torch(encode):
+    """Every finite fp16 value below the first magnitude that rounds past 448
+    (464), subnormals and both zeros included: the codes equal torch's cast."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    x = bits.view(np.float16).astype(np.float32)
+    keep = np.isfinite(x) & (np.abs(x) < 464.0)
+    got = encode(x[keep])
+    assert np.array_equal(got, _torch_e4m3(x[keep])), "E4M3 codes differ from torch's cast"
+
+
+def pin_e4m3_random_fp32_vs_torch(encode):
+    """Random fp32 magnitudes spread over 2^-12 .. 2^8.8 (exponents drawn
+    uniformly), both signs."""
+    rng = np.random.default_rng(401)
+    mag = np.exp2(rng.uniform(-12, 8.8, size=200000)).astype(np.float32)
+    x = np.where(rng.random(200000) < 0.5, -mag, mag).astype(np.float32)
+    assert np.array_equal(encode(x), _torch_e4m3(x)), "E4M3 codes differ from torch (fp32)"
+
+
+def pin_e4m3_closed_forms(encode, decode):
+    """The format's constants: largest finite 1.75 * 2^8 = 448 (code 0x7E),
+    smallest normal 2^-6 (0x08), smallest subnormal 2^-9 (0x01), NaN at
+    S.1111.111 only, 254 finite codes increasing with the code; saturation of
+    large magnitudes and infinities to +-448; signed zero; ties to even
+    worked by hand: with scale 0.5, 1.0 -> 2.0 = 0x40, -2.5 -> -5.0 = 0xCA,
+    0.3 -> 0.6 (nearer 0.625 = 0x32 than 0.5625), 500 -> 448 = 0x7E."""
+    v = decode(np.arange(256, dtype=np.uint8))
+    assert v[0x7E] == 448.0 and v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and np.isnan(v).sum() == 2
+    assert np.all(np.diff(v[:0x7F]) > 0) and np.array_equal(v[0x80:0xFF], -v[:0x7F])
+    big = np.array([1e6, -1e6, np.inf, -np.inf, 470.0], dtype=np.float32)
+    assert encode(big).tolist() == [0x7E, 0xFE, 0x7E, 0xFE, 0x7E]
+    assert encode(np.array([0.0, -0.0], dtype=np.float32)).tolist() == [0x00, 0x80]
+    assert encode(np.array([np.nan], dtype=np.float32)).tolist() == [0x7F]
+    x = np.array([1.0, -2.5, 0.3, 500.0], dtype=np.float32) / np.float32(0.5)
+    assert encode(x).tolist() == [0x40, 0xCA, 0x32, 0x7E]
+
+
+def pin_fp8_attention_on_representable_values(decode_fp8, quantize):
+    """Keys and values that E4M3 holds exactly (small multiples of powers of
+    two) times a power-of-two scale: quantizing them loses nothing, so
+    attention over the 8-bit cache equals attention over the same pool in
+    fp16, computed here with torch (fp64) on the unpaged texts."""
+    H, D, B = 2, 8, 4
+    lens = [6, 11, 1]
+    rng = np.random.default_rng(411)
+    mant = rng.integers(-15, 16, size=(64, H, B, D)).astype(np.float32) / 8.0
+    k_scale, v_scale = 0.25, 4.0
+    kc = mant * np.float32(k_scale)
+    vc = np.roll(mant, 1, axis=3) * np.float32(v_scale)
+    kq = quantize(kc, k_scale)
+    vq = quantize(vc, v_scale)
+    tables = rng.permutation(64)[:12].reshape(3, 4)
+    q = rng.standard_normal((3, H, D))
+    got = decode_fp8(q, kq, vq, tables, lens, 0.3, B, k_scale, v_scale)
+    Ks = [torch.from_numpy(np.stack([kc[tables[s, t // B], :, t % B] for t in range(L)]).astype(np.float64))
+          for s, L in enumerate(lens)]
+    Vs = [torch.from_numpy(np.stack([vc[tables[s, t // B], :, t % B] for t in range(L)]).astype(np.float64))
+          for s, L in enumerate(lens)]
+    ref = sdpa_contiguous(torch.from_numpy(q), Ks, Vs, 0.3)
+    assert np.abs(got - ref).max() <= 1e-12, "8-bit cache attention vs exact values"

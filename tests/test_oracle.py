@@ -68,3 +68,37 @@ def test_kv_head_of_rejects_uneven_groups():
     with pytest.raises(ValueError):
         oracle.kv_head_of(6, 4)
     assert list(oracle.kv_head_of(8, 2)) == [0, 0, 0, 0, 1, 1, 1, 1]
+
+
+def test_e4m3_codes_match_torch_on_every_fp16_value():
+    P.pin_e4m3_every_fp16_vs_torch(oracle.e4m3_encode)
+
+
+def test_e4m3_codes_match_torch_on_random_fp32():
+    P.pin_e4m3_random_fp32_vs_torch(oracle.e4m3_encode)
+
+
+def test_e4m3_closed_forms():
+    P.pin_e4m3_closed_forms(oracle.e4m3_encode, oracle.e4m3_decode)
+
+
+def test_fp8_attention_on_representable_values():
+    P.pin_fp8_attention_on_representable_values(oracle.paged_decode_fp8, oracle.quantize)
+
+
+def test_fp8_cache_write_stores_the_codes_at_the_slots():
+    """The 8-bit write puts quantize(token) at each slot, plain indexing
+    checked here, and skips negative slots."""
+    rng = np.random.default_rng(421)
+    H, D, B, N = 2, 8, 4, 6
+    kc = rng.integers(0, 256, size=(N, H, B, D), dtype=np.uint8)
+    vc = rng.integers(0, 256, size=(N, H, B, D), dtype=np.uint8)
+    k = rng.standard_normal((3, H, D)).astype(np.float32)
+    v = rng.standard_normal((3, H, D)).astype(np.float32)
+    slots = [5, -1, 22]
+    k2, v2 = oracle.cache_write_fp8(kc, vc, k, v, slots, B, 0.5, 0.125)
+    ek, ev = kc.copy(), vc.copy()
+    for t, sl in ((0, 5), (2, 22)):
+        ek[sl // B, :, sl % B] = oracle.e4m3_encode(k[t] / np.float32(0.5))
+        ev[sl // B, :, sl % B] = oracle.e4m3_encode(v[t] / np.float32(0.125))
+    assert np.array_equal(k2, ek) and np.array_equal(v2, ev)

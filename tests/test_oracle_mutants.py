@@ -223,3 +223,76 @@ def test_planted_copy_mistake_is_caught(fn):
 def test_unmodified_oracle_passes_copy_pins():
     for pin in P.COPY_PINS:
         pin(oracle.copy_blocks)
+
+
+
+# --- 8-bit cache: planted mistakes --------------------------------------------
+
+def _encode_variant(x, ties_even=True, saturate=True, keep_sign=True):
+    """The E4M3 rounding with one rule changed (a planted mistake)."""
+    vals = np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros(x.shape, dtype=np.uint8)
+    for i, v in np.ndenumerate(x):
+        if np.isnan(v):
+            out[i] = 0x7F
+            continue
+        a = abs(v)
+        if a > 448.0 and not saturate:
+            out[i] = 0x7F
+            continue
+        a = min(a, 448.0)
+        hi = int(np.searchsorted(vals, a))
+        lo = max(hi - 1, 0)
+        if vals[hi] == a:
+            c = hi
+        elif a - vals[lo] < vals[hi] - a:
+            c = lo
+        elif a - vals[lo] > vals[hi] - a:
+            c = hi
+        else:
+            c = (lo if lo % 2 == 0 else hi) if ties_even else hi
+        out[i] = (0x80 if (np.signbit(v) and keep_sign) else 0) | c
+    return out
+
+
+def encode_ties_away(x):
+    return _encode_variant(x, ties_even=False)
+
+
+def encode_without_saturation(x):
+    return _encode_variant(x, saturate=False)
+
+
+def encode_drops_sign(x):
+    return _encode_variant(x, keep_sign=False)
+
+
+def test_planted_e4m3_encoding_mistakes_are_caught():
+    for fn in (encode_ties_away, encode_without_saturation, encode_drops_sign):
+        failed = 0
+        for pin in (P.pin_e4m3_every_fp16_vs_torch,
+                    lambda e: P.pin_e4m3_closed_forms(e, oracle.e4m3_decode)):
+            try:
+                pin(fn)
+            except AssertionError:
+                failed += 1
+        assert failed, fn.__name__
+
+
+def decode_with_bias_8(codes):
+    return oracle.e4m3_decode(codes) / 2.0
+
+
+def test_planted_e4m3_decoding_mistake_is_caught():
+    with pytest.raises(AssertionError):
+        P.pin_e4m3_closed_forms(oracle.e4m3_encode, decode_with_bias_8)
+
+
+def quantize_multiplying(x, scale):
+    return oracle.e4m3_encode(np.asarray(x, dtype=np.float32) * np.float32(scale))
+
+
+def test_planted_scale_mistake_is_caught():
+    with pytest.raises(AssertionError):
+        P.pin_fp8_attention_on_representable_values(oracle.paged_decode_fp8, quantize_multiplying)
