@@ -157,7 +157,7 @@ def oracle_runner(w, num_pairs):
     workload, in text-major order.  Inputs are prepared outside the timed
     region.  Returns (run, kv_bytes_of_the_sample)."""
     from threadpoolctl import threadpool_limits
-    from tests.gpu_helpers import oracle_inputs, run_oracle
+    from tests.gpu_helpers import oracle_inputs, run_oracle, run_oracle_fp8
     H = w.num_heads
     pairs = [(p // H, p % H) for p in range(num_pairs)]
     seqs = sorted({s for s, _ in pairs})
@@ -167,14 +167,21 @@ def oracle_runner(w, num_pairs):
     full = num_pairs == len(seqs) * H
     # bytes of the KV cache the sample covers (each key/value head once)
     Hkv = w.k_cache.shape[1]
+    cb = w.k_cache.element_size()
     if full:
-        sample_bytes = sum(lens[s] for s in seqs) * 2 * Hkv * w.head_dim * w.q.element_size()
+        sample_bytes = sum(lens[s] for s in seqs) * 2 * Hkv * w.head_dim * cb
     else:
-        sample_bytes = sum(lens[s] for s, _ in pairs) * 2 * w.head_dim * w.q.element_size()
+        sample_bytes = sum(lens[s] for s, _ in pairs) * 2 * w.head_dim * cb
+
+    fp8 = w.k_cache.dtype == torch.uint8
 
     def run():
         with threadpool_limits(limits=1):
-            run_oracle(oi, w.scale, w.block_size, None if full else pairs)
+            if fp8:
+                run_oracle_fp8(oi, w.scale, w.block_size, w.meta["k_scale"], w.meta["v_scale"],
+                               None if full else pairs)
+            else:
+                run_oracle(oi, w.scale, w.block_size, None if full else pairs)
     return run, sample_bytes
 
 
@@ -354,6 +361,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
+    ap.add_argument("--kv-dtype", choices=["f16", "fp8"], default="f16",
+                    help="fp8: the batch-64 step over 8-bit E4M3 caches (two calls)")
     ap.add_argument("--gqa-kernel", choices=["auto", "cores", "tensor"], default="auto",
                     help="grouped-query workload: kernel choice (PA_OPT_GQA_KERNEL)")
     ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa", "cow_copy"],
@@ -386,18 +395,25 @@ def main():
     gqa = args.workload == "llama2_70b_gqa"
     P.pa_set_option(P.PA_OPT_GQA_KERNEL, {"auto": 0, "cores": 1, "tensor": 2}[args.gqa_kernel])
     gqa_kernel = "CUDA-core" if args.gqa_kernel == "cores" else "tensor-core"
+    fp8 = args.kv_dtype == "fp8"
+    if gqa and fp8:
+        raise SystemExit("the 8-bit cache is multi-head only")
     if gqa:
         args.path = "calls"   # the one-launch step is multi-head only
         w = W.llama2_70b_gqa(seed=dist.batch_seed(6, ranks), device=dev)
+    elif fp8:
+        args.path = "calls"   # the one-launch step stores 16-bit values
+        w = W.opt13b_batch64_fp8(seed=dist.batch_seed(2, ranks), device=dev)
     else:
         w = W.opt13b_batch64(seed=dist.batch_seed(2, ranks), device=dev)
     S, H, D = w.q.shape
     Hkv = w.k_cache.shape[1]
     eb = w.q.element_size()
+    cb = w.k_cache.element_size()                 # cache bytes per number (1 for 8-bit)
     lens = w.context_lens.tolist()
-    step_kv = kv_bytes(lens, Hkv, D, eb)
+    step_kv = kv_bytes(lens, Hkv, D, cb)
     decode_bytes = step_kv + 2 * S * H * D * eb + sum(4 * -(-L // w.block_size) for L in lens) + 4 * S
-    write_bytes = 4 * S * Hkv * D * eb + 8 * S   # k, v read and stored; slots
+    write_bytes = 2 * S * Hkv * D * (eb + cb) + 8 * S   # k, v read and stored; slots
     fused = args.path == "fused"
     if fused:
         decode_bytes += write_bytes
@@ -406,7 +422,10 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def write_part(k, v, slots):
-        if not fused:
+        if fp8:
+            P.pa_kv_cache_write_fp8(k, v, w.k_cache, w.v_cache, slots, w.meta["k_scale"],
+                                    w.meta["v_scale"], status=status)
+        elif not fused:
             P.pa_kv_cache_write(k, v, w.k_cache, w.v_cache, slots, status=status)
 
     def decode_part(q, k, v, slots, tables, lens):
@@ -416,6 +435,10 @@ def main():
         elif gqa:
             P.pa_paged_attn_decode_gqa(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
                                        workspace=ws, status=status)
+        elif fp8:
+            P.pa_paged_attn_decode_fp8(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
+                                       w.meta["k_scale"], w.meta["v_scale"], workspace=ws,
+                                       status=status)
         else:
             P.pa_paged_attn_decode(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
                                    workspace=ws, status=status)
@@ -505,7 +528,10 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload, "num_seqs": S, "num_heads": H,
+        "config": {"workload": args.workload + ("_fp8" if fp8 else ""), "num_seqs": S,
+                   "num_heads": H,
+                   "kv_cache": ("e4m3, per-tensor scales k %g, v %g" %
+                                (w.meta["k_scale"], w.meta["v_scale"]) if fp8 else "f16"),
                    "num_kv_heads": Hkv, "head_dim": D, "block_size": w.block_size,
                    "context_lens": ("uniform [128, 4096], seed 6+rank" if gqa else
                                     "uniform [128, 2048], seed 2+rank"),
@@ -514,6 +540,7 @@ def main():
                    "parallelism": f"independent batch per GPU x{world}",
                    "path": ("pa_decode_step" if fused else
                             f"pa_kv_cache_write + pa_paged_attn_decode_gqa ({gqa_kernel})" if gqa
+                            else "pa_kv_cache_write_fp8 + pa_paged_attn_decode_fp8" if fp8
                             else "pa_kv_cache_write + pa_paged_attn_decode")},
         "decode_tokens_per_s": world * S / (ms_step * 1e-3),
         "pct_of_nominal_8tbs": 100.0 * (value / world) / NOMINAL_HBM_GBS,
@@ -521,10 +548,11 @@ def main():
                       {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": traffic_per_launch(args.workload, args.path),
+                     "traffic": (None if fp8 else traffic_per_launch(args.workload, args.path)),
                      "kernel": ("pa_decode_step (decode kernel with the cache write, + merge kernel)"
                                 if fused else
                                 f"pa_paged_attn_decode_gqa ({gqa_kernel} decode kernel + merge kernel)" if gqa
+                                else "pa_paged_attn_decode_fp8 (8-bit decode kernel + merge kernel)" if fp8
                                 else "pa_paged_attn_decode (decode kernel + merge kernel)"),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": decode_bytes},
         "e2e": {"value": world * step_kv / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",

@@ -48,7 +48,10 @@ extern "C" {
 struct CUstream_st;                       /* same type as cudaStream_t */
 typedef struct CUstream_st* pa_stream_t;
 
-typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+/* Element types.  PA_E4M3 (8-bit cache codes) only where a call says so:
+ * pa_copy_blocks's pools; the 8-bit entry points take their fp16/bf16
+ * tensors' type as dt and the cache as raw codes. */
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2 } pa_dtype;
 
 enum {
   PA_OK = 0,
@@ -216,6 +219,53 @@ int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, cons
                              size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
 
 /*
+ * 8-bit KV cache ("The KV Cache and PagedAttention", section "What Came
+ * After": one byte per cached number instead of two, so about twice the
+ * tokens fit).  The pages fix no format; this library's reading:
+ *  - each cached number is an E4M3 code (1 sign, 4 exponent bits with bias
+ *    7, 3 mantissa bits; finite values only, largest 448; S.1111.111 is NaN);
+ *  - one fp32 scale per cache tensor: code c of the key cache stands for
+ *    value(c) * k_scale, of the value cache value(c) * v_scale;
+ *  - the pools are laid out as the 16-bit ones, one byte per number:
+ *    [num_blocks][num_heads][block_size][head_dim] uint8 codes.
+ * Scales must be finite and positive (else PA_ERR_INVALID).
+ */
+
+/*
+ * pa_kv_cache_write_fp8 — pa_kv_cache_write into 8-bit caches: element x of
+ * k[t] (v[t]) is stored as the E4M3 code of the fp32 quotient x / k_scale
+ * (x / v_scale), IEEE division, rounded to the nearest code with ties to the
+ * even one, magnitudes past 448 saturating to +-448, NaN to NaN.
+ *   k, v           [num_tokens][num_heads][head_dim] dt (fp16 or bf16)
+ *   k_cache,v_cache 8-bit pools (above); other arguments and errors as for
+ *                  pa_kv_cache_write.
+ */
+int pa_kv_cache_write_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                          const int64_t* slot_mapping, float k_scale, float v_scale,
+                          int num_tokens, int num_heads, int head_dim, int block_size,
+                          int64_t num_blocks, pa_dtype dt, int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_paged_attn_decode_fp8 — pa_paged_attn_decode over 8-bit caches:
+ *     z_t = scale * sum_d q[s][h][d] * value(K_t[d]) * k_scale,
+ *     out[s][h][:] = sum_t softmax(z)_t * value(V_t[:]) * v_scale.
+ * Codes are widened exactly; arithmetic as for pa_paged_attn_decode (fp32).
+ *   q, out         [num_seqs][num_heads][head_dim] dt (fp16 or bf16)
+ *   k_cache,v_cache 8-bit pools; the workspace is
+ *                  pa_paged_attn_decode_workspace_size(...) bytes (the same
+ *                  sizes as the 16-bit call).  Multi-head only.  Other
+ *                  arguments and errors as for pa_paged_attn_decode.
+ * Each chunk of work is 4096/head_dim tokens (32 at head_dim 128), so every
+ * copy still moves 4 KB of keys and 4 KB of values.
+ */
+int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             float scale, float k_scale, float v_scale, int num_seqs,
+                             int num_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                             int64_t num_blocks, pa_dtype dt, void* workspace,
+                             size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
+
+/*
  * pa_copy_blocks — copy whole blocks from one pool to another, or within one
  * pool: the device side of copy-on-write ("The KV Cache and
  * PagedAttention", section "Shared, Copied on Write": before a text writes
@@ -225,6 +275,7 @@ int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, cons
  * "When Memory Runs Out": blocks set aside in CPU memory).
  *
  *   src_k, src_v   [src_num_blocks][num_heads][block_size][head_dim] dt
+ *                  (PA_F16, PA_BF16, or PA_E4M3 for 8-bit pools)
  *   dst_k, dst_v   [dst_num_blocks][num_heads][block_size][head_dim] dt; may
  *                  be src_k, src_v (copy-on-write)
  *   block_pairs    [num_pairs][2] int32: (source block, destination block)

@@ -34,6 +34,7 @@ PA_ERR_TOO_LARGE = -12
 
 PA_F16 = 0
 PA_BF16 = 1
+PA_E4M3 = 2
 
 PA_OPT_WAIT_LIMIT_NS = 1
 PA_OPT_DECODE_WARPS = 2
@@ -72,6 +73,10 @@ _SIGNATURES = {
                               _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_paged_attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
                                             _i32, _i32, _i64, _i32, _vp, _vp]),
+    "pa_kv_cache_write_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _f32, _f32, _i32, _i32, _i32, _i32,
+                                     _i64, _i32, _vp, _vp]),
+    "pa_paged_attn_decode_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _f32, _f32, _i32, _i32,
+                                        _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32,
                               _vp, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
@@ -168,6 +173,59 @@ def pa_kv_cache_write(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
     _check(code, "pa_kv_cache_write")
 
 
+def _codes(t: torch.Tensor, name: str) -> int:
+    """An 8-bit cache pool: uint8 or float8_e4m3fn, on the GPU."""
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise TypeError(f"{name} must hold 8-bit codes (uint8 or float8_e4m3fn), got {t.dtype}")
+    return _cuda(t, name)
+
+
+def pa_kv_cache_write_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
+                          v_cache: torch.Tensor, slot_mapping: torch.Tensor, k_scale: float,
+                          v_scale: float, status: Optional[torch.Tensor] = None,
+                          stream=None) -> None:
+    """k, v: [T][H][D] fp16/bf16; 8-bit caches [N][H][B][D]; slot_mapping [T]
+    int64; per-tensor scales."""
+    T, H, D = k.shape
+    N, H2, B, D2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
+        raise ValueError("shape mismatch between k/v and the caches")
+    if slot_mapping.shape != (T,) or v.dtype != k.dtype:
+        raise ValueError("slot_mapping must be [num_tokens]; k and v must share a dtype")
+    code = lib().pa_kv_cache_write_fp8(
+        _cuda(k, "k"), _cuda(v, "v"), _codes(k_cache, "k_cache"), _codes(v_cache, "v_cache"),
+        _cuda(slot_mapping, "slot_mapping", torch.int64), float(k_scale), float(v_scale), T, H, D,
+        B, N, _dtype_code(k), _status_ptr(status), _stream(stream, k.device))
+    _check(code, "pa_kv_cache_write_fp8")
+
+
+def pa_paged_attn_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                             v_cache: torch.Tensor, block_tables: torch.Tensor,
+                             context_lens: torch.Tensor, scale: float, k_scale: float,
+                             v_scale: float, workspace: Optional[torch.Tensor] = None,
+                             status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out, q: [S][H][D] fp16/bf16; 8-bit caches [N][H][B][D]."""
+    S, H, D = q.shape
+    N, H2, B, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S][max_blocks], context_lens [S]")
+    if out.dtype != q.dtype:
+        raise TypeError("q and out must share a dtype")
+    MB = block_tables.shape[1]
+    if workspace is None:
+        workspace = workspace_for(q, B, MB)
+    code = lib().pa_paged_attn_decode_fp8(
+        _cuda(out, "out"), _cuda(q, "q"), _codes(k_cache, "k_cache"), _codes(v_cache, "v_cache"),
+        _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(context_lens, "context_lens", torch.int32), float(scale), float(k_scale),
+        float(v_scale), S, H, D, B, MB, N, _dtype_code(q), _cuda(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _status_ptr(status), _stream(stream, q.device))
+    _check(code, "pa_paged_attn_decode_fp8")
+    return out
+
+
 def _pool(t: torch.Tensor, name: str) -> int:
     """A pool the GPU can address: a CUDA tensor, or a pinned CPU tensor (the
     library checks the mapping before launch)."""
@@ -195,11 +253,11 @@ def pa_copy_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor
         if t.dtype != src_k.dtype:
             raise TypeError("pools must share a dtype")
     dev = block_pairs.device
+    dt = PA_E4M3 if src_k.dtype in (torch.uint8, torch.float8_e4m3fn) else _dtype_code(src_k)
     code = lib().pa_copy_blocks(
         _pool(src_k, "src_k"), _pool(src_v, "src_v"), Ns, _pool(dst_k, "dst_k"),
         _pool(dst_v, "dst_v"), Nd, _cuda(block_pairs, "block_pairs", torch.int32),
-        block_pairs.shape[0], H, D, B, _dtype_code(src_k), _status_ptr(status),
-        _stream(stream, dev))
+        block_pairs.shape[0], H, D, B, dt, _status_ptr(status), _stream(stream, dev))
     _check(code, "pa_copy_blocks")
 
 

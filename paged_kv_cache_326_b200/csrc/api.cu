@@ -39,6 +39,9 @@ bool device_accessible(const void* p) {
   return false;
 }
 
+// A usable per-tensor scale of the 8-bit cache: finite and positive.
+bool scale_ok(float s) { return s > 0.f && s <= 3.402823466e38f; }
+
 int from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return PA_OK;
   if (e == cudaErrorInvalidValue) return PA_ERR_INVALID;
@@ -127,8 +130,10 @@ int decode_common(void* out, const void* q, const void* k_cache, const void* v_c
                   int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                   int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt, void* workspace,
                   size_t workspace_bytes, int32_t* d_status, pa_stream_t stream,
-                  const void* k_new, const void* v_new, const int64_t* slot_mapping) {
+                  const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                  bool fp8 = false, float k_scale = 1.f, float v_scale = 1.f) {
   if (num_seqs == 0) return PA_OK;
+  if (fp8 && !(scale_ok(k_scale) && scale_ok(v_scale))) return PA_ERR_INVALID;
   if (!pa::decode_sizes_supported(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                   max_blocks_per_seq) ||
       num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16))
@@ -164,6 +169,9 @@ int decode_common(void* out, const void* q, const void* k_cache, const void* v_c
   a.k_new = k_new;
   a.v_new = v_new;
   a.slot_mapping = slot_mapping;
+  a.fp8 = fp8;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   return from_cuda(pa::launch_paged_attn_decode(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -182,12 +190,40 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
                        dt, workspace, workspace_bytes, d_status, stream, nullptr, nullptr, nullptr);
 }
 
+int pa_kv_cache_write_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                          const int64_t* slot_mapping, float k_scale, float v_scale,
+                          int num_tokens, int num_heads, int head_dim, int block_size,
+                          int64_t num_blocks, pa_dtype dt, int32_t* d_status, pa_stream_t stream) {
+  if (num_tokens < 0 || !shape_ok(num_heads, head_dim, block_size) || num_blocks <= 0 ||
+      (dt != PA_F16 && dt != PA_BF16) || !scale_ok(k_scale) || !scale_ok(v_scale))
+    return PA_ERR_INVALID;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  return from_cuda(pa::launch_kv_cache_write_fp8(
+      k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale, num_tokens, num_heads, head_dim,
+      block_size, num_blocks, dt == PA_BF16, d_status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             float scale, float k_scale, float v_scale, int num_seqs,
+                             int num_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                             int64_t num_blocks, pa_dtype dt, void* workspace,
+                             size_t workspace_bytes, int32_t* d_status, pa_stream_t stream) {
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       dt, workspace, workspace_bytes, d_status, stream, nullptr, nullptr, nullptr,
+                       true, k_scale, v_scale);
+}
+
 int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks, void* dst_k,
                    void* dst_v, int64_t dst_num_blocks, const int32_t* block_pairs,
                    int num_pairs, int num_heads, int head_dim, int block_size, pa_dtype dt,
                    int32_t* d_status, pa_stream_t stream) {
   if (num_pairs < 0 || !shape_ok(num_heads, head_dim, block_size) || src_num_blocks <= 0 ||
-      dst_num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16))
+      dst_num_blocks <= 0 || (dt != PA_F16 && dt != PA_BF16 && dt != PA_E4M3))
     return PA_ERR_INVALID;
   if (num_pairs == 0) return PA_OK;
   if (!src_k || !src_v || !dst_k || !dst_v || !block_pairs) return PA_ERR_INVALID;
@@ -197,7 +233,8 @@ int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks,
   if (!device_accessible(src_k) || !device_accessible(src_v) || !device_accessible(dst_k) ||
       !device_accessible(dst_v) || !device_accessible(block_pairs))
     return PA_ERR_INVALID;
-  const int64_t block_bytes = static_cast<int64_t>(num_heads) * block_size * head_dim * 2;
+  const int64_t block_bytes =
+      static_cast<int64_t>(num_heads) * block_size * head_dim * (dt == PA_E4M3 ? 1 : 2);
   return from_cuda(pa::launch_copy_blocks(src_k, src_v, dst_k, dst_v, block_pairs, num_pairs,
                                           block_bytes, src_num_blocks, dst_num_blocks, d_status,
                                           reinterpret_cast<cudaStream_t>(stream)));

@@ -74,7 +74,8 @@ struct DecodeParams {
   const void* v_cache;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  float qk_scale_log2;
+  float qk_scale_log2;  // scale * log2(e) (* the keys' scale for an 8-bit cache)
+  float v_scale;        // the values' scale for an 8-bit cache, else 1
   int num_seqs;
   int num_heads;      // virtual heads: key/value heads x subsets (the flat order's heads)
   int num_q_heads;    // query heads of q and out

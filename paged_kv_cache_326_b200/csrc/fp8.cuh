@@ -1,0 +1,40 @@
+// 8-bit (E4M3) cache codes: conversions through the hardware's cvt forms.
+// E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits, finite values only
+// (largest 448, S.1111.111 is NaN).  Every E4M3 value is exact in fp16.
+#pragma once
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+namespace pa {
+
+// Two floats -> two codes, `lo` in the low byte: round to nearest even,
+// magnitudes past 448 (infinities too) saturate to 448, NaN stays NaN.
+__device__ __forceinline__ uint16_t e4m3x2_from_floats(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two codes (low byte first) -> their values as a half2 (exact).
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t x) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(x));
+  return *reinterpret_cast<__half2*>(&r);
+}
+
+// Sixteen codes (one 16-byte vector) -> sixteen floats.
+__device__ __forceinline__ void unpack16_e4m3(const uint4& v, float (&f)[16]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 a = __half22float2(e4m3x2_to_half2(static_cast<uint16_t>(w[i] & 0xffffu)));
+    const float2 b = __half22float2(e4m3x2_to_half2(static_cast<uint16_t>(w[i] >> 16)));
+    f[4 * i + 0] = a.x;
+    f[4 * i + 1] = a.y;
+    f[4 * i + 2] = b.x;
+    f[4 * i + 3] = b.y;
+  }
+}
+
+}  // namespace pa

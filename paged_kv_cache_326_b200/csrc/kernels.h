@@ -7,6 +7,14 @@
 
 namespace pa {
 
+// The 8-bit cache's write: codes of k / k_scale and v / v_scale (E4M3, round
+// to nearest even, saturating); k, v are fp16 (bf16 if `bf16`).
+cudaError_t launch_kv_cache_write_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                                      const int64_t* slot_mapping, float k_scale, float v_scale,
+                                      int num_tokens, int num_heads, int head_dim, int block_size,
+                                      int64_t num_blocks, bool bf16, int32_t* status,
+                                      cudaStream_t stream);
+
 cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
                                   const int64_t* slot_mapping, int num_tokens, int num_heads,
                                   int head_dim, int block_size, int64_t num_blocks,
@@ -41,6 +49,10 @@ struct DecodeArgs {
   int32_t* status;
   int64_t wait_limit_ns;
   int64_t forced_warps;  // 0 = fill the device
+  // 8-bit (E4M3) cache with per-tensor scales (pa_paged_attn_decode_fp8).
+  bool fp8 = false;
+  float k_scale = 1.f;
+  float v_scale = 1.f;
   // Fused decode step (pa_decode_step) only; all null otherwise.
   const void* k_new = nullptr;
   const void* v_new = nullptr;

@@ -52,6 +52,7 @@
 #include <cstdint>
 
 #include "decode_common.cuh"
+#include "fp8.cuh"
 #include "kernels.h"
 
 namespace pa {
@@ -80,18 +81,33 @@ __host__ __device__ constexpr int warp_area_bytes(int D, int stages, int gs) {
 // GS: query heads per work unit (1 = multi-head attention).  With grouped-
 // query attention the GS query heads of a unit share one key/value head, so
 // every K/V row copied is used GS times from registers.
-template <typename T, int D, int B, int WARPS, int STAGES, bool FUSED, int GS>
+// F8: the cache holds 8-bit E4M3 codes (one byte per number, per-tensor
+// scales) instead of T; a chunk is then twice the tokens for the same 4 KB,
+// and each lane dequantizes 16 codes per 16-byte vector in registers.
+template <typename T, int D, int B, int WARPS, int STAGES, bool FUSED, int GS, bool F8>
 __global__ void __launch_bounds__(WARPS * 32, 2)
 paged_decode_kernel(const DecodeParams p) {
-  constexpr int CH = chunk_tokens(D);        // tokens per chunk
-  constexpr int LPT = D / 8;                 // lanes per token row (16-byte vectors)
+  constexpr int EB = F8 ? 1 : 2;             // cache bytes per number
+  constexpr int CH = 4096 / (D * EB);        // tokens per chunk (4 KB of keys)
+  constexpr int VEC = 16 / EB;               // numbers per 16-byte vector
+  constexpr int LPT = D / VEC;               // lanes per token row
   constexpr int TPI = 32 / LPT;              // token rows per warp-wide load
   constexpr int ITERS = CH / TPI;            // loads per chunk (8)
   constexpr int NB = CH >= B ? CH / B : 1;   // physical blocks a chunk touches
-  constexpr int TILE = CH * D;               // elements of K (or V) per chunk
+  constexpr int ROWB = D * EB;               // bytes per cache row
   constexpr int STRIDE = stage_bytes(D, GS);
   constexpr int AREA = warp_area_bytes(D, STAGES, GS);
   static_assert(CH % TPI == 0 && (CH % B == 0 || B % CH == 0), "shape");
+  static_assert(!(F8 && FUSED), "the one-launch step stores T");
+  // one 16-byte vector of cache numbers -> VEC floats
+  auto load_vec = [](const uint8_t* src, float (&f)[VEC]) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    if constexpr (F8) {
+      unpack16_e4m3(v, f);
+    } else {
+      unpack8<T>(v, f);
+    }
+  };
 
   extern __shared__ __align__(128) uint8_t smem[];
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + WARPS * AREA);
@@ -139,8 +155,8 @@ paged_decode_kernel(const DecodeParams p) {
   __syncwarp();
 
   const uint64_t policy = l2_evict_first_policy();
-  const T* __restrict__ kc = static_cast<const T*>(p.k_cache);
-  const T* __restrict__ vc = static_cast<const T*>(p.v_cache);
+  const uint8_t* __restrict__ kc = static_cast<const uint8_t*>(p.k_cache);
+  const uint8_t* __restrict__ vc = static_cast<const uint8_t*>(p.v_cache);
   const T* __restrict__ qg = static_cast<const T*>(p.q);
 
   Scheduler<CH, B, NB> sched(p, prefix, sp, w, lane);
@@ -181,9 +197,9 @@ paged_decode_kernel(const DecodeParams p) {
     ++issued;
     if (lane == 0) {
       uint8_t* stage = area + st * STRIDE;
-      T* sK = reinterpret_cast<T*>(stage);
-      T* sV = sK + TILE;
-      T* sQ = sV + TILE;
+      uint8_t* sK = stage;
+      uint8_t* sV = stage + 4096;
+      T* sQ = reinterpret_cast<T*>(stage + 8192);
       int32_t* flag = reinterpret_cast<int32_t*>(stage + 2 * 4096 + GS * 2 * D);
       const int len = min(max(len_raw, 0), cap);
       const int nvalid = min(CH, len - j * CH);
@@ -199,7 +215,7 @@ paged_decode_kernel(const DecodeParams p) {
       fence_proxy_async_smem();
       *flag = bad ? 1 : 0;
       const uint32_t qbytes = first ? GS * D * 2 : 0;
-      const uint32_t kvbytes = bad ? 0 : 2u * nvalid * D * 2;
+      const uint32_t kvbytes = bad ? 0 : 2u * nvalid * ROWB;
       mbar_arrive_expect_tx(&bars[st], qbytes + kvbytes);
       if (first)
         bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D, GS * D * 2, &bars[st],
@@ -214,24 +230,24 @@ paged_decode_kernel(const DecodeParams p) {
           for (int k = 0; k < NB; ++k) {
             const int rows = min(B, pool_rows - k * B);
             if (rows > 0) {
-              const int64_t off = (static_cast<int64_t>(blk[k]) * Hkv + kv_head(h)) * B * D;
-              bulk_copy_g2s(sK + k * B * D, kc + off, rows * D * 2, &bars[st], policy);
-              bulk_copy_g2s(sV + k * B * D, vc + off, rows * D * 2, &bars[st], policy);
+              const int64_t off = (static_cast<int64_t>(blk[k]) * Hkv + kv_head(h)) * B * ROWB;
+              bulk_copy_g2s(sK + k * B * ROWB, kc + off, rows * ROWB, &bars[st], policy);
+              bulk_copy_g2s(sV + k * B * ROWB, vc + off, rows * ROWB, &bars[st], policy);
             }
           }
         } else {
           const int row0 = (j * CH) % B;
-          const int64_t off = ((static_cast<int64_t>(blk[0]) * Hkv + kv_head(h)) * B + row0) * D;
+          const int64_t off = ((static_cast<int64_t>(blk[0]) * Hkv + kv_head(h)) * B + row0) * ROWB;
           if (pool_rows > 0) {
-            bulk_copy_g2s(sK, kc + off, pool_rows * D * 2, &bars[st], policy);
-            bulk_copy_g2s(sV, vc + off, pool_rows * D * 2, &bars[st], policy);
+            bulk_copy_g2s(sK, kc + off, pool_rows * ROWB, &bars[st], policy);
+            bulk_copy_g2s(sV, vc + off, pool_rows * ROWB, &bars[st], policy);
           }
         }
         if (new_row) {
           const int64_t src_off = (static_cast<int64_t>(s) * Hkv + kv_head(h)) * D;
-          bulk_copy_g2s(sK + pool_rows * D, static_cast<const T*>(p.k_new) + src_off, D * 2,
+          bulk_copy_g2s(sK + pool_rows * ROWB, static_cast<const T*>(p.k_new) + src_off, ROWB,
                         &bars[st], policy);
-          bulk_copy_g2s(sV + pool_rows * D, static_cast<const T*>(p.v_new) + src_off, D * 2,
+          bulk_copy_g2s(sV + pool_rows * ROWB, static_cast<const T*>(p.v_new) + src_off, ROWB,
                         &bars[st], policy);
         }
       }
@@ -245,8 +261,8 @@ paged_decode_kernel(const DecodeParams p) {
   const int dchunk = lane % LPT;
   const int tsub = lane / LPT;
   // Per query head of this unit (GS of them share every K/V row read).
-  float qf[GS][8];
-  float acc[GS][8];
+  float qf[GS][VEC];
+  float acc[GS][VEC];
   float m[GS], lsum[GS];
   int piece_j0 = 0;
   int prev_unit = -1;
@@ -267,21 +283,24 @@ paged_decode_kernel(const DecodeParams p) {
     }
 
     const uint8_t* stage = area + st * STRIDE;
-    const T* sK = reinterpret_cast<const T*>(stage);
-    const T* sV = sK + TILE;
-    const T* sQ = sV + TILE;
+    const uint8_t* sK = stage;
+    const uint8_t* sV = stage + 4096;
+    const T* sQ = reinterpret_cast<const T*>(stage + 8192);
     const int bad = *reinterpret_cast<const int32_t*>(stage + 2 * 4096 + GS * 2 * D);
 
     if (j == 0 || wu0 != prev_unit) {
       piece_j0 = j;
 #pragma unroll
       for (int g = 0; g < GS; ++g) {
-        float qraw[8];
-        unpack8<T>(*reinterpret_cast<const uint4*>(sQ + g * D + dchunk * 8), qraw);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          qf[g][k] = qraw[k] * p.qk_scale_log2;
-          acc[g][k] = 0.f;
+        for (int h8 = 0; h8 < VEC / 8; ++h8) {
+          float qraw[8];
+          unpack8<T>(*reinterpret_cast<const uint4*>(sQ + g * D + dchunk * VEC + h8 * 8), qraw);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            qf[g][h8 * 8 + k] = qraw[k] * p.qk_scale_log2;
+            acc[g][h8 * 8 + k] = 0.f;
+          }
         }
         m[g] = -INFINITY;
         lsum[g] = 0.f;
@@ -293,13 +312,13 @@ paged_decode_kernel(const DecodeParams p) {
     float sc[GS][ITERS];
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-      float kf[8];
-      unpack8<T>(*reinterpret_cast<const uint4*>(sK + (it * TPI + tsub) * D + dchunk * 8), kf);
+      float kf[VEC];
+      load_vec(sK + (it * TPI + tsub) * ROWB + dchunk * 16, kf);
 #pragma unroll
       for (int g = 0; g < GS; ++g) {
         float d0 = qf[g][0] * kf[0];
 #pragma unroll
-        for (int k = 1; k < 8; ++k) d0 = fmaf(qf[g][k], kf[k], d0);
+        for (int k = 1; k < VEC; ++k) d0 = fmaf(qf[g][k], kf[k], d0);
         sc[g][it] = d0;
       }
     }
@@ -337,7 +356,7 @@ paged_decode_kernel(const DecodeParams p) {
         }
         lsum[g] = fmaf(lsum[g], alpha, psum);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[g][k] *= alpha;
+        for (int k = 0; k < VEC; ++k) acc[g][k] *= alpha;
         m[g] = m_new;
       } else {
 #pragma unroll
@@ -347,23 +366,23 @@ paged_decode_kernel(const DecodeParams p) {
     if (nvalid == CH) {
 #pragma unroll
       for (int it = 0; it < ITERS; ++it) {
-        float vf[8];
-        unpack8<T>(*reinterpret_cast<const uint4*>(sV + (it * TPI + tsub) * D + dchunk * 8), vf);
+        float vf[VEC];
+        load_vec(sV + (it * TPI + tsub) * ROWB + dchunk * 16, vf);
 #pragma unroll
         for (int g = 0; g < GS; ++g)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
+          for (int k = 0; k < VEC; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
       }
     } else {
 #pragma unroll
       for (int it = 0; it < ITERS; ++it) {
         if (it * TPI + tsub < nvalid) {
-          float vf[8];
-          unpack8<T>(*reinterpret_cast<const uint4*>(sV + (it * TPI + tsub) * D + dchunk * 8), vf);
+          float vf[VEC];
+          load_vec(sV + (it * TPI + tsub) * ROWB + dchunk * 16, vf);
 #pragma unroll
           for (int g = 0; g < GS; ++g)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
+            for (int k = 0; k < VEC; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
         }
       }
     }
@@ -383,22 +402,27 @@ paged_decode_kernel(const DecodeParams p) {
 #pragma unroll
       for (int g = 0; g < GS; ++g) {
         float l_all = lsum[g];
-        float o[8];
+        float o[VEC];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = acc[g][k];
+        for (int k = 0; k < VEC; ++k) o[k] = acc[g][k];
 #pragma unroll
         for (int off = LPT; off < 32; off <<= 1) {
           l_all += __shfl_xor_sync(0xffffffffu, l_all, off);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
+          for (int k = 0; k < VEC; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
         }
         if (whole) {
           if (tsub == 0) {
-            const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+            // v_scale (1 for a T cache) turns sums of codes into values
+            const float inv = l_all > 0.f ? p.v_scale / l_all : 0.f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) o[k] *= inv;
-            *reinterpret_cast<uint4*>(static_cast<T*>(p.out) + (qrow + g) * D + dchunk * 8) =
-                pack8<T>(o);
+            for (int h8 = 0; h8 < VEC / 8; ++h8) {
+              float o8[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) o8[k] = o[h8 * 8 + k] * inv;
+              *reinterpret_cast<uint4*>(static_cast<T*>(p.out) + (qrow + g) * D + dchunk * VEC +
+                                        h8 * 8) = pack8<T>(o8);
+            }
           }
         } else {
           float* rec = recs + g * (D + 4);
@@ -407,9 +431,11 @@ paged_decode_kernel(const DecodeParams p) {
             rec[1] = l_all;
           }
           if (tsub == 0) {
-            float4* dst = reinterpret_cast<float4*>(rec + 4 + dchunk * 8);
-            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+            float4* dst = reinterpret_cast<float4*>(rec + 4 + dchunk * VEC);
+#pragma unroll
+            for (int k4 = 0; k4 < VEC / 4; ++k4)
+              dst[k4] = make_float4(o[4 * k4] * p.v_scale, o[4 * k4 + 1] * p.v_scale,
+                                    o[4 * k4 + 2] * p.v_scale, o[4 * k4 + 3] * p.v_scale);
           }
         }
       }
@@ -449,22 +475,22 @@ HeadLayout head_layout(int num_heads, int num_kv_heads) {
 
 // Persistent grid for one decode kernel variant.
 Plan plan_variant(const void* kernel, int D, int B, int num_seqs, int vheads,
-                  int max_blocks_per_seq, int64_t forced_warps, int gs) {
+                  int max_blocks_per_seq, int64_t forced_warps, int gs, bool fp8) {
   return plan_decode(kernel, decode_smem_bytes(D, num_seqs, gs), decode_smem_bytes(D, kMaxSeqs, gs),
-                     kDecodeWarps, chunk_tokens(D), B, num_seqs, vheads, max_blocks_per_seq,
-                     forced_warps);
+                     kDecodeWarps, fp8 ? 4096 / D : chunk_tokens(D), B, num_seqs, vheads,
+                     max_blocks_per_seq, forced_warps);
 }
 
-template <typename T, int D, int B, bool FUSED, int GS>
+template <typename T, int D, int B, bool FUSED, int GS, bool F8>
 const void* decode_kernel_ptr() {
   return reinterpret_cast<const void*>(
-      &paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS>);
+      &paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS, F8>);
 }
 
-template <typename T, int D, int B, bool FUSED, int GS>
+template <typename T, int D, int B, bool FUSED, int GS, bool F8>
 cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
-  const Plan pl = plan_variant(decode_kernel_ptr<T, D, B, FUSED, GS>(), D, B, a.num_seqs,
-                               hl.vheads, a.max_blocks_per_seq, a.forced_warps, GS);
+  const Plan pl = plan_variant(decode_kernel_ptr<T, D, B, FUSED, GS, F8>(), D, B, a.num_seqs,
+                               hl.vheads, a.max_blocks_per_seq, a.forced_warps, GS, F8);
   if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
   const int64_t segs = static_cast<int64_t>(a.num_seqs) * hl.vheads;
   const size_t need = header_bytes(a.num_seqs) + kGrabBytes +
@@ -477,7 +503,10 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   p.v_cache = a.v_cache;
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
-  p.qk_scale_log2 = a.scale * 1.4426950408889634f;  // log2(e)
+  // log2(e), and for an 8-bit cache the keys' scale, folded into the
+  // query; the values' scale multiplies the output
+  p.qk_scale_log2 = a.scale * 1.4426950408889634f * (F8 ? a.k_scale : 1.f);
+  p.v_scale = F8 ? a.v_scale : 1.f;
   p.num_seqs = a.num_seqs;
   p.num_heads = hl.vheads;
   p.num_q_heads = a.num_heads;
@@ -508,63 +537,67 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(
-      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS>, p);
+      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS, F8>, p);
   if (err != cudaSuccess) return err;
   err = launch_merge<T, D>(p, GS, stream);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
-template <typename T, int D, bool FUSED, int GS>
+template <typename T, int D, bool FUSED, int GS, bool F8>
 cudaError_t dispatch_block(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
   switch (a.block_size) {
-    case 4: return launch_typed<T, D, 4, FUSED, GS>(a, hl, stream);
-    case 8: return launch_typed<T, D, 8, FUSED, GS>(a, hl, stream);
-    case 16: return launch_typed<T, D, 16, FUSED, GS>(a, hl, stream);
-    case 32: return launch_typed<T, D, 32, FUSED, GS>(a, hl, stream);
+    case 4: return launch_typed<T, D, 4, FUSED, GS, F8>(a, hl, stream);
+    case 8: return launch_typed<T, D, 8, FUSED, GS, F8>(a, hl, stream);
+    case 16: return launch_typed<T, D, 16, FUSED, GS, F8>(a, hl, stream);
+    case 32: return launch_typed<T, D, 32, FUSED, GS, F8>(a, hl, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T, bool FUSED, int GS>
+template <typename T, bool FUSED, int GS, bool F8>
 cudaError_t dispatch_dim(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
   switch (a.head_dim) {
-    case 64: return dispatch_block<T, 64, FUSED, GS>(a, hl, stream);
-    case 128: return dispatch_block<T, 128, FUSED, GS>(a, hl, stream);
+    case 64: return dispatch_block<T, 64, FUSED, GS, F8>(a, hl, stream);
+    case 128: return dispatch_block<T, 128, FUSED, GS, F8>(a, hl, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <typename T>
 cudaError_t dispatch_heads(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
+  if (a.fp8)  // 8-bit cache: multi-head, two calls
+    return hl.gs == 1 && !a.slot_mapping ? dispatch_dim<T, false, 1, true>(a, hl, stream)
+                                         : cudaErrorInvalidValue;
   if (a.slot_mapping)  // fused decode step: multi-head only
-    return hl.gs == 1 ? dispatch_dim<T, true, 1>(a, hl, stream) : cudaErrorInvalidValue;
+    return hl.gs == 1 ? dispatch_dim<T, true, 1, false>(a, hl, stream) : cudaErrorInvalidValue;
   switch (hl.gs) {
-    case 1: return dispatch_dim<T, false, 1>(a, hl, stream);
-    case 2: return dispatch_dim<T, false, 2>(a, hl, stream);
-    case 4: return dispatch_dim<T, false, 4>(a, hl, stream);
+    case 1: return dispatch_dim<T, false, 1, false>(a, hl, stream);
+    case 2: return dispatch_dim<T, false, 2, false>(a, hl, stream);
+    case 4: return dispatch_dim<T, false, 4, false>(a, hl, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D, bool FUSED, int GS>
+template <int D, bool FUSED, int GS, bool F8>
 const void* kernel_for(int block_size, bool bf16) {
   switch (block_size) {
-    case 4: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 4, FUSED, GS>() : decode_kernel_ptr<__half, D, 4, FUSED, GS>();
-    case 8: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 8, FUSED, GS>() : decode_kernel_ptr<__half, D, 8, FUSED, GS>();
-    case 16: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 16, FUSED, GS>() : decode_kernel_ptr<__half, D, 16, FUSED, GS>();
-    case 32: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 32, FUSED, GS>() : decode_kernel_ptr<__half, D, 32, FUSED, GS>();
+    case 4: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 4, FUSED, GS, F8>() : decode_kernel_ptr<__half, D, 4, FUSED, GS, F8>();
+    case 8: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 8, FUSED, GS, F8>() : decode_kernel_ptr<__half, D, 8, FUSED, GS, F8>();
+    case 16: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 16, FUSED, GS, F8>() : decode_kernel_ptr<__half, D, 16, FUSED, GS, F8>();
+    case 32: return bf16 ? decode_kernel_ptr<__nv_bfloat16, D, 32, FUSED, GS, F8>() : decode_kernel_ptr<__half, D, 32, FUSED, GS, F8>();
     default: return nullptr;
   }
 }
 
 template <int D>
-const void* kernel_for_variant(int block_size, bool bf16, bool fused, int gs) {
-  if (fused) return gs == 1 ? kernel_for<D, true, 1>(block_size, bf16) : nullptr;
+const void* kernel_for_variant(int block_size, bool bf16, bool fused, int gs, bool fp8) {
+  if (fp8) return gs == 1 && !fused ? kernel_for<D, false, 1, true>(block_size, bf16) : nullptr;
+  if (fused) return gs == 1 ? kernel_for<D, true, 1, false>(block_size, bf16) : nullptr;
   switch (gs) {
-    case 1: return kernel_for<D, false, 1>(block_size, bf16);
-    case 2: return kernel_for<D, false, 2>(block_size, bf16);
-    case 4: return kernel_for<D, false, 4>(block_size, bf16);
+    case 1: return kernel_for<D, false, 1, false>(block_size, bf16);
+    case 2: return kernel_for<D, false, 2, false>(block_size, bf16);
+    case 4: return kernel_for<D, false, 4, false>(block_size, bf16);
     default: return nullptr;
   }
 }
@@ -592,13 +625,16 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
     return 0;
   const HeadLayout hl = head_layout(num_heads, num_kv_heads);
   int64_t warps = 0;
-  for (int variant = 0; variant < 4; ++variant) {
-    const bool bf16 = variant & 1, fused = variant & 2;
-    if (fused && hl.gs != 1) continue;
-    const void* k = head_dim == 128 ? kernel_for_variant<128>(block_size, bf16, fused, hl.gs)
-                                    : kernel_for_variant<64>(block_size, bf16, fused, hl.gs);
+  // every kernel these sizes may run: fp16 / bf16, two calls / one launch,
+  // 16-bit / 8-bit cache
+  for (int variant = 0; variant < 8; ++variant) {
+    const bool bf16 = variant & 1, fused = variant & 2, fp8 = variant & 4;
+    if ((fused || fp8) && hl.gs != 1) continue;
+    if (fused && fp8) continue;
+    const void* k = head_dim == 128 ? kernel_for_variant<128>(block_size, bf16, fused, hl.gs, fp8)
+                                    : kernel_for_variant<64>(block_size, bf16, fused, hl.gs, fp8);
     const Plan pl = plan_variant(k, head_dim, block_size, num_seqs, hl.vheads, max_blocks_per_seq,
-                                 forced_warps, hl.gs);
+                                 forced_warps, hl.gs, fp8);
     if (pl.grid <= 0) return 0;
     if (pl.work_warps > warps) warps = pl.work_warps;
   }
@@ -622,7 +658,7 @@ cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
   // Grouped-query attention: tensor cores unless PA_OPT_GQA_KERNEL asks for
   // the CUDA cores (or the shape or pool does not suit them).
   const int64_t mode = option_gqa_kernel();
-  const bool mma_ok = !a.slot_mapping &&
+  const bool mma_ok = !a.slot_mapping && !a.fp8 &&
                       mma_decode_shape_ok(a.num_heads, a.num_kv_heads, a.head_dim, a.block_size) &&
                       mma_decode_pool_ok(a.num_kv_heads, a.block_size, a.num_blocks);
   if (mode == 2 && !mma_ok) return cudaErrorInvalidValue;

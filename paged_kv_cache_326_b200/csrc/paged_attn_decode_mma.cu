@@ -609,6 +609,7 @@ cudaError_t launch_mma_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStre
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
   p.qk_scale_log2 = a.scale * 1.4426950408889634f;  // log2(e)
+  p.v_scale = 1.f;
   p.num_seqs = a.num_seqs;
   p.num_heads = hl.vheads;
   p.num_q_heads = a.num_heads;

@@ -433,3 +433,60 @@ def cow_bursts(seed: int = 4, device="cpu", dtype=torch.float16, num_bursts: int
     g = _gen(seed + 1000003, dev)
     shape = (num_blocks, num_heads, block_size, head_dim)
     return _randn(shape, dtype, g, dev), _randn(shape, dtype, g, dev), bursts
+
+
+# ---------------------------------------------------------------------------
+# 8-bit (E4M3) caches
+# ---------------------------------------------------------------------------
+
+# Per-tensor scales of the 8-bit workloads: N(0,1) numbers divided by them
+# spread over about +-100, well inside E4M3's +-448, so no code saturates.
+FP8_K_SCALE = 0.05
+FP8_V_SCALE = 0.04
+NAN_CODE = 0x7F
+
+
+def to_codes(x: torch.Tensor, scale: float) -> torch.Tensor:
+    """E4M3 codes (uint8) of x / scale through torch's float8_e4m3fn cast
+    (round to nearest even), computed in fp32 on x's device."""
+    return (x.float() / scale).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def make_decode_fp8(name: str, context_lens: Sequence[int], num_heads: int, head_dim: int,
+                    block_size: int, num_blocks: int, dtype: torch.dtype, seed: int,
+                    device="cpu", max_blocks_per_seq: Optional[int] = None,
+                    k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE) -> DecodeInputs:
+    """make_decode with 8-bit caches: the pools hold E4M3 codes of seeded
+    N(0,1) numbers over the scales (``meta['k_scale']``, ``meta['v_scale']``);
+    rows that hold no earlier token hold the NaN code.  q, k, v stay in
+    ``dtype``."""
+    w = make_decode(name, context_lens, num_heads, head_dim, block_size, num_blocks, dtype, seed,
+                    device, max_blocks_per_seq, poison=False)
+    dev = w.q.device
+    g = _gen(seed + 2000003, dev)
+    shape = w.k_cache.shape
+    kc = torch.empty(shape, dtype=torch.uint8, device=dev)
+    vc = torch.empty(shape, dtype=torch.uint8, device=dev)
+    for dst, sc in ((kc, k_scale), (vc, v_scale)):
+        flat = dst.view(shape[0], -1)
+        step = max(1, (1 << 26) // flat.shape[1])
+        for i in range(0, shape[0], step):
+            j = min(shape[0], i + step)
+            flat[i:j] = to_codes(torch.randn((j - i, flat.shape[1]), generator=g, device=dev), sc)
+    fill = history_fill_of([w.block_tables], [w.context_lens], num_blocks, block_size, dev)
+    rows = torch.arange(block_size, device=dev)
+    dead = (rows[None, :] >= fill[:, None])[:, None, :, None]
+    kc.masked_fill_(dead, NAN_CODE)
+    vc.masked_fill_(dead, NAN_CODE)
+    w.k_cache, w.v_cache = kc, vc
+    w.name = name
+    w.meta.update(k_scale=k_scale, v_scale=v_scale)
+    return w
+
+
+def opt13b_batch64_fp8(seed: int = 2, device="cpu") -> DecodeInputs:
+    """The batch-64 OPT-13B-shaped step (lengths, tables, q, k, v as
+    opt13b_batch64) over 8-bit caches."""
+    return make_decode_fp8("opt13b_batch64_fp8", opt13b_batch64_lens(seed), num_heads=40,
+                           head_dim=128, block_size=16, num_blocks=8192, dtype=torch.float16,
+                           seed=seed, device=device, max_blocks_per_seq=128)

@@ -71,7 +71,8 @@ def oracle_inputs(q, k, v, k_cache, v_cache, block_tables, context_lens, slot_ma
     """Copy to the host only the pool blocks that the chosen texts reference,
     renumbered 0..n-1 (renumbering is pinned not to change the oracle's
     output), and the writes that land in them.  Call BEFORE the GPU step: the
-    pool must be the pre-write one."""
+    pool must be the pre-write one.  8-bit (uint8) pools are copied as raw
+    codes."""
     S = q.shape[0]
     seqs = np.arange(S) if seqs is None else np.asarray(seqs)
     sel = torch.as_tensor(seqs, device=block_tables.device, dtype=torch.long)
@@ -85,10 +86,11 @@ def oracle_inputs(q, k, v, k_cache, v_cache, block_tables, context_lens, slot_ma
     blk = (slots // block_size).clamp(min=0, max=N - 1)
     nb = torch.where(slots >= 0, remap[blk], torch.full_like(slots, -1))
     new_slots = torch.where(nb >= 0, nb * block_size + slots % block_size, torch.full_like(slots, -1))
+    pool = (lambda t: t.cpu().numpy()) if k_cache.dtype == torch.uint8 else host_f32
     return OracleInputs(
         q=host_f32(q.index_select(0, sel)), k=host_f32(k), v=host_f32(v),
-        k_cache=host_f32(k_cache.index_select(0, used)),
-        v_cache=host_f32(v_cache.index_select(0, used)),
+        k_cache=pool(k_cache.index_select(0, used)),
+        v_cache=pool(v_cache.index_select(0, used)),
         tables=new_t.cpu().numpy(), lens=context_lens.index_select(0, sel).cpu().numpy(),
         slots=new_slots.cpu().numpy(), seqs=seqs)
 
@@ -101,6 +103,31 @@ def run_oracle(oi: OracleInputs, scale: float, block_size: int, pairs=None) -> n
         pos = {int(s): i for i, s in enumerate(oi.seqs)}
         local_pairs = [(pos[int(s)], int(h)) for s, h in pairs]
     return oracle.paged_decode(oi.q, kc, vc, oi.tables, oi.lens, scale, block_size, local_pairs)
+
+
+def run_oracle_fp8(oi: OracleInputs, scale: float, block_size: int, k_scale: float,
+                   v_scale: float, pairs=None) -> np.ndarray:
+    """Oracle decode step over 8-bit caches (quantizing write, then attend)."""
+    kc, vc = oracle.cache_write_fp8(oi.k_cache, oi.v_cache, oi.k, oi.v, oi.slots, block_size,
+                                    k_scale, v_scale)
+    local_pairs = None
+    if pairs is not None:
+        pos = {int(s): i for i, s in enumerate(oi.seqs)}
+        local_pairs = [(pos[int(s)], int(h)) for s, h in pairs]
+    return oracle.paged_decode_fp8(oi.q, kc, vc, oi.tables, oi.lens, scale, block_size, k_scale,
+                                   v_scale, local_pairs)
+
+
+def gpu_step_fp8(w, status=None, out=None):
+    """Quantizing write, then decode, over the workload's 8-bit caches."""
+    import paged_kv_cache_326_b200 as P
+    ks, vs = w.meta["k_scale"], w.meta["v_scale"]
+    P.pa_kv_cache_write_fp8(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, ks, vs, status=status)
+    if out is None:
+        out = torch.empty_like(w.q)
+    P.pa_paged_attn_decode_fp8(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                               w.scale, ks, vs, status=status)
+    return out
 
 
 def gpu_step(w, status=None, out=None):

@@ -1,0 +1,148 @@
+"""The 8-bit (E4M3) KV cache on the GPU against the oracle: the quantizing
+write bit for bit over whole pools, decode attention within the fp16/bf16
+tolerance (the oracle attends over the same codes, widened exactly)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_326_b200 import workloads as W
+from tests.gpu_helpers import (compare, gpu_step_fp8, new_status, oracle_inputs, run_oracle_fp8)
+
+pytestmark = pytest.mark.gpu
+
+SHAPE_LENS = [0, 1, 3, 16, 17, 33, 64, 100, 129, 160]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    from paged_kv_cache_326_b200 import build
+    build.build()
+    import paged_kv_cache_326_b200 as P
+    return P.lib()
+
+
+def parity_fp8(w, seqs=None, heads_per_seq=None, seed=0):
+    S, H, D = w.q.shape
+    seqs = np.arange(S) if seqs is None else np.asarray(seqs)
+    pairs = None
+    if heads_per_seq is not None and heads_per_seq < H:
+        rng = np.random.default_rng(seed)
+        pairs = [(int(s), int(h)) for s in seqs for h in rng.choice(H, heads_per_seq, replace=False)]
+    oi = oracle_inputs(w.q, w.k, w.v, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                       w.slot_mapping, w.block_size, seqs)
+    kb, vb = w.k_cache.cpu().numpy(), w.v_cache.cpu().numpy()
+    st = new_status()
+    out = gpu_step_fp8(w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, st.item()
+    ks, vs = w.meta["k_scale"], w.meta["v_scale"]
+    ek, ev = oracle.cache_write_fp8(kb, vb, w.k.float().cpu().numpy(), w.v.float().cpu().numpy(),
+                                    w.slot_mapping.cpu().numpy(), w.block_size, ks, vs)
+    assert np.array_equal(w.k_cache.cpu().numpy(), ek), "8-bit k pool differs"
+    assert np.array_equal(w.v_cache.cpu().numpy(), ev), "8-bit v pool differs"
+    ref = run_oracle_fp8(oi, w.scale, w.block_size, ks, vs, pairs)
+    got = out.index_select(0, torch.as_tensor(seqs, device=out.device))
+    mask = None
+    if pairs is not None:
+        pos = {int(s): i for i, s in enumerate(seqs)}
+        mask = np.zeros((len(seqs), H, D), dtype=bool)
+        for s, h in pairs:
+            mask[pos[s], h] = True
+    c = compare(got, ref, w.q.dtype, mask)
+    assert c.ok, f"{w.name}: {c}"
+    return c
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("head_dim", [64, 128])
+@pytest.mark.parametrize("block_size", [4, 8, 16, 32])
+def test_fp8_every_shape_ragged(dtype, head_dim, block_size):
+    w = W.make_decode_fp8("fp8_shape", SHAPE_LENS, num_heads=3, head_dim=head_dim,
+                          block_size=block_size,
+                          num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in SHAPE_LENS),
+                          dtype=dtype, seed=head_dim + block_size, device="cuda",
+                          max_blocks_per_seq=160 // block_size)
+    parity_fp8(w)
+
+
+def test_fp8_opt13b_batch64():
+    w = W.opt13b_batch64_fp8(device="cuda")
+    c = parity_fp8(w, heads_per_seq=6, seed=3)
+    print("fp8 opt13b", c)
+
+
+def test_fp8_write_rounds_saturates_and_keeps_signs():
+    """Inputs at ties, past the largest code (saturating), subnormal and
+    signed zero, through both scales: codes equal the oracle's."""
+    import paged_kv_cache_326_b200 as P
+    H, D, B, N = 2, 64, 8, 4
+    ks, vs = 0.5, 2.0
+    base = torch.tensor([0.0, -0.0, 1.0625, 1.1875, 600.0, -1e4, 2.0 ** -11, 0.3, -2.5, 447.9],
+                        dtype=torch.float32)
+    row = torch.cat([base, torch.linspace(-300, 300, D - base.numel())])
+    k = torch.stack([row * ks, -row * ks]).view(1, 2, D).repeat(3, 1, 1).to(torch.float16)
+    v = torch.stack([row * vs, row * vs * 0.5]).view(1, 2, D).repeat(3, 1, 1).to(torch.float16)
+    kc = torch.full((N, H, B, D), 0x55, dtype=torch.uint8)
+    vc = kc.clone()
+    slots = torch.tensor([3, -1, 17])
+    ek, ev = oracle.cache_write_fp8(kc.numpy(), vc.numpy(), k.float().numpy(), v.float().numpy(),
+                                    slots.numpy(), B, ks, vs)
+    kd, vd = kc.cuda(), vc.cuda()
+    st = new_status()
+    P.pa_kv_cache_write_fp8(k.cuda(), v.cuda(), kd, vd, slots.cuda(), ks, vs, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert np.array_equal(kd.cpu().numpy(), ek) and np.array_equal(vd.cpu().numpy(), ev)
+
+
+def test_fp8_single_token_returns_its_value():
+    """One stored token: the output is value(code) * v_scale rounded to the
+    output type, bit for bit."""
+    w = W.make_decode_fp8("fp8_one", [1] * 6, num_heads=5, head_dim=128, block_size=16,
+                          num_blocks=16, dtype=torch.float16, seed=3, device="cuda")
+    out = gpu_step_fp8(w)
+    torch.cuda.synchronize()
+    vs = np.float32(w.meta["v_scale"])
+    codes = oracle.quantize(w.v.float().cpu().numpy(), vs)          # IEEE fp32 quotient
+    vals = torch.from_numpy(oracle.e4m3_decode(codes).astype(np.float32))
+    want = (vals * torch.tensor(vs)).to(out.dtype)                   # fp32 product, then RN
+    assert torch.equal(out.cpu(), want)
+
+
+def test_fp8_split_and_single_pass_agree():
+    import paged_kv_cache_326_b200 as P
+    for warps in (1, 4096):
+        P.pa_set_option(P.binding.PA_OPT_DECODE_WARPS, warps)
+        try:
+            parity_fp8(W.make_decode_fp8("fp8_split", [300, 17, 1, 1000, 64, 0, 511, 129],
+                                         num_heads=4, head_dim=128, block_size=16,
+                                         num_blocks=256, dtype=torch.bfloat16, seed=9,
+                                         device="cuda", max_blocks_per_seq=64))
+        finally:
+            P.pa_set_option(P.binding.PA_OPT_DECODE_WARPS, 0)
+
+
+def test_fp8_pools_copy_bit_exact():
+    import paged_kv_cache_326_b200 as P
+    g = torch.Generator().manual_seed(5)
+    kc = torch.randint(0, 256, (40, 3, 16, 128), generator=g, dtype=torch.uint8).cuda()
+    vc = torch.randint(0, 256, (40, 3, 16, 128), generator=g, dtype=torch.uint8).cuda()
+    pairs = [(1, 30), (2, 31), (2, 32), (39, 0)]
+    ek, ev = oracle.copy_blocks(kc.cpu().numpy(), vc.cpu().numpy(), kc.cpu().numpy(),
+                                vc.cpu().numpy(), pairs)
+    P.pa_copy_blocks(kc, vc, kc, vc, torch.tensor(pairs, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert np.array_equal(kc.cpu().numpy(), ek) and np.array_equal(vc.cpu().numpy(), ev)
+
+
+@pytest.mark.parametrize("bad", [0.0, -1.0, float("inf"), float("nan")])
+def test_fp8_scales_must_be_finite_and_positive(bad):
+    import paged_kv_cache_326_b200 as P
+    w = W.make_decode_fp8("fp8_bad", [5, 9], num_heads=2, head_dim=64, block_size=8,
+                          num_blocks=8, dtype=torch.float16, seed=1, device="cuda")
+    with pytest.raises(P.PagedAttnError):
+        P.pa_kv_cache_write_fp8(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, bad, 1.0)
+    with pytest.raises(P.PagedAttnError):
+        P.pa_paged_attn_decode_fp8(torch.empty_like(w.q), w.q, w.k_cache, w.v_cache,
+                                   w.block_tables, w.context_lens, w.scale, 1.0, bad)
