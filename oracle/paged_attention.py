@@ -33,6 +33,10 @@ Precision: inputs are the exact fp16/bf16 values widened to fp64; every step
 is fp64; softmax subtracts the maximum before exponentiating (an identity, so
 the result is the same number up to rounding).
 
+Prompt phase (``prefill``): causal attention of a prompt's tokens over the
+prompt itself, whose keys and values are then stored in the cache (the
+write is ``cache_write``).
+
 Block copies (``copy_blocks``): whole blocks copied from a source pool to a
 destination pool ("The KV Cache and PagedAttention", §Shared, Copied on
 Write: a text about to write into a block it shares gets its own copy of the
@@ -170,6 +174,39 @@ def paged_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
         full = attend(q[s][heads], K[:, sel, :], V[:, sel, :], scale)
         for i, h in enumerate(heads):
             out[s, h] = full[i]
+    return out
+
+
+def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: Sequence[int],
+            scale: float) -> np.ndarray:
+    """Prompt phase, fp64: every prompt's tokens attend causally over the
+    prompt's own keys and values ("The KV Cache and PagedAttention", §One Token
+    at a Time: the prompt is processed all at once, and its keys and values
+    are what later steps reuse; "KV cache", §How it works: position t attends
+    over positions 0..t).  Tokens of all prompts are packed: prompt s holds
+    rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of q ``[T][H][D]`` and of k, v
+    ``[T][H_kv][D]`` (query head h reads key/value head ``kv_head_of``).
+
+    For prompt s, head h and position t:
+        z_u = scale * q[t] . k[u] for u <= t,  out[t] = softmax(z) . v[0..t]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    T, H, D = q.shape
+    kvh = kv_head_of(H, k.shape[1])
+    out = np.zeros((T, H, D), dtype=np.float64)
+    for s in range(len(cu_seqlens) - 1):
+        a, b = int(cu_seqlens[s]), int(cu_seqlens[s + 1])
+        L = b - a
+        if L == 0:
+            continue
+        causal = np.tril(np.ones((L, L), dtype=bool))
+        for h in range(H):
+            z = float(scale) * (q[a:b, h, :] @ k[a:b, kvh[h], :].T)     # [L][L]
+            z = np.where(causal, z, -np.inf)
+            e = np.exp(z - z.max(axis=1, keepdims=True))
+            w = e / e.sum(axis=1, keepdims=True)
+            out[a:b, h, :] = w @ v[a:b, kvh[h], :]
     return out
 
 

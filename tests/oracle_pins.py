@@ -503,3 +503,71 @@ def pin_fp8_attention_on_representable_values(decode_fp8, quantize):
           for s, L in enumerate(lens)]
     ref = sdpa_contiguous(torch.from_numpy(q), Ks, Vs, 0.3)
     assert np.abs(got - ref).max() <= 1e-12, "8-bit cache attention vs exact values"
+
+
+# ---------------------------------------------------------------------------
+# prompt phase (prefill)
+# ---------------------------------------------------------------------------
+
+def _packed_prompts(lens, H, Hkv, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    T = sum(lens)
+    q = torch.randn(T, H, D, generator=g).to(torch.float16)
+    k = torch.randn(T, Hkv, D, generator=g).to(torch.float16)
+    v = torch.randn(T, Hkv, D, generator=g).to(torch.float16)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    return q, k, v, cu
+
+
+def pin_prefill_vs_torch_causal(prefill_fn):
+    """torch's fp64 attention with is_causal=True on each prompt (key/value
+    heads repeated for grouped-query prompts)."""
+    lens, H, Hkv, D = [1, 7, 20, 3], 4, 2, 16
+    q, k, v, cu = _packed_prompts(lens, H, Hkv, D, 501)
+    got = prefill_fn(f64(q), f64(k), f64(v), cu, 0.3)
+    for s in range(len(lens)):
+        a, b = cu[s], cu[s + 1]
+        qs = q[a:b].double().permute(1, 0, 2)
+        ks = k[a:b].double().repeat_interleave(H // Hkv, dim=1).permute(1, 0, 2)
+        vs = v[a:b].double().repeat_interleave(H // Hkv, dim=1).permute(1, 0, 2)
+        ref = torch.nn.functional.scaled_dot_product_attention(qs, ks, vs, is_causal=True,
+                                                               scale=0.3)
+        assert np.abs(got[a:b] - ref.permute(1, 0, 2).numpy()).max() <= 1e-12, "prefill vs sdpa"
+
+
+def pin_prefill_last_row_is_decode(prefill_fn):
+    """The prompt's last position sees the whole prompt: its output equals the
+    decode-phase attention of that token over the prompt stored in a paged
+    pool (the decode oracle, pinned on its own)."""
+    from oracle import paged_decode
+    lens, H, D, B = [9, 4, 13], 2, 8, 4
+    q, k, v, cu = _packed_prompts(lens, H, H, D, 511)
+    got = prefill_fn(f64(q), f64(k), f64(v), cu, 0.25)
+    Ks = [k[cu[s]:cu[s + 1]] for s in range(3)]
+    Vs = [v[cu[s]:cu[s + 1]] for s in range(3)]
+    kc, vc, tables = scatter_to_pool(Ks, Vs, B, 16, 512)
+    last = np.stack([f64(q[cu[s + 1] - 1]) for s in range(3)])
+    ref = paged_decode(last, f64(kc), f64(vc), tables, lens, 0.25, B)
+    for s in range(3):
+        assert np.abs(got[cu[s + 1] - 1] - ref[s]).max() <= 1e-12, "last row vs decode"
+
+
+def pin_prefill_first_row_and_brute_force(prefill_fn):
+    """Position 0 sees only itself: its output is its value, exactly.  Every
+    row of a tiny prompt against scalar brute force with math.fsum."""
+    lens, H, D = [5], 1, 4
+    q, k, v, cu = _packed_prompts(lens, H, H, D, 521)
+    got = prefill_fn(f64(q), f64(k), f64(v), cu, 0.5)
+    assert np.array_equal(got[0], f64(v[0])), "first row is not its value"
+    Q, K, V = f64(q)[:, 0], f64(k)[:, 0], f64(v)[:, 0]
+    for t in range(5):
+        z = [0.5 * math.fsum(Q[t, d] * K[u, d] for d in range(D)) for u in range(t + 1)]
+        m = max(z)
+        e = [math.exp(x - m) for x in z]
+        den = math.fsum(e)
+        want = [math.fsum(e[u] * V[u, d] for u in range(t + 1)) / den for d in range(D)]
+        assert np.abs(got[t, 0] - np.array(want)).max() <= 1e-12, f"row {t} vs brute force"
+
+
+PREFILL_PINS = [pin_prefill_vs_torch_causal, pin_prefill_last_row_is_decode,
+                pin_prefill_first_row_and_brute_force]

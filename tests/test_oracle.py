@@ -102,3 +102,8 @@ def test_fp8_cache_write_stores_the_codes_at_the_slots():
         ek[sl // B, :, sl % B] = oracle.e4m3_encode(k[t] / np.float32(0.5))
         ev[sl // B, :, sl % B] = oracle.e4m3_encode(v[t] / np.float32(0.125))
     assert np.array_equal(k2, ek) and np.array_equal(v2, ev)
+
+
+@pytest.mark.parametrize("pin", P.PREFILL_PINS, ids=lambda f: f.__name__)
+def test_prefill_pin(pin):
+    pin(oracle.prefill)

@@ -296,3 +296,42 @@ def quantize_multiplying(x, scale):
 def test_planted_scale_mistake_is_caught():
     with pytest.raises(AssertionError):
         P.pin_fp8_attention_on_representable_values(oracle.paged_decode_fp8, quantize_multiplying)
+
+
+# --- prompt phase: planted mistakes -------------------------------------------
+
+def prefill_not_causal(q, k, v, cu, scale):
+    """Planted mistake: every position sees the whole prompt."""
+    out = np.zeros(q.shape)
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        for t in range(a, b):
+            out[t] = oracle.attend(q[t], k[a:b], v[a:b], scale)
+    return out
+
+
+def prefill_excludes_self(q, k, v, cu, scale):
+    """Planted mistake: position t sees 0..t-1 only (the first sees nothing)."""
+    out = np.zeros(q.shape)
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        for t in range(a, b):
+            out[t] = oracle.attend(q[t], k[a:t], v[a:t], scale)
+    return out
+
+
+def prefill_crosses_prompts(q, k, v, cu, scale):
+    """Planted mistake: the prompts are treated as one long prompt."""
+    return oracle.prefill(q, k, v, [0, cu[-1]], scale)
+
+
+@pytest.mark.parametrize("fn", [prefill_not_causal, prefill_excludes_self,
+                                prefill_crosses_prompts], ids=lambda f: f.__name__)
+def test_planted_prefill_mistake_is_caught(fn):
+    failed = 0
+    for pin in P.PREFILL_PINS:
+        try:
+            pin(fn)
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    assert failed, fn.__name__
