@@ -239,6 +239,121 @@ def run_reference(args, world, rank):
     return 0
 
 
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return (float(json.load(f)["bf16_tflops"]),
+                    "measured (MEASURED_PEAKS.json bf16_tflops: cuBLAS dense, burst; fp16 runs "
+                    "at the same tensor rate)")
+    except Exception:
+        return 1590.0, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+
+
+def run_prefill_bench(args, ranks, world, rank, local):
+    """The prompt phase: 16 prompts of 2,048 tokens x 40 heads x 128, fp16 --
+    each step stores the prompts' keys and values in their blocks and runs
+    causal attention (pa_prefill)."""
+    import paged_kv_cache_326_b200 as P
+    from paged_kv_cache_326_b200 import dist, workloads as W
+    P.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    w = W.opt13b_prefill(seed=dist.batch_seed(7, ranks), device=dev)
+    T, H, D = w.q.shape
+    flops = 4.0 * D * H * sum(L * (L + 1) / 2 for L in w.lens)   # causal QK^T and PV
+    out = torch.empty_like(w.q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        P.pa_prefill(out, w.q, w.k, w.v, w.cu_seqlens, w.max_seqlen, w.scale, w.k_cache,
+                     w.v_cache, w.slot_mapping, status=status)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    K = args.steps
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        dist.barrier(ranks)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(K):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier(ranks)
+    clk = clocks.summary()
+    ms_step = start.elapsed_time(stop) / K
+    # end to end: q, k, v from pinned host memory, out back to the host
+    hq, hk, hv = (t.cpu().pin_memory() for t in (w.q, w.k, w.v))
+    hout = torch.empty_like(hq).pin_memory()
+    Ke = max(1, K // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Ke):
+        w.q.copy_(hq, non_blocking=True)
+        w.k.copy_(hk, non_blocking=True)
+        w.v.copy_(hv, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    ms_step, e2e_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms], dev)
+    peak, peak_src = tensor_peak()
+    tflops = flops / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": "prefill TFLOP/s (causal attention, 4*D flops per query-key pair)",
+        "value": world * tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
+        "data": "synthetic",
+        "config": {"workload": "opt13b_prefill", "prompts": len(w.lens), "prompt_len": w.lens[0],
+                   "num_heads": H, "head_dim": D, "block_size": w.block_size,
+                   "l2": "q, k, v, out 1.3 GB per step >> 126 MB L2",
+                   "parallelism": f"independent prompts per GPU x{world}",
+                   "path": "pa_prefill (cache write + causal attention)"},
+        "prefill_tokens_per_s": world * T / (ms_step * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None,
+                     "kernel": "prefill_kernel (mma.sync m16n8k16) + kv_cache_write_kernel",
+                     "peak_source": peak_src, "algorithmic_flops_per_launch": flops},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": 3 * w.q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        # one prompt's first 512 tokens, 4 heads: about ten seconds of host work
+        L, Hs = 512, 4
+        q = w.q[:L, :Hs].float().cpu().numpy()
+        k = w.k[:L, :Hs].float().cpu().numpy()
+        v = w.v[:L, :Hs].float().cpu().numpy()
+        sample_flops = 4.0 * D * Hs * L * (L + 1) / 2
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.prefill(q, k, v, [0, L], w.scale)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= 10.0 or reps >= 200:
+                break
+        line["cpu_baseline"] = {
+            "value": sample_flops * reps / el / 1e12, "unit": "TFLOP/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"one prompt's first {L} tokens x {Hs} heads, {reps} run(s), {el:.1f} s, "
+                      f"numpy fp64 (BLAS threads as installed)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_cow_copy(args, ranks, world, rank, local):
     """Copy-on-write bursts: each step copies one burst of 224 whole blocks
     (32 prompts x 7 samples, 40 heads x 16 x 128 fp16, K and V) with
@@ -365,10 +480,12 @@ def main():
                     help="fp8: the batch-64 step over 8-bit E4M3 caches (two calls)")
     ap.add_argument("--gqa-kernel", choices=["auto", "cores", "tensor"], default="auto",
                     help="grouped-query workload: kernel choice (PA_OPT_GQA_KERNEL)")
-    ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa", "cow_copy"],
+    ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa", "cow_copy",
+                                           "prefill"],
                     default="opt13b_batch64",
                     help="llama2_70b_gqa: 64 query heads on 8 key/value heads (two calls); "
-                         "cow_copy: copy-on-write bursts of whole blocks (pa_copy_blocks)")
+                         "cow_copy: copy-on-write bursts of whole blocks (pa_copy_blocks); "
+                         "prefill: the prompt phase of 16 prompts of 2,048 tokens (pa_prefill)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -382,6 +499,10 @@ def main():
 
     if args.workload == "cow_copy":
         rc = run_cow_copy(args, ranks, world, rank, local)
+        dist.finish(ranks)
+        return rc
+    if args.workload == "prefill":
+        rc = run_prefill_bench(args, ranks, world, rank, local)
         dist.finish(ranks)
         return rc
 

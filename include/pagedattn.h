@@ -266,6 +266,39 @@ int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, cons
                              size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
 
 /*
+ * pa_prefill — the prompt phase: every prompt's tokens attend causally over
+ * the prompt's own keys and values, which are also stored in their blocks
+ * ("The KV Cache and PagedAttention", section "One Token at a Time": the
+ * prompt is processed all at once, and its keys and values are what later
+ * steps reuse; "KV cache", section "How it works": position t attends over
+ * positions 0..t).  Prompts are packed: prompt s is rows cu_seqlens[s] ..
+ * cu_seqlens[s+1]-1 of q, k, v and out.  For prompt s, query head h and
+ * position t (query head h reads key/value head h / (num_heads/num_kv_heads)):
+ *     out[t][h] = sum_{u <= t in prompt s} softmax_u(scale * q[t][h] . k[u]) v[u].
+ * Arithmetic: products on the tensor cores with fp32 sums, online softmax in
+ * fp32; for bf16 the softmax weights enter the weighted sum of values as two
+ * bf16 values (about 16 significant bits).
+ *
+ *   out, q         [num_tokens][num_heads][head_dim] dt, device
+ *   k, v           [num_tokens][num_kv_heads][head_dim] dt, device
+ *   cu_seqlens     [num_seqs + 1] int32, device: 0 = cu[0] <= cu[1] <= ... <=
+ *                  cu[num_seqs] = num_tokens (a prompt outside [0,
+ *                  num_tokens] is skipped with PA_ERR_BAD_LEN in *d_status)
+ *   max_seqlen     at least the longest prompt (a longer one is reported as
+ *                  PA_ERR_BAD_LEN and its tail positions are not computed)
+ *   k_cache, v_cache, slot_mapping, block_size, num_blocks
+ *                  the pool and each token's slot, as for pa_kv_cache_write;
+ *                  k_cache NULL skips the store (attention only)
+ * Support: head_dim 64 or 128; num_seqs <= 65535.  Returns PA_OK or
+ * PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_cache,
+               void* v_cache, const int64_t* slot_mapping, const int32_t* cu_seqlens,
+               int num_seqs, int num_tokens, int max_seqlen, float scale, int num_heads,
+               int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, pa_dtype dt,
+               int32_t* d_status, pa_stream_t stream);
+
+/*
  * pa_copy_blocks — copy whole blocks from one pool to another, or within one
  * pool: the device side of copy-on-write ("The KV Cache and
  * PagedAttention", section "Shared, Copied on Write": before a text writes

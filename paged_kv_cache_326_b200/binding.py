@@ -77,6 +77,8 @@ _SIGNATURES = {
                                      _i64, _i32, _vp, _vp]),
     "pa_paged_attn_decode_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _f32, _f32, _i32, _i32,
                                         _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
+    "pa_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _f32, _i32,
+                          _i32, _i32, _i32, _i64, _i32, _vp, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32,
                               _vp, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
@@ -223,6 +225,40 @@ def pa_paged_attn_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.
         float(v_scale), S, H, D, B, MB, N, _dtype_code(q), _cuda(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _status_ptr(status), _stream(stream, q.device))
     _check(code, "pa_paged_attn_decode_fp8")
+    return out
+
+
+def pa_prefill(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+               cu_seqlens: torch.Tensor, max_seqlen: int, scale: float,
+               k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
+               slot_mapping: Optional[torch.Tensor] = None,
+               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Prompt phase over packed prompts: out, q [T][H][D]; k, v [T][H_kv][D];
+    cu_seqlens [S+1] int32.  With caches and slot_mapping [T] int64, the
+    prompts' keys and values are stored in their blocks first."""
+    T, H, D = q.shape
+    Tk, Hkv, Dk = k.shape
+    if out.shape != q.shape or v.shape != k.shape or Tk != T or Dk != D or H % Hkv:
+        raise ValueError("shape mismatch")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be [num_seqs + 1]")
+    for t in (out, k, v):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v and out must share a dtype")
+    S = cu_seqlens.numel() - 1
+    B, N, kc, vc, sm = 16, 0, None, None, None
+    if k_cache is not None:
+        N, Hc, B, Dc = k_cache.shape
+        if v_cache is None or slot_mapping is None or v_cache.shape != k_cache.shape or \
+                (Hc, Dc) != (Hkv, D) or slot_mapping.shape != (T,) or k_cache.dtype != q.dtype:
+            raise ValueError("caches must be [N][H_kv][B][D] of q's dtype with slot_mapping [T]")
+        kc, vc = _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache")
+        sm = _cuda(slot_mapping, "slot_mapping", torch.int64)
+    code = lib().pa_prefill(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), kc, vc, sm,
+        _cuda(cu_seqlens, "cu_seqlens", torch.int32), S, T, int(max_seqlen), float(scale), H, Hkv,
+        D, B, N, _dtype_code(q), _status_ptr(status), _stream(stream, q.device))
+    _check(code, "pa_prefill")
     return out
 
 

@@ -218,6 +218,46 @@ int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, cons
                        true, k_scale, v_scale);
 }
 
+int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_cache,
+               void* v_cache, const int64_t* slot_mapping, const int32_t* cu_seqlens,
+               int num_seqs, int num_tokens, int max_seqlen, float scale, int num_heads,
+               int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, pa_dtype dt,
+               int32_t* d_status, pa_stream_t stream) {
+  if (num_seqs < 0 || num_seqs > 65535 || num_tokens < 0 || max_seqlen < 0 ||
+      num_heads < 1 || num_heads > 65535 || num_kv_heads < 1 || num_heads % num_kv_heads ||
+      (head_dim != 64 && head_dim != 128) || (dt != PA_F16 && dt != PA_BF16))
+    return PA_ERR_INVALID;
+  if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+  if (!out || !q || !k || !v || !cu_seqlens) return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return PA_ERR_INVALID;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (k_cache) {  // store the prompts' keys and values in their blocks first
+    if (!v_cache || !slot_mapping || !shape_ok(num_kv_heads, head_dim, block_size) ||
+        num_blocks <= 0 || !aligned16(k_cache) || !aligned16(v_cache))
+      return PA_ERR_INVALID;
+    const int rc = from_cuda(pa::launch_kv_cache_write(k, v, k_cache, v_cache, slot_mapping,
+                                                       num_tokens, num_kv_heads, head_dim,
+                                                       block_size, num_blocks, d_status, st));
+    if (rc != PA_OK) return rc;
+  }
+  pa::PrefillArgs a;
+  a.out = out;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.cu_seqlens = cu_seqlens;
+  a.num_seqs = num_seqs;
+  a.num_tokens = num_tokens;
+  a.max_seqlen = max_seqlen;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.scale = scale;
+  a.is_bf16 = dt == PA_BF16;
+  a.status = d_status;
+  return from_cuda(pa::launch_prefill(a, st));
+}
+
 int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks, void* dst_k,
                    void* dst_v, int64_t dst_num_blocks, const int32_t* block_pairs,
                    int num_pairs, int num_heads, int head_dim, int block_size, pa_dtype dt,

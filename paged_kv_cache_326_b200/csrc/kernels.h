@@ -28,6 +28,25 @@ cudaError_t launch_copy_blocks(const void* src_k, const void* src_v, void* dst_k
                                int64_t src_num_blocks, int64_t dst_num_blocks, int32_t* status,
                                cudaStream_t stream);
 
+// Prompt phase: causal attention within each packed prompt (prefill.cu).
+struct PrefillArgs {
+  void* out;
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* cu_seqlens;
+  int num_seqs;
+  int num_tokens;
+  int max_seqlen;
+  int num_heads;
+  int num_kv_heads;
+  int head_dim;
+  float scale;
+  int is_bf16;
+  int32_t* status;
+};
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+
 struct DecodeArgs {
   void* out;
   const void* q;

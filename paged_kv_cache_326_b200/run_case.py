@@ -7,8 +7,9 @@ For profilers: it makes no timing claims.  Workloads: ``opt13b_batch64``
 (optionally cut to the first S texts, pool sized 1.5x what they need),
 ``tiny``, ``skewed`` (bf16, blocks of 16), ``llama2_70b_gqa`` (64 query heads
 on 8 key/value heads; always the two-call path, the one-launch step being
-multi-head only).  ``--gqa-kernel`` picks its kernel (0 automatic, 1 CUDA
-cores, 2 tensor cores).
+multi-head only), ``opt13b_batch64_fp8`` (the batch-64 step over 8-bit
+caches, two calls).  ``--gqa-kernel`` picks the grouped-query kernel (0
+automatic, 1 CUDA cores, 2 tensor cores).
 """
 from __future__ import annotations
 
@@ -25,6 +26,8 @@ def make(name: str, num_seqs: int, device):
         return W.tiny(device=device)
     if name == "skewed":
         return W.skewed(device=device)
+    if name == "opt13b_batch64_fp8":
+        return W.opt13b_batch64_fp8(device=device)
     if name == "llama2_70b_gqa":
         return W.llama2_70b_gqa(device=device, num_seqs=num_seqs if num_seqs > 0 else 64)
     if name == "opt13b_batch64":
@@ -49,11 +52,18 @@ def main():
     dev = torch.device("cuda", 0)
     w = make(args.workload, args.num_seqs, dev)
     gqa = w.k_cache.shape[1] != w.num_heads
+    fp8 = w.k_cache.dtype == torch.uint8
     P.pa_set_option(P.PA_OPT_GQA_KERNEL, args.gqa_kernel)
     out = torch.empty_like(w.q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     for _ in range(args.reps):
-        if gqa:
+        if fp8:
+            ks, vs = w.meta["k_scale"], w.meta["v_scale"]
+            P.pa_kv_cache_write_fp8(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, ks, vs,
+                                    status=status)
+            P.pa_paged_attn_decode_fp8(out, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                       w.context_lens, w.scale, ks, vs, status=status)
+        elif gqa:
             P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
             P.pa_paged_attn_decode_gqa(out, w.q, w.k_cache, w.v_cache, w.block_tables,
                                        w.context_lens, w.scale, status=status)
@@ -67,7 +77,8 @@ def main():
     torch.cuda.synchronize()
     if status.item() != 0:
         raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
-    kv = sum(w.context_lens.tolist()) * 2 * w.k_cache.shape[1] * w.head_dim * w.q.element_size()
+    kv = (sum(w.context_lens.tolist()) * 2 * w.k_cache.shape[1] * w.head_dim *
+          w.k_cache.element_size())
     print(f"{w.name}: {w.num_seqs} texts, KV bytes per step {kv}, status ok")
 
 

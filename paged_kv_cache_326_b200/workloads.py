@@ -490,3 +490,71 @@ def opt13b_batch64_fp8(seed: int = 2, device="cpu") -> DecodeInputs:
     return make_decode_fp8("opt13b_batch64_fp8", opt13b_batch64_lens(seed), num_heads=40,
                            head_dim=128, block_size=16, num_blocks=8192, dtype=torch.float16,
                            seed=seed, device=device, max_blocks_per_seq=128)
+
+
+# ---------------------------------------------------------------------------
+# Prompt phase (prefill)
+# ---------------------------------------------------------------------------
+
+@dataclass
+class PrefillInputs:
+    """Packed prompts: prompt s is rows cu_seqlens[s]..cu_seqlens[s+1]-1."""
+
+    name: str
+    q: torch.Tensor             # [T][H][D]
+    k: torch.Tensor             # [T][H_kv][D]
+    v: torch.Tensor             # [T][H_kv][D]
+    cu_seqlens: torch.Tensor    # [S+1] int32
+    max_seqlen: int
+    k_cache: torch.Tensor       # [N][H_kv][B][D], NaN before the store
+    v_cache: torch.Tensor
+    slot_mapping: torch.Tensor  # [T] int64: each token's slot through its prompt's table
+    block_tables: torch.Tensor  # [S][max_blocks] int32
+    scale: float
+    block_size: int
+    lens: List[int]
+
+
+def make_prefill(name: str, lens: Sequence[int], num_heads: int, num_kv_heads: int,
+                 head_dim: int, dtype: torch.dtype, seed: int, device="cpu",
+                 block_size: int = 16, spare_blocks: int = 8) -> PrefillInputs:
+    """Seeded N(0,1) prompts packed back to back; each prompt gets blocks from
+    a seeded permutation of a pool with ``spare_blocks`` extra blocks, and
+    token t of prompt s has slot table[s][t // B] * B + t % B."""
+    dev = torch.device(device)
+    lens = [int(x) for x in lens]
+    T, S = sum(lens), len(lens)
+    nb = [blocks_needed(L, block_size) for L in lens]
+    N = sum(nb) + spare_blocks
+    order = torch.randperm(N, generator=_gen(seed, "cpu"))
+    mb = max([1] + nb)
+    tables = torch.full((S, mb), -1, dtype=torch.int32)
+    slots = torch.empty(T, dtype=torch.int64)
+    at = pos = 0
+    for s, L in enumerate(lens):
+        tables[s, :nb[s]] = order[at:at + nb[s]].to(torch.int32)
+        at += nb[s]
+        t = torch.arange(L)
+        slots[pos:pos + L] = tables[s, t // block_size].to(torch.int64) * block_size + t % block_size
+        pos += L
+    g = _gen(seed + 1000003, dev)
+    q = _randn((max(T, 1), num_heads, head_dim), dtype, g, dev)[:T]
+    k = _randn((max(T, 1), num_kv_heads, head_dim), dtype, g, dev)[:T]
+    v = _randn((max(T, 1), num_kv_heads, head_dim), dtype, g, dev)[:T]
+    cache_shape = (N, num_kv_heads, block_size, head_dim)
+    k_cache = torch.full(cache_shape, NAN16, dtype=dtype, device=dev)
+    v_cache = torch.full(cache_shape, NAN16, dtype=dtype, device=dev)
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    return PrefillInputs(name=name, q=q.contiguous(), k=k.contiguous(), v=v.contiguous(),
+                         cu_seqlens=cu.to(dev), max_seqlen=max([0] + lens), k_cache=k_cache,
+                         v_cache=v_cache, slot_mapping=slots.to(dev), block_tables=tables.to(dev),
+                         scale=fp32_scale(head_dim), block_size=block_size, lens=lens)
+
+
+def opt13b_prefill(seed: int = 7, device="cpu", num_prompts: int = 16,
+                   prompt_len: int = 2048) -> PrefillInputs:
+    """OPT-13B-shaped prompt phase: 16 prompts of 2,048 tokens (the model's
+    longest), 40 heads of 128, fp16, blocks of 16."""
+    return make_prefill("opt13b_prefill", [prompt_len] * num_prompts, num_heads=40,
+                        num_kv_heads=40, head_dim=128, dtype=torch.float16, seed=seed,
+                        device=device)
