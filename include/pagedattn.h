@@ -277,7 +277,8 @@ int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, cons
  *     out[t][h] = sum_{u <= t in prompt s} softmax_u(scale * q[t][h] . k[u]) v[u].
  * Arithmetic: products on the tensor cores with fp32 sums, online softmax in
  * fp32; for bf16 the softmax weights enter the weighted sum of values as two
- * bf16 values (about 16 significant bits).
+ * bf16 values (about 16 significant bits).  Every wait is bounded
+ * (PA_OPT_WAIT_LIMIT_NS); one that gives up records PA_ERR_TIMEOUT.
  *
  *   out, q         [num_tokens][num_heads][head_dim] dt, device
  *   k, v           [num_tokens][num_kv_heads][head_dim] dt, device
@@ -381,9 +382,14 @@ int pa_paged_attn_decode_noalloc(void* out, const void* q, const void* k_cache,
  *                         tensor-core kernel carries the softmax weights into
  *                         the weighted sum of values as the sum of two dt
  *                         values (about 16 significant bits).
+ *   PA_OPT_PREFILL_KERNEL which kernel pa_prefill runs: 0 (default) or 2 the
+ *                         5th-generation tensor cores (tcgen05, accumulators
+ *                         in tensor memory, 128 queries per CTA); 1 the
+ *                         warp-level tensor cores (mma.sync).  Same function.
  * Returns PA_OK or PA_ERR_INVALID for an unknown key or value.
  */
-enum { PA_OPT_WAIT_LIMIT_NS = 1, PA_OPT_DECODE_WARPS = 2, PA_OPT_GQA_KERNEL = 3 };
+enum { PA_OPT_WAIT_LIMIT_NS = 1, PA_OPT_DECODE_WARPS = 2, PA_OPT_GQA_KERNEL = 3,
+       PA_OPT_PREFILL_KERNEL = 4 };
 int pa_set_option(int key, int64_t value);
 
 /* ------------------------------------------------------------------------ */

@@ -39,6 +39,7 @@ PA_E4M3 = 2
 PA_OPT_WAIT_LIMIT_NS = 1
 PA_OPT_DECODE_WARPS = 2
 PA_OPT_GQA_KERNEL = 3
+PA_OPT_PREFILL_KERNEL = 4
 
 _KIND = {PA_ERR_INVALID: "invalid", PA_ERR_CUDA: "cuda", PA_ERR_OUT_OF_BLOCKS: "out_of_blocks",
          PA_ERR_NO_SEQ: "no_seq", PA_ERR_EXISTS: "exists", PA_ERR_TABLE_FULL: "table_full",

@@ -14,6 +14,7 @@ namespace {
 std::atomic<int64_t> g_wait_limit_ns{1000000000};
 std::atomic<int64_t> g_decode_warps{0};
 std::atomic<int64_t> g_gqa_kernel{0};
+std::atomic<int64_t> g_prefill_kernel{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -53,6 +54,7 @@ int from_cuda(cudaError_t e) {
 namespace pa {
 int64_t option_decode_warps() { return g_decode_warps.load(); }
 int64_t option_gqa_kernel() { return g_gqa_kernel.load(); }
+int64_t option_prefill_kernel() { return g_prefill_kernel.load(); }
 }  // namespace pa
 
 extern "C" {
@@ -86,6 +88,10 @@ int pa_set_option(int key, int64_t value) {
     case PA_OPT_GQA_KERNEL:
       if (value < 0 || value > 2) return PA_ERR_INVALID;
       g_gqa_kernel = value;
+      return PA_OK;
+    case PA_OPT_PREFILL_KERNEL:
+      if (value < 0 || value > 2) return PA_ERR_INVALID;
+      g_prefill_kernel = value;
       return PA_OK;
     default: return PA_ERR_INVALID;
   }
@@ -255,7 +261,9 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
   a.scale = scale;
   a.is_bf16 = dt == PA_BF16;
   a.status = d_status;
-  return from_cuda(pa::launch_prefill(a, st));
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  return from_cuda(g_prefill_kernel.load() == 1 ? pa::launch_prefill(a, st)
+                                                : pa::launch_prefill_tc(a, st));
 }
 
 int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks, void* dst_k,

@@ -1,5 +1,6 @@
 // Internal launcher declarations shared by the C-ABI layer and the kernels.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -14,6 +15,14 @@ cudaError_t launch_kv_cache_write_fp8(const void* k, const void* v, void* k_cach
                                       int num_tokens, int num_heads, int head_dim, int block_size,
                                       int64_t num_blocks, bool bf16, int32_t* status,
                                       cudaStream_t stream);
+
+// A tiled TMA map of a 16-bit (fp16 or bf16) tensor of `rank` dimensions
+// (innermost first; strides in bytes of dimensions 1..rank-1), boxes of
+// `box` elements, 128-byte swizzle, zero fill out of bounds.  False if the
+// driver refuses it.
+bool encode_swizzled_map(CUtensorMap* map, const void* base, bool bf16, int rank,
+                         const uint64_t* dims, const uint64_t* strides_bytes,
+                         const uint32_t* box);
 
 cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
                                   const int64_t* slot_mapping, int num_tokens, int num_heads,
@@ -44,8 +53,14 @@ struct PrefillArgs {
   float scale;
   int is_bf16;
   int32_t* status;
+  int64_t wait_limit_ns = 1000000000;
 };
+// Warp-level tensor cores (mma.sync, prefill.cu) and 5th-generation tensor
+// cores (tcgen05 with TMEM accumulators, prefill_tc.cu).
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
+// Current PA_OPT_PREFILL_KERNEL setting (0 automatic = tcgen05, 1 mma.sync, 2 tcgen05).
+int64_t option_prefill_kernel();
 
 struct DecodeArgs {
   void* out;

@@ -22,6 +22,19 @@ def lib():
     return P.lib()
 
 
+# PA_OPT_PREFILL_KERNEL values: 5th-generation tensor cores, warp-level MMA
+PREFILL_KERNELS = {"tcgen05": 2, "mma": 1}
+
+
+@pytest.fixture(params=list(PREFILL_KERNELS))
+def prefill_kernel(request):
+    """Run the test once on each prefill kernel."""
+    import paged_kv_cache_326_b200 as P
+    P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, PREFILL_KERNELS[request.param])
+    yield request.param
+    P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, 0)
+
+
 def run_prefill(w, status=None, store=True):
     import paged_kv_cache_326_b200 as P
     out = torch.empty_like(w.q)
@@ -58,15 +71,15 @@ def check(w, rows=None):
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
 @pytest.mark.parametrize("head_dim", [64, 128])
 @pytest.mark.parametrize("heads", [(4, 4), (8, 2), (6, 1)], ids=lambda hk: f"q{hk[0]}kv{hk[1]}")
-def test_prefill_ragged_prompts(dtype, head_dim, heads):
+def test_prefill_ragged_prompts(dtype, head_dim, heads, prefill_kernel):
     Hq, Hkv = heads
     w = W.make_prefill("prefill", LENS, Hq, Hkv, head_dim, dtype, seed=head_dim + Hq,
                        device="cuda")
     c = check(w)
-    print(f"prefill {dtype} D{head_dim} q{Hq}kv{Hkv}", c)
+    print(f"prefill {prefill_kernel} {dtype} D{head_dim} q{Hq}kv{Hkv}", c)
 
 
-def test_prefill_opt13b_sampled_rows():
+def test_prefill_opt13b_sampled_rows(prefill_kernel):
     """16 prompts of 2,048 tokens x 40 heads: a sample of rows spread over
     every tile, the diagonal ones and each prompt's last."""
     w = W.opt13b_prefill(device="cuda", num_prompts=4)
@@ -74,10 +87,10 @@ def test_prefill_opt13b_sampled_rows():
     rows = sorted(set(rng.choice(w.q.shape[0], 64, replace=False).tolist()) |
                   {int(x) - 1 for x in w.cu_seqlens[1:].tolist()} | {0, 63, 64, 2047, 2048})
     c = check(w, rows)
-    print("prefill opt13b", c)
+    print(f"prefill {prefill_kernel} opt13b", c)
 
 
-def test_prefill_first_position_returns_its_value():
+def test_prefill_first_position_returns_its_value(prefill_kernel):
     for dtype in (torch.float16, torch.bfloat16):
         w = W.make_prefill("first", [5, 1, 70], 4, 2, 128, dtype, seed=3, device="cuda")
         out = run_prefill(w, store=False)
@@ -87,7 +100,7 @@ def test_prefill_first_position_returns_its_value():
             assert torch.equal(out[a], w.v[a].repeat_interleave(2, dim=0)), dtype
 
 
-def test_prefill_bad_offsets_and_short_max_seqlen_are_reported():
+def test_prefill_bad_offsets_and_short_max_seqlen_are_reported(prefill_kernel):
     import paged_kv_cache_326_b200 as P
     w = W.make_prefill("bad", [10, 20], 2, 2, 64, torch.float16, seed=4, device="cuda")
     st = new_status()
@@ -140,3 +153,43 @@ def test_prefill_then_decode_continues_the_prompt():
     ref = oracle.paged_decode(host_f32(q), kc, vc, t2.cpu().numpy(), ctx.cpu().numpy(), w.scale, B)
     c = compare(out, ref, torch.float16)
     assert c.ok, c
+
+
+def test_prefill_kernels_agree_and_are_deterministic():
+    """Both prefill kernels compute the same function: equal within the
+    tolerance; each bitwise reproducible run to run."""
+    import paged_kv_cache_326_b200 as P
+    w = W.make_prefill("agree", [700, 129, 1, 64], 8, 2, 128, torch.bfloat16, seed=8,
+                       device="cuda")
+    res = {}
+    try:
+        for name, mode in PREFILL_KERNELS.items():
+            P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, mode)
+            a = run_prefill(w, store=False)
+            b = run_prefill(w, store=False)
+            torch.cuda.synchronize()
+            assert torch.equal(a, b), name
+            res[name] = a
+    finally:
+        P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, 0)
+    diff = (res["tcgen05"].float() - res["mma"].float()).abs().max().item()
+    assert diff <= 2e-2, diff
+
+
+def test_prefill_tcgen05_wait_limit_gives_up_cleanly():
+    """A wait limit below zero makes every barrier wait give up at once: the
+    kernel records PA_ERR_TIMEOUT, drains what it issued, frees its tensor
+    memory and returns; the next call is correct."""
+    import paged_kv_cache_326_b200 as P
+    w = W.make_prefill("timeout", [200, 70], 4, 4, 128, torch.float16, seed=9, device="cuda")
+    st = new_status()
+    P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, 2)
+    P.pa_set_option(P.binding.PA_OPT_WAIT_LIMIT_NS, -1)
+    try:
+        run_prefill(w, st, store=False)
+        torch.cuda.synchronize()
+    finally:
+        P.pa_set_option(P.binding.PA_OPT_WAIT_LIMIT_NS, 1_000_000_000)
+        P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, 0)
+    assert st.item() == P.binding.PA_ERR_TIMEOUT
+    check(W.make_prefill("after", [200, 70], 4, 4, 128, torch.float16, seed=9, device="cuda"))
