@@ -321,7 +321,7 @@ def run_prefill_bench(args, ranks, world, rank, local):
         "prefill_tokens_per_s": world * T / (ms_step * 1e-3),
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "traffic": None,
-                     "kernel": "prefill_kernel (mma.sync m16n8k16) + kv_cache_write_kernel",
+                     "kernel": "prefill_tc_kernel (tcgen05, TMEM accumulators) + kv_cache_write_kernel",
                      "peak_source": peak_src, "algorithmic_flops_per_launch": flops},
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 3 * w.q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
