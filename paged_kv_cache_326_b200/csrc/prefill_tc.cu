@@ -6,27 +6,33 @@
 //     out[t][h] = sum_{u <= t} softmax_u(scale * q[t][h] . k[u]) v[u],
 // query head h reading key/value head h / (Hq / Hkv).
 //
-// How (one CTA = 128 queries of one (prompt, head); 128 threads, one query
-// row each; two CTAs per SM):
-//   * Q (128 x D) and each 64-key block of K and V arrive by 3-D tiled TMA
-//     (the [T][H][D] tensors seen as (D, H, T); boxes 64 x 1 x rows, 128-byte
-//     swizzle) into shared memory; K and V are double-buffered in stages.
-//   * S = Q K^T: thread 0 issues tcgen05.mma (M = 128, N = 64, K = 16 per
-//     instruction, both operands K-major in shared memory) into tensor memory
-//     (TMEM); a commit signals an mbarrier.
-//   * Softmax: each thread reads its query's 64 scores from TMEM (its warp's
-//     32 lanes), so the row max and sum need no shuffles.  Base 2; the
-//     running max is raised only when a score passes it by more than 2^8,
-//     which then rescales that row of O in TMEM.  P (and for bf16 the rest
-//     P - P_hi, so P enters as about 16 significant bits) is written back to
-//     TMEM as packed 16-bit pairs.
-//   * O += P V: tcgen05.mma with A = P from TMEM and B = V (MN-major: head_dim
-//     contiguous) from shared memory; O accumulates in TMEM.
-//   * After the last block each thread reads its row of O, divides by its
+// How (FlashAttention-4's arrangement on sm_100a): one CTA takes two tiles of
+// 128 queries of one (prompt, head), 256 consecutive queries, and runs ten
+// warps with separate jobs:
+//   * warp 9 (one thread) loads: Q of both tiles once, then each 64-key block
+//     of K and V into a 3-stage ring, by 3-D tiled TMA (the [T][H][D] tensors
+//     seen as (D, H, T); boxes 64 x 1 x rows; 128-byte swizzle);
+//   * warp 8 (one thread) issues the tensor-core products, tcgen05.mma
+//     kind::f16, accumulating in tensor memory (TMEM): S_t = Q_t K^T (both
+//     operands K-major in shared memory) and O_t += P_t V (P_t from TMEM, V
+//     MN-major in shared memory), in the order S0, S1, then per block PV0,
+//     S0', PV1, S1': while one tile's softmax runs, the tensor pipe works on
+//     the other tile's products;
+//   * warps 0-3 and 4-7: the softmax of tile 0 and tile 1, one thread per
+//     query row (its warp's 32 TMEM lanes), so the row max and sum stay in
+//     the thread.  Base 2; the running max is raised only when a score
+//     passes it by more than 2^8, which then rescales that row of O in TMEM.
+//     P (and for bf16 the rest P - P_hi, so P enters as about 16 significant
+//     bits) goes back to TMEM as packed 16-bit pairs.
+//   * After its last block each softmax thread divides its row of O by its
 //     sum and stores it.
-// TMEM per CTA: S 64 columns, P 32 (+ 32 for bf16's low part), O head_dim.
-// Every wait is bounded: a wait that gives up records PA_ERR_TIMEOUT, the CTA
-// drains what it issued (bounded too), frees its TMEM and returns.
+// Barriers: per stage full (TMA bytes) and empty (last product that reads
+// it); per tile S ready, P ready (128 arrivals) and O done.  TMEM loads are
+// issued in groups of four under one wait.  TMEM per tile:
+// S 64 columns, P 32 + 32, O head_dim; 512 in all, one CTA per SM.
+// Every wait is bounded: a wait that gives up records PA_ERR_TIMEOUT and
+// raises a CTA-wide abort flag; each role then drains what it issued
+// (bounded), TMEM is freed and the CTA returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -44,21 +50,25 @@ namespace pa {
 
 namespace {
 
-constexpr int kTcThreads = 128;  // one per query row
-constexpr int kTcBM = 128;       // queries per CTA (MMA M)
-constexpr int kTcBN = 64;        // keys per block (MMA N of S, K of P V)
-constexpr uint32_t kColS = 0, kColPhi = 64, kColPlo = 96, kColO = 128, kTmemCols = 256;
+constexpr int kTcBM = 128;      // queries per tile (MMA M)
+constexpr int kTcBN = 64;       // keys per block (MMA N of S, K of P V)
+constexpr int kTcTiles = 2;     // query tiles per CTA
+constexpr int kTcStages = 3;    // K/V ring depth
+constexpr int kTcThreads = 320; // 8 softmax warps, the MMA warp, the load warp
+constexpr int kMmaWarp = 8, kLoadWarp = 9;
+constexpr uint32_t kColS = 0, kColPhi = 64, kColPlo = 96, kColO = 128;
+constexpr uint32_t kTileCols = 256, kTmemCols = 512;
 constexpr int64_t kTcDrainNs = 1000000000;
 
 template <int D>
 struct TcLayout {
-  static constexpr int HALVES = D / 64;             // 64-element (128-byte) column blocks
-  static constexpr int Q_BYTES = kTcBM * D * 2;     // 32 KB at head_dim 128
-  static constexpr int KV_BYTES = kTcBN * D * 2;    // 16 KB
-  static constexpr int STAGE = 2 * KV_BYTES;        // K block, then V block
-  // shared memory asked for: + 1 KB to align by hand; sized for head_dim 128
-  // at every head_dim, which keeps two CTAs (2 x 256 TMEM columns) per SM
-  static constexpr int SMEM = 1024 + 128 * 128 * 2 + 2 * 2 * 64 * 128 * 2;
+  static constexpr int HALVES = D / 64;           // 64-element (128-byte) column blocks
+  static constexpr int Q_BYTES = kTcBM * D * 2;   // one tile of Q: 32 KB at head_dim 128
+  static constexpr int KV_BYTES = kTcBN * D * 2;  // one block of K (or V): 16 KB
+  static constexpr int STAGE = 2 * KV_BYTES;      // K block, then V block
+  // shared memory asked for (+ 1 KB to align by hand): the head_dim-128
+  // amount at every head_dim, so one CTA holds an SM (its 512 TMEM columns)
+  static constexpr int SMEM = 1024 + kTcTiles * (kTcBM * 128 * 2) + kTcStages * (2 * kTcBN * 128 * 2);
 };
 
 struct TcParams {
@@ -74,7 +84,7 @@ struct TcParams {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kTcThreads, 2)
+__global__ void __launch_bounds__(kTcThreads, 1)
 prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using LY = TcLayout<D>;
@@ -84,10 +94,12 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 128-byte swizzle patterns repeat every 1024 bytes of shared address: align by hand
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + LY::Q_BYTES;
-  __shared__ uint64_t bar_q, bar_kv[2], bar_s, bar_o;
+  uint8_t* sQ = smem;                               // tile t at t * Q_BYTES
+  uint8_t* sKV = smem + kTcTiles * LY::Q_BYTES;     // stage i at i * STAGE
+  __shared__ uint64_t bar_q, bar_full[kTcStages], bar_empty[kTcStages];
+  __shared__ uint64_t bar_s[kTcTiles], bar_p[kTcTiles], bar_o[kTcTiles];
   __shared__ uint32_t tmem_base;
+  __shared__ volatile int abort_flag;
 
   griddep_wait();
   const int s = blockIdx.z, h = blockIdx.y;
@@ -99,22 +111,35 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   const int L = b - a;
   if (L > p.max_seqlen && blockIdx.x == 0 && h == 0 && threadIdx.x == 0)
     set_status(p.status, -8 /* PA_ERR_BAD_LEN: a prompt longer than max_seqlen */);
-  const int tile = gridDim.x - 1 - blockIdx.x;  // heaviest tiles first
-  if (tile * kTcBM >= L) return;                 // the whole CTA leaves: nothing allocated yet
+  const int pair = gridDim.x - 1 - blockIdx.x;       // heaviest pairs of tiles first
+  const int q0 = pair * kTcTiles * kTcBM;            // first query of tile 0
+  if (q0 >= L) return;                               // the whole CTA leaves: nothing allocated
   const int kvh = h / (p.Hq / p.Hkv);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int q_end = min(L, (tile + 1) * kTcBM);  // this tile's queries end here
-  const int nkb = (q_end + kTcBN - 1) / kTcBN;   // key blocks up to the diagonal
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // key blocks each tile needs (keys up to its last query); tile 1 may be empty
+  int nkb_t[kTcTiles];
+#pragma unroll
+  for (int t = 0; t < kTcTiles; ++t) {
+    const int lo = q0 + t * kTcBM;
+    const int hi = min(L, lo + kTcBM);
+    nkb_t[t] = lo < L ? (hi + kTcBN - 1) / kTcBN : 0;
+  }
+  const int nkb = nkb_t[kTcTiles - 1] > 0 ? nkb_t[kTcTiles - 1] : nkb_t[0];
 
   if (tid == 0) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+    abort_flag = 0;
     mbar_init(&bar_q, 1);
-    mbar_init(&bar_kv[0], 1);
-    mbar_init(&bar_kv[1], 1);
-    mbar_init(&bar_s, 1);
-    mbar_init(&bar_o, 1);
+#pragma unroll
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 1);
+    }
+#pragma unroll
+    for (int t = 0; t < kTcTiles; ++t) {
+      mbar_init(&bar_s[t], 1);
+      mbar_init(&bar_p[t], kTcBM);
+      mbar_init(&bar_o[t], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 0) tc::alloc(&tmem_base, kTmemCols);
@@ -122,103 +147,174 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_base;
-  const uint32_t row_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-
-  // Producer bookkeeping (thread 0): what was issued, for the drain.
-  int kv_issued = 0, s_commits = 0, o_commits = 0;
-  auto load_kv = [&](int j) {  // key block j into stage j % 2
-    uint8_t* st = sKV + (j & 1) * LY::STAGE;
-    uint64_t* bar = &bar_kv[j & 1];
-    mbar_arrive_expect_tx(bar, LY::STAGE);
-#pragma unroll
-    for (int hf = 0; hf < LY::HALVES; ++hf) {
-      tc::tma_load_3d(st + hf * (kTcBN * 128), &tm_k, hf * 64, kvh, a + j * kTcBN, bar);
-      tc::tma_load_3d(st + LY::KV_BYTES + hf * (kTcBN * 128), &tm_v, hf * 64, kvh, a + j * kTcBN,
-                      bar);
-    }
-    ++kv_issued;
+  const int64_t lim = p.wait_limit_ns;
+  auto give_up = [&]() {
+    set_status(p.status, -10 /* PA_ERR_TIMEOUT */);
+    abort_flag = 1;
   };
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bar_q, LY::Q_BYTES);
-#pragma unroll
-    for (int hf = 0; hf < LY::HALVES; ++hf)
-      tc::tma_load_3d(sQ + hf * (kTcBM * 128), &tm_q, hf * 64, h, a + tile * kTcBM, &bar_q);
-    load_kv(0);
-  }
+  // a bounded wait that also ends once the CTA has given up
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (abort_flag) return false;
+    if (!mbar_wait_bounded(bar, parity, lim)) {
+      give_up();
+      return false;
+    }
+    return true;
+  };
 
-  const int qpos = tile * kTcBM + tid;  // this thread's query, within the prompt
-  float m = -INFINITY, l = 0.f;
-  bool failed = false;
-  int j = 0;
-  for (; j < nkb; ++j) {
-    // ---- S = Q K^T (thread 0 issues) ----
-    if (tid == 0 && !failed) {
-      bool ok = mbar_wait_bounded(&bar_kv[j & 1], (j >> 1) & 1, p.wait_limit_ns);
-      if (ok && j == 0) ok = mbar_wait_bounded(&bar_q, 0, p.wait_limit_ns);
-      if (!ok) {
-        failed = true;
-      } else {
-        const uint32_t q0 = smem_addr(sQ), k0 = smem_addr(sKV + (j & 1) * LY::STAGE);
+  if (warp == kLoadWarp) {
+    // ---------------- loads ----------------
+    if (lane == 0) {
+      tc::prefetch_map(&tm_q);
+      tc::prefetch_map(&tm_k);
+      tc::prefetch_map(&tm_v);
+      const int nq = nkb_t[1] > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(&bar_q, nq * LY::Q_BYTES);
+      for (int t = 0; t < nq; ++t)
+#pragma unroll
+        for (int hf = 0; hf < LY::HALVES; ++hf)
+          tc::tma_load_3d(sQ + t * LY::Q_BYTES + hf * (kTcBM * 128), &tm_q, hf * 64, h,
+                          a + q0 + t * kTcBM, &bar_q);
+      int issued = 0;
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j % kTcStages;
+        if (j >= kTcStages && !wait(&bar_empty[st], ((j / kTcStages) - 1) & 1)) break;
+        uint8_t* dst = sKV + st * LY::STAGE;
+        mbar_arrive_expect_tx(&bar_full[st], LY::STAGE);
+#pragma unroll
+        for (int hf = 0; hf < LY::HALVES; ++hf) {
+          tc::tma_load_3d(dst + hf * (kTcBN * 128), &tm_k, hf * 64, kvh, a + j * kTcBN,
+                          &bar_full[st]);
+          tc::tma_load_3d(dst + LY::KV_BYTES + hf * (kTcBN * 128), &tm_v, hf * 64, kvh,
+                          a + j * kTcBN, &bar_full[st]);
+        }
+        issued = j + 1;
+      }
+      // drain: the copies in flight must land before this CTA's memory goes
+      mbar_wait_bounded(&bar_q, 0, kTcDrainNs);
+      for (int j = issued > kTcStages ? issued - kTcStages : 0; j < issued; ++j)
+        mbar_wait_bounded(&bar_full[j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------- tensor-core products ----------------
+    if (lane == 0) {
+      const uint32_t qa = smem_addr(sQ);
+      int s_done[kTcTiles] = {0, 0}, o_done[kTcTiles] = {0, 0}, empties = 0;
+      auto issue_s = [&](int t, int j) -> bool {  // S_t = Q_t K_j^T
+        // (the previous block's scores were read: its P is written, P V issued)
+        if (!wait(&bar_full[j % kTcStages], (j / kTcStages) & 1)) return false;
+        tc::fence_after_sync();
+        const uint32_t q = qa + t * LY::Q_BYTES;
+        const uint32_t k = smem_addr(sKV + (j % kTcStages) * LY::STAGE);
+        const uint32_t d = tmem + t * kTileCols + kColS;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          tc::mma_ss(tmem + kColS,
-                     tc::smem_desc(q0 + (ks >> 2) * (kTcBM * 128) + (ks & 3) * 32, 16, 1024),
-                     tc::smem_desc(k0 + (ks >> 2) * (kTcBN * 128) + (ks & 3) * 32, 16, 1024),
+          tc::mma_ss(d, tc::smem_desc(q + (ks >> 2) * (kTcBM * 128) + (ks & 3) * 32, 16, 1024),
+                     tc::smem_desc(k + (ks >> 2) * (kTcBN * 128) + (ks & 3) * 32, 16, 1024),
                      IDESC_S, ks > 0);
-        tc::commit(&bar_s);
-        ++s_commits;
+        tc::commit(&bar_s[t]);
+        ++s_done[t];
+        return true;
+      };
+      auto issue_pv = [&](int t, int j) -> bool {  // O_t += P_t V_j
+        if (!wait(&bar_p[t], j & 1)) return false;
+        tc::fence_after_sync();
+        const uint32_t v = smem_addr(sKV + (j % kTcStages) * LY::STAGE + LY::KV_BYTES);
+        const uint32_t base = tmem + t * kTileCols;
+#pragma unroll
+        for (int ks = 0; ks < kTcBN / 16; ++ks) {
+          const uint64_t dv = tc::smem_desc(v + ks * 2048, kTcBN * 128, 1024);
+          tc::mma_ts(base + kColO, base + kColPhi + ks * 8, dv, IDESC_O, j > 0 || ks > 0);
+          if constexpr (BF16) tc::mma_ts(base + kColO, base + kColPlo + ks * 8, dv, IDESC_O, true);
+        }
+        tc::commit(&bar_o[t]);
+        ++o_done[t];
+        return true;
+      };
+      bool ok = wait(&bar_q, 0);
+      for (int t = 0; t < kTcTiles && ok; ++t)
+        if (nkb_t[t] > 0) ok = issue_s(t, 0);
+      for (int j = 0; j < nkb && ok; ++j) {
+        for (int t = 0; t < kTcTiles && ok; ++t) {
+          if (j >= nkb_t[t]) continue;
+          ok = issue_pv(t, j);
+          if (ok && j + 1 < nkb_t[t]) ok = issue_s(t, j + 1);
+        }
+        if (ok) {
+          tc::commit(&bar_empty[j % kTcStages]);  // block j's stage is read for good
+          empties = j + 1;
+        }
+      }
+      // drain: every product issued must finish, and every commit arrive,
+      // before TMEM and this CTA's shared memory are given up
+      for (int j = empties > kTcStages ? empties - kTcStages : 0; j < empties; ++j)
+        mbar_wait_bounded(&bar_empty[j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
+#pragma unroll
+      for (int t = 0; t < kTcTiles; ++t) {
+        if (s_done[t] > 0) mbar_wait_bounded(&bar_s[t], (s_done[t] - 1) & 1, kTcDrainNs);
+        if (o_done[t] > 0) mbar_wait_bounded(&bar_o[t], (o_done[t] - 1) & 1, kTcDrainNs);
       }
     }
-    // ---- softmax of this thread's row ----
-    // tcgen05.ld/st are warp-collective: every guard around them is made
-    // uniform across the warp by a vote
-    float sv[kTcBN];
-    if (!failed) failed = !mbar_wait_bounded(&bar_s, j & 1, p.wait_limit_ns);
-    failed = __any_sync(0xffffffffu, failed);
-    tc::fence_after_sync();
-    if (!failed) {
+  } else {
+    // ---------------- softmax of one query row ----------------
+    const int t = warp >> 2;                     // tile of this warpgroup
+    const int row = tid & (kTcBM - 1);           // row within the tile = TMEM lane
+    const int qpos = q0 + t * kTcBM + row;       // query position within the prompt
+    const uint32_t rbase = tmem + t * kTileCols + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    float m = -INFINITY, l = 0.f;
+    bool failed = false;
+    const int nk = nkb_t[t];
+    for (int j = 0; j < nk; ++j) {
+      // tcgen05.ld/st are warp-collective: guards around them are warp-uniform
+      failed = __any_sync(0xffffffffu, failed || !wait(&bar_s[t], j & 1));
+      if (failed) break;
+      tc::fence_after_sync();
+      float sv[kTcBN];
+      {
+        // four loads in flight, one wait
+        uint32_t v[kTcBN / 16][16];
 #pragma unroll
-      for (int c0 = 0; c0 < kTcBN; c0 += 16) {
-        uint32_t v[16];
-        tc::ld16(row_addr + kColS + c0, v);
+        for (int i = 0; i < kTcBN / 16; ++i) tc::ld16(rbase + kColS + i * 16, v[i]);
         tc::wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; ++c) sv[c0 + c] = __uint_as_float(v[c]);
-      }
-    }
-    float rmax = -INFINITY;
+        for (int i = 0; i < kTcBN / 16; ++i)
 #pragma unroll
-    for (int c = 0; c < kTcBN; ++c) {
-      const int key = j * kTcBN + c;
-      sv[c] = key <= qpos ? sv[c] * p.scale_log2 : -INFINITY;
-      rmax = fmaxf(rmax, sv[c]);
-    }
-    // P and O are still in use by the previous block's P V until it completes
-    if (j > 0 && !failed) failed = !mbar_wait_bounded(&bar_o, (j - 1) & 1, p.wait_limit_ns);
-    failed = __any_sync(0xffffffffu, failed);
-    tc::fence_after_sync();
-    if (tid == 0 && !failed && j + 1 < nkb) load_kv(j + 1);  // its stage held block j - 1
-    // Raise the running max of a row only past a slack of 2^8; a row whose
-    // max rises after the first block rescales its O (the whole warp takes
-    // part in the TMEM traffic, with factor 1 on rows that do not rise).
-    const bool raise = rmax > m + 8.f;
-    const float m_new = raise ? rmax : m;
-    const float alpha = raise && m != -INFINITY ? fast_exp2(m - m_new) : 1.f;
-    if (!failed && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          for (int c = 0; c < 16; ++c) sv[i * 16 + c] = __uint_as_float(v[i][c]);
+      }
+      float rmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTcBN; ++c) {
+        const int key = j * kTcBN + c;
+        sv[c] = key <= qpos ? sv[c] * p.scale_log2 : -INFINITY;
+        rmax = fmaxf(rmax, sv[c]);
+      }
+      // P_t and O_t are in use by the previous block's product until it is done
+      if (j > 0) {
+        failed = __any_sync(0xffffffffu, !wait(&bar_o[t], (j - 1) & 1));
+        if (failed) break;
+        tc::fence_after_sync();
+      }
+      const bool raise = rmax > m + 8.f;
+      const float m_new = raise ? rmax : m;
+      const float alpha = raise && m != -INFINITY ? fast_exp2(m - m_new) : 1.f;
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t v[16];
-        tc::ld16(row_addr + kColO + c0, v);
-        tc::wait_ld();
+        for (int c0 = 0; c0 < D; c0 += 64) {
+          uint32_t v[4][16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * alpha);
-        tc::st16(row_addr + kColO + c0, v);
+          for (int i = 0; i < 4; ++i) tc::ld16(rbase + kColO + c0 + i * 16, v[i]);
+          tc::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              v[i][c] = __float_as_uint(__uint_as_float(v[i][c]) * alpha);
+            tc::st16(rbase + kColO + c0 + i * 16, v[i]);
+          }
+        }
       }
-      tc::wait_st();
-    }
-    l *= alpha;
-    m = m_new;
-    {
+      l *= alpha;
+      m = m_new;
       const float mm = m == -INFINITY ? 0.f : m;
       uint32_t ph[32], pl[32];
 #pragma unroll
@@ -231,79 +327,50 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
           pl[c / 2] = Elem<T>::from_float2(p0 - back.x, p1 - back.y);
         }
       }
+      tc::st16(rbase + kColPhi, *reinterpret_cast<uint32_t(*)[16]>(ph));
+      tc::st16(rbase + kColPhi + 16, *reinterpret_cast<uint32_t(*)[16]>(ph + 16));
+      if constexpr (BF16) {
+        tc::st16(rbase + kColPlo, *reinterpret_cast<uint32_t(*)[16]>(pl));
+        tc::st16(rbase + kColPlo + 16, *reinterpret_cast<uint32_t(*)[16]>(pl + 16));
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      mbar_arrive(&bar_p[t]);
+    }
+    if (!failed && nk > 0) {
+      // ---- epilogue: out = O / l ----
+      failed = __any_sync(0xffffffffu, !wait(&bar_o[t], (nk - 1) & 1));
       if (!failed) {
-        tc::st16(row_addr + kColPhi, *reinterpret_cast<uint32_t(*)[16]>(ph));
-        tc::st16(row_addr + kColPhi + 16, *reinterpret_cast<uint32_t(*)[16]>(ph + 16));
-        if constexpr (BF16) {
-          tc::st16(row_addr + kColPlo, *reinterpret_cast<uint32_t(*)[16]>(pl));
-          tc::st16(row_addr + kColPlo + 16, *reinterpret_cast<uint32_t(*)[16]>(pl + 16));
-        }
-        tc::wait_st();
-      }
-    }
-    tc::fence_before_sync();
-    if (__syncthreads_or(failed ? 1 : 0)) {
-      failed = true;
-      break;
-    }
-    tc::fence_after_sync();
-    // ---- O += P V (thread 0 issues) ----
-    if (tid == 0) {
-      const uint32_t v0 = smem_addr(sKV + (j & 1) * LY::STAGE + LY::KV_BYTES);
-#pragma unroll
-      for (int ks = 0; ks < kTcBN / 16; ++ks) {
-        const uint64_t dv = tc::smem_desc(v0 + ks * 2048, kTcBN * 128, 1024);
-        tc::mma_ts(tmem + kColO, tmem + kColPhi + ks * 8, dv, IDESC_O, j > 0 || ks > 0);
-        if constexpr (BF16) tc::mma_ts(tmem + kColO, tmem + kColPlo + ks * 8, dv, IDESC_O, true);
-      }
-      tc::commit(&bar_o);
-      ++o_commits;
-    }
-  }
-
-  if (!failed) {
-    // ---- epilogue: out = O / l ----
-    failed = !mbar_wait_bounded(&bar_o, (nkb - 1) & 1, p.wait_limit_ns);
-    failed = __any_sync(0xffffffffu, failed);
-    tc::fence_after_sync();
-    if (!failed) {
-      const bool store = qpos < L;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      T* orow = static_cast<T*>(p.out) + (static_cast<int64_t>(a + qpos) * p.Hq + h) * D;
+        tc::fence_after_sync();
+        const bool store = qpos < L;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        T* orow = static_cast<T*>(p.out) + (static_cast<int64_t>(a + qpos) * p.Hq + h) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t v[16];
-        tc::ld16(row_addr + kColO + c0, v);
-        tc::wait_ld();
-        float f[8];
-        if (store) {
+        for (int c0 = 0; c0 < D; c0 += 64) {
+          uint32_t v[4][16];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(v[k]) * inv;
-          *reinterpret_cast<uint4*>(orow + c0) = pack8<T>(f);
+          for (int i = 0; i < 4; ++i) tc::ld16(rbase + kColO + c0 + i * 16, v[i]);
+          tc::wait_ld();
+          if (store) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(v[8 + k]) * inv;
-          *reinterpret_cast<uint4*>(orow + c0 + 8) = pack8<T>(f);
+            for (int i = 0; i < 4; ++i) {
+              float f[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(v[i][k]) * inv;
+              *reinterpret_cast<uint4*>(orow + c0 + i * 16) = pack8<T>(f);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(v[i][8 + k]) * inv;
+              *reinterpret_cast<uint4*>(orow + c0 + i * 16 + 8) = pack8<T>(f);
+            }
+          }
         }
       }
-    }
-  }
-  if (failed) {
-    if (tid == 0) {
-      set_status(p.status, -10 /* PA_ERR_TIMEOUT */);
-      // drain what this CTA issued before its memory goes away (bounded):
-      // the last load into each stage, the last commit of each barrier
-      for (int i = kv_issued > 2 ? kv_issued - 2 : 0; i < kv_issued; ++i)
-        mbar_wait_bounded(&bar_kv[i & 1], (i >> 1) & 1, kTcDrainNs);
-      mbar_wait_bounded(&bar_q, 0, kTcDrainNs);
-      if (s_commits > 0) mbar_wait_bounded(&bar_s, (s_commits - 1) & 1, kTcDrainNs);
-      if (o_commits > 0) mbar_wait_bounded(&bar_o, (o_commits - 1) & 1, kTcDrainNs);
     }
   }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tc::dealloc(tmem, kTmemCols);
 }
-
 template <typename T, int D>
 cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
   using LY = TcLayout<D>;
@@ -321,7 +388,7 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
       raised.insert(dev);
     }
   }
-  const int tiles = (a.max_seqlen + kTcBM - 1) / kTcBM;
+  const int tiles = (a.max_seqlen + kTcTiles * kTcBM - 1) / (kTcTiles * kTcBM);  // pairs
   if (tiles <= 0) return cudaSuccess;
   // q as (D, Hq, T), k and v as (D, Hkv, T); boxes 64 x 1 x rows
   CUtensorMap tq, tk, tv;
@@ -332,7 +399,7 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
                           static_cast<uint64_t>(a.num_heads) * D * 2};
   const uint64_t sk[2] = {static_cast<uint64_t>(D) * 2,
                           static_cast<uint64_t>(a.num_kv_heads) * D * 2};
-  const uint32_t bq[3] = {64u, 1u, static_cast<uint32_t>(kTcBM)};
+  const uint32_t bq[3] = {64u, 1u, static_cast<uint32_t>(kTcBM)};  // one tile of Q
   const uint32_t bk[3] = {64u, 1u, static_cast<uint32_t>(kTcBN)};
   const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   if (!encode_swizzled_map(&tq, a.q, bf16, 3, dq, sq, bq) ||

@@ -1,7 +1,7 @@
 // Thin wrappers over the sm_90+/sm_100a PTX used by the kernels: shared-memory
 // mbarriers, the bulk (TMA) global->shared copy, proxy fences, the global
-// timer.  No tensor maps: every tile this library moves is one contiguous run
-// of bytes, so the untiled cp.async.bulk form is enough.  No multicast.
+// timer.  (Tiled tensor-map copies live in mma_ptx.cuh and tcgen05.cuh.)  No
+// multicast.
 #pragma once
 #include <cstdint>
 
@@ -31,6 +31,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
                    smem_addr(bar)),
                "r"(bytes)
+               : "memory");
+}
+
+// A plain arrival (release at CTA scope), no transaction bytes.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
                : "memory");
 }
 

@@ -109,6 +109,11 @@ __device__ __forceinline__ void wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Bring a tensor map (a __grid_constant__ parameter) into the descriptor cache.
+__device__ __forceinline__ void prefetch_map(const void* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 // 3-D tiled TMA load (no multicast) into shared memory, counted on `bar`.
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, int y, int z,
                                             uint64_t* bar) {

@@ -8,8 +8,10 @@ For profilers: it makes no timing claims.  Workloads: ``opt13b_batch64``
 ``tiny``, ``skewed`` (bf16, blocks of 16), ``llama2_70b_gqa`` (64 query heads
 on 8 key/value heads; always the two-call path, the one-launch step being
 multi-head only), ``opt13b_batch64_fp8`` (the batch-64 step over 8-bit
-caches, two calls).  ``--gqa-kernel`` picks the grouped-query kernel (0
-automatic, 1 CUDA cores, 2 tensor cores).
+caches, two calls), ``opt13b_prefill`` (the prompt phase: S prompts of 2,048
+tokens, 40 heads of 128; ``--prefill-kernel`` 0 automatic, 1 mma.sync, 2
+tcgen05).  ``--gqa-kernel`` picks the grouped-query kernel (0 automatic, 1
+CUDA cores, 2 tensor cores).
 """
 from __future__ import annotations
 
@@ -48,8 +50,22 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
     ap.add_argument("--gqa-kernel", type=int, choices=[0, 1, 2], default=0)
+    ap.add_argument("--prefill-kernel", type=int, choices=[0, 1, 2], default=0)
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
+    if args.workload == "opt13b_prefill":
+        P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, args.prefill_kernel)
+        w = W.opt13b_prefill(device=dev, num_prompts=args.num_seqs if args.num_seqs > 0 else 16)
+        out = torch.empty_like(w.q)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        for _ in range(args.reps):
+            P.pa_prefill(out, w.q, w.k, w.v, w.cu_seqlens, w.max_seqlen, w.scale, w.k_cache,
+                         w.v_cache, w.slot_mapping, status=status)
+        torch.cuda.synchronize()
+        if status.item() != 0:
+            raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
+        print(f"{len(w.lens)} prompts of {w.lens[0]} tokens, status ok")
+        return
     w = make(args.workload, args.num_seqs, dev)
     gqa = w.k_cache.shape[1] != w.num_heads
     fp8 = w.k_cache.dtype == torch.uint8
