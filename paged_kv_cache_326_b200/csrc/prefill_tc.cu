@@ -281,13 +281,16 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int c = 0; c < 16; ++c) sv[i * 16 + c] = __uint_as_float(v[i][c]);
       }
+      // keys past this query exist only in the diagonal blocks
+      if (j * kTcBN + kTcBN - 1 > qpos) {
+#pragma unroll
+        for (int c = 0; c < kTcBN; ++c)
+          if (j * kTcBN + c > qpos) sv[c] = -INFINITY;
+      }
       float rmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kTcBN; ++c) {
-        const int key = j * kTcBN + c;
-        sv[c] = key <= qpos ? sv[c] * p.scale_log2 : -INFINITY;
-        rmax = fmaxf(rmax, sv[c]);
-      }
+      for (int c = 0; c < kTcBN; ++c) rmax = fmaxf(rmax, sv[c]);
+      rmax *= p.scale_log2;  // base-2 logits: the scale (> 0) is applied in the exponent
       // P_t and O_t are in use by the previous block's product until it is done
       if (j > 0) {
         failed = __any_sync(0xffffffffu, !wait(&bar_o[t], (j - 1) & 1));
@@ -319,7 +322,9 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       uint32_t ph[32], pl[32];
 #pragma unroll
       for (int c = 0; c < kTcBN; c += 2) {
-        const float p0 = fast_exp2(sv[c] - mm), p1 = fast_exp2(sv[c + 1] - mm);
+        // 2^(scale * s - m): one fma per score (masked scores are -inf: weight 0)
+        const float p0 = fast_exp2(fmaf(sv[c], p.scale_log2, -mm));
+        const float p1 = fast_exp2(fmaf(sv[c + 1], p.scale_log2, -mm));
         l += p0 + p1;
         ph[c / 2] = Elem<T>::from_float2(p0, p1);
         if constexpr (BF16) {
