@@ -287,10 +287,12 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
         for (int c = 0; c < kTcBN; ++c)
           if (j * kTcBN + c > qpos) sv[c] = -INFINITY;
       }
-      float rmax = -INFINITY;
+      // four independent partial maxima: no 64-long dependent chain
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kTcBN; ++c) rmax = fmaxf(rmax, sv[c]);
-      rmax *= p.scale_log2;  // base-2 logits: the scale (> 0) is applied in the exponent
+      for (int c = 0; c < kTcBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+      // base-2 logits: the scale (> 0) is applied in the exponent
+      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
       // P_t and O_t are in use by the previous block's product until it is done
       if (j > 0) {
         failed = __any_sync(0xffffffffu, !wait(&bar_o[t], (j - 1) & 1));
@@ -320,18 +322,20 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       m = m_new;
       const float mm = m == -INFINITY ? 0.f : m;
       uint32_t ph[32], pl[32];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
 #pragma unroll
       for (int c = 0; c < kTcBN; c += 2) {
         // 2^(scale * s - m): one fma per score (masked scores are -inf: weight 0)
         const float p0 = fast_exp2(fmaf(sv[c], p.scale_log2, -mm));
         const float p1 = fast_exp2(fmaf(sv[c + 1], p.scale_log2, -mm));
-        l += p0 + p1;
+        ls[(c >> 1) & 3] += p0 + p1;
         ph[c / 2] = Elem<T>::from_float2(p0, p1);
         if constexpr (BF16) {
           const float2 back = Elem<T>::to_float2(ph[c / 2]);
           pl[c / 2] = Elem<T>::from_float2(p0 - back.x, p1 - back.y);
         }
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tc::st16(rbase + kColPhi, *reinterpret_cast<uint32_t(*)[16]>(ph));
       tc::st16(rbase + kColPhi + 16, *reinterpret_cast<uint32_t(*)[16]>(ph + 16));
       if constexpr (BF16) {
