@@ -354,6 +354,168 @@ def run_prefill_bench(args, ranks, world, rank, local):
     return 0
 
 
+def read_probe_gbs(dev, gib: int = 4) -> float:
+    """Read-only streaming ceiling of this GPU, measured in the same process:
+    the median rate of the library's read probe (pa_read_probe) over a `gib`
+    GiB buffer, larger than L2."""
+    import paged_kv_cache_326_b200 as P
+    buf = torch.empty(gib << 30, dtype=torch.uint8, device=dev)
+    buf.fill_(1)
+    sink = torch.empty(4096, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        P.binding.pa_read_probe(buf, sink)
+    times = []
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        P.binding.pa_read_probe(buf, sink)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    del buf
+    torch.cuda.empty_cache()
+    return (gib << 30) / (statistics.median(times) * 1e-3) / 1e9
+
+
+def shared_prefix_inputs(P, W, seed, dev):
+    """The shared-prefix workload built by the C++ block manager (copy-on-write
+    copies applied while the samples generate)."""
+    bm = P.BlockManager(8192, 16)
+
+    class Adapter:
+        add_seq = staticmethod(bm.add_seq)
+        fork = staticmethod(bm.fork)
+        append_slot = staticmethod(bm.append_slot)
+
+        @staticmethod
+        def export(ids, mb):
+            t, l = bm.export(ids, mb)
+            return t.numpy(), l.numpy()
+
+    return W.shared_prefix(Adapter(), num_blocks=8192, seed=seed, device=dev)
+
+
+def unique_kv_bytes(w, num_kv_heads, head_dim, elem_bytes) -> int:
+    """KV bytes that the texts' reads cover, each stored (block, row) once."""
+    import numpy as np
+    tables = w.block_tables.cpu().numpy()
+    lens = w.context_lens.cpu().numpy()
+    B = w.block_size
+    rows = {}
+    for s in range(tables.shape[0]):
+        L = int(lens[s])
+        for j in range(-(-L // B)):
+            b = int(tables[s, j])
+            rows[b] = max(rows.get(b, 0), min(B, L - j * B))
+    return sum(rows.values()) * 2 * num_kv_heads * head_dim * elem_bytes
+
+
+def run_full_step(args, ranks, world, rank, local):
+    """The full OPT-13B-shaped decode step: 40 layers x (write + attend) for
+    256 texts, one 131,072-block pool (42.9 GB) shared by the layers; each
+    layer streams its own ~5.5 GB of KV.  decode tokens/s = texts / step."""
+    import paged_kv_cache_326_b200 as P
+    from paged_kv_cache_326_b200 import dist, workloads as W
+    P.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    fs = W.full_step(seed=dist.batch_seed(5, ranks), device=dev)
+    S, H, D = fs.q[0].shape
+    lens = fs.context_lens.tolist()
+    layer_kv = kv_bytes(lens, H, D, 2)
+    step_kv = layer_kv * fs.num_layers
+    out = torch.empty_like(fs.q[0])
+    ws = P.binding.workspace_for(fs.q[0], fs.block_size, fs.block_tables[0].shape[1])
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        for layer in range(fs.num_layers):
+            P.pa_decode_step(out, fs.q[layer], fs.k[layer], fs.v[layer], fs.k_cache, fs.v_cache,
+                             fs.slot_mapping[layer], fs.block_tables[layer], fs.context_lens,
+                             fs.scale, workspace=ws, status=status)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    K = args.steps
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        dist.barrier(ranks)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(K):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier(ranks)
+    clk = clocks.summary()
+    ms_step = start.elapsed_time(stop) / K
+    # end to end: every layer's q, k, v and slots from pinned host memory, every
+    # layer's output back to the host
+    hq = [t.cpu().pin_memory() for t in fs.q]
+    hk = [t.cpu().pin_memory() for t in fs.k]
+    hv = [t.cpu().pin_memory() for t in fs.v]
+    hs = [t.cpu().pin_memory() for t in fs.slot_mapping]
+    hout = torch.empty_like(hq[0]).pin_memory()
+    dq, dk, dv, dsl = (torch.empty_like(fs.q[0]), torch.empty_like(fs.k[0]),
+                       torch.empty_like(fs.v[0]), torch.empty_like(fs.slot_mapping[0]))
+    Ke = max(1, min(K, 10))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        for layer in range(fs.num_layers):
+            dq.copy_(hq[layer], non_blocking=True)
+            dk.copy_(hk[layer], non_blocking=True)
+            dv.copy_(hv[layer], non_blocking=True)
+            dsl.copy_(hs[layer], non_blocking=True)
+            P.pa_decode_step(out, dq, dk, dv, fs.k_cache, fs.v_cache, dsl,
+                             fs.block_tables[layer], fs.context_lens, fs.scale, workspace=ws,
+                             status=status)
+            hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    ms_step, e2e_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms], dev)
+    peak, peak_src = hbm_peak()
+    per_layer_bytes = (layer_kv + 2 * S * H * D * 2 + 4 * S * H * D * 2 +
+                       sum(4 * -(-L // fs.block_size) for L in lens) + 12 * S)
+    achieved = per_layer_bytes * fs.num_layers / (ms_step * 1e-3) / 1e9
+    h2d = fs.num_layers * sum(t.numel() * t.element_size() for t in (hq[0], hk[0], hv[0], hs[0]))
+    d2h = fs.num_layers * hout.numel() * hout.element_size()
+    line = {
+        "metric": METRIC, "value": world * step_kv / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "accumulate": "f32", "data": "synthetic",
+        "config": {"workload": "full_step", "layers": fs.num_layers, "num_seqs": S,
+                   "num_heads": H, "head_dim": D, "block_size": fs.block_size,
+                   "context_lens": "uniform [64, 2048], seed 5+rank",
+                   "num_blocks": fs.k_cache.shape[0], "kv_bytes_per_step": step_kv,
+                   "pool": "one 131,072-block pool shared by the 40 layers (tables drawn per layer)",
+                   "l2": "inputs larger than L2 (5.5 GB of KV per layer)",
+                   "parallelism": f"independent batch per GPU x{world}",
+                   "path": "pa_decode_step per layer"},
+        "decode_tokens_per_s": world * S / (ms_step * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "pa_decode_step x 40 layers (decode kernel + merge kernel)",
+                     "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": per_layer_bytes},
+        "e2e": {"value": world * step_kv / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * fs.num_layers * K,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_cow_copy(args, ranks, world, rank, local):
     """Copy-on-write bursts: each step copies one burst of 224 whole blocks
     (32 prompts x 7 samples, 40 heads x 16 x 128 fp16, K and V) with
@@ -481,11 +643,14 @@ def main():
     ap.add_argument("--gqa-kernel", choices=["auto", "cores", "tensor"], default="auto",
                     help="grouped-query workload: kernel choice (PA_OPT_GQA_KERNEL)")
     ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa", "cow_copy",
-                                           "prefill"],
+                                           "prefill", "skewed", "shared_prefix", "full_step"],
                     default="opt13b_batch64",
                     help="llama2_70b_gqa: 64 query heads on 8 key/value heads (two calls); "
                          "cow_copy: copy-on-write bursts of whole blocks (pa_copy_blocks); "
-                         "prefill: the prompt phase of 16 prompts of 2,048 tokens (pa_prefill)")
+                         "prefill: the prompt phase of 16 prompts of 2,048 tokens (pa_prefill); "
+                         "skewed: 256 texts, lognormal lengths, bf16; shared_prefix: 32 prompts "
+                         "x 8 samples built by the block manager; full_step: 40 layers x 256 "
+                         "texts over one 42.9 GB pool")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -503,6 +668,10 @@ def main():
         return rc
     if args.workload == "prefill":
         rc = run_prefill_bench(args, ranks, world, rank, local)
+        dist.finish(ranks)
+        return rc
+    if args.workload == "full_step":
+        rc = run_full_step(args, ranks, world, rank, local)
         dist.finish(ranks)
         return rc
 
@@ -525,6 +694,10 @@ def main():
     elif fp8:
         args.path = "calls"   # the one-launch step stores 16-bit values
         w = W.opt13b_batch64_fp8(seed=dist.batch_seed(2, ranks), device=dev)
+    elif args.workload == "skewed":
+        w = W.skewed(seed=dist.batch_seed(3, ranks), device=dev)
+    elif args.workload == "shared_prefix":
+        w = shared_prefix_inputs(P, W, dist.batch_seed(4, ranks), dev)
     else:
         w = W.opt13b_batch64(seed=dist.batch_seed(2, ranks), device=dev)
     S, H, D = w.q.shape
@@ -533,6 +706,10 @@ def main():
     cb = w.k_cache.element_size()                 # cache bytes per number (1 for 8-bit)
     lens = w.context_lens.tolist()
     step_kv = kv_bytes(lens, Hkv, D, cb)
+    logical_kv = step_kv
+    if args.workload == "shared_prefix":
+        # texts share their prompt's blocks: count each stored row once
+        step_kv = unique_kv_bytes(w, Hkv, D, cb)
     decode_bytes = step_kv + 2 * S * H * D * eb + sum(4 * -(-L // w.block_size) for L in lens) + 4 * S
     write_bytes = 2 * S * Hkv * D * (eb + cb) + 8 * S   # k, v read and stored; slots
     fused = args.path == "fused"
@@ -644,10 +821,12 @@ def main():
     peak, peak_src = hbm_peak()
     achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
     value = world * step_kv / (ms_step * 1e-3) / 1e9
+    probe_gbs = read_probe_gbs(dev)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.q.dtype == torch.bfloat16 else "f16", "accumulate": "f32",
         "data": "synthetic",
         "config": {"workload": args.workload + ("_fp8" if fp8 else ""), "num_seqs": S,
                    "num_heads": H,
@@ -655,6 +834,10 @@ def main():
                                 (w.meta["k_scale"], w.meta["v_scale"]) if fp8 else "f16"),
                    "num_kv_heads": Hkv, "head_dim": D, "block_size": w.block_size,
                    "context_lens": ("uniform [128, 4096], seed 6+rank" if gqa else
+                                    "lognormal (median 300, sigma 1.0) clipped [16, 2048], 8 at "
+                                    "2,048, seed 3+rank" if args.workload == "skewed" else
+                                    "prompts U[256, 1024] x 8 samples, generated U[1, 256], "
+                                    "seed 4+rank" if args.workload == "shared_prefix" else
                                     "uniform [128, 2048], seed 2+rank"),
                    "num_blocks": w.num_blocks, "kv_bytes_per_step": step_kv,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB)",
@@ -664,7 +847,17 @@ def main():
                             else "pa_kv_cache_write_fp8 + pa_paged_attn_decode_fp8" if fp8
                             else "pa_kv_cache_write + pa_paged_attn_decode")},
         "decode_tokens_per_s": world * S / (ms_step * 1e-3),
+        **({"logical_kv_gbs": world * logical_kv / (ms_step * 1e-3) / 1e9,
+            "value_counts": "distinct (block, row) KV bytes; logical_kv_gbs counts every "
+                            "text's reads"} if args.workload == "shared_prefix" else {}),
         "pct_of_nominal_8tbs": 100.0 * (value / world) / NOMINAL_HBM_GBS,
+        # the decode call against three ceilings: the nominal spec, the
+        # measured copy bandwidth, and a read-only stream measured here
+        "ceilings": {"nominal_gbs": NOMINAL_HBM_GBS, "measured_copy_gbs": peak,
+                     "read_probe_gbs": probe_gbs,
+                     "decode_frac_of": {"nominal": achieved / NOMINAL_HBM_GBS,
+                                        "measured_copy": achieved / peak,
+                                        "read_probe": achieved / probe_gbs}},
         "kernel_ms": ({"pa_decode_step": decode_ms} if fused else
                       {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -333,6 +333,18 @@ int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks,
                    int32_t* d_status, pa_stream_t stream);
 
 /*
+ * pa_read_probe — a diagnostic with no counterpart in the pages: read `bytes`
+ * (a multiple of 16) of device buffer `buf` once with a read-only streaming
+ * kernel (a persistent grid, four 16-byte loads in flight per thread), to
+ * measure the GPU's HBM read ceiling beside the decode kernels.  The loads
+ * are folded with XOR into one word per CTA in d_sink (device, sink_words
+ * words; 4 x the SM count is enough).  Returns PA_OK or PA_ERR_INVALID /
+ * PA_ERR_CUDA.
+ */
+int pa_read_probe(const void* buf, size_t bytes, uint32_t* d_sink, int sink_words,
+                  pa_stream_t stream);
+
+/*
  * pa_paged_attn_decode_noalloc — pa_paged_attn_decode without a caller
  * workspace, for callers that cannot allocate device memory (a host framework
  * that owns every device allocation, a fixed memory budget, a loop where an

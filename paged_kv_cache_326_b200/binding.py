@@ -80,6 +80,7 @@ _SIGNATURES = {
                                         _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _f32, _i32,
                           _i32, _i32, _i32, _i64, _i32, _vp, _vp]),
+    "pa_read_probe": (_i32, [_vp, _sz, _vp, _i32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32,
                               _vp, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
@@ -261,6 +262,14 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Ten
         D, B, N, _dtype_code(q), _status_ptr(status), _stream(stream, q.device))
     _check(code, "pa_prefill")
     return out
+
+
+def pa_read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
+    """Read every byte of the CUDA tensor `buf` once (the HBM read ceiling);
+    sink: a CUDA int32 tensor of at least 4 x the SM count words."""
+    nbytes = buf.numel() * buf.element_size()
+    _check(lib().pa_read_probe(_cuda(buf, "buf"), nbytes & ~15, _cuda(sink, "sink", torch.int32),
+                               sink.numel(), _stream(stream, buf.device)), "pa_read_probe")
 
 
 def _pool(t: torch.Tensor, name: str) -> int:

@@ -266,6 +266,14 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
                                                 : pa::launch_prefill_tc(a, st));
 }
 
+int pa_read_probe(const void* buf, size_t bytes, uint32_t* d_sink, int sink_words,
+                  pa_stream_t stream) {
+  if (!buf || !d_sink || bytes == 0 || (bytes & 15u) || sink_words < 1 || !aligned16(buf))
+    return PA_ERR_INVALID;
+  return from_cuda(pa::launch_read_probe(buf, static_cast<int64_t>(bytes), d_sink, sink_words,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int pa_copy_blocks(const void* src_k, const void* src_v, int64_t src_num_blocks, void* dst_k,
                    void* dst_v, int64_t dst_num_blocks, const int32_t* block_pairs,
                    int num_pairs, int num_heads, int head_dim, int block_size, pa_dtype dt,

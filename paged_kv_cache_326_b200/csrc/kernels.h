@@ -62,6 +62,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
 // Current PA_OPT_PREFILL_KERNEL setting (0 automatic = tcgen05, 1 mma.sync, 2 tcgen05).
 int64_t option_prefill_kernel();
 
+// Read-only streaming probe: reads `bytes` (a multiple of 16) of `buf` once;
+// one word per CTA lands in sink[0 .. sink_words).
+cudaError_t launch_read_probe(const void* buf, int64_t bytes, uint32_t* sink, int sink_words,
+                              cudaStream_t stream);
+
 struct DecodeArgs {
   void* out;
   const void* q;
