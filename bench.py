@@ -640,6 +640,9 @@ def main():
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
     ap.add_argument("--kv-dtype", choices=["f16", "fp8"], default="f16",
                     help="fp8: the batch-64 step over 8-bit E4M3 caches (two calls)")
+    ap.add_argument("--shared-path", choices=["cascade", "plain"], default="cascade",
+                    help="shared_prefix workload: pa_paged_attn_decode_shared over the split "
+                         "tables (cascade) or pa_paged_attn_decode over the joined ones (plain)")
     ap.add_argument("--gqa-kernel", choices=["auto", "cores", "tensor"], default="auto",
                     help="grouped-query workload: kernel choice (PA_OPT_GQA_KERNEL)")
     ap.add_argument("--workload", choices=["opt13b_batch64", "llama2_70b_gqa", "cow_copy",
@@ -712,11 +715,26 @@ def main():
         step_kv = unique_kv_bytes(w, Hkv, D, cb)
     decode_bytes = step_kv + 2 * S * H * D * eb + sum(4 * -(-L // w.block_size) for L in lens) + 4 * S
     write_bytes = 2 * S * Hkv * D * (eb + cb) + 8 * S   # k, v read and stored; slots
+    cascade = args.workload == "shared_prefix" and args.shared_path == "cascade"
+    if cascade:
+        # the host splits the exported tables once per step, as it exports
+        # them: a prefix per prompt, a tail per sample
+        args.path = "calls"
+        gs = w.meta["samples"]
+        split = P.split_shared_prefix(w.block_tables.cpu(), w.context_lens.cpu(), w.block_size, gs)
+        split_d = [t.to(dev) for t in split]
+        pl, tl = split[1].tolist(), split[3].tolist()
+        decode_bytes = (step_kv + 2 * S * H * D * eb + 4 * S + 4 * len(pl) +
+                        sum(4 * -(-L // w.block_size) for L in pl + tl))
     fused = args.path == "fused"
     if fused:
         decode_bytes += write_bytes
     out = torch.empty_like(w.q)
     ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq, Hkv)
+    if cascade:
+        ws_shared = torch.empty(P.pa_paged_attn_decode_shared_workspace_size(
+            len(pl), gs, H, D, w.block_size, split[0].shape[1], split[2].shape[1]),
+            dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def write_part(k, v, slots):
@@ -726,8 +744,12 @@ def main():
         elif not fused:
             P.pa_kv_cache_write(k, v, w.k_cache, w.v_cache, slots, status=status)
 
-    def decode_part(q, k, v, slots, tables, lens):
-        if fused:
+    def decode_part(q, k, v, slots, tables, lens, shared_tables=None):
+        if cascade:
+            pt, pl_d, tt, tl_d = shared_tables if shared_tables is not None else split_d
+            P.pa_paged_attn_decode_shared(out, q, w.k_cache, w.v_cache, pt, pl_d, tt, tl_d,
+                                          w.scale, gs, workspace=ws_shared, status=status)
+        elif fused:
             P.pa_decode_step(out, q, k, v, w.k_cache, w.v_cache, slots, tables, lens, w.scale,
                              workspace=ws, status=status)
         elif gqa:
@@ -784,14 +806,29 @@ def main():
     hslot = w.slot_mapping.cpu().pin_memory()
     htab = w.block_tables.cpu().pin_memory()
     hlen = w.context_lens.cpu().pin_memory()
+    if cascade:   # the split tables stand in for the joined ones
+        hsplit = [t.pin_memory() for t in split]
+        dsplit = [torch.empty_like(t) for t in split_d]
+        htab, hlen = hsplit[0], hsplit[1]
     hout = torch.empty_like(hq).pin_memory()
     dq, dk, dv = torch.empty_like(w.q), torch.empty_like(w.k), torch.empty_like(w.v)
     dslot, dtab, dlen = (torch.empty_like(w.slot_mapping), torch.empty_like(w.block_tables),
                          torch.empty_like(w.context_lens))
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hslot, htab, hlen))
+    if cascade:
+        h2d += sum(t.numel() * t.element_size() for t in hsplit[2:])
     d2h = hout.numel() * hout.element_size()
 
     def e2e_step():
+        if cascade:
+            for d, h in zip(dsplit, hsplit):
+                d.copy_(h, non_blocking=True)
+            for d, h in ((dq, hq), (dk, hk), (dv, hv), (dslot, hslot)):
+                d.copy_(h, non_blocking=True)
+            write_part(dk, dv, dslot)
+            decode_part(dq, dk, dv, dslot, None, None, shared_tables=dsplit)
+            hout.copy_(out, non_blocking=True)
+            return
         for d, h in ((dq, hq), (dk, hk), (dv, hv), (dslot, hslot), (dtab, htab), (dlen, hlen)):
             d.copy_(h, non_blocking=True)
         write_part(dk, dv, dslot)
@@ -842,7 +879,9 @@ def main():
                    "num_blocks": w.num_blocks, "kv_bytes_per_step": step_kv,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB)",
                    "parallelism": f"independent batch per GPU x{world}",
-                   "path": ("pa_decode_step" if fused else
+                   "path": ("pa_kv_cache_write + pa_paged_attn_decode_shared (tables split "
+                            "by pa_split_shared_prefix)" if cascade else
+                            "pa_decode_step" if fused else
                             f"pa_kv_cache_write + pa_paged_attn_decode_gqa ({gqa_kernel})" if gqa
                             else "pa_kv_cache_write_fp8 + pa_paged_attn_decode_fp8" if fp8
                             else "pa_kv_cache_write + pa_paged_attn_decode")},
@@ -863,7 +902,9 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
                      "traffic": (None if fp8 else traffic_per_launch(args.workload, args.path)),
-                     "kernel": ("pa_decode_step (decode kernel with the cache write, + merge kernel)"
+                     "kernel": ("pa_paged_attn_decode_shared (prefix pass on the tensor cores, "
+                                "tail pass, merge kernel)" if cascade else
+                                "pa_decode_step (decode kernel with the cache write, + merge kernel)"
                                 if fused else
                                 f"pa_paged_attn_decode_gqa ({gqa_kernel} decode kernel + merge kernel)" if gqa
                                 else "pa_paged_attn_decode_fp8 (8-bit decode kernel + merge kernel)" if fp8
@@ -871,7 +912,7 @@ def main():
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": decode_bytes},
         "e2e": {"value": world * step_kv / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": (2 if fused else 3) * K,
+        "gpu_launches": (2 if fused else 4 if cascade else 3) * K,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

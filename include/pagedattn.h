@@ -179,6 +179,69 @@ int pa_decode_step(void* out, const void* q, const void* k, const void* v, void*
                    pa_stream_t stream);
 
 /*
+ * pa_paged_attn_decode_shared_workspace_size — device scratch bytes that
+ * pa_paged_attn_decode_shared needs for these sizes on the current device.
+ * Host only.  Returns 0 for unsupported sizes.
+ */
+size_t pa_paged_attn_decode_shared_workspace_size(int num_groups, int group_size, int num_heads,
+                                                  int head_dim, int block_size,
+                                                  int max_prefix_blocks, int max_tail_blocks);
+
+/*
+ * pa_paged_attn_decode_shared — pa_paged_attn_decode for groups of texts that
+ * share the leading blocks of one prompt ("The KV Cache and PagedAttention",
+ * section "Shared, Copied on Write": the samples of one prompt point at the
+ * same physical blocks).  Texts come in num_groups groups of group_size
+ * consecutive texts (text t is in group t / group_size).  Text t attends over
+ * its group's PREFIX (prefix_lens[g] tokens in the blocks of
+ * prefix_tables[g]) followed by its own TAIL (tail_lens[t] tokens in the
+ * blocks of tail_tables[t]):
+ *     out[t][h][:] = sum over prefix and tail tokens of softmax(z) * V,
+ * the same result as pa_paged_attn_decode over the joined table (up to
+ * rounding).  Each shared key and value is read once per group, not once per
+ * text: the group's queries run together on the tensor cores, the tails on
+ * the multi-head kernel, and a log-sum-exp merge joins the two.
+ *
+ *   out, q         [num_groups * group_size][num_heads][head_dim] dt, device
+ *   k_cache,v_cache multi-head pool (layout above), device
+ *   prefix_tables  [num_groups][max_prefix_blocks] int32, device
+ *   prefix_lens    [num_groups] int32, device (0 allowed)
+ *   tail_tables    [num_groups * group_size][max_tail_blocks] int32, device
+ *   tail_lens      [num_groups * group_size] int32, device (0 allowed)
+ *   group_size     1 .. 16; block_size 8, 16 or 32
+ *   workspace      at least pa_paged_attn_decode_shared_workspace_size(...)
+ *                  bytes, 256-byte aligned, not shared with concurrent calls
+ * A text with no tokens at all gets zeros.  pa_split_shared_prefix builds the
+ * four tables from ordinary block tables.  Data errors as for
+ * pa_paged_attn_decode.  Bitwise reproducible for fixed inputs and device.
+ * Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_paged_attn_decode_shared(void* out, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* prefix_tables,
+                                const int32_t* prefix_lens, int max_prefix_blocks,
+                                const int32_t* tail_tables, const int32_t* tail_lens,
+                                int max_tail_blocks, float scale, int num_groups, int group_size,
+                                int num_heads, int head_dim, int block_size, int64_t num_blocks,
+                                pa_dtype dt, void* workspace, size_t workspace_bytes,
+                                int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_split_shared_prefix — host only: cut ordinary block tables (as
+ * pa_bm_export writes them) of num_seqs = groups * group_size texts into the
+ * inputs of pa_paged_attn_decode_shared.  A group's prefix is its longest run
+ * of leading table entries that all its texts hold at the same index and have
+ * filled completely (at most max_prefix_blocks); each text's tail is the rest
+ * of its table.  Unused entries are -1.  All pointers are HOST pointers.
+ * PA_ERR_TABLE_FULL if a tail needs more than max_tail_blocks blocks,
+ * PA_ERR_INVALID for bad sizes or a length outside the table; nothing is
+ * written on error.
+ */
+int pa_split_shared_prefix(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                           int max_blocks_per_seq, int block_size, int group_size,
+                           int32_t* prefix_tables, int max_prefix_blocks, int32_t* prefix_lens,
+                           int32_t* tail_tables, int max_tail_blocks, int32_t* tail_lens);
+
+/*
  * pa_paged_attn_decode_gqa_workspace_size — as
  * pa_paged_attn_decode_workspace_size, for pa_paged_attn_decode_gqa with
  * num_kv_heads key/value heads.  Returns 0 for unsupported sizes (including

@@ -37,6 +37,11 @@ Prompt phase (``prefill``): causal attention of a prompt's tokens over the
 prompt itself, whose keys and values are then stored in the cache (the
 write is ``cache_write``).
 
+Shared prefixes (``split_shared_prefix``, ``paged_decode_shared``): texts
+in groups that share the leading blocks of one prompt attend over the group's
+prefix followed by their own tail, which is the same token sequence as their
+joined table.
+
 Block copies (``copy_blocks``): whole blocks copied from a source pool to a
 destination pool ("The KV Cache and PagedAttention", §Shared, Copied on
 Write: a text about to write into a block it shares gets its own copy of the
@@ -54,7 +59,9 @@ attention on repeated heads, and brute force for one shared head; block
 copies against the worked copy-on-write example of the pages (each answer
 reads the prompt plus its own token and nothing of the other's), torch's
 index_copy_ on raw bit patterns, and a copy out and back that restores every
-block.
+block; shared prefixes against ``paged_decode`` on the joined tables (bit for
+bit), a prefix and tail written out by hand for a forked prompt, scalar brute
+force, and the order of prefix and tail swapped (softmax ignores order).
 """
 from __future__ import annotations
 
@@ -174,6 +181,68 @@ def paged_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
         full = attend(q[s][heads], K[:, sel, :], V[:, sel, :], scale)
         for i, h in enumerate(heads):
             out[s, h] = full[i]
+    return out
+
+
+def split_shared_prefix(block_tables: np.ndarray, context_lens: Sequence[int], block_size: int,
+                        group_size: int):
+    """Cut the tables of groups of ``group_size`` consecutive texts into a
+    shared prefix per group and a private tail per text ("The KV Cache and
+    PagedAttention", §Shared, Copied on Write: the samples of one prompt point
+    at the same physical blocks).  A group's prefix is the longest run of
+    leading table entries that every text of the group holds at the same
+    index and has filled completely.  Returns (prefix_tables as a list of
+    lists, prefix_lens, tail_tables, tail_lens)."""
+    S = len(context_lens)
+    if group_size < 1 or S % group_size:
+        raise ValueError("the number of texts must be a multiple of group_size")
+    prefix_tables, prefix_lens, tail_tables, tail_lens = [], [], [], []
+    for g in range(S // group_size):
+        members = range(g * group_size, (g + 1) * group_size)
+        first = block_tables[g * group_size]
+        p = 0
+        while p < len(first) and all(
+                int(block_tables[s][p]) == int(first[p]) and (p + 1) * block_size <= int(context_lens[s])
+                for s in members):
+            p += 1
+        prefix_tables.append([int(b) for b in first[:p]])
+        prefix_lens.append(p * block_size)
+        for s in members:
+            tail = int(context_lens[s]) - p * block_size
+            nb = -(-tail // block_size)
+            tail_tables.append([int(b) for b in block_tables[s][p:p + nb]])
+            tail_lens.append(tail)
+    return prefix_tables, prefix_lens, tail_tables, tail_lens
+
+
+def paged_decode_shared(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                        prefix_tables, prefix_lens: Sequence[int], tail_tables,
+                        tail_lens: Sequence[int], group_size: int, scale: float,
+                        block_size: int,
+                        pairs: Optional[Iterable[Tuple[int, int]]] = None) -> np.ndarray:
+    """Decode attention for texts that share a prefix, fp64 ``[S][H][D]``:
+    text t (group t // group_size) attends over its group's prefix tokens
+    followed by its own tail tokens, i.e. the tokens of the joined table, with
+    the plain definition of ``attend``.  ``pairs`` as in ``paged_decode``."""
+    S, H, D = q.shape
+    out = np.zeros((S, H, D), dtype=np.float64)
+    wanted = None
+    if pairs is not None:
+        wanted = {}
+        for s, h in pairs:
+            wanted.setdefault(int(s), []).append(int(h))
+    for t in range(S):
+        if wanted is not None and t not in wanted:
+            continue
+        g = t // group_size
+        K = np.concatenate([gather_context(k_cache, prefix_tables[g], prefix_lens[g], block_size),
+                            gather_context(k_cache, tail_tables[t], tail_lens[t], block_size)])
+        V = np.concatenate([gather_context(v_cache, prefix_tables[g], prefix_lens[g], block_size),
+                            gather_context(v_cache, tail_tables[t], tail_lens[t], block_size)])
+        heads = list(range(H)) if wanted is None else wanted[t]
+        full = attend(q[t][heads], K[:, heads, :], V[:, heads, :], scale)
+        for i, h in enumerate(heads):
+            out[t, h] = full[i]
     return out
 
 

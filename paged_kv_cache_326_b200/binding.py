@@ -83,6 +83,13 @@ _SIGNATURES = {
     "pa_read_probe": (_i32, [_vp, _sz, _vp, _i32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32,
                               _vp, _vp]),
+    "pa_paged_attn_decode_shared_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32,
+                                                           _i32]),
+    "pa_paged_attn_decode_shared": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32,
+                                           _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _vp,
+                                           _sz, _vp, _vp]),
+    "pa_split_shared_prefix": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp,
+                                      _i32, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_i32, [_vp, _i64, _i32]),
@@ -399,6 +406,88 @@ def pa_paged_attn_decode_gqa(out: torch.Tensor, q: torch.Tensor, k_cache: torch.
         _status_ptr(status), _stream(stream, q.device))
     _check(code, "pa_paged_attn_decode_gqa")
     return out
+
+
+def pa_paged_attn_decode_shared_workspace_size(num_groups: int, group_size: int, num_heads: int,
+                                               head_dim: int, block_size: int,
+                                               max_prefix_blocks: int, max_tail_blocks: int) -> int:
+    return int(lib().pa_paged_attn_decode_shared_workspace_size(
+        num_groups, group_size, num_heads, head_dim, block_size, max_prefix_blocks,
+        max_tail_blocks))
+
+
+def pa_paged_attn_decode_shared(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                                v_cache: torch.Tensor, prefix_tables: torch.Tensor,
+                                prefix_lens: torch.Tensor, tail_tables: torch.Tensor,
+                                tail_lens: torch.Tensor, scale: float, group_size: int,
+                                workspace: Optional[torch.Tensor] = None,
+                                status: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """Decode for groups of ``group_size`` consecutive texts sharing a prefix:
+    out, q [G*group_size][H][D]; caches [N][H][B][D]; prefix_tables
+    [G][max_prefix_blocks], prefix_lens [G]; tail_tables
+    [G*group_size][max_tail_blocks], tail_lens [G*group_size] (int32)."""
+    S, H, D = q.shape
+    N, H2, B, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
+        raise ValueError("shape mismatch")
+    if group_size < 1 or S % group_size:
+        raise ValueError("the number of texts must be a multiple of group_size")
+    G = S // group_size
+    if prefix_tables.dim() != 2 or prefix_tables.shape[0] != G or prefix_lens.shape != (G,):
+        raise ValueError("prefix_tables must be [G][max_prefix_blocks], prefix_lens [G]")
+    if tail_tables.dim() != 2 or tail_tables.shape[0] != S or tail_lens.shape != (S,):
+        raise ValueError("tail_tables must be [S][max_tail_blocks], tail_lens [S]")
+    for t in (out, k_cache, v_cache):
+        if t.dtype != q.dtype:
+            raise TypeError("q, out and the caches must share a dtype")
+    MP, MT = prefix_tables.shape[1], tail_tables.shape[1]
+    if workspace is None:
+        need = pa_paged_attn_decode_shared_workspace_size(G, group_size, H, D, B, MP, MT)
+        if need == 0:
+            raise PagedAttnError(PA_ERR_INVALID, "pa_paged_attn_decode_shared_workspace_size")
+        key = (q.device.index if q.device.index is not None else torch.cuda.current_device(),
+               need)
+        workspace = _ws_cache.get(key)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            _ws_cache[key] = workspace
+    code = lib().pa_paged_attn_decode_shared(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(prefix_tables, "prefix_tables", torch.int32),
+        _cuda(prefix_lens, "prefix_lens", torch.int32), MP,
+        _cuda(tail_tables, "tail_tables", torch.int32),
+        _cuda(tail_lens, "tail_lens", torch.int32), MT, float(scale), G, int(group_size), H, D,
+        B, N, _dtype_code(q), _cuda(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _status_ptr(status),
+        _stream(stream, q.device))
+    _check(code, "pa_paged_attn_decode_shared")
+    return out
+
+
+def split_shared_prefix(block_tables: torch.Tensor, context_lens: torch.Tensor,
+                        block_size: int, group_size: int, max_prefix_blocks: Optional[int] = None,
+                        max_tail_blocks: Optional[int] = None):
+    """Host: cut block tables of groups of ``group_size`` consecutive texts
+    into (prefix_tables, prefix_lens, tail_tables, tail_lens), CPU int32
+    tensors, with pa_split_shared_prefix."""
+    bt = block_tables.detach().to("cpu", torch.int32).contiguous()
+    cl = context_lens.detach().to("cpu", torch.int32).contiguous()
+    S, MB = bt.shape
+    if cl.shape != (S,) or group_size < 1 or S % group_size:
+        raise ValueError("block_tables [S][max_blocks], context_lens [S], S % group_size == 0")
+    MP = MB if max_prefix_blocks is None else int(max_prefix_blocks)
+    MT = MB if max_tail_blocks is None else int(max_tail_blocks)
+    G = S // group_size
+    pt = torch.empty((G, MP), dtype=torch.int32)
+    pl = torch.empty(G, dtype=torch.int32)
+    tt = torch.empty((S, MT), dtype=torch.int32)
+    tl = torch.empty(S, dtype=torch.int32)
+    _check(lib().pa_split_shared_prefix(bt.data_ptr(), cl.data_ptr(), S, MB, int(block_size),
+                                        int(group_size), pt.data_ptr(), MP, pl.data_ptr(),
+                                        tt.data_ptr(), MT, tl.data_ptr()),
+           "pa_split_shared_prefix")
+    return pt, pl, tt, tl
 
 
 def pa_decode_step(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

@@ -176,4 +176,59 @@ int pa_bm_export(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* block_
   return PA_OK;
 }
 
+int pa_split_shared_prefix(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                           int max_blocks_per_seq, int block_size, int group_size,
+                           int32_t* prefix_tables, int max_prefix_blocks, int32_t* prefix_lens,
+                           int32_t* tail_tables, int max_tail_blocks, int32_t* tail_lens) {
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || group_size <= 0 ||
+      num_seqs % group_size != 0 || max_prefix_blocks <= 0 || max_tail_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!block_tables || !context_lens || !prefix_tables || !prefix_lens || !tail_tables ||
+      !tail_lens)
+    return PA_ERR_INVALID;
+  const int64_t cap = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+  for (int s = 0; s < num_seqs; ++s)
+    if (context_lens[s] < 0 || context_lens[s] > cap) return PA_ERR_INVALID;
+  const int groups = num_seqs / group_size;
+  std::vector<int> shared(groups);
+  // Shared blocks of a group: the leading table entries that every text of
+  // the group holds at the same index and has filled completely.
+  for (int g = 0; g < groups; ++g) {
+    const int s0 = g * group_size;
+    const int32_t* row0 = block_tables + static_cast<int64_t>(s0) * max_blocks_per_seq;
+    int p = 0;
+    while (p < max_prefix_blocks && p < max_blocks_per_seq) {
+      bool same = true;
+      for (int s = s0; s < s0 + group_size && same; ++s) {
+        const int32_t* row = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq;
+        same = row[p] == row0[p] && static_cast<int64_t>(p + 1) * block_size <= context_lens[s];
+      }
+      if (!same) break;
+      ++p;
+    }
+    shared[g] = p;
+    for (int s = s0; s < s0 + group_size; ++s) {
+      const int64_t tail = context_lens[s] - static_cast<int64_t>(p) * block_size;
+      if ((tail + block_size - 1) / block_size > max_tail_blocks) return PA_ERR_TABLE_FULL;
+    }
+  }
+  for (int g = 0; g < groups; ++g) {
+    const int p = shared[g];
+    const int32_t* row0 = block_tables + static_cast<int64_t>(g) * group_size * max_blocks_per_seq;
+    int32_t* prow = prefix_tables + static_cast<int64_t>(g) * max_prefix_blocks;
+    for (int k = 0; k < max_prefix_blocks; ++k) prow[k] = k < p ? row0[k] : -1;
+    prefix_lens[g] = p * block_size;
+    for (int s = g * group_size; s < (g + 1) * group_size; ++s) {
+      const int32_t* row = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq;
+      int32_t* trow = tail_tables + static_cast<int64_t>(s) * max_tail_blocks;
+      const int tail = context_lens[s] - p * block_size;
+      const int nb = (tail + block_size - 1) / block_size;
+      for (int k = 0; k < max_tail_blocks; ++k) trow[k] = k < nb ? row[p + k] : -1;
+      tail_lens[s] = tail;
+    }
+  }
+  return PA_OK;
+}
+
 }  // extern "C"

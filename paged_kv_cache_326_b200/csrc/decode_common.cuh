@@ -94,6 +94,12 @@ struct DecodeParams {
   float* records;
   int32_t* status;
   int64_t wait_limit_ns;
+  // Shared-prefix (cascade) passes: every unit leaves a partial record, even
+  // for a (text, head) it covers whole, and no output is written (a third
+  // kernel merges the records of both passes).  In the grouped-query kernel
+  // the gs query heads of virtual text s and head h are then the same head h
+  // of texts s * gs .. s * gs + gs - 1 (q laid out [texts][heads][D]).
+  int cascade = 0;
 };
 
 // The work split of one launch; every CTA computes the same one.
@@ -174,7 +180,7 @@ __device__ __forceinline__ WorkSplit decode_prologue(const DecodeParams& p, int3
     for (int i = tid; i <= S; i += NTHREADS) p.header[kHeaderInts + i] = prefix[i];
   }
   const int Hq = p.num_q_heads;
-  for (int s = blockIdx.x; s < S; s += gridDim.x) {
+  for (int s = p.cascade ? S : blockIdx.x; s < S; s += gridDim.x) {
     if (prefix[s + 1] == prefix[s]) {
       uint4* o = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + static_cast<int64_t>(s) * Hq * D);
       for (int i = tid; i < Hq * D / 8; i += NTHREADS) o[i] = make_uint4(0u, 0u, 0u, 0u);

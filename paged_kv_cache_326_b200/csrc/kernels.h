@@ -96,6 +96,9 @@ struct DecodeArgs {
   const void* k_new = nullptr;
   const void* v_new = nullptr;
   const int64_t* slot_mapping = nullptr;
+  // One pass of the shared-prefix decode: partial records only, no merge
+  // (and, on the grouped-query kernel, queries taken from a group's texts).
+  bool cascade = false;
 };
 
 bool decode_sizes_supported(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
@@ -119,6 +122,48 @@ bool mma_decode_pool_ok(int num_kv_heads, int block_size, int64_t num_blocks);
 size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                   int block_size, int max_blocks_per_seq, int64_t forced_warps);
 cudaError_t launch_paged_attn_decode_mma(const DecodeArgs& a, cudaStream_t stream);
+
+// The shared-prefix pass of the grouped-query kernel (a.cascade set, a
+// multi-head pool): a.num_seqs groups of `group_size` texts, each group's
+// texts' queries as the columns of one key/value head.  Partial records
+// only, no merge.
+bool mma_cascade_ok(int num_heads, int group_size, int head_dim, int block_size);
+size_t mma_cascade_workspace_bytes(int num_groups, int group_size, int num_heads, int head_dim,
+                                   int block_size, int max_blocks_per_seq, int64_t forced_warps);
+cudaError_t launch_paged_attn_decode_mma_cascade(const DecodeArgs& a, int group_size,
+                                                 cudaStream_t stream);
+
+// Shared-prefix decode (shared_prefix.cu): the prefix pass, the tail pass,
+// then the merge of both passes' records.
+struct SharedPrefixArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* prefix_tables;
+  const int32_t* prefix_lens;
+  int max_prefix_blocks;
+  const int32_t* tail_tables;
+  const int32_t* tail_lens;
+  int max_tail_blocks;
+  float scale;
+  int num_groups;
+  int group_size;
+  int num_heads;
+  int head_dim;
+  int block_size;
+  int64_t num_blocks;
+  int is_bf16;
+  void* workspace;
+  size_t workspace_bytes;
+  int32_t* status;
+  int64_t wait_limit_ns;
+  int64_t forced_warps;
+};
+size_t shared_prefix_workspace_bytes(int num_groups, int group_size, int num_heads, int head_dim,
+                                     int block_size, int max_prefix_blocks, int max_tail_blocks,
+                                     int64_t forced_warps);
+cudaError_t launch_paged_attn_decode_shared(const SharedPrefixArgs& a, cudaStream_t stream);
 
 // Launches the decode kernel and the split reduce on `stream`.
 // Returns cudaErrorInvalidValue for unsupported sizes or a short workspace.

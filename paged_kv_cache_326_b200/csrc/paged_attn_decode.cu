@@ -397,7 +397,7 @@ paged_decode_kernel(const DecodeParams p) {
     if (unit_ends || j == ns - 1) {
       const int64_t sh = static_cast<int64_t>(s) * H + h;          // (text, virtual head)
       const int64_t qrow = static_cast<int64_t>(s) * Hq + q_head0(h);  // first query head
-      const bool whole = piece_j0 == 0 && j == ns - 1;
+      const bool whole = piece_j0 == 0 && j == ns - 1 && !p.cascade;
       float* recs = p.records + (static_cast<int64_t>(wu0) + sh) * (GS * (D + 4));
 #pragma unroll
       for (int g = 0; g < GS; ++g) {
@@ -526,6 +526,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   p.k_new = a.k_new;
   p.v_new = a.v_new;
   p.slot_mapping = a.slot_mapping;
+  p.cascade = a.cascade ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(kDecodeWarps * 32);
@@ -539,6 +540,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   cudaError_t err = cudaLaunchKernelEx(
       &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS, F8>, p);
   if (err != cudaSuccess) return err;
+  if (p.cascade) return cudaGetLastError();  // the caller merges
   err = launch_merge<T, D>(p, GS, stream);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();

@@ -199,9 +199,17 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
       const uint32_t qbytes = first ? GS * D * 2 : 0;
       const uint32_t kvbytes = bad ? 0 : 2u * HALVES * boxes * BOX_BYTES;
       mbar_arrive_expect_tx(&bars[st], qbytes + kvbytes);
-      if (first)
-        bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D, GS * D * 2,
-                      &bars[st], policy);
+      if (first) {
+        if (!p.cascade) {
+          bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D, GS * D * 2,
+                        &bars[st], policy);
+        } else {
+          // head h of the group's GS texts: rows Hq * D elements apart
+          for (int g = 0; g < GS; ++g)
+            bulk_copy_g2s(sQ + g * D * 2, qg + ((static_cast<int64_t>(s) * GS + g) * Hq + h) * D,
+                          D * 2, &bars[st], policy);
+        }
+      }
       if (!bad) {
         const int kvh = kv_head(h);
         const int row0 = CH >= B ? 0 : (j * CH) % B;
@@ -439,7 +447,7 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
     if (unit_ends || j == ns - 1) {
       const int64_t sh = static_cast<int64_t>(s) * p.num_heads + h;  // (text, virtual head)
       const int64_t qrow = static_cast<int64_t>(s) * Hq + q_head0(h);  // first query head
-      const bool whole = piece_j0 == 0 && j == ns - 1;
+      const bool whole = piece_j0 == 0 && j == ns - 1 && !p.cascade;
       float lt[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
@@ -601,6 +609,7 @@ cudaError_t launch_mma_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStre
   p.k_new = nullptr;
   p.v_new = nullptr;
   p.slot_mapping = nullptr;
+  p.cascade = a.cascade ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(kMmaWarps * 32);
@@ -614,6 +623,7 @@ cudaError_t launch_mma_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStre
   cudaError_t err = cudaLaunchKernelEx(
       &cfg, paged_decode_mma_kernel<T, D, B, kMmaWarps, kMmaStages, NT>, p, tm_k, tm_v);
   if (err != cudaSuccess) return err;
+  if (p.cascade) return cudaGetLastError();  // the caller merges
   err = launch_merge<T, D>(p, hl.gs, stream);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
@@ -665,9 +675,10 @@ bool mma_decode_pool_ok(int num_kv_heads, int block_size, int64_t num_blocks) {
   return num_blocks > 0 && num_blocks * num_kv_heads * block_size < (int64_t{1} << 31);
 }
 
-size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                                  int block_size, int max_blocks_per_seq, int64_t forced_warps) {
-  const HeadLayout hl = mma_head_layout(num_heads, num_kv_heads);
+namespace {
+
+size_t mma_workspace_for(int num_seqs, const HeadLayout& hl, int head_dim, int block_size,
+                         int max_blocks_per_seq, int64_t forced_warps) {
   if (hl.vheads < 1) return 0;
   const int nt = column_tiles(hl.gs);
   int64_t warps = 0;
@@ -686,6 +697,49 @@ size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
   const int64_t segs = static_cast<int64_t>(num_seqs) * hl.vheads;
   return header_bytes(num_seqs) + kGrabBytes +
          records_bytes(max_units(warps) + segs, head_dim, hl.gs);
+}
+
+// The shared-prefix pass: one virtual text per group, one subset of
+// `group_size` query columns (the group's texts) per head.
+HeadLayout cascade_head_layout(int num_heads, int group_size) {
+  HeadLayout l;
+  l.group = 1;
+  l.gs = group_size;
+  l.nsub = 1;
+  l.vheads = num_heads;
+  return l;
+}
+
+}  // namespace
+
+size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int max_blocks_per_seq, int64_t forced_warps) {
+  return mma_workspace_for(num_seqs, mma_head_layout(num_heads, num_kv_heads), head_dim,
+                           block_size, max_blocks_per_seq, forced_warps);
+}
+
+bool mma_cascade_ok(int num_heads, int group_size, int head_dim, int block_size) {
+  return num_heads >= 1 && group_size >= 1 && group_size <= 16 &&
+         (head_dim == 64 || head_dim == 128) &&
+         (block_size == 8 || block_size == 16 || block_size == 32);
+}
+
+size_t mma_cascade_workspace_bytes(int num_groups, int group_size, int num_heads, int head_dim,
+                                   int block_size, int max_blocks_per_seq, int64_t forced_warps) {
+  if (!mma_cascade_ok(num_heads, group_size, head_dim, block_size)) return 0;
+  return mma_workspace_for(num_groups, cascade_head_layout(num_heads, group_size), head_dim,
+                           block_size, max_blocks_per_seq, forced_warps);
+}
+
+cudaError_t launch_paged_attn_decode_mma_cascade(const DecodeArgs& a, int group_size,
+                                                 cudaStream_t stream) {
+  if (!a.cascade || a.slot_mapping || a.fp8 || a.num_heads != a.num_kv_heads ||
+      !mma_cascade_ok(a.num_heads, group_size, a.head_dim, a.block_size) ||
+      !mma_decode_pool_ok(a.num_kv_heads, a.block_size, a.num_blocks))
+    return cudaErrorInvalidValue;
+  const HeadLayout hl = cascade_head_layout(a.num_heads, group_size);
+  return a.is_bf16 ? mma_dispatch<__nv_bfloat16>(a, hl, stream)
+                   : mma_dispatch<__half>(a, hl, stream);
 }
 
 cudaError_t launch_paged_attn_decode_mma(const DecodeArgs& a, cudaStream_t stream) {

@@ -571,3 +571,134 @@ def pin_prefill_first_row_and_brute_force(prefill_fn):
 
 PREFILL_PINS = [pin_prefill_vs_torch_causal, pin_prefill_last_row_is_decode,
                 pin_prefill_first_row_and_brute_force]
+
+
+# ---------------------------------------------------------------------------
+# shared prefixes
+# ---------------------------------------------------------------------------
+
+def _forked_groups(prompt_lens, tail_lens, group_size, H, D, B, seed, dtype=torch.float16):
+    """Groups of texts built as the block manager builds them, written out by
+    hand: the prompt's full blocks are stored once and listed first in every
+    member's table; a partial last prompt block is copied into each member's
+    first private block (copy on write), followed by the member's own tokens.
+    Returns q, the contiguous K and V of every text, the pool, and the prefix
+    and tail tables and lengths."""
+    g = torch.Generator().manual_seed(seed)
+    G = len(prompt_lens)
+    S = G * group_size
+    prompts = [(torch.randn(L, H, D, generator=g).to(dtype), torch.randn(L, H, D, generator=g).to(dtype))
+               for L in prompt_lens]
+    tails = [(torch.randn(L, H, D, generator=g).to(dtype), torch.randn(L, H, D, generator=g).to(dtype))
+             for L in tail_lens]
+    q = torch.randn(S, H, D, generator=g).to(dtype)
+    nb = sum(L // B for L in prompt_lens) + 8
+    nb += sum(-(-(prompt_lens[s // group_size] % B + tail_lens[s]) // B) for s in range(S))
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(seed + 5)).tolist()
+    kc = torch.full((nb, H, B, D), float("nan"), dtype=dtype)
+    vc = torch.full((nb, H, B, D), float("nan"), dtype=dtype)
+    at = 0
+    prefix_tables, prefix_lens, tail_tables, K, V = [], [], [], [], []
+    for gi, L in enumerate(prompt_lens):
+        pk, pv = prompts[gi]
+        full = L // B
+        row = []
+        for j in range(full):
+            phys = perm[at]
+            at += 1
+            kc[phys] = pk[j * B:(j + 1) * B].permute(1, 0, 2)
+            vc[phys] = pv[j * B:(j + 1) * B].permute(1, 0, 2)
+            row.append(phys)
+        prefix_tables.append(row)
+        prefix_lens.append(full * B)
+        for m in range(group_size):
+            s = gi * group_size + m
+            tk, tv = tails[s]
+            own_k = torch.cat([pk[full * B:], tk])
+            own_v = torch.cat([pv[full * B:], tv])
+            trow = []
+            for j in range(-(-own_k.shape[0] // B)):
+                phys = perm[at]
+                at += 1
+                lo, hi = j * B, min(own_k.shape[0], (j + 1) * B)
+                kc[phys, :, :hi - lo] = own_k[lo:hi].permute(1, 0, 2)
+                vc[phys, :, :hi - lo] = own_v[lo:hi].permute(1, 0, 2)
+                trow.append(phys)
+            tail_tables.append(trow)
+            K.append(torch.cat([pk, tk]))
+            V.append(torch.cat([pv, tv]))
+    t_lens = [K[s].shape[0] - prefix_lens[s // group_size] for s in range(S)]
+    return q, K, V, kc, vc, prefix_tables, prefix_lens, tail_tables, t_lens
+
+
+def pin_shared_vs_unpaged_sdpa(shared_fn):
+    """Two groups of three forked texts (prompts of 13 and 8 tokens, B = 4)
+    against torch's fp64 attention on each text's contiguous tokens."""
+    H, D, B, gs = 2, 8, 4, 3
+    q, K, V, kc, vc, pt, pl, tt, tl = _forked_groups([13, 8], [1, 5, 3, 2, 0, 7], gs, H, D, B, 601)
+    got = shared_fn(f64(q), f64(kc), f64(vc), pt, pl, tt, tl, gs, 0.35, B)
+    ref = sdpa_contiguous(q, K, V, 0.35)
+    err = np.abs(got - ref).max()
+    assert err <= 1e-12, f"shared prefix vs unpaged sdpa: max err {err}"
+
+
+def pin_shared_brute_force_and_empty(shared_fn):
+    """Scalar brute force on a tiny group; a group with no shared block (a
+    prompt shorter than a block) and a text with no tokens at all."""
+    H, D, B, gs = 1, 4, 4, 2
+    q, K, V, kc, vc, pt, pl, tt, tl = _forked_groups([9, 3], [2, 1, 0, 4], gs, H, D, B, 611)
+    assert pl[1] == 0, "the second prompt has no full block"
+    got = shared_fn(f64(q), f64(kc), f64(vc), pt, pl, tt, tl, gs, 0.5, B)
+    ref = brute_force(q, K, V, 0.5)
+    assert np.abs(got - ref).max() <= 1e-12, "shared prefix vs brute force"
+    q2, K2, V2, kc2, vc2, pt2, pl2, tt2, tl2 = _forked_groups([0], [0, 2], 2, H, D, B, 612)
+    got2 = shared_fn(f64(q2), f64(kc2), f64(vc2), pt2, pl2, tt2, tl2, 2, 0.5, B)
+    assert np.array_equal(got2[0], np.zeros((H, D))), "a text with no tokens is not zero"
+    assert np.abs(got2[1] - brute_force(q2[1:], K2[1:], V2[1:], 0.5)[0]).max() <= 1e-12
+
+
+def pin_split_worked_example(split_fn):
+    """Hand-worked splits (B = 16): two pairs whose first two blocks agree,
+    then diverge; a pair right after a fork, whose shared second block is
+    only partly filled (so it stays out of the prefix); a trio whose third
+    member differs at block 1; a pair with nothing in common."""
+    bt = [[5, 6, 7, -1], [5, 6, 8, -1], [5, 9, 10, 11], [5, 9, 12, -1]]
+    got = split_fn(np.array(bt), [40, 36, 64, 48], 16, 2)
+    want = ([[5, 6], [5, 9]], [32, 32], [[7], [8], [10, 11], [12]], [8, 4, 32, 16])
+    assert [list(map(list, got[0])), list(got[1]), list(map(list, got[2])), list(got[3])] == \
+        [want[0], want[1], want[2], want[3]], f"worked split: {got}"
+    got = split_fn(np.array([[3, 4], [3, 4]]), [20, 20], 16, 2)
+    assert list(map(list, got[0])) == [[3]] and list(got[1]) == [16], "partial shared block"
+    assert list(map(list, got[2])) == [[4], [4]] and list(got[3]) == [4, 4]
+    got = split_fn(np.array([[1, 2, 3], [1, 2, 4], [1, 7, 8]]), [48, 48, 48], 16, 3)
+    assert list(map(list, got[0])) == [[1]] and list(got[1]) == [16], "trio"
+    assert list(map(list, got[2])) == [[2, 3], [2, 4], [7, 8]] and list(got[3]) == [32, 32, 32]
+    got = split_fn(np.array([[1, 2], [3, 2]]), [32, 32], 16, 2)
+    assert list(map(list, got[0])) == [[]] and list(got[1]) == [0], "nothing shared"
+    assert list(map(list, got[2])) == [[1, 2], [3, 2]] and list(got[3]) == [32, 32]
+
+
+def pin_split_then_shared_is_decode(split_fn, shared_fn):
+    """Splitting forked tables and attending over prefix then tail reads the
+    same tokens in the same order as the joined table: the output equals
+    plain paged decode bit for bit."""
+    from oracle import paged_decode
+    H, D, B, gs = 2, 8, 4, 4
+    q, K, V, kc, vc, pt, pl, tt, tl = _forked_groups([14, 4, 17], [3, 1, 6, 2, 5, 0, 4, 4, 1, 2, 3, 9],
+                                                     gs, H, D, B, 621)
+    S = q.shape[0]
+    width = max(len(pt[s // gs]) + len(tt[s]) for s in range(S))
+    joined = np.full((S, width), -1, dtype=np.int64)
+    lens = []
+    for s in range(S):
+        row = pt[s // gs] + tt[s]
+        joined[s, :len(row)] = row
+        lens.append(pl[s // gs] + tl[s])
+    ref = paged_decode(f64(q), f64(kc), f64(vc), joined, lens, 0.3, B)
+    spt, spl, stt, stl = split_fn(joined, lens, B, gs)
+    got = shared_fn(f64(q), f64(kc), f64(vc), spt, spl, stt, stl, gs, 0.3, B)
+    assert np.array_equal(got, ref), "split + shared decode differs from paged decode"
+
+
+SHARED_PINS = [pin_shared_vs_unpaged_sdpa, pin_shared_brute_force_and_empty]
+SPLIT_PINS = [pin_split_worked_example]

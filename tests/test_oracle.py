@@ -107,3 +107,17 @@ def test_fp8_cache_write_stores_the_codes_at_the_slots():
 @pytest.mark.parametrize("pin", P.PREFILL_PINS, ids=lambda f: f.__name__)
 def test_prefill_pin(pin):
     pin(oracle.prefill)
+
+
+@pytest.mark.parametrize("pin", P.SHARED_PINS, ids=lambda f: f.__name__)
+def test_shared_prefix_oracle_pin(pin):
+    pin(oracle.paged_decode_shared)
+
+
+@pytest.mark.parametrize("pin", P.SPLIT_PINS, ids=lambda f: f.__name__)
+def test_split_oracle_pin(pin):
+    pin(oracle.split_shared_prefix)
+
+
+def test_split_then_shared_is_paged_decode():
+    P.pin_split_then_shared_is_decode(oracle.split_shared_prefix, oracle.paged_decode_shared)

@@ -335,3 +335,100 @@ def test_planted_prefill_mistake_is_caught(fn):
         except (AssertionError, ValueError, IndexError):
             failed += 1
     assert failed, fn.__name__
+
+
+# --- shared prefixes: planted mistakes ----------------------------------------
+
+def _shared_with(group_of=None, use_prefix=True, use_tail=True):
+    def fn(q, kc, vc, pt, pl, tt, tl, gs, scale, B):
+        S, H, D = q.shape
+        out = np.zeros((S, H, D))
+        G = len(pl)
+        for t in range(S):
+            g = group_of(t, gs, G) if group_of else t // gs
+            parts_k, parts_v = [], []
+            if use_prefix:
+                parts_k.append(oracle.gather_context(kc, pt[g], pl[g], B))
+                parts_v.append(oracle.gather_context(vc, pt[g], pl[g], B))
+            if use_tail:
+                parts_k.append(oracle.gather_context(kc, tt[t], tl[t], B))
+                parts_v.append(oracle.gather_context(vc, tt[t], tl[t], B))
+            K = np.concatenate(parts_k) if parts_k else np.zeros((0, H, D))
+            V = np.concatenate(parts_v) if parts_v else np.zeros((0, H, D))
+            out[t] = oracle.attend(q[t], K, V, scale)
+        return out
+    return fn
+
+
+SHARED_MUTANTS = {
+    "prefix_of_wrong_group": _shared_with(group_of=lambda t, gs, G: t % G),
+    "prefix_dropped": _shared_with(use_prefix=False),
+    "tail_dropped": _shared_with(use_tail=False),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SHARED_MUTANTS))
+def test_planted_shared_prefix_mistake_is_caught(name):
+    failed = 0
+    for pin in P.SHARED_PINS:
+        try:
+            pin(SHARED_MUTANTS[name])
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    assert failed, name
+
+
+def split_ignores_fill(bt, lens, B, gs):
+    """Planted mistake: a shared block counts even when partly filled."""
+    S = len(lens)
+    pt, pl, tt, tl = [], [], [], []
+    for g in range(S // gs):
+        first = bt[g * gs]
+        p = 0
+        while p < len(first) and first[p] >= 0 and all(bt[s][p] == first[p]
+                                                       for s in range(g * gs, (g + 1) * gs)):
+            p += 1
+        pt.append([int(b) for b in first[:p]])
+        pl.append(min(p * B, min(lens[g * gs:(g + 1) * gs])))
+        for s in range(g * gs, (g + 1) * gs):
+            rest = lens[s] - pl[-1]
+            tt.append([int(b) for b in bt[s][p:p + -(-rest // B)]])
+            tl.append(rest)
+    return pt, pl, tt, tl
+
+
+def split_first_member_only(bt, lens, B, gs):
+    """Planted mistake: the prefix is read off the group's first table only."""
+    S = len(lens)
+    pt, pl, tt, tl = [], [], [], []
+    for g in range(S // gs):
+        first = bt[g * gs]
+        p = 0
+        while p < len(first) and (p + 1) * B <= lens[g * gs]:
+            p += 1
+        pt.append([int(b) for b in first[:p]])
+        pl.append(p * B)
+        for s in range(g * gs, (g + 1) * gs):
+            rest = lens[s] - p * B
+            tt.append([int(b) for b in bt[s][p:p + -(-rest // B)]])
+            tl.append(rest)
+    return pt, pl, tt, tl
+
+
+@pytest.mark.parametrize("fn", [split_ignores_fill, split_first_member_only],
+                         ids=lambda f: f.__name__)
+def test_planted_split_mistake_is_caught(fn):
+    failed = 0
+    for pin in P.SPLIT_PINS:
+        try:
+            pin(fn)
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    assert failed, fn.__name__
+
+
+def test_unmodified_oracle_passes_shared_pins():
+    for pin in P.SHARED_PINS:
+        pin(oracle.paged_decode_shared)
+    for pin in P.SPLIT_PINS:
+        pin(oracle.split_shared_prefix)
