@@ -99,6 +99,8 @@ struct DecodeParams {
   // kernel merges the records of both passes).  In the grouped-query kernel
   // the gs query heads of virtual text s and head h are then the same head h
   // of texts s * gs .. s * gs + gs - 1 (q laid out [texts][heads][D]).
+  // 2: as 1, for a pass whose predecessor on the stream is the other pass
+  // (it waits for that grid at its exit instead of its start).
   int cascade = 0;
 };
 

@@ -99,6 +99,10 @@ struct DecodeArgs {
   // One pass of the shared-prefix decode: partial records only, no merge
   // (and, on the grouped-query kernel, queries taken from a group's texts).
   bool cascade = false;
+  // With cascade: the kernel launched just before this one (on the same
+  // stream, also a cascade pass) triggers its dependents early and writes
+  // nothing this pass reads; this pass then waits for it only at its exit.
+  bool cascade_overlap = false;
 };
 
 bool decode_sizes_supported(int num_seqs, int num_heads, int num_kv_heads, int head_dim,

@@ -126,7 +126,11 @@ paged_decode_kernel(const DecodeParams p) {
   const int warp = tid >> 5;
 
   // Inputs may come from the kernel launched just before (the cache write).
-  griddep_wait();
+  // The tail pass of a shared-prefix decode reads nothing the pass before it
+  // writes: it starts at once and waits for that pass only on its way out,
+  // so that the merge launched after it sees both passes' records.
+  const bool wait_at_exit = p.cascade == 2;
+  if (!wait_at_exit) griddep_wait();
 
   const WorkSplit sp = decode_prologue<T, D, CH, WARPS * 32>(p, prefix, warp_tot, cap);
   const int total = sp.total;
@@ -139,9 +143,13 @@ paged_decode_kernel(const DecodeParams p) {
   auto fused_write = [&]() {
     if constexpr (FUSED) fused_cache_write<D, B>(p, w, W, lane);
   };
-  if (w >= W) return;
+  if (w >= W) {
+    if (wait_at_exit) griddep_wait();
+    return;
+  }
   if (total == 0) {
     fused_write();
+    if (wait_at_exit) griddep_wait();
     return;
   }
 
@@ -279,6 +287,7 @@ paged_decode_kernel(const DecodeParams p) {
       set_status(p.status, -10 /* PA_ERR_TIMEOUT */);
       for (int d = pos; d < issued; ++d)
         mbar_wait_bounded(&bars[d % STAGES], (d / STAGES) & 1, kDrainLimitNs);
+      if (wait_at_exit) griddep_wait();
       return;
     }
 
@@ -452,6 +461,7 @@ paged_decode_kernel(const DecodeParams p) {
       i0 = 0;
     }
   }
+  if (wait_at_exit) griddep_wait();
 }
 
 namespace {
@@ -526,7 +536,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   p.k_new = a.k_new;
   p.v_new = a.v_new;
   p.slot_mapping = a.slot_mapping;
-  p.cascade = a.cascade ? 1 : 0;
+  p.cascade = a.cascade ? (a.cascade_overlap ? 2 : 1) : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(kDecodeWarps * 32);

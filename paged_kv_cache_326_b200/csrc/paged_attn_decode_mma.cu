@@ -116,6 +116,8 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
   }
   // Inputs may come from the kernel launched just before (the cache write).
   griddep_wait();
+  // A shared-prefix pass lets the tail pass after it start on SMs it leaves.
+  if (p.cascade) griddep_launch_dependents();
 
   const WorkSplit sp = decode_prologue<T, D, CH, WARPS * 32>(p, prefix, warp_tot, cap);
   const int W = sp.W;

@@ -19,7 +19,11 @@
 //                rounding: the log-sum-exp merge is exact algebra).
 //
 // Both passes run with their `cascade` flag set: every work unit leaves a
-// record, none writes an output, so the merge sees every partial.
+// record, none writes an output, so the merge sees every partial.  The prefix
+// pass triggers its dependents as soon as its inputs are ready, so the tail
+// pass (which reads nothing the prefix pass writes) fills SMs as prefix CTAs
+// finish; the tail pass waits for the prefix grid on its way out, so the
+// merge, which waits for the tail grid, sees both passes' records.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -230,6 +234,7 @@ cudaError_t launch_paged_attn_decode_shared(const SharedPrefixArgs& a, cudaStrea
   tp.max_blocks_per_seq = a.max_tail_blocks;
   tp.workspace = ws_t;
   tp.workspace_bytes = t_bytes;
+  tp.cascade_overlap = true;
   err = launch_paged_attn_decode(tp, stream);
   if (err != cudaSuccess) return err;
 

@@ -10,8 +10,10 @@ on 8 key/value heads; always the two-call path, the one-launch step being
 multi-head only), ``opt13b_batch64_fp8`` (the batch-64 step over 8-bit
 caches, two calls), ``opt13b_prefill`` (the prompt phase: S prompts of 2,048
 tokens, 40 heads of 128; ``--prefill-kernel`` 0 automatic, 1 mma.sync, 2
-tcgen05).  ``--gqa-kernel`` picks the grouped-query kernel (0 automatic, 1
-CUDA cores, 2 tensor cores).
+tcgen05), ``shared_prefix`` (32 prompts x 8 samples built by the block
+manager, through pa_paged_attn_decode_shared over the split tables).
+``--gqa-kernel`` picks the grouped-query kernel (0 automatic, 1 CUDA cores, 2
+tensor cores).
 """
 from __future__ import annotations
 
@@ -65,6 +67,30 @@ def main():
         if status.item() != 0:
             raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
         print(f"{len(w.lens)} prompts of {w.lens[0]} tokens, status ok")
+        return
+    if args.workload == "shared_prefix":
+        bm = P.BlockManager(8192, 16)
+
+        class Adapter:
+            add_seq = staticmethod(bm.add_seq)
+            fork = staticmethod(bm.fork)
+            append_slot = staticmethod(bm.append_slot)
+            export = staticmethod(lambda ids, m: tuple(t.numpy() for t in bm.export(ids, m)))
+
+        w = W.shared_prefix(Adapter, num_blocks=8192, seed=4, device=dev)
+        gs = w.meta["samples"]
+        pt, pl, tt, tl = [t.to(dev) for t in P.split_shared_prefix(
+            w.block_tables.cpu(), w.context_lens.cpu(), w.block_size, gs)]
+        out = torch.empty_like(w.q)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        for _ in range(args.reps):
+            P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+            P.pa_paged_attn_decode_shared(out, w.q, w.k_cache, w.v_cache, pt, pl, tt, tl,
+                                          w.scale, gs, status=status)
+        torch.cuda.synchronize()
+        if status.item() != 0:
+            raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
+        print(f"shared_prefix: {w.num_seqs} texts in groups of {gs}, status ok")
         return
     w = make(args.workload, args.num_seqs, dev)
     gqa = w.k_cache.shape[1] != w.num_heads
