@@ -52,6 +52,12 @@ TRAFFIC = {
          "paged_kv_cache_326_b200/csrc/decode_common.cuh",
          "paged_kv_cache_326_b200/csrc/mma_ptx.cuh",
          "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
+    "opt13b_batch64_fp8": (
+        os.path.join(ROOT, "profiles", "paged_decode_fp8_opt13b_batch64_traffic.json"),
+        ["paged_kv_cache_326_b200/csrc/paged_attn_decode.cu",
+         "paged_kv_cache_326_b200/csrc/decode_common.cuh",
+         "paged_kv_cache_326_b200/csrc/fp8.cuh",
+         "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
     # the shared-prefix call: prefix pass + tail pass + merge, summed
     "shared_prefix": (
         os.path.join(ROOT, "profiles", "paged_decode_shared_prefix_c4_traffic.json"),
@@ -910,7 +916,8 @@ def main():
                       {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": (None if fp8 else traffic_per_launch(args.workload, args.path)),
+                     "traffic": traffic_per_launch(args.workload + ("_fp8" if fp8 else ""),
+                                                   args.path),
                      "kernel": ("pa_paged_attn_decode_shared (prefix pass on the tensor cores, "
                                 "tail pass, merge kernel)" if cascade else
                                 "pa_decode_step (decode kernel with the cache write, + merge kernel)"

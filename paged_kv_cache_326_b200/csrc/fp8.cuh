@@ -23,6 +23,27 @@ __device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t x) {
   return *reinterpret_cast<__half2*>(&r);
 }
 
+// Four codes (one 32-bit word, low byte first) -> two half2 words: codes 0, 1
+// in `lo`, codes 2, 3 in `hi` (exact).
+__device__ __forceinline__ void e4m3x4_to_half2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// c + a.x * b.x + a.y * b.y for two fp16 pairs (a, b packed as half2 words),
+// summed in fp32: each fp16 x fp16 product is exact in fp32.
+__device__ __forceinline__ float dot2_f16_f32(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 t, a0, b0, %3;\n\tfma.rn.f32.f16 %0, a1, b1, t;\n\t}"
+      : "=f"(d)
+      : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+
 // Sixteen codes (one 16-byte vector) -> sixteen floats.
 __device__ __forceinline__ void unpack16_e4m3(const uint4& v, float (&f)[16]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};

@@ -50,6 +50,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "decode_common.cuh"
 #include "fp8.cuh"
@@ -269,7 +270,12 @@ paged_decode_kernel(const DecodeParams p) {
   const int dchunk = lane % LPT;
   const int tsub = lane / LPT;
   // Per query head of this unit (GS of them share every K/V row read).
+  // An 8-bit cache with fp16 queries keeps the query as raw fp16 pairs and
+  // forms the scores with fp16 x fp16 -> fp32 FMAs straight from the widened
+  // codes (exact products; the scale is applied to the sum).
+  constexpr bool MIXED = F8 && std::is_same<T, __half>::value;
   float qf[GS][VEC];
+  uint32_t qh[GS][MIXED ? VEC / 2 : 1];
   float acc[GS][VEC];
   float m[GS], lsum[GS];
   int piece_j0 = 0;
@@ -303,13 +309,20 @@ paged_decode_kernel(const DecodeParams p) {
       for (int g = 0; g < GS; ++g) {
 #pragma unroll
         for (int h8 = 0; h8 < VEC / 8; ++h8) {
-          float qraw[8];
-          unpack8<T>(*reinterpret_cast<const uint4*>(sQ + g * D + dchunk * VEC + h8 * 8), qraw);
+          const uint4 qv = *reinterpret_cast<const uint4*>(sQ + g * D + dchunk * VEC + h8 * 8);
+          if constexpr (MIXED) {
+            qh[g][h8 * 4 + 0] = qv.x;
+            qh[g][h8 * 4 + 1] = qv.y;
+            qh[g][h8 * 4 + 2] = qv.z;
+            qh[g][h8 * 4 + 3] = qv.w;
+          } else {
+            float qraw[8];
+            unpack8<T>(qv, qraw);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            qf[g][h8 * 8 + k] = qraw[k] * p.qk_scale_log2;
-            acc[g][h8 * 8 + k] = 0.f;
+            for (int k = 0; k < 8; ++k) qf[g][h8 * 8 + k] = qraw[k] * p.qk_scale_log2;
           }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[g][h8 * 8 + k] = 0.f;
         }
         m[g] = -INFINITY;
         lsum[g] = 0.f;
@@ -321,14 +334,32 @@ paged_decode_kernel(const DecodeParams p) {
     float sc[GS][ITERS];
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-      float kf[VEC];
-      load_vec(sK + (it * TPI + tsub) * ROWB + dchunk * 16, kf);
+      if constexpr (MIXED) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(sK + (it * TPI + tsub) * ROWB + dchunk * 16);
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t kh[VEC / 2];
 #pragma unroll
-      for (int g = 0; g < GS; ++g) {
-        float d0 = qf[g][0] * kf[0];
+        for (int i = 0; i < 4; ++i) e4m3x4_to_half2x2(kw[i], kh[2 * i], kh[2 * i + 1]);
 #pragma unroll
-        for (int k = 1; k < VEC; ++k) d0 = fmaf(qf[g][k], kf[k], d0);
-        sc[g][it] = d0;
+        for (int g = 0; g < GS; ++g) {
+          float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+          for (int i = 0; i < VEC / 2; i += 2) {
+            d0 = dot2_f16_f32(qh[g][i], kh[i], d0);
+            d1 = dot2_f16_f32(qh[g][i + 1], kh[i + 1], d1);
+          }
+          sc[g][it] = (d0 + d1) * p.qk_scale_log2;
+        }
+      } else {
+        float kf[VEC];
+        load_vec(sK + (it * TPI + tsub) * ROWB + dchunk * 16, kf);
+#pragma unroll
+        for (int g = 0; g < GS; ++g) {
+          float d0 = qf[g][0] * kf[0];
+#pragma unroll
+          for (int k = 1; k < VEC; ++k) d0 = fmaf(qf[g][k], kf[k], d0);
+          sc[g][it] = d0;
+        }
       }
     }
 #pragma unroll
@@ -372,28 +403,34 @@ paged_decode_kernel(const DecodeParams p) {
         for (int it = 0; it < ITERS; ++it) sc[g][it] = 0.f;
       }
     }
-    if (nvalid == CH) {
+    // acc += p * v for one token row (packed fp32 FMAs on the 8-bit cache)
+    auto accumulate = [&](int it) {
+      float vf[VEC];
+      load_vec(sV + (it * TPI + tsub) * ROWB + dchunk * 16, vf);
 #pragma unroll
-      for (int it = 0; it < ITERS; ++it) {
-        float vf[VEC];
-        load_vec(sV + (it * TPI + tsub) * ROWB + dchunk * 16, vf);
+      for (int g = 0; g < GS; ++g) {
+        if constexpr (F8) {
+          const float2 p2 = make_float2(sc[g][it], sc[g][it]);
 #pragma unroll
-        for (int g = 0; g < GS; ++g)
+          for (int k = 0; k < VEC; k += 2) {
+            const float2 r = __ffma2_rn(p2, make_float2(vf[k], vf[k + 1]),
+                                        make_float2(acc[g][k], acc[g][k + 1]));
+            acc[g][k] = r.x;
+            acc[g][k + 1] = r.y;
+          }
+        } else {
 #pragma unroll
           for (int k = 0; k < VEC; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
-      }
-    } else {
-#pragma unroll
-      for (int it = 0; it < ITERS; ++it) {
-        if (it * TPI + tsub < nvalid) {
-          float vf[VEC];
-          load_vec(sV + (it * TPI + tsub) * ROWB + dchunk * 16, vf);
-#pragma unroll
-          for (int g = 0; g < GS; ++g)
-#pragma unroll
-            for (int k = 0; k < VEC; ++k) acc[g][k] = fmaf(sc[g][it], vf[k], acc[g][k]);
         }
       }
+    };
+    if (nvalid == CH) {
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) accumulate(it);
+    } else {
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it)
+        if (it * TPI + tsub < nvalid) accumulate(it);
     }
 
     // This stage is consumed: refill it before the epilogue, whose global

@@ -60,7 +60,8 @@ __device__ __forceinline__ void unit_range(const int32_t* header, int s, int h, 
 
 // One warp per (text, head): the prefix pass's records for column j of group
 // t / gs, then the tail pass's records for text t, merged in that fixed order
-// (so the result does not depend on which warp produced a record).
+// (so the result does not depend on which warp produced a record).  Every
+// lane reads the same records, so the running maximum is warp-uniform.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_p,
@@ -88,16 +89,14 @@ shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_
                   : rec_t + (tu + (i - pn) + seg_t) * RS;
   };
 
+  // One pass over the records, four loads in flight at a time; the running
+  // maximum rises batch by batch (a single batch in the usual case: a prefix
+  // and a tail each covered by one or two units).
   float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(rec(i)));
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-
   float L = 0.f;
   float acc[PER];
 #pragma unroll
   for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  // four records' loads in flight at a time
   for (int i0 = 0; i0 < n; i0 += 4) {
     float mv[4], lv[4], o[4][PER];
 #pragma unroll
@@ -117,10 +116,22 @@ shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_
         o[u][1] = v.y;
       }
     }
+    float Mb = M;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (i0 + u < n) Mb = fmaxf(Mb, mv[u]);
+    if (Mb != M) {  // rescale what is summed so far (nothing, in the first batch)
+      const float a = M == -INFINITY ? 0.f : fast_exp2(M - Mb);
+      L *= a;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) acc[k] *= a;
+      M = Mb;
+    }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       if (i0 + u < n) {
-        const float f = fast_exp2(mv[u] - M);
+        // a record of skipped (bad) blocks only carries m = -inf: weight 0
+        const float f = mv[u] == -INFINITY ? 0.f : fast_exp2(mv[u] - M);
         L = fmaf(f, lv[u], L);
 #pragma unroll
         for (int k = 0; k < PER; ++k) acc[k] = fmaf(f, o[u][k], acc[k]);
