@@ -68,6 +68,16 @@ namespace {
 #endif
 constexpr int kDecodeWarps = PA_DECODE_WARPS;    // warps per CTA
 constexpr int kDecodeStages = PA_DECODE_STAGES;  // ring depth per warp
+// The 8-bit kernel is bound by instruction latency more than by copies in
+// flight: two stages let three CTAs (12 warps) share an SM with the same
+// bytes in flight as two CTAs of three stages.
+#ifndef PA_DECODE_STAGES_F8
+#define PA_DECODE_STAGES_F8 2
+#endif
+constexpr int kDecodeStagesF8 = PA_DECODE_STAGES_F8;
+__host__ __device__ constexpr int decode_stages(bool f8) {
+  return f8 ? kDecodeStagesF8 : kDecodeStages;
+}
 // One stage: K rows (4 KB), V rows (4 KB), the unit's GS query rows, a flag.
 __host__ __device__ constexpr int stage_bytes(int D, int gs) { return 2 * 4096 + gs * 2 * D + 128; }
 __host__ __device__ constexpr int warp_area_bytes(int D, int stages, int gs) {
@@ -503,8 +513,8 @@ paged_decode_kernel(const DecodeParams p) {
 
 namespace {
 
-size_t decode_smem_bytes(int D, int num_seqs, int gs) {
-  return static_cast<size_t>(kDecodeWarps) * warp_area_bytes(D, kDecodeStages, gs) +
+size_t decode_smem_bytes(int D, int num_seqs, int gs, bool fp8) {
+  return static_cast<size_t>(kDecodeWarps) * warp_area_bytes(D, decode_stages(fp8), gs) +
          align_up(sizeof(int32_t) * (num_seqs + 1), 16);
 }
 
@@ -523,7 +533,8 @@ HeadLayout head_layout(int num_heads, int num_kv_heads) {
 // Persistent grid for one decode kernel variant.
 Plan plan_variant(const void* kernel, int D, int B, int num_seqs, int vheads,
                   int max_blocks_per_seq, int64_t forced_warps, int gs, bool fp8) {
-  return plan_decode(kernel, decode_smem_bytes(D, num_seqs, gs), decode_smem_bytes(D, kMaxSeqs, gs),
+  return plan_decode(kernel, decode_smem_bytes(D, num_seqs, gs, fp8),
+                     decode_smem_bytes(D, kMaxSeqs, gs, fp8),
                      kDecodeWarps, fp8 ? 4096 / D : chunk_tokens(D), B, num_seqs, vheads,
                      max_blocks_per_seq, forced_warps);
 }
@@ -531,7 +542,7 @@ Plan plan_variant(const void* kernel, int D, int B, int num_seqs, int vheads,
 template <typename T, int D, int B, bool FUSED, int GS, bool F8>
 const void* decode_kernel_ptr() {
   return reinterpret_cast<const void*>(
-      &paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS, F8>);
+      &paged_decode_kernel<T, D, B, kDecodeWarps, decode_stages(F8), FUSED, GS, F8>);
 }
 
 template <typename T, int D, int B, bool FUSED, int GS, bool F8>
@@ -585,7 +596,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(
-      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, kDecodeStages, FUSED, GS, F8>, p);
+      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, decode_stages(F8), FUSED, GS, F8>, p);
   if (err != cudaSuccess) return err;
   if (p.cascade) return cudaGetLastError();  // the caller merges
   err = launch_merge<T, D>(p, GS, stream);
