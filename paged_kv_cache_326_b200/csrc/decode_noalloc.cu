@@ -59,8 +59,10 @@ extern "C" int pa_paged_attn_decode_noalloc(void* out, const void* q, const void
                                             int64_t num_blocks, pa_dtype dt, int32_t* d_status,
                                             pa_stream_t stream) {
   if (num_seqs == 0) return PA_OK;
-  const size_t need = pa::decode_workspace_bytes(num_seqs, num_heads, num_heads, head_dim, block_size,
-                                                 max_blocks_per_seq, pa::option_decode_warps());
+  // only the 16-bit kernels run here
+  const size_t need =
+      pa::decode_workspace_bytes(num_seqs, num_heads, num_heads, head_dim, block_size,
+                                 max_blocks_per_seq, pa::option_decode_warps(), false);
   if (need == 0) return PA_ERR_INVALID;
   if (need > kScratchBytes) return PA_ERR_TOO_LARGE;
   void* scratch = nullptr;

@@ -109,9 +109,11 @@ bool decode_sizes_supported(int num_seqs, int num_heads, int num_kv_heads, int h
                             int block_size, int max_blocks_per_seq);
 
 // Size of the decode workspace for these sizes on the current device, or 0
-// if the sizes are unsupported.
+// if the sizes are unsupported: the most any decode kernel these sizes may
+// run needs (without the 8-bit kernel when with_fp8 is false).
 size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                              int block_size, int max_blocks_per_seq, int64_t forced_warps);
+                              int block_size, int max_blocks_per_seq, int64_t forced_warps,
+                              bool with_fp8 = true);
 
 // Current PA_OPT_DECODE_WARPS setting.
 int64_t option_decode_warps();

@@ -679,7 +679,8 @@ bool decode_sizes_supported(int num_seqs, int num_heads, int num_kv_heads, int h
 }
 
 size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                              int block_size, int max_blocks_per_seq, int64_t forced_warps) {
+                              int block_size, int max_blocks_per_seq, int64_t forced_warps,
+                              bool with_fp8) {
   if (!decode_sizes_supported(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                               max_blocks_per_seq))
     return 0;
@@ -691,6 +692,7 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
     const bool bf16 = variant & 1, fused = variant & 2, fp8 = variant & 4;
     if ((fused || fp8) && hl.gs != 1) continue;
     if (fused && fp8) continue;
+    if (fp8 && !with_fp8) continue;
     const void* k = head_dim == 128 ? kernel_for_variant<128>(block_size, bf16, fused, hl.gs, fp8)
                                     : kernel_for_variant<64>(block_size, bf16, fused, hl.gs, fp8);
     const Plan pl = plan_variant(k, head_dim, block_size, num_seqs, hl.vheads, max_blocks_per_seq,
