@@ -66,3 +66,30 @@ def test_cpp_split_rejects_bad_arguments():
     with pytest.raises(PK.PagedAttnError):  # a tail longer than the tail table
         PK.split_shared_prefix(apart, torch.tensor([32, 32], dtype=torch.int32), 16, 2,
                                max_tail_blocks=1)
+
+
+def test_shared_decode_rejects_bad_arguments_before_launch():
+    """Argument errors return PA_ERR_INVALID before any CUDA call (no GPU)."""
+    import paged_kv_cache_326_b200 as PK
+    lib = PK.lib()
+    bad = PK.binding.PA_ERR_INVALID
+    args = dict(out=None, q=None, kc=None, vc=None, pt=None, pl=None, mp=4, tt=None, tl=None,
+                mt=4, scale=0.1, G=2, gs=8, H=8, D=128, B=16, N=64, dt=0, ws=None, wsb=0,
+                st=None, stream=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.pa_paged_attn_decode_shared(a["out"], a["q"], a["kc"], a["vc"], a["pt"], a["pl"],
+                                               a["mp"], a["tt"], a["tl"], a["mt"], a["scale"],
+                                               a["G"], a["gs"], a["H"], a["D"], a["B"], a["N"],
+                                               a["dt"], a["ws"], a["wsb"], a["st"], a["stream"])
+    assert call(G=0) == PK.binding.PA_OK          # nothing to do
+    assert call() == bad                          # null pointers
+    assert call(gs=17) == bad                     # more texts per group than tile columns
+    assert call(gs=0) == bad
+    assert call(G=513, gs=8) == bad               # more than 4,096 texts
+    assert call(B=4) == bad                       # blocks of 4 do not suit the tensor cores
+    assert call(D=96) == bad
+    assert call(mp=0) == bad and call(mt=0) == bad
+    assert lib.pa_paged_attn_decode_shared_workspace_size(2, 17, 8, 128, 16, 4, 4) == 0
+    assert lib.pa_paged_attn_decode_shared_workspace_size(2, 8, 8, 128, 16, 0, 4) == 0
