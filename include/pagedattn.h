@@ -7,8 +7,8 @@
  * "Shared, Copied on Write") and "KV cache" ("How it works"): each text's keys
  * and values are cut into fixed-size blocks that may sit anywhere in a pool;
  * a per-text block table maps logical to physical blocks; in each generation
- * step the new token's key and value are written into their slot and its
- * query attends over every stored key of its text, the new one included.
+ * step the new token's key and value go to their slot and its query
+ * attends over every stored key of its text, the new one included.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -75,10 +75,10 @@ const char* pa_status_string(int code);
 /*
  * pa_kv_cache_write — store each new token's key and value in its slot.
  *
- * Definition: "KV cache", section "How it works" (the token's own key and
- * value are written into the cache) and "The KV Cache and PagedAttention",
- * section "One Token at a Time" (only the new token's key and value are
- * computed; earlier ones are kept).  For t < num_tokens with slot_mapping[t]
+ * Definition: "KV cache", section "How it works" (each generated token's
+ * key and value join the cache) and "The KV Cache and PagedAttention",
+ * section "One Token at a Time" (a step computes keys and values for the new
+ * token alone and keeps the older ones).  For t < num_tokens with slot_mapping[t]
  * >= 0:  k_cache[slot/B][h][slot%B][:] = k[t][h][:]  (and v likewise), for
  * every head h.  A pure copy: the stored bits equal the input bits.
  *
@@ -108,11 +108,12 @@ size_t pa_paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head
 /*
  * pa_paged_attn_decode — decode-phase attention through block tables.
  *
- * Definition: "KV cache", section "How it works": the query of the new
- * position is compared against the stored keys (the new key included) and the
- * attention weights mix the stored values; "The KV Cache and PagedAttention",
- * section "The Block Table": attention follows the block table and fetches
- * each block's keys and values.  For text s with L = context_lens[s] tokens
+ * Definition: "KV cache", section "How it works": the new token's query is
+ * scored against every key in the cache, its own among them, and the
+ * resulting weights blend the cached values; "The KV Cache and
+ * PagedAttention", section "The Block Table": the kernel looks up each
+ * logical block's physical block in the table and reads its keys and values
+ * from there.  For text s with L = context_lens[s] tokens
  * and every head h:
  *     z_t = scale * sum_d q[s][h][d] * K_t[d],   t < L,
  *     out[s][h][:] = sum_t softmax(z)_t * V_t[:],
@@ -156,7 +157,7 @@ int pa_paged_attn_decode(void* out, const void* q, const void* k_cache, const vo
  * merge): the cache write of pa_kv_cache_write for one new token per text,
  * then the attention of pa_paged_attn_decode.  A B200 fusion of the pages'
  * two steps ("KV cache", section "How it works": the new token's key and
- * value are written into the cache and take part in its own attention).
+ * value join the cache and take part in its own attention).
  *
  *   k, v           [num_seqs][num_heads][head_dim] dt: each text's new token
  *   slot_mapping   [num_seqs] int64: its slot (negative: not stored)
@@ -255,8 +256,8 @@ size_t pa_paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int 
  * pa_paged_attn_decode_gqa — pa_paged_attn_decode for a pool holding fewer
  * key/value heads than there are query heads (grouped-query attention; one
  * key/value head is multi-query attention): "The KV Cache and
- * PagedAttention", section "What Came After" (several query heads share one
- * set of stored keys and values, shrinking the cache).  With
+ * PagedAttention", section "What Came After" (groups of query heads use
+ * common stored keys and values, so the cache is smaller).  With
  * G = num_heads / num_kv_heads, query head h reads key/value head h / G:
  *     z_t = scale * sum_d q[s][h][d] * K_t[h / G][d],
  *     out[s][h][:] = sum_t softmax(z)_t * V_t[h / G][:].
@@ -365,10 +366,10 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
 /*
  * pa_copy_blocks — copy whole blocks from one pool to another, or within one
  * pool: the device side of copy-on-write ("The KV Cache and
- * PagedAttention", section "Shared, Copied on Write": before a text writes
- * into a block it shares, the block is copied to a free one, the text writes
- * into the copy and the original's count drops by one; pa_bm_append_slot
- * returns the pair) and of moving blocks out of the pool and back (section
+ * PagedAttention", section "Shared, Copied on Write": a text that must
+ * change a block it shares first has that block duplicated into a free one,
+ * then changes the duplicate, and the original's count falls by one;
+ * pa_bm_append_slot returns the pair) and of moving blocks out of the pool and back (section
  * "When Memory Runs Out": blocks set aside in CPU memory).
  *
  *   src_k, src_v   [src_num_blocks][num_heads][block_size][head_dim] dt
@@ -488,8 +489,8 @@ int pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int num_tokens);
 int pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child);
 
 /* Room for the text's next token.  A fresh block is taken only when the last
- * block is full ("a new block only when the earlier ones are full").  If the
- * last block is partial and shared, it is copied first: *cow_src/*cow_dst
+ * block is full (blocks are allocated one at a time, as earlier ones fill).  If the
+ * last block is partial and shared, it is copied first: *cow_src and *cow_dst
  * receive the pair (the caller copies the block's rows on the device before
  * writing), the original's count drops by one; otherwise both are -1.
  * *slot receives the token's slot.  All or nothing. */

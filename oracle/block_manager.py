@@ -6,16 +6,16 @@ in ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may use it.
 Rules, from "The KV Cache and PagedAttention":
   * a text's cache is cut into equal blocks; its logical blocks map to
     physical blocks anywhere in the pool (§Like Pages of Memory);
-  * the block table holds, per logical block, the physical block and how many
-    places are filled; a new physical block is handed out only when all the
-    text's earlier blocks are full (§The Block Table);
-  * when a text is done its blocks go back to the pool (§The Block Table);
+  * the block table records, per logical block, its physical block and its
+    filled places; a text receives a further block only once its current
+    blocks are full (§The Block Table);
+  * a finished text returns its blocks to the pool (§The Block Table);
   * parallel samples of one prompt point at the same physical blocks, each
-    block counting the texts that use it; a text about to write into a shared
-    block first gets a copy, writes there, and the original's count drops by
-    one (§Shared, Copied on Write);
-  * a text holds all its blocks or none (§When Memory Runs Out): an operation
-    that cannot get every block it needs changes nothing.
+    block counting the texts that use it; a text that must change a shared
+    block copies it, changes the copy, and the original's count falls by one
+    (§Shared, Copied on Write);
+  * a text either has every block it needs or none (§When Memory Runs Out):
+    an operation that cannot get every block it needs changes nothing.
 
 Free-list policy (the pages leave it open): blocks are taken from the front of
 the free list and returned to its back; the initial order is given.  The

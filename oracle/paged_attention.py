@@ -7,13 +7,13 @@ It shares no code with the CUDA path and imports nothing from the package.
 What it computes is the plain definition.  Paging changes where the keys and
 values live, not what attention computes ("The KV Cache and PagedAttention",
 §Like Pages of Memory: logical blocks are contiguous to the text, physical
-blocks sit anywhere; §The Block Table: attention follows the block table and
-fetches each block's keys and values).  So the oracle
+blocks sit anywhere; §The Block Table: the kernel finds each logical block's
+physical block in the table and reads it there).  So the oracle
 
   1. writes the new token's key and value into its slot ("KV cache", §How it
-     works: the new position's key and value are written into the cache;
-     "The KV Cache and PagedAttention", §One Token at a Time: only the new
-     token's key and value are computed, the earlier ones are kept);
+     works: each generated token's key and value join the cache; "The KV
+     Cache and PagedAttention", §One Token at a Time: a step computes keys
+     and values for the new token alone and keeps the older ones);
   2. gathers each text's tokens through its block table into one contiguous
      fp64 buffer (token t sits in logical block t // B at place t % B);
   3. runs textbook attention for the one new query: weights
@@ -44,8 +44,8 @@ joined table.
 
 Block copies (``copy_blocks``): whole blocks copied from a source pool to a
 destination pool ("The KV Cache and PagedAttention", §Shared, Copied on
-Write: a text about to write into a block it shares gets its own copy of the
-block first; §When Memory Runs Out: blocks are moved out of the pool to CPU
+Write: a text that must change a block it shares first receives a duplicate
+of it; §When Memory Runs Out: blocks are moved out of the pool to CPU
 memory and back).
 
 Pinned by tests/test_oracle.py against: torch's fp64 attention on unpaged
@@ -142,7 +142,7 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> np.ndar
 
 def kv_head_of(num_heads: int, num_kv_heads: int) -> np.ndarray:
     """Query head h reads key/value head h // (num_heads / num_kv_heads):
-    consecutive query heads share one set of keys and values ("The KV Cache
+    consecutive query heads use common keys and values ("The KV Cache
     and PagedAttention", §What Came After; num_kv_heads == num_heads is plain
     multi-head attention, num_kv_heads == 1 one set for all heads)."""
     if num_kv_heads <= 0 or num_heads % num_kv_heads:

@@ -1,10 +1,10 @@
 """Byte accounting for the KV cache.
 
-"The KV Cache and PagedAttention", section "800 KB a Token": each token keeps a
-key and a value in every layer, so one token costs
+"The KV Cache and PagedAttention", section "800 KB a Token": a token leaves
+two vectors (its key and its value) behind in each layer, so one token costs
 2 x hidden x layers x bytes-per-number (OPT-13B: 2 x 5,120 x 40 x 2 = 819,200
-bytes).  Section "What Came After": when several heads share one set of keys
-and values, only the shared sets count (hidden = kv_heads x head_dim).
+bytes).  Section "What Came After": when groups of heads use common keys and
+values, only those common sets count (hidden = kv_heads x head_dim).
 """
 from __future__ import annotations
 

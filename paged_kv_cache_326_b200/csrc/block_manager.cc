@@ -1,13 +1,14 @@
 // Host block manager: free list, per-block reference counts, copy-on-write.
 //
 // "The KV Cache and PagedAttention": a text's logical blocks map to physical
-// blocks anywhere in the pool (section "Like Pages of Memory"); a new block is
-// handed out only when all the text's earlier blocks are full and a finished
-// text's blocks go back to the pool (section "The Block Table"); samples of one
-// prompt share its blocks, each block counting its users, and a text about to
-// write into a shared block first gets a copy (section "Shared, Copied on
-// Write"); a text holds all its blocks or none (section "When Memory Runs
-// Out"), so every operation here either succeeds completely or changes nothing.
+// blocks anywhere in the pool (section "Like Pages of Memory"); a text gets
+// its next block once its current ones are full, and returns them all when it
+// finishes (section "The Block Table"); samples of one prompt share its
+// blocks, each block counting its users, and a text that needs to change a
+// shared block copies it first (section "Shared, Copied on Write"); a text
+// either has every block it needs or none of them (section "When Memory Runs
+// Out"), so every operation here either succeeds completely or changes
+// nothing.
 #include <cstdint>
 #include <deque>
 #include <new>

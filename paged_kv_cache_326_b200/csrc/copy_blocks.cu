@@ -1,7 +1,7 @@
 // copy_blocks: whole-block copies between two pools (or within one): the
 // device side of copy-on-write ("The KV Cache and PagedAttention", section
-// "Shared, Copied on Write": a text about to write into a block it shares
-// first gets its own copy) and of moving blocks out of a pool and back
+// "Shared, Copied on Write": a text that must change a block it shares
+// first receives a duplicate of it) and of moving blocks out of a pool and back
 // (section "When Memory Runs Out").
 //
 // A block of one pool tensor is one contiguous run of H * B * D elements, so

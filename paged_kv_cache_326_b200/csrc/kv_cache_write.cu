@@ -1,8 +1,8 @@
 // kv_cache_write: scatter each new token's key and value into its slot.
 //
-// "KV cache", section "How it works": the new position's key and value are
-// written into the cache; "The KV Cache and PagedAttention", section "One Token
-// at a Time": only the new token's key and value are computed each iteration.
+// "KV cache", section "How it works": each generated token's key and value
+// join the cache; "The KV Cache and PagedAttention", section "One Token at a
+// Time": a step computes keys and values for the new token alone.
 //
 // One thread moves one 16-byte vector of K and the matching one of V.  A
 // token's H*D elements are contiguous in the input and land in H tiles of the

@@ -11,8 +11,8 @@ PagedAttention" (§800 KB a Token: 40 layers, 5,120 = 40 heads x 128 numbers,
 2-byte floats, texts up to 2,048 tokens) and its default block of 16 tokens
 (§Like Pages of Memory).  Every value is N(0, 1) cast to the storage dtype.
 
-Layout of the pool (chosen here; the pages only say a block holds the keys and
-values of a fixed number of tokens): ``k_cache`` and ``v_cache`` are each
+Layout of the pool (chosen here; the pages only say that every block stores
+keys and values for the same count of tokens): ``k_cache`` and ``v_cache`` are each
 ``[num_blocks][num_heads][block_size][head_dim]``.
 
 Decode-step convention: ``context_lens[s]`` counts the token written in this

@@ -37,8 +37,8 @@ def run_golden_two_answers(make):
 
 def check_invariants(bm, live, num_blocks, block_size, max_blocks):
     """Free + distinct live blocks = pool; counts equal the number of tables
-    holding the block; every text wastes less than one block (a new block
-    only when the earlier ones are full)."""
+    holding the block; every text wastes less than one block (it receives a
+    further block only once its current ones are full)."""
     if not live:
         assert bm.num_free() == num_blocks
         return

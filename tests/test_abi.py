@@ -76,3 +76,13 @@ def test_invalid_arguments_are_rejected_before_launch(built_lib):
     assert lib.pa_paged_attn_decode(None, None, None, None, None, None, 1.0, 4, 8, 100, 4, 8, 64,
                                     0, None, 0, None, None) == P.binding.PA_ERR_INVALID
     assert lib.pa_set_option(99, 0) == P.binding.PA_ERR_INVALID
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/pagedattn.h compiles as strict C99 with every warning an error."""
+    src = tmp_path / "use.c"
+    src.write_text('#include "pagedattn.h"\nint main(void) { return PA_OK; }\n')
+    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                          f"-I{os.path.join(ROOT, 'include')}", "-c", str(src), "-o",
+                          str(tmp_path / "use.o")], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr

@@ -24,7 +24,7 @@ def test_copy_pin(pin):
 
 def test_step_writes_before_attending():
     """The token written in this step is one of the keys the query attends to
-    ("KV cache", How it works: the stored keys plus the new key)."""
+    ("KV cache", How it works: the cached keys and the new token's own)."""
     H, D, B = 2, 8, 4
     q, K, V = P.random_texts([7], H, D, 111)
     kc, vc, tables = P.scatter_to_pool([K[0][:6]], [V[0][:6]], B, 4, 111)
