@@ -514,6 +514,32 @@ int64_t pa_bm_num_tokens(const pa_bm* bm, int64_t seq_id);
 int pa_bm_export(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* block_tables,
                  int max_blocks_per_seq, int32_t* context_lens);
 
+/* Prefix reuse ("The KV Cache and PagedAttention", section "What Came After":
+ * each full block is identified by a hash of its tokens chained with the
+ * hash of all tokens before it; a text that begins like an earlier one takes
+ * over the earlier text's blocks).
+ *
+ * pa_bm_add_seq_tokens adds a text from its prompt's token ids (host array of
+ * num_tokens int32).  It walks the prompt's full blocks in order and takes
+ * over cached blocks with the same chained hash up to the first miss (each
+ * count rises by one; a cached block waiting in the free list leaves it).
+ * The rest are fresh blocks from the front of the free list, as in
+ * pa_bm_add_seq.  The new full blocks are then cached; a partial last block
+ * never is.  *num_cached_tokens (nullable) receives the number of leading
+ * tokens whose blocks were taken over (a multiple of block_size): their keys
+ * and values are already in the pool.  The caller stores the rest (a
+ * negative slot skips the first tokens in pa_kv_cache_write and pa_prefill).
+ *
+ * A cached block whose count falls to zero stays cached while it waits in
+ * the free list.  When the free list hands it out again it is evicted: its
+ * hash is dropped.  Blocks added by pa_bm_add_seq or filled by appends are
+ * not cached.  The chained hash is a 64-bit SplitMix64-style mix: two
+ * different prefixes with equal hashes would share blocks.  All or nothing.
+ * pa_bm_num_cached_blocks counts the hashes currently held. */
+int pa_bm_add_seq_tokens(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                         int* num_cached_tokens);
+int64_t pa_bm_num_cached_blocks(const pa_bm* bm);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,13 +22,41 @@ the free list and returned to its back; the initial order is given.  The
 "places filled" field is kept as the text's token count (filled places of
 block j = min(B, n - j*B)).
 
+Prefix reuse ("The KV Cache and PagedAttention", §What Came After): a full
+block is identified by a hash of its tokens chained with the hash of all
+tokens before it; a text that begins like an earlier one takes over the
+earlier text's blocks.  ``add_seq_tokens`` takes over cached blocks up to the
+first miss and caches the prompt's new full blocks; a cached block with count
+zero keeps its hash while it waits in the free list, a hit takes it back out,
+and handing it out again from the free list drops the hash.  The chained hash
+is SplitMix64's output mix applied token by token (defined below).
+
 Pinned by tests/golden/cow_two_answers.json (the pages' two-answer example)
-and by invariants checked in tests/test_block_manager.py.
+and by invariants checked in tests/test_block_manager.py; prefix reuse by the
+hand-worked sessions in tests/test_prefix_reuse.py.
 """
 from __future__ import annotations
 
 from collections import deque
 from typing import Dict, List, Optional, Sequence, Tuple
+
+_M64 = (1 << 64) - 1
+
+
+def _mix64(z: int) -> int:
+    """SplitMix64's output mix (Steele, Lea, Flood, OOPSLA 2014)."""
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def block_hash(prev: int, tokens: Sequence[int]) -> int:
+    """Hash of one full block: the hash of everything before it (0 for the
+    first block), then each token id taken as an unsigned 32-bit number."""
+    h = prev
+    for t in tokens:
+        h = _mix64(h ^ (((int(t) & 0xFFFFFFFF) + 0x9E3779B97F4A7C15) & _M64))
+    return h
 
 
 class BlockManagerError(Exception):
@@ -51,10 +79,15 @@ class BlockManagerModel:
         self.ref: List[int] = [0] * num_blocks
         self.tables: Dict[int, List[int]] = {}
         self.tokens: Dict[int, int] = {}
+        self.cache: Dict[int, int] = {}        # chained hash -> block
+        self.cached: Dict[int, int] = {}       # block -> its hash
 
     # -- helpers -----------------------------------------------------------
     def _take(self) -> int:
         b = self.free.popleft()
+        h = self.cached.pop(b, None)
+        if h is not None and self.cache.get(h) == b:
+            del self.cache[h]
         self.ref[b] = 1
         return b
 
@@ -74,6 +107,46 @@ class BlockManagerModel:
         self._need(n_blocks)
         self.tables[seq_id] = [self._take() for _ in range(n_blocks)]
         self.tokens[seq_id] = num_tokens
+
+    def add_seq_tokens(self, seq_id: int, tokens: Sequence[int]) -> int:
+        """A new text from its prompt's token ids.  Its leading full blocks
+        whose chained hashes are cached (up to the first miss) are taken over;
+        the rest are fresh.  Returns the number of tokens taken over."""
+        if seq_id in self.tables:
+            raise BlockManagerError("exists", str(seq_id))
+        B = self.block_size
+        n = len(tokens)
+        full = n // B
+        hashes, hits, prev, run = [], [], 0, True
+        for j in range(full):
+            prev = block_hash(prev, tokens[j * B:(j + 1) * B])
+            hashes.append(prev)
+            if run and prev in self.cache:
+                hits.append(self.cache[prev])
+            else:
+                run = False
+        n_blocks = -(-n // B)
+        waiting = sum(1 for b in hits if self.ref[b] == 0)
+        if len(self.free) - waiting < n_blocks - len(hits):
+            raise BlockManagerError("out_of_blocks", f"need {n_blocks - len(hits)}")
+        table = []
+        for b in hits:
+            if self.ref[b] == 0:
+                self.free.remove(b)
+            self.ref[b] += 1
+            table.append(b)
+        for j in range(len(hits), n_blocks):
+            b = self._take()
+            table.append(b)
+            if j < full and hashes[j] not in self.cache:
+                self.cache[hashes[j]] = b
+                self.cached[b] = hashes[j]
+        self.tables[seq_id] = table
+        self.tokens[seq_id] = n
+        return len(hits) * B
+
+    def num_cached_blocks(self) -> int:
+        return len(self.cache)
 
     def fork(self, parent: int, child: int) -> None:
         """The child shares every block of the parent; each count goes up by one."""

@@ -101,6 +101,8 @@ _SIGNATURES = {
     "pa_bm_refcount": (_i32, [_vp, ctypes.c_int32]),
     "pa_bm_num_tokens": (_i64, [_vp, _i64]),
     "pa_bm_export": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp]),
+    "pa_bm_add_seq_tokens": (_i32, [_vp, _i64, _vp, _i32, ctypes.POINTER(ctypes.c_int)]),
+    "pa_bm_num_cached_blocks": (_i64, [_vp]),
 }
 
 
@@ -578,6 +580,20 @@ class BlockManager:
 
     def add_seq(self, seq_id: int, num_tokens: int) -> None:
         _check(lib().pa_bm_add_seq(self._h, int(seq_id), int(num_tokens)), "pa_bm_add_seq")
+
+    def add_seq_tokens(self, seq_id: int, tokens: Sequence[int]) -> int:
+        """A new text from its prompt's token ids, taking over cached blocks
+        of an earlier text that began the same way.  Returns the number of
+        leading tokens whose blocks were taken over."""
+        t = torch.tensor(list(tokens), dtype=torch.int32)
+        cached = ctypes.c_int(0)
+        _check(lib().pa_bm_add_seq_tokens(self._h, int(seq_id), t.data_ptr() if t.numel() else None,
+                                          int(t.numel()), ctypes.byref(cached)),
+               "pa_bm_add_seq_tokens")
+        return cached.value
+
+    def num_cached_blocks(self) -> int:
+        return int(lib().pa_bm_num_cached_blocks(self._h))
 
     def fork(self, parent: int, child: int) -> None:
         _check(lib().pa_bm_fork(self._h, int(parent), int(child)), "pa_bm_fork")

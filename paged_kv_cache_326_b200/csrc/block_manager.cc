@@ -9,6 +9,16 @@
 // either has every block it needs or none of them (section "When Memory Runs
 // Out"), so every operation here either succeeds completely or changes
 // nothing.
+//
+// Prefix reuse ("The KV Cache and PagedAttention", section "What Came After":
+// every full block is identified by a hash of its own tokens chained with
+// the hash of everything before it, and a new text that begins like an
+// earlier one takes over the earlier text's blocks).  pa_bm_add_seq_tokens
+// walks the prompt's full blocks in order and reuses cached blocks up to
+// the first miss.  A cached block whose count falls to zero stays cached
+// while it waits in the free list; a hit takes it back out; the allocator
+// evicts it (drops its hash) when it hands the block out again.  Only
+// prompt blocks registered by pa_bm_add_seq_tokens are cached.
 #include <cstdint>
 #include <deque>
 #include <new>
@@ -20,8 +30,19 @@
 struct pa_bm {
   int64_t num_blocks;
   int block_size;
-  std::deque<int32_t> free_list;                 // take front, return back
+  // Free list: take from the front, return to the back.  A cached block can
+  // leave it from the middle (a prefix hit), so entries carry the stamp the
+  // block got when it was returned; an entry whose block has since left, or
+  // was returned again later, is stale and skipped.
+  std::deque<std::pair<int32_t, uint32_t>> free_list;
+  std::vector<uint8_t> in_free;
+  std::vector<uint32_t> free_stamp;
+  int64_t free_count = 0;
   std::vector<int32_t> ref;                      // texts using each block
+  // prefix cache: chained hash -> block, and each cached block's hash
+  std::unordered_map<uint64_t, int32_t> cache;
+  std::vector<uint8_t> cached;
+  std::vector<uint64_t> cached_hash;
   struct Seq {
     std::vector<int32_t> blocks;
     int64_t tokens;
@@ -41,11 +62,54 @@ uint64_t splitmix64(uint64_t& x) {
   return z ^ (z >> 31);
 }
 
+void drop_stale(pa_bm* bm) {
+  while (!bm->free_list.empty()) {
+    const auto& f = bm->free_list.front();
+    if (bm->in_free[f.first] && bm->free_stamp[f.first] == f.second) return;
+    bm->free_list.pop_front();
+  }
+}
+
+void give_back(pa_bm* bm, int32_t b) {
+  bm->in_free[b] = 1;
+  bm->free_stamp[b] += 1;
+  bm->free_list.emplace_back(b, bm->free_stamp[b]);
+  bm->free_count += 1;
+}
+
+void uncache(pa_bm* bm, int32_t b) {
+  if (!bm->cached[b]) return;
+  auto it = bm->cache.find(bm->cached_hash[b]);
+  if (it != bm->cache.end() && it->second == b) bm->cache.erase(it);
+  bm->cached[b] = 0;
+}
+
+// The front of the free list; a block handed out again leaves the cache.
 int32_t take(pa_bm* bm) {
-  int32_t b = bm->free_list.front();
+  drop_stale(bm);
+  const int32_t b = bm->free_list.front().first;
   bm->free_list.pop_front();
+  bm->in_free[b] = 0;
+  bm->free_count -= 1;
+  uncache(bm, b);
   bm->ref[b] = 1;
   return b;
+}
+
+// SplitMix64's output mix (the same paper) as the step of the chained hash.
+uint64_t mix64(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Hash of one full block: the hash of everything before it, then its tokens.
+uint64_t block_hash(uint64_t prev, const int32_t* tokens, int n) {
+  uint64_t h = prev;
+  for (int i = 0; i < n; ++i)
+    h = mix64(h ^ (static_cast<uint64_t>(static_cast<uint32_t>(tokens[i])) +
+                   0x9E3779B97F4A7C15ull));
+  return h;
 }
 
 }  // namespace
@@ -67,8 +131,12 @@ pa_bm* pa_bm_create(int64_t num_blocks, int block_size, uint64_t shuffle_seed) {
       std::swap(order[i], order[j]);
     }
   }
-  bm->free_list.assign(order.begin(), order.end());
+  bm->in_free.assign(static_cast<size_t>(num_blocks), 0);
+  bm->free_stamp.assign(static_cast<size_t>(num_blocks), 0);
+  for (int32_t b : order) give_back(bm, b);
   bm->ref.assign(static_cast<size_t>(num_blocks), 0);
+  bm->cached.assign(static_cast<size_t>(num_blocks), 0);
+  bm->cached_hash.assign(static_cast<size_t>(num_blocks), 0);
   return bm;
 }
 
@@ -78,7 +146,7 @@ int pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int num_tokens) {
   if (!bm || num_tokens < 0) return PA_ERR_INVALID;
   if (bm->seqs.count(seq_id)) return PA_ERR_EXISTS;
   int64_t need = (static_cast<int64_t>(num_tokens) + bm->block_size - 1) / bm->block_size;
-  if (static_cast<int64_t>(bm->free_list.size()) < need) return PA_ERR_OUT_OF_BLOCKS;
+  if (bm->free_count < need) return PA_ERR_OUT_OF_BLOCKS;
   pa_bm::Seq s;
   s.tokens = num_tokens;
   s.blocks.reserve(static_cast<size_t>(need));
@@ -107,12 +175,12 @@ int pa_bm_append_slot(pa_bm* bm, int64_t seq_id, int64_t* slot, int32_t* cow_src
   const int64_t place = s.tokens % bm->block_size;
   int32_t src = -1, dst = -1;
   if (place == 0) {
-    if (bm->free_list.empty()) return PA_ERR_OUT_OF_BLOCKS;
+    if (bm->free_count == 0) return PA_ERR_OUT_OF_BLOCKS;
     s.blocks.push_back(take(bm));
   } else {
     int32_t last = s.blocks.back();
     if (bm->ref[last] > 1) {
-      if (bm->free_list.empty()) return PA_ERR_OUT_OF_BLOCKS;
+      if (bm->free_count == 0) return PA_ERR_OUT_OF_BLOCKS;
       dst = take(bm);
       bm->ref[last] -= 1;
       s.blocks.back() = dst;
@@ -133,14 +201,69 @@ int pa_bm_free_seq(pa_bm* bm, int64_t seq_id) {
   for (int32_t b : it->second.blocks)
     if (bm->ref[b] <= 0) return PA_ERR_CORRUPT;
   for (int32_t b : it->second.blocks) {
-    if (--bm->ref[b] == 0) bm->free_list.push_back(b);
+    if (--bm->ref[b] == 0) give_back(bm, b);
   }
   bm->seqs.erase(it);
   return PA_OK;
 }
 
-int64_t pa_bm_num_free(const pa_bm* bm) {
-  return bm ? static_cast<int64_t>(bm->free_list.size()) : PA_ERR_INVALID;
+int64_t pa_bm_num_free(const pa_bm* bm) { return bm ? bm->free_count : PA_ERR_INVALID; }
+
+int64_t pa_bm_num_cached_blocks(const pa_bm* bm) {
+  return bm ? static_cast<int64_t>(bm->cache.size()) : PA_ERR_INVALID;
+}
+
+int pa_bm_add_seq_tokens(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                         int* num_cached_tokens) {
+  if (!bm || num_tokens < 0 || (num_tokens > 0 && !tokens)) return PA_ERR_INVALID;
+  if (bm->seqs.count(seq_id)) return PA_ERR_EXISTS;
+  const int B = bm->block_size;
+  const int64_t full = num_tokens / B;
+  const int64_t need = (static_cast<int64_t>(num_tokens) + B - 1) / B;
+  // the chained hashes of the full blocks, and the cached run at the front
+  std::vector<uint64_t> h(static_cast<size_t>(full));
+  std::vector<int32_t> hit;
+  bool run = true;
+  uint64_t prev = 0;
+  for (int64_t j = 0; j < full; ++j) {
+    prev = block_hash(prev, tokens + j * B, B);
+    h[j] = prev;
+    if (run) {
+      auto it = bm->cache.find(prev);
+      if (it == bm->cache.end()) {
+        run = false;
+      } else {
+        hit.push_back(it->second);
+      }
+    }
+  }
+  int64_t hits_free = 0;
+  for (int32_t b : hit) hits_free += bm->in_free[b] ? 1 : 0;
+  const int64_t fresh = need - static_cast<int64_t>(hit.size());
+  if (bm->free_count - hits_free < fresh) return PA_ERR_OUT_OF_BLOCKS;
+  pa_bm::Seq s;
+  s.tokens = num_tokens;
+  s.blocks.reserve(static_cast<size_t>(need));
+  for (int32_t b : hit) {  // reuse: a waiting block leaves the free list
+    if (bm->in_free[b]) {
+      bm->in_free[b] = 0;
+      bm->free_count -= 1;
+    }
+    bm->ref[b] += 1;
+    s.blocks.push_back(b);
+  }
+  for (int64_t j = static_cast<int64_t>(hit.size()); j < need; ++j) {
+    const int32_t b = take(bm);
+    s.blocks.push_back(b);
+    if (j < full && !bm->cache.count(h[j])) {  // register a new full block
+      bm->cache.emplace(h[j], b);
+      bm->cached[b] = 1;
+      bm->cached_hash[b] = h[j];
+    }
+  }
+  bm->seqs.emplace(seq_id, std::move(s));
+  if (num_cached_tokens) *num_cached_tokens = static_cast<int>(hit.size()) * B;
+  return PA_OK;
 }
 
 int pa_bm_refcount(const pa_bm* bm, int32_t block) {

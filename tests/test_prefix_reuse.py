@@ -1,0 +1,270 @@
+"""Prefix reuse in the block manager ("The KV Cache and PagedAttention",
+section "What Came After": every full block is identified by a hash of its
+tokens chained with the hash of all tokens before it, and a text that begins
+like an earlier one takes over the earlier text's blocks).
+
+The oracle's model is pinned by hand-worked sessions and planted mistakes;
+the C++ manager must match the model exactly on seeded random sessions
+(CPU only)."""
+import random
+
+import pytest
+
+from oracle import BlockManagerError, BlockManagerModel
+
+
+class Cpp:
+    """The C++ manager through the binding, with the model's interface."""
+
+    def __init__(self, n, b):
+        import paged_kv_cache_326_b200 as P
+        self.P = P
+        self.bm = P.BlockManager(n, b)
+        self.block_size = b
+
+    def _run(self, fn, *a):
+        try:
+            return fn(*a)
+        except self.P.PagedAttnError as e:
+            kind = {-3: "out_of_blocks", -4: "no_seq", -5: "exists", -6: "table_full",
+                    -1: "invalid"}.get(e.code, str(e.code))
+            raise BlockManagerError(kind) from None
+
+    def add_seq_tokens(self, s, toks):
+        return self._run(self.bm.add_seq_tokens, s, toks)
+
+    def add_seq(self, s, n):
+        return self._run(self.bm.add_seq, s, n)
+
+    def fork(self, p, c):
+        return self._run(self.bm.fork, p, c)
+
+    def append_slot(self, s):
+        return self._run(self.bm.append_slot, s)
+
+    def free_seq(self, s):
+        return self._run(self.bm.free_seq, s)
+
+    def num_free(self):
+        return self.bm.num_free()
+
+    def num_cached_blocks(self):
+        return self.bm.num_cached_blocks()
+
+    def refcount(self, b):
+        return self.bm.refcount(b)
+
+    def export(self, ids, mb):
+        t, l = self.bm.export(ids, mb)
+        return t.tolist(), l.tolist()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from paged_kv_cache_326_b200 import build
+    build.build()
+
+
+# ---------------------------------------------------------------------------
+# pins of the rules (hand-worked sessions, blocks of 4, free list in order)
+# ---------------------------------------------------------------------------
+
+def pin_same_beginning_takes_over_full_blocks(make):
+    bm = make(16, 4)
+    assert bm.add_seq_tokens(1, list(range(1, 11))) == 0        # blocks 0, 1 full, 2 partial
+    assert bm.num_cached_blocks() == 2
+    assert bm.add_seq_tokens(2, list(range(1, 9)) + [99, 98]) == 8
+    tables, lens = bm.export([1, 2], 4)
+    assert tables == [[0, 1, 2, -1], [0, 1, 3, -1]] and lens == [10, 10]
+    assert [bm.refcount(b) for b in range(4)] == [2, 2, 1, 1]
+    assert bm.num_free() == 12
+
+
+def pin_partial_last_block_is_never_shared(make):
+    bm = make(16, 4)
+    toks = list(range(1, 11))
+    bm.add_seq_tokens(1, toks)
+    assert bm.add_seq_tokens(2, toks) == 8                       # identical prompts
+    tables, _ = bm.export([1, 2], 4)
+    assert tables[0][:2] == tables[1][:2] and tables[0][2] != tables[1][2]
+
+
+def pin_hash_covers_everything_before(make):
+    """Equal second blocks after different first blocks share nothing."""
+    bm = make(16, 4)
+    bm.add_seq_tokens(1, [1, 2, 3, 4, 5, 6, 7, 8])
+    assert bm.add_seq_tokens(2, [0, 2, 3, 4, 5, 6, 7, 8]) == 0
+    tables, _ = bm.export([1, 2], 2)
+    assert set(tables[0]).isdisjoint(tables[1])
+    assert bm.num_cached_blocks() == 4
+
+
+def pin_waiting_blocks_are_taken_back(make):
+    """A finished text's cached blocks wait in the free list; a text that
+    begins the same way takes them back out."""
+    bm = make(8, 4)
+    bm.add_seq_tokens(1, list(range(12)))
+    bm.free_seq(1)
+    assert bm.num_free() == 8 and bm.num_cached_blocks() == 3
+    assert bm.add_seq_tokens(2, list(range(12)) + [5]) == 12
+    tables, _ = bm.export([2], 4)
+    assert tables == [[0, 1, 2, 3]]
+    assert bm.num_free() == 4 and [bm.refcount(b) for b in range(4)] == [1, 1, 1, 1]
+
+
+def pin_handing_out_evicts_and_reuse_stops_at_the_first_miss(make):
+    """Blocks 0, 1 (cached, waiting) sit at the back of the free list after
+    blocks 2..5; taking five fresh blocks hands out block 0 again, which
+    drops its hash.  The same prompt then misses at its first block and takes
+    over nothing, although its second block's hash is still cached."""
+    bm = make(6, 4)
+    bm.add_seq_tokens(1, list(range(8)))                          # blocks 0, 1
+    bm.free_seq(1)                                                # free list: 2 3 4 5 0 1
+    bm.add_seq(2, 20)                                             # takes 2 3 4 5 0
+    assert bm.num_cached_blocks() == 1                            # block 1 keeps its hash
+    bm.free_seq(2)                                                # free list: 1 2 3 4 5 0
+    assert bm.add_seq_tokens(3, list(range(8))) == 0
+    tables, _ = bm.export([3], 2)
+    # fresh blocks from the front: block 1 is handed out (its old hash goes),
+    # and both new full blocks are cached under the prompt's hashes
+    assert tables == [[1, 2]]
+    assert [bm.refcount(b) for b in range(3)] == [0, 1, 1]
+    assert bm.num_cached_blocks() == 2
+    assert bm.add_seq_tokens(4, list(range(8))) == 8              # now a full takeover
+
+
+def pin_out_of_blocks_changes_nothing(make):
+    bm = make(4, 4)
+    bm.add_seq_tokens(1, list(range(8)))
+    before = (bm.export([1], 2), bm.num_free(), bm.num_cached_blocks())
+    with pytest.raises(BlockManagerError) as e:
+        bm.add_seq_tokens(2, list(range(8)) + list(range(100, 112)))   # 2 reused + 3 fresh > 2
+    assert e.value.kind == "out_of_blocks"
+    assert (bm.export([1], 2), bm.num_free(), bm.num_cached_blocks()) == before
+    assert bm.add_seq_tokens(2, list(range(8)) + [1, 2]) == 8            # 1 fresh fits
+
+
+PINS = [pin_same_beginning_takes_over_full_blocks, pin_partial_last_block_is_never_shared,
+        pin_hash_covers_everything_before, pin_waiting_blocks_are_taken_back,
+        pin_handing_out_evicts_and_reuse_stops_at_the_first_miss,
+        pin_out_of_blocks_changes_nothing]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
+def test_model_pin(pin):
+    pin(BlockManagerModel)
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
+def test_cpp_pin(pin):
+    pin(Cpp)
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes in copies of the model
+# ---------------------------------------------------------------------------
+
+class NoChain(BlockManagerModel):
+    """Planted mistake: each block hashed on its own tokens only."""
+
+    def add_seq_tokens(self, seq_id, tokens):
+        import oracle.block_manager as M
+        real = M.block_hash
+        M.block_hash = lambda prev, toks: real(0, toks)
+        try:
+            return super().add_seq_tokens(seq_id, tokens)
+        finally:
+            M.block_hash = real
+
+
+class CachesPartial(BlockManagerModel):
+    """Planted mistake: the partial last block is cached and shared too."""
+
+    def add_seq_tokens(self, seq_id, tokens):
+        B = self.block_size
+        pad = (-len(tokens)) % B
+        got = super().add_seq_tokens(seq_id, list(tokens) + [-1] * pad)
+        self.tokens[seq_id] = len(tokens)
+        return min(got, len(tokens))
+
+
+class NoEviction(BlockManagerModel):
+    """Planted mistake: handing a block out again keeps its hash."""
+
+    def _take(self):
+        b = self.free.popleft()
+        self.ref[b] = 1
+        return b
+
+
+@pytest.mark.parametrize("cls", [NoChain, CachesPartial, NoEviction], ids=lambda c: c.__name__)
+def test_planted_prefix_mistake_is_caught(cls):
+    failed = 0
+    for pin in PINS:
+        try:
+            pin(cls)
+        except (AssertionError, BlockManagerError, ValueError, KeyError):
+            failed += 1
+    assert failed, cls.__name__
+
+
+# ---------------------------------------------------------------------------
+# the C++ manager against the model
+# ---------------------------------------------------------------------------
+
+def _session(make, seed):
+    """Random operations over prompts from a few shared beginnings (so blocks
+    are taken over, wait in the free list, are taken back and evicted); every
+    result and the full state after each operation are logged."""
+    rnd = random.Random(seed)
+    B = rnd.choice([2, 4, 8])
+    bm = make(48, B)
+    stems = [[rnd.randrange(50) for _ in range(rnd.randrange(0, 5 * B))] for _ in range(4)]
+    live, next_id, log = [], 0, []
+    for _ in range(300):
+        op = rnd.random()
+        try:
+            if op < 0.35 or not live:
+                toks = list(rnd.choice(stems))[:rnd.randrange(0, 5 * B + 1)]
+                toks += [rnd.randrange(50) for _ in range(rnd.randrange(0, B + 2))]
+                log.append(("tok", bm.add_seq_tokens(next_id, toks)))
+                live.append(next_id)
+                next_id += 1
+            elif op < 0.45:
+                bm.add_seq(next_id, rnd.randrange(0, 3 * B))
+                live.append(next_id)
+                next_id += 1
+                log.append(("add",))
+            elif op < 0.55:
+                p = rnd.choice(live)
+                bm.fork(p, next_id)
+                live.append(next_id)
+                next_id += 1
+                log.append(("fork",))
+            elif op < 0.8:
+                log.append(("app", tuple(bm.append_slot(rnd.choice(live)))))
+            else:
+                s = rnd.choice(live)
+                bm.free_seq(s)
+                live.remove(s)
+                log.append(("free",))
+        except BlockManagerError as e:
+            log.append(("err", e.kind))
+            if e.kind == "out_of_blocks" and live:
+                s = live.pop(0)
+                bm.free_seq(s)
+        tables, lens = bm.export(live, 64) if live else ([], [])
+        log.append((tuple(map(tuple, tables)), tuple(lens), bm.num_free(),
+                    bm.num_cached_blocks(), tuple(bm.refcount(b) for b in range(48))))
+    return log
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_cpp_matches_model_exactly(seed):
+    assert _session(Cpp, seed) == _session(BlockManagerModel, seed)
+
+
+def test_sessions_do_reuse_and_evict():
+    """The sessions exercise what they are meant to: takeovers happen."""
+    log = _session(BlockManagerModel, 3)
+    assert any(e[0] == "tok" and e[1] > 0 for e in log if isinstance(e[0], str))
