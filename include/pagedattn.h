@@ -272,8 +272,8 @@ size_t pa_paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int 
  * equal subsets that each read the rows).  The tensor-core kernel (see
  * PA_OPT_GQA_KERNEL) copies whole 16-token (32 at head_dim 64) runs of a
  * block, so rows past L in a text's last block are read and ignored; they
- * lie inside the pool, and their contents (NaN included) do not affect out.  num_heads must be a multiple of num_kv_heads
- * (else PA_ERR_INVALID).
+ * lie inside the pool, and their contents (NaN included) do not affect out.
+ * num_heads must be a multiple of num_kv_heads (else PA_ERR_INVALID).
  */
 int pa_paged_attn_decode_gqa(void* out, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* block_tables, const int32_t* context_lens,
@@ -369,8 +369,8 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
  * PagedAttention", section "Shared, Copied on Write": a text that must
  * change a block it shares first has that block duplicated into a free one,
  * then changes the duplicate, and the original's count falls by one;
- * pa_bm_append_slot returns the pair) and of moving blocks out of the pool and back (section
- * "When Memory Runs Out": blocks set aside in CPU memory).
+ * pa_bm_append_slot returns the pair) and of moving blocks out of the pool
+ * and back (section "When Memory Runs Out": blocks set aside in CPU memory).
  *
  *   src_k, src_v   [src_num_blocks][num_heads][block_size][head_dim] dt
  *                  (PA_F16, PA_BF16, or PA_E4M3 for 8-bit pools)
