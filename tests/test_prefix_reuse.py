@@ -268,3 +268,47 @@ def test_sessions_do_reuse_and_evict():
     """The sessions exercise what they are meant to: takeovers happen."""
     log = _session(BlockManagerModel, 3)
     assert any(e[0] == "tok" and e[1] > 0 for e in log if isinstance(e[0], str))
+
+
+def test_taken_over_blocks_attend_like_private_ones():
+    """Two prompts begin with the same 8 tokens (blocks of 4).  The second
+    text takes over the first's two full blocks and stores only its own
+    remaining tokens (negative slots for the taken-over ones).  Its decode
+    through the oracle then equals torch's fp64 attention on its contiguous
+    keys and values, i.e. the shared blocks hold exactly its prefix."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from tests.oracle_pins import f64, sdpa_contiguous
+
+    B, H, D, N = 4, 2, 8, 16
+    bm = Cpp(N, B)
+    g = torch.Generator().manual_seed(7)
+    prefix = [5, 6, 7, 8, 9, 10, 11, 12]
+    prompts = [prefix + [1, 2], prefix + [3, 4, 13, 14, 15]]
+    # a token's key and value depend only on the token and its position here,
+    # as in a model whose prefix is the same
+    table_k = torch.randn(64, 32, H, D, generator=g).half()   # [token id][position]
+    table_v = torch.randn(64, 32, H, D, generator=g).half()
+    kc = torch.full((N, H, B, D), float("nan"), dtype=torch.float16)
+    vc = torch.full((N, H, B, D), float("nan"), dtype=torch.float16)
+    reused = []
+    for sid, toks in enumerate(prompts):
+        cached = bm.add_seq_tokens(sid, toks)
+        reused.append(cached)
+        tables, _ = bm.export([sid], 8)
+        ks = torch.stack([table_k[t, p] for p, t in enumerate(toks)])
+        vs = torch.stack([table_v[t, p] for p, t in enumerate(toks)])
+        slots = np.array([tables[0][p // B] * B + p % B if p >= cached else -1
+                          for p in range(len(toks))])
+        kc_new, vc_new = oracle.cache_write(f64(kc), f64(vc), f64(ks), f64(vs), slots, B)
+        kc, vc = torch.from_numpy(kc_new).half(), torch.from_numpy(vc_new).half()
+    assert reused == [0, 8]
+    tables, lens = bm.export([0, 1], 8)
+    q = torch.randn(2, H, D, generator=g).half()
+    got = oracle.paged_decode(f64(q), f64(kc), f64(vc), np.array(tables), lens, 0.3, B)
+    K = [torch.stack([table_k[t, p] for p, t in enumerate(toks)]) for toks in prompts]
+    V = [torch.stack([table_v[t, p] for p, t in enumerate(toks)]) for toks in prompts]
+    ref = sdpa_contiguous(q, K, V, 0.3)
+    assert np.abs(got - ref).max() <= 1e-12
