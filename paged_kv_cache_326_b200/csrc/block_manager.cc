@@ -70,6 +70,16 @@ void drop_stale(pa_bm* bm) {
   }
 }
 
+// Drop every stale entry, keeping the order of the live ones, once they
+// outnumber the live ones (prefix hits leave one behind each).
+void compact(pa_bm* bm) {
+  if (static_cast<int64_t>(bm->free_list.size()) <= 2 * bm->free_count + 64) return;
+  std::deque<std::pair<int32_t, uint32_t>> live;
+  for (const auto& f : bm->free_list)
+    if (bm->in_free[f.first] && bm->free_stamp[f.first] == f.second) live.push_back(f);
+  bm->free_list.swap(live);
+}
+
 void give_back(pa_bm* bm, int32_t b) {
   bm->in_free[b] = 1;
   bm->free_stamp[b] += 1;
@@ -252,6 +262,7 @@ int pa_bm_add_seq_tokens(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int n
     bm->ref[b] += 1;
     s.blocks.push_back(b);
   }
+  compact(bm);
   for (int64_t j = static_cast<int64_t>(hit.size()); j < need; ++j) {
     const int32_t b = take(bm);
     s.blocks.push_back(b);

@@ -312,3 +312,20 @@ def test_taken_over_blocks_attend_like_private_ones():
     V = [torch.stack([table_v[t, p] for p, t in enumerate(toks)]) for toks in prompts]
     ref = sdpa_contiguous(q, K, V, 0.3)
     assert np.abs(got - ref).max() <= 1e-12
+
+
+def test_many_takebacks_keep_the_free_list_order():
+    """Thousands of take-backs of waiting blocks (each leaves a stale entry
+    behind in the C++ free list, compacted from time to time) give the same
+    tables as the model."""
+    def run(make):
+        bm = make(64, 4)
+        out = []
+        for i in range(3000):
+            toks = list(range(i % 5, i % 5 + 8)) + [i % 3]
+            out.append(bm.add_seq_tokens(i, toks))
+            out.append(tuple(bm.export([i], 4)[0][0]))
+            bm.free_seq(i)
+            out.append((bm.num_free(), bm.num_cached_blocks()))
+        return out
+    assert run(Cpp) == run(BlockManagerModel)
