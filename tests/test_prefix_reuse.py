@@ -329,3 +329,37 @@ def test_many_takebacks_keep_the_free_list_order():
             out.append((bm.num_free(), bm.num_cached_blocks()))
         return out
     assert run(Cpp) == run(BlockManagerModel)
+
+
+def test_reuse_across_requests_feeds_the_shared_prefix_split():
+    """Four requests that begin with the same 12-token system prompt (blocks
+    of 4) take over its three blocks; the host splitter then finds those
+    blocks as the group's prefix, and the oracle's shared-prefix form over
+    the split equals its plain decode over the tables bit for bit."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import paged_kv_cache_326_b200 as P
+
+    B, H, D, N = 4, 2, 8, 32
+    bm = Cpp(N, B)
+    system = list(range(100, 112))
+    asks = [[1, 2], [3, 4, 5, 6, 7], [8], [9, 10, 11, 12]]
+    got = [bm.add_seq_tokens(i, system + a) for i, a in enumerate(asks)]
+    assert got == [0, 12, 12, 12]
+    tables, lens = bm.export(list(range(4)), 8)
+    pt, pl, tt, tl = P.split_shared_prefix(torch.tensor(tables, dtype=torch.int32),
+                                           torch.tensor(lens, dtype=torch.int32), B, 4)
+    assert pl.tolist() == [12] and pt.tolist()[0][:3] == tables[0][:3]
+    assert tl.tolist() == [len(a) for a in asks]
+    g = torch.Generator().manual_seed(3)
+    kc = torch.randn(N, H, B, D, generator=g).double().numpy()
+    vc = torch.randn(N, H, B, D, generator=g).double().numpy()
+    q = torch.randn(4, H, D, generator=g).double().numpy()
+    plain = oracle.paged_decode(q, kc, vc, np.array(tables), lens, 0.3, B)
+    prows = [[b for b in r if b >= 0] for r in pt.tolist()]
+    trows = [[b for b in r if b >= 0] for r in tt.tolist()]
+    shared = oracle.paged_decode_shared(q, kc, vc, prows, pl.tolist(), trows, tl.tolist(), 4,
+                                        0.3, B)
+    assert np.array_equal(plain, shared)
