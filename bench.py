@@ -83,7 +83,7 @@ def hbm_peak():
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: copy, burst)"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, an earlier copy measurement on B200)"
 
 
 def traffic_per_launch(workload: str, path: str):
@@ -261,7 +261,7 @@ def tensor_peak():
                     "measured (MEASURED_PEAKS.json bf16_tflops: cuBLAS dense, burst; fp16 runs "
                     "at the same tensor rate)")
     except Exception:
-        return 1590.0, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+        return 1590.0, "fallback (1.59 PFLOP/s, an earlier cuBLAS bf16 measurement on B200)"
 
 
 def run_prefill_bench(args, ranks, world, rank, local):

@@ -19,7 +19,7 @@ cudaError_t launch_kv_cache_write_fp8(const void* k, const void* v, void* k_cach
 // A tiled TMA map of a 16-bit (fp16 or bf16) tensor of `rank` dimensions
 // (innermost first; strides in bytes of dimensions 1..rank-1), boxes of
 // `box` elements, 128-byte swizzle, zero fill out of bounds.  False if the
-// driver refuses it.
+// CUDA driver's encoder refuses it.
 bool encode_swizzled_map(CUtensorMap* map, const void* base, bool bf16, int rank,
                          const uint64_t* dims, const uint64_t* strides_bytes,
                          const uint32_t* box);
