@@ -86,3 +86,18 @@ def test_header_is_plain_c(tmp_path):
                           f"-I{os.path.join(ROOT, 'include')}", "-c", str(src), "-o",
                           str(tmp_path / "use.o")], capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_plain_c_program_uses_the_host_calls(tmp_path, built_lib):
+    """A C99 program links libpagedattn.so and drives the block manager,
+    prefix reuse and the shared-prefix splitter (no GPU needed)."""
+    exe = tmp_path / "c_abi_host"
+    lib_dir = os.path.dirname(built_lib)
+    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                          f"-I{os.path.join(ROOT, 'include')}",
+                          os.path.join(ROOT, "tests", "c_abi_host.c"), "-o", str(exe),
+                          f"-L{lib_dir}", "-l:libpagedattn.so", f"-Wl,-rpath,{lib_dir}"],
+                         capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stderr
