@@ -8,12 +8,13 @@ path and never imports the product package.
 """
 from .paged_attention import (attend, cache_write, copy_blocks, decode_step, gather_context,
                               kv_head_of, paged_decode, paged_decode_shared, prefill,
-                              split_shared_prefix)
+                              prefill_with_prefix, split_shared_prefix)
 from .block_manager import BlockManagerError, BlockManagerModel
 from .fp8 import (cache_write_fp8, e4m3_decode, e4m3_encode, e4m3_value, paged_decode_fp8,
                   quantize)
 
-__all__ = ["attend", "cache_write", "copy_blocks", "decode_step", "gather_context", "kv_head_of", "paged_decode", "prefill",
+__all__ = ["attend", "cache_write", "copy_blocks", "decode_step", "gather_context", "kv_head_of",
+           "paged_decode", "prefill", "prefill_with_prefix",
            "paged_decode_shared", "split_shared_prefix",
            "BlockManagerError", "BlockManagerModel", "cache_write_fp8", "e4m3_decode",
            "e4m3_encode", "e4m3_value", "paged_decode_fp8", "quantize"]

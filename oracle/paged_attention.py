@@ -279,6 +279,48 @@ def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: Sequence[in
     return out
 
 
+def prefill_with_prefix(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: Sequence[int],
+                        k_cache: np.ndarray, v_cache: np.ndarray, block_tables: np.ndarray,
+                        cached_lens: Sequence[int], scale: float,
+                        block_size: int) -> np.ndarray:
+    """Prompt phase of prompts whose first tokens are already in the paged
+    cache, fp64 ("The KV Cache and PagedAttention", §What Came After: a prompt
+    that begins like an earlier one reuses the earlier one's blocks, which
+    saves the time spent on the prompt).
+
+    Prompt s has ``cached_lens[s]`` tokens in the caches, found through
+    ``block_tables[s]`` as in decode; its other tokens are rows
+    cu_seqlens[s] .. cu_seqlens[s+1]-1 of q ``[T][H][D]`` and k, v
+    ``[T][H_kv][D]``, at positions cached_lens[s] + i.  With K the cached keys
+    followed by k[a:b] (V likewise), row a + i (position P = cached_lens[s] + i)
+    is
+        z_u = scale * q[a+i] . K[u] for u <= P,  out[a+i] = softmax(z) . V[0..P],
+    i.e. the rows of the ordinary prompt phase over the whole prompt that
+    belong to the new tokens."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    T, H, D = q.shape
+    kvh = kv_head_of(H, k.shape[1])
+    out = np.zeros((T, H, D), dtype=np.float64)
+    for s in range(len(cu_seqlens) - 1):
+        a, b = int(cu_seqlens[s]), int(cu_seqlens[s + 1])
+        n = b - a
+        if n == 0:
+            continue
+        c = int(cached_lens[s])
+        K = np.concatenate([gather_context(k_cache, block_tables[s], c, block_size), k[a:b]])
+        V = np.concatenate([gather_context(v_cache, block_tables[s], c, block_size), v[a:b]])
+        allowed = np.arange(c + n)[None, :] <= (c + np.arange(n))[:, None]   # [n][c + n]
+        for h in range(H):
+            z = float(scale) * (q[a:b, h, :] @ K[:, kvh[h], :].T)
+            z = np.where(allowed, z, -np.inf)
+            e = np.exp(z - z.max(axis=1, keepdims=True))
+            w = e / e.sum(axis=1, keepdims=True)
+            out[a:b, h, :] = w @ V[:, kvh[h], :]
+    return out
+
+
 def decode_step(q, k, v, k_cache, v_cache, slot_mapping, block_tables, context_lens,
                 scale, block_size, pairs=None):
     """One decode step of one layer: write the new tokens, then attend.

@@ -574,6 +574,83 @@ PREFILL_PINS = [pin_prefill_vs_torch_causal, pin_prefill_last_row_is_decode,
 
 
 # ---------------------------------------------------------------------------
+# prompt phase over a stored prefix (fn(q, k, v, cu, k_cache, v_cache,
+# tables, cached_lens, scale, block_size) -> out)
+# ---------------------------------------------------------------------------
+
+def _prefixed_prompts(prefix_lens, new_lens, H, Hkv, D, B, seed, num_blocks=64):
+    """Whole prompts drawn as contiguous tensors; each prompt's first
+    prefix_lens[s] tokens' keys and values scattered into a paged pool (the
+    pin's own scatter), the rest packed as the new rows."""
+    g = torch.Generator().manual_seed(seed)
+    whole = [(torch.randn(c + n, H, D, generator=g).to(torch.float16),
+              torch.randn(c + n, Hkv, D, generator=g).to(torch.float16),
+              torch.randn(c + n, Hkv, D, generator=g).to(torch.float16))
+             for c, n in zip(prefix_lens, new_lens)]
+    kc, vc, tables = scatter_to_pool([w[1][:c] for w, c in zip(whole, prefix_lens)],
+                                     [w[2][:c] for w, c in zip(whole, prefix_lens)], B,
+                                     num_blocks, seed)
+    q = torch.cat([w[0][c:] for w, c in zip(whole, prefix_lens)])
+    k = torch.cat([w[1][c:] for w, c in zip(whole, prefix_lens)])
+    v = torch.cat([w[2][c:] for w, c in zip(whole, prefix_lens)])
+    cu = np.concatenate([[0], np.cumsum(new_lens)]).astype(np.int64)
+    return whole, q, k, v, cu, kc, vc, tables
+
+
+def pin_prefix_rows_of_the_whole_prompt(fn):
+    """The new rows equal torch's fp64 causal attention over the whole prompt
+    (prefix and new tokens contiguous, key/value heads repeated), restricted
+    to the new rows; a zero-length prefix is the ordinary prompt phase."""
+    pre, new, H, Hkv, D, B = [8, 0, 24, 4, 16], [5, 9, 1, 12, 0], 4, 2, 8, 4
+    whole, q, k, v, cu, kc, vc, tables = _prefixed_prompts(pre, new, H, Hkv, D, B, 531)
+    got = fn(f64(q), f64(k), f64(v), cu, f64(kc), f64(vc), tables, pre, 0.35, B)
+    for s, (c, n) in enumerate(zip(pre, new)):
+        if n == 0:
+            continue
+        qw, kw, vw = (t.double().permute(1, 0, 2) for t in whole[s])
+        kw = kw.repeat_interleave(H // Hkv, dim=0)
+        vw = vw.repeat_interleave(H // Hkv, dim=0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qw, kw, vw, is_causal=True,
+                                                               scale=0.35)
+        ref = ref.permute(1, 0, 2)[c:].numpy()
+        assert np.abs(got[cu[s]:cu[s + 1]] - ref).max() <= 1e-12, f"prompt {s} vs whole"
+
+
+def pin_prefix_brute_force(fn):
+    """Every new row of a tiny prompt (6 stored tokens in blocks of 2, 3 new)
+    against scalar brute force with math.fsum over the contiguous prompt."""
+    pre, new, D, B = [6], [3], 4, 2
+    whole, q, k, v, cu, kc, vc, tables = _prefixed_prompts(pre, new, 1, 1, D, B, 541)
+    got = fn(f64(q), f64(k), f64(v), cu, f64(kc), f64(vc), tables, pre, 0.5, B)
+    Q, K, V = (f64(t)[:, 0] for t in whole[0])
+    for i in range(3):
+        P = 6 + i
+        z = [0.5 * math.fsum(Q[P, d] * K[u, d] for d in range(D)) for u in range(P + 1)]
+        m = max(z)
+        e = [math.exp(x - m) for x in z]
+        den = math.fsum(e)
+        want = [math.fsum(e[u] * V[u, d] for u in range(P + 1)) / den for d in range(D)]
+        assert np.abs(got[i, 0] - np.array(want)).max() <= 1e-12, f"new row {i}"
+
+
+def pin_prefix_blocks_can_sit_anywhere(fn):
+    """The same stored prefixes under another seeded placement of their
+    blocks in the pool give bit-identical rows."""
+    pre, new, H, D, B = [12, 20], [7, 3], 2, 8, 4
+    _, q, k, v, cu, kc, vc, tables = _prefixed_prompts(pre, new, H, H, D, B, 551)
+    _, q2, k2, v2, cu2, kc2, vc2, tables2 = _prefixed_prompts(pre, new, H, H, D, B, 551,
+                                                              num_blocks=97)
+    assert not np.array_equal(tables, tables2)
+    a = fn(f64(q), f64(k), f64(v), cu, f64(kc), f64(vc), tables, pre, 0.3, B)
+    b = fn(f64(q2), f64(k2), f64(v2), cu2, f64(kc2), f64(vc2), tables2, pre, 0.3, B)
+    assert np.array_equal(a, b), "placement changed the result"
+
+
+PREFIX_PINS = [pin_prefix_rows_of_the_whole_prompt, pin_prefix_brute_force,
+               pin_prefix_blocks_can_sit_anywhere]
+
+
+# ---------------------------------------------------------------------------
 # shared prefixes
 # ---------------------------------------------------------------------------
 

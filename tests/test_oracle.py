@@ -86,27 +86,34 @@ def test_fp8_attention_on_representable_values():
     P.pin_fp8_attention_on_representable_values(oracle.paged_decode_fp8, oracle.quantize)
 
 
-def test_fp8_cache_write_stores_the_codes_at_the_slots():
-    """The 8-bit write puts quantize(token) at each slot, plain indexing
-    checked here, and skips negative slots."""
-    rng = np.random.default_rng(421)
-    H, D, B, N = 2, 8, 4, 6
-    kc = rng.integers(0, 256, size=(N, H, B, D), dtype=np.uint8)
-    vc = rng.integers(0, 256, size=(N, H, B, D), dtype=np.uint8)
-    k = rng.standard_normal((3, H, D)).astype(np.float32)
-    v = rng.standard_normal((3, H, D)).astype(np.float32)
-    slots = [5, -1, 22]
-    k2, v2 = oracle.cache_write_fp8(kc, vc, k, v, slots, B, 0.5, 0.125)
-    ek, ev = kc.copy(), vc.copy()
-    for t, sl in ((0, 5), (2, 22)):
-        ek[sl // B, :, sl % B] = oracle.e4m3_encode(k[t] / np.float32(0.5))
-        ev[sl // B, :, sl % B] = oracle.e4m3_encode(v[t] / np.float32(0.125))
-    assert np.array_equal(k2, ek) and np.array_equal(v2, ev)
+def test_fp8_cache_write_matches_hand_worked_golden():
+    """The 8-bit write against codes worked out by hand from the E4M3 format
+    (tests/golden/cache_write_fp8_tiny.json): division by the scale, ties to
+    the even mantissa, saturation at 448, subnormals, negative zero, the
+    slot's block and place, a skipped padding token, untouched rows."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                    "cache_write_fp8_tiny.json")))
+    shape = (g["num_blocks"], g["num_heads"], g["block_size"], g["head_dim"])
+    kc = np.full(shape, g["fill"], dtype=np.uint8)
+    vc = np.full(shape, g["fill"], dtype=np.uint8)
+    k = np.array(g["k"], dtype=np.float32)
+    v = np.array(g["v"], dtype=np.float32)
+    k2, v2 = oracle.cache_write_fp8(kc, vc, k, v, g["slot_mapping"], g["block_size"],
+                                    g["k_scale"], g["v_scale"])
+    assert k2.tolist() == g["expected_k_cache"]
+    assert v2.tolist() == g["expected_v_cache"]
 
 
 @pytest.mark.parametrize("pin", P.PREFILL_PINS, ids=lambda f: f.__name__)
 def test_prefill_pin(pin):
     pin(oracle.prefill)
+
+
+@pytest.mark.parametrize("pin", P.PREFIX_PINS, ids=lambda f: f.__name__)
+def test_prefill_with_prefix_pin(pin):
+    pin(oracle.prefill_with_prefix)
 
 
 @pytest.mark.parametrize("pin", P.SHARED_PINS, ids=lambda f: f.__name__)

@@ -337,6 +337,72 @@ def test_planted_prefill_mistake_is_caught(fn):
     assert failed, fn.__name__
 
 
+# --- prompt phase over a stored prefix: planted mistakes ---------------------
+
+def prefix_ignored(q, k, v, cu, kc, vc, tables, cached, scale, B):
+    """Planted mistake: the stored prefix is left out."""
+    return oracle.prefill(q, k, v, cu, scale)
+
+
+def prefix_offset_dropped(q, k, v, cu, kc, vc, tables, cached, scale, B):
+    """Planted mistake: new row i sees keys 0..i of the joined list, as if it
+    sat at position i instead of cached + i."""
+    out = np.zeros(q.shape)
+    for s in range(len(cu) - 1):
+        a, b, c = int(cu[s]), int(cu[s + 1]), int(cached[s])
+        K = np.concatenate([oracle.gather_context(kc, tables[s], c, B), k[a:b]])
+        V = np.concatenate([oracle.gather_context(vc, tables[s], c, B), v[a:b]])
+        kvh = oracle.kv_head_of(q.shape[1], k.shape[1])
+        for i in range(b - a):
+            out[a + i] = oracle.attend(q[a + i], K[:i + 1][:, kvh], V[:i + 1][:, kvh], scale)
+    return out
+
+
+def prefix_sees_the_future(q, k, v, cu, kc, vc, tables, cached, scale, B):
+    """Planted mistake: new rows see every new token, not just the earlier ones."""
+    out = np.zeros(q.shape)
+    for s in range(len(cu) - 1):
+        a, b, c = int(cu[s]), int(cu[s + 1]), int(cached[s])
+        K = np.concatenate([oracle.gather_context(kc, tables[s], c, B), k[a:b]])
+        V = np.concatenate([oracle.gather_context(vc, tables[s], c, B), v[a:b]])
+        kvh = oracle.kv_head_of(q.shape[1], k.shape[1])
+        for i in range(b - a):
+            out[a + i] = oracle.attend(q[a + i], K[:, kvh], V[:, kvh], scale)
+    return out
+
+
+def prefix_gathered_block_major(q, k, v, cu, kc, vc, tables, cached, scale, B):
+    """Planted mistake: a stored token's row is taken as place t // B of
+    block table[t % B] (the block and place indices swapped)."""
+    def gather(cache, table, c):
+        out = np.empty((c, cache.shape[1], cache.shape[3]))
+        for t in range(c):
+            out[t] = cache[int(table[min(t % B, len(table) - 1)]), :, min(t // B, B - 1), :]
+        return out
+    out = np.zeros(q.shape)
+    kvh = oracle.kv_head_of(q.shape[1], k.shape[1])
+    for s in range(len(cu) - 1):
+        a, b, c = int(cu[s]), int(cu[s + 1]), int(cached[s])
+        K = np.concatenate([gather(kc, tables[s], c), k[a:b]])
+        V = np.concatenate([gather(vc, tables[s], c), v[a:b]])
+        for i in range(b - a):
+            out[a + i] = oracle.attend(q[a + i], K[:c + i + 1][:, kvh], V[:c + i + 1][:, kvh],
+                                       scale)
+    return out
+
+
+@pytest.mark.parametrize("fn", [prefix_ignored, prefix_offset_dropped, prefix_sees_the_future,
+                                prefix_gathered_block_major], ids=lambda f: f.__name__)
+def test_planted_prefix_prefill_mistake_is_caught(fn):
+    failed = 0
+    for pin in P.PREFIX_PINS:
+        try:
+            pin(fn)
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    assert failed, fn.__name__
+
+
 # --- shared prefixes: planted mistakes ----------------------------------------
 
 def _shared_with(group_of=None, use_prefix=True, use_tail=True):
