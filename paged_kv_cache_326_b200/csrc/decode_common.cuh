@@ -54,11 +54,14 @@ inline size_t header_bytes(int num_seqs) {
   return align_up(sizeof(int32_t) * (kHeaderInts + num_seqs + 1), 256);
 }
 constexpr size_t kGrabBytes = 256;
-// The grain counter holds the call's epoch above bit 30; a stale epoch (an
-// earlier call's, or never set) reads as zero, so the workspace never needs
-// clearing.
+// The grain counter holds the call's epoch in bits 30-63 and the chunks
+// handed out below them.  A stale epoch (an earlier call's, or never set)
+// reads as zero, so the workspace never needs clearing before a call; the
+// merge kernel also resets the counter to zero once the decode grid is done,
+// so a call replayed with the same epoch (a captured CUDA graph) starts from
+// zero too.
 constexpr unsigned long long kGrabMask = (1ull << 30) - 1;
-constexpr unsigned long long kEpochMask = (1ull << 40) - 1;
+constexpr unsigned long long kEpochMask = (1ull << 34) - 1;
 
 // Units a launch with `warps` working warps can create (static runs plus at
 // most kGrainsPerWarp grains per warp).
@@ -90,7 +93,7 @@ struct DecodeParams {
   const int64_t* slot_mapping;    // one-launch step only: their slots
   int32_t* header;                // work split + prefix, for the merge kernel
   unsigned long long* grab;       // grain counter
-  unsigned long long epoch;       // 40-bit, never 0
+  unsigned long long epoch;       // 34-bit, never 0
   float* records;
   int32_t* status;
   int64_t wait_limit_ns;
@@ -225,7 +228,7 @@ struct Scheduler {
         sp(sp_), w(w_), lane(lane_) {
     step = 1;
     while (step * 2 <= S) step *= 2;
-    e34 = p.epoch & ((1ull << 34) - 1);
+    e34 = p.epoch & kEpochMask;
   }
 
   // Chunk offset of the grain whose counter value is `old` (lane 0).  A
@@ -448,9 +451,11 @@ __device__ __forceinline__ void merge_partials(const float* records, int64_t rec
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 split_reduce_kernel(T* __restrict__ out, const int32_t* __restrict__ header,
-                    const float* __restrict__ records, int num_seqs, int num_vheads,
-                    int num_q_heads, int nsub, int gs) {
+                    const float* __restrict__ records, unsigned long long* __restrict__ grab,
+                    int num_seqs, int num_vheads, int num_q_heads, int nsub, int gs) {
   griddep_wait();
+  // The decode grid is done with its grain counter: zero it for the next call
+  if (blockIdx.x == 0 && threadIdx.x == 0) *grab = 0ull;
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (item >= num_seqs * num_vheads * gs) return;
@@ -490,7 +495,7 @@ inline int device_sm_count() {
   return sms;
 }
 
-// A fresh 40-bit epoch per launch (never 0, so a zeroed workspace holds no
+// A fresh 34-bit epoch per launch (never 0, so a zeroed workspace holds no
 // live counts).
 inline unsigned long long next_epoch() {
   static std::atomic<unsigned long long> counter{0};
@@ -587,8 +592,8 @@ cudaError_t launch_merge(const DecodeParams& p, int gs, cudaStream_t stream) {
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, split_reduce_kernel<T, D>, static_cast<T*>(p.out),
                             static_cast<const int32_t*>(p.header),
-                            static_cast<const float*>(p.records), p.num_seqs, p.num_heads,
-                            p.num_q_heads, p.nsub, gs);
+                            static_cast<const float*>(p.records), p.grab, p.num_seqs,
+                            p.num_heads, p.num_q_heads, p.nsub, gs);
 }
 
 }  // namespace pa

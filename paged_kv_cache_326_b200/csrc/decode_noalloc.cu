@@ -8,10 +8,13 @@
 // is not allowed.  This entry point runs the same kernels as
 // pa_paged_attn_decode, but its scratch is a file-scope device array that the
 // library carries with it, so the caller passes only inputs and outputs.
+#include <cuda.h>  // CUcontext and CUresult, for the two driver entry points below
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "kernels.h"
 #include "pagedattn.h"
@@ -23,29 +26,71 @@ namespace {
 constexpr size_t kScratchBytes = size_t{16} << 20;
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_decode_scratch on the current device, looked up once
-// per device.  In host code the array's name is only a host-side stand-in,
-// never a device address, so it is resolved with cudaGetSymbolAddress.
+// Unique id of the calling thread's current context (0 if there is none or
+// the driver cannot say).  A device reset ends the primary context; the one
+// the runtime makes next has a new id, and the module holding
+// g_decode_scratch is loaded again into it, possibly at another address.
+unsigned long long current_context_id() {
+  static std::once_flag once;
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+    cudaGetLastError();
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, never a device address, so it is
+// resolved with cudaGetSymbolAddress: once per (device, context), the first
+// time a call runs there.  The lookup itself makes the device's primary
+// context current if no runtime call has yet.
 int scratch_address(void** out) {
   static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
+  static std::map<std::pair<int, unsigned long long>, void*> addr;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();
     return PA_ERR_CUDA;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return PA_ERR_CUDA;
+  const unsigned long long ctx = current_context_id();
+  if (ctx != 0) {
+    const auto it = addr.find({dev, ctx});
+    if (it != addr.end()) {
+      *out = it->second;
+      return PA_OK;
     }
-    addr[dev] = p;
   }
-  *out = addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  // cache it under the context the lookup ran in (made current by it if
+  // there was none); without a context id, look it up on every call
+  const unsigned long long ctx_now = ctx != 0 ? ctx : current_context_id();
+  if (ctx_now != 0) addr[{dev, ctx_now}] = p;
+  *out = p;
   return PA_OK;
 }
 

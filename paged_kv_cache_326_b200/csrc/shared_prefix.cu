@@ -66,8 +66,14 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256)
 shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_p,
                            const float* __restrict__ rec_p, const int32_t* __restrict__ hdr_t,
-                           const float* __restrict__ rec_t, int num_groups, int gs, int H) {
+                           const float* __restrict__ rec_t, unsigned long long* __restrict__ grab_p,
+                           unsigned long long* __restrict__ grab_t, int num_groups, int gs, int H) {
   griddep_wait();
+  // Both passes are done with their grain counters: zero them for the next call
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *grab_p = 0ull;
+    *grab_t = 0ull;
+  }
   constexpr int PER = D / 32;
   constexpr int RS = D + 4;  // floats per record
   const int lane = threadIdx.x & 31;
@@ -169,8 +175,10 @@ cudaError_t launch_shared_merge(const SharedPrefixArgs& a, const char* ws_p, int
       reinterpret_cast<const int32_t*>(ws_p),
       reinterpret_cast<const float*>(ws_p + header_bytes(S_p) + kGrabBytes),
       reinterpret_cast<const int32_t*>(ws_t),
-      reinterpret_cast<const float*>(ws_t + header_bytes(S_t) + kGrabBytes), a.num_groups,
-      a.group_size, a.num_heads);
+      reinterpret_cast<const float*>(ws_t + header_bytes(S_t) + kGrabBytes),
+      reinterpret_cast<unsigned long long*>(const_cast<char*>(ws_p) + header_bytes(S_p)),
+      reinterpret_cast<unsigned long long*>(const_cast<char*>(ws_t) + header_bytes(S_t)),
+      a.num_groups, a.group_size, a.num_heads);
 }
 
 // The two passes' workspaces, one after the other (256-byte aligned).

@@ -80,3 +80,26 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(P):
                                           ctypes.c_void_p(status.data_ptr()), None)
     assert rc == P.binding.PA_ERR_TOO_LARGE
     assert "scratch" in P.pa_status_string(rc)
+
+
+def test_noalloc_limit_is_the_16bit_kernels_need(P):
+    """The 16 MiB limit applies to what the 16-bit kernels, the only ones
+    this call runs, need.  At 256 texts x 40 heads x 128 (blocks of 16, 128
+    per text) the general workspace query, which also sizes for the 8-bit
+    kernel's larger grid, asks for more than 16 MiB; the call still accepts
+    the size and matches the workspace entry point."""
+    w = W.skewed(block_size=16, device="cuda")
+    assert (w.num_seqs, w.num_heads, w.head_dim, w.max_blocks_per_seq) == (256, 40, 128, 128)
+    assert P.pa_paged_attn_decode_workspace_size(256, 40, 128, 16, 128) > (16 << 20)
+    P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping)
+    ref = torch.empty_like(w.q)
+    P.pa_paged_attn_decode(ref, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                           w.scale)
+    out = torch.full_like(w.q, float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = _noalloc_raw(P, out, w, status)
+    torch.cuda.synchronize()
+    assert rc == 0, P.pa_status_string(rc)
+    assert status.item() == 0
+    c = compare(out, ref.double().cpu().numpy(), w.q.dtype)
+    assert c.ok, str(c)
