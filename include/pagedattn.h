@@ -133,8 +133,10 @@ size_t pa_paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head
  *   workspace      device scratch of at least
  *                  pa_paged_attn_decode_workspace_size(...) bytes, 256-byte
  *                  aligned; no initial contents needed (its grain counter is
- *                  tagged with a per-call epoch); must not be shared by
- *                  calls that may run at the same time
+ *                  tagged with a per-call epoch, and the call's last kernel
+ *                  zeroes it, so a call replayed from a captured CUDA graph
+ *                  starts clean too); must not be shared by calls that may
+ *                  run at the same time
  *   d_status       nullable device int32 (see conventions)
  * Work is split over all SMs in 16-token (head_dim 128) or 32-token
  * (head_dim 64) chunks: static runs, then grains from a shared counter; a
@@ -320,7 +322,10 @@ int pa_kv_cache_write_fp8(const void* k, const void* v, void* k_cache, void* v_c
  *                  sizes as the 16-bit call).  Multi-head only.  Other
  *                  arguments and errors as for pa_paged_attn_decode.
  * Each chunk of work is 4096/head_dim tokens (32 at head_dim 128), so every
- * copy still moves 4 KB of keys and 4 KB of values.
+ * copy still moves 4 KB of keys and 4 KB of values.  With fp16 queries,
+ * head_dim 128 and blocks of 8, 16 or 32 the products run on the tensor
+ * cores (PA_OPT_FP8_KERNEL picks the kernel): the codes are widened exactly
+ * to fp16 and multiplied with fp32 accumulation.
  */
 int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* block_tables, const int32_t* context_lens,
@@ -354,6 +359,12 @@ int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, cons
  *   k_cache, v_cache, slot_mapping, block_size, num_blocks
  *                  the pool and each token's slot, as for pa_kv_cache_write;
  *                  k_cache NULL skips the store (attention only)
+ * On the tcgen05 kernel (the default) with block_size 8, 16 or 32 the store
+ * is done by the attention kernel itself, from the key and value tiles it
+ * has loaded: a block of block_size tokens whose slots fill one physical
+ * block in order goes out as one tiled copy, other tokens row by row;
+ * otherwise a separate cache write runs first.  Either way the pool holds
+ * the same bits afterwards.
  * Support: head_dim 64 or 128; num_seqs <= 65535.  Returns PA_OK or
  * PA_ERR_INVALID / PA_ERR_CUDA.
  */
@@ -362,6 +373,47 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
                int num_seqs, int num_tokens, int max_seqlen, float scale, int num_heads,
                int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, pa_dtype dt,
                int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_prefill_with_prefix — the prompt phase of prompts whose first tokens are
+ * already in the cache ("The KV Cache and PagedAttention", section "What Came
+ * After": a prompt that begins like an earlier one reuses the earlier one's
+ * blocks, which saves the time spent on the prompt; pa_bm_add_seq_tokens
+ * reports how many leading tokens were taken over).
+ *
+ * Prompt s has cached_lens[s] tokens stored in the pool, in the blocks
+ * block_tables[s][0 .. cached_lens[s] / block_size - 1] (a multiple of
+ * block_size); rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of q, k, v and out are
+ * its other tokens, at positions cached_lens[s] + i.  With K the stored keys
+ * followed by the new ones (V likewise), row a + i is
+ *     out[a+i][h] = sum_{u <= cached_lens[s] + i} softmax_u(scale * q[a+i][h] . K[u]) V[u],
+ * which equals the rows of pa_prefill over the whole prompt that belong to
+ * the new tokens (up to rounding).  The stored keys and values are read
+ * through the table by the tensor-core kernel; nothing is recomputed for
+ * them.  With slot_mapping non-NULL the new tokens' keys and values are
+ * stored at their slots as pa_prefill does.
+ *
+ *   out, q, k, v   the new tokens only, as for pa_prefill
+ *   k_cache, v_cache the pool (layout above), device; read through the
+ *                  tables, written at slot_mapping
+ *   slot_mapping   [num_tokens] int64, device, or NULL (no store)
+ *   block_tables   [num_seqs][max_blocks_per_seq] int32, device
+ *   cached_lens    [num_seqs] int32, device: 0 <= cached_lens[s] <=
+ *                  max_blocks_per_seq * block_size, a multiple of block_size
+ *                  (else PA_ERR_BAD_LEN in *d_status and prompt s is skipped);
+ *                  a table entry outside [0, num_blocks) is PA_ERR_BAD_BLOCK
+ *                  and its rows read as zeros
+ * Support: the tcgen05 kernel only (PA_OPT_PREFILL_KERNEL 0 or 2), head_dim
+ * 64 or 128, block_size 8, 16 or 32.  Returns PA_OK or PA_ERR_INVALID /
+ * PA_ERR_CUDA.
+ */
+int pa_prefill_with_prefix(void* out, const void* q, const void* k, const void* v,
+                           void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                           const int32_t* cu_seqlens, const int32_t* block_tables,
+                           const int32_t* cached_lens, int num_seqs, int num_tokens,
+                           int max_seqlen, int max_blocks_per_seq, float scale, int num_heads,
+                           int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                           pa_dtype dt, int32_t* d_status, pa_stream_t stream);
 
 /*
  * pa_copy_blocks — copy whole blocks from one pool to another, or within one
@@ -409,6 +461,28 @@ int pa_read_probe(const void* buf, size_t bytes, uint32_t* d_sink, int sink_word
                   pa_stream_t stream);
 
 /*
+ * pa_write_probe — a diagnostic with no counterpart in the pages: write
+ * `bytes` (a multiple of 16) of device buffer `buf` once with a write-only
+ * streaming kernel (a persistent grid, four 16-byte streaming stores per
+ * thread per round; the contents become an index pattern), to measure the
+ * write ceiling that block copies (pa_copy_blocks) are compared with.
+ * Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_write_probe(void* buf, size_t bytes, pa_stream_t stream);
+
+/*
+ * pa_exp2_probe — a diagnostic with no counterpart in the pages: d_y[i] =
+ * 2^d_x[i] for i < n (device float arrays), computed the way the prompt-phase
+ * kernel computes part of its softmax weights: method 0 the FMA-pipe
+ * polynomial (range reduction to [-1/2, 1/2], degree-5 minimax polynomial,
+ * exponent insertion; inputs below -125 give 2^-125), method 1 the
+ * exponential unit (ex2.approx.ftz).  Lets a test hold the polynomial to
+ * its error bound on the GPU itself.  Returns PA_OK or PA_ERR_INVALID /
+ * PA_ERR_CUDA.
+ */
+int pa_exp2_probe(const float* d_x, float* d_y, int64_t n, int method, pa_stream_t stream);
+
+/*
  * pa_paged_attn_decode_noalloc — pa_paged_attn_decode without a caller
  * workspace, for callers that cannot allocate device memory (a host framework
  * that owns every device allocation, a fixed memory budget, a loop where an
@@ -418,14 +492,19 @@ int pa_read_probe(const void* buf, size_t bytes, uint32_t* d_sink, int sink_word
  * Same arguments, computation, result and errors as pa_paged_attn_decode,
  * minus workspace/workspace_bytes.  Its scratch is a static device array of
  * 16 MiB inside the library; every GPU that loads the library holds it until
- * the process exits.  Sizes whose workspace
- * (pa_paged_attn_decode_workspace_size) exceeds 16 MiB are rejected with
- * PA_ERR_TOO_LARGE before anything is launched (16 MiB covers, e.g., 256 texts
- * x 40 heads x 128 on a 148-SM B200).  The call allocates and frees nothing.
+ * the process exits.  Only the 16-bit kernels run here, so the limit applies
+ * to what they need: sizes whose 16-bit scratch need exceeds 16 MiB are
+ * rejected with PA_ERR_TOO_LARGE before anything is launched.  That need can
+ * be below pa_paged_attn_decode_workspace_size, which also covers the 8-bit
+ * kernels: 256 texts x 40 heads x 128 (blocks of 16, 128 per text) on a
+ * 148-SM B200 needs less than 16 MiB here but more from that query.  The
+ * call allocates and frees nothing.
  *
  * The first call on each device looks up the array's device address (a host
  * runtime call, cudaGetSymbolAddress); make that first call before any
- * stream capture.  All calls share the one array and leave their contents in
+ * stream capture.  The address is kept per device and context: after a
+ * device reset (cudaDeviceReset), the first call in the new context looks it
+ * up again.  All calls share the one array and leave their contents in
  * it (nothing in it needs to start at zero): calls that may overlap on the
  * GPU, on any streams, race and must be serialised by the caller.
  */
@@ -462,10 +541,27 @@ int pa_paged_attn_decode_noalloc(void* out, const void* q, const void* k_cache,
  *                         5th-generation tensor cores (tcgen05, accumulators
  *                         in tensor memory, 128 queries per CTA); 1 the
  *                         warp-level tensor cores (mma.sync).  Same function.
+ *   PA_OPT_FP8_KERNEL     which kernel pa_paged_attn_decode_fp8 runs: 0
+ *                         (default) the tensor-core kernel where it applies
+ *                         (fp16 queries, head_dim 128, block_size 8, 16 or
+ *                         32, num_blocks * num_heads * block_size < 2^31),
+ *                         else the CUDA-core one; 1 always the CUDA-core
+ *                         kernel; 2 always the tensor-core kernel
+ *                         (PA_ERR_INVALID where it does not apply).  Both
+ *                         widen the codes exactly and sum in fp32; the
+ *                         tensor-core kernel carries the softmax weights into
+ *                         the weighted sum of values as the sum of two fp16
+ *                         values.
+ *   PA_OPT_PREFIX_KEY_BITS bits of the chained prefix hash that block
+ *                         managers created after the call use as their
+ *                         lookup key, 1..64 (default 64).  Fewer bits make
+ *                         different prefixes share keys; a test uses that to
+ *                         exercise the checks that keep such prefixes from
+ *                         sharing blocks.
  * Returns PA_OK or PA_ERR_INVALID for an unknown key or value.
  */
 enum { PA_OPT_WAIT_LIMIT_NS = 1, PA_OPT_DECODE_WARPS = 2, PA_OPT_GQA_KERNEL = 3,
-       PA_OPT_PREFILL_KERNEL = 4 };
+       PA_OPT_PREFILL_KERNEL = 4, PA_OPT_PREFIX_KEY_BITS = 5, PA_OPT_FP8_KERNEL = 6 };
 int pa_set_option(int key, int64_t value);
 
 /* ------------------------------------------------------------------------ */
@@ -533,8 +629,14 @@ int pa_bm_export(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* block_
  * A cached block whose count falls to zero stays cached while it waits in
  * the free list.  When the free list hands it out again it is evicted: its
  * hash is dropped.  Blocks added by pa_bm_add_seq or filled by appends are
- * not cached.  The chained hash is a 64-bit SplitMix64-style mix: two
- * different prefixes with equal hashes would share blocks.  All or nothing.
+ * not cached.  The chained hash is a 64-bit SplitMix64-style mix, used as
+ * the lookup key.  A key match alone is not a hit: the cached block's own
+ * token ids must equal the prompt's, and a second 64-bit hash of the whole
+ * prefix (FNV-1a over the token ids' bytes), kept per cached block, must
+ * match too.  Two different prefixes could share a block only if both
+ * 64-bit hashes collided while the last block's ids agree.  A key already
+ * held by a block whose check fails stays with that block; the new block
+ * is then not cached.  All or nothing.
  * pa_bm_num_cached_blocks counts the hashes currently held. */
 int pa_bm_add_seq_tokens(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
                          int* num_cached_tokens);

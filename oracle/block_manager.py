@@ -29,7 +29,13 @@ earlier text's blocks.  ``add_seq_tokens`` takes over cached blocks up to the
 first miss and caches the prompt's new full blocks; a cached block with count
 zero keeps its hash while it waits in the free list, a hit takes it back out,
 and handing it out again from the free list drops the hash.  The chained hash
-is SplitMix64's output mix applied token by token (defined below).
+is SplitMix64's output mix applied token by token (defined below).  A hash is
+how a block is looked up, not proof that it holds the same text: a cached
+block is taken over only if the whole prefix it was cached for (every token
+up to its end) equals the new prompt's, compared here token by token.
+``key_bits`` keeps only the low bits of the hash as the lookup key, so that
+tests can make different prefixes meet on one key; a key already held stays
+with its block.
 
 Pinned by tests/golden/cow_two_answers.json (the pages' two-answer example)
 and by invariants checked in tests/test_block_manager.py; prefix reuse by the
@@ -67,7 +73,7 @@ class BlockManagerError(Exception):
 
 class BlockManagerModel:
     def __init__(self, num_blocks: int, block_size: int,
-                 initial_order: Optional[Sequence[int]] = None):
+                 initial_order: Optional[Sequence[int]] = None, key_bits: int = 64):
         if num_blocks <= 0 or block_size <= 0:
             raise BlockManagerError("invalid", "num_blocks and block_size must be > 0")
         self.num_blocks = num_blocks
@@ -79,13 +85,16 @@ class BlockManagerModel:
         self.ref: List[int] = [0] * num_blocks
         self.tables: Dict[int, List[int]] = {}
         self.tokens: Dict[int, int] = {}
-        self.cache: Dict[int, int] = {}        # chained hash -> block
-        self.cached: Dict[int, int] = {}       # block -> its hash
+        self.cache: Dict[int, int] = {}        # lookup key -> block
+        self.cached: Dict[int, int] = {}       # block -> its key
+        self.prefix_of: Dict[int, tuple] = {}  # block -> every token up to its end
+        self.key_mask = (1 << key_bits) - 1
 
     # -- helpers -----------------------------------------------------------
     def _take(self) -> int:
         b = self.free.popleft()
         h = self.cached.pop(b, None)
+        self.prefix_of.pop(b, None)
         if h is not None and self.cache.get(h) == b:
             del self.cache[h]
         self.ref[b] = 1
@@ -120,9 +129,11 @@ class BlockManagerModel:
         hashes, hits, prev, run = [], [], 0, True
         for j in range(full):
             prev = block_hash(prev, tokens[j * B:(j + 1) * B])
-            hashes.append(prev)
-            if run and prev in self.cache:
-                hits.append(self.cache[prev])
+            key = prev & self.key_mask
+            hashes.append(key)
+            prefix = tuple(int(t) for t in tokens[:(j + 1) * B])
+            if run and key in self.cache and self.prefix_of[self.cache[key]] == prefix:
+                hits.append(self.cache[key])
             else:
                 run = False
         n_blocks = -(-n // B)
@@ -141,6 +152,7 @@ class BlockManagerModel:
             if j < full and hashes[j] not in self.cache:
                 self.cache[hashes[j]] = b
                 self.cached[b] = hashes[j]
+                self.prefix_of[b] = tuple(int(t) for t in tokens[:(j + 1) * B])
         self.tables[seq_id] = table
         self.tokens[seq_id] = n
         return len(hits) * B

@@ -40,6 +40,8 @@ PA_OPT_WAIT_LIMIT_NS = 1
 PA_OPT_DECODE_WARPS = 2
 PA_OPT_GQA_KERNEL = 3
 PA_OPT_PREFILL_KERNEL = 4
+PA_OPT_PREFIX_KEY_BITS = 5
+PA_OPT_FP8_KERNEL = 6
 
 _KIND = {PA_ERR_INVALID: "invalid", PA_ERR_CUDA: "cuda", PA_ERR_OUT_OF_BLOCKS: "out_of_blocks",
          PA_ERR_NO_SEQ: "no_seq", PA_ERR_EXISTS: "exists", PA_ERR_TABLE_FULL: "table_full",
@@ -80,7 +82,12 @@ _SIGNATURES = {
                                         _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _f32, _i32,
                           _i32, _i32, _i32, _i64, _i32, _vp, _vp]),
+    "pa_prefill_with_prefix": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                                      _i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64,
+                                      _i32, _vp, _vp]),
     "pa_read_probe": (_i32, [_vp, _sz, _vp, _i32, _vp]),
+    "pa_exp2_probe": (_i32, [_vp, _vp, _i64, _i32, _vp]),
+    "pa_write_probe": (_i32, [_vp, _sz, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32,
                               _vp, _vp]),
     "pa_paged_attn_decode_shared_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32,
@@ -273,12 +280,68 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Ten
     return out
 
 
+def pa_prefill_with_prefix(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor,
+                           v: torch.Tensor, cu_seqlens: torch.Tensor, max_seqlen: int,
+                           scale: float, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                           block_tables: torch.Tensor, cached_lens: torch.Tensor,
+                           slot_mapping: Optional[torch.Tensor] = None,
+                           status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Prompt phase of prompts whose first cached_lens[s] tokens are stored
+    in the caches (blocks block_tables[s]): out, q [T][H][D] and k, v
+    [T][H_kv][D] hold the other tokens; slot_mapping [T] int64 (optional)
+    stores their keys and values."""
+    T, H, D = q.shape
+    Tk, Hkv, Dk = k.shape
+    if out.shape != q.shape or v.shape != k.shape or Tk != T or Dk != D or H % Hkv:
+        raise ValueError("shape mismatch")
+    S = cu_seqlens.numel() - 1
+    N, Hc, B, Dc = k_cache.shape
+    if v_cache.shape != k_cache.shape or (Hc, Dc) != (Hkv, D) or k_cache.dtype != q.dtype:
+        raise ValueError("caches must be [N][H_kv][B][D] of q's dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or cached_lens.shape != (S,):
+        raise ValueError("block_tables must be [S][max_blocks], cached_lens [S]")
+    sm = None
+    if slot_mapping is not None:
+        if slot_mapping.shape != (T,):
+            raise ValueError("slot_mapping must be [T]")
+        sm = _cuda(slot_mapping, "slot_mapping", torch.int64)
+    for t in (out, k, v):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v and out must share a dtype")
+    code = lib().pa_prefill_with_prefix(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"),
+        _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"), sm,
+        _cuda(cu_seqlens, "cu_seqlens", torch.int32),
+        _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(cached_lens, "cached_lens", torch.int32), S, T, int(max_seqlen),
+        block_tables.shape[1], float(scale), H, Hkv, D, B, N, _dtype_code(q),
+        _status_ptr(status), _stream(stream, q.device))
+    _check(code, "pa_prefill_with_prefix")
+    return out
+
+
 def pa_read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
     """Read every byte of the CUDA tensor `buf` once (the HBM read ceiling);
     sink: a CUDA int32 tensor of at least 4 x the SM count words."""
     nbytes = buf.numel() * buf.element_size()
     _check(lib().pa_read_probe(_cuda(buf, "buf"), nbytes & ~15, _cuda(sink, "sink", torch.int32),
                                sink.numel(), _stream(stream, buf.device)), "pa_read_probe")
+
+
+def pa_write_probe(buf: torch.Tensor, stream=None) -> None:
+    """Write the whole (contiguous, device) buffer once: the write ceiling."""
+    _check(lib().pa_write_probe(_cuda(buf, "buf"), buf.numel() * buf.element_size(),
+                                _stream(stream, buf.device)), "pa_write_probe")
+
+
+def pa_exp2_probe(x: torch.Tensor, y: torch.Tensor, method: int, stream=None) -> None:
+    """y = 2^x (float32 device tensors) by the softmax polynomial (method 0)
+    or the exponential unit (method 1)."""
+    if x.shape != y.shape:
+        raise ValueError("x and y must have one shape")
+    _check(lib().pa_exp2_probe(_cuda(x, "x", torch.float32), _cuda(y, "y", torch.float32),
+                               x.numel(), int(method), _stream(stream, x.device)),
+           "pa_exp2_probe")
 
 
 def _pool(t: torch.Tensor, name: str) -> int:

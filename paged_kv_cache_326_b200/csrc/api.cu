@@ -15,6 +15,8 @@ std::atomic<int64_t> g_wait_limit_ns{1000000000};
 std::atomic<int64_t> g_decode_warps{0};
 std::atomic<int64_t> g_gqa_kernel{0};
 std::atomic<int64_t> g_prefill_kernel{0};
+std::atomic<int64_t> g_prefix_key_bits{64};
+std::atomic<int64_t> g_fp8_kernel{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -55,6 +57,8 @@ namespace pa {
 int64_t option_decode_warps() { return g_decode_warps.load(); }
 int64_t option_gqa_kernel() { return g_gqa_kernel.load(); }
 int64_t option_prefill_kernel() { return g_prefill_kernel.load(); }
+int64_t option_prefix_key_bits() { return g_prefix_key_bits.load(); }
+int64_t option_fp8_kernel() { return g_fp8_kernel.load(); }
 }  // namespace pa
 
 extern "C" {
@@ -92,6 +96,14 @@ int pa_set_option(int key, int64_t value) {
     case PA_OPT_PREFILL_KERNEL:
       if (value < 0 || value > 2) return PA_ERR_INVALID;
       g_prefill_kernel = value;
+      return PA_OK;
+    case PA_OPT_FP8_KERNEL:
+      if (value < 0 || value > 2) return PA_ERR_INVALID;
+      g_fp8_kernel = value;
+      return PA_OK;
+    case PA_OPT_PREFIX_KEY_BITS:
+      if (value < 1 || value > 64) return PA_ERR_INVALID;
+      g_prefix_key_bits = value;
       return PA_OK;
     default: return PA_ERR_INVALID;
   }
@@ -237,14 +249,21 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
   if (!out || !q || !k || !v || !cu_seqlens) return PA_ERR_INVALID;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return PA_ERR_INVALID;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (k_cache) {  // store the prompts' keys and values in their blocks first
+  const bool tc = g_prefill_kernel.load() != 1;
+  bool fused_store = false;
+  if (k_cache) {  // store the prompts' keys and values in their blocks
     if (!v_cache || !slot_mapping || !shape_ok(num_kv_heads, head_dim, block_size) ||
         num_blocks <= 0 || !aligned16(k_cache) || !aligned16(v_cache))
       return PA_ERR_INVALID;
-    const int rc = from_cuda(pa::launch_kv_cache_write(k, v, k_cache, v_cache, slot_mapping,
-                                                       num_tokens, num_kv_heads, head_dim,
-                                                       block_size, num_blocks, d_status, st));
-    if (rc != PA_OK) return rc;
+    // the tcgen05 kernel stores them from its own tiles; otherwise a cache
+    // write runs first
+    fused_store = tc && pa::prefill_tc_paged_ok(block_size, num_blocks);
+    if (!fused_store) {
+      const int rc = from_cuda(pa::launch_kv_cache_write(k, v, k_cache, v_cache, slot_mapping,
+                                                         num_tokens, num_kv_heads, head_dim,
+                                                         block_size, num_blocks, d_status, st));
+      if (rc != PA_OK) return rc;
+    }
   }
   pa::PrefillArgs a;
   a.out = out;
@@ -262,8 +281,61 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
   a.is_bf16 = dt == PA_BF16;
   a.status = d_status;
   a.wait_limit_ns = g_wait_limit_ns.load();
-  return from_cuda(g_prefill_kernel.load() == 1 ? pa::launch_prefill(a, st)
-                                                : pa::launch_prefill_tc(a, st));
+  if (fused_store) {
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_size = block_size;
+    a.num_blocks = num_blocks;
+    a.slot_mapping = slot_mapping;
+  }
+  return from_cuda(tc ? pa::launch_prefill_tc(a, st) : pa::launch_prefill(a, st));
+}
+
+int pa_prefill_with_prefix(void* out, const void* q, const void* k, const void* v,
+                           void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                           const int32_t* cu_seqlens, const int32_t* block_tables,
+                           const int32_t* cached_lens, int num_seqs, int num_tokens,
+                           int max_seqlen, int max_blocks_per_seq, float scale, int num_heads,
+                           int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                           pa_dtype dt, int32_t* d_status, pa_stream_t stream) {
+  if (num_seqs < 0 || num_seqs > 65535 || num_tokens < 0 || max_seqlen < 0 ||
+      max_blocks_per_seq < 1 || num_heads < 1 || num_heads > 65535 || num_kv_heads < 1 ||
+      num_heads % num_kv_heads || (head_dim != 64 && head_dim != 128) ||
+      (dt != PA_F16 && dt != PA_BF16) || g_prefill_kernel.load() == 1 ||
+      !pa::prefill_tc_paged_ok(block_size, num_blocks))
+    return PA_ERR_INVALID;
+  if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+  if (!out || !q || !k || !v || !cu_seqlens || !k_cache || !v_cache || !block_tables ||
+      !cached_lens)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  pa::PrefillArgs a;
+  a.out = out;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.cu_seqlens = cu_seqlens;
+  a.num_seqs = num_seqs;
+  a.num_tokens = num_tokens;
+  a.max_seqlen = max_seqlen;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.scale = scale;
+  a.is_bf16 = dt == PA_BF16;
+  a.status = d_status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.block_tables = block_tables;
+  a.cached_lens = cached_lens;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.slot_mapping = slot_mapping;
+  return from_cuda(pa::launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int pa_read_probe(const void* buf, size_t bytes, uint32_t* d_sink, int sink_words,
@@ -271,6 +343,18 @@ int pa_read_probe(const void* buf, size_t bytes, uint32_t* d_sink, int sink_word
   if (!buf || !d_sink || bytes == 0 || (bytes & 15u) || sink_words < 1 || !aligned16(buf))
     return PA_ERR_INVALID;
   return from_cuda(pa::launch_read_probe(buf, static_cast<int64_t>(bytes), d_sink, sink_words,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pa_write_probe(void* buf, size_t bytes, pa_stream_t stream) {
+  if (!buf || bytes == 0 || (bytes & 15u) || !aligned16(buf)) return PA_ERR_INVALID;
+  return from_cuda(pa::launch_write_probe(buf, static_cast<int64_t>(bytes),
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pa_exp2_probe(const float* d_x, float* d_y, int64_t n, int method, pa_stream_t stream) {
+  if (n < 0 || (method != 0 && method != 1) || (n > 0 && (!d_x || !d_y))) return PA_ERR_INVALID;
+  return from_cuda(pa::launch_exp2_probe(d_x, d_y, n, method,
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 

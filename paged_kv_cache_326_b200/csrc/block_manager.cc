@@ -18,14 +18,22 @@
 // the first miss.  A cached block whose count falls to zero stays cached
 // while it waits in the free list; a hit takes it back out; the allocator
 // evicts it (drops its hash) when it hands the block out again.  Only
-// prompt blocks registered by pa_bm_add_seq_tokens are cached.
+// prompt blocks registered by pa_bm_add_seq_tokens are cached.  A hash match
+// alone never shares a block: a hit also needs the block's own token ids to
+// be equal, and a second, independent 64-bit hash of the whole prefix (FNV-1a)
+// to be equal, so a collision of the chained hash is caught.
 #include <cstdint>
+#include <cstring>
 #include <deque>
 #include <new>
 #include <unordered_map>
 #include <vector>
 
 #include "pagedattn.h"
+
+namespace pa {
+int64_t option_prefix_key_bits();
+}
 
 struct pa_bm {
   int64_t num_blocks;
@@ -39,10 +47,14 @@ struct pa_bm {
   std::vector<uint32_t> free_stamp;
   int64_t free_count = 0;
   std::vector<int32_t> ref;                      // texts using each block
-  // prefix cache: chained hash -> block, and each cached block's hash
+  // prefix cache: key (the chained hash, masked by key_mask) -> block; each
+  // cached block's key, its token ids and the second hash of its prefix
   std::unordered_map<uint64_t, int32_t> cache;
   std::vector<uint8_t> cached;
   std::vector<uint64_t> cached_hash;
+  std::vector<uint64_t> cached_check;  // FNV-1a of every token up to the block's end
+  std::vector<int32_t> cached_tokens;  // block_size ids per block, sized on first use
+  uint64_t key_mask = ~0ull;
   struct Seq {
     std::vector<int32_t> blocks;
     int64_t tokens;
@@ -122,6 +134,23 @@ uint64_t block_hash(uint64_t prev, const int32_t* tokens, int n) {
   return h;
 }
 
+// The check hash: 64-bit FNV-1a (Fowler, Noll, Vo) over the four
+// little-endian bytes of every token id, continued from `prev` (the FNV
+// offset basis before the first block).  Independent of the chained hash, so
+// two different prefixes pass as equal only if both 64-bit hashes collide.
+constexpr uint64_t kFnvBasis = 0xcbf29ce484222325ull;
+uint64_t check_hash(uint64_t prev, const int32_t* tokens, int n) {
+  uint64_t h = prev;
+  for (int i = 0; i < n; ++i) {
+    const uint32_t t = static_cast<uint32_t>(tokens[i]);
+    for (int b = 0; b < 4; ++b) {
+      h ^= (t >> (8 * b)) & 0xffu;
+      h *= 0x100000001b3ull;
+    }
+  }
+  return h;
+}
+
 }  // namespace
 
 extern "C" {
@@ -147,6 +176,9 @@ pa_bm* pa_bm_create(int64_t num_blocks, int block_size, uint64_t shuffle_seed) {
   bm->ref.assign(static_cast<size_t>(num_blocks), 0);
   bm->cached.assign(static_cast<size_t>(num_blocks), 0);
   bm->cached_hash.assign(static_cast<size_t>(num_blocks), 0);
+  bm->cached_check.assign(static_cast<size_t>(num_blocks), 0);
+  const int64_t bits = pa::option_prefix_key_bits();
+  bm->key_mask = bits >= 64 ? ~0ull : ((1ull << bits) - 1);
   return bm;
 }
 
@@ -230,20 +262,30 @@ int pa_bm_add_seq_tokens(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int n
   const int B = bm->block_size;
   const int64_t full = num_tokens / B;
   const int64_t need = (static_cast<int64_t>(num_tokens) + B - 1) / B;
-  // the chained hashes of the full blocks, and the cached run at the front
-  std::vector<uint64_t> h(static_cast<size_t>(full));
+  if (full > 0 && bm->cached_tokens.empty())
+    bm->cached_tokens.assign(static_cast<size_t>(bm->num_blocks) * B, 0);
+  // the keys of the full blocks, and the cached run at the front: a cached
+  // block is a hit only if its token ids and its prefix's check hash agree
+  std::vector<uint64_t> h(static_cast<size_t>(full)), chk(static_cast<size_t>(full));
   std::vector<int32_t> hit;
   bool run = true;
-  uint64_t prev = 0;
+  uint64_t prev = 0, prev_chk = kFnvBasis;
   for (int64_t j = 0; j < full; ++j) {
-    prev = block_hash(prev, tokens + j * B, B);
-    h[j] = prev;
+    const int32_t* tj = tokens + j * B;
+    prev = block_hash(prev, tj, B);
+    prev_chk = check_hash(prev_chk, tj, B);
+    h[j] = prev & bm->key_mask;
+    chk[j] = prev_chk;
     if (run) {
-      auto it = bm->cache.find(prev);
-      if (it == bm->cache.end()) {
-        run = false;
-      } else {
+      auto it = bm->cache.find(h[j]);
+      const bool same =
+          it != bm->cache.end() && bm->cached_check[it->second] == prev_chk &&
+          std::memcmp(bm->cached_tokens.data() + static_cast<size_t>(it->second) * B, tj,
+                      sizeof(int32_t) * B) == 0;
+      if (same) {
         hit.push_back(it->second);
+      } else {
+        run = false;
       }
     }
   }
@@ -270,6 +312,9 @@ int pa_bm_add_seq_tokens(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int n
       bm->cache.emplace(h[j], b);
       bm->cached[b] = 1;
       bm->cached_hash[b] = h[j];
+      bm->cached_check[b] = chk[j];
+      std::memcpy(bm->cached_tokens.data() + static_cast<size_t>(b) * B, tokens + j * B,
+                  sizeof(int32_t) * B);
     }
   }
   bm->seqs.emplace(seq_id, std::move(s));

@@ -5,10 +5,13 @@
 // (section "When Memory Runs Out").
 //
 // A block of one pool tensor is one contiguous run of H * B * D elements, so
-// a copy is a plain stream of 16-byte vectors.  Each CTA copies one piece of
-// one (pair, K-or-V) block with every thread keeping kUnroll vectors in
-// flight; the grid covers all pieces of all pairs at once.  The kernel is
-// HBM-bound (every byte read once and written once).
+// a copy is a plain stream of 16-byte vectors.  All copies of a call (pair p
+// and K or V: copy 2p or 2p+1) form one flat order of vectors, and a
+// persistent grid (kCopyCtasPerSm CTAs per SM) cuts it into equal contiguous
+// shares, one per CTA: no CTA waits on a partial second wave, and a share
+// may run across the end of one copy into the next.  Each thread keeps
+// kUnroll vectors in flight.  The kernel is HBM-bound (every distinct byte
+// read once and written once).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -22,42 +25,74 @@ namespace {
 
 constexpr int kCopyThreads = 256;
 constexpr int kUnroll = 4;
-constexpr int64_t kVecsPerCta = kCopyThreads * kUnroll * 2;  // 32 KB per CTA
+constexpr int kCopyCtasPerSm = 3;
 
-__global__ void __launch_bounds__(kCopyThreads)
+__global__ void __launch_bounds__(kCopyThreads, kCopyCtasPerSm)
 copy_blocks_kernel(const uint4* src_k, const uint4* src_v, uint4* dst_k, uint4* dst_v,
-                   const int32_t* __restrict__ pairs, int64_t vecs_per_block, int ctas_per_copy,
+                   const int32_t* __restrict__ pairs, int64_t vecs_per_block, int64_t total,
                    int64_t src_num_blocks, int64_t dst_num_blocks, int32_t* status) {
   // The pairs or the source blocks may come from the kernel launched just
   // before; a kernel launched after this one waits for all of it.
   griddep_wait();
   griddep_launch_dependents();
-  const int64_t copy = blockIdx.x / ctas_per_copy;  // (pair, K or V)
-  const int piece = static_cast<int>(blockIdx.x - copy * ctas_per_copy);
-  const int64_t pair = copy >> 1;
-  const bool is_v = copy & 1;
-  const int64_t s = __ldg(pairs + 2 * pair);
-  const int64_t d = __ldg(pairs + 2 * pair + 1);
-  if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) {
-    if (piece == 0 && !is_v && threadIdx.x == 0) set_status(status, -7 /* PA_ERR_BAD_BLOCK */);
-    return;
+  constexpr int kStep = kCopyThreads * kUnroll;
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  const int64_t lo = blockIdx.x * per;
+  // vectors in this CTA's share (fewer than 2^31: the grid has at least
+  // one CTA per SM and the host limits the total)
+  const int n = static_cast<int>(max(int64_t{0}, min(per, total - lo)));
+  const int vpb = static_cast<int>(vecs_per_block);
+  // Lane u of this thread walks vectors i = u * kCopyThreads + tid of the
+  // share, + kStep each round, keeping its copy index and offset up to date
+  // (one division to start with, then additions).
+  int i[kUnroll], copy[kUnroll], off[kUnroll];
+  const uint4* src[kUnroll];
+  uint4* dst[kUnroll];
+  // the endpoints of copy c (pair c / 2, K or V); null if the pair is bad,
+  // which the thread that meets the copy's first vector reports
+  auto endpoints = [&](int u) {
+    const int pair = copy[u] >> 1;
+    const int64_t s = __ldg(pairs + 2 * pair);
+    const int64_t d = __ldg(pairs + 2 * pair + 1);
+    if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) {
+      src[u] = nullptr;
+      dst[u] = nullptr;
+      return;
+    }
+    src[u] = ((copy[u] & 1) ? src_v : src_k) + s * vecs_per_block;
+    dst[u] = ((copy[u] & 1) ? dst_v : dst_k) + d * vecs_per_block;
+  };
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    i[u] = u * kCopyThreads + threadIdx.x;
+    const int64_t j = lo + i[u];
+    copy[u] = static_cast<int>(j / vecs_per_block);
+    off[u] = static_cast<int>(j - static_cast<int64_t>(copy[u]) * vecs_per_block);
+    if (i[u] < n) endpoints(u);
   }
-  const uint4* src = (is_v ? src_v : src_k) + s * vecs_per_block;
-  uint4* dst = (is_v ? dst_v : dst_k) + d * vecs_per_block;
-  const int64_t per = (vecs_per_block + ctas_per_copy - 1) / ctas_per_copy;
-  const int64_t lo = piece * per;
-  const int64_t hi = lo + per < vecs_per_block ? lo + per : vecs_per_block;
-  for (int64_t i = lo + threadIdx.x; i < hi; i += kCopyThreads * kUnroll) {
+  while (i[0] < n) {
     uint4 r[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t j = i + u * kCopyThreads;
-      if (j < hi) r[u] = src[j];
-    }
+    for (int u = 0; u < kUnroll; ++u)
+      if (i[u] < n && src[u]) r[u] = src[u][off[u]];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t j = i + u * kCopyThreads;
-      if (j < hi) dst[j] = r[u];
+      if (i[u] < n) {
+        if (dst[u]) {
+          dst[u][off[u]] = r[u];
+        } else if (off[u] == 0 && !(copy[u] & 1)) {
+          set_status(status, -7 /* PA_ERR_BAD_BLOCK */);
+        }
+      }
+      i[u] += kStep;
+      off[u] += kStep;
+      if (off[u] >= vpb) {
+        while (off[u] >= vpb) {
+          off[u] -= vpb;
+          ++copy[u];
+        }
+        if (i[u] < n) endpoints(u);
+      }
     }
   }
 }
@@ -69,9 +104,18 @@ cudaError_t launch_copy_blocks(const void* src_k, const void* src_v, void* dst_k
                                int64_t src_num_blocks, int64_t dst_num_blocks, int32_t* status,
                                cudaStream_t stream) {
   const int64_t vecs = block_bytes / 16;
-  const int ctas_per_copy = static_cast<int>((vecs + kVecsPerCta - 1) / kVecsPerCta);
-  const int64_t grid = static_cast<int64_t>(num_pairs) * 2 * ctas_per_copy;
-  if (grid <= 0 || grid > 0x7fffffff) return cudaErrorInvalidValue;
+  const int64_t total = static_cast<int64_t>(num_pairs) * 2 * vecs;
+  // 32-bit offsets in the kernel: a block under 32 GB, a call under 16 TB
+  if (total <= 0 || vecs >= (int64_t{1} << 31) || total >= (int64_t{1} << 40))
+    return cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaGetLastError();
+  // persistent grid, never more CTAs than there are vectors for each to copy
+  int64_t grid = static_cast<int64_t>(sms) * kCopyCtasPerSm;
+  const int64_t most = (total + kCopyThreads - 1) / kCopyThreads;
+  if (grid > most) grid = most;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kCopyThreads);
@@ -83,8 +127,8 @@ cudaError_t launch_copy_blocks(const void* src_k, const void* src_v, void* dst_k
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(
       &cfg, copy_blocks_kernel, static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v),
-      static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), pairs, vecs, ctas_per_copy,
-      src_num_blocks, dst_num_blocks, status);
+      static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), pairs, vecs, total, src_num_blocks,
+      dst_num_blocks, status);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

@@ -23,6 +23,9 @@ cudaError_t launch_kv_cache_write_fp8(const void* k, const void* v, void* k_cach
 bool encode_swizzled_map(CUtensorMap* map, const void* base, bool bf16, int rank,
                          const uint64_t* dims, const uint64_t* strides_bytes,
                          const uint32_t* box);
+// The same for any element type the driver names (one-byte codes among them).
+bool encode_tiled_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
 
 cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
                                   const int64_t* slot_mapping, int num_tokens, int num_heads,
@@ -54,17 +57,38 @@ struct PrefillArgs {
   int is_bf16;
   int32_t* status;
   int64_t wait_limit_ns = 1000000000;
+  // tcgen05 kernel only.  The paged cache: with cached_lens, prompt s's first
+  // cached_lens[s] tokens are read from it through block_tables (q, k, v and
+  // out then hold the other tokens); with slot_mapping, the prompt tokens'
+  // keys and values are stored in it by the kernel itself.
+  void* k_cache = nullptr;
+  void* v_cache = nullptr;
+  int block_size = 0;
+  int64_t num_blocks = 0;
+  const int32_t* block_tables = nullptr;
+  const int32_t* cached_lens = nullptr;
+  int max_blocks_per_seq = 0;
+  const int64_t* slot_mapping = nullptr;
 };
 // Warp-level tensor cores (mma.sync, prefill.cu) and 5th-generation tensor
 // cores (tcgen05 with TMEM accumulators, prefill_tc.cu).
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
+// Block sizes and pool sizes for which the tcgen05 kernel reads and writes
+// the paged cache itself.
+bool prefill_tc_paged_ok(int block_size, int64_t num_blocks);
 // Current PA_OPT_PREFILL_KERNEL setting (0 automatic = tcgen05, 1 mma.sync, 2 tcgen05).
 int64_t option_prefill_kernel();
 
 // Read-only streaming probe: reads `bytes` (a multiple of 16) of `buf` once;
 // one word per CTA lands in sink[0 .. sink_words).
 cudaError_t launch_read_probe(const void* buf, int64_t bytes, uint32_t* sink, int sink_words,
+                              cudaStream_t stream);
+// Write-only streaming probe: writes `bytes` (a multiple of 16) of `buf`.
+cudaError_t launch_write_probe(void* buf, int64_t bytes, cudaStream_t stream);
+// y = 2^x elementwise: method 0 the FMA-pipe polynomial of the softmax
+// kernels (exp2poly.cuh), 1 the exponential unit (ex2.approx).
+cudaError_t launch_exp2_probe(const float* x, float* y, int64_t n, int method,
                               cudaStream_t stream);
 
 struct DecodeArgs {
@@ -119,6 +143,16 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
 int64_t option_decode_warps();
 // Current PA_OPT_GQA_KERNEL setting (0 automatic, 1 CUDA cores, 2 tensor cores).
 int64_t option_gqa_kernel();
+// Current PA_OPT_FP8_KERNEL setting (0 automatic, 1 CUDA cores, 2 tensor cores).
+int64_t option_fp8_kernel();
+
+// Tensor-core decode over an 8-bit cache (paged_attn_decode_mma_fp8.cu):
+// fp16 queries, head_dim 128, multi-head, blocks of 8, 16 or 32, a pool that
+// fits 32-bit TMA row coordinates.
+bool mma_fp8_decode_ok(const DecodeArgs& a);
+size_t mma_fp8_workspace_bytes(int num_seqs, int num_heads, int block_size,
+                               int max_blocks_per_seq, int64_t forced_warps);
+cudaError_t launch_paged_attn_decode_mma_fp8(const DecodeArgs& a, cudaStream_t stream);
 
 // Tensor-core grouped-query decode (paged_attn_decode_mma.cu): whether the
 // head layout and block size suit it, whether the pool fits its 32-bit TMA

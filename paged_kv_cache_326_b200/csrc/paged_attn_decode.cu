@@ -703,6 +703,14 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
   const int64_t segs = static_cast<int64_t>(num_seqs) * hl.vheads;
   size_t bytes =
       header_bytes(num_seqs) + kGrabBytes + records_bytes(max_units(warps) + segs, head_dim, hl.gs);
+  // The 8-bit cache may run on the tensor-core kernel: size for it too.
+  if (with_fp8 && hl.gs == 1 && head_dim == 128 &&
+      (block_size == 8 || block_size == 16 || block_size == 32)) {
+    const size_t f8 = mma_fp8_workspace_bytes(num_seqs, num_heads, block_size,
+                                              max_blocks_per_seq, forced_warps);
+    if (f8 == 0) return 0;
+    if (f8 > bytes) bytes = f8;
+  }
   // Grouped-query shapes may run on either kernel: size for both.
   if (mma_decode_shape_ok(num_heads, num_kv_heads, head_dim, block_size)) {
     const size_t mma = mma_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
@@ -717,6 +725,14 @@ cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (!decode_sizes_supported(a.num_seqs, a.num_heads, a.num_kv_heads, a.head_dim, a.block_size,
                               a.max_blocks_per_seq))
     return cudaErrorInvalidValue;
+  // 8-bit cache: tensor cores unless PA_OPT_FP8_KERNEL asks for the CUDA
+  // cores (or the query type, shape or pool does not suit them).
+  if (a.fp8) {
+    const int64_t f8mode = option_fp8_kernel();
+    const bool f8_ok = mma_fp8_decode_ok(a);
+    if (f8mode == 2 && !f8_ok) return cudaErrorInvalidValue;
+    if (f8_ok && f8mode != 1) return launch_paged_attn_decode_mma_fp8(a, stream);
+  }
   // Grouped-query attention: tensor cores unless PA_OPT_GQA_KERNEL asks for
   // the CUDA cores (or the shape or pool does not suit them).
   const int64_t mode = option_gqa_kernel();

@@ -4,14 +4,26 @@
 // PagedAttention", section "One Token at a Time"; "KV cache", section "How it
 // works"): for prompt s, query head h and position t,
 //     out[t][h] = sum_{u <= t} softmax_u(scale * q[t][h] . k[u]) v[u],
-// query head h reading key/value head h / (Hq / Hkv).
+// query head h reading key/value head h / (Hq / Hkv).  With a stored prefix
+// (section "What Came After": a prompt that begins like an earlier one reuses
+// the earlier one's blocks and skips their compute), prompt s's first
+// cached_lens[s] tokens are not in q, k, v: their keys and values are read
+// from the paged cache through block_tables[s], and the new rows are the
+// positions after them.
 //
 // How (FlashAttention-4's arrangement on sm_100a): one CTA takes two tiles of
 // 128 queries of one (prompt, head), 256 consecutive queries, and runs ten
 // warps with separate jobs:
-//   * warp 9 (one thread) loads: Q of both tiles once, then each 64-key block
-//     of K and V into a 3-stage ring, by 3-D tiled TMA (the [T][H][D] tensors
-//     seen as (D, H, T); boxes 64 x 1 x rows; 128-byte swizzle);
+//   * warp 9 loads: Q of both tiles once, then each 64-key block of K and V
+//     into a 3-stage ring, by tiled TMA with the 128-byte swizzle: the new
+//     tokens from q, k, v (the [T][H][D] tensors seen as (D, H, T); boxes
+//     64 x 1 x rows), the stored prefix from the cache pools (seen as
+//     (D, B, H, N); one box of 64 x B rows per physical block, found in the
+//     block table).  The CTA that holds a key block's own queries also
+//     stores that block of the new keys and values in the cache: TMA stores
+//     of the tiles already in shared memory, one box per physical block, when
+//     the block's slots fill whole physical blocks in order (the usual case),
+//     else row by row from the warp's lanes;
 //   * warp 8 (one thread) issues the tensor-core products, tcgen05.mma
 //     kind::f16, accumulating in tensor memory (TMEM): S_t = Q_t K^T (both
 //     operands K-major in shared memory) and O_t += P_t V (P_t from TMEM, V
@@ -22,8 +34,12 @@
 //     query row (its warp's 32 TMEM lanes), so the row max and sum stay in
 //     the thread.  Base 2; the running max is raised only when a score
 //     passes it by more than 2^8, which then rescales that row of O in TMEM.
-//     P (and for bf16 the rest P - P_hi, so P enters as about 16 significant
-//     bits) goes back to TMEM as packed 16-bit pairs.
+//     Two scores per packed fp32 instruction, maxima three at a time; in
+//     blocks with no masked score half of the weights come from an FMA-pipe
+//     polynomial (exp2poly.cuh) and half from the exponential unit, which
+//     alone would take as long as the products.  P (and for bf16 the rest
+//     P - P_hi, so P enters as about 16 significant bits) goes back to TMEM
+//     as packed 16-bit pairs.
 //   * After its last block each softmax thread divides its row of O by its
 //     sum and stores it.
 // Barriers: per stage full (TMA bytes) and empty (last product that reads
@@ -42,6 +58,7 @@
 #include <type_traits>
 
 #include "dtype.cuh"
+#include "exp2poly.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tcgen05.cuh"
@@ -59,6 +76,20 @@ constexpr int kMmaWarp = 8, kLoadWarp = 9;
 constexpr uint32_t kColS = 0, kColPhi = 64, kColPlo = 96, kColO = 128;
 constexpr uint32_t kTileCols = 256, kTmemCols = 512;
 constexpr int64_t kTcDrainNs = 1000000000;
+#ifndef PA_TC_POLY_PAIRS
+#define PA_TC_POLY_PAIRS 2
+#endif
+// Of every four pairs of softmax weights in a block below the diagonal, this
+// many are computed by the FMA-pipe polynomial (exp2poly.cuh), the rest by
+// the exponential unit.
+constexpr int kTcPolyPairs = PA_TC_POLY_PAIRS;
+
+// max(a, b, c) in one instruction (three-input max.f32 of sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
 template <int D>
 struct TcLayout {
@@ -81,12 +112,24 @@ struct TcParams {
   float scale_log2;
   int32_t* status;
   int64_t wait_limit_ns;
+  // The paged cache (block size B, num_blocks blocks): a stored prefix is
+  // read from it through block_tables / cached_lens (null: none), and the new
+  // tokens' keys and values are written to it at slot_mapping (null: not).
+  int B;
+  int64_t num_blocks;
+  const int32_t* block_tables;
+  const int32_t* cached_lens;
+  int max_blocks;
+  const int64_t* slot_mapping;
+  void* k_cache;
+  void* v_cache;
 };
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
 prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc) {
   using LY = TcLayout<D>;
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t IDESC_S = tc::idesc_f16(kTcBM, kTcBN, BF16, false);
@@ -108,21 +151,29 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
     return;
   }
-  const int L = b - a;
+  const int L = b - a;  // new tokens of this prompt
   if (L > p.max_seqlen && blockIdx.x == 0 && h == 0 && threadIdx.x == 0)
     set_status(p.status, -8 /* PA_ERR_BAD_LEN: a prompt longer than max_seqlen */);
+  // stored prefix: a whole number of blocks that the table holds
+  const int cl = p.cached_lens ? __ldg(p.cached_lens + s) : 0;
+  if (cl < 0 || cl % p.B || cl > p.max_blocks * p.B) {
+    if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
+    return;
+  }
+  const int npre = (cl + kTcBN - 1) / kTcBN;        // key blocks of the stored prefix
   const int pair = gridDim.x - 1 - blockIdx.x;       // heaviest pairs of tiles first
-  const int q0 = pair * kTcTiles * kTcBM;            // first query of tile 0
+  const int q0 = pair * kTcTiles * kTcBM;            // first new row of tile 0
   if (q0 >= L) return;                               // the whole CTA leaves: nothing allocated
   const int kvh = h / (p.Hq / p.Hkv);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // key blocks each tile needs (keys up to its last query); tile 1 may be empty
+  // key blocks each tile needs: the prefix's, then the new keys up to its
+  // last row; tile 1 may be empty
   int nkb_t[kTcTiles];
 #pragma unroll
   for (int t = 0; t < kTcTiles; ++t) {
     const int lo = q0 + t * kTcBM;
     const int hi = min(L, lo + kTcBM);
-    nkb_t[t] = lo < L ? (hi + kTcBN - 1) / kTcBN : 0;
+    nkb_t[t] = lo < L ? npre + (hi + kTcBN - 1) / kTcBN : 0;
   }
   const int nkb = nkb_t[kTcTiles - 1] > 0 ? nkb_t[kTcTiles - 1] : nkb_t[0];
 
@@ -163,11 +214,15 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   };
 
   if (warp == kLoadWarp) {
-    // ---------------- loads ----------------
+    // ---------------- loads (lane 0) and stores of the new keys ----------------
     if (lane == 0) {
       tc::prefetch_map(&tm_q);
       tc::prefetch_map(&tm_k);
       tc::prefetch_map(&tm_v);
+      if (p.cached_lens || p.slot_mapping) {
+        tc::prefetch_map(&tm_kc);
+        tc::prefetch_map(&tm_vc);
+      }
       const int nq = nkb_t[1] > 0 ? 2 : 1;
       mbar_arrive_expect_tx(&bar_q, nq * LY::Q_BYTES);
       for (int t = 0; t < nq; ++t)
@@ -175,12 +230,39 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
         for (int hf = 0; hf < LY::HALVES; ++hf)
           tc::tma_load_3d(sQ + t * LY::Q_BYTES + hf * (kTcBM * 128), &tm_q, hf * 64, h,
                           a + q0 + t * kTcBM, &bar_q);
-      int issued = 0;
-      for (int j = 0; j < nkb; ++j) {
-        const int st = j % kTcStages;
-        if (j >= kTcStages && !wait(&bar_empty[st], ((j / kTcStages) - 1) & 1)) break;
-        uint8_t* dst = sKV + st * LY::STAGE;
-        mbar_arrive_expect_tx(&bar_full[st], LY::STAGE);
+    }
+    // Key block jj: the stored prefix's block jj (jj < npre), else block
+    // jj - npre of the new keys.
+    const int32_t* table = p.cached_lens ? p.block_tables + static_cast<int64_t>(s) * p.max_blocks
+                                         : nullptr;
+    auto load_block = [&](int jj, int st) {  // lane 0
+      uint8_t* dst = sKV + st * LY::STAGE;
+      mbar_arrive_expect_tx(&bar_full[st], LY::STAGE);
+      if (jj < npre) {
+        // one box of B rows per physical block; rows past the prefix (and bad
+        // table entries) are read from block num_blocks, outside the pool:
+        // zeros, so their scores are finite and their values add nothing
+        for (int r0 = 0; r0 < kTcBN; r0 += p.B) {
+          const int pos = jj * kTcBN + r0;
+          int blk = static_cast<int>(p.num_blocks);
+          if (pos < cl) {
+            const int e = __ldg(table + pos / p.B);
+            if (e >= 0 && e < p.num_blocks) {
+              blk = e;
+            } else {
+              set_status(p.status, -7 /* PA_ERR_BAD_BLOCK */);
+            }
+          }
+#pragma unroll
+          for (int hf = 0; hf < LY::HALVES; ++hf) {
+            tc::tma_load_4d(dst + hf * (kTcBN * 128) + r0 * 128, &tm_kc, hf * 64, 0, kvh, blk,
+                            &bar_full[st]);
+            tc::tma_load_4d(dst + LY::KV_BYTES + hf * (kTcBN * 128) + r0 * 128, &tm_vc, hf * 64,
+                            0, kvh, blk, &bar_full[st]);
+          }
+        }
+      } else {
+        const int j = jj - npre;
 #pragma unroll
         for (int hf = 0; hf < LY::HALVES; ++hf) {
           tc::tma_load_3d(dst + hf * (kTcBN * 128), &tm_k, hf * 64, kvh, a + j * kTcBN,
@@ -188,9 +270,92 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
           tc::tma_load_3d(dst + LY::KV_BYTES + hf * (kTcBN * 128), &tm_v, hf * 64, kvh,
                           a + j * kTcBN, &bar_full[st]);
         }
-        issued = j + 1;
       }
-      // drain: the copies in flight must land before this CTA's memory goes
+    };
+    // The new keys' blocks whose rows are this CTA's own queries go to the
+    // cache from here (one query head per key/value head stores them).
+    const bool stores = p.slot_mapping && h % (p.Hq / p.Hkv) == 0;
+    const int own_lo = npre + q0 / kTcBN;
+    const int64_t num_slots = p.num_blocks * p.B;
+    // a wait whose outcome the whole warp shares (the stores use warp votes)
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return !__any_sync(0xffffffffu, !wait(bar, parity));
+    };
+    auto store_block = [&](int jj) -> bool {  // whole warp; block jj's data has landed
+      const int st = jj % kTcStages;
+      if (!wwait(&bar_full[st], (jj / kTcStages) & 1)) return false;
+      const uint8_t* sK = sKV + st * LY::STAGE;
+      const uint8_t* sV = sK + LY::KV_BYTES;
+      const int j = jj - npre;
+      bool plain = false;
+      for (int r0 = 0; r0 < kTcBN; r0 += p.B) {
+        // lane r < B takes row r0 + r of the block: new token j*64 + r0 + r
+        const int pos = j * kTcBN + r0 + lane;
+        int64_t slot = -2;  // no token
+        if (lane < p.B && pos < L) slot = __ldg(p.slot_mapping + a + pos);
+        const int64_t s0 = __shfl_sync(0xffffffffu, slot, 0);
+        const bool in_order = lane >= p.B || slot == s0 + lane;
+        if (__all_sync(0xffffffffu, in_order) && s0 >= 0 && s0 % p.B == 0 &&
+            s0 + p.B <= num_slots) {
+          // the B rows fill physical block s0 / B in order: one box per half
+          if (lane == 0) {
+            const int blk = static_cast<int>(s0 / p.B);
+#pragma unroll
+            for (int hf = 0; hf < LY::HALVES; ++hf) {
+              tc::tma_store_4d(&tm_kc, sK + hf * (kTcBN * 128) + r0 * 128, hf * 64, 0, kvh, blk);
+              tc::tma_store_4d(&tm_vc, sV + hf * (kTcBN * 128) + r0 * 128, hf * 64, 0, kvh, blk);
+            }
+            tc::bulk_commit();
+          }
+        } else if (lane < p.B && slot >= num_slots) {
+          set_status(p.status, -9 /* PA_ERR_BAD_SLOT */);
+        } else if (lane < p.B && slot >= 0) {
+          // row by row: undo the swizzle (16-byte piece c of row r sits at
+          // piece c ^ (r % 8)) and write the row at its slot
+          const int r = r0 + lane;
+          const int64_t row = ((slot / p.B) * p.Hkv + kvh) * p.B + slot % p.B;
+          uint4* dk = reinterpret_cast<uint4*>(static_cast<T*>(p.k_cache) + row * D);
+          uint4* dv = reinterpret_cast<uint4*>(static_cast<T*>(p.v_cache) + row * D);
+#pragma unroll
+          for (int hf = 0; hf < LY::HALVES; ++hf)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int off = hf * (kTcBN * 128) + r * 128 + ((c ^ (r & 7)) << 4);
+              dk[hf * 8 + c] = *reinterpret_cast<const uint4*>(sK + off);
+              dv[hf * 8 + c] = *reinterpret_cast<const uint4*>(sV + off);
+            }
+          plain = true;
+        }
+      }
+      // generic reads of the stage before the next TMA load writes it
+      if (plain) fence_proxy_async_smem();
+      __syncwarp();
+      return true;
+    };
+    int issued = 0, stored = own_lo;
+    bool ok = true;
+    for (int jj = 0; jj < nkb; ++jj) {
+      const int st = jj % kTcStages;
+      if (jj >= kTcStages) {
+        if (!wwait(&bar_empty[st], ((jj / kTcStages) - 1) & 1)) break;
+        // the stage still holds block jj - kTcStages: store it if it is ours,
+        // and let the stores finish reading it before it is refilled
+        if (stores && jj - kTcStages >= own_lo) {
+          if (!(ok = store_block(jj - kTcStages))) break;
+          stored = jj - kTcStages + 1;
+          if (lane == 0) tc::bulk_wait_read_all();
+          __syncwarp();
+        }
+      }
+      if (lane == 0) load_block(jj, st);
+      issued = jj + 1;
+    }
+    // our blocks still in the ring
+    for (int jj = stored; stores && ok && jj < issued; ++jj) ok = store_block(jj);
+    if (lane == 0) {
+      // drain: the stores must complete, and the copies in flight land,
+      // before this CTA's memory goes
+      tc::bulk_wait_all();
       mbar_wait_bounded(&bar_q, 0, kTcDrainNs);
       for (int j = issued > kTcStages ? issued - kTcStages : 0; j < issued; ++j)
         mbar_wait_bounded(&bar_full[j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
@@ -259,14 +424,14 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     // ---------------- softmax of one query row ----------------
     const int t = warp >> 2;                     // tile of this warpgroup
     const int row = tid & (kTcBM - 1);           // row within the tile = TMEM lane
-    const int qpos = q0 + t * kTcBM + row;       // query position within the prompt
+    const int qpos = q0 + t * kTcBM + row;       // new row within the prompt (position cl + qpos)
     const uint32_t rbase = tmem + t * kTileCols + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     float m = -INFINITY, l = 0.f;
     bool failed = false;
     const int nk = nkb_t[t];
-    for (int j = 0; j < nk; ++j) {
+    for (int jj = 0; jj < nk; ++jj) {
       // tcgen05.ld/st are warp-collective: guards around them are warp-uniform
-      failed = __any_sync(0xffffffffu, failed || !wait(&bar_s[t], j & 1));
+      failed = __any_sync(0xffffffffu, failed || !wait(&bar_s[t], jj & 1));
       if (failed) break;
       tc::fence_after_sync();
       float sv[kTcBN];
@@ -281,28 +446,47 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int c = 0; c < 16; ++c) sv[i * 16 + c] = __uint_as_float(v[i][c]);
       }
-      // keys past this query exist only in the diagonal blocks
-      if (j * kTcBN + kTcBN - 1 > qpos) {
+      // `below`: no score of this warp's rows is masked in this block, so part
+      // of the weights may come from the polynomial
+      bool below;
+      if (jj < npre) {
+        // stored prefix: its keys precede every new row; the last block may
+        // run past the prefix (rows read as zeros), which is masked
+        below = jj * kTcBN + kTcBN <= cl;
+        if (!below) {
 #pragma unroll
-        for (int c = 0; c < kTcBN; ++c)
-          if (j * kTcBN + c > qpos) sv[c] = -INFINITY;
+          for (int c = 0; c < kTcBN; ++c)
+            if (jj * kTcBN + c >= cl) sv[c] = -INFINITY;
+        }
+      } else {
+        // new keys: those past this row exist only in the diagonal blocks
+        const int j = jj - npre;
+        if (j * kTcBN + kTcBN - 1 > qpos) {
+#pragma unroll
+          for (int c = 0; c < kTcBN; ++c)
+            if (j * kTcBN + c > qpos) sv[c] = -INFINITY;
+        }
+        below = j * kTcBN + kTcBN - 1 <= q0 + t * kTcBM + (warp & 3) * 32;
       }
-      // four independent partial maxima: no 64-long dependent chain
+      // four independent partial maxima of three-input maxima
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kTcBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+      for (int c = 0; c < kTcBN; c += 8) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
+      }
       // base-2 logits: the scale (> 0) is applied in the exponent
       const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
       // P_t and O_t are in use by the previous block's product until it is done
-      if (j > 0) {
-        failed = __any_sync(0xffffffffu, !wait(&bar_o[t], (j - 1) & 1));
+      if (jj > 0) {
+        failed = __any_sync(0xffffffffu, !wait(&bar_o[t], (jj - 1) & 1));
         if (failed) break;
         tc::fence_after_sync();
       }
       const bool raise = rmax > m + 8.f;
       const float m_new = raise ? rmax : m;
       const float alpha = raise && m != -INFINITY ? fast_exp2(m - m_new) : 1.f;
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 64) {
           uint32_t v[4][16];
@@ -322,20 +506,31 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       m = m_new;
       const float mm = m == -INFINITY ? 0.f : m;
       uint32_t ph[32], pl[32];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
-#pragma unroll
-      for (int c = 0; c < kTcBN; c += 2) {
-        // 2^(scale * s - m): one fma per score (masked scores are -inf: weight 0)
-        const float p0 = fast_exp2(fmaf(sv[c], p.scale_log2, -mm));
-        const float p1 = fast_exp2(fmaf(sv[c + 1], p.scale_log2, -mm));
-        ls[(c >> 1) & 3] += p0 + p1;
-        ph[c / 2] = Elem<T>::from_float2(p0, p1);
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // partial sums
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nm2 = make_float2(-mm, -mm);
+      // 2^(scale * s - m), two scores per packed fma (masked scores are -inf:
+      // weight 0).  Below the diagonal, kTcPolyPairs of every four pairs of
+      // weights come from the FMA-pipe polynomial and the rest from the
+      // exponential unit, so the two units share the work.
+      auto weights = [&](int c, bool poly) {
+        const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sc2, nm2);
+        const float2 pw = poly ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        ls[(c >> 1) & 1] = __fadd2_rn(ls[(c >> 1) & 1], pw);
+        ph[c / 2] = Elem<T>::from_float2(pw.x, pw.y);
         if constexpr (BF16) {
           const float2 back = Elem<T>::to_float2(ph[c / 2]);
-          pl[c / 2] = Elem<T>::from_float2(p0 - back.x, p1 - back.y);
+          pl[c / 2] = Elem<T>::from_float2(pw.x - back.x, pw.y - back.y);
         }
+      };
+      if (below) {
+#pragma unroll
+        for (int c = 0; c < kTcBN; c += 2) weights(c, ((c >> 1) & 3) >= 4 - kTcPolyPairs);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kTcBN; c += 2) weights(c, false);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
       tc::st16(rbase + kColPhi, *reinterpret_cast<uint32_t(*)[16]>(ph));
       tc::st16(rbase + kColPhi + 16, *reinterpret_cast<uint32_t(*)[16]>(ph + 16));
       if constexpr (BF16) {
@@ -415,6 +610,22 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
       !encode_swizzled_map(&tk, a.k, bf16, 3, dk, sk, bk) ||
       !encode_swizzled_map(&tv, a.v, bf16, 3, dk, sk, bk))
     return cudaErrorInvalidValue;
+  // the cache pools [N][Hkv][B][D] as (D, B, Hkv, N); one physical block of
+  // one head per box of 64 x B (only when the kernel reads or writes them)
+  CUtensorMap tkc = tk, tvc = tv;
+  const bool paged = a.cached_lens || a.slot_mapping;
+  if (paged) {
+    const uint64_t dc[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.block_size),
+                            static_cast<uint64_t>(a.num_kv_heads),
+                            static_cast<uint64_t>(a.num_blocks)};
+    const uint64_t sc[3] = {static_cast<uint64_t>(D) * 2,
+                            static_cast<uint64_t>(a.block_size) * D * 2,
+                            static_cast<uint64_t>(a.num_kv_heads) * a.block_size * D * 2};
+    const uint32_t bc[4] = {64u, static_cast<uint32_t>(a.block_size), 1u, 1u};
+    if (!encode_swizzled_map(&tkc, a.k_cache, bf16, 4, dc, sc, bc) ||
+        !encode_swizzled_map(&tvc, a.v_cache, bf16, 4, dc, sc, bc))
+      return cudaErrorInvalidValue;
+  }
   TcParams p;
   p.out = a.out;
   p.cu_seqlens = a.cu_seqlens;
@@ -425,6 +636,14 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.B = paged ? a.block_size : 1;
+  p.num_blocks = a.num_blocks;
+  p.block_tables = a.block_tables;
+  p.cached_lens = a.cached_lens;
+  p.max_blocks = a.max_blocks_per_seq;
+  p.slot_mapping = a.slot_mapping;
+  p.k_cache = a.k_cache;
+  p.v_cache = a.v_cache;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles, a.num_heads, a.num_seqs);
   cfg.blockDim = dim3(kTcThreads);
@@ -435,14 +654,26 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<T, D>, p, tq, tk, tv);
+  cudaError_t err = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<T, D>, p, tq, tk, tv, tkc, tvc);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
 }  // namespace
 
+bool prefill_tc_paged_ok(int block_size, int64_t num_blocks) {
+  // boxes of B rows start on 1024-byte boundaries of the swizzled tiles;
+  // block indices (num_blocks itself reads as zeros) fit the 32-bit
+  // coordinates of the tensor map
+  return (block_size == 8 || block_size == 16 || block_size == 32) && num_blocks > 0 &&
+         num_blocks < (int64_t{1} << 31) - 1;
+}
+
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
+  if ((a.cached_lens || a.slot_mapping) &&
+      (!a.k_cache || !a.v_cache || !prefill_tc_paged_ok(a.block_size, a.num_blocks) ||
+       (a.cached_lens && (!a.block_tables || a.max_blocks_per_seq < 1))))
+    return cudaErrorInvalidValue;
   if (a.head_dim == 128)
     return a.is_bf16 ? launch_prefill_tc_typed<__nv_bfloat16, 128>(a, stream)
                      : launch_prefill_tc_typed<__half, 128>(a, stream);

@@ -2,7 +2,8 @@
 // sm_100a: tensor-memory (TMEM) allocation, the single-thread MMA with
 // operands in shared memory (SS) or A in TMEM (TS), completion through an
 // mbarrier, TMEM loads and stores, and the ordering fences; plus the shared-
-// memory matrix descriptors and the instruction descriptor of kind::f16.
+// memory matrix descriptors and the instruction descriptor of kind::f16; and
+// the 3-D and 4-D tiled TMA loads and 4-D stores of the prompt-phase kernel.
 // 1-CTA forms only; no multicast.
 #pragma once
 #include <cstdint>
@@ -122,6 +123,41 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, i
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
       : "memory");
+}
+
+// 4-D tiled TMA load (no multicast) into shared memory, counted on `bar`.
+// Coordinates outside the tensor read as zeros.
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// 4-D tiled TMA store of a shared-memory box to global memory (the box's
+// swizzle undone by the map), tracked by this thread's bulk async-groups.
+__device__ __forceinline__ void tma_store_4d(const void* map, const void* src, int x, int y, int z,
+                                             int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(src))
+      : "memory");
+}
+
+// Close the current bulk async-group of this thread.
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's bulk stores have finished reading shared memory ...
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... or have completed their global writes.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 }  // namespace tc

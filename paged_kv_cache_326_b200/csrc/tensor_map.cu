@@ -1,4 +1,5 @@
-// Tiled TMA tensor maps of 16-bit tensors with the 128-byte swizzle, encoded
+// Tiled TMA tensor maps with the 128-byte swizzle (16-bit tensors, and the
+// 8-bit cache's one-byte codes), encoded
 // through the driver's cuTensorMapEncodeTiled, which is looked up once
 // through the runtime (the library does not link the driver library).
 #include <cuda.h>
@@ -35,6 +36,13 @@ EncodeTiledFn encode_tiled() {
 bool encode_swizzled_map(CUtensorMap* map, const void* base, bool bf16, int rank,
                          const uint64_t* dims, const uint64_t* strides_bytes,
                          const uint32_t* box) {
+  return encode_tiled_map(map, base,
+                          bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                          rank, dims, strides_bytes, box);
+}
+
+bool encode_tiled_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   const EncodeTiledFn fn = encode_tiled();
   if (!fn || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], st[4];
@@ -45,8 +53,7 @@ bool encode_swizzled_map(CUtensorMap* map, const void* base, bool bf16, int rank
     e[i] = 1u;
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
-  return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-            static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, b, e,
+  return fn(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, b, e,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

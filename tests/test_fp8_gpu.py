@@ -22,6 +22,16 @@ def lib():
     return P.lib()
 
 
+@pytest.fixture(params=[1, 0], ids=["cuda_cores", "auto"])
+def fp8_kernel(request):
+    """PA_OPT_FP8_KERNEL: 1 the CUDA-core kernel everywhere; 0 the default
+    (tensor cores for fp16 queries, head_dim 128, blocks of 8-32)."""
+    import paged_kv_cache_326_b200 as P
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, request.param)
+    yield request.param
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
+
+
 def parity_fp8(w, seqs=None, heads_per_seq=None, seed=0):
     S, H, D = w.q.shape
     seqs = np.arange(S) if seqs is None else np.asarray(seqs)
@@ -57,7 +67,7 @@ def parity_fp8(w, seqs=None, heads_per_seq=None, seed=0):
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
 @pytest.mark.parametrize("head_dim", [64, 128])
 @pytest.mark.parametrize("block_size", [4, 8, 16, 32])
-def test_fp8_every_shape_ragged(dtype, head_dim, block_size):
+def test_fp8_every_shape_ragged(dtype, head_dim, block_size, fp8_kernel):
     w = W.make_decode_fp8("fp8_shape", SHAPE_LENS, num_heads=3, head_dim=head_dim,
                           block_size=block_size,
                           num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in SHAPE_LENS),
@@ -66,10 +76,46 @@ def test_fp8_every_shape_ragged(dtype, head_dim, block_size):
     parity_fp8(w)
 
 
-def test_fp8_opt13b_batch64():
+def test_fp8_opt13b_batch64(fp8_kernel):
     w = W.opt13b_batch64_fp8(device="cuda")
     c = parity_fp8(w, heads_per_seq=6, seed=3)
-    print("fp8 opt13b", c)
+    print("fp8 opt13b", fp8_kernel, c)
+
+
+def test_fp8_tensor_cores_all_outputs_of_a_large_batch():
+    """The tensor-core kernel forced on 24 texts of the batch-64 shapes
+    (lengths 128..2048), every head against the oracle."""
+    import paged_kv_cache_326_b200 as P
+    lens = W.opt13b_batch64_lens()[:24]
+    need = sum(W.blocks_needed(L, 16) for L in lens)
+    w = W.make_decode_fp8("fp8_first24", lens, num_heads=40, head_dim=128, block_size=16,
+                          num_blocks=(3 * need + 1) // 2, dtype=torch.float16, seed=12,
+                          device="cuda", max_blocks_per_seq=128)
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, 2)
+    try:
+        c = parity_fp8(w)
+    finally:
+        P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
+    print("fp8 tensor cores, 24 texts", c)
+
+
+def test_fp8_tensor_cores_refuse_what_they_do_not_cover():
+    """Forcing the tensor-core kernel where it does not apply (bf16 queries,
+    head_dim 64, blocks of 4) is an argument error, not a silent fallback."""
+    import paged_kv_cache_326_b200 as P
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, 2)
+    try:
+        for dtype, D, B in ((torch.bfloat16, 128, 16), (torch.float16, 64, 16),
+                            (torch.float16, 128, 4)):
+            w = W.make_decode_fp8("fp8_refuse", [5, 40], num_heads=2, head_dim=D, block_size=B,
+                                  num_blocks=32, dtype=dtype, seed=1, device="cuda",
+                                  max_blocks_per_seq=64 // B)
+            with pytest.raises(P.PagedAttnError):
+                P.pa_paged_attn_decode_fp8(torch.empty_like(w.q), w.q, w.k_cache, w.v_cache,
+                                           w.block_tables, w.context_lens, w.scale,
+                                           w.meta["k_scale"], w.meta["v_scale"])
+    finally:
+        P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
 
 
 def test_fp8_write_rounds_saturates_and_keeps_signs():
@@ -96,7 +142,7 @@ def test_fp8_write_rounds_saturates_and_keeps_signs():
     assert np.array_equal(kd.cpu().numpy(), ek) and np.array_equal(vd.cpu().numpy(), ev)
 
 
-def test_fp8_single_token_returns_its_value():
+def test_fp8_single_token_returns_its_value(fp8_kernel):
     """One stored token: the output is value(code) * v_scale rounded to the
     output type, bit for bit."""
     w = W.make_decode_fp8("fp8_one", [1] * 6, num_heads=5, head_dim=128, block_size=16,
@@ -110,14 +156,15 @@ def test_fp8_single_token_returns_its_value():
     assert torch.equal(out.cpu(), want)
 
 
-def test_fp8_split_and_single_pass_agree():
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+def test_fp8_split_and_single_pass_agree(dtype, fp8_kernel):
     import paged_kv_cache_326_b200 as P
     for warps in (1, 4096):
         P.pa_set_option(P.binding.PA_OPT_DECODE_WARPS, warps)
         try:
             parity_fp8(W.make_decode_fp8("fp8_split", [300, 17, 1, 1000, 64, 0, 511, 129],
                                          num_heads=4, head_dim=128, block_size=16,
-                                         num_blocks=256, dtype=torch.bfloat16, seed=9,
+                                         num_blocks=256, dtype=dtype, seed=9,
                                          device="cuda", max_blocks_per_seq=64))
         finally:
             P.pa_set_option(P.binding.PA_OPT_DECODE_WARPS, 0)

@@ -109,12 +109,13 @@ def test_shared_prefix_through_block_manager():
 
 @pytest.mark.slow
 def test_full_step_40_layers():
-    """40 layers x (write + attend) over one shared pool; the oracle replays
-    every layer's writes and checks sampled texts and heads of 3 layers."""
+    """40 layers x (write + attend) over one shared pool (blocks alias across
+    layers); the oracle replays every layer's writes and checks every head of
+    6 sampled texts on 5 layers."""
     import paged_kv_cache_326_b200 as P
     fs = W.full_step(device="cuda")
     B = fs.block_size
-    check_layers = [0, 21, 39]
+    check_layers = [0, 9, 21, 30, 39]
     rng = np.random.default_rng(5)
     seqs = np.sort(rng.choice(fs.context_lens.numel(), 6, replace=False))
     sel = torch.as_tensor(seqs, device="cuda")
@@ -159,8 +160,7 @@ def test_full_step_40_layers():
         t = torch.where(t >= 0, remap[t.clamp(min=0)], torch.full_like(t, -1)).cpu().numpy()
         assert (t[t >= 0] >= 0).all()
         q = fs.q[layer].index_select(0, sel).float().cpu().numpy()
-        heads = rng.choice(H, 5, replace=False)
-        pairs = [(i, int(h)) for i in range(len(seqs)) for h in heads]
+        pairs = [(i, h) for i in range(len(seqs)) for h in range(H)]
         ref = oracle.paged_decode(q, kc, vc, t, fs.context_lens.index_select(0, sel).cpu().numpy(),
                                   fs.scale, B, pairs)
         mask = np.zeros(ref.shape, dtype=bool)

@@ -16,10 +16,14 @@ from oracle import BlockManagerError, BlockManagerModel
 class Cpp:
     """The C++ manager through the binding, with the model's interface."""
 
-    def __init__(self, n, b):
+    def __init__(self, n, b, key_bits=64):
         import paged_kv_cache_326_b200 as P
         self.P = P
-        self.bm = P.BlockManager(n, b)
+        P.pa_set_option(P.PA_OPT_PREFIX_KEY_BITS, key_bits)
+        try:
+            self.bm = P.BlockManager(n, b)
+        finally:
+            P.pa_set_option(P.PA_OPT_PREFIX_KEY_BITS, 64)
         self.block_size = b
 
     def _run(self, fn, *a):
@@ -144,10 +148,55 @@ def pin_out_of_blocks_changes_nothing(make):
     assert bm.add_seq_tokens(2, list(range(8)) + [1, 2]) == 8            # 1 fresh fits
 
 
+def _key(tokens, B, bits):
+    """Lookup key of the last full block of `tokens` with `bits` key bits
+    (test set-up only: used to find prompts whose keys meet)."""
+    from oracle.block_manager import block_hash
+    h = 0
+    for j in range(len(tokens) // B):
+        h = block_hash(h, tokens[j * B:(j + 1) * B])
+    return h & ((1 << bits) - 1)
+
+
+def pin_equal_keys_of_different_blocks_share_nothing(make):
+    """With 4 key bits, two different one-block prompts whose keys meet: the
+    second takes over nothing, and its block is not cached (the key stays
+    with the first block)."""
+    bits, B = 4, 4
+    a = [1, 2, 3, 4]
+    b = next([5, 6, 7, t] for t in range(1000) if _key([5, 6, 7, t], B, bits) == _key(a, B, bits))
+    bm = make(8, B, key_bits=bits)
+    assert bm.add_seq_tokens(1, a) == 0
+    assert bm.add_seq_tokens(2, b) == 0
+    tables, _ = bm.export([1, 2], 1)
+    assert tables[0] != tables[1]
+    assert bm.num_cached_blocks() == 1
+    assert bm.add_seq_tokens(3, a + [9]) == 4                      # the first still hits
+
+
+def pin_equal_last_blocks_after_different_prefixes_share_nothing(make):
+    """With 4 key bits: text 1 is [P, X], text 2 is [Q] alone (so Q's block is
+    cached), text 3 is [Q, X] where the keys of [P, X] and [Q, X] meet.  Text 3
+    takes over Q's block, but not text 1's X block, although the key and X's
+    own token ids agree: the whole prefix before X differs."""
+    bits, B = 4, 4
+    P_, X = [1, 2, 3, 4], [7, 7, 7, 7]
+    Q = next([9, 9, 9, t] for t in range(1000)
+             if _key([9, 9, 9, t], B, bits) not in (_key(P_, B, bits), _key(P_ + X, B, bits))
+             and _key([9, 9, 9, t] + X, B, bits) == _key(P_ + X, B, bits))
+    bm = make(8, B, key_bits=bits)
+    assert bm.add_seq_tokens(1, P_ + X) == 0
+    assert bm.add_seq_tokens(2, Q) == 0
+    assert bm.add_seq_tokens(3, Q + X) == 4
+    tables, _ = bm.export([1, 2, 3], 2)
+    assert tables[2][0] == tables[1][0] and tables[2][1] != tables[0][1]
+
+
 PINS = [pin_same_beginning_takes_over_full_blocks, pin_partial_last_block_is_never_shared,
         pin_hash_covers_everything_before, pin_waiting_blocks_are_taken_back,
         pin_handing_out_evicts_and_reuse_stops_at_the_first_miss,
-        pin_out_of_blocks_changes_nothing]
+        pin_out_of_blocks_changes_nothing, pin_equal_keys_of_different_blocks_share_nothing,
+        pin_equal_last_blocks_after_different_prefixes_share_nothing]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -197,7 +246,50 @@ class NoEviction(BlockManagerModel):
         return b
 
 
-@pytest.mark.parametrize("cls", [NoChain, CachesPartial, NoEviction], ids=lambda c: c.__name__)
+class KeyOnly(BlockManagerModel):
+    """Planted mistake: a key match is taken as a hit, with no check of the
+    cached block's prefix."""
+
+    def add_seq_tokens(self, seq_id, tokens):
+        self.prefix_of = _Anything()
+        return super().add_seq_tokens(seq_id, tokens)
+
+
+class _Anything(dict):
+    def __getitem__(self, k):
+        return _Equal()
+
+
+class _Equal:
+    def __eq__(self, other):
+        return True
+
+
+class LastBlockOnly(BlockManagerModel):
+    """Planted mistake: only the cached block's own token ids are compared,
+    not the prefix before it."""
+
+    def add_seq_tokens(self, seq_id, tokens):
+        B = self.block_size
+        real = self.prefix_of
+        self.prefix_of = {b: _Tail(p, B) for b, p in real.items()}
+        try:
+            return super().add_seq_tokens(seq_id, tokens)
+        finally:
+            merged = {b: (p.full if isinstance(p, _Tail) else p) for b, p in self.prefix_of.items()}
+            self.prefix_of = merged
+
+
+class _Tail:
+    def __init__(self, full, B):
+        self.full, self.B = full, B
+
+    def __eq__(self, other):
+        return tuple(self.full[-self.B:]) == tuple(other[-self.B:])
+
+
+@pytest.mark.parametrize("cls", [NoChain, CachesPartial, NoEviction, KeyOnly, LastBlockOnly],
+                         ids=lambda c: c.__name__)
 def test_planted_prefix_mistake_is_caught(cls):
     failed = 0
     for pin in PINS:
@@ -262,6 +354,17 @@ def _session(make, seed):
 @pytest.mark.parametrize("seed", range(8))
 def test_cpp_matches_model_exactly(seed):
     assert _session(Cpp, seed) == _session(BlockManagerModel, seed)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_cpp_matches_model_when_keys_collide(seed):
+    """3 key bits: prompts meet on keys all the time; the C++ manager (token
+    ids plus a check hash) still shares exactly what the model (whole
+    prefixes compared) shares."""
+    import functools
+    cpp = functools.partial(Cpp, key_bits=3)
+    model = functools.partial(BlockManagerModel, key_bits=3)
+    assert _session(cpp, 100 + seed) == _session(model, 100 + seed)
 
 
 def test_sessions_do_reuse_and_evict():
