@@ -162,6 +162,65 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max((num(r[3]) or 0) for r in rows)}
 
 
+class StagedInputs:
+    """A step's input tensors packed into one pinned host buffer (each piece
+    256-byte aligned) and ``copies`` device buffers of the same layout, so a
+    step moves all its inputs with one host-to-device copy."""
+
+    def __init__(self, tensors, dev, copies: int = 2):
+        offs, total = [], 0
+        for t in tensors:
+            total = -(-total // 256) * 256
+            offs.append(total)
+            total += t.numel() * t.element_size()
+        self.nbytes = total
+        self.host = torch.empty(total, dtype=torch.uint8).pin_memory()
+        self.dev = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(copies)]
+
+        def views(buf):
+            return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                    for t, o in zip(tensors, offs)]
+        for hv, t in zip(views(self.host), tensors):
+            hv.copy_(t.cpu())
+        self.views = [views(d) for d in self.dev]
+
+
+def e2e_pipelined(run, staged: StagedInputs, outs, houts, steps: int, stream, copy_stream):
+    """Time ``steps`` end-to-end steps on the device.  Step i: the copy stream
+    uploads the inputs into device buffer i % 2 (once step i - 2 is done with
+    it), the compute stream runs ``run(inputs, out)`` on it, and the copy
+    stream reads that step's output back into pinned host memory.  So one
+    step's copies overlap the neighbouring steps' kernels.  Returns ms/step."""
+    n = len(staged.dev)
+    in_ready = [torch.cuda.Event() for _ in range(n)]
+    computed = [torch.cuda.Event() for _ in range(n)]
+    drained = [torch.cuda.Event() for _ in range(n)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    copy_stream.wait_stream(stream)
+    for i in range(steps):
+        b = i % n
+        with torch.cuda.stream(copy_stream):
+            if i >= n:
+                copy_stream.wait_event(computed[b])
+            staged.dev[b].copy_(staged.host, non_blocking=True)
+            in_ready[b].record(copy_stream)
+        stream.wait_event(in_ready[b])
+        if i >= n:
+            stream.wait_event(drained[b])
+        run(staged.views[b], outs[b])
+        computed[b].record(stream)
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(computed[b])
+            houts[b].copy_(outs[b], non_blocking=True)
+            drained[b].record(copy_stream)
+    stream.wait_stream(copy_stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def kv_bytes(context_lens, num_heads, head_dim, elem_bytes) -> int:
     from paged_kv_cache_326_b200.accounting import decode_kv_bytes
     return decode_kv_bytes(context_lens, num_heads, head_dim, elem_bytes)
@@ -214,6 +273,363 @@ def cpu_baseline(w, budget_s=12.0):
     return {"value": sample_bytes * reps / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"all {w.num_seqs} texts x {w.num_heads} query heads of the step ({w.name}), "
                       f"{reps} run(s), {el:.1f} s, numpy fp64, BLAS limited to 1 thread"}
+
+
+def host_cores() -> dict:
+    """What the host offers the oracle: usable cores, all cores, BLAS threads."""
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except Exception:
+        aff = os.cpu_count() or 1
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()
+                    if i.get("user_api") == "blas"), default=None)
+    except Exception:
+        blas = None
+    return {"affinity_cores": aff, "cpu_count": os.cpu_count(), "blas_threads_default": blas}
+
+
+def cpu_baseline_pool(w, budget_s=10.0, max_workers=128):
+    """The oracle over the whole step, spread over the host's cores: one
+    worker process per usable core (``python -m tests.oracle_pool_worker``,
+    numpy and the oracle only, BLAS limited to one thread each).  The
+    (text, head) pairs, in text-major order, are cut into one contiguous run
+    per worker with about equal token counts; each worker holds the pool
+    blocks of its texts and runs the cache write and its pairs.  A run is
+    timed from the moment all workers are told to start until the last one
+    is done; runs repeat until ``budget_s`` seconds have passed."""
+    import pickle
+    import threading
+
+    from tests.gpu_helpers import oracle_inputs
+    cores = host_cores()
+    S, H = w.num_seqs, w.num_heads
+    n = max(1, min(cores["affinity_cores"], max_workers, S * H))
+    lens = w.context_lens.tolist()
+    cost = [lens[s] for s in range(S) for _ in range(H)]
+    total = sum(cost)
+    cuts, acc = [0], 0
+    for i, c in enumerate(cost):
+        acc += c
+        if len(cuts) < n and acc >= total * len(cuts) / n:
+            cuts.append(i + 1)
+    cuts.append(S * H)
+    cuts = sorted(set(cuts))
+    fp8 = w.k_cache.dtype == torch.uint8
+    shares = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        pairs = [(p // H, p % H) for p in range(a, b)]
+        seqs = sorted({s for s, _ in pairs})
+        oi = oracle_inputs(w.q, w.k, w.v, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                           w.slot_mapping, w.block_size, seqs)
+        pos = {s: i for i, s in enumerate(seqs)}
+        shares.append({"q": oi.q, "k": oi.k, "v": oi.v, "k_cache": oi.k_cache,
+                       "v_cache": oi.v_cache, "tables": oi.tables, "lens": oi.lens,
+                       "slots": oi.slots, "scale": w.scale, "block_size": w.block_size,
+                       "pairs": [(pos[s], h) for s, h in pairs],
+                       "fp8": (w.meta["k_scale"], w.meta["v_scale"]) if fp8 else None})
+    env = dict(os.environ, OMP_NUM_THREADS="1", OPENBLAS_NUM_THREADS="1", MKL_NUM_THREADS="1")
+    procs = [subprocess.Popen([sys.executable, "-m", "tests.oracle_pool_worker"], cwd=ROOT,
+                              env=env, stdin=subprocess.PIPE, stdout=subprocess.PIPE)
+             for _ in shares]
+    try:
+        def send(p, x):
+            pickle.dump(x, p.stdin, protocol=5)
+            p.stdin.flush()
+        ths = [threading.Thread(target=send, args=(p, x)) for p, x in zip(procs, shares)]
+        for t in ths:
+            t.start()
+        for t in ths:
+            t.join()
+        del shares
+        for p in procs:
+            if p.stdout.readline().strip() != b"ready":
+                raise RuntimeError("oracle worker failed to start")
+        reps, spent = 0, 0.0
+        while True:
+            t0 = time.perf_counter()
+            for p in procs:
+                p.stdin.write(b"run\n")
+                p.stdin.flush()
+            for p in procs:
+                if p.stdout.readline().strip() != b"done":
+                    raise RuntimeError("oracle worker failed")
+            spent += time.perf_counter() - t0
+            reps += 1
+            if spent >= budget_s or reps >= 200:
+                break
+    finally:
+        for p in procs:
+            try:
+                p.stdin.write(b"quit\n")
+                p.stdin.close()
+            except Exception:
+                pass
+        for p in procs:
+            try:
+                p.wait(timeout=30)
+            except Exception:
+                p.kill()
+    Hkv = w.k_cache.shape[1]
+    step_bytes = sum(lens) * 2 * Hkv * w.head_dim * w.k_cache.element_size()
+    return {"value": step_bytes * reps / spent / 1e9, "unit": "GB/s", "cores": len(procs),
+            "kind": "oracle",
+            "sample": f"all {S} texts x {H} query heads of the step ({w.name}) over "
+                      f"{len(procs)} worker processes (one per usable core, contiguous runs of "
+                      f"(text, head) pairs of about equal tokens), {reps} run(s), {spent:.1f} s, "
+                      f"numpy fp64, BLAS limited to 1 thread per worker",
+            **cores}
+
+
+def time_call(fn, stream, reps=20, warm=3, flush=None):
+    """Median and minimum device time (ms) of ``fn`` over ``reps`` calls after
+    ``warm`` untimed ones, each bracketed by CUDA events on ``stream``;
+    ``flush`` (if given) runs before each timed call, outside its events."""
+    for _ in range(warm):
+        fn()
+    marks = []
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        marks.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in marks]
+    return statistics.median(ms), min(ms)
+
+
+def oracle_check(w, out, seqs):
+    """CPU-baseline leg of one configuration: the oracle (one core, fp64) over
+    every head of the chosen texts, timed, and the GPU's outputs for them
+    compared with its result (max-abs, max-rel over |ref| >= 0.2, and the
+    tests' pass/fail rule)."""
+    from threadpoolctl import threadpool_limits
+    from tests.gpu_helpers import compare, oracle_inputs, run_oracle
+    seqs = [int(s) for s in seqs]
+    oi = oracle_inputs(w.q, w.k, w.v, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                       w.slot_mapping, w.block_size, seqs)
+    t0 = time.perf_counter()
+    with threadpool_limits(limits=1):
+        ref = run_oracle(oi, w.scale, w.block_size)
+    el = time.perf_counter() - t0
+    c = compare(out.index_select(0, torch.as_tensor(seqs, device=out.device)), ref, w.q.dtype)
+    lens = w.context_lens.tolist()
+    kv = sum(lens[s] for s in seqs) * 2 * w.k_cache.shape[1] * w.head_dim * w.k_cache.element_size()
+    return ({"max_abs": c.max_abs, "max_rel": c.max_rel, "ok": c.ok,
+             "outputs_checked": len(seqs) * w.num_heads, "texts_checked": len(seqs)},
+            {"value": kv / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+             "sample": f"{len(seqs)} seeded texts x {w.num_heads} heads, one run, {el:.2f} s"})
+
+
+def sample_texts(w, n, seed):
+    """n seeded texts of the batch, the longest one always among them (sorted)."""
+    import numpy as np
+    lens = w.context_lens.tolist()
+    longest = max(range(len(lens)), key=lambda s: lens[s])
+    rest = [s for s in range(len(lens)) if s != longest]
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(len(rest), min(n - 1, len(rest)), replace=False)
+    return sorted([longest] + [rest[int(i)] for i in pick])
+
+
+def decode_step_config(P, w, stream, peak, flush=None):
+    """pa_decode_step (write + attention, one launch, plus the merge kernel)
+    on one workload: the call's device time and rates."""
+    S, H, D = w.q.shape
+    Hkv = w.k_cache.shape[1]
+    eb = w.q.element_size()
+    lens = w.context_lens.tolist()
+    kv = kv_bytes(lens, Hkv, D, eb)
+    nbytes = (kv + 2 * S * H * D * eb + sum(4 * -(-L // w.block_size) for L in lens) + 4 * S +
+              2 * S * Hkv * D * 2 * eb + 8 * S)
+    out = torch.empty_like(w.q)
+    ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq)
+    status = torch.zeros(1, dtype=torch.int32, device=w.q.device)
+
+    def fn():
+        P.pa_decode_step(out, w.q, w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping,
+                         w.block_tables, w.context_lens, w.scale, workspace=ws, status=status)
+    med, mn = time_call(fn, stream, flush=flush)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    gbs = nbytes / (med * 1e-3) / 1e9
+    return {"path": "pa_decode_step", "call_ms": med, "call_ms_min": mn,
+            "algorithmic_bytes": nbytes, "kv_bytes": kv, "gbs": gbs,
+            "kv_gbs": kv / (med * 1e-3) / 1e9, "frac_of_measured_copy": gbs / peak,
+            "decode_tokens_per_s": S / (med * 1e-3)}, out
+
+
+def full_step_config(P, W, dev, stream, peak, with_oracle):
+    """The 40-layer step (pa_decode_step per layer over one 42.9 GB pool).
+    With the oracle: every head of 4 seeded texts at layers 0 and 39, from the
+    first step on the initial pool (the oracle replays every layer's writes
+    into the blocks those texts read, in layer order)."""
+    import numpy as np
+    fs = W.full_step(device=dev)
+    S, H, D = fs.q[0].shape
+    B, L = fs.block_size, fs.num_layers
+    check_layers = [0, L - 1]
+    seqs = np.sort(np.random.default_rng(5).choice(S, 4, replace=False))
+    if with_oracle:
+        sel = torch.as_tensor(seqs, device=dev)
+        need = torch.unique(torch.cat([fs.block_tables[l].index_select(0, sel).flatten()
+                                       for l in check_layers]))
+        need = need[need >= 0]
+        remap = torch.full((fs.k_cache.shape[0],), -1, dtype=torch.int64, device=dev)
+        remap[need] = torch.arange(need.numel(), device=dev)
+        kc = fs.k_cache.index_select(0, need).float().cpu().numpy()
+        vc = fs.v_cache.index_select(0, need).float().cpu().numpy()
+    out = torch.empty_like(fs.q[0])
+    ws = P.binding.workspace_for(fs.q[0], B, fs.block_tables[0].shape[1])
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    kept = {}
+
+    def step(keep=False):
+        for layer in range(L):
+            o = torch.empty_like(out) if keep and layer in check_layers else out
+            P.pa_decode_step(o, fs.q[layer], fs.k[layer], fs.v[layer], fs.k_cache, fs.v_cache,
+                             fs.slot_mapping[layer], fs.block_tables[layer], fs.context_lens,
+                             fs.scale, workspace=ws, status=status)
+            if keep and layer in check_layers:
+                kept[layer] = o
+    step(keep=True)
+    med, mn = time_call(step, stream, reps=5, warm=2)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    lens = fs.context_lens.tolist()
+    layer_kv = kv_bytes(lens, H, D, 2)
+    per_layer = (layer_kv + 2 * S * H * D * 2 + 4 * S * H * D * 2 +
+                 sum(4 * -(-x // B) for x in lens) + 12 * S)
+    gbs = per_layer * L / (med * 1e-3) / 1e9
+    rec = {"path": "pa_decode_step x 40 layers", "step_ms": med, "step_ms_min": mn,
+           "call_ms": med / L, "algorithmic_bytes_per_layer": per_layer,
+           "kv_bytes_per_step": layer_kv * L, "gbs": gbs,
+           "kv_gbs": layer_kv * L / (med * 1e-3) / 1e9, "frac_of_measured_copy": gbs / peak,
+           "decode_tokens_per_s": S / (med * 1e-3),
+           "pool": "one 131,072-block pool (42.9 GB) shared by the 40 layers, tables drawn "
+                   "per layer, so blocks alias across layers"}
+    if with_oracle:
+        from threadpoolctl import threadpool_limits
+
+        import oracle
+        from tests.gpu_helpers import compare
+        worst = {"max_abs": 0.0, "max_rel": 0.0, "ok": True, "outputs_checked": 0,
+                 "texts_checked": len(seqs), "layers_checked": check_layers}
+        t0 = time.perf_counter()
+        done = 0
+        with threadpool_limits(limits=1):
+            for layer in check_layers:
+                for l2 in range(done, layer + 1):
+                    sl = fs.slot_mapping[l2]
+                    nb = remap[(sl // B).clamp(min=0)]
+                    idx = torch.nonzero((sl >= 0) & (nb >= 0)).flatten()
+                    kc, vc = oracle.cache_write(
+                        kc, vc, fs.k[l2].index_select(0, idx).float().cpu().numpy(),
+                        fs.v[l2].index_select(0, idx).float().cpu().numpy(),
+                        (nb[idx] * B + sl[idx] % B).cpu().numpy(), B)
+                done = layer + 1
+                t = fs.block_tables[layer].index_select(0, sel).to(torch.int64)
+                t = torch.where(t >= 0, remap[t.clamp(min=0)], torch.full_like(t, -1)).cpu().numpy()
+                q = fs.q[layer].index_select(0, sel).float().cpu().numpy()
+                ref = oracle.paged_decode(q, kc, vc, t,
+                                          fs.context_lens.index_select(0, sel).cpu().numpy(),
+                                          fs.scale, B)
+                c = compare(kept[layer].index_select(0, sel), ref, torch.float16)
+                worst["max_abs"] = max(worst["max_abs"], c.max_abs)
+                worst["max_rel"] = max(worst["max_rel"], c.max_rel)
+                worst["ok"] = worst["ok"] and c.ok
+                worst["outputs_checked"] += len(seqs) * H
+        el = time.perf_counter() - t0
+        rec["parity"] = worst
+        rec["cpu_baseline"] = {
+            "value": sum(lens[s] for s in seqs) * 2 * H * D * 2 * len(check_layers) / el / 1e9,
+            "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(seqs)} texts x {H} heads at layers {check_layers} with every "
+                      f"layer's writes replayed, {el:.1f} s"}
+    del fs
+    torch.cuda.empty_cache()
+    return rec
+
+
+def other_configs(P, W, dev, stream, peak, with_oracle=True):
+    """The other configurations of the study, each on the path the headline
+    uses (or the shared-prefix call for the shared-prefix one): device time of
+    the decode call, GB/s, fraction of the measured copy bandwidth, decode
+    tokens/s, and, in the CPU-baseline leg, parity against the oracle on a
+    seeded sample of outputs."""
+    res = {}
+    # tiny: 108 KB of KV, so L2 is flushed (a 256 MB write) before each call
+    w = W.tiny(device=dev)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rec, out = decode_step_config(P, w, stream, peak, flush=lambda: flush_buf.zero_())
+    rec["l2"] = "flushed before each call (256 MB write)"
+    if with_oracle:
+        rec["parity"], rec["cpu_baseline"] = oracle_check(w, out, range(w.num_seqs))
+    res["tiny"] = rec
+    del w, out, flush_buf
+    # skewed lengths, bf16, blocks of 8, 16 and 32
+    for B in (8, 16, 32):
+        w = W.skewed(block_size=B, device=dev)
+        rec, out = decode_step_config(P, w, stream, peak)
+        if with_oracle:
+            rec["parity"], rec["cpu_baseline"] = oracle_check(w, out, sample_texts(w, 24, 30 + B))
+        res[f"skewed_b{B}"] = rec
+        del w, out
+        torch.cuda.empty_cache()
+    # shared prefixes: 32 prompts x 8 samples built by the block manager
+    w = shared_prefix_inputs(P, W, 4, dev)
+    S, H, D = w.q.shape
+    gs = w.meta["samples"]
+    lens = w.context_lens.tolist()
+    distinct = unique_kv_bytes(w, H, D, 2)
+    logical = kv_bytes(lens, H, D, 2)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    P.pa_kv_cache_write(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, status=status)
+    split = P.split_shared_prefix(w.block_tables.cpu(), w.context_lens.cpu(), w.block_size, gs)
+    pt, pl, tt, tl = [t.to(dev) for t in split]
+    ws_sh = torch.empty(P.pa_paged_attn_decode_shared_workspace_size(
+        pt.shape[0], gs, H, D, w.block_size, pt.shape[1], tt.shape[1]), dtype=torch.uint8,
+        device=dev)
+    out_sh = torch.empty_like(w.q)
+    out_pl = torch.empty_like(w.q)
+    ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq)
+    small = 2 * S * H * D * 2 + 4 * S
+    tab_sh = 4 * len(split[1]) + sum(4 * -(-x // w.block_size) for x in split[1].tolist() +
+                                     split[3].tolist())
+    tab_pl = sum(4 * -(-x // w.block_size) for x in lens)
+    for name, fn, out, tab in (
+            ("shared_prefix_cascade",
+             lambda: P.pa_paged_attn_decode_shared(out_sh, w.q, w.k_cache, w.v_cache, pt, pl, tt,
+                                                   tl, w.scale, gs, workspace=ws_sh,
+                                                   status=status), out_sh, tab_sh),
+            ("shared_prefix_plain",
+             lambda: P.pa_paged_attn_decode(out_pl, w.q, w.k_cache, w.v_cache, w.block_tables,
+                                            w.context_lens, w.scale, workspace=ws,
+                                            status=status), out_pl, tab_pl)):
+        med, mn = time_call(fn, stream)
+        if status.item() != 0:
+            raise RuntimeError(f"device status {status.item()}")
+        nbytes = distinct + small + tab
+        gbs = nbytes / (med * 1e-3) / 1e9
+        rec = {"path": ("pa_paged_attn_decode_shared (split by pa_split_shared_prefix)"
+                        if name.endswith("cascade") else
+                        "pa_paged_attn_decode over the joined tables"),
+               "call_ms": med, "call_ms_min": mn, "algorithmic_bytes": nbytes,
+               "distinct_kv_bytes": distinct, "logical_kv_bytes": logical, "gbs": gbs,
+               "logical_kv_gbs": logical / (med * 1e-3) / 1e9,
+               "frac_of_measured_copy": gbs / peak, "counts": "distinct (block, row) KV bytes",
+               "decode_tokens_per_s": S / (med * 1e-3)}
+        if with_oracle:
+            rec["parity"], rec["cpu_baseline"] = oracle_check(w, out, sample_texts(w, 24, 44))
+        res[name] = rec
+    del w, out_sh, out_pl, ws_sh, ws
+    torch.cuda.empty_cache()
+    res["full_step"] = full_step_config(P, W, dev, stream, peak, with_oracle)
+    return res
 
 
 def run_reference(args, world, rank):
@@ -319,6 +735,32 @@ def run_prefill_bench(args, ranks, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / Ke
+    # Prompt time against the reused fraction: the same prompts with their
+    # first c tokens already in the cache (stored by the steps above), only
+    # the other 2048 - c tokens computed (pa_prefill_with_prefix).
+    sweep = []
+    L0 = w.lens[0]
+    for frac in (0.25, 0.5, 0.75):
+        c = int(L0 * frac) // w.block_size * w.block_size
+        n = L0 - c
+        rows = torch.cat([torch.arange(int(w.cu_seqlens[s]) + c, int(w.cu_seqlens[s + 1]),
+                                       device=dev) for s in range(len(w.lens))])
+        qn, kn, vn = w.q[rows].contiguous(), w.k[rows].contiguous(), w.v[rows].contiguous()
+        sn = w.slot_mapping[rows].contiguous()
+        cun = torch.arange(0, (len(w.lens) + 1) * n, n, dtype=torch.int32, device=dev)
+        cached = torch.full((len(w.lens),), c, dtype=torch.int32, device=dev)
+        outn = torch.empty_like(qn)
+
+        def reuse_step():
+            P.pa_prefill_with_prefix(outn, qn, kn, vn, cun, n, w.scale, w.k_cache, w.v_cache,
+                                     w.block_tables, cached, sn, status=status)
+        med, mn = time_call(reuse_step, stream, reps=max(5, min(K, 20)))
+        if status.item() != 0:
+            raise RuntimeError(f"device status {status.item()}")
+        fl = 4.0 * D * H * len(w.lens) * sum(c + i + 1 for i in range(n))
+        sweep.append({"cached_tokens": c, "new_tokens": n, "ms": med, "ms_min": mn,
+                      "ms_vs_no_reuse": med / ms_step, "tflops": fl / (med * 1e-3) / 1e12,
+                      "new_tokens_per_s": len(w.lens) * n / (med * 1e-3)})
     ms_step, e2e_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms], dev)
     peak, peak_src = tensor_peak()
     tflops = flops / (ms_step * 1e-3) / 1e12
@@ -332,16 +774,19 @@ def run_prefill_bench(args, ranks, world, rank, local):
                    "num_heads": H, "head_dim": D, "block_size": w.block_size,
                    "l2": "q, k, v, out 1.3 GB per step >> 126 MB L2",
                    "parallelism": f"independent prompts per GPU x{world}",
-                   "path": "pa_prefill (cache write + causal attention)"},
+                   "path": "pa_prefill (causal attention; the kernel stores the prompts' keys "
+                           "and values from its tiles)"},
         "prefill_tokens_per_s": world * T / (ms_step * 1e-3),
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "traffic": None,
-                     "kernel": "prefill_tc_kernel (tcgen05, TMEM accumulators) + kv_cache_write_kernel",
+                     "kernel": "prefill_tc_kernel (tcgen05, TMEM accumulators, cache store "
+                               "from the K/V tiles)",
                      "peak_source": peak_src, "algorithmic_flops_per_launch": flops},
+        "reuse_sweep": sweep,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 3 * w.q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
                 "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -597,9 +1042,28 @@ def run_cow_copy(args, ranks, world, rank, local):
     e2e_ms = e0.elapsed_time(e1) / Ke
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()}")
-    ms_step, e2e_ms, kernel_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms, kernel_ms], dev)
+    # The write ceiling for a launch of this size: the write-only probe on
+    # the same number of bytes as a burst writes, rotating over as many
+    # buffers as there are bursts (so L2 holds the same share of them).
+    write_bytes = n * 2 * block_bytes
+    wbuf = torch.empty(len(bursts) * write_bytes, dtype=torch.uint8, device=dev)
+    wslices = [wbuf[i * write_bytes:(i + 1) * write_bytes] for i in range(len(bursts))]
+    for i in range(3):
+        P.binding.pa_write_probe(wslices[i % len(wslices)])
+    wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(max(K, 20))]
+    for i, (e0, e1) in enumerate(wev):
+        e0.record(stream)
+        P.binding.pa_write_probe(wslices[i % len(wslices)])
+        e1.record(stream)
+    torch.cuda.synchronize()
+    probe_ms = statistics.median(a.elapsed_time(b) for a, b in wev)
+    del wbuf, wslices
+    ms_step, e2e_ms, kernel_ms, probe_ms = dist.max_over_ranks(
+        ranks, [ms_step, e2e_ms, kernel_ms, probe_ms], dev)
     peak, peak_src = hbm_peak()
     achieved = step_bytes / (kernel_ms * 1e-3) / 1e9
+    write_gbs = write_bytes / (kernel_ms * 1e-3) / 1e9
+    probe_gbs = write_bytes / (probe_ms * 1e-3) / 1e9
     line = {
         "metric": "paged block copy GB/s (distinct blocks read + blocks written)",
         "value": world * step_bytes / (ms_step * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
@@ -612,6 +1076,11 @@ def run_cow_copy(args, ranks, world, rank, local):
                          f"({len(bursts) * step_bytes / 1e9:.2f} GB of blocks >> 126 MB L2)",
                    "parallelism": f"independent pool per GPU x{world}"},
         "kernel_ms": {"copy_blocks": kernel_ms},
+        "write_ceiling": {"probe_ms": probe_ms, "probe_gbs": probe_gbs,
+                          "copy_write_gbs": write_gbs, "frac": write_gbs / probe_gbs,
+                          "how": f"pa_write_probe over {write_bytes} bytes (a burst's "
+                                 f"destination blocks), {len(bursts)} buffers in rotation, "
+                                 "median launch"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None, "kernel": "copy_blocks_kernel",
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": step_bytes},
@@ -652,6 +1121,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the tiny, skewed, shared-prefix and 40-layer configurations that "
+                         "the default run reports under other_configs")
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
     ap.add_argument("--kv-dtype", choices=["f16", "fp8"], default="f16",
                     help="fp8: the batch-64 step over 8-bit E4M3 caches (two calls)")
@@ -744,7 +1216,7 @@ def main():
     fused = args.path == "fused"
     if fused:
         decode_bytes += write_bytes
-    out = torch.empty_like(w.q)
+    out0 = torch.empty_like(w.q)
     ws = P.binding.workspace_for(w.q, w.block_size, w.max_blocks_per_seq, Hkv)
     if cascade:
         ws_shared = torch.empty(P.pa_paged_attn_decode_shared_workspace_size(
@@ -759,7 +1231,8 @@ def main():
         elif not fused:
             P.pa_kv_cache_write(k, v, w.k_cache, w.v_cache, slots, status=status)
 
-    def decode_part(q, k, v, slots, tables, lens, shared_tables=None):
+    def decode_part(q, k, v, slots, tables, lens, shared_tables=None, out_=None):
+        out = out_ if out_ is not None else out0
         if cascade:
             pt, pl_d, tt, tl_d = shared_tables if shared_tables is not None else split_d
             P.pa_paged_attn_decode_shared(out, q, w.k_cache, w.v_cache, pt, pl_d, tt, tl_d,
@@ -814,56 +1287,35 @@ def main():
     decode_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
     write_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
 
-    # end to end: inputs from pinned host memory, output back to the host
-    hq = w.q.cpu().pin_memory()
-    hk = w.k.cpu().pin_memory()
-    hv = w.v.cpu().pin_memory()
-    hslot = w.slot_mapping.cpu().pin_memory()
-    htab = w.block_tables.cpu().pin_memory()
-    hlen = w.context_lens.cpu().pin_memory()
+    # end to end: each step's inputs from pinned host memory (one packed copy),
+    # its output back to pinned host memory, copies overlapped with the
+    # neighbouring steps' kernels on a second stream
     if cascade:   # the split tables stand in for the joined ones
-        hsplit = [t.pin_memory() for t in split]
-        dsplit = [torch.empty_like(t) for t in split_d]
-        htab, hlen = hsplit[0], hsplit[1]
-    hout = torch.empty_like(hq).pin_memory()
-    dq, dk, dv = torch.empty_like(w.q), torch.empty_like(w.k), torch.empty_like(w.v)
-    dslot, dtab, dlen = (torch.empty_like(w.slot_mapping), torch.empty_like(w.block_tables),
-                         torch.empty_like(w.context_lens))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hslot, htab, hlen))
-    if cascade:
-        h2d += sum(t.numel() * t.element_size() for t in hsplit[2:])
-    d2h = hout.numel() * hout.element_size()
+        inputs = [w.q, w.k, w.v, w.slot_mapping, *split_d]
+    else:
+        inputs = [w.q, w.k, w.v, w.slot_mapping, w.block_tables, w.context_lens]
+    staged = StagedInputs(inputs, dev)
+    outs = [torch.empty_like(w.q) for _ in staged.dev]
+    houts = [torch.empty(w.q.shape, dtype=w.q.dtype).pin_memory() for _ in staged.dev]
+    h2d = staged.nbytes
+    d2h = outs[0].numel() * outs[0].element_size()
 
-    def e2e_step():
+    def e2e_run(x, o):
         if cascade:
-            for d, h in zip(dsplit, hsplit):
-                d.copy_(h, non_blocking=True)
-            for d, h in ((dq, hq), (dk, hk), (dv, hv), (dslot, hslot)):
-                d.copy_(h, non_blocking=True)
-            write_part(dk, dv, dslot)
-            decode_part(dq, dk, dv, dslot, None, None, shared_tables=dsplit)
-            hout.copy_(out, non_blocking=True)
-            return
-        for d, h in ((dq, hq), (dk, hk), (dv, hv), (dslot, hslot), (dtab, htab), (dlen, hlen)):
-            d.copy_(h, non_blocking=True)
-        write_part(dk, dv, dslot)
-        decode_part(dq, dk, dv, dslot, dtab, dlen)
-        hout.copy_(out, non_blocking=True)
+            q, k, v, slots, pt, pl_d, tt, tl_d = x
+            write_part(k, v, slots)
+            decode_part(q, k, v, slots, None, None, shared_tables=(pt, pl_d, tt, tl_d), out_=o)
+        else:
+            q, k, v, slots, tables, lens = x
+            write_part(k, v, slots)
+            decode_part(q, k, v, slots, tables, lens, out_=o)
 
+    copy_stream = torch.cuda.Stream(dev)
     Ke = max(3, min(K, 1000))
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
+    e2e_pipelined(e2e_run, staged, outs, houts, 3, stream, copy_stream)
     barrier()
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_stop = torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for _ in range(Ke):
-        e2e_step()
-    e_stop.record(stream)
-    torch.cuda.synchronize()
+    e2e_ms = e2e_pipelined(e2e_run, staged, outs, houts, Ke, stream, copy_stream)
     barrier()
-    e2e_ms = e_start.elapsed_time(e_stop) / Ke
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()}: {P.pa_status_string(status.item())}")
 
@@ -932,8 +1384,18 @@ def main():
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        w_cpu = w
-        line["cpu_baseline"] = cpu_baseline(w_cpu)
+        single = cpu_baseline(w)
+        try:
+            line["cpu_baseline"] = cpu_baseline_pool(w)
+            line["cpu_baseline"]["single_core"] = single
+        except Exception as e:   # the pool is a report, never a reason to lose the line
+            line["cpu_baseline"] = dict(single, pool_error=str(e)[:200], **host_cores())
+    if (world == 1 and args.workload == "opt13b_batch64" and not fp8 and args.path == "fused"
+            and not args.no_other_configs):
+        del w, staged, outs, houts, ws
+        torch.cuda.empty_cache()
+        line["other_configs"] = other_configs(P, W, dev, stream, peak,
+                                              with_oracle=not args.no_cpu_baseline)
     if rank == 0:
         print(json.dumps(line), flush=True)
     dist.finish(ranks)

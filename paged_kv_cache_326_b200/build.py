@@ -4,12 +4,15 @@
 
 Compiles every .cu / .cc under csrc/ with nvcc (CUDA runtime linked
 statically) into paged_kv_cache_326_b200/libpagedattn.so.  Object files go to
-_build/ at the repository root.  Nothing here needs a GPU.
+_build/ at the repository root.  Nothing here needs a GPU.  An existing
+library is reused only if the SHA-256 of the sources, headers and flags it
+was built from (kept in libpagedattn.so.sha256) matches the current ones.
 """
 from __future__ import annotations
 
 import argparse
 import concurrent.futures as cf
+import hashlib
 import os
 import subprocess
 import sys
@@ -20,6 +23,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedattn.so")
+# digest of the sources the library was built from, written beside it
+STAMP = LIB + ".sha256"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3", f"-I{INCLUDE}", f"-I{CSRC}"]
@@ -49,15 +54,28 @@ def _compile(src: str, ptxas_verbose: bool) -> str:
     return obj
 
 
+def _digest(paths) -> str:
+    """SHA-256 over the build inputs' names and contents and the compiler
+    flags: the library is reused only if it was built from exactly these."""
+    h = hashlib.sha256()
+    h.update(" ".join(ARCH + COMMON).encode())
+    for p in sorted(paths):
+        h.update(os.path.relpath(p, ROOT).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def build(ptxas_verbose: bool = False, force: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = sources()
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     headers.append(os.path.join(INCLUDE, "pagedattn.h"))
-    if not force and os.path.exists(LIB):
-        newest = max(os.path.getmtime(p) for p in srcs + headers + [__file__])
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
+    digest = _digest(srcs + headers + [__file__])
+    if not force and os.path.exists(LIB) and os.path.exists(STAMP):
+        with open(STAMP) as f:
+            if f.read().strip() == digest:
+                return LIB
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(lambda s: _compile(s, ptxas_verbose), srcs))
     tmp = LIB + ".tmp"
@@ -66,6 +84,8 @@ def build(ptxas_verbose: bool = False, force: bool = False) -> str:
     if res.returncode != 0:
         raise RuntimeError(f"link failed: {' '.join(cmd)}\n{res.stdout}\n{res.stderr}")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(digest + "\n")
     return LIB
 
 
