@@ -13,7 +13,10 @@ tokens, 40 heads of 128; ``--prefill-kernel`` 0 automatic, 1 mma.sync, 2
 tcgen05), ``shared_prefix`` (32 prompts x 8 samples built by the block
 manager, through pa_paged_attn_decode_shared over the split tables).
 ``--gqa-kernel`` picks the grouped-query kernel (0 automatic, 1 CUDA cores, 2
-tensor cores).
+tensor cores), ``--fp8-kernel`` the 8-bit one (same values).
+``opt13b_prefill_reuse``: the prompt phase of the same prompts with their
+first half already stored (pa_prefill_with_prefix; the first repetition
+stores the whole prompts).
 """
 from __future__ import annotations
 
@@ -53,8 +56,33 @@ def main():
     ap.add_argument("--path", choices=["fused", "calls"], default="fused")
     ap.add_argument("--gqa-kernel", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--prefill-kernel", type=int, choices=[0, 1, 2], default=0)
+    ap.add_argument("--fp8-kernel", type=int, choices=[0, 1, 2], default=0)
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, args.fp8_kernel)
+    if args.workload == "opt13b_prefill_reuse":
+        w = W.opt13b_prefill(device=dev, num_prompts=args.num_seqs if args.num_seqs > 0 else 16)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        out = torch.empty_like(w.q)
+        P.pa_prefill(out, w.q, w.k, w.v, w.cu_seqlens, w.max_seqlen, w.scale, w.k_cache,
+                     w.v_cache, w.slot_mapping, status=status)
+        L = w.lens[0]
+        c = L // 2
+        rows = torch.cat([torch.arange(int(w.cu_seqlens[s]) + c, int(w.cu_seqlens[s + 1]),
+                                       device=dev) for s in range(len(w.lens))])
+        qn, kn, vn = w.q[rows].contiguous(), w.k[rows].contiguous(), w.v[rows].contiguous()
+        sn = w.slot_mapping[rows].contiguous()
+        cun = torch.arange(0, (len(w.lens) + 1) * (L - c), L - c, dtype=torch.int32, device=dev)
+        cached = torch.full((len(w.lens),), c, dtype=torch.int32, device=dev)
+        outn = torch.empty_like(qn)
+        for _ in range(args.reps):
+            P.pa_prefill_with_prefix(outn, qn, kn, vn, cun, L - c, w.scale, w.k_cache, w.v_cache,
+                                     w.block_tables, cached, sn, status=status)
+        torch.cuda.synchronize()
+        if status.item() != 0:
+            raise SystemExit(f"device status {status.item()}: {P.pa_status_string(status.item())}")
+        print(f"{len(w.lens)} prompts, {c} tokens stored, {L - c} new each, status ok")
+        return
     if args.workload == "opt13b_prefill":
         P.pa_set_option(P.PA_OPT_PREFILL_KERNEL, args.prefill_kernel)
         w = W.opt13b_prefill(device=dev, num_prompts=args.num_seqs if args.num_seqs > 0 else 16)
