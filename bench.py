@@ -523,14 +523,17 @@ def full_step_config(P, W, dev, stream, peak, with_oracle):
         done = 0
         with threadpool_limits(limits=1):
             for layer in check_layers:
+                # the writes of the layers since the last check, in layer order
+                ks, vs, slots = [], [], []
                 for l2 in range(done, layer + 1):
                     sl = fs.slot_mapping[l2]
                     nb = remap[(sl // B).clamp(min=0)]
                     idx = torch.nonzero((sl >= 0) & (nb >= 0)).flatten()
-                    kc, vc = oracle.cache_write(
-                        kc, vc, fs.k[l2].index_select(0, idx).float().cpu().numpy(),
-                        fs.v[l2].index_select(0, idx).float().cpu().numpy(),
-                        (nb[idx] * B + sl[idx] % B).cpu().numpy(), B)
+                    ks.append(fs.k[l2].index_select(0, idx).float().cpu().numpy())
+                    vs.append(fs.v[l2].index_select(0, idx).float().cpu().numpy())
+                    slots.append((nb[idx] * B + sl[idx] % B).cpu().numpy())
+                kc, vc = oracle.cache_write(kc, vc, np.concatenate(ks), np.concatenate(vs),
+                                            np.concatenate(slots), B)
                 done = layer + 1
                 t = fs.block_tables[layer].index_select(0, sel).to(torch.int64)
                 t = torch.where(t >= 0, remap[t.clamp(min=0)], torch.full_like(t, -1)).cpu().numpy()
