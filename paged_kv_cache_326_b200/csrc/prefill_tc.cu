@@ -83,6 +83,14 @@ constexpr int64_t kTcDrainNs = 1000000000;
 // many are computed by the FMA-pipe polynomial (exp2poly.cuh), the rest by
 // the exponential unit.
 constexpr int kTcPolyPairs = PA_TC_POLY_PAIRS;
+#ifndef PA_TC_EARLY_S
+#define PA_TC_EARLY_S 1
+#endif
+// 1: the softmax warps release S as soon as they hold the scores in
+// registers, and the next block's S is issued then, ahead of this block's
+// P V; each softmax waits for the previous P V only before it stores P and
+// rescales O.  0: S(j+1) is issued after P(j) V.
+constexpr bool kTcEarlyS = PA_TC_EARLY_S != 0;
 
 // max(a, b, c) in one instruction (three-input max.f32 of sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -140,7 +148,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   uint8_t* sQ = smem;                               // tile t at t * Q_BYTES
   uint8_t* sKV = smem + kTcTiles * LY::Q_BYTES;     // stage i at i * STAGE
   __shared__ uint64_t bar_q, bar_full[kTcStages], bar_empty[kTcStages];
-  __shared__ uint64_t bar_s[kTcTiles], bar_p[kTcTiles], bar_o[kTcTiles];
+  __shared__ uint64_t bar_s[kTcTiles], bar_p[kTcTiles], bar_o[kTcTiles], bar_sfree[kTcTiles];
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
 
@@ -190,6 +198,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&bar_s[t], 1);
       mbar_init(&bar_p[t], kTcBM);
       mbar_init(&bar_o[t], 1);
+      mbar_init(&bar_sfree[t], kTcBM / 32);  // one arrival per softmax warp
     }
     fence_barrier_init();
   }
@@ -400,10 +409,21 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       for (int t = 0; t < kTcTiles && ok; ++t)
         if (nkb_t[t] > 0) ok = issue_s(t, 0);
       for (int j = 0; j < nkb && ok; ++j) {
-        for (int t = 0; t < kTcTiles && ok; ++t) {
-          if (j >= nkb_t[t]) continue;
-          ok = issue_pv(t, j);
-          if (ok && j + 1 < nkb_t[t]) ok = issue_s(t, j + 1);
+        if constexpr (kTcEarlyS) {
+          // S(j+1) as soon as the softmax holds S(j) in registers, then P(j) V
+          for (int t = 0; t < kTcTiles && ok; ++t) {
+            if (j + 1 >= nkb_t[t]) continue;
+            ok = wait(&bar_sfree[t], j & 1);
+            if (ok) ok = issue_s(t, j + 1);
+          }
+          for (int t = 0; t < kTcTiles && ok; ++t)
+            if (j < nkb_t[t]) ok = issue_pv(t, j);
+        } else {
+          for (int t = 0; t < kTcTiles && ok; ++t) {
+            if (j >= nkb_t[t]) continue;
+            ok = issue_pv(t, j);
+            if (ok && j + 1 < nkb_t[t]) ok = issue_s(t, j + 1);
+          }
         }
         if (ok) {
           tc::commit(&bar_empty[j % kTcStages]);  // block j's stage is read for good
@@ -446,6 +466,12 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int c = 0; c < 16; ++c) sv[i * 16 + c] = __uint_as_float(v[i][c]);
       }
+      if constexpr (kTcEarlyS) {
+        // the scores are in registers: the next block's S may overwrite them
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_sfree[t]);
+      }
       // `below`: no score of this warp's rows is masked in this block, so part
       // of the weights may come from the polynomial
       bool below;
@@ -477,16 +503,24 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       }
       // base-2 logits: the scale (> 0) is applied in the exponent
       const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
-      // P_t and O_t are in use by the previous block's product until it is done
-      if (jj > 0) {
-        failed = __any_sync(0xffffffffu, !wait(&bar_o[t], (jj - 1) & 1));
+      // P_t and O_t are in use by the previous block's product until it is
+      // done (here, or after the weights when S runs a block ahead)
+      auto wait_pv = [&]() -> bool {
+        if (jj > 0) {
+          if (__any_sync(0xffffffffu, !wait(&bar_o[t], (jj - 1) & 1))) return false;
+          tc::fence_after_sync();
+        }
+        return true;
+      };
+      if constexpr (!kTcEarlyS) {
+        failed = !wait_pv();
         if (failed) break;
-        tc::fence_after_sync();
       }
       const bool raise = rmax > m + 8.f;
       const float m_new = raise ? rmax : m;
       const float alpha = raise && m != -INFINITY ? fast_exp2(m - m_new) : 1.f;
-      if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      auto rescale_o = [&]() {
+        if (!(jj > 0 && __any_sync(0xffffffffu, alpha != 1.f))) return;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 64) {
           uint32_t v[4][16];
@@ -501,7 +535,8 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
             tc::st16(rbase + kColO + c0 + i * 16, v[i]);
           }
         }
-      }
+      };
+      if constexpr (!kTcEarlyS) rescale_o();
       l *= alpha;
       m = m_new;
       const float mm = m == -INFINITY ? 0.f : m;
@@ -531,6 +566,11 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
         for (int c = 0; c < kTcBN; c += 2) weights(c, false);
       }
       l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+      if constexpr (kTcEarlyS) {
+        failed = !wait_pv();
+        if (failed) break;
+        rescale_o();
+      }
       tc::st16(rbase + kColPhi, *reinterpret_cast<uint32_t(*)[16]>(ph));
       tc::st16(rbase + kColPhi + 16, *reinterpret_cast<uint32_t(*)[16]>(ph + 16));
       if constexpr (BF16) {

@@ -198,3 +198,53 @@ def test_parallel_sampling_session_with_device_copies():
                               lens.numpy(), float(np.float32(D ** -0.5)), B)
     c = compare(out, ref, dt)
     assert c.ok, c
+
+
+@pytest.mark.parametrize("count", [1, 7, 700])
+def test_copy_shares_cross_copy_boundaries(count):
+    """The grid cuts all copies of a call into equal shares of 16-byte
+    vectors: with blocks of 512 bytes (1 head x 4 x 64, 32 vectors) a
+    thread's lanes step across many copies per round, with one pair only a
+    few threads work, and with 700 pairs shares start and end inside
+    copies.  Bit-exact in every case."""
+    import paged_kv_cache_326_b200 as P
+    H, D, B, N = 1, 64, 4, 1600
+    kc, vc = (_bits_pool(N, H, B, D, torch.float16, 11 + i) for i in range(2))
+    pairs = _pairs(N, N, count, 12 + count, same_pool=True)
+    ek, ev = oracle.copy_blocks(_i16(kc), _i16(vc), _i16(kc), _i16(vc), pairs)
+    st = new_status()
+    P.pa_copy_blocks(kc, vc, kc, vc, torch.tensor(pairs, dtype=torch.int32, device="cuda"),
+                     status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert np.array_equal(_i16(kc), ek) and np.array_equal(_i16(vc), ev)
+
+
+def test_copy_bad_pair_in_the_middle_is_reported_and_skipped():
+    """A pair naming a block outside the pool, between good ones: the status
+    word says PA_ERR_BAD_BLOCK, that pair copies nothing, every other pair
+    is exact."""
+    import paged_kv_cache_326_b200 as P
+    H, D, B, N = 8, 128, 16, 64
+    kc, vc = (_bits_pool(N, H, B, D, torch.bfloat16, 21 + i) for i in range(2))
+    good = _pairs(N, N, 20, 23, same_pool=True)
+    pairs = good[:10] + [(N + 5, good[10][1])] + good[11:]
+    ek, ev = oracle.copy_blocks(_i16(kc), _i16(vc), _i16(kc), _i16(vc),
+                                good[:10] + good[11:])
+    st = new_status()
+    P.pa_copy_blocks(kc, vc, kc, vc, torch.tensor(pairs, dtype=torch.int32, device="cuda"),
+                     status=st)
+    torch.cuda.synchronize()
+    assert st.item() == P.binding.PA_ERR_BAD_BLOCK
+    assert np.array_equal(_i16(kc), ek) and np.array_equal(_i16(vc), ev)
+
+
+def test_write_probe_writes_the_whole_buffer():
+    import paged_kv_cache_326_b200 as P
+    buf = torch.zeros(3 << 20, dtype=torch.uint8, device="cuda")
+    P.binding.pa_write_probe(buf)
+    torch.cuda.synchronize()
+    w = buf.view(torch.int32).view(-1, 4).cpu()
+    idx = torch.arange(w.shape[0], dtype=torch.int64)
+    assert torch.equal(w[:, 0].to(torch.int64) & 0xFFFFFFFF, idx & 0xFFFFFFFF)
+    assert torch.equal(w[:, 2], ~w[:, 0])
