@@ -25,7 +25,7 @@ namespace {
 
 constexpr int kCopyThreads = 256;
 constexpr int kUnroll = 4;
-constexpr int kCopyCtasPerSm = 3;
+constexpr int kCopyCtasPerSm = 8;
 
 __global__ void __launch_bounds__(kCopyThreads, kCopyCtasPerSm)
 copy_blocks_kernel(const uint4* src_k, const uint4* src_v, uint4* dst_k, uint4* dst_v,
@@ -35,63 +35,36 @@ copy_blocks_kernel(const uint4* src_k, const uint4* src_v, uint4* dst_k, uint4* 
   // before; a kernel launched after this one waits for all of it.
   griddep_wait();
   griddep_launch_dependents();
-  constexpr int kStep = kCopyThreads * kUnroll;
   const int64_t per = (total + gridDim.x - 1) / gridDim.x;
   const int64_t lo = blockIdx.x * per;
-  // vectors in this CTA's share (fewer than 2^31: the grid has at least
-  // one CTA per SM and the host limits the total)
-  const int n = static_cast<int>(max(int64_t{0}, min(per, total - lo)));
-  const int vpb = static_cast<int>(vecs_per_block);
-  // Lane u of this thread walks vectors i = u * kCopyThreads + tid of the
-  // share, + kStep each round, keeping its copy index and offset up to date
-  // (one division to start with, then additions).
-  int i[kUnroll], copy[kUnroll], off[kUnroll];
-  const uint4* src[kUnroll];
-  uint4* dst[kUnroll];
-  // the endpoints of copy c (pair c / 2, K or V); null if the pair is bad,
-  // which the thread that meets the copy's first vector reports
-  auto endpoints = [&](int u) {
-    const int pair = copy[u] >> 1;
+  const int64_t hi = lo + per < total ? lo + per : total;
+  // The share [lo, hi) covers the end of one copy, whole copies, the start
+  // of another: walk it copy by copy, each piece a contiguous range.
+  for (int64_t c = lo / vecs_per_block; c * vecs_per_block < hi; ++c) {
+    const int64_t base = c * vecs_per_block;
+    const int64_t a = lo > base ? lo - base : 0;
+    const int64_t b = hi < base + vecs_per_block ? hi - base : vecs_per_block;
+    const int64_t pair = c >> 1;
     const int64_t s = __ldg(pairs + 2 * pair);
     const int64_t d = __ldg(pairs + 2 * pair + 1);
     if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) {
-      src[u] = nullptr;
-      dst[u] = nullptr;
-      return;
+      // reported by the CTA whose share holds the pair's first vector
+      if (a == 0 && !(c & 1) && threadIdx.x == 0) set_status(status, -7 /* PA_ERR_BAD_BLOCK */);
+      continue;
     }
-    src[u] = ((copy[u] & 1) ? src_v : src_k) + s * vecs_per_block;
-    dst[u] = ((copy[u] & 1) ? dst_v : dst_k) + d * vecs_per_block;
-  };
+    const uint4* src = ((c & 1) ? src_v : src_k) + s * vecs_per_block;
+    uint4* dst = ((c & 1) ? dst_v : dst_k) + d * vecs_per_block;
+    for (int64_t i = a + threadIdx.x; i < b; i += kCopyThreads * kUnroll) {
+      uint4 r[kUnroll];
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    i[u] = u * kCopyThreads + threadIdx.x;
-    const int64_t j = lo + i[u];
-    copy[u] = static_cast<int>(j / vecs_per_block);
-    off[u] = static_cast<int>(j - static_cast<int64_t>(copy[u]) * vecs_per_block);
-    if (i[u] < n) endpoints(u);
-  }
-  while (i[0] < n) {
-    uint4 r[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      if (i[u] < n && src[u]) r[u] = src[u][off[u]];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (i[u] < n) {
-        if (dst[u]) {
-          dst[u][off[u]] = r[u];
-        } else if (off[u] == 0 && !(copy[u] & 1)) {
-          set_status(status, -7 /* PA_ERR_BAD_BLOCK */);
-        }
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t j = i + u * kCopyThreads;
+        if (j < b) r[u] = src[j];
       }
-      i[u] += kStep;
-      off[u] += kStep;
-      if (off[u] >= vpb) {
-        while (off[u] >= vpb) {
-          off[u] -= vpb;
-          ++copy[u];
-        }
-        if (i[u] < n) endpoints(u);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t j = i + u * kCopyThreads;
+        if (j < b) dst[j] = r[u];
       }
     }
   }
@@ -105,9 +78,7 @@ cudaError_t launch_copy_blocks(const void* src_k, const void* src_v, void* dst_k
                                cudaStream_t stream) {
   const int64_t vecs = block_bytes / 16;
   const int64_t total = static_cast<int64_t>(num_pairs) * 2 * vecs;
-  // 32-bit offsets in the kernel: a block under 32 GB, a call under 16 TB
-  if (total <= 0 || vecs >= (int64_t{1} << 31) || total >= (int64_t{1} << 40))
-    return cudaErrorInvalidValue;
+  if (total <= 0) return cudaErrorInvalidValue;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

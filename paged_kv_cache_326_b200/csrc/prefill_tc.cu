@@ -362,9 +362,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     // our blocks still in the ring
     for (int jj = stored; stores && ok && jj < issued; ++jj) ok = store_block(jj);
     if (lane == 0) {
-      // drain: the stores must complete, and the copies in flight land,
-      // before this CTA's memory goes
-      tc::bulk_wait_all();
+      // drain: the stores must have read their tiles, and the copies in
+      // flight landed, before this CTA's shared memory goes (the stores'
+      // global writes complete with the grid, like any other store)
+      tc::bulk_wait_read_all();
       mbar_wait_bounded(&bar_q, 0, kTcDrainNs);
       for (int j = issued > kTcStages ? issued - kTcStages : 0; j < issued; ++j)
         mbar_wait_bounded(&bar_full[j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);

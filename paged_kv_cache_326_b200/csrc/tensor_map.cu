@@ -11,6 +11,19 @@ namespace pa {
 
 namespace {
 
+#ifndef PA_TMA_L2_PROMOTION
+#define PA_TMA_L2_PROMOTION 256
+#endif
+// L2 promotion of the tiled loads' requests (0, 64, 128 or 256 bytes).
+CUtensorMapL2promotion l2_promotion() {
+  switch (PA_TMA_L2_PROMOTION) {
+    case 0: return CU_TENSOR_MAP_L2_PROMOTION_NONE;
+    case 64: return CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+    case 128: return CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+    default: return CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+  }
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -55,7 +68,7 @@ bool encode_tiled_map(CUtensorMap* map, const void* base, CUtensorMapDataType ty
   }
   return fn(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, b, e,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            l2_promotion(), CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace pa

@@ -52,7 +52,7 @@ def test_replayed_decode_matches_oracle_each_time(P, kind):
     if kv is None:
         ws_bytes = P.pa_paged_attn_decode_workspace_size(S, H, D, 16, live.max_blocks_per_seq)
     else:
-        ws_bytes = P.pa_paged_attn_decode_gqa_workspace_size(S, H, kv, D, 16,
+        ws_bytes = P.binding.pa_paged_attn_decode_gqa_workspace_size(S, H, kv, D, 16,
                                                              live.max_blocks_per_seq)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
 
