@@ -54,9 +54,9 @@ TRAFFIC = {
          "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
     "opt13b_batch64_fp8": (
         os.path.join(ROOT, "profiles", "paged_decode_fp8_opt13b_batch64_traffic.json"),
-        ["paged_kv_cache_326_b200/csrc/paged_attn_decode.cu",
+        ["paged_kv_cache_326_b200/csrc/paged_attn_decode_mma_fp8.cu",
          "paged_kv_cache_326_b200/csrc/decode_common.cuh",
-         "paged_kv_cache_326_b200/csrc/fp8.cuh",
+         "paged_kv_cache_326_b200/csrc/fp8.cuh", "paged_kv_cache_326_b200/csrc/mma_ptx.cuh",
          "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
     # the shared-prefix call: prefix pass + tail pass + merge, summed
     "shared_prefix": (
