@@ -17,6 +17,12 @@ std::atomic<int64_t> g_gqa_kernel{0};
 std::atomic<int64_t> g_prefill_kernel{0};
 std::atomic<int64_t> g_prefix_key_bits{64};
 std::atomic<int64_t> g_fp8_kernel{0};
+#ifndef PA_TC_FUSED_STORE
+#define PA_TC_FUSED_STORE 1
+#endif
+// 1: the tcgen05 prompt-phase kernel stores the prompts' keys and values
+// from its own tiles; 0: a separate cache write runs first.
+constexpr bool kPrefillFusedStore = PA_TC_FUSED_STORE != 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -257,7 +263,7 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
       return PA_ERR_INVALID;
     // the tcgen05 kernel stores them from its own tiles; otherwise a cache
     // write runs first
-    fused_store = tc && pa::prefill_tc_paged_ok(block_size, num_blocks);
+    fused_store = kPrefillFusedStore && tc && pa::prefill_tc_paged_ok(block_size, num_blocks);
     if (!fused_store) {
       const int rc = from_cuda(pa::launch_kv_cache_write(k, v, k_cache, v_cache, slot_mapping,
                                                          num_tokens, num_kv_heads, head_dim,

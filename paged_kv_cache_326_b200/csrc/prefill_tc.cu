@@ -83,6 +83,12 @@ constexpr int64_t kTcDrainNs = 1000000000;
 // many are computed by the FMA-pipe polynomial (exp2poly.cuh), the rest by
 // the exponential unit.
 constexpr int kTcPolyPairs = PA_TC_POLY_PAIRS;
+#ifndef PA_TC_PACKED
+#define PA_TC_PACKED 1
+#endif
+// 1: the softmax's scores go through packed fp32 instructions two at a time
+// and three-input maxima; 0: one score per instruction.
+constexpr bool kTcPacked = PA_TC_PACKED != 0;
 #ifndef PA_TC_EARLY_S
 #define PA_TC_EARLY_S 1
 #endif
@@ -495,12 +501,17 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
         }
         below = j * kTcBN + kTcBN - 1 <= q0 + t * kTcBM + (warp & 3) * 32;
       }
-      // four independent partial maxima of three-input maxima
+      // four independent partial maxima (of three-input maxima)
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if constexpr (kTcPacked) {
 #pragma unroll
-      for (int c = 0; c < kTcBN; c += 8) {
+        for (int c = 0; c < kTcBN; c += 8) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
+          for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kTcBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
       }
       // base-2 logits: the scale (> 0) is applied in the exponent
       const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
@@ -550,9 +561,16 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       // weights come from the FMA-pipe polynomial and the rest from the
       // exponential unit, so the two units share the work.
       auto weights = [&](int c, bool poly) {
-        const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sc2, nm2);
-        const float2 pw = poly ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
-        ls[(c >> 1) & 1] = __fadd2_rn(ls[(c >> 1) & 1], pw);
+        float2 pw;
+        if constexpr (kTcPacked) {
+          const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sc2, nm2);
+          pw = poly ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          ls[(c >> 1) & 1] = __fadd2_rn(ls[(c >> 1) & 1], pw);
+        } else {
+          pw = make_float2(fast_exp2(fmaf(sv[c], p.scale_log2, -mm)),
+                           fast_exp2(fmaf(sv[c + 1], p.scale_log2, -mm)));
+          ls[(c >> 1) & 1].x += pw.x + pw.y;
+        }
         ph[c / 2] = Elem<T>::from_float2(pw.x, pw.y);
         if constexpr (BF16) {
           const float2 back = Elem<T>::to_float2(ph[c / 2]);
