@@ -18,7 +18,7 @@ std::atomic<int64_t> g_prefill_kernel{0};
 std::atomic<int64_t> g_prefix_key_bits{64};
 std::atomic<int64_t> g_fp8_kernel{0};
 #ifndef PA_TC_FUSED_STORE
-#define PA_TC_FUSED_STORE 1
+#define PA_TC_FUSED_STORE 0
 #endif
 // 1: the tcgen05 prompt-phase kernel stores the prompts' keys and values
 // from its own tiles; 0: a separate cache write runs first.

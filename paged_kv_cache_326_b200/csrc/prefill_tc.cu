@@ -77,7 +77,7 @@ constexpr uint32_t kColS = 0, kColPhi = 64, kColPlo = 96, kColO = 128;
 constexpr uint32_t kTileCols = 256, kTmemCols = 512;
 constexpr int64_t kTcDrainNs = 1000000000;
 #ifndef PA_TC_POLY_PAIRS
-#define PA_TC_POLY_PAIRS 2
+#define PA_TC_POLY_PAIRS 0
 #endif
 // Of every four pairs of softmax weights in a block below the diagonal, this
 // many are computed by the FMA-pipe polynomial (exp2poly.cuh), the rest by
@@ -90,7 +90,7 @@ constexpr int kTcPolyPairs = PA_TC_POLY_PAIRS;
 // and three-input maxima; 0: one score per instruction.
 constexpr bool kTcPacked = PA_TC_PACKED != 0;
 #ifndef PA_TC_EARLY_S
-#define PA_TC_EARLY_S 1
+#define PA_TC_EARLY_S 0
 #endif
 // 1: the softmax warps release S as soon as they hold the scores in
 // registers, and the next block's S is issued then, ahead of this block's

@@ -40,10 +40,35 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                : "memory");
 }
 
-// One probe of the barrier's phase; the hardware may suspend the thread for a
-// bounded time before answering false.
+#ifndef PA_MBAR_TEST_WAIT
+#define PA_MBAR_TEST_WAIT 0
+#endif
+#ifndef PA_MBAR_SUSPEND_NS
+#define PA_MBAR_SUSPEND_NS 0
+#endif
+// One probe of the barrier's phase.  try_wait may suspend the thread for a
+// bounded time before answering false (PA_MBAR_SUSPEND_NS > 0: at most that
+// many nanoseconds, as a hint); test_wait (PA_MBAR_TEST_WAIT=1) answers at
+// once.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
+#if PA_MBAR_SUSPEND_NS > 0
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(static_cast<uint32_t>(PA_MBAR_SUSPEND_NS))
+      : "memory");
+#elif PA_MBAR_TEST_WAIT
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
@@ -51,6 +76,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
+#endif
   return ok != 0;
 }
 
