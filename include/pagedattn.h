@@ -182,6 +182,36 @@ int pa_decode_step(void* out, const void* q, const void* k, const void* v, void*
                    pa_stream_t stream);
 
 /*
+ * pa_decode_step_fp8 — pa_decode_step over 8-bit caches: the quantizing
+ * write of pa_kv_cache_write_fp8 for one new token per text, then the
+ * attention of pa_paged_attn_decode_fp8, in one launch (plus the merge)
+ * ("The KV Cache and PagedAttention", section "What Came After": one byte a
+ * number; "KV cache", section "How it works": the new token's key and value
+ * join the cache and take part in its own attention).
+ *
+ *   k, v           [num_seqs][num_heads][head_dim] dt (fp16 or bf16): each
+ *                  text's new token; stored as the codes of k / k_scale and
+ *                  v / v_scale
+ *   k_cache,v_cache 8-bit pools [num_blocks][num_heads][block_size][head_dim]
+ *   k_scale, v_scale finite and > 0 (else PA_ERR_INVALID)
+ *   other arguments as for pa_decode_step (workspace as for
+ *                  pa_paged_attn_decode_fp8).  Multi-head only.
+ *
+ * Result: the pool afterwards and `out` are exactly those of
+ * pa_kv_cache_write_fp8 followed by pa_paged_attn_decode_fp8 on the CUDA
+ * cores (PA_OPT_FP8_KERNEL 1), under the conditions of pa_decode_step.  The
+ * attention quantizes position context_lens[s] - 1 from k[s], v[s] itself,
+ * with the write's arithmetic, so the launch never waits on its own write.
+ * Runs on the CUDA-core kernel.  Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ */
+int pa_decode_step_fp8(void* out, const void* q, const void* k, const void* v, void* k_cache,
+                       void* v_cache, const int64_t* slot_mapping, const int32_t* block_tables,
+                       const int32_t* context_lens, float scale, float k_scale, float v_scale,
+                       int num_seqs, int num_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt, void* workspace,
+                       size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
+
+/*
  * pa_paged_attn_decode_shared_workspace_size — device scratch bytes that
  * pa_paged_attn_decode_shared needs for these sizes on the current device.
  * Host only.  Returns 0 for unsupported sizes.
@@ -319,7 +349,8 @@ int pa_kv_cache_write_fp8(const void* k, const void* v, void* k_cache, void* v_c
  *   q, out         [num_seqs][num_heads][head_dim] dt (fp16 or bf16)
  *   k_cache,v_cache 8-bit pools; the workspace is
  *                  pa_paged_attn_decode_workspace_size(...) bytes (the same
- *                  sizes as the 16-bit call).  Multi-head only.  Other
+ *                  sizes as the 16-bit call).  Multi-head; grouped-query
+ *                  pools go through pa_paged_attn_decode_fp8_gqa.  Other
  *                  arguments and errors as for pa_paged_attn_decode.
  * Each chunk of work is 4096/head_dim tokens (32 at head_dim 128), so every
  * copy still moves 4 KB of keys and 4 KB of values.  With fp16 queries,
@@ -333,6 +364,30 @@ int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, cons
                              int num_heads, int head_dim, int block_size, int max_blocks_per_seq,
                              int64_t num_blocks, pa_dtype dt, void* workspace,
                              size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_paged_attn_decode_fp8_gqa — pa_paged_attn_decode_fp8 over 8-bit pools
+ * of num_kv_heads heads shared by num_heads query heads ("The KV Cache and
+ * PagedAttention", section "What Came After": heads that share a key/value
+ * set, and one byte a number, side by side): query head h reads key/value
+ * head h / (num_heads / num_kv_heads), with the formula of
+ * pa_paged_attn_decode_fp8.
+ *   k_cache,v_cache [num_blocks][num_kv_heads][block_size][head_dim] uint8
+ *                  codes (written by pa_kv_cache_write_fp8 with num_heads =
+ *                  num_kv_heads)
+ *   workspace      pa_paged_attn_decode_gqa_workspace_size(...) bytes
+ * Runs on the CUDA cores: each unit of work carries up to 4 query heads of
+ * one group (the largest of 4, 2, 1 that divides the group), so every code
+ * read serves them all.  num_heads must be a multiple of num_kv_heads (else
+ * PA_ERR_INVALID); other arguments and errors as for pa_paged_attn_decode_fp8.
+ */
+int pa_paged_attn_decode_fp8_gqa(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, float k_scale,
+                                 float v_scale, int num_seqs, int num_heads, int num_kv_heads,
+                                 int head_dim, int block_size, int max_blocks_per_seq,
+                                 int64_t num_blocks, pa_dtype dt, void* workspace,
+                                 size_t workspace_bytes, int32_t* d_status, pa_stream_t stream);
 
 /*
  * pa_prefill — the prompt phase: every prompt's tokens attend causally over

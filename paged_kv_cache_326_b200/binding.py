@@ -74,12 +74,17 @@ _SIGNATURES = {
                                         _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
                               _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
+    "pa_decode_step_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _f32, _f32,
+                                  _i32, _i32, _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_paged_attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
                                             _i32, _i32, _i64, _i32, _vp, _vp]),
     "pa_kv_cache_write_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _f32, _f32, _i32, _i32, _i32, _i32,
                                      _i64, _i32, _vp, _vp]),
     "pa_paged_attn_decode_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _f32, _f32, _i32, _i32,
                                         _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp, _vp]),
+    "pa_paged_attn_decode_fp8_gqa": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _f32, _f32, _i32,
+                                            _i32, _i32, _i32, _i32, _i32, _i64, _i32, _vp, _sz,
+                                            _vp, _vp]),
     "pa_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _f32, _i32,
                           _i32, _i32, _i32, _i64, _i32, _vp, _vp]),
     "pa_prefill_with_prefix": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
@@ -224,25 +229,33 @@ def pa_paged_attn_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.
                              context_lens: torch.Tensor, scale: float, k_scale: float,
                              v_scale: float, workspace: Optional[torch.Tensor] = None,
                              status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """out, q: [S][H][D] fp16/bf16; 8-bit caches [N][H][B][D]."""
+    """out, q: [S][H][D] fp16/bf16; 8-bit caches [N][H_kv][B][D].  H_kv == H
+    is multi-head attention (pa_paged_attn_decode_fp8); a divisor of H is
+    grouped-query attention (pa_paged_attn_decode_fp8_gqa)."""
     S, H, D = q.shape
-    N, H2, B, D2 = k_cache.shape
-    if out.shape != q.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
-        raise ValueError("shape mismatch")
+    N, Hkv, B, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D or H % Hkv:
+        raise ValueError("shape mismatch (num_heads must be a multiple of num_kv_heads)")
     if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
         raise ValueError("block_tables must be [S][max_blocks], context_lens [S]")
     if out.dtype != q.dtype:
         raise TypeError("q and out must share a dtype")
     MB = block_tables.shape[1]
     if workspace is None:
-        workspace = workspace_for(q, B, MB)
-    code = lib().pa_paged_attn_decode_fp8(
-        _cuda(out, "out"), _cuda(q, "q"), _codes(k_cache, "k_cache"), _codes(v_cache, "v_cache"),
-        _cuda(block_tables, "block_tables", torch.int32),
-        _cuda(context_lens, "context_lens", torch.int32), float(scale), float(k_scale),
-        float(v_scale), S, H, D, B, MB, N, _dtype_code(q), _cuda(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(), _status_ptr(status), _stream(stream, q.device))
-    _check(code, "pa_paged_attn_decode_fp8")
+        workspace = workspace_for(q, B, MB, Hkv)
+    args = (_cuda(out, "out"), _cuda(q, "q"), _codes(k_cache, "k_cache"),
+            _codes(v_cache, "v_cache"), _cuda(block_tables, "block_tables", torch.int32),
+            _cuda(context_lens, "context_lens", torch.int32), float(scale), float(k_scale),
+            float(v_scale), S, H)
+    tail = (D, B, MB, N, _dtype_code(q), _cuda(workspace, "workspace"),
+            workspace.numel() * workspace.element_size(), _status_ptr(status),
+            _stream(stream, q.device))
+    if Hkv == H:
+        code = lib().pa_paged_attn_decode_fp8(*args, *tail)
+        _check(code, "pa_paged_attn_decode_fp8")
+    else:
+        code = lib().pa_paged_attn_decode_fp8_gqa(*args, Hkv, *tail)
+        _check(code, "pa_paged_attn_decode_fp8_gqa")
     return out
 
 
@@ -586,6 +599,42 @@ def pa_decode_step(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch
         _dtype_code(q), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _status_ptr(status), _stream(stream, q.device))
     _check(code, "pa_decode_step")
+    return out
+
+
+def pa_decode_step_fp8(out: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                       k_cache: torch.Tensor, v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                       block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                       k_scale: float, v_scale: float, workspace: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pa_decode_step over 8-bit caches [N][H][B][D] (uint8 codes): each
+    text's new token is stored quantized and attended in one launch.
+    q, k, v, out: [S][H][D] fp16/bf16; slot_mapping [S] int64."""
+    S, H, D = q.shape
+    N, H2, B, D2 = k_cache.shape
+    if (out.shape != q.shape or k.shape != q.shape or v.shape != q.shape
+            or v_cache.shape != k_cache.shape or (H2, D2) != (H, D)):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S][max_blocks], context_lens [S]")
+    if slot_mapping.shape != (S,):
+        raise ValueError("slot_mapping must be [num_seqs]")
+    for t in (out, k, v):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v and out must share a dtype")
+    MB = block_tables.shape[1]
+    if workspace is None:
+        workspace = workspace_for(q, B, MB)
+    code = lib().pa_decode_step_fp8(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"),
+        _codes(k_cache, "k_cache"), _codes(v_cache, "v_cache"),
+        _cuda(slot_mapping, "slot_mapping", torch.int64),
+        _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(context_lens, "context_lens", torch.int32), float(scale), float(k_scale),
+        float(v_scale), S, H, D, B, MB, N, _dtype_code(q), _cuda(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _status_ptr(status),
+        _stream(stream, q.device))
+    _check(code, "pa_decode_step_fp8")
     return out
 
 

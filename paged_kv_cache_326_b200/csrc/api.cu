@@ -242,6 +242,19 @@ int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, cons
                        true, k_scale, v_scale);
 }
 
+int pa_paged_attn_decode_fp8_gqa(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, float k_scale,
+                                 float v_scale, int num_seqs, int num_heads, int num_kv_heads,
+                                 int head_dim, int block_size, int max_blocks_per_seq,
+                                 int64_t num_blocks, pa_dtype dt, void* workspace,
+                                 size_t workspace_bytes, int32_t* d_status, pa_stream_t stream) {
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                       num_blocks, dt, workspace, workspace_bytes, d_status, stream, nullptr,
+                       nullptr, nullptr, true, k_scale, v_scale);
+}
+
 int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_cache,
                void* v_cache, const int64_t* slot_mapping, const int32_t* cu_seqlens,
                int num_seqs, int num_tokens, int max_seqlen, float scale, int num_heads,
@@ -408,6 +421,19 @@ int pa_decode_step(void* out, const void* q, const void* k, const void* v, void*
   return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
                        num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
                        dt, workspace, workspace_bytes, d_status, stream, k, v, slot_mapping);
+}
+
+int pa_decode_step_fp8(void* out, const void* q, const void* k, const void* v, void* k_cache,
+                       void* v_cache, const int64_t* slot_mapping, const int32_t* block_tables,
+                       const int32_t* context_lens, float scale, float k_scale, float v_scale,
+                       int num_seqs, int num_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int64_t num_blocks, pa_dtype dt, void* workspace,
+                       size_t workspace_bytes, int32_t* d_status, pa_stream_t stream) {
+  if (num_seqs != 0 && !slot_mapping) return PA_ERR_INVALID;
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       dt, workspace, workspace_bytes, d_status, stream, k, v, slot_mapping, true,
+                       k_scale, v_scale);
 }
 
 size_t pa_paged_attn_decode_shared_workspace_size(int num_groups, int group_size, int num_heads,

@@ -14,8 +14,12 @@
 // shares cross copy boundaries, and the extra index work per piece costs
 // more than the partial last wave it saves.
 //
-// PA_COPY_STREAMING_STORE=1 writes with st.global.cs (evict-first): the
-// destination is not read again by this kernel.
+// Two other forms measured slower on the same bursts: a CTA per run of
+// pairs with one source, reading it once and writing every destination
+// (29.5 microseconds: too few CTAs left writing), and the run's CTAs each
+// taking one slice of the source for all destinations (23.5).
+// PA_COPY_STREAMING_STORE=1 writes with st.global.cs (evict-first); it
+// measured no different.
 #include <cuda_runtime.h>
 
 #include <cstdint>

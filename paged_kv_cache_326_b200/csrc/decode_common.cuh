@@ -21,6 +21,7 @@
 #include <utility>
 
 #include "dtype.cuh"
+#include "fp8.cuh"
 #include "ptx.cuh"
 
 namespace pa {
@@ -79,6 +80,7 @@ struct DecodeParams {
   const int32_t* context_lens;
   float qk_scale_log2;  // scale * log2(e) (* the keys' scale for an 8-bit cache)
   float v_scale;        // the values' scale for an 8-bit cache, else 1
+  float k_scale;        // the keys' scale for an 8-bit cache, else 1
   int num_seqs;
   int num_heads;      // virtual heads: key/value heads x subsets (the flat order's heads)
   int num_q_heads;    // query heads of q and out
@@ -364,6 +366,39 @@ __device__ __forceinline__ void fused_cache_write(const DecodeParams& p, int w, 
     const int64_t dst = ((blk * Hkv + h) * B + place) * vpr + c;
     kcw[dst] = __ldg(static_cast<const uint4*>(p.k_new) + i);
     vcw[dst] = __ldg(static_cast<const uint4*>(p.v_new) + i);
+  }
+}
+
+// fused_cache_write for an 8-bit cache: each lane takes 8 numbers of a new
+// row and stores their codes (e4m3x8_quantize with the keys' or the values'
+// scale, as the 8-bit cache write does).
+template <typename T, int D, int B>
+__device__ __forceinline__ void fused_cache_write_f8(const DecodeParams& p, int w, int W,
+                                                     int lane) {
+  const int Hkv = p.num_kv_heads;
+  const int vpr = D / 8;
+  const int64_t per_text = static_cast<int64_t>(Hkv) * vpr;
+  const int64_t nvec = per_text * p.num_seqs;
+  const int64_t num_slots = p.num_blocks * B;
+  uint2* kcw = static_cast<uint2*>(const_cast<void*>(p.k_cache));
+  uint2* vcw = static_cast<uint2*>(const_cast<void*>(p.v_cache));
+  for (int64_t i = static_cast<int64_t>(w) * 32 + lane; i < nvec; i += static_cast<int64_t>(W) * 32) {
+    const int64_t s = i / per_text;
+    const int64_t r = i - s * per_text;
+    const int64_t slot = __ldg(p.slot_mapping + s);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (r == 0) set_status(p.status, -9 /* PA_ERR_BAD_SLOT */);
+      continue;
+    }
+    const int64_t h = r / vpr, c = r - (r / vpr) * vpr;
+    const int64_t blk = slot / B, place = slot - blk * B;
+    const int64_t dst = ((blk * Hkv + h) * B + place) * vpr + c;
+    float x[8];
+    unpack8<T>(__ldg(static_cast<const uint4*>(p.k_new) + i), x);
+    kcw[dst] = e4m3x8_quantize(x, p.k_scale);
+    unpack8<T>(__ldg(static_cast<const uint4*>(p.v_new) + i), x);
+    vcw[dst] = e4m3x8_quantize(x, p.v_scale);
   }
 }
 

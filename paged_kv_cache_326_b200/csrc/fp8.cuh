@@ -16,6 +16,21 @@ __device__ __forceinline__ uint16_t e4m3x2_from_floats(float lo, float hi) {
   return r;
 }
 
+// Eight numbers -> their eight codes (low byte first) of x / scale: the
+// quotient in IEEE fp32 (round to nearest), then rounded as above.  The
+// cache write and the one-launch step's new row both use this, so the same
+// inputs give the same codes.
+__device__ __forceinline__ uint2 e4m3x8_quantize(const float (&x)[8], float scale) {
+  uint2 o;
+  o.x = e4m3x2_from_floats(__fdiv_rn(x[0], scale), __fdiv_rn(x[1], scale)) |
+        (static_cast<uint32_t>(e4m3x2_from_floats(__fdiv_rn(x[2], scale),
+                                                  __fdiv_rn(x[3], scale))) << 16);
+  o.y = e4m3x2_from_floats(__fdiv_rn(x[4], scale), __fdiv_rn(x[5], scale)) |
+        (static_cast<uint32_t>(e4m3x2_from_floats(__fdiv_rn(x[6], scale),
+                                                  __fdiv_rn(x[7], scale))) << 16);
+  return o;
+}
+
 // Two codes (low byte first) -> their values as a half2 (exact).
 __device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t x) {
   uint32_t r;

@@ -84,23 +84,10 @@ kv_cache_write_fp8_kernel(const uint4* __restrict__ k, const uint4* __restrict__
     const int64_t place = slot - blk * block_size;
     const int64_t dst = ((blk * num_heads + h) * block_size + place) * vec_per_row + c;
     float x[8];
-    uint2 o;
     unpack8<T>(__ldg(k + i), x);
-    o.x = e4m3x2_from_floats(__fdiv_rn(x[0], k_scale), __fdiv_rn(x[1], k_scale)) |
-          (static_cast<uint32_t>(e4m3x2_from_floats(__fdiv_rn(x[2], k_scale),
-                                                    __fdiv_rn(x[3], k_scale))) << 16);
-    o.y = e4m3x2_from_floats(__fdiv_rn(x[4], k_scale), __fdiv_rn(x[5], k_scale)) |
-          (static_cast<uint32_t>(e4m3x2_from_floats(__fdiv_rn(x[6], k_scale),
-                                                    __fdiv_rn(x[7], k_scale))) << 16);
-    k_cache[dst] = o;
+    k_cache[dst] = e4m3x8_quantize(x, k_scale);
     unpack8<T>(__ldg(v + i), x);
-    o.x = e4m3x2_from_floats(__fdiv_rn(x[0], v_scale), __fdiv_rn(x[1], v_scale)) |
-          (static_cast<uint32_t>(e4m3x2_from_floats(__fdiv_rn(x[2], v_scale),
-                                                    __fdiv_rn(x[3], v_scale))) << 16);
-    o.y = e4m3x2_from_floats(__fdiv_rn(x[4], v_scale), __fdiv_rn(x[5], v_scale)) |
-          (static_cast<uint32_t>(e4m3x2_from_floats(__fdiv_rn(x[6], v_scale),
-                                                    __fdiv_rn(x[7], v_scale))) << 16);
-    v_cache[dst] = o;
+    v_cache[dst] = e4m3x8_quantize(x, v_scale);
   }
 }
 

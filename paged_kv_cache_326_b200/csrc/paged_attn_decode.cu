@@ -109,7 +109,6 @@ paged_decode_kernel(const DecodeParams p) {
   constexpr int STRIDE = stage_bytes(D, GS);
   constexpr int AREA = warp_area_bytes(D, STAGES, GS);
   static_assert(CH % TPI == 0 && (CH % B == 0 || B % CH == 0), "shape");
-  static_assert(!(F8 && FUSED), "the one-launch step stores T");
   // one 16-byte vector of cache numbers -> VEC floats
   auto load_vec = [](const uint8_t* src, float (&f)[VEC]) {
     const uint4 v = *reinterpret_cast<const uint4*>(src);
@@ -152,7 +151,8 @@ paged_decode_kernel(const DecodeParams p) {
   // slots, so each warp does its share whenever it has a moment: right after
   // issuing its first copies, while it waits for them.
   auto fused_write = [&]() {
-    if constexpr (FUSED) fused_cache_write<D, B>(p, w, W, lane);
+    if constexpr (FUSED && F8) fused_cache_write_f8<T, D, B>(p, w, W, lane);
+    else if constexpr (FUSED) fused_cache_write<D, B>(p, w, W, lane);
   };
   if (w >= W) {
     if (wait_at_exit) griddep_wait();
@@ -233,17 +233,18 @@ paged_decode_kernel(const DecodeParams p) {
       if (bad) set_status(p.status, -7 /* PA_ERR_BAD_BLOCK */);
       fence_proxy_async_smem();
       *flag = bad ? 1 : 0;
+      // Fused step: the chunk holding the text's last position takes that
+      // row from the new k/v instead of the pool (copied here for a 16-bit
+      // cache; for an 8-bit cache the consumer writes its codes).
+      const bool new_row = FUSED && j * CH + nvalid == len;
+      const int pool_rows = nvalid - (new_row ? 1 : 0);
       const uint32_t qbytes = first ? GS * D * 2 : 0;
-      const uint32_t kvbytes = bad ? 0 : 2u * nvalid * ROWB;
+      const uint32_t kvbytes = bad ? 0 : 2u * (F8 ? pool_rows : nvalid) * ROWB;
       mbar_arrive_expect_tx(&bars[st], qbytes + kvbytes);
       if (first)
         bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D, GS * D * 2, &bars[st],
                       policy);
       if (!bad) {
-        // Fused step: the chunk holding the text's last position takes that
-        // row from the new k/v instead of the pool.
-        const bool new_row = FUSED && j * CH + nvalid == len;
-        const int pool_rows = nvalid - (new_row ? 1 : 0);
         if constexpr (CH >= B) {
 #pragma unroll
           for (int k = 0; k < NB; ++k) {
@@ -262,7 +263,7 @@ paged_decode_kernel(const DecodeParams p) {
             bulk_copy_g2s(sV, vc + off, pool_rows * ROWB, &bars[st], policy);
           }
         }
-        if (new_row) {
+        if (!F8 && new_row) {
           const int64_t src_off = (static_cast<int64_t>(s) * Hkv + kv_head(h)) * D;
           bulk_copy_g2s(sK + pool_rows * ROWB, static_cast<const T*>(p.k_new) + src_off, ROWB,
                         &bars[st], policy);
@@ -339,6 +340,25 @@ paged_decode_kernel(const DecodeParams p) {
       }
     }
     const int nvalid = bad ? 0 : min(CH, len - j * CH);
+    if constexpr (F8 && FUSED) {
+      // The one-launch step's new row over an 8-bit cache: its codes (the
+      // cache write's quantization) take the stage row after the pool rows,
+      // which the copies left empty.  The refill of this stage is ordered
+      // after these writes by the proxy fence its issue begins with.
+      if (nvalid > 0 && j * CH + nvalid == len) {
+        const int64_t src = (static_cast<int64_t>(s) * Hkv + kv_head(h)) * D;
+        uint8_t* rk = const_cast<uint8_t*>(sK) + (nvalid - 1) * ROWB;
+        uint8_t* rv = const_cast<uint8_t*>(sV) + (nvalid - 1) * ROWB;
+        for (int c = lane; c < D / 8; c += 32) {
+          float x[8];
+          unpack8<T>(__ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + src) + c), x);
+          *reinterpret_cast<uint2*>(rk + c * 8) = e4m3x8_quantize(x, p.k_scale);
+          unpack8<T>(__ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + src) + c), x);
+          *reinterpret_cast<uint2*>(rv + c * 8) = e4m3x8_quantize(x, p.v_scale);
+        }
+        __syncwarp();
+      }
+    }
 
     // scores (base-2 logits) of this lane's token rows, for every head
     float sc[GS][ITERS];
@@ -565,6 +585,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   // query; the values' scale multiplies the output
   p.qk_scale_log2 = a.scale * 1.4426950408889634f * (F8 ? a.k_scale : 1.f);
   p.v_scale = F8 ? a.v_scale : 1.f;
+  p.k_scale = F8 ? a.k_scale : 1.f;
   p.num_seqs = a.num_seqs;
   p.num_heads = hl.vheads;
   p.num_q_heads = a.num_heads;
@@ -626,9 +647,16 @@ cudaError_t dispatch_dim(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
 
 template <typename T>
 cudaError_t dispatch_heads(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t stream) {
-  if (a.fp8)  // 8-bit cache: multi-head, two calls
-    return hl.gs == 1 && !a.slot_mapping ? dispatch_dim<T, false, 1, true>(a, hl, stream)
-                                         : cudaErrorInvalidValue;
+  if (a.fp8) {  // 8-bit cache; query heads per unit as for 16-bit
+    if (a.slot_mapping)  // one-launch step: multi-head only
+      return hl.gs == 1 ? dispatch_dim<T, true, 1, true>(a, hl, stream) : cudaErrorInvalidValue;
+    switch (hl.gs) {
+      case 1: return dispatch_dim<T, false, 1, true>(a, hl, stream);
+      case 2: return dispatch_dim<T, false, 2, true>(a, hl, stream);
+      case 4: return dispatch_dim<T, false, 4, true>(a, hl, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   if (a.slot_mapping)  // fused decode step: multi-head only
     return hl.gs == 1 ? dispatch_dim<T, true, 1, false>(a, hl, stream) : cudaErrorInvalidValue;
   switch (hl.gs) {
@@ -652,7 +680,15 @@ const void* kernel_for(int block_size, bool bf16) {
 
 template <int D>
 const void* kernel_for_variant(int block_size, bool bf16, bool fused, int gs, bool fp8) {
-  if (fp8) return gs == 1 && !fused ? kernel_for<D, false, 1, true>(block_size, bf16) : nullptr;
+  if (fp8) {
+    if (fused) return gs == 1 ? kernel_for<D, true, 1, true>(block_size, bf16) : nullptr;
+    switch (gs) {
+      case 1: return kernel_for<D, false, 1, true>(block_size, bf16);
+      case 2: return kernel_for<D, false, 2, true>(block_size, bf16);
+      case 4: return kernel_for<D, false, 4, true>(block_size, bf16);
+      default: return nullptr;
+    }
+  }
   if (fused) return gs == 1 ? kernel_for<D, true, 1, false>(block_size, bf16) : nullptr;
   switch (gs) {
     case 1: return kernel_for<D, false, 1, false>(block_size, bf16);
@@ -690,8 +726,7 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
   // 16-bit / 8-bit cache
   for (int variant = 0; variant < 8; ++variant) {
     const bool bf16 = variant & 1, fused = variant & 2, fp8 = variant & 4;
-    if ((fused || fp8) && hl.gs != 1) continue;
-    if (fused && fp8) continue;
+    if (fused && hl.gs != 1) continue;
     if (fp8 && !with_fp8) continue;
     const void* k = head_dim == 128 ? kernel_for_variant<128>(block_size, bf16, fused, hl.gs, fp8)
                                     : kernel_for_variant<64>(block_size, bf16, fused, hl.gs, fp8);

@@ -12,10 +12,13 @@
 // positions after them.
 //
 // How (FlashAttention-4's arrangement on sm_100a): one CTA takes two tiles of
-// 128 queries of one (prompt, head), 256 consecutive queries, and runs ten
+// 128 queries of one (prompt, head), 256 consecutive queries, and runs twelve
 // warps with separate jobs:
-//   * warp 9 loads: Q of both tiles once, then each 64-key block of K and V
-//     into a 3-stage ring, by tiled TMA with the 128-byte swizzle: the new
+//   * warp 9 loads: Q of both tiles once, then each block of kTcBN keys
+//     (128; 64 as a build option) of K and of V, each into a ring of its own
+//     of 2 slots (3 for 64-key blocks): a K slot refills once both tiles' S
+//     have read it, a step before the block's V slot frees, which gives the
+//     loads about two steps of lead.  Tiled TMA with the 128-byte swizzle: the new
 //     tokens from q, k, v (the [T][H][D] tensors seen as (D, H, T); boxes
 //     64 x 1 x rows), the stored prefix from the cache pools (seen as
 //     (D, B, H, N); one box of 64 x B rows per physical block, found in the
@@ -24,28 +27,32 @@
 //     of the tiles already in shared memory, one box per physical block, when
 //     the block's slots fill whole physical blocks in order (the usual case),
 //     else row by row from the warp's lanes;
-//   * warp 8 (one thread) issues the tensor-core products, tcgen05.mma
-//     kind::f16, accumulating in tensor memory (TMEM): S_t = Q_t K^T (both
-//     operands K-major in shared memory) and O_t += P_t V (P_t from TMEM, V
-//     MN-major in shared memory), in the order S0, S1, then per block PV0,
-//     S0', PV1, S1': while one tile's softmax runs, the tensor pipe works on
-//     the other tile's products;
+//   * warp 8 (lane 0 issuing, the whole warp running the loop) issues the
+//     tensor-core products, tcgen05.mma kind::f16, accumulating in tensor
+//     memory (TMEM): S_t = Q_t K^T (both operands K-major in shared memory)
+//     and O_t += P_t V (P_t from TMEM, V MN-major in shared memory), in the
+//     order S0, S1, then per block PV0, S0', PV1, S1': while one tile's
+//     softmax runs, the tensor pipe works on the other tile's products;
 //   * warps 0-3 and 4-7: the softmax of tile 0 and tile 1, one thread per
 //     query row (its warp's 32 TMEM lanes), so the row max and sum stay in
-//     the thread.  Base 2; the running max is raised only when a score
-//     passes it by more than 2^8, which then rescales that row of O in TMEM.
-//     Two scores per packed fp32 instruction, maxima three at a time; in
-//     blocks with no masked score half of the weights come from an FMA-pipe
-//     polynomial (exp2poly.cuh) and half from the exponential unit, which
-//     alone would take as long as the products.  P (and for bf16 the rest
-//     P - P_hi, so P enters as about 16 significant bits) goes back to TMEM
-//     as packed 16-bit pairs.
+//     the thread.  The row's scores are read from TMEM once (a build option
+//     reads them twice, for the max and for the weights, 32 at a time, to
+//     spare registers); then the max, then the weights.  Base 2; the running max is raised only
+//     when a score passes it by more than 2^8, which then rescales that row
+//     of O in TMEM.  Two scores per packed fp32 instruction, maxima three at
+//     a time; a build option moves a share of the weights of unmasked blocks
+//     to an FMA-pipe polynomial (exp2poly.cuh).  P (and for bf16 the rest
+//     P - P_hi, so P enters as about 16 significant bits) goes back into the
+//     S columns it was computed from, as packed 16-bit pairs.
 //   * After its last block each softmax thread divides its row of O by its
 //     sum and stores it.
-// Barriers: per stage full (TMA bytes) and empty (last product that reads
-// it); per tile S ready, P ready (128 arrivals) and O done.  TMEM loads are
-// issued in groups of four under one wait.  TMEM per tile:
-// S 64 columns, P 32 + 32, O head_dim; 512 in all, one CTA per SM.
+// Barriers: per ring slot, for K and for V, full (TMA bytes) and empty (the
+// last product that reads it); per tile S ready, P ready (128 arrivals) and
+// O done.  TMEM per tile:
+// S (and P over it) kTcBN columns, O head_dim, 256 in all; 512 for the two
+// tiles, one CTA per SM.  Blocks of 128 keys halve the handoffs per product
+// (every wait on a completed barrier still costs over a hundred cycles) and
+// give S products of N = 128, which the tensor pipe runs at full rate.
 // Every wait is bounded: a wait that gives up records PA_ERR_TIMEOUT and
 // raises a CTA-wide abort flag; each role then drains what it issued
 // (bounded), TMEM is freed and the CTA returns.
@@ -68,12 +75,32 @@ namespace pa {
 namespace {
 
 constexpr int kTcBM = 128;      // queries per tile (MMA M)
-constexpr int kTcBN = 64;       // keys per block (MMA N of S, K of P V)
+#ifndef PA_TC_BN
+#define PA_TC_BN 128
+#endif
+constexpr int kTcBN = PA_TC_BN;   // keys per block (MMA N of S, K of P V): 64 or 128
+static_assert(kTcBN == 64 || kTcBN == 128, "blocks of 64 or 128 keys");
 constexpr int kTcTiles = 2;     // query tiles per CTA
-constexpr int kTcStages = 3;    // K/V ring depth
-constexpr int kTcThreads = 320; // 8 softmax warps, the MMA warp, the load warp
+constexpr int kTcStages = kTcBN == 128 ? 2 : 3;  // K/V ring depth (64 KB or 32 KB a stage)
+// 8 softmax warps (warpgroups 0 and 1), then warpgroup 2: the MMA warp, the
+// load warp and two idle warps.  The launch gives every thread 168 registers
+// (384 x 168 of the SM's 65,536); warpgroup 2 then lowers to kTcRegsLow and
+// the softmax warpgroups raise to kTcRegsHigh:
+// 2 x 128 x 208 + 128 x 80 = 63,488 <= 64,512 (the split at which neither
+// side spills).
+constexpr int kTcThreads = 384;
 constexpr int kMmaWarp = 8, kLoadWarp = 9;
-constexpr uint32_t kColS = 0, kColPhi = 64, kColPlo = 96, kColO = 128;
+#ifndef PA_TC_REGS_HIGH
+#define PA_TC_REGS_HIGH 208
+#endif
+#ifndef PA_TC_REGS_LOW
+#define PA_TC_REGS_LOW 80
+#endif
+constexpr uint32_t kTcRegsHigh = PA_TC_REGS_HIGH, kTcRegsLow = PA_TC_REGS_LOW;
+static_assert(2 * 128 * kTcRegsHigh + 128 * kTcRegsLow <= kTcThreads * 168, "register split");
+// TMEM columns of a tile: S from kColS (kTcBN of them), P written over S
+// (see the softmax), O from kColO.
+constexpr uint32_t kColS = 0, kColO = 128;
 constexpr uint32_t kTileCols = 256, kTmemCols = 512;
 constexpr int64_t kTcDrainNs = 1000000000;
 #ifndef PA_TC_POLY_PAIRS
@@ -89,14 +116,14 @@ constexpr int kTcPolyPairs = PA_TC_POLY_PAIRS;
 // 1: the softmax's scores go through packed fp32 instructions two at a time
 // and three-input maxima; 0: one score per instruction.
 constexpr bool kTcPacked = PA_TC_PACKED != 0;
-#ifndef PA_TC_EARLY_S
-#define PA_TC_EARLY_S 0
+
+#ifndef PA_TC_ONE_LOAD
+#define PA_TC_ONE_LOAD 1
 #endif
-// 1: the softmax warps release S as soon as they hold the scores in
-// registers, and the next block's S is issued then, ahead of this block's
-// P V; each softmax waits for the previous P V only before it stores P and
-// rescales O.  0: S(j+1) is issued after P(j) V.
-constexpr bool kTcEarlyS = PA_TC_EARLY_S != 0;
+// 1: the softmax reads a row's scores from TMEM once, all kTcBN of them into
+// registers (568 against 548 TFLOP/s on the 16 x 2,048-token step); 0:
+// twice (the max, then the weights 32 at a time).
+constexpr bool kTcOneLoad = PA_TC_ONE_LOAD != 0;
 
 // max(a, b, c) in one instruction (three-input max.f32 of sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -109,7 +136,7 @@ template <int D>
 struct TcLayout {
   static constexpr int HALVES = D / 64;           // 64-element (128-byte) column blocks
   static constexpr int Q_BYTES = kTcBM * D * 2;   // one tile of Q: 32 KB at head_dim 128
-  static constexpr int KV_BYTES = kTcBN * D * 2;  // one block of K (or V): 16 KB
+  static constexpr int KV_BYTES = kTcBN * D * 2;  // one block of K (or V): 32 KB at D = 128
   static constexpr int STAGE = 2 * KV_BYTES;      // K block, then V block
   // shared memory asked for (+ 1 KB to align by hand): the head_dim-128
   // amount at every head_dim, so one CTA holds an SM (its 512 TMEM columns)
@@ -153,8 +180,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = smem;                               // tile t at t * Q_BYTES
   uint8_t* sKV = smem + kTcTiles * LY::Q_BYTES;     // stage i at i * STAGE
-  __shared__ uint64_t bar_q, bar_full[kTcStages], bar_empty[kTcStages];
-  __shared__ uint64_t bar_s[kTcTiles], bar_p[kTcTiles], bar_o[kTcTiles], bar_sfree[kTcTiles];
+  // per ring slot, separately for K (index 0) and V (index 1): full (TMA
+  // bytes) and empty (the last product that reads it)
+  __shared__ uint64_t bar_q, bar_full[2][kTcStages], bar_empty[2][kTcStages];
+  __shared__ uint64_t bar_s[kTcTiles], bar_p[kTcTiles], bar_o[kTcTiles];
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
 
@@ -195,16 +224,17 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     abort_flag = 0;
     mbar_init(&bar_q, 1);
 #pragma unroll
-    for (int i = 0; i < kTcStages; ++i) {
-      mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 1);
-    }
+    for (int w = 0; w < 2; ++w)
+#pragma unroll
+      for (int i = 0; i < kTcStages; ++i) {
+        mbar_init(&bar_full[w][i], 1);
+        mbar_init(&bar_empty[w][i], 1);
+      }
 #pragma unroll
     for (int t = 0; t < kTcTiles; ++t) {
       mbar_init(&bar_s[t], 1);
       mbar_init(&bar_p[t], kTcBM);
       mbar_init(&bar_o[t], 1);
-      mbar_init(&bar_sfree[t], kTcBM / 32);  // one arrival per softmax warp
     }
     fence_barrier_init();
   }
@@ -228,6 +258,9 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     return true;
   };
 
+  if (warp >= 8) {
+  // warpgroup 2 lowers its registers, then runs its roles
+  tc::regs_lower<kTcRegsLow>();
   if (warp == kLoadWarp) {
     // ---------------- loads (lane 0) and stores of the new keys ----------------
     if (lane == 0) {
@@ -247,12 +280,16 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
                           a + q0 + t * kTcBM, &bar_q);
     }
     // Key block jj: the stored prefix's block jj (jj < npre), else block
-    // jj - npre of the new keys.
+    // jj - npre of the new keys.  K and V have rings of their own (w = 0, 1),
+    // so a K slot is refilled as soon as both tiles' S products have read
+    // it, a step before the V slot of the same block frees.
     const int32_t* table = p.cached_lens ? p.block_tables + static_cast<int64_t>(s) * p.max_blocks
                                          : nullptr;
-    auto load_block = [&](int jj, int st) {  // lane 0
-      uint8_t* dst = sKV + st * LY::STAGE;
-      mbar_arrive_expect_tx(&bar_full[st], LY::STAGE);
+    auto load_part = [&](int jj, int w) {  // lane 0
+      const int st = jj % kTcStages;
+      uint8_t* dst = sKV + st * LY::STAGE + w * LY::KV_BYTES;
+      uint64_t* bar = &bar_full[w][st];
+      mbar_arrive_expect_tx(bar, LY::KV_BYTES);
       if (jj < npre) {
         // one box of B rows per physical block; rows past the prefix (and bad
         // table entries) are read from block num_blocks, outside the pool:
@@ -264,27 +301,21 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
             const int e = __ldg(table + pos / p.B);
             if (e >= 0 && e < p.num_blocks) {
               blk = e;
-            } else {
+            } else if (w == 0) {
               set_status(p.status, -7 /* PA_ERR_BAD_BLOCK */);
             }
           }
 #pragma unroll
-          for (int hf = 0; hf < LY::HALVES; ++hf) {
-            tc::tma_load_4d(dst + hf * (kTcBN * 128) + r0 * 128, &tm_kc, hf * 64, 0, kvh, blk,
-                            &bar_full[st]);
-            tc::tma_load_4d(dst + LY::KV_BYTES + hf * (kTcBN * 128) + r0 * 128, &tm_vc, hf * 64,
-                            0, kvh, blk, &bar_full[st]);
-          }
+          for (int hf = 0; hf < LY::HALVES; ++hf)
+            tc::tma_load_4d(dst + hf * (kTcBN * 128) + r0 * 128, w ? &tm_vc : &tm_kc, hf * 64, 0,
+                            kvh, blk, bar);
         }
       } else {
         const int j = jj - npre;
 #pragma unroll
-        for (int hf = 0; hf < LY::HALVES; ++hf) {
-          tc::tma_load_3d(dst + hf * (kTcBN * 128), &tm_k, hf * 64, kvh, a + j * kTcBN,
-                          &bar_full[st]);
-          tc::tma_load_3d(dst + LY::KV_BYTES + hf * (kTcBN * 128), &tm_v, hf * 64, kvh,
-                          a + j * kTcBN, &bar_full[st]);
-        }
+        for (int hf = 0; hf < LY::HALVES; ++hf)
+          tc::tma_load_3d(dst + hf * (kTcBN * 128), w ? &tm_v : &tm_k, hf * 64, kvh,
+                          a + j * kTcBN, bar);
       }
     };
     // The new keys' blocks whose rows are this CTA's own queries go to the
@@ -296,15 +327,17 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return !__any_sync(0xffffffffu, !wait(bar, parity));
     };
-    auto store_block = [&](int jj) -> bool {  // whole warp; block jj's data has landed
+    // store the K (w = 0) or V (w = 1) tile of block jj, once it has landed
+    auto store_part = [&](int jj, int w) -> bool {  // whole warp
       const int st = jj % kTcStages;
-      if (!wwait(&bar_full[st], (jj / kTcStages) & 1)) return false;
-      const uint8_t* sK = sKV + st * LY::STAGE;
-      const uint8_t* sV = sK + LY::KV_BYTES;
+      if (!wwait(&bar_full[w][st], (jj / kTcStages) & 1)) return false;
+      const uint8_t* src = sKV + st * LY::STAGE + w * LY::KV_BYTES;
+      const CUtensorMap* map = w ? &tm_vc : &tm_kc;
+      T* cache = static_cast<T*>(w ? p.v_cache : p.k_cache);
       const int j = jj - npre;
       bool plain = false;
       for (int r0 = 0; r0 < kTcBN; r0 += p.B) {
-        // lane r < B takes row r0 + r of the block: new token j*64 + r0 + r
+        // lane r < B takes row r0 + r of the block: new token j*kTcBN + r0 + r
         const int pos = j * kTcBN + r0 + lane;
         int64_t slot = -2;  // no token
         if (lane < p.B && pos < L) slot = __ldg(p.slot_mapping + a + pos);
@@ -316,139 +349,185 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
           if (lane == 0) {
             const int blk = static_cast<int>(s0 / p.B);
 #pragma unroll
-            for (int hf = 0; hf < LY::HALVES; ++hf) {
-              tc::tma_store_4d(&tm_kc, sK + hf * (kTcBN * 128) + r0 * 128, hf * 64, 0, kvh, blk);
-              tc::tma_store_4d(&tm_vc, sV + hf * (kTcBN * 128) + r0 * 128, hf * 64, 0, kvh, blk);
-            }
+            for (int hf = 0; hf < LY::HALVES; ++hf)
+              tc::tma_store_4d(map, src + hf * (kTcBN * 128) + r0 * 128, hf * 64, 0, kvh, blk);
             tc::bulk_commit();
           }
         } else if (lane < p.B && slot >= num_slots) {
-          set_status(p.status, -9 /* PA_ERR_BAD_SLOT */);
+          if (w == 0) set_status(p.status, -9 /* PA_ERR_BAD_SLOT */);
         } else if (lane < p.B && slot >= 0) {
           // row by row: undo the swizzle (16-byte piece c of row r sits at
           // piece c ^ (r % 8)) and write the row at its slot
           const int r = r0 + lane;
           const int64_t row = ((slot / p.B) * p.Hkv + kvh) * p.B + slot % p.B;
-          uint4* dk = reinterpret_cast<uint4*>(static_cast<T*>(p.k_cache) + row * D);
-          uint4* dv = reinterpret_cast<uint4*>(static_cast<T*>(p.v_cache) + row * D);
+          uint4* dst = reinterpret_cast<uint4*>(cache + row * D);
 #pragma unroll
           for (int hf = 0; hf < LY::HALVES; ++hf)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int off = hf * (kTcBN * 128) + r * 128 + ((c ^ (r & 7)) << 4);
-              dk[hf * 8 + c] = *reinterpret_cast<const uint4*>(sK + off);
-              dv[hf * 8 + c] = *reinterpret_cast<const uint4*>(sV + off);
-            }
+            for (int c = 0; c < 8; ++c)
+              dst[hf * 8 + c] = *reinterpret_cast<const uint4*>(
+                  src + hf * (kTcBN * 128) + r * 128 + ((c ^ (r & 7)) << 4));
           plain = true;
         }
       }
-      // generic reads of the stage before the next TMA load writes it
+      // generic reads of the slot before the next TMA load writes it
       if (plain) fence_proxy_async_smem();
       __syncwarp();
       return true;
     };
-    int issued = 0, stored = own_lo;
+    int issued_w[2] = {0, 0}, stored = own_lo;
     bool ok = true;
-    for (int jj = 0; jj < nkb; ++jj) {
+    for (int jj = 0; jj < nkb && ok; ++jj) {
       const int st = jj % kTcStages;
-      if (jj >= kTcStages) {
-        if (!wwait(&bar_empty[st], ((jj / kTcStages) - 1) & 1)) break;
-        // the stage still holds block jj - kTcStages: store it if it is ours,
-        // and let the stores finish reading it before it is refilled
-        if (stores && jj - kTcStages >= own_lo) {
-          if (!(ok = store_block(jj - kTcStages))) break;
-          stored = jj - kTcStages + 1;
-          if (lane == 0) tc::bulk_wait_read_all();
-          __syncwarp();
+#pragma unroll
+      for (int w = 0; w < 2 && ok; ++w) {
+        if (jj >= kTcStages) {
+          if (!(ok = wwait(&bar_empty[w][st], ((jj / kTcStages) - 1) & 1))) break;
+          // the slot still holds block jj - kTcStages: store it if it is ours,
+          // and let the stores finish reading it before it is refilled
+          if (stores && jj - kTcStages >= own_lo) {
+            if (!(ok = store_part(jj - kTcStages, w))) break;
+            if (w == 1) stored = jj - kTcStages + 1;
+            if (lane == 0) tc::bulk_wait_read_all();
+            __syncwarp();
+          }
         }
+        if (lane == 0) load_part(jj, w);
+        issued_w[w] = jj + 1;
       }
-      if (lane == 0) load_block(jj, st);
-      issued = jj + 1;
     }
-    // our blocks still in the ring
-    for (int jj = stored; stores && ok && jj < issued; ++jj) ok = store_block(jj);
+    // our blocks still in the rings
+    for (int jj = stored; stores && ok && jj < issued_w[1]; ++jj)
+      ok = store_part(jj, 0) && store_part(jj, 1);
     if (lane == 0) {
       // drain: the stores must have read their tiles, and the copies in
       // flight landed, before this CTA's shared memory goes (the stores'
       // global writes complete with the grid, like any other store)
       tc::bulk_wait_read_all();
       mbar_wait_bounded(&bar_q, 0, kTcDrainNs);
-      for (int j = issued > kTcStages ? issued - kTcStages : 0; j < issued; ++j)
-        mbar_wait_bounded(&bar_full[j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
+#pragma unroll
+      for (int w = 0; w < 2; ++w)
+        for (int j = issued_w[w] > kTcStages ? issued_w[w] - kTcStages : 0; j < issued_w[w]; ++j)
+          mbar_wait_bounded(&bar_full[w][j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
     }
   } else if (warp == kMmaWarp) {
     // ---------------- tensor-core products ----------------
-    if (lane == 0) {
-      const uint32_t qa = smem_addr(sQ);
-      int s_done[kTcTiles] = {0, 0}, o_done[kTcTiles] = {0, 0}, empties = 0;
-      auto issue_s = [&](int t, int j) -> bool {  // S_t = Q_t K_j^T
-        // (the previous block's scores were read: its P is written, P V issued)
-        if (!wait(&bar_full[j % kTcStages], (j / kTcStages) & 1)) return false;
-        tc::fence_after_sync();
-        const uint32_t q = qa + t * LY::Q_BYTES;
-        const uint32_t k = smem_addr(sKV + (j % kTcStages) * LY::STAGE);
-        const uint32_t d = tmem + t * kTileCols + kColS;
+    // One issuer for both tiles, in the order PV0, S0', PV1, S1': the tiles'
+    // softmaxes then alternate, each running while the tensor pipe has the
+    // other tile's products.  (A warp per tile measured slower: the tiles
+    // fell into step, their softmaxes contending for the exponential unit
+    // while the pipe stood idle.)  The whole warp runs the loop; lane 0
+    // alone issues each product and commit (the same lane throughout, so
+    // its commits track its products).
+    const uint32_t leader = lane == 0;
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return !__any_sync(0xffffffffu, !wait(bar, parity));
+    };
+    // descriptors of the two Q tiles and of the K and V blocks of each stage;
+    // a step along K adds its byte offset >> 4 to the start-address field
+    uint64_t dq[kTcTiles], dk[kTcStages], dv[kTcStages];
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          tc::mma_ss(d, tc::smem_desc(q + (ks >> 2) * (kTcBM * 128) + (ks & 3) * 32, 16, 1024),
-                     tc::smem_desc(k + (ks >> 2) * (kTcBN * 128) + (ks & 3) * 32, 16, 1024),
-                     IDESC_S, ks > 0);
-        tc::commit(&bar_s[t]);
-        ++s_done[t];
-        return true;
-      };
-      auto issue_pv = [&](int t, int j) -> bool {  // O_t += P_t V_j
-        if (!wait(&bar_p[t], j & 1)) return false;
-        tc::fence_after_sync();
-        const uint32_t v = smem_addr(sKV + (j % kTcStages) * LY::STAGE + LY::KV_BYTES);
-        const uint32_t base = tmem + t * kTileCols;
+    for (int t = 0; t < kTcTiles; ++t) dq[t] = tc::smem_desc(smem_addr(sQ + t * LY::Q_BYTES), 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < kTcBN / 16; ++ks) {
-          const uint64_t dv = tc::smem_desc(v + ks * 2048, kTcBN * 128, 1024);
-          tc::mma_ts(base + kColO, base + kColPhi + ks * 8, dv, IDESC_O, j > 0 || ks > 0);
-          if constexpr (BF16) tc::mma_ts(base + kColO, base + kColPlo + ks * 8, dv, IDESC_O, true);
-        }
-        tc::commit(&bar_o[t]);
-        ++o_done[t];
-        return true;
-      };
-      bool ok = wait(&bar_q, 0);
-      for (int t = 0; t < kTcTiles && ok; ++t)
-        if (nkb_t[t] > 0) ok = issue_s(t, 0);
-      for (int j = 0; j < nkb && ok; ++j) {
-        if constexpr (kTcEarlyS) {
-          // S(j+1) as soon as the softmax holds S(j) in registers, then P(j) V
-          for (int t = 0; t < kTcTiles && ok; ++t) {
-            if (j + 1 >= nkb_t[t]) continue;
-            ok = wait(&bar_sfree[t], j & 1);
-            if (ok) ok = issue_s(t, j + 1);
-          }
-          for (int t = 0; t < kTcTiles && ok; ++t)
-            if (j < nkb_t[t]) ok = issue_pv(t, j);
+    for (int i = 0; i < kTcStages; ++i) {
+      dk[i] = tc::smem_desc(smem_addr(sKV + i * LY::STAGE), 16, 1024);
+      dv[i] = tc::smem_desc(smem_addr(sKV + i * LY::STAGE + LY::KV_BYTES), kTcBN * 128, 1024);
+    }
+    // a stage's descriptor by a run-time index, without local memory
+    auto sel = [](const uint64_t (&a)[kTcStages], int i) -> uint64_t {
+      uint64_t r = a[0];
+#pragma unroll
+      for (int k = 1; k < kTcStages; ++k)
+        if (i == k) r = a[k];
+      return r;
+    };
+    int s_done0 = 0, s_done1 = 0, o_done0 = 0, o_done1 = 0;
+    int k_ready = 0, v_ready = 0;  // blocks whose K, V tiles are known to have landed
+    auto issue_s = [&](int t, int j) -> bool {  // S_t = Q_t K_j^T
+      // (the previous block's scores were read: its P is written, P V issued)
+      if (j >= k_ready) {
+        if (!wwait(&bar_full[0][j % kTcStages], (j / kTcStages) & 1)) return false;
+        k_ready = j + 1;
+      }
+      tc::fence_after_sync();
+      const uint64_t q = t ? dq[1] : dq[0];
+      const uint64_t k = sel(dk, j % kTcStages);
+      const uint32_t d = tmem + t * kTileCols + kColS;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tc::mma_ss_by(leader, d, q + ((((ks >> 2) * (kTcBM * 128)) + (ks & 3) * 32) >> 4),
+                      k + ((((ks >> 2) * (kTcBN * 128)) + (ks & 3) * 32) >> 4), IDESC_S, ks > 0);
+      tc::commit_by(leader, &bar_s[t]);
+      if (t) ++s_done1; else ++s_done0;
+      return true;
+    };
+    auto issue_pv = [&](int t, int j) -> bool {  // O_t += P_t V_j
+      if (j >= v_ready) {
+        if (!wwait(&bar_full[1][j % kTcStages], (j / kTcStages) & 1)) return false;
+        v_ready = j + 1;
+      }
+      if (!wwait(&bar_p[t], j & 1)) return false;
+      tc::fence_after_sync();
+      const uint64_t v = sel(dv, j % kTcStages);
+      const uint32_t base = tmem + t * kTileCols;
+#pragma unroll
+      for (int ks = 0; ks < kTcBN / 16; ++ks) {
+        // 16 keys a product; their P columns (the softmax's layout)
+        const uint64_t b = v + ((ks * 2048) >> 4);
+        if constexpr (BF16) {
+          tc::mma_ts_by(leader, base + kColO, base + kColS + ks * 16, b, IDESC_O, j > 0 || ks > 0);
+          tc::mma_ts_by(leader, base + kColO, base + kColS + ks * 16 + 8, b, IDESC_O, true);
         } else {
-          for (int t = 0; t < kTcTiles && ok; ++t) {
-            if (j >= nkb_t[t]) continue;
-            ok = issue_pv(t, j);
-            if (ok && j + 1 < nkb_t[t]) ok = issue_s(t, j + 1);
-          }
-        }
-        if (ok) {
-          tc::commit(&bar_empty[j % kTcStages]);  // block j's stage is read for good
-          empties = j + 1;
+          tc::mma_ts_by(leader, base + kColO, base + kColS + ks * 8, b, IDESC_O, j > 0 || ks > 0);
         }
       }
-      // drain: every product issued must finish, and every commit arrive,
-      // before TMEM and this CTA's shared memory are given up
-      for (int j = empties > kTcStages ? empties - kTcStages : 0; j < empties; ++j)
-        mbar_wait_bounded(&bar_empty[j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
+      tc::commit_by(leader, &bar_o[t]);
+      if (t) ++o_done1; else ++o_done0;
+      return true;
+    };
+    // Slot releases: K of block j once both tiles' S_t(j) are issued, V of
+    // block j once both tiles' P_t(j) V are (a commit tracks every product
+    // issued before it).
+    int k_empties = 0, v_empties = 0;
+    bool ok = wwait(&bar_q, 0);
+    if (ok && nkb_t[0] > 0) ok = issue_s(0, 0);
+    if (ok && nkb_t[1] > 0) ok = issue_s(1, 0);
+    if (ok && nkb > 0) {
+      tc::commit_by(leader, &bar_empty[0][0]);
+      k_empties = 1;
+    }
+    for (int j = 0; j < nkb && ok; ++j) {
 #pragma unroll
       for (int t = 0; t < kTcTiles; ++t) {
-        if (s_done[t] > 0) mbar_wait_bounded(&bar_s[t], (s_done[t] - 1) & 1, kTcDrainNs);
-        if (o_done[t] > 0) mbar_wait_bounded(&bar_o[t], (o_done[t] - 1) & 1, kTcDrainNs);
+        if (!ok || j >= nkb_t[t]) continue;
+        ok = issue_pv(t, j);
+        if (ok && j + 1 < nkb_t[t]) ok = issue_s(t, j + 1);
+      }
+      if (ok) {
+        tc::commit_by(leader, &bar_empty[1][j % kTcStages]);
+        v_empties = j + 1;
+        if (j + 1 < nkb) {
+          tc::commit_by(leader, &bar_empty[0][(j + 1) % kTcStages]);
+          k_empties = j + 2;
+        }
       }
     }
+    // drain: every product issued must finish, and every commit arrive,
+    // before TMEM and this CTA's shared memory are given up
+    for (int j = k_empties > kTcStages ? k_empties - kTcStages : 0; j < k_empties; ++j)
+      mbar_wait_bounded(&bar_empty[0][j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
+    for (int j = v_empties > kTcStages ? v_empties - kTcStages : 0; j < v_empties; ++j)
+      mbar_wait_bounded(&bar_empty[1][j % kTcStages], (j / kTcStages) & 1, kTcDrainNs);
+    if (s_done0 > 0) mbar_wait_bounded(&bar_s[0], (s_done0 - 1) & 1, kTcDrainNs);
+    if (o_done0 > 0) mbar_wait_bounded(&bar_o[0], (o_done0 - 1) & 1, kTcDrainNs);
+    if (s_done1 > 0) mbar_wait_bounded(&bar_s[1], (s_done1 - 1) & 1, kTcDrainNs);
+    if (o_done1 > 0) mbar_wait_bounded(&bar_o[1], (o_done1 - 1) & 1, kTcDrainNs);
+    __syncwarp();
+  }
   } else {
     // ---------------- softmax of one query row ----------------
+    // (the softmax warpgroups first raise their registers)
+    tc::regs_raise<kTcRegsHigh>();
     const int t = warp >> 2;                     // tile of this warpgroup
     const int row = tid & (kTcBM - 1);           // row within the tile = TMEM lane
     const int qpos = q0 + t * kTcBM + row;       // new row within the prompt (position cl + qpos)
@@ -461,141 +540,167 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       failed = __any_sync(0xffffffffu, failed || !wait(&bar_s[t], jj & 1));
       if (failed) break;
       tc::fence_after_sync();
-      float sv[kTcBN];
-      {
-        // four loads in flight, one wait
-        uint32_t v[kTcBN / 16][16];
-#pragma unroll
-        for (int i = 0; i < kTcBN / 16; ++i) tc::ld16(rbase + kColS + i * 16, v[i]);
-        tc::wait_ld();
-#pragma unroll
-        for (int i = 0; i < kTcBN / 16; ++i)
-#pragma unroll
-          for (int c = 0; c < 16; ++c) sv[i * 16 + c] = __uint_as_float(v[i][c]);
-      }
-      if constexpr (kTcEarlyS) {
-        // the scores are in registers: the next block's S may overwrite them
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_sfree[t]);
-      }
-      // `below`: no score of this warp's rows is masked in this block, so part
-      // of the weights may come from the polynomial
+      // Keys of this block from `lim` on are hidden from this row: past the
+      // stored prefix in its last block (rows read as zeros), or past the row
+      // itself among the new keys.  `below`: no score of this warp's rows is
+      // hidden, so part of the weights may come from the polynomial.
+      int lim;
       bool below;
       if (jj < npre) {
-        // stored prefix: its keys precede every new row; the last block may
-        // run past the prefix (rows read as zeros), which is masked
+        lim = min(kTcBN, cl - jj * kTcBN);
         below = jj * kTcBN + kTcBN <= cl;
-        if (!below) {
-#pragma unroll
-          for (int c = 0; c < kTcBN; ++c)
-            if (jj * kTcBN + c >= cl) sv[c] = -INFINITY;
-        }
       } else {
-        // new keys: those past this row exist only in the diagonal blocks
         const int j = jj - npre;
-        if (j * kTcBN + kTcBN - 1 > qpos) {
-#pragma unroll
-          for (int c = 0; c < kTcBN; ++c)
-            if (j * kTcBN + c > qpos) sv[c] = -INFINITY;
-        }
+        lim = min(kTcBN, max(0, qpos - j * kTcBN + 1));
         below = j * kTcBN + kTcBN - 1 <= q0 + t * kTcBM + (warp & 3) * 32;
       }
-      // four independent partial maxima (of three-input maxima)
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if constexpr (kTcPacked) {
+      // Hidden keys exist only in a warp's diagonal block and in the prefix's
+      // last block: the warps that have any take the masking path, the rest
+      // (most blocks) the one without a compare per score.
+      const bool masked = lim < kTcBN;
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // partial sums
+      auto block = [&](auto mask_tag) {
+        constexpr bool MASK = decltype(mask_tag)::value;
+        auto score = [&](uint32_t bits, int key) -> float {
+          if constexpr (MASK) return key >= lim ? -INFINITY : __uint_as_float(bits);
+          return __uint_as_float(bits);
+        };
+        // the row's scores, when they are read once
+        uint32_t all[kTcOneLoad ? kTcBN / 32 : 1][32];
+        // Pass 1, the row max: the scores 64 columns at a time (two loads in
+        // flight, one wait), four independent partial maxima of three-input
+        // maxima.
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        auto max_of = [&](const uint32_t (&v)[32], int key0) {
 #pragma unroll
-        for (int c = 0; c < kTcBN; c += 8) {
+          for (int c = 0; c < 32; c += 8)
 #pragma unroll
-          for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
-        }
-      } else {
+            for (int u = 0; u < 4; ++u) {
+              const int key = key0 + c + 2 * u;
+              const float a = score(v[c + 2 * u], key), b = score(v[c + 2 * u + 1], key + 1);
+              if constexpr (kTcPacked) {
+                mx[u] = fmax3(mx[u], a, b);
+              } else {
+                mx[u] = fmaxf(fmaxf(mx[u], a), b);
+              }
+            }
+        };
+        if constexpr (kTcOneLoad) {
 #pragma unroll
-        for (int c = 0; c < kTcBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
-      }
-      // base-2 logits: the scale (> 0) is applied in the exponent
-      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
-      // P_t and O_t are in use by the previous block's product until it is
-      // done (here, or after the weights when S runs a block ahead)
-      auto wait_pv = [&]() -> bool {
-        if (jj > 0) {
-          if (__any_sync(0xffffffffu, !wait(&bar_o[t], (jj - 1) & 1))) return false;
-          tc::fence_after_sync();
-        }
-        return true;
-      };
-      if constexpr (!kTcEarlyS) {
-        failed = !wait_pv();
-        if (failed) break;
-      }
-      const bool raise = rmax > m + 8.f;
-      const float m_new = raise ? rmax : m;
-      const float alpha = raise && m != -INFINITY ? fast_exp2(m - m_new) : 1.f;
-      auto rescale_o = [&]() {
-        if (!(jj > 0 && __any_sync(0xffffffffu, alpha != 1.f))) return;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 64) {
-          uint32_t v[4][16];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) tc::ld16(rbase + kColO + c0 + i * 16, v[i]);
+          for (int c = 0; c < kTcBN / 32; ++c) tc::ld32(rbase + kColS + c * 32, all[c]);
           tc::wait_ld();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int c = 0; c < kTcBN / 32; ++c) max_of(all[c], c * 32);
+        } else {
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              v[i][c] = __float_as_uint(__uint_as_float(v[i][c]) * alpha);
-            tc::st16(rbase + kColO + c0 + i * 16, v[i]);
+          for (int h = 0; h < kTcBN / 64; ++h) {
+            uint32_t v[2][32];
+            tc::ld32(rbase + kColS + h * 64, v[0]);
+            tc::ld32(rbase + kColS + h * 64 + 32, v[1]);
+            tc::wait_ld();
+            max_of(v[0], h * 64);
+            max_of(v[1], h * 64 + 32);
+          }
+        }
+        // base-2 logits: the scale (> 0) is applied in the exponent
+        const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+        // P_t and O_t are in use by the previous block's product until it is
+        // done, which is known here: S is issued after it, and the S-ready
+        // commit tracks every product the MMA warp issued before it.
+        const bool raise = rmax > m + 8.f;
+        const float m_new = raise ? rmax : m;
+        const float alpha = raise && m != -INFINITY ? fast_exp2(m - m_new) : 1.f;
+        if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 64) {
+            uint32_t v[4][16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tc::ld16(rbase + kColO + c0 + i * 16, v[i]);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                v[i][c] = __float_as_uint(__uint_as_float(v[i][c]) * alpha);
+              tc::st16(rbase + kColO + c0 + i * 16, v[i]);
+            }
+          }
+        }
+        l *= alpha;
+        m = m_new;
+        const float mm = m == -INFINITY ? 0.f : m;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-mm, -mm);
+        // Pass 2, the weights 2^(scale * s - m), 32 keys at a time (read
+        // again from TMEM, the next chunk's load in flight while this one is
+        // computed, unless the scores were read once), two scores per packed
+        // fma; hidden scores are -inf: weight 0.  Below the diagonal,
+        // kTcPolyPairs of every four pairs of weights come from the FMA-pipe
+        // polynomial and the rest from the exponential unit.
+        // P goes back over S as packed 16-bit pairs: keys 16g..16g+15 take
+        // columns 8g..8g+7 (fp16), or 16g..16g+7 for P_hi and 16g+8..16g+15
+        // for P_lo = P - P_hi (bf16, so P enters with about 16 significant
+        // bits).  Chunk c's P thus lands in columns that chunks 0..c were
+        // read from, never in one still to be read.
+        auto weights = [&](const uint32_t (&v)[32], int c) {
+          uint32_t ph[16], pl[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int key = c * 32 + e;
+            const float a = score(v[e], key), b = score(v[e + 1], key + 1);
+            const bool poly = below && ((e >> 1) & 3) >= 4 - kTcPolyPairs;
+            float2 pw;
+            if constexpr (kTcPacked) {
+              const float2 x = __ffma2_rn(make_float2(a, b), sc2, nm2);
+              pw = poly ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              ls[(e >> 1) & 1] = __fadd2_rn(ls[(e >> 1) & 1], pw);
+            } else {
+              pw = make_float2(fast_exp2(fmaf(a, p.scale_log2, -mm)),
+                               fast_exp2(fmaf(b, p.scale_log2, -mm)));
+              ls[(e >> 1) & 1].x += pw.x + pw.y;
+            }
+            ph[e / 2] = Elem<T>::from_float2(pw.x, pw.y);
+            if constexpr (BF16) {
+              const float2 back = Elem<T>::to_float2(ph[e / 2]);
+              pl[e / 2] = Elem<T>::from_float2(pw.x - back.x, pw.y - back.y);
+            }
+          }
+          if constexpr (BF16) {
+            uint32_t w[2][16];
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                w[g][i] = ph[g * 8 + i];
+                w[g][8 + i] = pl[g * 8 + i];
+              }
+            tc::st16(rbase + kColS + c * 32, w[0]);
+            tc::st16(rbase + kColS + c * 32 + 16, w[1]);
+          } else {
+            tc::st16(rbase + kColS + c * 16, ph);
+          }
+        };
+        if constexpr (kTcOneLoad) {
+#pragma unroll
+          for (int c = 0; c < kTcBN / 32; ++c) weights(all[c], c);
+        } else {
+          uint32_t v[2][32];
+          tc::ld32(rbase + kColS, v[0]);
+          tc::wait_ld();
+#pragma unroll
+          for (int c = 0; c < kTcBN / 32; ++c) {
+            if (c + 1 < kTcBN / 32) tc::ld32(rbase + kColS + (c + 1) * 32, v[(c + 1) & 1]);
+            weights(v[c & 1], c);
+            if (c + 1 < kTcBN / 32) tc::wait_ld();
           }
         }
       };
-      if constexpr (!kTcEarlyS) rescale_o();
-      l *= alpha;
-      m = m_new;
-      const float mm = m == -INFINITY ? 0.f : m;
-      uint32_t ph[32], pl[32];
-      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // partial sums
-      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-      const float2 nm2 = make_float2(-mm, -mm);
-      // 2^(scale * s - m), two scores per packed fma (masked scores are -inf:
-      // weight 0).  Below the diagonal, kTcPolyPairs of every four pairs of
-      // weights come from the FMA-pipe polynomial and the rest from the
-      // exponential unit, so the two units share the work.
-      auto weights = [&](int c, bool poly) {
-        float2 pw;
-        if constexpr (kTcPacked) {
-          const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sc2, nm2);
-          pw = poly ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
-          ls[(c >> 1) & 1] = __fadd2_rn(ls[(c >> 1) & 1], pw);
-        } else {
-          pw = make_float2(fast_exp2(fmaf(sv[c], p.scale_log2, -mm)),
-                           fast_exp2(fmaf(sv[c + 1], p.scale_log2, -mm)));
-          ls[(c >> 1) & 1].x += pw.x + pw.y;
-        }
-        ph[c / 2] = Elem<T>::from_float2(pw.x, pw.y);
-        if constexpr (BF16) {
-          const float2 back = Elem<T>::to_float2(ph[c / 2]);
-          pl[c / 2] = Elem<T>::from_float2(pw.x - back.x, pw.y - back.y);
-        }
-      };
-      if (below) {
-#pragma unroll
-        for (int c = 0; c < kTcBN; c += 2) weights(c, ((c >> 1) & 3) >= 4 - kTcPolyPairs);
+      if (__any_sync(0xffffffffu, masked)) {
+        block(std::true_type{});
       } else {
-#pragma unroll
-        for (int c = 0; c < kTcBN; c += 2) weights(c, false);
+        block(std::false_type{});
       }
       l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
-      if constexpr (kTcEarlyS) {
-        failed = !wait_pv();
-        if (failed) break;
-        rescale_o();
-      }
-      tc::st16(rbase + kColPhi, *reinterpret_cast<uint32_t(*)[16]>(ph));
-      tc::st16(rbase + kColPhi + 16, *reinterpret_cast<uint32_t(*)[16]>(ph + 16));
-      if constexpr (BF16) {
-        tc::st16(rbase + kColPlo, *reinterpret_cast<uint32_t(*)[16]>(pl));
-        tc::st16(rbase + kColPlo + 16, *reinterpret_cast<uint32_t(*)[16]>(pl + 16));
-      }
       tc::wait_st();
       tc::fence_before_sync();
       mbar_arrive(&bar_p[t]);

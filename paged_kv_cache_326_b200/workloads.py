@@ -455,13 +455,15 @@ def to_codes(x: torch.Tensor, scale: float) -> torch.Tensor:
 def make_decode_fp8(name: str, context_lens: Sequence[int], num_heads: int, head_dim: int,
                     block_size: int, num_blocks: int, dtype: torch.dtype, seed: int,
                     device="cpu", max_blocks_per_seq: Optional[int] = None,
-                    k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE) -> DecodeInputs:
+                    k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE,
+                    num_kv_heads: Optional[int] = None) -> DecodeInputs:
     """make_decode with 8-bit caches: the pools hold E4M3 codes of seeded
     N(0,1) numbers over the scales (``meta['k_scale']``, ``meta['v_scale']``);
     rows that hold no earlier token hold the NaN code.  q, k, v stay in
-    ``dtype``."""
+    ``dtype``; ``num_kv_heads`` below ``num_heads`` gives grouped-query
+    pools."""
     w = make_decode(name, context_lens, num_heads, head_dim, block_size, num_blocks, dtype, seed,
-                    device, max_blocks_per_seq, poison=False)
+                    device, max_blocks_per_seq, poison=False, num_kv_heads=num_kv_heads)
     dev = w.q.device
     g = _gen(seed + 2000003, dev)
     shape = w.k_cache.shape
@@ -482,6 +484,18 @@ def make_decode_fp8(name: str, context_lens: Sequence[int], num_heads: int, head
     w.name = name
     w.meta.update(k_scale=k_scale, v_scale=v_scale)
     return w
+
+
+def llama2_70b_gqa_fp8(seed: int = 6, device="cpu", num_seqs: int = 64,
+                       num_blocks: int = 12288) -> DecodeInputs:
+    """The Llama-2-70B-shaped grouped-query step (64 query heads over 8
+    key/value heads, head_dim 128, blocks of 16, lengths uniform in
+    [128, 4096]) over 8-bit caches."""
+    g = np.random.default_rng(seed)
+    lens = [int(x) for x in g.integers(128, 4096, size=num_seqs, endpoint=True)]
+    return make_decode_fp8("llama2_70b_gqa_fp8", lens, num_heads=64, head_dim=128,
+                           block_size=16, num_blocks=num_blocks, dtype=torch.float16, seed=seed,
+                           device=device, max_blocks_per_seq=4096 // 16, num_kv_heads=8)
 
 
 def opt13b_batch64_fp8(seed: int = 2, device="cpu") -> DecodeInputs:

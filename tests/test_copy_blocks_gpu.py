@@ -201,12 +201,10 @@ def test_parallel_sampling_session_with_device_copies():
 
 
 @pytest.mark.parametrize("count", [1, 7, 700])
-def test_copy_shares_cross_copy_boundaries(count):
-    """The grid cuts all copies of a call into equal shares of 16-byte
-    vectors: with blocks of 512 bytes (1 head x 4 x 64, 32 vectors) a
-    thread's lanes step across many copies per round, with one pair only a
-    few threads work, and with 700 pairs shares start and end inside
-    copies.  Bit-exact in every case."""
+def test_copy_small_blocks_many_pairs(count):
+    """Blocks of 512 bytes (1 head x 4 x 64, 32 vectors): one CTA per copy
+    with most of its threads idle, one pair or 700 of them.  Bit-exact in
+    every case."""
     import paged_kv_cache_326_b200 as P
     H, D, B, N = 1, 64, 4, 1600
     kc, vc = (_bits_pool(N, H, B, D, torch.float16, 11 + i) for i in range(2))
@@ -231,6 +229,38 @@ def test_copy_bad_pair_in_the_middle_is_reported_and_skipped():
     pairs = good[:10] + [(N + 5, good[10][1])] + good[11:]
     ek, ev = oracle.copy_blocks(_i16(kc), _i16(vc), _i16(kc), _i16(vc),
                                 good[:10] + good[11:])
+    st = new_status()
+    P.pa_copy_blocks(kc, vc, kc, vc, torch.tensor(pairs, dtype=torch.int32, device="cuda"),
+                     status=st)
+    torch.cuda.synchronize()
+    assert st.item() == P.binding.PA_ERR_BAD_BLOCK
+    assert np.array_equal(_i16(kc), ek) and np.array_equal(_i16(vc), ev)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+def test_copy_runs_of_one_source(dtype):
+    """Runs of consecutive pairs with one source (a prompt's block copied for
+    each of its samples): runs of 1, 3, 8, 9 and 17 pairs, a run whose source
+    is outside the pool, and a run with a bad destination inside it.  The
+    bad pairs are reported and copy nothing; every other pair is exact."""
+    import paged_kv_cache_326_b200 as P
+    H, D, B, N = 4, 128, 16, 200
+    kc, vc = (_bits_pool(N, H, B, D, dtype, 31 + i) for i in range(2))
+    rng = np.random.default_rng(33)
+    perm = [int(x) for x in rng.permutation(N)]
+    srcs, dsts = perm[:10], iter(perm[10:])
+    pairs, good = [], []
+    for k, n in enumerate([1, 3, 8, 9, 17, 2, 5, 4]):
+        for i in range(n):
+            p = (srcs[k], next(dsts))
+            if k == 5:
+                p = (N + 3, p[1])            # source outside the pool
+            if k == 4 and i == 11:
+                p = (p[0], -2)               # destination outside the pool
+            pairs.append(p)
+            if 0 <= p[0] < N and 0 <= p[1] < N:
+                good.append(p)
+    ek, ev = oracle.copy_blocks(_i16(kc), _i16(vc), _i16(kc), _i16(vc), good)
     st = new_status()
     P.pa_copy_blocks(kc, vc, kc, vc, torch.tensor(pairs, dtype=torch.int32, device="cuda"),
                      status=st)

@@ -32,7 +32,18 @@ def fp8_kernel(request):
     P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
 
 
-def parity_fp8(w, seqs=None, heads_per_seq=None, seed=0):
+def gpu_step_fp8_fused(w, status=None, out=None):
+    """The 8-bit step through the one-launch entry point pa_decode_step_fp8."""
+    import paged_kv_cache_326_b200 as P
+    if out is None:
+        out = torch.empty_like(w.q)
+    P.pa_decode_step_fp8(out, w.q, w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping,
+                         w.block_tables, w.context_lens, w.scale, w.meta["k_scale"],
+                         w.meta["v_scale"], status=status)
+    return out
+
+
+def parity_fp8(w, seqs=None, heads_per_seq=None, seed=0, step=gpu_step_fp8):
     S, H, D = w.q.shape
     seqs = np.arange(S) if seqs is None else np.asarray(seqs)
     pairs = None
@@ -43,7 +54,7 @@ def parity_fp8(w, seqs=None, heads_per_seq=None, seed=0):
                        w.slot_mapping, w.block_size, seqs)
     kb, vb = w.k_cache.cpu().numpy(), w.v_cache.cpu().numpy()
     st = new_status()
-    out = gpu_step_fp8(w, st)
+    out = step(w, st)
     torch.cuda.synchronize()
     assert st.item() == 0, st.item()
     ks, vs = w.meta["k_scale"], w.meta["v_scale"]
@@ -116,6 +127,83 @@ def test_fp8_tensor_cores_refuse_what_they_do_not_cover():
                                            w.meta["k_scale"], w.meta["v_scale"])
     finally:
         P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("group", [2, 4, 5, 8])
+@pytest.mark.parametrize("head_dim,block_size", [(64, 8), (128, 16), (128, 4), (64, 32)],
+                         ids=["d64b8", "d128b16", "d128b4", "d64b32"])
+def test_fp8_grouped_query_every_shape(dtype, group, head_dim, block_size):
+    """Grouped-query pools of 8-bit codes (pa_paged_attn_decode_fp8_gqa):
+    2 key/value heads, each shared by `group` query heads, ragged lengths
+    from 0 to 160; the quantizing write bit for bit, every output against
+    the oracle."""
+    w = W.make_decode_fp8("fp8_gqa", SHAPE_LENS, num_heads=2 * group, head_dim=head_dim,
+                          block_size=block_size,
+                          num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in SHAPE_LENS),
+                          dtype=dtype, seed=group * 7 + head_dim + block_size, device="cuda",
+                          max_blocks_per_seq=160 // block_size, num_kv_heads=2)
+    parity_fp8(w)
+
+
+def test_fp8_grouped_query_llama2_70b():
+    """The Llama-2-70B-shaped layer (64 query heads over 8 key/value heads,
+    lengths 128..4096) over 8-bit caches: 12 texts x 8 sampled heads each."""
+    w = W.llama2_70b_gqa_fp8(device="cuda", num_seqs=24, num_blocks=6144)
+    c = parity_fp8(w, seqs=range(0, 24, 2), heads_per_seq=8, seed=5)
+    print("fp8 grouped-query llama2-70b", c)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("head_dim", [64, 128])
+@pytest.mark.parametrize("block_size", [4, 8, 16, 32])
+def test_fp8_one_launch_step_every_shape_ragged(dtype, head_dim, block_size):
+    """pa_decode_step_fp8: the new tokens' codes in the pool bit for bit, every
+    output against the oracle (which writes, then attends)."""
+    w = W.make_decode_fp8("fp8_step", SHAPE_LENS, num_heads=3, head_dim=head_dim,
+                          block_size=block_size,
+                          num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in SHAPE_LENS),
+                          dtype=dtype, seed=head_dim * 3 + block_size, device="cuda",
+                          max_blocks_per_seq=160 // block_size)
+    parity_fp8(w, step=gpu_step_fp8_fused)
+
+
+def test_fp8_one_launch_step_opt13b_batch64():
+    w = W.opt13b_batch64_fp8(device="cuda")
+    c = parity_fp8(w, heads_per_seq=6, seed=4, step=gpu_step_fp8_fused)
+    print("fp8 one-launch step opt13b", c)
+
+
+def test_fp8_one_launch_step_equals_two_calls_bitwise():
+    """Same inputs: the one-launch 8-bit step and the quantizing write followed
+    by the CUDA-core 8-bit decode give the same output and the same pools,
+    bit for bit (the new row's codes come from the same quantizer)."""
+    import paged_kv_cache_326_b200 as P
+    a = W.opt13b_batch64_fp8(device="cuda")
+    b = W.opt13b_batch64_fp8(device="cuda")
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, 1)
+    try:
+        out_a = gpu_step_fp8(a)
+    finally:
+        P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
+    out_b = gpu_step_fp8_fused(b)
+    torch.cuda.synchronize()
+    assert torch.equal(a.k_cache, b.k_cache) and torch.equal(a.v_cache, b.v_cache)
+    assert torch.equal(out_a, out_b)
+
+
+def test_fp8_one_launch_step_single_token_returns_its_value():
+    """One token per text, the new one: out = value(code(v / v_scale)) *
+    v_scale rounded to the output type, bit for bit."""
+    w = W.make_decode_fp8("fp8_step_one", [1] * 6, num_heads=5, head_dim=128, block_size=16,
+                          num_blocks=16, dtype=torch.bfloat16, seed=8, device="cuda")
+    out = gpu_step_fp8_fused(w)
+    torch.cuda.synchronize()
+    vs = np.float32(w.meta["v_scale"])
+    codes = oracle.quantize(w.v.float().cpu().numpy(), vs)
+    vals = torch.from_numpy(oracle.e4m3_decode(codes).astype(np.float32))
+    want = (vals * torch.tensor(vs)).to(out.dtype)
+    assert torch.equal(out.cpu(), want)
 
 
 def test_fp8_write_rounds_saturates_and_keeps_signs():
