@@ -764,9 +764,14 @@ def run_prefill_bench(args, ranks, world, rank, local):
         sweep.append({"cached_tokens": c, "new_tokens": n, "ms": med, "ms_min": mn,
                       "ms_vs_no_reuse": med / ms_step, "tflops": fl / (med * 1e-3) / 1e12,
                       "new_tokens_per_s": len(w.lens) * n / (med * 1e-3)})
-    ms_step, e2e_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms], dev)
+    # the attention without the store of the keys and values, for reference
+    def attention_only():
+        P.pa_prefill(out, w.q, w.k, w.v, w.cu_seqlens, w.max_seqlen, w.scale, status=status)
+    attn_ms, attn_min = time_call(attention_only, stream, reps=max(5, min(K, 20)))
+    ms_step, e2e_ms, attn_ms = dist.max_over_ranks(ranks, [ms_step, e2e_ms, attn_ms], dev)
     peak, peak_src = tensor_peak()
     tflops = flops / (ms_step * 1e-3) / 1e12
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     line = {
         "metric": "prefill TFLOP/s (causal attention, 4*D flops per query-key pair)",
         "value": world * tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
@@ -777,14 +782,16 @@ def run_prefill_bench(args, ranks, world, rank, local):
                    "num_heads": H, "head_dim": D, "block_size": w.block_size,
                    "l2": "q, k, v, out 1.3 GB per step >> 126 MB L2",
                    "parallelism": f"independent prompts per GPU x{world}",
-                   "path": "pa_prefill (causal attention; the kernel stores the prompts' keys "
-                           "and values from its tiles)"},
+                   "path": "pa_prefill (causal attention; two warps of each CTA store the "
+                           "prompts' keys and values in the same launch)"},
         "prefill_tokens_per_s": world * T / (ms_step * 1e-3),
-        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": tflops / peak, "traffic": None,
-                     "kernel": "prefill_tc_kernel (tcgen05, TMEM accumulators, cache store "
-                               "from the K/V tiles)",
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None,
+                     "kernel": "prefill_tc_kernel (tcgen05, TMEM accumulators; the one launch "
+                               "of the step)",
                      "peak_source": peak_src, "algorithmic_flops_per_launch": flops},
+        "attention_without_store": {"ms": attn_ms, "ms_min": attn_min,
+                                    "tflops": attn_tflops},
         "reuse_sweep": sweep,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 3 * w.q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,

@@ -414,12 +414,13 @@ int pa_paged_attn_decode_fp8_gqa(void* out, const void* q, const void* k_cache,
  *   k_cache, v_cache, slot_mapping, block_size, num_blocks
  *                  the pool and each token's slot, as for pa_kv_cache_write;
  *                  k_cache NULL skips the store (attention only)
- * On the tcgen05 kernel (the default) with block_size 8, 16 or 32 the store
- * is done by the attention kernel itself, from the key and value tiles it
- * has loaded: a block of block_size tokens whose slots fill one physical
- * block in order goes out as one tiled copy, other tokens row by row;
- * otherwise a separate cache write runs first.  Either way the pool holds
- * the same bits afterwards.
+ * On the tcgen05 kernel (the default) the store is done inside the
+ * attention launch, by warps of its own that copy the prompts' key and
+ * value rows to their slots while the others compute; on the warp-level
+ * kernel a separate cache write runs first.  Either way the pool holds the
+ * bits of pa_kv_cache_write afterwards (tokens of a prompt longer than
+ * max_seqlen past max_seqlen are neither computed nor, on the tcgen05
+ * kernel, stored).
  * Support: head_dim 64 or 128; num_seqs <= 65535.  Returns PA_OK or
  * PA_ERR_INVALID / PA_ERR_CUDA.
  */

@@ -17,12 +17,6 @@ std::atomic<int64_t> g_gqa_kernel{0};
 std::atomic<int64_t> g_prefill_kernel{0};
 std::atomic<int64_t> g_prefix_key_bits{64};
 std::atomic<int64_t> g_fp8_kernel{0};
-#ifndef PA_TC_FUSED_STORE
-#define PA_TC_FUSED_STORE 0
-#endif
-// 1: the tcgen05 prompt-phase kernel stores the prompts' keys and values
-// from its own tiles; 0: a separate cache write runs first.
-constexpr bool kPrefillFusedStore = PA_TC_FUSED_STORE != 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -269,15 +263,13 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
   if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return PA_ERR_INVALID;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool tc = g_prefill_kernel.load() != 1;
-  bool fused_store = false;
   if (k_cache) {  // store the prompts' keys and values in their blocks
     if (!v_cache || !slot_mapping || !shape_ok(num_kv_heads, head_dim, block_size) ||
         num_blocks <= 0 || !aligned16(k_cache) || !aligned16(v_cache))
       return PA_ERR_INVALID;
-    // the tcgen05 kernel stores them from its own tiles; otherwise a cache
-    // write runs first
-    fused_store = kPrefillFusedStore && tc && pa::prefill_tc_paged_ok(block_size, num_blocks);
-    if (!fused_store) {
+    // the tcgen05 kernel stores them itself, alongside the attention; the
+    // warp-level kernel after a separate cache write
+    if (!tc) {
       const int rc = from_cuda(pa::launch_kv_cache_write(k, v, k_cache, v_cache, slot_mapping,
                                                          num_tokens, num_kv_heads, head_dim,
                                                          block_size, num_blocks, d_status, st));
@@ -300,7 +292,7 @@ int pa_prefill(void* out, const void* q, const void* k, const void* v, void* k_c
   a.is_bf16 = dt == PA_BF16;
   a.status = d_status;
   a.wait_limit_ns = g_wait_limit_ns.load();
-  if (fused_store) {
+  if (tc && k_cache) {
     a.k_cache = k_cache;
     a.v_cache = v_cache;
     a.block_size = block_size;
@@ -330,6 +322,8 @@ int pa_prefill_with_prefix(void* out, const void* q, const void* k, const void* 
   if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
       !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (slot_mapping && !shape_ok(num_kv_heads, head_dim, block_size)) return PA_ERR_INVALID;
   pa::PrefillArgs a;
   a.out = out;
   a.q = q;
@@ -353,8 +347,8 @@ int pa_prefill_with_prefix(void* out, const void* q, const void* k, const void* 
   a.block_tables = block_tables;
   a.cached_lens = cached_lens;
   a.max_blocks_per_seq = max_blocks_per_seq;
-  a.slot_mapping = slot_mapping;
-  return from_cuda(pa::launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream)));
+  a.slot_mapping = slot_mapping;  // the kernel stores the new tokens' keys and values
+  return from_cuda(pa::launch_prefill_tc(a, st));
 }
 
 int pa_read_probe(const void* buf, size_t bytes, uint32_t* d_sink, int sink_words,

@@ -59,8 +59,8 @@ struct PrefillArgs {
   int64_t wait_limit_ns = 1000000000;
   // tcgen05 kernel only.  The paged cache: with cached_lens, prompt s's first
   // cached_lens[s] tokens are read from it through block_tables (q, k, v and
-  // out then hold the other tokens); with slot_mapping, the prompt tokens'
-  // keys and values are stored in it by the kernel itself.
+  // out then hold the other tokens); with slot_mapping, the new tokens' keys
+  // and values are stored in it by the kernel itself.
   void* k_cache = nullptr;
   void* v_cache = nullptr;
   int block_size = 0;

@@ -200,6 +200,14 @@ __device__ __forceinline__ void tma_store_4d(const void* map, const void* src, i
 }
 
 // Close the current bulk async-group of this thread.
+// Untiled bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from this CTA's shared memory to global memory; completes in
+// this thread's bulk group.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_addr(ssrc)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
