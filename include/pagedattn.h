@@ -232,8 +232,10 @@ size_t pa_paged_attn_decode_shared_workspace_size(int num_groups, int group_size
  *     out[t][h][:] = sum over prefix and tail tokens of softmax(z) * V,
  * the same result as pa_paged_attn_decode over the joined table (up to
  * rounding).  Each shared key and value is read once per group, not once per
- * text: the group's queries run together on the tensor cores, the tails on
- * the multi-head kernel, and a log-sum-exp merge joins the two.
+ * text: the group's queries run together on the tensor cores (a group of
+ * more than 16 texts in subsets of at most 16, the smallest number of equal
+ * subsets, each reading the prefix once), the tails on the multi-head
+ * kernel, and a log-sum-exp merge joins the two.
  *
  *   out, q         [num_groups * group_size][num_heads][head_dim] dt, device
  *   k_cache,v_cache multi-head pool (layout above), device
@@ -241,7 +243,8 @@ size_t pa_paged_attn_decode_shared_workspace_size(int num_groups, int group_size
  *   prefix_lens    [num_groups] int32, device (0 allowed)
  *   tail_tables    [num_groups * group_size][max_tail_blocks] int32, device
  *   tail_lens      [num_groups * group_size] int32, device (0 allowed)
- *   group_size     1 .. 16; block_size 8, 16 or 32
+ *   group_size     1 .. 1024 (num_groups * group_size <= 4096); block_size
+ *                  8, 16 or 32
  *   workspace      at least pa_paged_attn_decode_shared_workspace_size(...)
  *                  bytes, 256-byte aligned, not shared with concurrent calls
  * A text with no tokens at all gets zeros.  pa_split_shared_prefix builds the
@@ -528,12 +531,13 @@ int pa_write_probe(void* buf, size_t bytes, pa_stream_t stream);
 
 /*
  * pa_exp2_probe — a diagnostic with no counterpart in the pages: d_y[i] =
- * 2^d_x[i] for i < n (device float arrays), computed the way the prompt-phase
- * kernel computes part of its softmax weights: method 0 the FMA-pipe
- * polynomial (range reduction to [-1/2, 1/2], degree-5 minimax polynomial,
- * exponent insertion; inputs below -125 give 2^-125), method 1 the
- * exponential unit (ex2.approx.ftz).  Lets a test hold the polynomial to
- * its error bound on the GPU itself.  Returns PA_OK or PA_ERR_INVALID /
+ * 2^d_x[i] for i < n (device float arrays): method 0 an FMA-pipe polynomial
+ * (range reduction to [-1/2, 1/2], degree-5 minimax polynomial, exponent
+ * insertion; inputs below -125 give 2^-125), method 1 the exponential unit
+ * (ex2.approx.ftz), which the softmax kernels use.  The polynomial was
+ * built to take part of the prompt phase's exponentials and measured
+ * slower there; this entry point lets a test hold it to its error bound on
+ * the GPU itself.  Returns PA_OK or PA_ERR_INVALID /
  * PA_ERR_CUDA.
  */
 int pa_exp2_probe(const float* d_x, float* d_y, int64_t n, int method, pa_stream_t stream);

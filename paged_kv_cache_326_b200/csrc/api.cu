@@ -448,7 +448,7 @@ int pa_paged_attn_decode_shared(void* out, const void* q, const void* k_cache,
                                 pa_dtype dt, void* workspace, size_t workspace_bytes,
                                 int32_t* d_status, pa_stream_t stream) {
   if (num_groups == 0) return PA_OK;
-  if (num_groups < 0 || group_size < 1 || group_size > 16 ||
+  if (num_groups < 0 || group_size < 1 || group_size > 1024 ||
       static_cast<int64_t>(num_groups) * group_size > 4096 || max_prefix_blocks < 1 ||
       max_tail_blocks < 1 || num_blocks <= 0 || !shape_ok(num_heads, head_dim, block_size) ||
       block_size < 8 || (dt != PA_F16 && dt != PA_BF16))

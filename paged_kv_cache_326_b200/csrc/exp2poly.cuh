@@ -1,7 +1,9 @@
-// 2^x on the FMA pipe, for softmax weights: the exponential unit (MUFU) does
-// one exp2 per lane every four cycles per SM sub-partition, which in the
-// prompt phase is as slow as the tensor cores' products, so part of the
-// weights is computed here instead.
+// 2^x on the FMA pipe.  Built to take part of the prompt phase's softmax
+// weights off the exponential unit (which does 4 exp2 a clock per SM
+// sub-partition, as slow as the tensor cores' products there); on sm_100 it
+// costs about 12 cycles a value against 8.5 on that unit, and every split
+// measured slower, so the softmax kernels do not use it.  It stays for
+// pa_exp2_probe and its test.
 //
 // Method (Cody and Waite's additive range reduction, which for base 2 is
 // exact): x = n + f with n the integer nearest x and f in [-1/2, 1/2]; 2^f

@@ -206,10 +206,12 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
           bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D, GS * D * 2,
                         &bars[st], policy);
         } else {
-          // head h of the group's GS texts: rows Hq * D elements apart
+          // head kv_head(h) of the GS texts of subset h % NSUB of group s
+          // (a group of NSUB * GS texts): rows Hq * D elements apart
+          const int64_t t0 = static_cast<int64_t>(s) * GS * NSUB + (NSUB == 1 ? 0 : h % NSUB) * GS;
           for (int g = 0; g < GS; ++g)
-            bulk_copy_g2s(sQ + g * D * 2, qg + ((static_cast<int64_t>(s) * GS + g) * Hq + h) * D,
-                          D * 2, &bars[st], policy);
+            bulk_copy_g2s(sQ + g * D * 2, qg + ((t0 + g) * Hq + kv_head(h)) * D, D * 2,
+                          &bars[st], policy);
         }
       }
       if (!bad) {
@@ -703,12 +705,18 @@ size_t mma_workspace_for(int num_seqs, const HeadLayout& hl, int head_dim, int b
 
 // The shared-prefix pass: one virtual text per group, one subset of
 // `group_size` query columns (the group's texts) per head.
+// Shared-prefix pass: a group's texts are the columns; a group of more than
+// 16 is split into nsub subsets of gs <= 16 (the smallest count that
+// divides it), one virtual head per (head, subset), each reading the
+// prefix once.
 HeadLayout cascade_head_layout(int num_heads, int group_size) {
   HeadLayout l;
   l.group = 1;
-  l.gs = group_size;
-  l.nsub = 1;
-  l.vheads = num_heads;
+  int nsub = (group_size + 15) / 16;
+  while (group_size % nsub) ++nsub;
+  l.nsub = nsub;
+  l.gs = group_size / nsub;
+  l.vheads = num_heads * nsub;
   return l;
 }
 
@@ -721,7 +729,7 @@ size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
 }
 
 bool mma_cascade_ok(int num_heads, int group_size, int head_dim, int block_size) {
-  return num_heads >= 1 && group_size >= 1 && group_size <= 16 &&
+  return num_heads >= 1 && group_size >= 1 && group_size <= 1024 &&
          (head_dim == 64 || head_dim == 128) &&
          (block_size == 8 || block_size == 16 || block_size == 32);
 }

@@ -64,7 +64,7 @@ write_probe_kernel(uint4* __restrict__ buf, int64_t nvec) {
   }
 }
 
-// y[i] = 2^x[i], by the softmax kernels' FMA-pipe polynomial (method 0) or by
+// y[i] = 2^x[i], by the FMA-pipe polynomial of exp2poly.cuh (method 0) or by
 // the exponential unit's ex2.approx (method 1).
 __global__ void __launch_bounds__(256)
 exp2_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n, int method) {

@@ -58,8 +58,10 @@ __device__ __forceinline__ void unit_range(const int32_t* header, int s, int h, 
   n = sp.unit_of(a + ns - 1) - u_lo + 1;
 }
 
-// One warp per (text, head): the prefix pass's records for column j of group
-// t / gs, then the tail pass's records for text t, merged in that fixed order
+// One warp per (text, head): the prefix pass's records for text j of group
+// t / gs (column j % gsub of the subset j / gsub, which the prefix pass ran
+// as virtual head h * nsub + j / gsub), then the tail pass's records for
+// text t, merged in that fixed order
 // (so the result does not depend on which warp produced a record).  Every
 // lane reads the same records, so the running maximum is warp-uniform.
 template <typename T, int D>
@@ -67,7 +69,8 @@ __global__ void __launch_bounds__(256)
 shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_p,
                            const float* __restrict__ rec_p, const int32_t* __restrict__ hdr_t,
                            const float* __restrict__ rec_t, unsigned long long* __restrict__ grab_p,
-                           unsigned long long* __restrict__ grab_t, int num_groups, int gs, int H) {
+                           unsigned long long* __restrict__ grab_t, int num_groups, int gs, int H,
+                           int nsub) {
   griddep_wait();
   // Both passes are done with their grain counters: zero them for the next call
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -84,14 +87,17 @@ shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_
   const int h = item - t * H;
   const int g = t / gs;
   const int j = t - g * gs;
+  const int gsub = gs / nsub;                    // texts per subset
+  const int vh = h * nsub + j / gsub, col = j % gsub;
+  const int Hp = H * nsub;                       // virtual heads of the prefix pass
   int pu, pn, tu, tn;
-  unit_range(hdr_p, g, h, H, pu, pn);
+  unit_range(hdr_p, g, vh, Hp, pu, pn);
   unit_range(hdr_t, t, h, H, tu, tn);
-  const int64_t seg_p = static_cast<int64_t>(g) * H + h;
+  const int64_t seg_p = static_cast<int64_t>(g) * Hp + vh;
   const int64_t seg_t = static_cast<int64_t>(t) * H + h;
   const int n = pn + tn;
   auto rec = [&](int i) -> const float* {
-    return i < pn ? rec_p + ((pu + i + seg_p) * gs + j) * RS
+    return i < pn ? rec_p + ((pu + i + seg_p) * gsub + col) * RS
                   : rec_t + (tu + (i - pn) + seg_t) * RS;
   };
 
@@ -156,6 +162,15 @@ shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_
   }
 }
 
+// subsets of the prefix pass for a group of `group_size` texts (as the
+// grouped-query kernel's cascade layout: the smallest count of at most 16
+// texts each that divides the group)
+int nsub_of(int group_size) {
+  int nsub = (group_size + 15) / 16;
+  while (group_size % nsub) ++nsub;
+  return nsub;
+}
+
 template <typename T, int D>
 cudaError_t launch_shared_merge(const SharedPrefixArgs& a, const char* ws_p, int S_p,
                                 const char* ws_t, int S_t, cudaStream_t stream) {
@@ -178,7 +193,7 @@ cudaError_t launch_shared_merge(const SharedPrefixArgs& a, const char* ws_p, int
       reinterpret_cast<const float*>(ws_t + header_bytes(S_t) + kGrabBytes),
       reinterpret_cast<unsigned long long*>(const_cast<char*>(ws_p) + header_bytes(S_p)),
       reinterpret_cast<unsigned long long*>(const_cast<char*>(ws_t) + header_bytes(S_t)),
-      a.num_groups, a.group_size, a.num_heads);
+      a.num_groups, a.group_size, a.num_heads, nsub_of(a.group_size));
 }
 
 // The two passes' workspaces, one after the other (256-byte aligned).

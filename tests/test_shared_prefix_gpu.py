@@ -65,6 +65,11 @@ CASES = [
     (torch.float16, 64, 32, 2, 16, (20, 130), (1, 50), 2),
     (torch.bfloat16, 64, 16, 5, 1, (1, 60), (1, 20), 2),
     (torch.float16, 128, 32, 3, 5, (2, 9), (1, 6), 2),   # prompts shorter than a block
+    # groups of more than 16 texts: the prefix pass in subsets of at most 16
+    (torch.float16, 128, 16, 2, 24, (30, 120), (1, 40), 3),   # 2 subsets of 12
+    (torch.bfloat16, 64, 8, 1, 40, (10, 80), (1, 30), 2),     # 4 subsets of 10
+    (torch.float16, 128, 16, 1, 17, (20, 60), (1, 20), 2),    # 17 subsets of 1
+    (torch.float16, 128, 32, 2, 32, (40, 150), (1, 50), 2),   # 2 subsets of 16
 ]
 
 
