@@ -188,10 +188,13 @@ class StagedInputs:
 def e2e_pipelined(run, staged: StagedInputs, outs, houts, steps: int, stream, copy_stream):
     """Time ``steps`` end-to-end steps on the device.  Step i: the copy stream
     uploads the inputs into device buffer i % 2 (once step i - 2 is done with
-    it), the compute stream runs ``run(inputs, out)`` on it, and the copy
-    stream reads that step's output back into pinned host memory.  So one
+    it), the compute stream runs ``run(inputs, out)`` on it, and a second copy
+    stream reads that step's output back into pinned host memory.  Uploads
+    and readbacks have streams of their own, so step i + 1's upload does not
+    queue behind step i's readback (which waits for step i's kernels): one
     step's copies overlap the neighbouring steps' kernels.  Returns ms/step."""
     n = len(staged.dev)
+    read_stream = torch.cuda.Stream(device=stream.device)
     in_ready = [torch.cuda.Event() for _ in range(n)]
     computed = [torch.cuda.Event() for _ in range(n)]
     drained = [torch.cuda.Event() for _ in range(n)]
@@ -199,6 +202,7 @@ def e2e_pipelined(run, staged: StagedInputs, outs, houts, steps: int, stream, co
     torch.cuda.synchronize()
     e0.record(stream)
     copy_stream.wait_stream(stream)
+    read_stream.wait_stream(stream)
     for i in range(steps):
         b = i % n
         with torch.cuda.stream(copy_stream):
@@ -211,11 +215,12 @@ def e2e_pipelined(run, staged: StagedInputs, outs, houts, steps: int, stream, co
             stream.wait_event(drained[b])
         run(staged.views[b], outs[b])
         computed[b].record(stream)
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(computed[b])
+        with torch.cuda.stream(read_stream):
+            read_stream.wait_event(computed[b])
             houts[b].copy_(outs[b], non_blocking=True)
-            drained[b].record(copy_stream)
+            drained[b].record(read_stream)
     stream.wait_stream(copy_stream)
+    stream.wait_stream(read_stream)
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / steps

@@ -50,6 +50,12 @@
 
 namespace pa {
 
+#ifndef PA_DECODE_SPLIT_P_F16
+#define PA_DECODE_SPLIT_P_F16 0
+#endif
+// 1: fp16 weights also enter the value products as P_hi + P_lo
+constexpr bool kSplitPF16 = PA_DECODE_SPLIT_P_F16 != 0;
+
 namespace {
 
 #ifndef PA_MMA_WARPS
@@ -392,12 +398,14 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
 
     // ---- O^T += V^T P^T ----
     // P^T operand of token tile mt: rows 0-7 and 8-15 of S^T, each an 8x8
-    // block transposed in registers.  The weights are kept as the sum of two
-    // T values, P = P_hi + P_lo (P_hi = P rounded to T, P_lo = the rest
-    // rounded to T), about 16 significant bits, and both parts are applied:
-    // one T value alone (8 bits for bf16) can cost more than the fp32
-    // contract's error where the weighted values nearly cancel.
-    uint32_t pb[TM][NT][2], pl[TM][NT][2];
+    // block transposed in registers.  For bf16 the weights are kept as the
+    // sum of two bf16 values, P = P_hi + P_lo (P_hi = P rounded, P_lo = the
+    // rest rounded), about 16 significant bits, and both parts are applied:
+    // one bf16 value alone (8 bits) can cost more than the fp32 contract's
+    // error where the weighted values nearly cancel.  fp16 weights (11 bits)
+    // enter once (PA_DECODE_SPLIT_P_F16=1 splits them too).
+    constexpr bool SPLIT = std::is_same<T, __nv_bfloat16>::value || kSplitPF16;
+    uint32_t pb[TM][NT][2], pl[TM][NT][SPLIT ? 2 : 1];
 #pragma unroll
     for (int mt = 0; mt < TM; ++mt)
 #pragma unroll
@@ -408,7 +416,8 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
           const uint32_t hi = Elem<T>::from_float2(x0, x1);
           const float2 back = Elem<T>::to_float2(hi);
           pb[mt][nt][r] = movmatrix_trans(hi);
-          pl[mt][nt][r] = movmatrix_trans(Elem<T>::from_float2(x0 - back.x, x1 - back.y));
+          if constexpr (SPLIT)
+            pl[mt][nt][r] = movmatrix_trans(Elem<T>::from_float2(x0 - back.x, x1 - back.y));
         }
     // Tokens past nvalid hold whatever the pool has there (possibly NaN);
     // their weights are zero, but 0 * NaN is not, so zero those V elements.
@@ -436,7 +445,7 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_16816<T>(o[md][nt], a, pb[mt][nt][0], pb[mt][nt][1]);
-          mma_16816<T>(o[md][nt], a, pl[mt][nt][0], pl[mt][nt][1]);
+          if constexpr (SPLIT) mma_16816<T>(o[md][nt], a, pl[mt][nt][0], pl[mt][nt][1]);
         }
       }
     }

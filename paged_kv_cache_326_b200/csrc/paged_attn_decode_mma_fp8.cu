@@ -38,8 +38,9 @@
 //     pair), and the lane's four value rows fall into eight distinct pieces
 //     per load phase.  The lane owns output dimensions [16g, 16g + 16): one
 //     16-byte piece of each of its rows, bytes of two rows interleaved by
-//     prmt into code pairs for cvt.  P enters as P_hi + P_lo (two fp16
-//     values, about 22 significant bits).
+//     prmt into code pairs for cvt.  P enters rounded to fp16 (11
+//     significant bits, as in the CUDA-core kernels; PA_DECODE_SPLIT_P_F16=1
+//     applies P_hi + P_lo, about 22 bits, at twice the value products).
 // Everything else (the flat chunk order, static runs then grains, partial
 // records and the log-sum-exp merge, bounded waits, programmatic dependent
 // launch) is shared with the other decode kernels.
@@ -54,6 +55,12 @@
 #include "mma_ptx.cuh"
 
 namespace pa {
+
+#ifndef PA_DECODE_SPLIT_P_F16
+#define PA_DECODE_SPLIT_P_F16 0
+#endif
+// 1: the weights enter the value products as P_hi + P_lo
+constexpr bool kSplitPF16 = PA_DECODE_SPLIT_P_F16 != 0;
 
 namespace {
 
@@ -314,13 +321,16 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
 #pragma unroll
     for (int i = 0; i < 4; ++i) pr[i] = fast_exp2(sc[i] - mm);
     l += (pr[0] + pr[1]) + (pr[2] + pr[3]);
-    // P pairs (token g, token g + 8) of each 16-token tile as hi + lo fp16
-    uint32_t ph[2], pl[2];
+    // P pairs (token g, token g + 8) of each 16-token tile in fp16 (and the
+    // rest, when split)
+    uint32_t ph[2], pl[2] = {0u, 0u};
 #pragma unroll
     for (int kt = 0; kt < 2; ++kt) {
       ph[kt] = Elem<__half>::from_float2(pr[2 * kt], pr[2 * kt + 1]);
-      const float2 back = Elem<__half>::to_float2(ph[kt]);
-      pl[kt] = Elem<__half>::from_float2(pr[2 * kt] - back.x, pr[2 * kt + 1] - back.y);
+      if constexpr (kSplitPF16) {
+        const float2 back = Elem<__half>::to_float2(ph[kt]);
+        pl[kt] = Elem<__half>::from_float2(pr[2 * kt] - back.x, pr[2 * kt + 1] - back.y);
+      }
     }
 
     // ---- O^T += V^T P^T ----
@@ -330,8 +340,8 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
       // K positions 2c+8, 2c+9 <- tokens 2c+1, 2c+9 (lane g = 2c + 1)
       const uint32_t b0h = __shfl_sync(0xffffffffu, ph[kt], (2 * c) * 4);
       const uint32_t b1h = __shfl_sync(0xffffffffu, ph[kt], (2 * c + 1) * 4);
-      const uint32_t b0l = __shfl_sync(0xffffffffu, pl[kt], (2 * c) * 4);
-      const uint32_t b1l = __shfl_sync(0xffffffffu, pl[kt], (2 * c + 1) * 4);
+      const uint32_t b0l = kSplitPF16 ? __shfl_sync(0xffffffffu, pl[kt], (2 * c) * 4) : 0u;
+      const uint32_t b1l = kSplitPF16 ? __shfl_sync(0xffffffffu, pl[kt], (2 * c + 1) * 4) : 0u;
       const int t0 = kt * 16 + 2 * c;
       uint4 v0 = lds128(sV + t0 * 128 + ((g ^ (2 * c)) << 4));
       uint4 v1 = lds128(sV + (t0 + 8) * 128 + ((g ^ (2 * c)) << 4));
@@ -356,11 +366,11 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
         e4m3x4_to_half2x2(__byte_perm(x0[wd], x1[wd], 0x5140), a[0], a[1]);
         e4m3x4_to_half2x2(__byte_perm(x2[wd], x3[wd], 0x5140), a[2], a[3]);
         mma_16816<__half>(o[2 * wd], a, b0h, b1h);
-        mma_16816<__half>(o[2 * wd], a, b0l, b1l);
+        if constexpr (kSplitPF16) mma_16816<__half>(o[2 * wd], a, b0l, b1l);
         e4m3x4_to_half2x2(__byte_perm(x0[wd], x1[wd], 0x7362), a[0], a[1]);
         e4m3x4_to_half2x2(__byte_perm(x2[wd], x3[wd], 0x7362), a[2], a[3]);
         mma_16816<__half>(o[2 * wd + 1], a, b0h, b1h);
-        mma_16816<__half>(o[2 * wd + 1], a, b0l, b1l);
+        if constexpr (kSplitPF16) mma_16816<__half>(o[2 * wd + 1], a, b0l, b1l);
       }
     }
 
