@@ -110,11 +110,18 @@ constexpr uint32_t kTileCols = 256, kTmemCols = 512;
 constexpr int64_t kTcDrainNs = 1000000000;
 
 #ifndef PA_TC_PREFETCH
-#define PA_TC_PREFETCH 0
+#define PA_TC_PREFETCH 2
 #endif
-// 1: the softmax's second read of keys 0-31 is issued before the exchange of
-// maxima (more registers live across it); 0: after keys 32-63's weights.
-constexpr bool kTcPrefetch = PA_TC_PREFETCH != 0;
+// When the softmax's second read of keys 0-31 is issued: 1 before the
+// exchange of maxima, 2 right after it (before keys 32-63's weights; 705
+// against 697 TFLOP/s for the attention alone), 0 after keys 32-63's
+// weights (fewest registers live).
+constexpr int kTcPrefetch = PA_TC_PREFETCH;
+#ifndef PA_TC_MAX_ONE_WAIT
+#define PA_TC_MAX_ONE_WAIT 0
+#endif
+// 1: the max pass issues both of its TMEM loads under one wait
+constexpr bool kTcMaxOneWait = PA_TC_MAX_ONE_WAIT != 0;
 
 // max(a, b, c) in one instruction (three-input max.f32 of sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -575,14 +582,30 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
             for (int u = 0; u < 4; ++u)
               mx[u] = fmax3(mx[u], __uint_as_float(v[c + 2 * u]), __uint_as_float(v[c + 2 * u + 1]));
         };
-        load32(0, v0);
-        max_of(v0);
-        load32(1, v1);  // kept for the weights
-        max_of(v1);
+        if constexpr (kTcMaxOneWait) {
+          // both loads in flight, one wait
+          tc::ld32(rbase + kColS + hf * kTcHalf, v0);
+          tc::ld32(rbase + kColS + hf * kTcHalf + 32, v1);
+          tc::wait_ld();
+          if (mask) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (c >= lim_h) v0[c] = __float_as_uint(-INFINITY);
+              if (32 + c >= lim_h) v1[c] = __float_as_uint(-INFINITY);
+            }
+          }
+          max_of(v0);
+          max_of(v1);
+        } else {
+          load32(0, v0);
+          max_of(v0);
+          load32(1, v1);  // kept for the weights
+          max_of(v1);
+        }
         pm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         xmax[jj & 1][t][hf][row] = pm;
         // keys 0-31 again, their load in flight across the exchange
-        if constexpr (kTcPrefetch) tc::ld32(rbase + kColS + hf * kTcHalf, v0);
+        if constexpr (kTcPrefetch == 1) tc::ld32(rbase + kColS + hf * kTcHalf, v0);
       }
       // the pair's maxima meet here; every thread of the tile learns whether
       // any gave up, so all leave together
@@ -623,7 +646,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // partial sums
       // The weights 2^(scale * s - m), two per packed fma; hidden scores are
       // -inf: weight 0.  Keys 32-63 of the half first (still in registers),
-      // then keys 0-31 (read again, the load issued before the exchange).
+      // then keys 0-31 (read again, the load in flight meanwhile).
       // P goes back over the S columns of its own 32 keys as packed 16-bit
       // pairs: keys 16g..16g+15 (g = 0..7 over the block) take columns
       // 32 (g / 2) + 8 (g % 2) .. +7 (fp16), or 16g..16g+7 for P_hi and
@@ -661,8 +684,9 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
         }
       }
       };
+      if constexpr (kTcPrefetch == 2) tc::ld32(rbase + kColS + hf * kTcHalf, v0);
       chunk(v1, 1);
-      if constexpr (!kTcPrefetch) tc::ld32(rbase + kColS + hf * kTcHalf, v0);
+      if constexpr (kTcPrefetch == 0) tc::ld32(rbase + kColS + hf * kTcHalf, v0);
       tc::wait_ld();
       if (mask) {
 #pragma unroll
