@@ -19,7 +19,9 @@
 // (29.5 microseconds: too few CTAs left writing), and the run's CTAs each
 // taking one slice of the source for all destinations (23.5).
 // PA_COPY_STREAMING_STORE=1 writes with st.global.cs (evict-first); it
-// measured no different.
+// measured no different, nor did 8 vectors in flight (21.2 us), 512 threads
+// (21.9) or 128 threads of 8 vectors (21.3); 64 KB pieces were slower
+// (23.3-25.0).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -31,9 +33,18 @@ namespace pa {
 
 namespace {
 
-constexpr int kCopyThreads = 256;
-constexpr int kUnroll = 4;
-constexpr int64_t kVecsPerCta = kCopyThreads * kUnroll * 2;  // 32 KB per CTA
+#ifndef PA_COPY_THREADS
+#define PA_COPY_THREADS 256
+#endif
+#ifndef PA_COPY_UNROLL
+#define PA_COPY_UNROLL 4
+#endif
+#ifndef PA_COPY_ROUNDS
+#define PA_COPY_ROUNDS 2
+#endif
+constexpr int kCopyThreads = PA_COPY_THREADS;
+constexpr int kUnroll = PA_COPY_UNROLL;  // 16-byte vectors in flight per thread
+constexpr int64_t kVecsPerCta = kCopyThreads * kUnroll * PA_COPY_ROUNDS;  // 32 KB per CTA
 
 #ifndef PA_COPY_STREAMING_STORE
 #define PA_COPY_STREAMING_STORE 0
