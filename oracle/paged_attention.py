@@ -223,8 +223,12 @@ def paged_decode_shared(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
     """Decode attention for texts that share a prefix, fp64 ``[S][H][D]``:
     text t (group t // group_size) attends over its group's prefix tokens
     followed by its own tail tokens, i.e. the tokens of the joined table, with
-    the plain definition of ``attend``.  ``pairs`` as in ``paged_decode``."""
+    the plain definition of ``attend``.  The pools may hold fewer heads than q
+    (grouped-query attention): query head h then reads key/value head
+    ``kv_head_of(H, H_kv)[h]``, as in ``paged_decode``.  ``pairs`` as in
+    ``paged_decode``."""
     S, H, D = q.shape
+    kvh = kv_head_of(H, k_cache.shape[1])
     out = np.zeros((S, H, D), dtype=np.float64)
     wanted = None
     if pairs is not None:
@@ -240,7 +244,7 @@ def paged_decode_shared(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
         V = np.concatenate([gather_context(v_cache, prefix_tables[g], prefix_lens[g], block_size),
                             gather_context(v_cache, tail_tables[t], tail_lens[t], block_size)])
         heads = list(range(H)) if wanted is None else wanted[t]
-        full = attend(q[t][heads], K[:, heads, :], V[:, heads, :], scale)
+        full = attend(q[t][heads], K[:, kvh[heads], :], V[:, kvh[heads], :], scale)
         for i, h in enumerate(heads):
             out[t, h] = full[i]
     return out

@@ -654,13 +654,16 @@ PREFIX_PINS = [pin_prefix_rows_of_the_whole_prompt, pin_prefix_brute_force,
 # shared prefixes
 # ---------------------------------------------------------------------------
 
-def _forked_groups(prompt_lens, tail_lens, group_size, H, D, B, seed, dtype=torch.float16):
+def _forked_groups(prompt_lens, tail_lens, group_size, H, D, B, seed, dtype=torch.float16,
+                   Hq=None):
     """Groups of texts built as the block manager builds them, written out by
     hand: the prompt's full blocks are stored once and listed first in every
     member's table; a partial last prompt block is copied into each member's
     first private block (copy on write), followed by the member's own tokens.
     Returns q, the contiguous K and V of every text, the pool, and the prefix
-    and tail tables and lengths."""
+    and tail tables and lengths.  H is the pool's head count; Hq (default H)
+    the query heads."""
+    Hq = H if Hq is None else Hq
     g = torch.Generator().manual_seed(seed)
     G = len(prompt_lens)
     S = G * group_size
@@ -668,7 +671,7 @@ def _forked_groups(prompt_lens, tail_lens, group_size, H, D, B, seed, dtype=torc
                for L in prompt_lens]
     tails = [(torch.randn(L, H, D, generator=g).to(dtype), torch.randn(L, H, D, generator=g).to(dtype))
              for L in tail_lens]
-    q = torch.randn(S, H, D, generator=g).to(dtype)
+    q = torch.randn(S, Hq, D, generator=g).to(dtype)
     nb = sum(L // B for L in prompt_lens) + 8
     nb += sum(-(-(prompt_lens[s // group_size] % B + tail_lens[s]) // B) for s in range(S))
     perm = torch.randperm(nb, generator=torch.Generator().manual_seed(seed + 5)).tolist()
@@ -777,5 +780,23 @@ def pin_split_then_shared_is_decode(split_fn, shared_fn):
     assert np.array_equal(got, ref), "split + shared decode differs from paged decode"
 
 
-SHARED_PINS = [pin_shared_vs_unpaged_sdpa, pin_shared_brute_force_and_empty]
+def pin_shared_grouped_query_vs_unpaged_sdpa(shared_fn):
+    """Grouped-query pools: two groups of three forked texts, 6 query heads
+    over 2 key/value heads (query head h reads key/value head h // 3),
+    against torch's fp64 attention on each text's contiguous tokens with the
+    key/value heads repeated for their query heads; a mistake in the head
+    map (h for h // 3, or h % 2) fails it."""
+    H, Hq, D, B, gs = 2, 6, 8, 4, 3
+    q, K, V, kc, vc, pt, pl, tt, tl = _forked_groups([13, 8], [1, 5, 3, 2, 0, 7], gs, H, D, B,
+                                                     613, Hq=Hq)
+    got = shared_fn(f64(q), f64(kc), f64(vc), pt, pl, tt, tl, gs, 0.35, B)
+    rep = Hq // H
+    ref = sdpa_contiguous(q, [k.repeat_interleave(rep, dim=1) for k in K],
+                          [v.repeat_interleave(rep, dim=1) for v in V], 0.35)
+    err = np.abs(got - ref).max()
+    assert err <= 1e-12, f"grouped-query shared prefix vs unpaged sdpa: max err {err}"
+
+
+SHARED_PINS = [pin_shared_vs_unpaged_sdpa, pin_shared_brute_force_and_empty,
+               pin_shared_grouped_query_vs_unpaged_sdpa]
 SPLIT_PINS = [pin_split_worked_example]

@@ -426,10 +426,30 @@ def _shared_with(group_of=None, use_prefix=True, use_tail=True):
     return fn
 
 
+def _shared_head_map_mod():
+    """Grouped-query mistake: query head h reads key/value head h % H_kv
+    instead of h // (H / H_kv)."""
+    def fn(q, kc, vc, pt, pl, tt, tl, gs, scale, B):
+        S, H, D = q.shape
+        Hkv = kc.shape[1]
+        out = np.zeros((S, H, D))
+        for t in range(S):
+            g = t // gs
+            K = np.concatenate([oracle.gather_context(kc, pt[g], pl[g], B),
+                                oracle.gather_context(kc, tt[t], tl[t], B)])
+            V = np.concatenate([oracle.gather_context(vc, pt[g], pl[g], B),
+                                oracle.gather_context(vc, tt[t], tl[t], B)])
+            heads = np.arange(H) % Hkv
+            out[t] = oracle.attend(q[t], K[:, heads, :], V[:, heads, :], scale)
+        return out
+    return fn
+
+
 SHARED_MUTANTS = {
     "prefix_of_wrong_group": _shared_with(group_of=lambda t, gs, G: t % G),
     "prefix_dropped": _shared_with(use_prefix=False),
     "tail_dropped": _shared_with(use_tail=False),
+    "grouped_query_head_map_mod": _shared_head_map_mod(),
 }
 
 
