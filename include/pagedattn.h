@@ -262,6 +262,40 @@ int pa_paged_attn_decode_shared(void* out, const void* q, const void* k_cache,
                                 int32_t* d_status, pa_stream_t stream);
 
 /*
+ * pa_paged_attn_decode_shared_gqa_workspace_size — as
+ * pa_paged_attn_decode_shared_workspace_size, for pools of num_kv_heads
+ * key/value heads (num_heads a multiple of it; else 0).
+ */
+size_t pa_paged_attn_decode_shared_gqa_workspace_size(int num_groups, int group_size,
+                                                      int num_heads, int num_kv_heads,
+                                                      int head_dim, int block_size,
+                                                      int max_prefix_blocks, int max_tail_blocks);
+
+/*
+ * pa_paged_attn_decode_shared_gqa — pa_paged_attn_decode_shared over a pool
+ * of num_kv_heads key/value heads shared by num_heads query heads ("The KV
+ * Cache and PagedAttention", section "What Came After": heads that share a
+ * key/value set; section "Shared, Copied on Write": samples that share a
+ * prompt's blocks): query head h reads key/value head
+ * h / (num_heads / num_kv_heads).  The prefix pass takes, per key/value
+ * head, the group's (text, query head) pairs as its tensor-core columns, in
+ * subsets of at most 16, so each shared key and value is read once per
+ * subset; the tails run on the grouped-query decode.
+ *   k_cache,v_cache [num_blocks][num_kv_heads][block_size][head_dim] dt
+ *   workspace      pa_paged_attn_decode_shared_gqa_workspace_size(...) bytes
+ * Other arguments and errors as for pa_paged_attn_decode_shared.
+ */
+int pa_paged_attn_decode_shared_gqa(void* out, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* prefix_tables,
+                                    const int32_t* prefix_lens, int max_prefix_blocks,
+                                    const int32_t* tail_tables, const int32_t* tail_lens,
+                                    int max_tail_blocks, float scale, int num_groups,
+                                    int group_size, int num_heads, int num_kv_heads,
+                                    int head_dim, int block_size, int64_t num_blocks, pa_dtype dt,
+                                    void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                    pa_stream_t stream);
+
+/*
  * pa_split_shared_prefix — host only: cut ordinary block tables (as
  * pa_bm_export writes them) of num_seqs = groups * group_size texts into the
  * inputs of pa_paged_attn_decode_shared.  A group's prefix is its longest run

@@ -100,6 +100,11 @@ _SIGNATURES = {
     "pa_paged_attn_decode_shared": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32,
                                            _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _vp,
                                            _sz, _vp, _vp]),
+    "pa_paged_attn_decode_shared_gqa_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32,
+                                                               _i32, _i32, _i32]),
+    "pa_paged_attn_decode_shared_gqa": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                               _i32, _f32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                               _i64, _i32, _vp, _sz, _vp, _vp]),
     "pa_split_shared_prefix": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp,
                                       _i32, _vp]),
     "pa_bm_create": (_vp, [_i64, _i32, _u64]),
@@ -488,10 +493,15 @@ def pa_paged_attn_decode_gqa(out: torch.Tensor, q: torch.Tensor, k_cache: torch.
 
 def pa_paged_attn_decode_shared_workspace_size(num_groups: int, group_size: int, num_heads: int,
                                                head_dim: int, block_size: int,
-                                               max_prefix_blocks: int, max_tail_blocks: int) -> int:
-    return int(lib().pa_paged_attn_decode_shared_workspace_size(
-        num_groups, group_size, num_heads, head_dim, block_size, max_prefix_blocks,
-        max_tail_blocks))
+                                               max_prefix_blocks: int, max_tail_blocks: int,
+                                               num_kv_heads: Optional[int] = None) -> int:
+    if num_kv_heads is None or num_kv_heads == num_heads:
+        return int(lib().pa_paged_attn_decode_shared_workspace_size(
+            num_groups, group_size, num_heads, head_dim, block_size, max_prefix_blocks,
+            max_tail_blocks))
+    return int(lib().pa_paged_attn_decode_shared_gqa_workspace_size(
+        num_groups, group_size, num_heads, num_kv_heads, head_dim, block_size,
+        max_prefix_blocks, max_tail_blocks))
 
 
 def pa_paged_attn_decode_shared(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
@@ -502,13 +512,14 @@ def pa_paged_attn_decode_shared(out: torch.Tensor, q: torch.Tensor, k_cache: tor
                                 status: Optional[torch.Tensor] = None,
                                 stream=None) -> torch.Tensor:
     """Decode for groups of ``group_size`` consecutive texts sharing a prefix:
-    out, q [G*group_size][H][D]; caches [N][H][B][D]; prefix_tables
-    [G][max_prefix_blocks], prefix_lens [G]; tail_tables
+    out, q [G*group_size][H][D]; caches [N][H_kv][B][D] (H_kv == H:
+    multi-head; a divisor of H: grouped-query, pa_paged_attn_decode_shared_gqa);
+    prefix_tables [G][max_prefix_blocks], prefix_lens [G]; tail_tables
     [G*group_size][max_tail_blocks], tail_lens [G*group_size] (int32)."""
     S, H, D = q.shape
-    N, H2, B, D2 = k_cache.shape
-    if out.shape != q.shape or v_cache.shape != k_cache.shape or (H2, D2) != (H, D):
-        raise ValueError("shape mismatch")
+    N, Hkv, B, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D or H % Hkv:
+        raise ValueError("shape mismatch (num_heads must be a multiple of num_kv_heads)")
     if group_size < 1 or S % group_size:
         raise ValueError("the number of texts must be a multiple of group_size")
     G = S // group_size
@@ -521,7 +532,7 @@ def pa_paged_attn_decode_shared(out: torch.Tensor, q: torch.Tensor, k_cache: tor
             raise TypeError("q, out and the caches must share a dtype")
     MP, MT = prefix_tables.shape[1], tail_tables.shape[1]
     if workspace is None:
-        need = pa_paged_attn_decode_shared_workspace_size(G, group_size, H, D, B, MP, MT)
+        need = pa_paged_attn_decode_shared_workspace_size(G, group_size, H, D, B, MP, MT, Hkv)
         if need == 0:
             raise PagedAttnError(PA_ERR_INVALID, "pa_paged_attn_decode_shared_workspace_size")
         key = (q.device.index if q.device.index is not None else torch.cuda.current_device(),
@@ -530,16 +541,19 @@ def pa_paged_attn_decode_shared(out: torch.Tensor, q: torch.Tensor, k_cache: tor
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
             _ws_cache[key] = workspace
-    code = lib().pa_paged_attn_decode_shared(
-        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
-        _cuda(prefix_tables, "prefix_tables", torch.int32),
-        _cuda(prefix_lens, "prefix_lens", torch.int32), MP,
-        _cuda(tail_tables, "tail_tables", torch.int32),
-        _cuda(tail_lens, "tail_lens", torch.int32), MT, float(scale), G, int(group_size), H, D,
-        B, N, _dtype_code(q), _cuda(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(), _status_ptr(status),
-        _stream(stream, q.device))
-    _check(code, "pa_paged_attn_decode_shared")
+    head = (_cuda(out, "out"), _cuda(q, "q"), _cuda(k_cache, "k_cache"),
+            _cuda(v_cache, "v_cache"), _cuda(prefix_tables, "prefix_tables", torch.int32),
+            _cuda(prefix_lens, "prefix_lens", torch.int32), MP,
+            _cuda(tail_tables, "tail_tables", torch.int32),
+            _cuda(tail_lens, "tail_lens", torch.int32), MT, float(scale), G, int(group_size), H)
+    tail = (D, B, N, _dtype_code(q), _cuda(workspace, "workspace"),
+            workspace.numel() * workspace.element_size(), _status_ptr(status),
+            _stream(stream, q.device))
+    if Hkv == H:
+        _check(lib().pa_paged_attn_decode_shared(*head, *tail), "pa_paged_attn_decode_shared")
+    else:
+        _check(lib().pa_paged_attn_decode_shared_gqa(*head, Hkv, *tail),
+               "pa_paged_attn_decode_shared_gqa")
     return out
 
 

@@ -61,6 +61,61 @@ int64_t option_prefix_key_bits() { return g_prefix_key_bits.load(); }
 int64_t option_fp8_kernel() { return g_fp8_kernel.load(); }
 }  // namespace pa
 
+namespace {
+
+// Checks shared by the shared-prefix entry points, then the launch.
+int shared_common(void* out, const void* q, const void* k_cache, const void* v_cache,
+                  const int32_t* prefix_tables, const int32_t* prefix_lens,
+                  int max_prefix_blocks, const int32_t* tail_tables, const int32_t* tail_lens,
+                  int max_tail_blocks, float scale, int num_groups, int group_size, int num_heads,
+                  int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                  pa_dtype dt, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                  pa_stream_t stream) {
+  if (num_groups == 0) return PA_OK;
+  if (num_groups < 0 || group_size < 1 || group_size > 1024 ||
+      static_cast<int64_t>(num_groups) * group_size > 4096 || max_prefix_blocks < 1 ||
+      max_tail_blocks < 1 || num_blocks <= 0 || num_heads < 1 || num_kv_heads < 1 ||
+      num_heads % num_kv_heads || !shape_ok(num_kv_heads, head_dim, block_size) ||
+      block_size < 8 || (dt != PA_F16 && dt != PA_BF16))
+    return PA_ERR_INVALID;
+  if (!out || !q || !k_cache || !v_cache || !prefix_tables || !prefix_lens || !tail_tables ||
+      !tail_lens || !workspace)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return PA_ERR_INVALID;
+  if (!pa::mma_decode_pool_ok(num_kv_heads, block_size, num_blocks)) return PA_ERR_INVALID;
+  pa::SharedPrefixArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.prefix_tables = prefix_tables;
+  a.prefix_lens = prefix_lens;
+  a.max_prefix_blocks = max_prefix_blocks;
+  a.tail_tables = tail_tables;
+  a.tail_lens = tail_lens;
+  a.max_tail_blocks = max_tail_blocks;
+  a.scale = scale;
+  a.num_groups = num_groups;
+  a.group_size = group_size;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.is_bf16 = dt == PA_BF16;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  a.status = d_status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.forced_warps = g_decode_warps.load();
+  return from_cuda(
+      pa::launch_paged_attn_decode_shared(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* pa_status_string(int code) {
@@ -434,9 +489,21 @@ size_t pa_paged_attn_decode_shared_workspace_size(int num_groups, int group_size
                                                   int head_dim, int block_size,
                                                   int max_prefix_blocks, int max_tail_blocks) {
   if (max_prefix_blocks < 1 || max_tail_blocks < 1) return 0;
-  return pa::shared_prefix_workspace_bytes(num_groups, group_size, num_heads, head_dim,
-                                           block_size, max_prefix_blocks, max_tail_blocks,
-                                           g_decode_warps.load());
+  return pa::shared_prefix_workspace_bytes(num_groups, group_size, num_heads, num_heads,
+                                           head_dim, block_size, max_prefix_blocks,
+                                           max_tail_blocks, g_decode_warps.load());
+}
+
+size_t pa_paged_attn_decode_shared_gqa_workspace_size(int num_groups, int group_size,
+                                                      int num_heads, int num_kv_heads,
+                                                      int head_dim, int block_size,
+                                                      int max_prefix_blocks, int max_tail_blocks) {
+  if (max_prefix_blocks < 1 || max_tail_blocks < 1 || num_kv_heads < 1 ||
+      num_heads % num_kv_heads)
+    return 0;
+  return pa::shared_prefix_workspace_bytes(num_groups, group_size, num_heads, num_kv_heads,
+                                           head_dim, block_size, max_prefix_blocks,
+                                           max_tail_blocks, g_decode_warps.load());
 }
 
 int pa_paged_attn_decode_shared(void* out, const void* q, const void* k_cache,
@@ -447,45 +514,25 @@ int pa_paged_attn_decode_shared(void* out, const void* q, const void* k_cache,
                                 int num_heads, int head_dim, int block_size, int64_t num_blocks,
                                 pa_dtype dt, void* workspace, size_t workspace_bytes,
                                 int32_t* d_status, pa_stream_t stream) {
-  if (num_groups == 0) return PA_OK;
-  if (num_groups < 0 || group_size < 1 || group_size > 1024 ||
-      static_cast<int64_t>(num_groups) * group_size > 4096 || max_prefix_blocks < 1 ||
-      max_tail_blocks < 1 || num_blocks <= 0 || !shape_ok(num_heads, head_dim, block_size) ||
-      block_size < 8 || (dt != PA_F16 && dt != PA_BF16))
-    return PA_ERR_INVALID;
-  if (!out || !q || !k_cache || !v_cache || !prefix_tables || !prefix_lens || !tail_tables ||
-      !tail_lens || !workspace)
-    return PA_ERR_INVALID;
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return PA_ERR_INVALID;
-  if (!pa::mma_decode_pool_ok(num_heads, block_size, num_blocks)) return PA_ERR_INVALID;
-  pa::SharedPrefixArgs a;
-  a.out = out;
-  a.q = q;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.prefix_tables = prefix_tables;
-  a.prefix_lens = prefix_lens;
-  a.max_prefix_blocks = max_prefix_blocks;
-  a.tail_tables = tail_tables;
-  a.tail_lens = tail_lens;
-  a.max_tail_blocks = max_tail_blocks;
-  a.scale = scale;
-  a.num_groups = num_groups;
-  a.group_size = group_size;
-  a.num_heads = num_heads;
-  a.head_dim = head_dim;
-  a.block_size = block_size;
-  a.num_blocks = num_blocks;
-  a.is_bf16 = dt == PA_BF16;
-  a.workspace = workspace;
-  a.workspace_bytes = workspace_bytes;
-  a.status = d_status;
-  a.wait_limit_ns = g_wait_limit_ns.load();
-  a.forced_warps = g_decode_warps.load();
-  return from_cuda(
-      pa::launch_paged_attn_decode_shared(a, reinterpret_cast<cudaStream_t>(stream)));
+  return shared_common(out, q, k_cache, v_cache, prefix_tables, prefix_lens, max_prefix_blocks,
+                       tail_tables, tail_lens, max_tail_blocks, scale, num_groups, group_size,
+                       num_heads, num_heads, head_dim, block_size, num_blocks, dt, workspace,
+                       workspace_bytes, d_status, stream);
+}
+
+int pa_paged_attn_decode_shared_gqa(void* out, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* prefix_tables,
+                                    const int32_t* prefix_lens, int max_prefix_blocks,
+                                    const int32_t* tail_tables, const int32_t* tail_lens,
+                                    int max_tail_blocks, float scale, int num_groups,
+                                    int group_size, int num_heads, int num_kv_heads,
+                                    int head_dim, int block_size, int64_t num_blocks, pa_dtype dt,
+                                    void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                    pa_stream_t stream) {
+  return shared_common(out, q, k_cache, v_cache, prefix_tables, prefix_lens, max_prefix_blocks,
+                       tail_tables, tail_lens, max_tail_blocks, scale, num_groups, group_size,
+                       num_heads, num_kv_heads, head_dim, block_size, num_blocks, dt, workspace,
+                       workspace_bytes, d_status, stream);
 }
 
 }  // extern "C"

@@ -163,13 +163,29 @@ size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
                                   int block_size, int max_blocks_per_seq, int64_t forced_warps);
 cudaError_t launch_paged_attn_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 
-// The shared-prefix pass of the grouped-query kernel (a.cascade set, a
-// multi-head pool): a.num_seqs groups of `group_size` texts, each group's
-// texts' queries as the columns of one key/value head.  Partial records
-// only, no merge.
-bool mma_cascade_ok(int num_heads, int group_size, int head_dim, int block_size);
-size_t mma_cascade_workspace_bytes(int num_groups, int group_size, int num_heads, int head_dim,
-                                   int block_size, int max_blocks_per_seq, int64_t forced_warps);
+// A decode launch's split of query heads: per key/value head nsub work
+// subsets of gs query heads (or, in the shared-prefix pass, of gs
+// (text, query head) columns), vheads virtual heads in all.  Records of a
+// unit hold gs columns.
+struct DecodeLayout {
+  int nsub;
+  int gs;
+  int vheads;
+};
+DecodeLayout mma_decode_layout(int num_heads, int num_kv_heads);
+DecodeLayout mma_cascade_layout(int num_heads, int num_kv_heads, int group_size);
+// The layout launch_paged_attn_decode uses for these arguments.
+DecodeLayout decode_layout(const DecodeArgs& a);
+
+// The shared-prefix pass of the grouped-query kernel (a.cascade set):
+// a.num_seqs groups of `group_size` texts; the columns of a key/value head
+// are the group's (text, query head) pairs.  Partial records only, no
+// merge.
+bool mma_cascade_ok(int num_heads, int num_kv_heads, int group_size, int head_dim,
+                    int block_size);
+size_t mma_cascade_workspace_bytes(int num_groups, int group_size, int num_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int max_blocks_per_seq, int64_t forced_warps);
 cudaError_t launch_paged_attn_decode_mma_cascade(const DecodeArgs& a, int group_size,
                                                  cudaStream_t stream);
 
@@ -190,6 +206,7 @@ struct SharedPrefixArgs {
   int num_groups;
   int group_size;
   int num_heads;
+  int num_kv_heads;
   int head_dim;
   int block_size;
   int64_t num_blocks;
@@ -200,8 +217,9 @@ struct SharedPrefixArgs {
   int64_t wait_limit_ns;
   int64_t forced_warps;
 };
-size_t shared_prefix_workspace_bytes(int num_groups, int group_size, int num_heads, int head_dim,
-                                     int block_size, int max_prefix_blocks, int max_tail_blocks,
+size_t shared_prefix_workspace_bytes(int num_groups, int group_size, int num_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int max_prefix_blocks, int max_tail_blocks,
                                      int64_t forced_warps);
 cudaError_t launch_paged_attn_decode_shared(const SharedPrefixArgs& a, cudaStream_t stream);
 

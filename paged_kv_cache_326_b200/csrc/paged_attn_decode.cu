@@ -756,6 +756,17 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
   return bytes;
 }
 
+DecodeLayout decode_layout(const DecodeArgs& a) {
+  // the same choice of kernel as launch_paged_attn_decode below
+  const int64_t mode = option_gqa_kernel();
+  const bool mma_ok = !a.slot_mapping && !a.fp8 &&
+                      mma_decode_shape_ok(a.num_heads, a.num_kv_heads, a.head_dim, a.block_size) &&
+                      mma_decode_pool_ok(a.num_kv_heads, a.block_size, a.num_blocks);
+  if (mma_ok && mode != 1) return mma_decode_layout(a.num_heads, a.num_kv_heads);
+  const HeadLayout hl = head_layout(a.num_heads, a.num_kv_heads);
+  return DecodeLayout{hl.nsub, hl.gs, hl.vheads};
+}
+
 cudaError_t launch_paged_attn_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (!decode_sizes_supported(a.num_seqs, a.num_heads, a.num_kv_heads, a.head_dim, a.block_size,
                               a.max_blocks_per_seq))

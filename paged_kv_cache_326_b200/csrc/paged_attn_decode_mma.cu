@@ -212,12 +212,18 @@ paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
           bulk_copy_g2s(sQ, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D, GS * D * 2,
                         &bars[st], policy);
         } else {
-          // head kv_head(h) of the GS texts of subset h % NSUB of group s
-          // (a group of NSUB * GS texts): rows Hq * D elements apart
-          const int64_t t0 = static_cast<int64_t>(s) * GS * NSUB + (NSUB == 1 ? 0 : h % NSUB) * GS;
-          for (int g = 0; g < GS; ++g)
-            bulk_copy_g2s(sQ + g * D * 2, qg + ((t0 + g) * Hq + kv_head(h)) * D, D * 2,
-                          &bars[st], policy);
+          // Shared-prefix pass: the columns of group s's key/value head
+          // kv_head(h) are its (text, query head) pairs, text-major, in
+          // NSUB subsets of GS; this unit has subset h % NSUB.  Column c is
+          // text c / G of the group and query head kv_head(h) * G + c % G.
+          const int sub = NSUB == 1 ? 0 : h % NSUB;
+          const int64_t text0 = static_cast<int64_t>(s) * (GS * NSUB / G);
+          for (int g = 0; g < GS; ++g) {
+            const int c = sub * GS + g;
+            const int64_t text = text0 + c / G;
+            const int qh = kv_head(h) * G + c % G;
+            bulk_copy_g2s(sQ + g * D * 2, qg + (text * Hq + qh) * D, D * 2, &bars[st], policy);
+          }
         }
       }
       if (!bad) {
@@ -714,18 +720,20 @@ size_t mma_workspace_for(int num_seqs, const HeadLayout& hl, int head_dim, int b
 
 // The shared-prefix pass: one virtual text per group, one subset of
 // `group_size` query columns (the group's texts) per head.
-// Shared-prefix pass: a group's texts are the columns; a group of more than
-// 16 is split into nsub subsets of gs <= 16 (the smallest count that
-// divides it), one virtual head per (head, subset), each reading the
-// prefix once.
-HeadLayout cascade_head_layout(int num_heads, int group_size) {
+// Shared-prefix pass: the columns of a key/value head are the group's
+// (text, query head) pairs, group_size * G of them; more than 16 are split
+// into nsub subsets of gs <= 16 (the smallest count that divides them), one
+// virtual head per (key/value head, subset), each reading the prefix once.
+HeadLayout cascade_head_layout(int num_heads, int num_kv_heads, int group_size) {
   HeadLayout l;
-  l.group = 1;
-  int nsub = (group_size + 15) / 16;
-  while (group_size % nsub) ++nsub;
+  if (num_kv_heads < 1 || num_heads < 1 || num_heads % num_kv_heads || group_size < 1) return l;
+  l.group = num_heads / num_kv_heads;
+  const int cols = group_size * l.group;
+  int nsub = (cols + 15) / 16;
+  while (cols % nsub) ++nsub;
   l.nsub = nsub;
-  l.gs = group_size / nsub;
-  l.vheads = num_heads * nsub;
+  l.gs = cols / nsub;
+  l.vheads = num_kv_heads * nsub;
   return l;
 }
 
@@ -737,26 +745,39 @@ size_t mma_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
                            block_size, max_blocks_per_seq, forced_warps);
 }
 
-bool mma_cascade_ok(int num_heads, int group_size, int head_dim, int block_size) {
-  return num_heads >= 1 && group_size >= 1 && group_size <= 1024 &&
+bool mma_cascade_ok(int num_heads, int num_kv_heads, int group_size, int head_dim,
+                    int block_size) {
+  return num_heads >= 1 && num_kv_heads >= 1 && num_heads % num_kv_heads == 0 &&
+         group_size >= 1 && group_size <= 1024 &&
          (head_dim == 64 || head_dim == 128) &&
          (block_size == 8 || block_size == 16 || block_size == 32);
 }
 
-size_t mma_cascade_workspace_bytes(int num_groups, int group_size, int num_heads, int head_dim,
-                                   int block_size, int max_blocks_per_seq, int64_t forced_warps) {
-  if (!mma_cascade_ok(num_heads, group_size, head_dim, block_size)) return 0;
-  return mma_workspace_for(num_groups, cascade_head_layout(num_heads, group_size), head_dim,
-                           block_size, max_blocks_per_seq, forced_warps);
+size_t mma_cascade_workspace_bytes(int num_groups, int group_size, int num_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int max_blocks_per_seq, int64_t forced_warps) {
+  if (!mma_cascade_ok(num_heads, num_kv_heads, group_size, head_dim, block_size)) return 0;
+  return mma_workspace_for(num_groups, cascade_head_layout(num_heads, num_kv_heads, group_size),
+                           head_dim, block_size, max_blocks_per_seq, forced_warps);
+}
+
+DecodeLayout mma_decode_layout(int num_heads, int num_kv_heads) {
+  const HeadLayout l = mma_head_layout(num_heads, num_kv_heads);
+  return DecodeLayout{l.nsub, l.gs, l.vheads};
+}
+
+DecodeLayout mma_cascade_layout(int num_heads, int num_kv_heads, int group_size) {
+  const HeadLayout l = cascade_head_layout(num_heads, num_kv_heads, group_size);
+  return DecodeLayout{l.nsub, l.gs, l.vheads};
 }
 
 cudaError_t launch_paged_attn_decode_mma_cascade(const DecodeArgs& a, int group_size,
                                                  cudaStream_t stream) {
-  if (!a.cascade || a.slot_mapping || a.fp8 || a.num_heads != a.num_kv_heads ||
-      !mma_cascade_ok(a.num_heads, group_size, a.head_dim, a.block_size) ||
+  if (!a.cascade || a.slot_mapping || a.fp8 ||
+      !mma_cascade_ok(a.num_heads, a.num_kv_heads, group_size, a.head_dim, a.block_size) ||
       !mma_decode_pool_ok(a.num_kv_heads, a.block_size, a.num_blocks))
     return cudaErrorInvalidValue;
-  const HeadLayout hl = cascade_head_layout(a.num_heads, group_size);
+  const HeadLayout hl = cascade_head_layout(a.num_heads, a.num_kv_heads, group_size);
   return a.is_bf16 ? mma_dispatch<__nv_bfloat16>(a, hl, stream)
                    : mma_dispatch<__half>(a, hl, stream);
 }

@@ -58,10 +58,12 @@ __device__ __forceinline__ void unit_range(const int32_t* header, int s, int h, 
   n = sp.unit_of(a + ns - 1) - u_lo + 1;
 }
 
-// One warp per (text, head): the prefix pass's records for text j of group
-// t / gs (column j % gsub of the subset j / gsub, which the prefix pass ran
-// as virtual head h * nsub + j / gsub), then the tail pass's records for
-// text t, merged in that fixed order
+// One warp per (text t, query head h): the prefix pass's records for
+// column c = j G + h % G of key/value head h / G of group t / gs (text j of
+// the group, G query heads per key/value head; the prefix pass ran the
+// columns in subsets of gs_p as virtual heads kvh * nsub_p + c / gs_p), then
+// the tail pass's records for text t and query head h (column h % G % gs_t
+// of virtual head kvh * nsub_t + (h % G) / gs_t), merged in that fixed order
 // (so the result does not depend on which warp produced a record).  Every
 // lane reads the same records, so the running maximum is warp-uniform.
 template <typename T, int D>
@@ -70,7 +72,7 @@ shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_
                            const float* __restrict__ rec_p, const int32_t* __restrict__ hdr_t,
                            const float* __restrict__ rec_t, unsigned long long* __restrict__ grab_p,
                            unsigned long long* __restrict__ grab_t, int num_groups, int gs, int H,
-                           int nsub) {
+                           int G, DecodeLayout lp, DecodeLayout lt) {
   griddep_wait();
   // Both passes are done with their grain counters: zero them for the next call
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -87,18 +89,19 @@ shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_
   const int h = item - t * H;
   const int g = t / gs;
   const int j = t - g * gs;
-  const int gsub = gs / nsub;                    // texts per subset
-  const int vh = h * nsub + j / gsub, col = j % gsub;
-  const int Hp = H * nsub;                       // virtual heads of the prefix pass
+  const int kvh = h / G, qq = h - kvh * G;
+  const int c = j * G + qq;                      // column in the prefix pass
+  const int vh_p = kvh * lp.nsub + c / lp.gs, col_p = c % lp.gs;
+  const int vh_t = kvh * lt.nsub + qq / lt.gs, col_t = qq % lt.gs;
   int pu, pn, tu, tn;
-  unit_range(hdr_p, g, vh, Hp, pu, pn);
-  unit_range(hdr_t, t, h, H, tu, tn);
-  const int64_t seg_p = static_cast<int64_t>(g) * Hp + vh;
-  const int64_t seg_t = static_cast<int64_t>(t) * H + h;
+  unit_range(hdr_p, g, vh_p, lp.vheads, pu, pn);
+  unit_range(hdr_t, t, vh_t, lt.vheads, tu, tn);
+  const int64_t seg_p = static_cast<int64_t>(g) * lp.vheads + vh_p;
+  const int64_t seg_t = static_cast<int64_t>(t) * lt.vheads + vh_t;
   const int n = pn + tn;
   auto rec = [&](int i) -> const float* {
-    return i < pn ? rec_p + ((pu + i + seg_p) * gsub + col) * RS
-                  : rec_t + (tu + (i - pn) + seg_t) * RS;
+    return i < pn ? rec_p + ((pu + i + seg_p) * lp.gs + col_p) * RS
+                  : rec_t + ((tu + (i - pn) + seg_t) * lt.gs + col_t) * RS;
   };
 
   // One pass over the records, four loads in flight at a time; the running
@@ -162,18 +165,10 @@ shared_prefix_merge_kernel(T* __restrict__ out, const int32_t* __restrict__ hdr_
   }
 }
 
-// subsets of the prefix pass for a group of `group_size` texts (as the
-// grouped-query kernel's cascade layout: the smallest count of at most 16
-// texts each that divides the group)
-int nsub_of(int group_size) {
-  int nsub = (group_size + 15) / 16;
-  while (group_size % nsub) ++nsub;
-  return nsub;
-}
-
 template <typename T, int D>
 cudaError_t launch_shared_merge(const SharedPrefixArgs& a, const char* ws_p, int S_p,
-                                const char* ws_t, int S_t, cudaStream_t stream) {
+                                const char* ws_t, int S_t, DecodeLayout lt,
+                                cudaStream_t stream) {
   const int64_t items = static_cast<int64_t>(a.num_groups) * a.group_size * a.num_heads;
   const int per_cta = 8;  // warps, one per (text, head)
   cudaLaunchConfig_t cfg = {};
@@ -193,13 +188,16 @@ cudaError_t launch_shared_merge(const SharedPrefixArgs& a, const char* ws_p, int
       reinterpret_cast<const float*>(ws_t + header_bytes(S_t) + kGrabBytes),
       reinterpret_cast<unsigned long long*>(const_cast<char*>(ws_p) + header_bytes(S_p)),
       reinterpret_cast<unsigned long long*>(const_cast<char*>(ws_t) + header_bytes(S_t)),
-      a.num_groups, a.group_size, a.num_heads, nsub_of(a.group_size));
+      a.num_groups, a.group_size, a.num_heads, a.num_heads / a.num_kv_heads,
+      mma_cascade_layout(a.num_heads, a.num_kv_heads, a.group_size), lt);
 }
 
 // The two passes' workspaces, one after the other (256-byte aligned).
-size_t prefix_part_bytes(int num_groups, int group_size, int num_heads, int head_dim,
-                         int block_size, int max_prefix_blocks, int64_t forced_warps) {
-  return align_up(mma_cascade_workspace_bytes(num_groups, group_size, num_heads, head_dim,
+size_t prefix_part_bytes(int num_groups, int group_size, int num_heads, int num_kv_heads,
+                         int head_dim, int block_size, int max_prefix_blocks,
+                         int64_t forced_warps) {
+  return align_up(mma_cascade_workspace_bytes(num_groups, group_size, num_heads, num_kv_heads,
+                                              head_dim,
                                               block_size, max_prefix_blocks, forced_warps),
                   256);
 }
@@ -212,7 +210,7 @@ DecodeArgs pass_args(const SharedPrefixArgs& a) {
   d.v_cache = a.v_cache;
   d.scale = a.scale;
   d.num_heads = a.num_heads;
-  d.num_kv_heads = a.num_heads;
+  d.num_kv_heads = a.num_kv_heads;
   d.head_dim = a.head_dim;
   d.block_size = a.block_size;
   d.num_blocks = a.num_blocks;
@@ -226,25 +224,27 @@ DecodeArgs pass_args(const SharedPrefixArgs& a) {
 
 }  // namespace
 
-size_t shared_prefix_workspace_bytes(int num_groups, int group_size, int num_heads, int head_dim,
-                                     int block_size, int max_prefix_blocks, int max_tail_blocks,
+size_t shared_prefix_workspace_bytes(int num_groups, int group_size, int num_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int max_prefix_blocks, int max_tail_blocks,
                                      int64_t forced_warps) {
   if (num_groups < 1 || group_size < 1 ||
       static_cast<int64_t>(num_groups) * group_size > kMaxSeqs)
     return 0;
-  const size_t p = prefix_part_bytes(num_groups, group_size, num_heads, head_dim, block_size,
-                                     max_prefix_blocks, forced_warps);
-  const size_t t = decode_workspace_bytes(num_groups * group_size, num_heads, num_heads, head_dim,
-                                          block_size, max_tail_blocks, forced_warps);
+  const size_t p = prefix_part_bytes(num_groups, group_size, num_heads, num_kv_heads, head_dim,
+                                     block_size, max_prefix_blocks, forced_warps);
+  const size_t t = decode_workspace_bytes(num_groups * group_size, num_heads, num_kv_heads,
+                                          head_dim, block_size, max_tail_blocks, forced_warps);
   if (p == 0 || t == 0) return 0;
   return p + t;
 }
 
 cudaError_t launch_paged_attn_decode_shared(const SharedPrefixArgs& a, cudaStream_t stream) {
   const int S = a.num_groups * a.group_size;
-  const size_t p_bytes = prefix_part_bytes(a.num_groups, a.group_size, a.num_heads, a.head_dim,
-                                           a.block_size, a.max_prefix_blocks, a.forced_warps);
-  const size_t t_bytes = decode_workspace_bytes(S, a.num_heads, a.num_heads, a.head_dim,
+  const size_t p_bytes = prefix_part_bytes(a.num_groups, a.group_size, a.num_heads,
+                                           a.num_kv_heads, a.head_dim, a.block_size,
+                                           a.max_prefix_blocks, a.forced_warps);
+  const size_t t_bytes = decode_workspace_bytes(S, a.num_heads, a.num_kv_heads, a.head_dim,
                                                 a.block_size, a.max_tail_blocks, a.forced_warps);
   if (p_bytes == 0 || t_bytes == 0 || a.workspace_bytes < p_bytes + t_bytes)
     return cudaErrorInvalidValue;
@@ -272,12 +272,15 @@ cudaError_t launch_paged_attn_decode_shared(const SharedPrefixArgs& a, cudaStrea
   err = launch_paged_attn_decode(tp, stream);
   if (err != cudaSuccess) return err;
 
+  const DecodeLayout lt = decode_layout(tp);  // the tail pass's split of query heads
   if (a.head_dim == 128)
-    err = a.is_bf16 ? launch_shared_merge<__nv_bfloat16, 128>(a, ws_p, a.num_groups, ws_t, S, stream)
-                    : launch_shared_merge<__half, 128>(a, ws_p, a.num_groups, ws_t, S, stream);
+    err = a.is_bf16
+              ? launch_shared_merge<__nv_bfloat16, 128>(a, ws_p, a.num_groups, ws_t, S, lt, stream)
+              : launch_shared_merge<__half, 128>(a, ws_p, a.num_groups, ws_t, S, lt, stream);
   else
-    err = a.is_bf16 ? launch_shared_merge<__nv_bfloat16, 64>(a, ws_p, a.num_groups, ws_t, S, stream)
-                    : launch_shared_merge<__half, 64>(a, ws_p, a.num_groups, ws_t, S, stream);
+    err = a.is_bf16
+              ? launch_shared_merge<__nv_bfloat16, 64>(a, ws_p, a.num_groups, ws_t, S, lt, stream)
+              : launch_shared_merge<__half, 64>(a, ws_p, a.num_groups, ws_t, S, lt, stream);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

@@ -277,7 +277,8 @@ def shared_prefix(allocator, num_blocks: int, seed: int = 4, device="cpu",
                   dtype=torch.float16, num_prompts: int = 32, samples: int = 8,
                   num_heads: int = 40, head_dim: int = 128, block_size: int = 16,
                   max_blocks_per_seq: int = (1024 + 256 + 15) // 16,
-                  prompt_range=(256, 1024), gen_range=(1, 256)) -> DecodeInputs:
+                  prompt_range=(256, 1024), gen_range=(1, 256),
+                  num_kv_heads: Optional[int] = None) -> DecodeInputs:
     """Shared-prefix parallel sampling, built by driving a block manager.
 
     Per prompt: add the prompt, fork it into ``samples`` texts, then append the
@@ -287,8 +288,10 @@ def shared_prefix(allocator, num_blocks: int, seed: int = 4, device="cpu",
 
     Block copies that the manager asks for are applied to the pool here, as a
     setup step: rows that already hold tokens are copied from source to
-    destination.  ``meta['cow']`` lists them in order."""
+    destination.  ``meta['cow']`` lists them in order.  ``num_kv_heads``
+    below ``num_heads`` gives grouped-query pools."""
     dev = torch.device(device)
+    Hkv = num_heads if num_kv_heads is None else num_kv_heads
     prompts, gens = shared_prefix_plan(seed, num_prompts, samples, *prompt_range, *gen_range)
     seq_ids: List[int] = []
     cows: List[Tuple[int, int, int]] = []      # (src, dst, rows filled when copied)
@@ -319,7 +322,7 @@ def shared_prefix(allocator, num_blocks: int, seed: int = 4, device="cpu",
     lens = torch.as_tensor(np.asarray(lens), dtype=torch.int32)
     S = len(seq_ids)
     g = _gen(seed + 1000003, dev)
-    shape_pool = (num_blocks, num_heads, block_size, head_dim)
+    shape_pool = (num_blocks, Hkv, block_size, head_dim)
     k_cache = _randn(shape_pool, dtype, g, dev)
     v_cache = _randn(shape_pool, dtype, g, dev)
     for src, dst, rows in cows:
@@ -327,8 +330,8 @@ def shared_prefix(allocator, num_blocks: int, seed: int = 4, device="cpu",
             k_cache[dst, :, :rows] = k_cache[src, :, :rows]
             v_cache[dst, :, :rows] = v_cache[src, :, :rows]
     q = _randn((S, num_heads, head_dim), dtype, g, dev)
-    k = _randn((S, num_heads, head_dim), dtype, g, dev)
-    v = _randn((S, num_heads, head_dim), dtype, g, dev)
+    k = _randn((S, Hkv, head_dim), dtype, g, dev)
+    v = _randn((S, Hkv, head_dim), dtype, g, dev)
     tables_d, lens_d = tables.to(dev), lens.to(dev)
     fill = history_fill_of([tables_d], [lens_d], num_blocks, block_size, dev)
     _poison_unwritten(k_cache, v_cache, fill, block_size)

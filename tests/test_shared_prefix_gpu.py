@@ -21,7 +21,8 @@ def lib():
     return P.lib()
 
 
-def build_case(dtype, D, B, prompts, samples, prompt_range, gen_range, H, seed, num_blocks=None):
+def build_case(dtype, D, B, prompts, samples, prompt_range, gen_range, H, seed, num_blocks=None,
+               Hkv=None):
     import paged_kv_cache_326_b200 as P
     mb = -(-(prompt_range[1] + gen_range[1]) // B) + 1
     if num_blocks is None:
@@ -41,7 +42,7 @@ def build_case(dtype, D, B, prompts, samples, prompt_range, gen_range, H, seed, 
     return W.shared_prefix(Adapter(), num_blocks=num_blocks, seed=seed, device="cuda",
                            dtype=dtype, num_prompts=prompts, samples=samples, num_heads=H,
                            head_dim=D, block_size=B, max_blocks_per_seq=mb,
-                           prompt_range=prompt_range, gen_range=gen_range)
+                           prompt_range=prompt_range, gen_range=gen_range, num_kv_heads=Hkv)
 
 
 def gpu_shared_step(w, status, out=None):
@@ -92,6 +93,36 @@ def test_shared_prefix_matches_oracle(idx):
     c = compare(out, ref, dtype)
     assert c.ok, str(c)
     assert list(split[1].tolist()) == list(pl) and list(split[3].tolist()) == list(tl)
+
+
+GQA_CASES = [
+    # dtype, D, B, prompts, samples, prompt range, generated range, query heads, kv heads
+    (torch.float16, 128, 16, 3, 8, (5, 90), (1, 40), 8, 1),     # 64 columns: 4 subsets of 16
+    (torch.bfloat16, 128, 8, 2, 4, (1, 70), (1, 30), 16, 2),    # 32 columns a kv head
+    (torch.float16, 64, 32, 2, 3, (20, 130), (1, 50), 6, 2),    # 9 columns
+    (torch.float16, 128, 16, 2, 2, (30, 120), (1, 40), 64, 8),  # Llama-2-70B heads, 16 columns
+]
+
+
+@pytest.mark.parametrize("idx", range(len(GQA_CASES)),
+                         ids=[f"{str(c[0])[6:]}-D{c[1]}-B{c[2]}-g{c[4]}-h{c[7]}kv{c[8]}"
+                              for c in GQA_CASES])
+def test_shared_prefix_grouped_query_matches_oracle(idx):
+    """Grouped-query pools (pa_paged_attn_decode_shared_gqa): every output
+    against the oracle's shared-prefix attention on the same pool."""
+    dtype, D, B, prompts, samples, pr, gr, H, Hkv = GQA_CASES[idx]
+    w = build_case(dtype, D, B, prompts, samples, pr, gr, H, seed=200 + idx, Hkv=Hkv)
+    oi = oracle_inputs(w.q, w.k, w.v, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                       w.slot_mapping, B)
+    st = new_status()
+    out, split = gpu_shared_step(w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, st.item()
+    kc, vc = oracle.cache_write(oi.k_cache, oi.v_cache, oi.k, oi.v, oi.slots, B)
+    pt, pl, tt, tl = oracle.split_shared_prefix(oi.tables, oi.lens, B, samples)
+    ref = oracle.paged_decode_shared(oi.q, kc, vc, pt, pl, tt, tl, samples, w.scale, B)
+    c = compare(out, ref, dtype)
+    assert c.ok, str(c)
 
 
 def test_shared_prefix_is_deterministic_and_close_to_plain_decode():
