@@ -21,7 +21,11 @@
 // PA_COPY_STREAMING_STORE=1 writes with st.global.cs (evict-first); it
 // measured no different, nor did 8 vectors in flight (21.2 us), 512 threads
 // (21.9) or 128 threads of 8 vectors (21.3); 64 KB pieces were slower
-// (23.3-25.0).
+// (23.3-25.0).  Moving the pieces through the bulk-copy unit instead (one
+// warp per piece: bulk loads into shared memory, each chunk written out by
+// a bulk store as soon as it lands; pieces of 16, 32 or 64 KB in 1 to 8
+// chunks) measured the same 21.1-21.3 microseconds: the bursts are bound by
+// the memory system's writes, not by how the copies are issued.
 #include <cuda_runtime.h>
 
 #include <cstdint>

@@ -45,16 +45,26 @@
 //     and stores it.
 //   * warps 18 and 19 store the new tokens' keys and values in the cache
 //     (when asked to): the CTAs of a key/value head's first query head copy
-//     the prompt's rows of k and v to their slots with plain 16-byte loads
-//     and stores, each a share of the tokens in proportion to its attention
-//     work, while the other warps compute; the attention is bound by the
-//     tensor and exponential units and leaves HBM mostly idle.
-//     (Storing from the K/V tiles in shared memory measured slower: the
-//     stores held the ring's slots.)
+//     the prompt's rows of k and v to their slots, a bulk copy into a
+//     staging row of shared memory and a bulk copy out of it per row, each
+//     CTA a share of the tokens in proportion to its attention work, while
+//     the other warps compute; the attention is bound by the tensor and
+//     exponential units and leaves HBM mostly idle.  (Storing from the K/V
+//     tiles in shared memory measured slower: the stores held the ring's
+//     slots; so did plain 16-byte loads and stores from registers.)
 // Why two threads a row: the exponential unit does 4 exp2 a clock per SM
 // sub-partition, so a block's 2 x 128 x 128 weights take as long as its
 // products; with one thread a row each tile's softmax ran twice as long as
-// the other tile's products, and the tensor pipe waited.
+// the other tile's products, and the tensor pipe waited.  Making the two
+// tiles take turns on the exponential unit (tile 1's weights of a block
+// after tile 0's, tile 0's of the next after tile 1's, through a pair of
+// barriers) measured slower: 670 against 712 TFLOP/s for the attention
+// alone.
+// Order of the CTAs: the hardware hands them out x fastest, then y, then
+// z; the grid is (head, pair, prompt), so each prompt's pairs of all heads
+// go heaviest first (0.7% faster than each (prompt, head)'s pairs in turn;
+// the heaviest pairs of the whole launch first lost 2.5%: a head's keys and
+// values no longer stay in L2 between its pairs).
 // Barriers: per ring slot, for K and for V, full (TMA bytes) and empty (the
 // last product that reads it); per tile S ready, P ready (256 arrivals) and
 // O done.  TMEM per tile: S (and P over it) 128 columns, O head_dim; 512 for
@@ -85,7 +95,7 @@ constexpr int kTcHalf = kTcBN / 2;  // keys per softmax thread and block
 constexpr int kTcTiles = 2;     // query tiles per CTA
 constexpr int kTcStages = 2;    // slots of each of the K and V rings (32 KB each)
 // Warpgroups 0-3: the softmax; warpgroup 4: the MMA warp, the load warp and
-// two idle warps.  The launch gives every thread 96 registers (640 x 96 of
+// the two store warps.  The launch gives every thread 96 registers (640 x 96 of
 // the SM's 65,536).  A build option splits them unevenly (warpgroup 4 lowers
 // to kTcRegsLow, the softmax warpgroups raise to kTcRegsHigh, with
 // 4 x 128 x high + 128 x low <= 640 x 96); with the softmax reading its
@@ -149,10 +159,9 @@ struct TcLayout {
   static constexpr int Q_BYTES = kTcBM * D * 2;   // one tile of Q: 32 KB at head_dim 128
   static constexpr int KV_BYTES = kTcBN * D * 2;  // one block of K (or V): 32 KB at D = 128
   static constexpr int STAGE = 2 * KV_BYTES;      // K slot i, then V slot i
-  // staging of the store warps: one row of k or v per thread
-  static constexpr int STORE_BYTES = 64 * D * 2;
   // shared memory asked for (+ 1 KB to align by hand): the head_dim-128
-  // amount at every head_dim, so one CTA holds an SM (its 512 TMEM columns)
+  // amount at every head_dim, so one CTA holds an SM (its 512 TMEM
+  // columns), and the store warps' staging (one 256-byte row per thread)
   static constexpr int SMEM = 1024 + kTcTiles * (kTcBM * 128 * 2) +
                               kTcStages * (2 * kTcBN * 128 * 2) + 64 * 128 * 2;
 };
@@ -210,23 +219,24 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   __shared__ volatile int abort_flag;
 
   griddep_wait();
-  const int s = blockIdx.z, h = blockIdx.y;
+  // (head h, pair index xp counted from the last pair, prompt s)
+  const int h = blockIdx.x, xp = blockIdx.y, s = blockIdx.z;
   const int a = __ldg(p.cu_seqlens + s), b = __ldg(p.cu_seqlens + s + 1);
   if (a < 0 || b < a || b > p.num_tokens) {
-    if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
+    if (xp == 0 && h == 0 && threadIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
     return;
   }
   const int L = b - a;  // new tokens of this prompt
-  if (L > p.max_seqlen && blockIdx.x == 0 && h == 0 && threadIdx.x == 0)
+  if (L > p.max_seqlen && xp == 0 && h == 0 && threadIdx.x == 0)
     set_status(p.status, -8 /* PA_ERR_BAD_LEN: a prompt longer than max_seqlen */);
   // stored prefix: a whole number of blocks that the table holds
   const int cl = p.cached_lens ? __ldg(p.cached_lens + s) : 0;
   if (cl < 0 || cl % p.B || cl > p.max_blocks * p.B) {
-    if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
+    if (xp == 0 && h == 0 && threadIdx.x == 0) set_status(p.status, -8 /* PA_ERR_BAD_LEN */);
     return;
   }
   const int npre = (cl + kTcBN - 1) / kTcBN;        // key blocks of the stored prefix
-  const int pair = gridDim.x - 1 - blockIdx.x;       // heaviest pairs of tiles first
+  const int pair = gridDim.y - 1 - xp;               // heaviest pairs of tiles first
   const int q0 = pair * kTcTiles * kTcBM;            // first new row of tile 0
   if (q0 >= L) return;                               // the whole CTA leaves: nothing allocated
   const int kvh = h / (p.Hq / p.Hkv);
@@ -474,15 +484,13 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     // ---------------- the new tokens' keys and values to the cache ----------------
     // The CTAs of a key/value head's first query head store the prompt's
     // tokens (each token of the prompt and head once): K and V rows from k,
-    // v to their slots, 16-byte vectors, kStoreVecs in flight per lane, by
-    // warps 18 and 19 while the others compute (the pool holds the bits of
-    // pa_kv_cache_write afterwards).  Pair p of tiles has about 4p + 3
-    // blocks of attention, so it takes that share of the prompt's tokens:
-    // [L c_p / c_P, L c_{p+1} / c_P) with c_p = 2p^2 + p (the sum of 4i + 3
-    // over i < p) and P pairs.  A slot outside the pool is recorded as
-    // PA_ERR_BAD_SLOT and that token skipped; a negative one skips it.
-    constexpr int kStoreVecs = 8;
-    constexpr int VPR = D / 8;                   // 16-byte vectors per row
+    // v to their slots, by warps 18 and 19 while the others compute (the
+    // pool holds the bits of pa_kv_cache_write afterwards).  Pair p of
+    // tiles has about 4p + 3 blocks of attention, so it takes that share of
+    // the prompt's tokens: [L c_p / c_P, L c_{p+1} / c_P) with
+    // c_p = 2p^2 + p (the sum of 4i + 3 over i < p) and P pairs.  A slot
+    // outside the pool is recorded as PA_ERR_BAD_SLOT and that token
+    // skipped; a negative one skips it.
     const int64_t npairs = (L + kTcTiles * kTcBM - 1) / (kTcTiles * kTcBM);
     const int64_t cP = 2 * npairs * npairs + npairs;
     auto cum = [](int64_t q) { return 2 * q * q + q; };
@@ -497,6 +505,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     uint8_t* stage_row = sKV + kTcStages * LY::STAGE + lid * ROW;
     const int rows = 2 * n_tok;
     uint32_t phase = 0;
+    // (The reads' L2 priority, evict-first, normal or evict-last, and an
+    // evict-first hint on the writes measured within 0.4% of each other; a
+    // barrier per thread instead of one for the 64, or 96 staging rows,
+    // measured slower.)
     for (int r0 = 0; r0 < rows; r0 += 64, phase ^= 1) {
       const int rr = r0 + lid;
       void* dst = nullptr;
@@ -821,7 +833,8 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
   p.B_shift = 0;
   while ((1 << p.B_shift) < p.B) ++p.B_shift;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(tiles, a.num_heads, a.num_seqs);
+  if (tiles > 65535) return cudaErrorInvalidValue;  // prompts of up to 16.7 M tokens
+  cfg.gridDim = dim3(a.num_heads, tiles, a.num_seqs);
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = LY::SMEM;
   cfg.stream = stream;

@@ -199,7 +199,6 @@ __device__ __forceinline__ void tma_store_4d(const void* map, const void* src, i
       : "memory");
 }
 
-// Close the current bulk async-group of this thread.
 // Untiled bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
 // aligned) from this CTA's shared memory to global memory; completes in
 // this thread's bulk group.
@@ -208,6 +207,7 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_
                "r"(smem_addr(ssrc)), "r"(bytes)
                : "memory");
 }
+// Close the current bulk async-group of this thread.
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
