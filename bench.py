@@ -1139,9 +1139,14 @@ def main():
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the tiny, skewed, shared-prefix and 40-layer configurations that "
                          "the default run reports under other_configs")
-    ap.add_argument("--path", choices=["fused", "calls"], default="fused")
+    ap.add_argument("--path", choices=["fused", "calls"], default=None,
+                    help="fused: one launch stores the new tokens and attends "
+                         "(pa_decode_step, pa_decode_step_fp8; multi-head pools); calls: the "
+                         "write, then the decode (default for the 8-bit and grouped-query "
+                         "workloads)")
     ap.add_argument("--kv-dtype", choices=["f16", "fp8"], default="f16",
-                    help="fp8: the batch-64 step over 8-bit E4M3 caches (two calls)")
+                    help="fp8: the step over 8-bit E4M3 caches (batch-64 OPT-13B, or with "
+                         "--workload llama2_70b_gqa the grouped-query step)")
     ap.add_argument("--shared-path", choices=["cascade", "plain"], default="cascade",
                     help="shared_prefix workload: pa_paged_attn_decode_shared over the split "
                          "tables (cascade) or pa_paged_attn_decode over the joined ones (plain)")
@@ -1191,13 +1196,13 @@ def main():
     P.pa_set_option(P.PA_OPT_GQA_KERNEL, {"auto": 0, "cores": 1, "tensor": 2}[args.gqa_kernel])
     gqa_kernel = "CUDA-core" if args.gqa_kernel == "cores" else "tensor-core"
     fp8 = args.kv_dtype == "fp8"
-    if gqa and fp8:
-        raise SystemExit("the 8-bit cache is multi-head only")
+    if args.path is None:
+        args.path = "calls" if (gqa or fp8) else "fused"
     if gqa:
         args.path = "calls"   # the one-launch step is multi-head only
-        w = W.llama2_70b_gqa(seed=dist.batch_seed(6, ranks), device=dev)
+        w = (W.llama2_70b_gqa_fp8 if fp8 else W.llama2_70b_gqa)(
+            seed=dist.batch_seed(6, ranks), device=dev)
     elif fp8:
-        args.path = "calls"   # the one-launch step stores 16-bit values
         w = W.opt13b_batch64_fp8(seed=dist.batch_seed(2, ranks), device=dev)
     elif args.workload == "skewed":
         w = W.skewed(seed=dist.batch_seed(3, ranks), device=dev)
@@ -1240,6 +1245,8 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def write_part(k, v, slots):
+        if fused:
+            return
         if fp8:
             P.pa_kv_cache_write_fp8(k, v, w.k_cache, w.v_cache, slots, w.meta["k_scale"],
                                     w.meta["v_scale"], status=status)
@@ -1252,9 +1259,17 @@ def main():
             pt, pl_d, tt, tl_d = shared_tables if shared_tables is not None else split_d
             P.pa_paged_attn_decode_shared(out, q, w.k_cache, w.v_cache, pt, pl_d, tt, tl_d,
                                           w.scale, gs, workspace=ws_shared, status=status)
+        elif fused and fp8:
+            P.pa_decode_step_fp8(out, q, k, v, w.k_cache, w.v_cache, slots, tables, lens,
+                                 w.scale, w.meta["k_scale"], w.meta["v_scale"], workspace=ws,
+                                 status=status)
         elif fused:
             P.pa_decode_step(out, q, k, v, w.k_cache, w.v_cache, slots, tables, lens, w.scale,
                              workspace=ws, status=status)
+        elif gqa and fp8:
+            P.pa_paged_attn_decode_fp8(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
+                                       w.meta["k_scale"], w.meta["v_scale"], workspace=ws,
+                                       status=status)
         elif gqa:
             P.pa_paged_attn_decode_gqa(out, q, w.k_cache, w.v_cache, tables, lens, w.scale,
                                        workspace=ws, status=status)
@@ -1363,7 +1378,10 @@ def main():
                    "parallelism": f"independent batch per GPU x{world}",
                    "path": ("pa_kv_cache_write + pa_paged_attn_decode_shared (tables split "
                             "by pa_split_shared_prefix)" if cascade else
+                            "pa_decode_step_fp8" if fused and fp8 else
                             "pa_decode_step" if fused else
+                            "pa_kv_cache_write_fp8 + pa_paged_attn_decode_fp8 (grouped-query "
+                            "pools)" if gqa and fp8 else
                             f"pa_kv_cache_write + pa_paged_attn_decode_gqa ({gqa_kernel})" if gqa
                             else "pa_kv_cache_write_fp8 + pa_paged_attn_decode_fp8" if fp8
                             else "pa_kv_cache_write + pa_paged_attn_decode")},
@@ -1379,7 +1397,7 @@ def main():
                      "decode_frac_of": {"nominal": achieved / NOMINAL_HBM_GBS,
                                         "measured_copy": achieved / peak,
                                         "read_probe": achieved / probe_gbs}},
-        "kernel_ms": ({"pa_decode_step": decode_ms} if fused else
+        "kernel_ms": ({"pa_decode_step_fp8" if fp8 else "pa_decode_step": decode_ms} if fused else
                       {"kv_cache_write": write_ms, "paged_attn_decode": decode_ms}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
@@ -1387,8 +1405,12 @@ def main():
                                                    args.path),
                      "kernel": ("pa_paged_attn_decode_shared (prefix pass on the tensor cores, "
                                 "tail pass, merge kernel)" if cascade else
+                                "pa_decode_step_fp8 (8-bit decode kernel with the cache write, "
+                                "+ merge kernel)" if fused and fp8 else
                                 "pa_decode_step (decode kernel with the cache write, + merge kernel)"
                                 if fused else
+                                "pa_paged_attn_decode_fp8 (8-bit grouped-query decode kernel + "
+                                "merge kernel)" if gqa and fp8 else
                                 f"pa_paged_attn_decode_gqa ({gqa_kernel} decode kernel + merge kernel)" if gqa
                                 else "pa_paged_attn_decode_fp8 (8-bit decode kernel + merge kernel)" if fp8
                                 else "pa_paged_attn_decode (decode kernel + merge kernel)"),

@@ -413,10 +413,15 @@ int pa_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache, cons
  *                  codes (written by pa_kv_cache_write_fp8 with num_heads =
  *                  num_kv_heads)
  *   workspace      pa_paged_attn_decode_gqa_workspace_size(...) bytes
- * Runs on the CUDA cores: each unit of work carries up to 4 query heads of
- * one group (the largest of 4, 2, 1 that divides the group), so every code
- * read serves them all.  num_heads must be a multiple of num_kv_heads (else
- * PA_ERR_INVALID); other arguments and errors as for pa_paged_attn_decode_fp8.
+ * With fp16 queries, head_dim 128 and blocks of 8, 16 or 32 it runs on the
+ * tensor cores (PA_OPT_FP8_KERNEL picks the kernel): the query heads of a
+ * key/value head are the columns of the product tile, up to 8 per pass
+ * (larger groups in the fewest equal subsets of at most 8), so every code
+ * read serves them all.  Otherwise it runs on the CUDA cores, each unit of
+ * work carrying up to 4 query heads of one group (the largest of 4, 2, 1
+ * that divides the group).  num_heads must be a multiple of num_kv_heads
+ * (else PA_ERR_INVALID); other arguments and errors as for
+ * pa_paged_attn_decode_fp8.
  */
 int pa_paged_attn_decode_fp8_gqa(void* out, const void* q, const void* k_cache,
                                  const void* v_cache, const int32_t* block_tables,

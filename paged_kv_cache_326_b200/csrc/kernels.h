@@ -147,10 +147,10 @@ int64_t option_gqa_kernel();
 int64_t option_fp8_kernel();
 
 // Tensor-core decode over an 8-bit cache (paged_attn_decode_mma_fp8.cu):
-// fp16 queries, head_dim 128, multi-head, blocks of 8, 16 or 32, a pool that
-// fits 32-bit TMA row coordinates.
+// fp16 queries, head_dim 128, multi-head or grouped-query pools, blocks of
+// 8, 16 or 32, a pool that fits 32-bit TMA row coordinates.
 bool mma_fp8_decode_ok(const DecodeArgs& a);
-size_t mma_fp8_workspace_bytes(int num_seqs, int num_heads, int block_size,
+size_t mma_fp8_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int block_size,
                                int max_blocks_per_seq, int64_t forced_warps);
 cudaError_t launch_paged_attn_decode_mma_fp8(const DecodeArgs& a, cudaStream_t stream);
 
@@ -173,6 +173,7 @@ struct DecodeLayout {
   int vheads;
 };
 DecodeLayout mma_decode_layout(int num_heads, int num_kv_heads);
+DecodeLayout mma_fp8_layout(int num_heads, int num_kv_heads);
 DecodeLayout mma_cascade_layout(int num_heads, int num_kv_heads, int group_size);
 // The layout launch_paged_attn_decode uses for these arguments.
 DecodeLayout decode_layout(const DecodeArgs& a);

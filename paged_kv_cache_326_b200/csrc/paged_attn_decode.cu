@@ -739,9 +739,8 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
   size_t bytes =
       header_bytes(num_seqs) + kGrabBytes + records_bytes(max_units(warps) + segs, head_dim, hl.gs);
   // The 8-bit cache may run on the tensor-core kernel: size for it too.
-  if (with_fp8 && hl.gs == 1 && head_dim == 128 &&
-      (block_size == 8 || block_size == 16 || block_size == 32)) {
-    const size_t f8 = mma_fp8_workspace_bytes(num_seqs, num_heads, block_size,
+  if (with_fp8 && head_dim == 128 && (block_size == 8 || block_size == 16 || block_size == 32)) {
+    const size_t f8 = mma_fp8_workspace_bytes(num_seqs, num_heads, num_kv_heads, block_size,
                                               max_blocks_per_seq, forced_warps);
     if (f8 == 0) return 0;
     if (f8 > bytes) bytes = f8;
@@ -758,6 +757,8 @@ size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int
 
 DecodeLayout decode_layout(const DecodeArgs& a) {
   // the same choice of kernel as launch_paged_attn_decode below
+  if (a.fp8 && mma_fp8_decode_ok(a) && option_fp8_kernel() != 1)
+    return mma_fp8_layout(a.num_heads, a.num_kv_heads);
   const int64_t mode = option_gqa_kernel();
   const bool mma_ok = !a.slot_mapping && !a.fp8 &&
                       mma_decode_shape_ok(a.num_heads, a.num_kv_heads, a.head_dim, a.block_size) &&

@@ -13,9 +13,16 @@
 // per number) that work, not HBM, set the pace.  Here every product runs as
 // mma.sync m16n8k16 (fp16 in, fp32 accumulate) on codes widened exactly to
 // fp16 by cvt.rn.f16x2.e4m3x2; only the conversions stay on the CUDA cores.
-// The single query is copied into all eight columns of the tile, so every
-// lane's accumulators hold finished scores and outputs: no cross-lane
-// reduction of dot products and no transpose of the scores.
+// Multi-head: the single query is copied into all eight columns of the
+// tile, so every lane's accumulators hold finished scores and outputs: no
+// cross-lane reduction of dot products and no transpose of the scores.
+// Grouped-query pools ("What Came After": heads that share a key/value set):
+// the columns are the query heads of one key/value head (up to 8 per pass;
+// a group of G in the fewest equal subsets of at most 8, a subset of gs < 8
+// repeating its heads over the spare columns), so one read of the codes
+// serves the whole subset; each lane then holds two columns' scores, keeps
+// a running max and sum per column, and fetches its column's weights for
+// the value products from the lane that computed them.
 //
 // A chunk is 32 tokens (4 KB of key codes, 4 KB of value codes), fetched by
 // 2-D tiled TMA with the 128-byte swizzle (16-byte piece k of row r stored at
@@ -70,17 +77,27 @@ namespace {
 #ifndef PA_F8MMA_STAGES
 #define PA_F8MMA_STAGES 2
 #endif
+#ifndef PA_F8MMA_WARPS_GQA
+#define PA_F8MMA_WARPS_GQA 4
+#endif
 constexpr int kF8Warps = PA_F8MMA_WARPS;    // warps per CTA
+// The grouped-query kernel's warps per CTA (its stages hold 8 query rows, so
+// its warps take 21 KB of shared memory against 17)
+constexpr int kF8WarpsGqa = PA_F8MMA_WARPS_GQA;
+__host__ __device__ constexpr int f8_warps(bool gqa) { return gqa ? kF8WarpsGqa : kF8Warps; }
 constexpr int kF8Stages = PA_F8MMA_STAGES;  // ring depth per warp
 constexpr int kF8D = 128;                   // head_dim
 constexpr int kF8CH = 32;                   // tokens per chunk: 4 KB of key codes
 
 // One warp's area: the stages' K and V tiles (4 KB each, every tile on a
-// 1024-byte boundary), then the stages' query rows (256 B each), barriers
-// and flags; rounded up to 1024 bytes.
-__host__ __device__ constexpr int f8_warp_bytes(int stages) {
-  return (stages * 8192 + stages * 256 + stages * 12 + 1023) / 1024 * 1024;
+// 1024-byte boundary), then the stages' query rows (qrows of 256 B each),
+// barriers and flags; rounded up to 1024 bytes.
+__host__ __device__ constexpr int f8_warp_bytes(int stages, int qrows) {
+  return (stages * 8192 + stages * 256 * qrows + stages * 12 + 1023) / 1024 * 1024;
 }
+// Query rows a stage holds: one (multi-head), or up to the tile's eight
+// columns (grouped-query).
+__host__ __device__ constexpr int f8_qrows(bool gqa) { return gqa ? 8 : 1; }
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
@@ -88,7 +105,7 @@ __device__ __forceinline__ uint4 lds128(const uint8_t* p) {
 
 }  // namespace
 
-template <int B, int WARPS, int STAGES>
+template <int B, int WARPS, int STAGES, bool GQA>
 __global__ void __launch_bounds__(WARPS * 32, 3)
 paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v) {
@@ -97,7 +114,8 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
   constexpr int NB = CH >= B ? CH / B : 1;  // physical blocks a chunk touches
   constexpr int R = CH >= B ? B : CH;       // rows per TMA box
   constexpr uint32_t BOX_BYTES = R * 128;
-  constexpr int AREA = f8_warp_bytes(STAGES);
+  constexpr int QR = f8_qrows(GQA);
+  constexpr int AREA = f8_warp_bytes(STAGES, QR);
   static_assert(B >= 8 && CH % B == 0, "block sizes 8, 16, 32");
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -106,7 +124,16 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + WARPS * AREA);
   __shared__ int32_t warp_tot[WARPS];
 
-  const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;  // equal: multi-head
+  const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
+  // Grouped-query: virtual head vh is subset vh % nsub of key/value head
+  // vh / nsub, query heads q_head0(vh) .. + GS - 1 (GS <= 8), one per
+  // column of the tile; multi-head: the head itself in every column.
+  const int NSUB = p.nsub, GS = GQA ? p.gs : 1;
+  const int G = Hq / Hkv;
+  auto kv_head = [&](int vh) { return !GQA ? vh : NSUB == 1 ? vh : vh / NSUB; };
+  auto q_head0 = [&](int vh) {
+    return !GQA ? vh : NSUB == 1 ? vh * G : (vh / NSUB) * G + (vh % NSUB) * GS;
+  };
   const int cap = p.max_blocks_per_seq * B;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -126,7 +153,7 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
 
   uint8_t* tiles = smem + warp * AREA;
   uint8_t* qbuf = tiles + STAGES * 8192;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + STAGES * 256);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + STAGES * 256 * QR);
   int32_t* flags = reinterpret_cast<int32_t*>(bars + STAGES);
   if (lane == 0) {
 #pragma unroll
@@ -190,18 +217,18 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
       if (bad) set_status(p.status, -7 /* PA_ERR_BAD_BLOCK */);
       flags[st] = bad ? 1 : 0;
       fence_proxy_async_smem();
-      const uint32_t qbytes = first ? D * 2 : 0;
+      const uint32_t qbytes = first ? GS * D * 2 : 0;
       const uint32_t kvbytes = bad ? 0 : 2u * boxes * BOX_BYTES;
       mbar_arrive_expect_tx(&bars[st], qbytes + kvbytes);
-      if (first)
-        bulk_copy_g2s(qbuf + st * 256, qg + (static_cast<int64_t>(s) * Hq + h) * D, D * 2,
-                      &bars[st], policy);
+      if (first)  // the unit's query rows (contiguous: GS heads in a row)
+        bulk_copy_g2s(qbuf + st * 256 * QR, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D,
+                      GS * D * 2, &bars[st], policy);
       if (!bad) {
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           const int rows = (CH >= B) ? min(B, nvalid - b * B) : nvalid;
           if (rows > 0) {
-            const int y = (blk[b] * Hkv + h) * B;
+            const int y = (blk[b] * Hkv + kv_head(h)) * B;
             tma_load_2d(sK + b * BOX_BYTES, &tm_k, 0, y, &bars[st], policy);
             tma_load_2d(sV + b * BOX_BYTES, &tm_v, 0, y, &bars[st], policy);
           }
@@ -214,9 +241,13 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
   for (int k = 0; k < STAGES; ++k) issue(k);
 
   const int g = lane >> 2, c = lane & 3;
-  uint32_t qh[16];   // query dimensions [32c, 32c + 32) as fp16 pairs
-  float o[8][4];     // O^T: dimension 16g + 2md (+1 for entries 2, 3), all columns alike
-  float m = -INFINITY, l = 0.f;  // running max (warp-uniform); this lane's share of the sum
+  uint32_t qh[16];   // query dimensions [32c, 32c + 32) of column g, as fp16 pairs
+  // O^T: dimension 16g + 2md (+1 for entries 2, 3), column 2c (entries 0, 2)
+  // and 2c + 1 (entries 1, 3); multi-head: all columns alike
+  float o[8][4];
+  float m = -INFINITY, l = 0.f;  // multi-head: running max (warp-uniform); this lane's share of the sum
+  // grouped-query: the same for columns 2c and 2c + 1 (the max uniform over g)
+  float mg[2] = {-INFINITY, -INFINITY}, lg[2] = {0.f, 0.f};
   int piece_j0 = 0;
   int prev_unit = -1;
   const float scale = p.qk_scale_log2;
@@ -242,7 +273,7 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
 
     if (j == 0 || wu0 != prev_unit) {
       piece_j0 = j;
-      const uint8_t* qrow = qbuf + st * 256 + c * 64;
+      const uint8_t* qrow = qbuf + st * 256 * QR + (GQA ? (g % GS) * 256 : 0) + c * 64;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint4 x = lds128(qrow + 16 * i);
@@ -253,6 +284,8 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
       }
       m = -INFINITY;
       l = 0.f;
+      mg[0] = mg[1] = -INFINITY;
+      lg[0] = lg[1] = 0.f;
 #pragma unroll
       for (int md = 0; md < 8; ++md)
 #pragma unroll
@@ -289,6 +322,63 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
     }
 
     // ---- online softmax (base 2): tokens g, g + 8, 16 + g, 24 + g ----
+    constexpr float kSlack = 8.f;
+    // P pairs (token g, token g + 8) of each 16-token tile in fp16 (and the
+    // rest, when split); grouped-query: [column 2c + j][tile]
+    uint32_t ph[2][2], pl[2][2] = {{0u, 0u}, {0u, 0u}};
+    if constexpr (GQA) {
+      float sc[2][4];
+#pragma unroll
+      for (int jc = 0; jc < 2; ++jc) {
+        sc[jc][0] = (sa[0][0][jc] + sa[1][0][jc]) * scale;
+        sc[jc][1] = (sa[0][0][2 + jc] + sa[1][0][2 + jc]) * scale;
+        sc[jc][2] = (sa[0][1][jc] + sa[1][1][jc]) * scale;
+        sc[jc][3] = (sa[0][1][2 + jc] + sa[1][1][2 + jc]) * scale;
+      }
+      if (nvalid < CH) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if ((i >> 1) * 16 + (i & 1) * 8 + g >= nvalid) sc[0][i] = sc[1][i] = -INFINITY;
+      }
+      float cm[2];
+#pragma unroll
+      for (int jc = 0; jc < 2; ++jc)
+        cm[jc] = fmaxf(fmaxf(sc[jc][0], sc[jc][1]), fmaxf(sc[jc][2], sc[jc][3]));
+      if (__any_sync(0xffffffffu, cm[0] > mg[0] + kSlack || cm[1] > mg[1] + kSlack)) {
+        float alpha[2];
+#pragma unroll
+        for (int jc = 0; jc < 2; ++jc) {
+          float x = cm[jc];  // the column's max over the warp's tokens (lanes of one c)
+          x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+          x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+          x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+          const float m_new = fmaxf(mg[jc], x);
+          alpha[jc] = m_new == mg[jc] ? 1.f : fast_exp2(mg[jc] - m_new);
+          lg[jc] *= alpha[jc];
+          mg[jc] = m_new;
+        }
+#pragma unroll
+        for (int md = 0; md < 8; ++md)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[md][e] *= alpha[e & 1];
+      }
+#pragma unroll
+      for (int jc = 0; jc < 2; ++jc) {
+        const float mm = mg[jc] == -INFINITY ? 0.f : mg[jc];
+        float pr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pr[i] = fast_exp2(sc[jc][i] - mm);
+        lg[jc] += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) {
+          ph[jc][kt] = Elem<__half>::from_float2(pr[2 * kt], pr[2 * kt + 1]);
+          if constexpr (kSplitPF16) {
+            const float2 back = Elem<__half>::to_float2(ph[jc][kt]);
+            pl[jc][kt] = Elem<__half>::from_float2(pr[2 * kt] - back.x, pr[2 * kt + 1] - back.y);
+          }
+        }
+      }
+    } else {
     float sc[4];
     sc[0] = (sa[0][0][0] + sa[1][0][0]) * scale;
     sc[1] = (sa[0][0][2] + sa[1][0][2]) * scale;
@@ -299,7 +389,6 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
       for (int i = 0; i < 4; ++i)
         if ((i >> 1) * 16 + (i & 1) * 8 + g >= nvalid) sc[i] = -INFINITY;
     }
-    constexpr float kSlack = 8.f;
     const float cm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
     if (__any_sync(0xffffffffu, cm > m + kSlack)) {
       float x = cm;
@@ -321,27 +410,49 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
 #pragma unroll
     for (int i = 0; i < 4; ++i) pr[i] = fast_exp2(sc[i] - mm);
     l += (pr[0] + pr[1]) + (pr[2] + pr[3]);
-    // P pairs (token g, token g + 8) of each 16-token tile in fp16 (and the
-    // rest, when split)
-    uint32_t ph[2], pl[2] = {0u, 0u};
 #pragma unroll
     for (int kt = 0; kt < 2; ++kt) {
-      ph[kt] = Elem<__half>::from_float2(pr[2 * kt], pr[2 * kt + 1]);
+      ph[0][kt] = Elem<__half>::from_float2(pr[2 * kt], pr[2 * kt + 1]);
       if constexpr (kSplitPF16) {
-        const float2 back = Elem<__half>::to_float2(ph[kt]);
-        pl[kt] = Elem<__half>::from_float2(pr[2 * kt] - back.x, pr[2 * kt + 1] - back.y);
+        const float2 back = Elem<__half>::to_float2(ph[0][kt]);
+        pl[0][kt] = Elem<__half>::from_float2(pr[2 * kt] - back.x, pr[2 * kt + 1] - back.y);
       }
+    }
     }
 
     // ---- O^T += V^T P^T ----
 #pragma unroll
     for (int kt = 0; kt < 2; ++kt) {
       // K positions 2c, 2c+1 <- tokens 2c, 2c+8 (held together by lane g = 2c);
-      // K positions 2c+8, 2c+9 <- tokens 2c+1, 2c+9 (lane g = 2c + 1)
-      const uint32_t b0h = __shfl_sync(0xffffffffu, ph[kt], (2 * c) * 4);
-      const uint32_t b1h = __shfl_sync(0xffffffffu, ph[kt], (2 * c + 1) * 4);
-      const uint32_t b0l = kSplitPF16 ? __shfl_sync(0xffffffffu, pl[kt], (2 * c) * 4) : 0u;
-      const uint32_t b1l = kSplitPF16 ? __shfl_sync(0xffffffffu, pl[kt], (2 * c + 1) * 4) : 0u;
+      // K positions 2c+8, 2c+9 <- tokens 2c+1, 2c+9 (lane g = 2c + 1).
+      // Grouped-query: this lane's column g is column 2(g/2) + (g%2) of the
+      // lane (2c or 2c + 1, g/2); both of its columns come over, one is kept.
+      uint32_t b0h, b1h, b0l = 0u, b1l = 0u;
+      if constexpr (GQA) {
+        const int src0 = (2 * c) * 4 + (g >> 1), src1 = (2 * c + 1) * 4 + (g >> 1);
+        const bool odd = g & 1;
+        uint32_t x0 = __shfl_sync(0xffffffffu, ph[0][kt], src0);
+        uint32_t x1 = __shfl_sync(0xffffffffu, ph[1][kt], src0);
+        b0h = odd ? x1 : x0;
+        x0 = __shfl_sync(0xffffffffu, ph[0][kt], src1);
+        x1 = __shfl_sync(0xffffffffu, ph[1][kt], src1);
+        b1h = odd ? x1 : x0;
+        if constexpr (kSplitPF16) {
+          x0 = __shfl_sync(0xffffffffu, pl[0][kt], src0);
+          x1 = __shfl_sync(0xffffffffu, pl[1][kt], src0);
+          b0l = odd ? x1 : x0;
+          x0 = __shfl_sync(0xffffffffu, pl[0][kt], src1);
+          x1 = __shfl_sync(0xffffffffu, pl[1][kt], src1);
+          b1l = odd ? x1 : x0;
+        }
+      } else {
+        b0h = __shfl_sync(0xffffffffu, ph[0][kt], (2 * c) * 4);
+        b1h = __shfl_sync(0xffffffffu, ph[0][kt], (2 * c + 1) * 4);
+        if constexpr (kSplitPF16) {
+          b0l = __shfl_sync(0xffffffffu, pl[0][kt], (2 * c) * 4);
+          b1l = __shfl_sync(0xffffffffu, pl[0][kt], (2 * c + 1) * 4);
+        }
+      }
       const int t0 = kt * 16 + 2 * c;
       uint4 v0 = lds128(sV + t0 * 128 + ((g ^ (2 * c)) << 4));
       uint4 v1 = lds128(sV + (t0 + 8) * 128 + ((g ^ (2 * c)) << 4));
@@ -382,8 +493,51 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
     const int ns = (len + CH - 1) / CH;
     const bool unit_ends = i0 + 1 == wc0 && (wc1 == 0 || wu1 != wu0);
     if (unit_ends || j == ns - 1) {
-      const int64_t sh = static_cast<int64_t>(s) * p.num_heads + h;  // (text, head)
+      const int64_t sh = static_cast<int64_t>(s) * p.num_heads + h;  // (text, virtual head)
       const bool whole = piece_j0 == 0 && j == ns - 1 && !p.cascade;
+      if constexpr (GQA) {
+        float lt[2];
+#pragma unroll
+        for (int jc = 0; jc < 2; ++jc) {
+          lt[jc] = lg[jc];
+          lt[jc] += __shfl_xor_sync(0xffffffffu, lt[jc], 4);
+          lt[jc] += __shfl_xor_sync(0xffffffffu, lt[jc], 8);
+          lt[jc] += __shfl_xor_sync(0xffffffffu, lt[jc], 16);
+        }
+        const int qh0 = q_head0(h);
+        float* recs = p.records + (static_cast<int64_t>(wu0) + sh) * (GS * (D + 4));
+#pragma unroll
+        for (int jc = 0; jc < 2; ++jc) {
+          const int col = 2 * c + jc;  // query head qh0 + col
+          if (col >= GS) continue;
+          if (whole) {
+            const float inv = lt[jc] > 0.f ? p.v_scale / lt[jc] : 0.f;
+            float f[8];
+            __half* orow =
+                static_cast<__half*>(p.out) + (static_cast<int64_t>(s) * Hq + qh0 + col) * D + 16 * g;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                f[2 * i] = o[4 * half + i][jc] * inv;
+                f[2 * i + 1] = o[4 * half + i][2 + jc] * inv;
+              }
+              *reinterpret_cast<uint4*>(orow + 8 * half) = pack8<__half>(f);
+            }
+          } else {
+            float* rec = recs + col * (D + 4);
+            if (g == 0) {
+              rec[0] = mg[jc];
+              rec[1] = lt[jc];
+            }
+            float4* dst = reinterpret_cast<float4*>(rec + 4 + 16 * g);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(o[2 * i][jc] * p.v_scale, o[2 * i][2 + jc] * p.v_scale,
+                                   o[2 * i + 1][jc] * p.v_scale, o[2 * i + 1][2 + jc] * p.v_scale);
+          }
+        }
+      } else {
       float lt = l;
       lt += __shfl_xor_sync(0xffffffffu, lt, 4);
       lt += __shfl_xor_sync(0xffffffffu, lt, 8);
@@ -418,6 +572,7 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
                                  o[2 * i + 1][0] * p.v_scale, o[2 * i + 1][2] * p.v_scale);
         }
       }
+      }
     }
 
     prev_unit = wu0;
@@ -439,29 +594,32 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
 
 namespace {
 
-size_t f8_smem_bytes(int num_seqs) {
-  return 1024 /* alignment slack */ + static_cast<size_t>(kF8Warps) * f8_warp_bytes(kF8Stages) +
+size_t f8_smem_bytes(int num_seqs, bool gqa) {
+  return 1024 /* alignment slack */ +
+         static_cast<size_t>(f8_warps(gqa)) * f8_warp_bytes(kF8Stages, f8_qrows(gqa)) +
          align_up(sizeof(int32_t) * (num_seqs + 1), 16);
 }
 
-template <int B>
+template <int B, bool GQA>
 const void* f8_kernel_ptr() {
-  return reinterpret_cast<const void*>(&paged_decode_mma_fp8_kernel<B, kF8Warps, kF8Stages>);
+  return reinterpret_cast<const void*>(
+      &paged_decode_mma_fp8_kernel<B, f8_warps(GQA), kF8Stages, GQA>);
 }
 
+template <bool GQA>
 const void* f8_kernel_for(int block_size) {
   switch (block_size) {
-    case 8: return f8_kernel_ptr<8>();
-    case 16: return f8_kernel_ptr<16>();
-    case 32: return f8_kernel_ptr<32>();
+    case 8: return f8_kernel_ptr<8, GQA>();
+    case 16: return f8_kernel_ptr<16, GQA>();
+    case 32: return f8_kernel_ptr<32, GQA>();
     default: return nullptr;
   }
 }
 
-Plan plan_f8(const void* kernel, int B, int num_seqs, int num_heads, int max_blocks_per_seq,
-             int64_t forced_warps) {
-  return plan_decode(kernel, f8_smem_bytes(num_seqs), f8_smem_bytes(kMaxSeqs), kF8Warps, kF8CH,
-                     B, num_seqs, num_heads, max_blocks_per_seq, forced_warps);
+Plan plan_f8(const void* kernel, bool gqa, int B, int num_seqs, int vheads,
+             int max_blocks_per_seq, int64_t forced_warps) {
+  return plan_decode(kernel, f8_smem_bytes(num_seqs, gqa), f8_smem_bytes(kMaxSeqs, gqa),
+                     f8_warps(gqa), kF8CH, B, num_seqs, vheads, max_blocks_per_seq, forced_warps);
 }
 
 // The 8-bit pool [num_blocks][H][B][128] seen as a 2-D tensor of
@@ -474,14 +632,14 @@ bool encode_code_map(CUtensorMap* map, const void* pool, int64_t rows, int box_r
   return encode_tiled_map(map, pool, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dims, strides, box);
 }
 
-template <int B>
-cudaError_t launch_f8_typed(const DecodeArgs& a, cudaStream_t stream) {
-  const Plan pl = plan_f8(f8_kernel_ptr<B>(), B, a.num_seqs, a.num_heads, a.max_blocks_per_seq,
-                          a.forced_warps);
+template <int B, bool GQA>
+cudaError_t launch_f8_typed(const DecodeArgs& a, const DecodeLayout& hl, cudaStream_t stream) {
+  const Plan pl = plan_f8(f8_kernel_ptr<B, GQA>(), GQA, B, a.num_seqs, hl.vheads,
+                          a.max_blocks_per_seq, a.forced_warps);
   if (pl.grid <= 0) return cudaErrorInvalidConfiguration;
-  const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_heads;
+  const int64_t segs = static_cast<int64_t>(a.num_seqs) * hl.vheads;
   const size_t need = header_bytes(a.num_seqs) + kGrabBytes +
-                      records_bytes(max_units(pl.work_warps) + segs, kF8D, 1);
+                      records_bytes(max_units(pl.work_warps) + segs, kF8D, hl.gs);
   if (a.workspace_bytes < need) return cudaErrorInvalidValue;
   const int64_t rows = a.num_blocks * a.num_kv_heads * B;
   CUtensorMap tm_k, tm_v;
@@ -500,11 +658,11 @@ cudaError_t launch_f8_typed(const DecodeArgs& a, cudaStream_t stream) {
   p.qk_scale_log2 = a.scale * 1.4426950408889634f * a.k_scale;
   p.v_scale = a.v_scale;
   p.num_seqs = a.num_seqs;
-  p.num_heads = a.num_heads;
+  p.num_heads = hl.vheads;
   p.num_q_heads = a.num_heads;
   p.num_kv_heads = a.num_kv_heads;
-  p.nsub = 1;
-  p.gs = 1;
+  p.nsub = hl.nsub;
+  p.gs = hl.gs;
   p.max_blocks_per_seq = a.max_blocks_per_seq;
   p.num_blocks = a.num_blocks;
   p.num_work_warps = pl.work_warps;
@@ -521,7 +679,7 @@ cudaError_t launch_f8_typed(const DecodeArgs& a, cudaStream_t stream) {
   p.cascade = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
-  cfg.blockDim = dim3(kF8Warps * 32);
+  cfg.blockDim = dim3(f8_warps(GQA) * 32);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -530,39 +688,62 @@ cudaError_t launch_f8_typed(const DecodeArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(
-      &cfg, paged_decode_mma_fp8_kernel<B, kF8Warps, kF8Stages>, p, tm_k, tm_v);
+      &cfg, paged_decode_mma_fp8_kernel<B, f8_warps(GQA), kF8Stages, GQA>, p, tm_k, tm_v);
   if (err != cudaSuccess) return err;
-  err = launch_merge<__half, kF8D>(p, 1, stream);
+  err = launch_merge<__half, kF8D>(p, hl.gs, stream);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
 }  // namespace
 
+// Grouped-query pools: a key/value head's G query heads in nsub equal
+// subsets of gs <= 8 (the smallest count that divides G), one subset per
+// pass over the key/value head's codes, a query head per tile column.
+DecodeLayout mma_fp8_layout(int num_heads, int num_kv_heads) {
+  const int G = num_kv_heads > 0 ? num_heads / num_kv_heads : 1;
+  int nsub = (G + 7) / 8;
+  while (G % nsub) ++nsub;
+  return DecodeLayout{nsub, G / nsub, num_kv_heads * nsub};
+}
+
 bool mma_fp8_decode_ok(const DecodeArgs& a) {
   return a.fp8 && !a.is_bf16 && !a.slot_mapping && !a.cascade && a.head_dim == kF8D &&
-         a.num_heads == a.num_kv_heads &&
+         a.num_kv_heads >= 1 && a.num_heads % a.num_kv_heads == 0 &&
          (a.block_size == 8 || a.block_size == 16 || a.block_size == 32) &&
          mma_decode_pool_ok(a.num_kv_heads, a.block_size, a.num_blocks);
 }
 
-size_t mma_fp8_workspace_bytes(int num_seqs, int num_heads, int block_size,
+size_t mma_fp8_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int block_size,
                                int max_blocks_per_seq, int64_t forced_warps) {
-  const void* k = f8_kernel_for(block_size);
+  if (num_kv_heads < 1 || num_heads % num_kv_heads) return 0;
+  const DecodeLayout hl = mma_fp8_layout(num_heads, num_kv_heads);
+  const bool gqa = num_heads != num_kv_heads;
+  const void* k = gqa ? f8_kernel_for<true>(block_size) : f8_kernel_for<false>(block_size);
   if (!k) return 0;
-  const Plan pl = plan_f8(k, block_size, num_seqs, num_heads, max_blocks_per_seq, forced_warps);
+  const Plan pl = plan_f8(k, gqa, block_size, num_seqs, hl.vheads, max_blocks_per_seq,
+                          forced_warps);
   if (pl.grid <= 0) return 0;
-  const int64_t segs = static_cast<int64_t>(num_seqs) * num_heads;
+  const int64_t segs = static_cast<int64_t>(num_seqs) * hl.vheads;
   return header_bytes(num_seqs) + kGrabBytes +
-         records_bytes(max_units(pl.work_warps) + segs, kF8D, 1);
+         records_bytes(max_units(pl.work_warps) + segs, kF8D, hl.gs);
 }
 
 cudaError_t launch_paged_attn_decode_mma_fp8(const DecodeArgs& a, cudaStream_t stream) {
   if (!mma_fp8_decode_ok(a)) return cudaErrorInvalidValue;
+  const DecodeLayout hl = mma_fp8_layout(a.num_heads, a.num_kv_heads);
+  if (a.num_heads == a.num_kv_heads) {
+    switch (a.block_size) {
+      case 8: return launch_f8_typed<8, false>(a, hl, stream);
+      case 16: return launch_f8_typed<16, false>(a, hl, stream);
+      case 32: return launch_f8_typed<32, false>(a, hl, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (a.block_size) {
-    case 8: return launch_f8_typed<8>(a, stream);
-    case 16: return launch_f8_typed<16>(a, stream);
-    case 32: return launch_f8_typed<32>(a, stream);
+    case 8: return launch_f8_typed<8, true>(a, hl, stream);
+    case 16: return launch_f8_typed<16, true>(a, hl, stream);
+    case 32: return launch_f8_typed<32, true>(a, hl, stream);
     default: return cudaErrorInvalidValue;
   }
 }

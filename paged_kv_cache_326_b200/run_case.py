@@ -8,7 +8,8 @@ For profilers: it makes no timing claims.  Workloads: ``opt13b_batch64``
 ``tiny``, ``skewed`` (bf16, blocks of 16), ``llama2_70b_gqa`` (64 query heads
 on 8 key/value heads; always the two-call path, the one-launch step being
 multi-head only), ``opt13b_batch64_fp8`` (the batch-64 step over 8-bit
-caches, two calls), ``opt13b_prefill`` (the prompt phase: S prompts of 2,048
+caches, two calls), ``llama2_70b_gqa_fp8`` (the grouped-query step over
+8-bit caches, two calls), ``opt13b_prefill`` (the prompt phase: S prompts of 2,048
 tokens, 40 heads of 128; ``--prefill-kernel`` 0 automatic, 1 mma.sync, 2
 tcgen05), ``shared_prefix`` (32 prompts x 8 samples built by the block
 manager, through pa_paged_attn_decode_shared over the split tables).
@@ -35,6 +36,8 @@ def make(name: str, num_seqs: int, device):
         return W.skewed(device=device)
     if name == "opt13b_batch64_fp8":
         return W.opt13b_batch64_fp8(device=device)
+    if name == "llama2_70b_gqa_fp8":
+        return W.llama2_70b_gqa_fp8(device=device, num_seqs=num_seqs if num_seqs > 0 else 64)
     if name == "llama2_70b_gqa":
         return W.llama2_70b_gqa(device=device, num_seqs=num_seqs if num_seqs > 0 else 64)
     if name == "opt13b_batch64":

@@ -146,12 +146,49 @@ def test_fp8_grouped_query_every_shape(dtype, group, head_dim, block_size):
     parity_fp8(w)
 
 
-def test_fp8_grouped_query_llama2_70b():
+def test_fp8_grouped_query_llama2_70b(fp8_kernel):
     """The Llama-2-70B-shaped layer (64 query heads over 8 key/value heads,
     lengths 128..4096) over 8-bit caches: 12 texts x 8 sampled heads each."""
     w = W.llama2_70b_gqa_fp8(device="cuda", num_seqs=24, num_blocks=6144)
     c = parity_fp8(w, seqs=range(0, 24, 2), heads_per_seq=8, seed=5)
-    print("fp8 grouped-query llama2-70b", c)
+    print("fp8 grouped-query llama2-70b", fp8_kernel, c)
+
+
+@pytest.mark.parametrize("group", [2, 3, 8, 12, 16])
+@pytest.mark.parametrize("block_size", [8, 16, 32])
+def test_fp8_grouped_query_tensor_cores(group, block_size):
+    """The tensor-core kernel forced on grouped-query 8-bit pools: a key/value
+    head's query heads are the tile's columns (groups above 8 in equal
+    subsets of at most 8: 12 as 2 x 6, 16 as 2 x 8; 3 leaves columns that
+    repeat a head); ragged lengths 0..300 spanning several chunks and a
+    partial last one; every output against the oracle."""
+    import paged_kv_cache_326_b200 as P
+    lens = [0, 1, 7, 31, 32, 33, 95, 160, 300, 257, 64, 5]
+    w = W.make_decode_fp8("fp8_gqa_tc", lens, num_heads=3 * group, head_dim=128,
+                          block_size=block_size,
+                          num_blocks=3 * sum(W.blocks_needed(L, block_size) for L in lens),
+                          dtype=torch.float16, seed=group * 11 + block_size, device="cuda",
+                          max_blocks_per_seq=320 // block_size, num_kv_heads=3)
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, 2)
+    try:
+        parity_fp8(w)
+    finally:
+        P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
+
+
+def test_fp8_grouped_query_tensor_cores_all_outputs_of_a_large_batch():
+    """The tensor-core kernel forced on 16 texts of the Llama-2-70B shape
+    (64 query heads over 8 key/value heads, lengths up to 4096): every head
+    of every text against the oracle, so texts split across many warps and
+    merged are covered."""
+    import paged_kv_cache_326_b200 as P
+    w = W.llama2_70b_gqa_fp8(device="cuda", num_seqs=16, num_blocks=4096)
+    P.pa_set_option(P.PA_OPT_FP8_KERNEL, 2)
+    try:
+        c = parity_fp8(w)
+    finally:
+        P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
+    print("fp8 grouped-query tensor cores, 16 texts", c)
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
