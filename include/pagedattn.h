@@ -198,11 +198,13 @@ int pa_decode_step(void* out, const void* q, const void* k, const void* v, void*
  *                  pa_paged_attn_decode_fp8).  Multi-head only.
  *
  * Result: the pool afterwards and `out` are exactly those of
- * pa_kv_cache_write_fp8 followed by pa_paged_attn_decode_fp8 on the CUDA
- * cores (PA_OPT_FP8_KERNEL 1), under the conditions of pa_decode_step.  The
- * attention quantizes position context_lens[s] - 1 from k[s], v[s] itself,
- * with the write's arithmetic, so the launch never waits on its own write.
- * Runs on the CUDA-core kernel.  Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
+ * pa_kv_cache_write_fp8 followed by pa_paged_attn_decode_fp8 on the same
+ * kernel, under the conditions of pa_decode_step.  The attention quantizes
+ * position context_lens[s] - 1 from k[s], v[s] itself, with the write's
+ * arithmetic, so the launch never waits on its own write.  With fp16
+ * queries, head_dim 128 and blocks of 8, 16 or 32 it runs on the tensor-core
+ * 8-bit kernel (PA_OPT_FP8_KERNEL picks the kernel), else on the CUDA cores.
+ * Returns PA_OK or PA_ERR_INVALID / PA_ERR_CUDA.
  */
 int pa_decode_step_fp8(void* out, const void* q, const void* k, const void* v, void* k_cache,
                        void* v_cache, const int64_t* slot_mapping, const int32_t* block_tables,

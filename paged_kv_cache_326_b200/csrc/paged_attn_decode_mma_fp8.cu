@@ -149,7 +149,14 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
   const WorkSplit sp = decode_prologue<__half, D, CH, WARPS * 32>(p, prefix, warp_tot, cap);
   const int W = sp.W;
   const int w = blockIdx.x * WARPS + warp;
-  if (w >= W || sp.total == 0) return;
+  if (w >= W) return;
+  // One-launch step (multi-head pools): the cache write of every text's new
+  // row, each warp a share, as in the CUDA-core kernel.
+  const bool fused = !GQA && p.slot_mapping != nullptr;
+  if (sp.total == 0) {
+    if (fused) fused_cache_write_f8<__half, D, B>(p, w, W, lane);
+    return;
+  }
 
   uint8_t* tiles = smem + warp * AREA;
   uint8_t* qbuf = tiles + STAGES * 8192;
@@ -239,6 +246,8 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
 
 #pragma unroll
   for (int k = 0; k < STAGES; ++k) issue(k);
+  // (the write while the first copies are in flight)
+  if (fused) fused_cache_write_f8<__half, D, B>(p, w, W, lane);
 
   const int g = lane >> 2, c = lane & 3;
   uint32_t qh[16];   // query dimensions [32c, 32c + 32) of column g, as fp16 pairs
@@ -292,6 +301,25 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
         for (int e = 0; e < 4; ++e) o[md][e] = 0.f;
     }
     const int nvalid = bad ? 0 : min(CH, len - j * CH);
+    if (fused && nvalid > 0 && j * CH + nvalid == len) {
+      // The chunk holding the text's last position takes that row from the
+      // new k, v: its codes (the cache write's quantization) replace stage
+      // row nvalid - 1, which the copies brought from the pool (possibly
+      // while another warp was writing the same codes there).  Lanes 0-15
+      // write the K row, 16-31 the V row, 8 codes each, at the swizzled
+      // place of their 16-byte piece.
+      const int r = nvalid - 1, part = lane & 15;
+      const bool isv = lane >= 16;
+      const __half* src = static_cast<const __half*>(isv ? p.v_new : p.k_new) +
+                          (static_cast<int64_t>(s) * Hkv + h) * D + 8 * part;
+      float x[8];
+      unpack8<__half>(__ldg(reinterpret_cast<const uint4*>(src)), x);
+      uint8_t* row = const_cast<uint8_t*>(isv ? sV : sK) + r * 128;
+      *reinterpret_cast<uint2*>(row + (((part >> 1) ^ (r & 7)) << 4) + (part & 1) * 8) =
+          e4m3x8_quantize(x, isv ? p.v_scale : p.k_scale);
+      fence_proxy_async_smem();  // before this stage's refill by the copy engine
+      __syncwarp();
+    }
 
     // ---- S^T = K Q^T: two 16-token tiles, two accumulators each ----
     float sa[2][2][4];
@@ -673,9 +701,11 @@ cudaError_t launch_f8_typed(const DecodeArgs& a, const DecodeLayout& hl, cudaStr
   p.records = reinterpret_cast<float*>(ws + header_bytes(a.num_seqs) + kGrabBytes);
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
-  p.k_new = nullptr;
-  p.v_new = nullptr;
-  p.slot_mapping = nullptr;
+  // one-launch step: the new rows and their slots (null otherwise)
+  p.k_new = a.k_new;
+  p.v_new = a.v_new;
+  p.slot_mapping = a.slot_mapping;
+  p.k_scale = a.k_scale;
   p.cascade = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
@@ -708,7 +738,9 @@ DecodeLayout mma_fp8_layout(int num_heads, int num_kv_heads) {
 }
 
 bool mma_fp8_decode_ok(const DecodeArgs& a) {
-  return a.fp8 && !a.is_bf16 && !a.slot_mapping && !a.cascade && a.head_dim == kF8D &&
+  // (the one-launch step, with slot_mapping, on multi-head pools only)
+  return a.fp8 && !a.is_bf16 && !a.cascade && a.head_dim == kF8D &&
+         (!a.slot_mapping || a.num_heads == a.num_kv_heads) &&
          a.num_kv_heads >= 1 && a.num_heads % a.num_kv_heads == 0 &&
          (a.block_size == 8 || a.block_size == 16 || a.block_size == 32) &&
          mma_decode_pool_ok(a.num_kv_heads, a.block_size, a.num_blocks);

@@ -194,7 +194,7 @@ def test_fp8_grouped_query_tensor_cores_all_outputs_of_a_large_batch():
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
 @pytest.mark.parametrize("head_dim", [64, 128])
 @pytest.mark.parametrize("block_size", [4, 8, 16, 32])
-def test_fp8_one_launch_step_every_shape_ragged(dtype, head_dim, block_size):
+def test_fp8_one_launch_step_every_shape_ragged(dtype, head_dim, block_size, fp8_kernel):
     """pa_decode_step_fp8: the new tokens' codes in the pool bit for bit, every
     output against the oracle (which writes, then attends)."""
     w = W.make_decode_fp8("fp8_step", SHAPE_LENS, num_heads=3, head_dim=head_dim,
@@ -211,29 +211,27 @@ def test_fp8_one_launch_step_opt13b_batch64():
     print("fp8 one-launch step opt13b", c)
 
 
-def test_fp8_one_launch_step_equals_two_calls_bitwise():
-    """Same inputs: the one-launch 8-bit step and the quantizing write followed
-    by the CUDA-core 8-bit decode give the same output and the same pools,
-    bit for bit (the new row's codes come from the same quantizer)."""
-    import paged_kv_cache_326_b200 as P
+def test_fp8_one_launch_step_equals_two_calls_bitwise(fp8_kernel):
+    """Same inputs, same kernel (CUDA cores, or the default: tensor cores):
+    the one-launch 8-bit step and the quantizing write followed by the 8-bit
+    decode give the same output and the same pools, bit for bit (the new
+    row's codes come from the same quantizer)."""
     a = W.opt13b_batch64_fp8(device="cuda")
     b = W.opt13b_batch64_fp8(device="cuda")
-    P.pa_set_option(P.PA_OPT_FP8_KERNEL, 1)
-    try:
-        out_a = gpu_step_fp8(a)
-    finally:
-        P.pa_set_option(P.PA_OPT_FP8_KERNEL, 0)
+    out_a = gpu_step_fp8(a)
     out_b = gpu_step_fp8_fused(b)
     torch.cuda.synchronize()
     assert torch.equal(a.k_cache, b.k_cache) and torch.equal(a.v_cache, b.v_cache)
     assert torch.equal(out_a, out_b)
 
 
-def test_fp8_one_launch_step_single_token_returns_its_value():
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+def test_fp8_one_launch_step_single_token_returns_its_value(dtype):
     """One token per text, the new one: out = value(code(v / v_scale)) *
-    v_scale rounded to the output type, bit for bit."""
+    v_scale rounded to the output type, bit for bit (fp16: the tensor-core
+    kernel, whose stage row is the new token's codes; bf16: CUDA cores)."""
     w = W.make_decode_fp8("fp8_step_one", [1] * 6, num_heads=5, head_dim=128, block_size=16,
-                          num_blocks=16, dtype=torch.bfloat16, seed=8, device="cuda")
+                          num_blocks=16, dtype=dtype, seed=8, device="cuda")
     out = gpu_step_fp8_fused(w)
     torch.cuda.synchronize()
     vs = np.float32(w.meta["v_scale"])
