@@ -78,11 +78,14 @@ namespace {
 #define PA_F8MMA_STAGES 2
 #endif
 #ifndef PA_F8MMA_WARPS_GQA
-#define PA_F8MMA_WARPS_GQA 4
+#define PA_F8MMA_WARPS_GQA 2
 #endif
 constexpr int kF8Warps = PA_F8MMA_WARPS;    // warps per CTA
-// The grouped-query kernel's warps per CTA (its stages hold 8 query rows, so
-// its warps take 21 KB of shared memory against 17)
+// The grouped-query kernel's warps per CTA.  On the Llama-2-70B-shaped 8-bit
+// step: 2 warps a CTA with the query rows read from global memory (12 warps
+// an SM) 87.4 us; with the query rows in the stages (21 KB a warp), 4 warps
+// a CTA (8 an SM) 89.0-89.3, 2 (10) 88.8, 3 (9) 93.4, 5 (register-capped)
+// 99.0, 6 (one CTA) 109.4; 4 warps with the rows from global memory 90.2.
 constexpr int kF8WarpsGqa = PA_F8MMA_WARPS_GQA;
 __host__ __device__ constexpr int f8_warps(bool gqa) { return gqa ? kF8WarpsGqa : kF8Warps; }
 constexpr int kF8Stages = PA_F8MMA_STAGES;  // ring depth per warp
@@ -95,9 +98,18 @@ constexpr int kF8CH = 32;                   // tokens per chunk: 4 KB of key cod
 __host__ __device__ constexpr int f8_warp_bytes(int stages, int qrows) {
   return (stages * 8192 + stages * 256 * qrows + stages * 12 + 1023) / 1024 * 1024;
 }
+#ifndef PA_F8_GQA_Q_GLOBAL
+#define PA_F8_GQA_Q_GLOBAL 1
+#endif
+// Grouped-query: 1 loads a unit's query rows from global memory straight
+// into registers at the unit's first chunk (the stages then hold no query
+// rows); 0 brings them with the chunk's copies, up to 8 rows per stage.
+constexpr bool kF8GqaQGlobal = PA_F8_GQA_Q_GLOBAL != 0;
 // Query rows a stage holds: one (multi-head), or up to the tile's eight
-// columns (grouped-query).
-__host__ __device__ constexpr int f8_qrows(bool gqa) { return gqa ? 8 : 1; }
+// columns (grouped-query), or none.
+__host__ __device__ constexpr int f8_qrows(bool gqa) {
+  return gqa ? (kF8GqaQGlobal ? 0 : 8) : 1;
+}
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
@@ -115,6 +127,7 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
   constexpr int R = CH >= B ? B : CH;       // rows per TMA box
   constexpr uint32_t BOX_BYTES = R * 128;
   constexpr int QR = f8_qrows(GQA);
+  constexpr bool QG = GQA && kF8GqaQGlobal;  // query rows from global memory
   constexpr int AREA = f8_warp_bytes(STAGES, QR);
   static_assert(B >= 8 && CH % B == 0, "block sizes 8, 16, 32");
 
@@ -224,10 +237,10 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
       if (bad) set_status(p.status, -7 /* PA_ERR_BAD_BLOCK */);
       flags[st] = bad ? 1 : 0;
       fence_proxy_async_smem();
-      const uint32_t qbytes = first ? GS * D * 2 : 0;
+      const uint32_t qbytes = first && !QG ? GS * D * 2 : 0;
       const uint32_t kvbytes = bad ? 0 : 2u * boxes * BOX_BYTES;
       mbar_arrive_expect_tx(&bars[st], qbytes + kvbytes);
-      if (first)  // the unit's query rows (contiguous: GS heads in a row)
+      if (first && !QG)  // the unit's query rows (contiguous: GS heads in a row)
         bulk_copy_g2s(qbuf + st * 256 * QR, qg + (static_cast<int64_t>(s) * Hq + q_head0(h)) * D,
                       GS * D * 2, &bars[st], policy);
       if (!bad) {
@@ -283,9 +296,11 @@ paged_decode_mma_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtens
     if (j == 0 || wu0 != prev_unit) {
       piece_j0 = j;
       const uint8_t* qrow = qbuf + st * 256 * QR + (GQA ? (g % GS) * 256 : 0) + c * 64;
+      const uint4* qrow_g = reinterpret_cast<const uint4*>(
+          qg + (static_cast<int64_t>(s) * Hq + q_head0(h) + g % GS) * D + c * 32);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint4 x = lds128(qrow + 16 * i);
+        const uint4 x = QG ? __ldg(qrow_g + i) : lds128(qrow + 16 * i);
         qh[4 * i + 0] = x.x;
         qh[4 * i + 1] = x.y;
         qh[4 * i + 2] = x.z;
