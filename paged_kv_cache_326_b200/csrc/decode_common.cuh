@@ -37,7 +37,10 @@ constexpr int kDrainLimitNs = 1000000000;
 #endif
 // Each warp's static run is about kStaticPermille per mille of an even share;
 // the rest goes out in grains of at least kMinGrain chunks, about
-// kGrainsPerWarp per warp.
+// kGrainsPerWarp per warp.  (Longer static runs, 850 or 930 per mille, or
+// grains of at least 32 chunks measured slower on the batch-64 multi-head
+// step and on the grouped-query steps, 16- and 8-bit: fewer partials to
+// merge, but a longer tail of warps finishing late.)
 constexpr int kStaticPermille = PA_STATIC_PERMILLE;
 constexpr int kGrainsPerWarp = 12;
 constexpr int kMinGrain = PA_MIN_GRAIN;
