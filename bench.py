@@ -58,6 +58,12 @@ TRAFFIC = {
          "paged_kv_cache_326_b200/csrc/decode_common.cuh",
          "paged_kv_cache_326_b200/csrc/fp8.cuh", "paged_kv_cache_326_b200/csrc/mma_ptx.cuh",
          "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
+    "llama2_70b_gqa_fp8": (
+        os.path.join(ROOT, "profiles", "paged_decode_mma_fp8_llama2_70b_gqa_fp8_traffic.json"),
+        ["paged_kv_cache_326_b200/csrc/paged_attn_decode_mma_fp8.cu",
+         "paged_kv_cache_326_b200/csrc/decode_common.cuh",
+         "paged_kv_cache_326_b200/csrc/fp8.cuh", "paged_kv_cache_326_b200/csrc/mma_ptx.cuh",
+         "paged_kv_cache_326_b200/csrc/ptx.cuh", "paged_kv_cache_326_b200/csrc/dtype.cuh"]),
     # the shared-prefix call: prefix pass + tail pass + merge, summed
     "shared_prefix": (
         os.path.join(ROOT, "profiles", "paged_decode_shared_prefix_c4_traffic.json"),
