@@ -26,6 +26,10 @@ bool encode_swizzled_map(CUtensorMap* map, const void* base, bool bf16, int rank
 // The same for any element type the driver names (one-byte codes among them).
 bool encode_tiled_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
+// The same without swizzle: a box lands in shared memory as a plain
+// row-major array (inner box of at most 256 elements).
+bool encode_plain_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
 
 cudaError_t launch_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
                                   const int64_t* slot_mapping, int num_tokens, int num_heads,

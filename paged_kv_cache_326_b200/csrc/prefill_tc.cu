@@ -127,6 +127,12 @@ constexpr int64_t kTcDrainNs = 1000000000;
 // against 697 TFLOP/s for the attention alone), 0 after keys 32-63's
 // weights (fewest registers live).
 constexpr int kTcPrefetch = PA_TC_PREFETCH;
+#ifndef PA_TC_STORE_BLOCKS
+#define PA_TC_STORE_BLOCKS 1
+#endif
+// 1: the store warps move a block's rows of k and v with one tiled load and
+// one bulk store each where the slots allow (else row by row)
+constexpr bool kTcStoreBlocks = PA_TC_STORE_BLOCKS != 0;
 #ifndef PA_TC_MAX_ONE_WAIT
 #define PA_TC_MAX_ONE_WAIT 0
 #endif
@@ -191,13 +197,16 @@ struct TcParams {
   const int32_t* cached_lens;
   int max_blocks;
   int B_shift;  // log2(B): block sizes are powers of two
+  // 1: the store warps move whole blocks (tm_ks / tm_vs are encoded)
+  int store_blocks;
 };
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
 prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc) {
+                  const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs) {
   using LY = TcLayout<D>;
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t IDESC_S = tc::idesc_f16(kTcBM, kTcBN, BF16, false);
@@ -211,6 +220,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
   // bytes) and empty (the last product that reads it)
   __shared__ uint64_t bar_q, bar_full[2][kTcStages], bar_empty[2][kTcStages];
   __shared__ uint64_t bar_s[kTcTiles], bar_p[kTcTiles], bar_o[kTcTiles], bar_st;
+  __shared__ uint64_t bar_stw[2];  // the store warps' own barriers (whole-block stores)
   // the two halves of a row trade partial maxima (two buffers, alternating
   // by block) and, at the end, partial sums
   __shared__ float xmax[2][kTcTiles][2][kTcBM];
@@ -269,6 +279,8 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&bar_o[t], 1);
     }
     mbar_init(&bar_st, 64);  // the store warps' 64 threads
+    mbar_init(&bar_stw[0], 32);
+    mbar_init(&bar_stw[1], 32);
     fence_barrier_init();
   }
   if (warp == 0) tc::alloc(&tmem_base, kTmemCols);
@@ -498,10 +510,105 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     const int n_tok = static_cast<int>(L * cum(pair + 1) / cP) - tok0;
     const int64_t num_slots = p.num_blocks * p.B;
     const int lid = (warp - kStoreWarp0) * 32 + lane;
+    const uint64_t read_pol = l2_evict_first_policy();
+    constexpr uint32_t ROW = D * 2;
+    if (p.store_blocks) {
+      // Whole blocks (a block's K and V rows of this head take at most 8 KB):
+      // the shares' bounds are rounded down to multiples of B, so each
+      // share is a run of groups of B tokens that start a block when the
+      // prompt's slots run in order.  Warp 18 takes the even groups, warp
+      // 19 the odd ones, each through its own 8 KB of staging.  A group
+      // whose B slots are one block's, in order, moves as two tiled loads
+      // (B rows of k, of v, from the [T][Hkv][D] tensors) and two bulk
+      // stores of B rows each: 4 copies for 2B rows.  Any other group (the
+      // prompt's last, partial one; slots out of order, negative or outside
+      // the pool) goes row by row as below.
+      const int Bq = p.B;
+      auto bound = [&](int64_t q) -> int {
+        if (q >= npairs) return L;
+        return static_cast<int>(L * cum(q) / cP) & ~(Bq - 1);
+      };
+      const int t_lo = bound(pair), t_hi = bound(pair + 1);
+      const int ws = warp - kStoreWarp0;
+      uint8_t* stg = sKV + kTcStages * LY::STAGE + ws * 8192;
+      uint64_t* wb = &bar_stw[ws];
+      uint32_t wph = 0;
+      const int ng = (t_hi - t_lo + Bq - 1) / Bq;
+      for (int gi = ws; gi < ng; gi += 2) {
+        const int t0 = t_lo + gi * Bq;
+        const int n = min(Bq, t_hi - t0);
+        const int64_t sl = lane < n ? __ldg(p.slot_mapping + a + t0 + lane) : -1;
+        const int64_t s0 = __shfl_sync(0xffffffffu, sl, 0);
+        const bool whole = n == Bq && s0 >= 0 && s0 < num_slots && (s0 & (Bq - 1)) == 0 &&
+                           __all_sync(0xffffffffu, lane >= n || sl == s0 + lane);
+        uint8_t* dst[2] = {nullptr, nullptr};
+        if (whole) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(wb, 2u * Bq * ROW);
+            tc::tma_load_3d(stg, &tm_ks, 0, kvh, a + t0, wb);
+            tc::tma_load_3d(stg + Bq * ROW, &tm_vs, 0, kvh, a + t0, wb);
+          } else {
+            mbar_arrive(wb);
+          }
+        } else {
+          // rows r = lane, lane + 32 of the group: K rows 0..n-1, then V rows
+          uint32_t bytes = 0;
+          const uint8_t* src[2] = {nullptr, nullptr};
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int r = lane + 32 * u;
+            if (r < 2 * n) {
+              const int kv = r >= n;
+              const int64_t row = a + t0 + (r - kv * n);
+              const int64_t slot = __ldg(p.slot_mapping + row);
+              if (slot >= num_slots) {
+                if (!kv) set_status(p.status, -9 /* PA_ERR_BAD_SLOT */);
+              } else if (slot >= 0) {
+                const int64_t blk = slot >> p.B_shift, place = slot & (p.B - 1);
+                dst[u] = static_cast<uint8_t*>(kv ? p.v_cache : p.k_cache) +
+                         (((blk * p.Hkv + kvh) << p.B_shift) + place) * ROW;
+                src[u] = static_cast<const uint8_t*>(kv ? p.v : p.k) + (row * p.Hkv + kvh) * ROW;
+                bytes += ROW;
+              }
+            }
+          }
+          if (bytes) {
+            mbar_arrive_expect_tx(wb, bytes);
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+              if (src[u]) bulk_copy_g2s(stg + (lane + 32 * u) * ROW, src[u], ROW, wb, read_pol);
+          } else {
+            mbar_arrive(wb);
+          }
+        }
+        // one outcome for the whole warp (its lanes time their waits apart)
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(wb, wph, lim));
+        if (!ok) {
+          give_up();
+          mbar_wait_bounded(wb, wph, kTcDrainNs);  // the copies still in flight
+          break;
+        }
+        wph ^= 1;
+        if (whole) {
+          if (lane == 0) {
+            const int64_t off = ((s0 >> p.B_shift) * p.Hkv + kvh) * Bq * ROW;
+            tc::bulk_store(static_cast<uint8_t*>(p.k_cache) + off, stg, Bq * ROW);
+            tc::bulk_store(static_cast<uint8_t*>(p.v_cache) + off, stg + Bq * ROW, Bq * ROW);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            if (dst[u]) tc::bulk_store(dst[u], stg + (lane + 32 * u) * ROW, ROW);
+        }
+        tc::bulk_commit();
+        tc::bulk_wait_read_all();  // the staging is read: it can be refilled
+        __syncwarp();
+      }
+      tc::bulk_wait_read_all();
+    } else {
     // Batches of 64 rows (K rows, then V rows), one per thread: a bulk copy
     // brings the row into the staging area, a bulk copy takes it to its
     // slot; the staging row is reused once that copy has read it.
-    constexpr uint32_t ROW = D * 2;
     uint8_t* stage_row = sKV + kTcStages * LY::STAGE + lid * ROW;
     const int rows = 2 * n_tok;
     uint32_t phase = 0;
@@ -525,7 +632,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
           mbar_arrive_expect_tx(&bar_st, ROW);
           bulk_copy_g2s(stage_row, static_cast<const uint8_t*>(kv ? p.v : p.k) +
                                        (row * p.Hkv + kvh) * ROW,
-                        ROW, &bar_st, l2_evict_first_policy());
+                        ROW, &bar_st, read_pol);
         }
       }
       if (!dst) mbar_arrive(&bar_st);
@@ -540,6 +647,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       }
     }
     tc::bulk_wait_read_all();
+    }
   }
   } else {
     // ---------------- softmax: half of one query row ----------------
@@ -809,7 +917,21 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
         !encode_swizzled_map(&tvc, a.v_cache, bf16, 4, dc, sc, bc))
       return cudaErrorInvalidValue;
   }
+  // the new tokens' k and v as (D, Hkv, T) again, unswizzled boxes of D x 1
+  // x B: one block's rows of one head, row-major, for whole-block stores
+  CUtensorMap tks = tk, tvs = tv;
+  const bool store_blocks = kTcStoreBlocks && a.slot_mapping && a.block_size <= 32 &&
+                            2 * a.block_size * D * 2 <= 8192;
+  if (store_blocks) {
+    const uint32_t bs[3] = {static_cast<uint32_t>(D), 1u, static_cast<uint32_t>(a.block_size)};
+    const CUtensorMapDataType ty =
+        bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!encode_plain_map(&tks, a.k, ty, 3, dk, sk, bs) ||
+        !encode_plain_map(&tvs, a.v, ty, 3, dk, sk, bs))
+      return cudaErrorInvalidValue;
+  }
   TcParams p;
+  p.store_blocks = store_blocks ? 1 : 0;
   p.out = a.out;
   p.cu_seqlens = a.cu_seqlens;
   p.num_tokens = a.num_tokens;
@@ -843,7 +965,8 @@ cudaError_t launch_prefill_tc_typed(const PrefillArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<T, D>, p, tq, tk, tv, tkc, tvc);
+  cudaError_t err =
+      cudaLaunchKernelEx(&cfg, prefill_tc_kernel<T, D>, p, tq, tk, tv, tkc, tvc, tks, tvs);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

@@ -54,8 +54,10 @@ bool encode_swizzled_map(CUtensorMap* map, const void* base, bool bf16, int rank
                           rank, dims, strides_bytes, box);
 }
 
-bool encode_tiled_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
-                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+namespace {
+bool encode_with(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle) {
   const EncodeTiledFn fn = encode_tiled();
   if (!fn || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], st[4];
@@ -67,8 +69,19 @@ bool encode_tiled_map(CUtensorMap* map, const void* base, CUtensorMapDataType ty
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
   return fn(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, b, e,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            l2_promotion(), CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, l2_promotion(),
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+bool encode_tiled_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_with(map, base, type, rank, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool encode_plain_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_with(map, base, type, rank, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace pa
