@@ -658,7 +658,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
     const int row = (warp & 3) * 32 + lane;      // row within the tile = TMEM lane
     const int qpos = q0 + t * kTcBM + row;       // new row within the prompt (position cl + qpos)
     const uint32_t rbase = tmem + t * kTileCols + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t tile_bar = 1 + t;             // named barrier of the tile's 256 threads
+    // Named barrier of the exchange: the tile's 256 threads.  (One barrier
+    // per pair of warps that share rows, 64 threads, measured 0.5% slower.)
+    const uint32_t tile_bar = 1 + t;
+    constexpr uint32_t kBarThreads = 2 * kTcBM;
     float m = -INFINITY, l = 0.f;
     bool failed = false;
     const int nk = nkb_t[t];
@@ -729,7 +732,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       }
       // the pair's maxima meet here; every thread of the tile learns whether
       // any gave up, so all leave together
-      if (bar_any(tile_bar, 2 * kTcBM, failed)) {
+      if (bar_any(tile_bar, kBarThreads, failed)) {
         failed = true;
         break;
       }
@@ -823,7 +826,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_q,
       // ---- epilogue: out = O / l, each thread its half of head_dim ----
       failed = __any_sync(0xffffffffu, failed || !wait(&bar_o[t], (nk - 1) & 1));
       xsum[t][hf][row] = l;
-      if (!bar_any(tile_bar, 2 * kTcBM, failed)) {
+      if (!bar_any(tile_bar, kBarThreads, failed)) {
         tc::fence_after_sync();
         const float lt = l + xsum[t][hf ^ 1][row];
         const bool store = qpos < L;
