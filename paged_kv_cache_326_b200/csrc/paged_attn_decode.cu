@@ -75,8 +75,16 @@ constexpr int kDecodeStages = PA_DECODE_STAGES;  // ring depth per warp
 #define PA_DECODE_STAGES_F8 2
 #endif
 constexpr int kDecodeStagesF8 = PA_DECODE_STAGES_F8;
-__host__ __device__ constexpr int decode_stages(bool f8) {
-  return f8 ? kDecodeStagesF8 : kDecodeStages;
+// Blocks of 8 or fewer rows: a chunk takes two or more copies of K and of V,
+// and two stages, three CTAs an SM, beat three stages, two CTAs (skewed
+// lengths, bf16: 414 against 474 us at blocks of 8); at blocks of 16 and up
+// three stages stay (the batch-64 step: 238 against 246 us).
+#ifndef PA_DECODE_STAGES_SMALL_B
+#define PA_DECODE_STAGES_SMALL_B 2
+#endif
+constexpr int kDecodeStagesSmallB = PA_DECODE_STAGES_SMALL_B;
+__host__ __device__ constexpr int decode_stages(bool f8, int B) {
+  return f8 ? kDecodeStagesF8 : B <= 8 ? kDecodeStagesSmallB : kDecodeStages;
 }
 // One stage: K rows (4 KB), V rows (4 KB), the unit's GS query rows, a flag.
 __host__ __device__ constexpr int stage_bytes(int D, int gs) { return 2 * 4096 + gs * 2 * D + 128; }
@@ -533,8 +541,8 @@ paged_decode_kernel(const DecodeParams p) {
 
 namespace {
 
-size_t decode_smem_bytes(int D, int num_seqs, int gs, bool fp8) {
-  return static_cast<size_t>(kDecodeWarps) * warp_area_bytes(D, decode_stages(fp8), gs) +
+size_t decode_smem_bytes(int D, int num_seqs, int gs, bool fp8, int B) {
+  return static_cast<size_t>(kDecodeWarps) * warp_area_bytes(D, decode_stages(fp8, B), gs) +
          align_up(sizeof(int32_t) * (num_seqs + 1), 16);
 }
 
@@ -553,8 +561,8 @@ HeadLayout head_layout(int num_heads, int num_kv_heads) {
 // Persistent grid for one decode kernel variant.
 Plan plan_variant(const void* kernel, int D, int B, int num_seqs, int vheads,
                   int max_blocks_per_seq, int64_t forced_warps, int gs, bool fp8) {
-  return plan_decode(kernel, decode_smem_bytes(D, num_seqs, gs, fp8),
-                     decode_smem_bytes(D, kMaxSeqs, gs, fp8),
+  return plan_decode(kernel, decode_smem_bytes(D, num_seqs, gs, fp8, B),
+                     decode_smem_bytes(D, kMaxSeqs, gs, fp8, B),
                      kDecodeWarps, fp8 ? 4096 / D : chunk_tokens(D), B, num_seqs, vheads,
                      max_blocks_per_seq, forced_warps);
 }
@@ -562,7 +570,7 @@ Plan plan_variant(const void* kernel, int D, int B, int num_seqs, int vheads,
 template <typename T, int D, int B, bool FUSED, int GS, bool F8>
 const void* decode_kernel_ptr() {
   return reinterpret_cast<const void*>(
-      &paged_decode_kernel<T, D, B, kDecodeWarps, decode_stages(F8), FUSED, GS, F8>);
+      &paged_decode_kernel<T, D, B, kDecodeWarps, decode_stages(F8, B), FUSED, GS, F8>);
 }
 
 template <typename T, int D, int B, bool FUSED, int GS, bool F8>
@@ -617,7 +625,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const HeadLayout& hl, cudaStream_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(
-      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, decode_stages(F8), FUSED, GS, F8>, p);
+      &cfg, paged_decode_kernel<T, D, B, kDecodeWarps, decode_stages(F8, B), FUSED, GS, F8>, p);
   if (err != cudaSuccess) return err;
   if (p.cascade) return cudaGetLastError();  // the caller merges
   err = launch_merge<T, D>(p, GS, stream);
