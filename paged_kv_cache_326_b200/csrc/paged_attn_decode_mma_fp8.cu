@@ -75,7 +75,10 @@ namespace {
 #define PA_F8MMA_WARPS 4
 #endif
 #ifndef PA_F8MMA_STAGES
-#define PA_F8MMA_STAGES 2
+#define PA_F8MMA_STAGES 3
+#endif
+#ifndef PA_F8MMA_STAGES_GQA
+#define PA_F8MMA_STAGES_GQA 2
 #endif
 #ifndef PA_F8MMA_WARPS_GQA
 #define PA_F8MMA_WARPS_GQA 2
@@ -88,7 +91,12 @@ constexpr int kF8Warps = PA_F8MMA_WARPS;    // warps per CTA
 // 99.0, 6 (one CTA) 109.4; 4 warps with the rows from global memory 90.2.
 constexpr int kF8WarpsGqa = PA_F8MMA_WARPS_GQA;
 __host__ __device__ constexpr int f8_warps(bool gqa) { return gqa ? kF8WarpsGqa : kF8Warps; }
-constexpr int kF8Stages = PA_F8MMA_STAGES;  // ring depth per warp
+// Ring depth per warp.  Multi-head: 3 stages, 2 CTAs (8 warps) an SM, 136.2
+// us on the batch-64 step against 142.4 for 2 stages, 3 CTAs (12 warps) on
+// the same box; grouped-query: 2 (3 measured the same).
+constexpr int kF8Stages = PA_F8MMA_STAGES;
+constexpr int kF8StagesGqa = PA_F8MMA_STAGES_GQA;
+__host__ __device__ constexpr int f8_stages(bool gqa) { return gqa ? kF8StagesGqa : kF8Stages; }
 constexpr int kF8D = 128;                   // head_dim
 constexpr int kF8CH = 32;                   // tokens per chunk: 4 KB of key codes
 
@@ -639,14 +647,14 @@ namespace {
 
 size_t f8_smem_bytes(int num_seqs, bool gqa) {
   return 1024 /* alignment slack */ +
-         static_cast<size_t>(f8_warps(gqa)) * f8_warp_bytes(kF8Stages, f8_qrows(gqa)) +
+         static_cast<size_t>(f8_warps(gqa)) * f8_warp_bytes(f8_stages(gqa), f8_qrows(gqa)) +
          align_up(sizeof(int32_t) * (num_seqs + 1), 16);
 }
 
 template <int B, bool GQA>
 const void* f8_kernel_ptr() {
   return reinterpret_cast<const void*>(
-      &paged_decode_mma_fp8_kernel<B, f8_warps(GQA), kF8Stages, GQA>);
+      &paged_decode_mma_fp8_kernel<B, f8_warps(GQA), f8_stages(GQA), GQA>);
 }
 
 template <bool GQA>
@@ -733,7 +741,7 @@ cudaError_t launch_f8_typed(const DecodeArgs& a, const DecodeLayout& hl, cudaStr
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(
-      &cfg, paged_decode_mma_fp8_kernel<B, f8_warps(GQA), kF8Stages, GQA>, p, tm_k, tm_v);
+      &cfg, paged_decode_mma_fp8_kernel<B, f8_warps(GQA), f8_stages(GQA), GQA>, p, tm_k, tm_v);
   if (err != cudaSuccess) return err;
   err = launch_merge<__half, kF8D>(p, hl.gs, stream);
   if (err != cudaSuccess) return err;
